@@ -1,0 +1,120 @@
+/*
+ * zgcm_attn.h — C ABI of the ZGCM-1 gated window-attention layer on B200 (sm_100a).
+ *
+ * One attention layer of the ZGCM-1 hybrid decoder, forward and backward:
+ *
+ *   per-head QK-RMSNorm -> partial RoPE on the first `rope_dims` head dims ->
+ *   GQA (query head h reads KV head h / (Hq/Hkv)) -> causal attention restricted to
+ *   the `window` most recent keys (key j visible to query i iff i - window < j <= i) ->
+ *   output multiplied elementwise by sigmoid(g).
+ *
+ * Where each piece is defined:
+ *   - window of 128 nearest tokens, 5:1 local:global interleave, global layers at
+ *     6/12/18/24/30: ZGCM-1 summary (paper.rainbus.top), section "前置知识 / 滑动窗口注意力
+ *     (SWA)与混合注意力"; the same facts in the shibing624 review, section "架构：5:1 的门控滑窗注意力".
+ *   - QK-RMSNorm, RoPE ratio 0.33, GQA 32 query / 8 KV heads: shibing624 review, section
+ *     "架构"; ZGCM-1 summary, section "核心方法".
+ *   - the sigmoid output gate: shibing624 review, section "架构" (the sentence says the
+ *     local attention output is multiplied by a sigmoid gate; the formula itself was lost
+ *     from the page).  Read here as out = sigmoid(g) * attn with g supplied by the caller,
+ *     one logit per output element.
+ *   - gated sliding-window and full attention interleaved: yunkai-blog summary, section
+ *     "关键技术点 1 (Architecture & System Co-design)".
+ *   window >= S gives the full-causal global layer of the same model.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are DEVICE pointers, contiguous, BSHD order, bf16 (raw 16-bit storage)
+ *     unless stated: q, g, out, dout, dq, dg are [B, S, Hq, D]; k, v, dk, dv are
+ *     [B, S, Hkv, D]; lse is fp32 [B, Hq, S]; gamma_q, gamma_k, dgamma_q, dgamma_k are
+ *     fp32 [D].  Every pointer must be 16-byte aligned (ZGCM_ERR_ALIGNMENT otherwise).
+ *   - Ownership: the caller owns every buffer.  The library never allocates device memory
+ *     and keeps no state between calls.
+ *   - Streams: every call is asynchronous on `cuda_stream` (a cudaStream_t, NULL = legacy
+ *     default stream) and never synchronises the device.
+ *   - Errors: arguments are checked on the host before anything is launched; a failed
+ *     check returns a negative zgcm_status and launches nothing.  A failed launch returns
+ *     ZGCM_ERR_CUDA.  No kernel traps.
+ *   - Supported shapes: D == 128, Hq % Hkv == 0, Hq, Hkv >= 1, rope_dims even with
+ *     0 <= rope_dims <= D, window >= 1, causal == 1, B >= 0, S >= 0, B*S*Hq*D < 2^40.
+ *     B == 0 or S == 0 is a valid empty problem (backward still zeroes dgamma_*).
+ *   - Positions are 0..S-1 in every sequence of the batch.
+ *   - Thread-safe and re-entrant: no global mutable state.
+ */
+#ifndef ZGCM_ATTN_H
+#define ZGCM_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ZGCM_OK = 0,
+    ZGCM_ERR_INVALID_ARG = -1, /* null pointer, negative size, window < 1, eps < 0, ...   */
+    ZGCM_ERR_UNSUPPORTED = -2, /* valid but not implemented: D != 128, causal == 0, ...   */
+    ZGCM_ERR_ALIGNMENT = -3,   /* a tensor pointer is not 16-byte aligned                 */
+    ZGCM_ERR_WORKSPACE = -4,   /* workspace null or smaller than the size query returns  */
+    ZGCM_ERR_CUDA = -5,        /* a CUDA runtime call or a kernel launch failed          */
+    ZGCM_ERR_TIMEOUT = -6      /* reserved: a bounded device-side wait gave up           */
+} zgcm_status;
+
+/* Human-readable name of a zgcm_status value (static string, never NULL). */
+const char* zgcm_status_string(int status);
+
+/*
+ * Forward of one gated attention layer.
+ *
+ *   q_hat = RoPE(gamma_q * q / sqrt(mean_d q^2 + eps))     per (b, s, query head)
+ *   k_hat = RoPE(gamma_k * k / sqrt(mean_d k^2 + eps))     per (b, s, KV head)
+ *   s_ij  = scale * q_hat_i . k_hat_j            for max(0, i-window+1) <= j <= i
+ *   A_i   = sum_j softmax_j(s_ij) v_j ;  out_i = sigmoid(g_i) * A_i
+ *   lse_i = log sum_j exp(s_ij)                  (natural log, kept for backward)
+ *
+ * RoPE rotates pairs (t, t + rope_dims/2) for t < rope_dims/2 by angle pos * theta_t,
+ * theta_t = rope_base^(-2t/rope_dims); dims >= rope_dims pass through.
+ *
+ * In : q, g bf16 [B,S,Hq,D]; k, v bf16 [B,S,Hkv,D]; gamma_q, gamma_k fp32 [D].
+ * Out: out bf16 [B,S,Hq,D] (rounded once, to nearest even); lse fp32 [B,Hq,S].
+ * out/lse must not alias any input.
+ */
+int zgcm_attn_fwd(const void* q, const void* k, const void* v, const void* g,
+                  const float* gamma_q, const float* gamma_k,
+                  int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                  double rope_base, int window, int causal, float eps, float scale,
+                  void* out, float* lse, void* cuda_stream);
+
+/*
+ * Bytes of device workspace zgcm_attn_bwd needs for this problem (0 for an empty one).
+ * Returns 0 as well for arguments zgcm_attn_bwd would reject.
+ */
+size_t zgcm_attn_bwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int window);
+
+/*
+ * Backward of zgcm_attn_fwd: exact gradients of L = sum(dout * out) with respect to
+ * q, k, v, g, gamma_q and gamma_k.
+ *
+ * In : the forward's inputs and arguments, its outputs `out` (bf16) and `lse` (fp32),
+ *      and dout bf16 [B,S,Hq,D].
+ * Out: dq, dg bf16 [B,S,Hq,D] — gradients w.r.t. the RAW q (before RMSNorm) and the gate
+ *      logits; dk, dv bf16 [B,S,Hkv,D] — summed over the Hq/Hkv query heads that share
+ *      each KV head; dgamma_q, dgamma_k fp32 [D] — overwritten (not accumulated).
+ * workspace: device scratch of at least zgcm_attn_bwd_workspace_size(...) bytes, 256-byte
+ *      aligned, owned by the caller, contents on entry irrelevant; it must not be used by
+ *      another call that runs concurrently.
+ * Outputs must not alias inputs or each other.
+ */
+int zgcm_attn_bwd(const void* q, const void* k, const void* v, const void* g,
+                  const float* gamma_q, const float* gamma_k,
+                  const void* out, const float* lse, const void* dout,
+                  int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                  double rope_base, int window, int causal, float eps, float scale,
+                  void* dq, void* dk, void* dv, void* dg,
+                  float* dgamma_q, float* dgamma_k,
+                  void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZGCM_ATTN_H */
