@@ -1,0 +1,391 @@
+#!/usr/bin/env python3
+"""Benchmark of the gated window-attention layer (ZGCM-1) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload swa16k]
+
+A step is one pass of the whole hot path: forward + backward of one gated attention layer
+over one batch of seeded synthetic inputs already resident in HBM.  The default workload
+is the 16K gated sliding-window layer: B=4 sequences x S=16384 tokens, 32 query / 8 KV
+heads, head dim 128, window 128 (65,536 tokens per step per GPU).  Under torchrun each
+rank runs its own batch (independent sequences, no collective on the data path): weak
+scaling, value = tokens of all ranks / max-over-ranks device time.
+
+Prints ONE JSON line (rank 0).  --impl reference times the fp64 CPU oracle instead (rank 0
+only; a bounded sample of the same workload per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "gated SWA fwd+bwd tokens/s & % of roofline, 16K seq, GQA 32/8, d=128, 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOADS = {
+    # name: (B, S, window, backward?)
+    "swa16k": (4, 16384, 128, True),
+    "global64k": (1, 65536, 65536, True),
+    "swa256k_fwd": (1, 262144, 128, False),
+    "global256k_fwd": (1, 262144, 262144, False),
+    "tiny_fwd": (1, 1024, 128, False),
+}
+HQ, HKV, D = 32, 8, 128
+
+
+def pairs(S: int, W: int) -> int:
+    """Visible (i, j) pairs per (batch, head): sum_i min(i+1, W)."""
+    if W >= S:
+        return S * (S + 1) // 2
+    return W * S - W * (W - 1) // 2
+
+
+def work(B, S, W, bwd):
+    """Masked FLOPs and algorithmic HBM bytes of one step (and of each dominant kernel)."""
+    npair = pairs(S, W) * B * HQ
+    tok = B * S
+    qb = tok * HQ * D * 2            # q, g, out, dout, dq, dg (bf16 [B,S,Hq,D])
+    kb = tok * HKV * D * 2           # k, v, dk, dv
+    lse = tok * HQ * 4
+    fwd_bytes = 2 * qb + 2 * kb + qb + lse               # read q,k,v,g; write out, lse
+    fwd_flops = 4 * D * npair
+    bwd_bytes = 4 * qb + 2 * kb + lse + 2 * qb + 2 * kb  # read q,k,v,g,out,dout,lse; write dq,dk,dv,dg
+    bwd_flops = 10 * D * npair
+    # main backward kernel of this build: reads q, k, v, dA (bf16), lse, Delta;
+    # writes dk, dv and the fp32 dQ~ accumulation (each counted once)
+    main_bytes = qb + 2 * kb + qb + 2 * lse + 2 * kb + tok * HQ * D * 4
+    return dict(tokens=tok, npair=npair, fwd_bytes=fwd_bytes, fwd_flops=fwd_flops,
+                bwd_bytes=bwd_bytes if bwd else 0, bwd_flops=bwd_flops if bwd else 0,
+                main_bytes=main_bytes, main_flops=bwd_flops)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def traffic_for(kernel: str, workload: str):
+    """dram read+write bytes per launch from the committed ncu summary, if it was taken on
+    the kernel source as it is now (sha of the .cu file), else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        entries = json.load(f)
+    for e in entries:
+        if e.get("kernel") != kernel or e.get("workload") != workload:
+            continue
+        src = os.path.join(ROOT, e["source"])
+        if not os.path.exists(src):
+            return None
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        return e["bytes_per_launch"] if sha == e.get("source_sha") else None
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.index, self.rows, self.proc = gpu_id, [], None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+                for n, v in zip(names, r[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_oracle_run(B, S, W, bwd, seed=0):
+    """One fp64 oracle pass (forward + full backward) over B x S tokens; returns seconds."""
+    import oracle
+    from global_attention_b200.synth import make_inputs
+    t = make_inputs(B, S, seed=seed, with_dout=bwd)
+    P = oracle.Problem(t["q"], t["k"], t["v"], t["g"], t["gamma_q"], t["gamma_k"], window=W)
+    t0 = time.perf_counter()
+    P.forward()
+    if bwd:
+        P.backward(t["dout"])
+    return time.perf_counter() - t0
+
+
+def cpu_sample_shape(Bw, Sw, W):
+    """A bounded sample of the workload for the oracle: same heads and window, fewer and
+    shorter sequences (window work per token is the same once past the first W tokens)."""
+    if W >= Sw:            # global layer: a shorter causal sequence
+        return 1, 2048, 2048
+    return 4, 2048, W
+
+
+def run_reference(args):
+    """--impl reference: the fp64 CPU oracle as it stands, each step a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    Bw, Sw, W, bwd = WORKLOADS[args.workload]
+    B, S, Wc = (1, 512, 512) if W >= Sw else (1, 1024, W)
+    for _ in range(args.warmup):
+        cpu_oracle_run(B, S, Wc, bwd)
+    times = [cpu_oracle_run(B, S, Wc, bwd, seed=i) for i in range(args.steps)]
+    ms = 1e3 * sum(times) / len(times)
+    val = B * S / (ms / 1e3)
+    cores = oracle.num_threads()
+    sample = f"{B}x{S} tokens per step, window {Wc}, fwd{'+bwd' if bwd else ''}, fp64, {cores} threads"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_name(args.workload), "sample": sample},
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+    return 0
+
+
+def workload_name(w):
+    B, S, W, bwd = WORKLOADS[w]
+    kind = "global (full causal)" if W >= S else f"sliding window W={W}"
+    return f"gated {kind} attention {'fwd+bwd' if bwd else 'fwd'}, B={B} S={S} Hq={HQ} Hkv={HKV} D={D}"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="swa16k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    import global_attention_b200 as ga
+    from global_attention_b200.synth import make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    ga.load()
+
+    Bw, Sw, W, bwd = WORKLOADS[args.workload]
+    wk = work(Bw, Sw, W, bwd)
+    t = make_inputs(Bw, Sw, seed=rank, with_dout=bwd)
+    host = {k: v.pin_memory() for k, v in t.items()}
+    d = {k: v.to(dev) for k, v in host.items()}
+    stream = torch.cuda.current_stream()
+    out = torch.empty_like(d["q"])
+    lse = torch.empty((Bw, HQ, Sw), dtype=torch.float32, device=dev)
+    grads = ws = None
+    if bwd:
+        grads = dict(dq=torch.empty_like(d["q"]), dk=torch.empty_like(d["k"]), dv=torch.empty_like(d["v"]),
+                     dg=torch.empty_like(d["g"]), dgamma_q=torch.empty(D, device=dev),
+                     dgamma_k=torch.empty(D, device=dev))
+        ws = torch.empty(max(256, ga.zgcm_attn_bwd_workspace_size(Bw, Sw, HQ, HKV, D, W)),
+                         dtype=torch.uint8, device=dev)
+
+    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    ev_m = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+
+    def step(i=None, src=d):
+        if i is not None:
+            ev_f[i][0].record(stream)
+        ga.zgcm_attn_fwd(src["q"], src["k"], src["v"], src["g"], src["gamma_q"], src["gamma_k"],
+                         window=W, out=out, lse=lse, stream=stream)
+        if i is not None:
+            ev_f[i][1].record(stream)
+        if bwd:
+            ga.zgcm_attn_bwd(src["q"], src["k"], src["v"], src["g"], src["gamma_q"], src["gamma_k"],
+                             out, lse, src["dout"], window=W, grads=grads, workspace=ws, stream=stream,
+                             main_events=None if i is None else ev_m[i])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, inputs resident in HBM (5.6 GB per step >> 126 MB L2)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_f)
+    main_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_m) if bwd else 0.0
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_step = ms / args.steps
+
+    # ---- end to end through the public API: pinned host inputs -> HBM -> fwd+bwd -> host
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    outs_host = {"out": torch.empty_like(out, device="cpu").pin_memory(),
+                 "lse": torch.empty_like(lse, device="cpu").pin_memory()}
+    if bwd:
+        for k, v in grads.items():
+            outs_host[k] = torch.empty_like(v, device="cpu").pin_memory()
+    d2h = sum(v.numel() * v.element_size() for v in outs_host.values())
+    dst = {k: torch.empty_like(v) for k, v in d.items()}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        for k in dst:
+            dst[k].copy_(host[k], non_blocking=True)
+        step(src=dst)
+        outs_host["out"].copy_(out, non_blocking=True)
+        outs_host["lse"].copy_(lse, non_blocking=True)
+        if bwd:
+            for k, v in grads.items():
+                outs_host[k].copy_(v, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+        dist.barrier()
+
+    if rank != 0:
+        dist.destroy_process_group()
+        return 0
+
+    peaks, peak_src = load_peaks()
+    tokens_step = wk["tokens"] * world
+    value = tokens_step / (ms_step / 1e3)
+    # roofline of the whole step and of the dominant kernel
+    step_bytes = wk["fwd_bytes"] + wk["bwd_bytes"]
+    step_flops = wk["fwd_flops"] + wk["bwd_flops"]
+    t_roof = max(step_bytes / (peaks["hbm_gbs"] * 1e9), step_flops / (peaks["bf16_tflops"] * 1e12))
+    kern = {"fwd_mma_kernel": (fwd_ms, wk["fwd_bytes"], wk["fwd_flops"], "global_attention_b200/csrc/fwd_mma.cu")}
+    if bwd:
+        kern["bwd_main_kernel"] = (main_ms, wk["main_bytes"], wk["main_flops"], "global_attention_b200/csrc/bwd_mma.cu")
+    name = max(kern, key=lambda k: kern[k][0])
+    kms, kbytes, kflops, _ = kern[name]
+    t_hbm = kbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = kflops / (peaks["bf16_tflops_sustained"] * 1e12)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": kbytes / (kms / 1e3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": kflops / (kms / 1e3) / 1e12,
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic_for(name, args.workload)
+    roof.update({"kernel": name, "kernel_ms": kms, "algorithmic_bytes": kbytes, "flops": kflops,
+                 "peak_source": peak_src, "other_kernels_ms": {k: v[0] for k, v in kern.items() if k != name}})
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        Bc, Sc, Wc = cpu_sample_shape(Bw, Sw, W)
+        secs = cpu_oracle_run(Bc, Sc, Wc, bwd)
+        cpu = {"value": Bc * Sc / secs, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+               "sample": f"{Bc}x{Sc} tokens, window {Wc}, fwd{'+bwd' if bwd else ''} in fp64 "
+                         f"({secs:.1f} s); same heads/window as the workload"}
+
+    launches_per_step = 1 + (5 if bwd else 0)   # fwd; pre, main, dq, 2 x d_gamma reduce
+    rec = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) bf16 q,k,v,g,dout; gamma U(0.5,1.5) fp32",
+        "config": {"workload": workload_name(args.workload), "global_batch": Bw * world, "seq_len": Sw,
+                   "window": W, "parallelism": f"dp{world} (independent batches, no collective)",
+                   "l2": f"inputs larger than L2 ({(step_bytes) / 1e9:.2f} GB moved per step)"},
+        "tflops": step_flops / (ms_step / 1e3) / 1e12 * world,
+        "pct_of_roofline": t_roof / (ms_step / 1e3),
+        "roofline_step_ms": t_roof * 1e3,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": tokens_step / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(rec))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,146 @@
+"""ZGCM-1 gated window-attention layer on B200: Python binding of the C ABI.
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels of
+``libzgcm_attn.so`` (built in-tree by ``python -m global_attention_b200.build``).  There is
+no CPU fallback; if the library is missing, loading fails loudly.
+
+The functions carry the C names (include/zgcm_attn.h) and take torch CUDA tensors:
+
+    out, lse = zgcm_attn_fwd(q, k, v, g, gamma_q, gamma_k, window=128)
+    grads = zgcm_attn_bwd(q, k, v, g, gamma_q, gamma_k, out, lse, dout, window=128)
+
+q, g, dout: bf16 [B,S,Hq,128]; k, v: bf16 [B,S,Hkv,128]; gamma_*: fp32 [128].
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libzgcm_attn.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "zgcm_attn.h")
+
+ZGCM_OK = 0
+_lib = None
+
+
+class ZgcmError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {zgcm_status_string(status)} ({status})")
+        self.status = status
+
+
+def load() -> ctypes.CDLL:
+    """Load libzgcm_attn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m global_attention_b200.build` (no CPU fallback exists)")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, i, d, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_float
+        lib.zgcm_status_string.argtypes = [i]
+        lib.zgcm_status_string.restype = ctypes.c_char_p
+        lib.zgcm_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, d, i, i, f, f, vp, vp, vp]
+        lib.zgcm_attn_fwd.restype = i
+        lib.zgcm_attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
+        lib.zgcm_attn_bwd_workspace_size.restype = ctypes.c_size_t
+        lib.zgcm_attn_bwd.argtypes = ([vp] * 9 + [i] * 6 + [d, i, i, f, f] + [vp] * 7 +
+                                      [ctypes.c_size_t, vp])
+        lib.zgcm_attn_bwd.restype = i
+        lib.zgcm_attn_bwd_timed.argtypes = lib.zgcm_attn_bwd.argtypes + [vp, vp]
+        lib.zgcm_attn_bwd_timed.restype = i
+        _lib = lib
+    return _lib
+
+
+def zgcm_status_string(status: int) -> str:
+    return load().zgcm_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(t, name, dtype, ndim):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype or t.dim() != ndim or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous {dtype} tensor of rank {ndim}")
+
+
+def zgcm_attn_fwd(q, k, v, g, gamma_q, gamma_k, *, rope_dims=42, rope_base=10000.0, window=128,
+                  causal=1, eps=1e-6, scale=None, out=None, lse=None, stream=None):
+    """Gated window-attention forward.  Returns (out bf16 [B,S,Hq,D], lse fp32 [B,Hq,S])."""
+    import torch
+    for n, t in (("q", q), ("k", k), ("v", v), ("g", g)):
+        _check(t, n, torch.bfloat16, 4)
+    _check(gamma_q, "gamma_q", torch.float32, 1)
+    _check(gamma_k, "gamma_k", torch.float32, 1)
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    st = load().zgcm_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma_q), _ptr(gamma_k),
+                              B, S, Hq, Hkv, D, int(rope_dims), float(rope_base), int(window),
+                              int(causal), float(eps), float(scale), _ptr(out), _ptr(lse),
+                              _stream(stream))
+    if st != ZGCM_OK:
+        raise ZgcmError(st, "zgcm_attn_fwd")
+    return out, lse
+
+
+def zgcm_attn_bwd_workspace_size(B, S, Hq, Hkv, D=128, window=128) -> int:
+    return int(load().zgcm_attn_bwd_workspace_size(int(B), int(S), int(Hq), int(Hkv), int(D), int(window)))
+
+
+def zgcm_attn_bwd(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dims=42, rope_base=10000.0,
+                  window=128, causal=1, eps=1e-6, scale=None, grads=None, workspace=None, stream=None,
+                  main_events=None):
+    """Gated window-attention backward.  Returns dict dq, dk, dv, dg (bf16) and dgamma_q,
+    dgamma_k (fp32 [D]).  `grads` may supply preallocated outputs, `workspace` a uint8
+    CUDA tensor of at least zgcm_attn_bwd_workspace_size(...) bytes.  `main_events`, a pair
+    of torch.cuda.Event, brackets the main kernel (zgcm_attn_bwd_timed)."""
+    import torch
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    for n, t in (("q", q), ("k", k), ("v", v), ("g", g), ("out", out), ("dout", dout)):
+        _check(t, n, torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
+    if grads is None:
+        grads = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+                     dg=torch.empty_like(g),
+                     dgamma_q=torch.empty(D, dtype=torch.float32, device=q.device),
+                     dgamma_k=torch.empty(D, dtype=torch.float32, device=q.device))
+    need = zgcm_attn_bwd_workspace_size(B, S, Hq, Hkv, D, window)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma_q), _ptr(gamma_k),
+            _ptr(out), _ptr(lse), _ptr(dout), B, S, Hq, Hkv, D, int(rope_dims),
+            float(rope_base), int(window), int(causal), float(eps), float(scale),
+            _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]), _ptr(grads["dg"]),
+            _ptr(grads["dgamma_q"]), _ptr(grads["dgamma_k"]), _ptr(workspace),
+            workspace.numel(), _stream(stream))
+    if main_events is None:
+        st = load().zgcm_attn_bwd(*args)
+    else:
+        ev = [ctypes.c_void_p(e.cuda_event) for e in main_events]
+        st = load().zgcm_attn_bwd_timed(*args, *ev)
+    if st != ZGCM_OK:
+        raise ZgcmError(st, "zgcm_attn_bwd")
+    return grads

@@ -1,0 +1,194 @@
+// zgcm_attn.cu — the C ABI (include/zgcm_attn.h): argument checks, parameter set-up,
+// workspace layout and kernel launches.  Host code only; the kernels live in the other
+// .cu files of this directory.
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/zgcm_attn.h"
+#include "common.cuh"
+
+namespace zgcm {
+cudaError_t launch_fwd_mma(const FwdParams& p, cudaStream_t stream);
+cudaError_t launch_bwd_mma(const BwdParams& p, cudaStream_t stream, cudaEvent_t ev0, cudaEvent_t ev1);
+int bwd_mma_n_k_parts(int B, int S, int Hkv);
+long long bwd_mma_n_q_parts(int B, int S, int Hq);
+}  // namespace zgcm
+
+using namespace zgcm;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks shared by forward and backward.  Returns ZGCM_OK or the first failing status.
+int check_shape(int B, int S, int Hq, int Hkv, int D, int rope_dims, double rope_base, int window,
+                int causal, float eps, float scale) {
+    if (B < 0 || S < 0 || Hq < 1 || Hkv < 1 || D < 1) return ZGCM_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return ZGCM_ERR_INVALID_ARG;
+    if (rope_dims < 0 || rope_dims > D || (rope_dims & 1)) return ZGCM_ERR_INVALID_ARG;
+    if (rope_dims > 0 && !(rope_base > 0.0 && isfinite(rope_base))) return ZGCM_ERR_INVALID_ARG;
+    if (window < 1) return ZGCM_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || !isfinite(eps)) return ZGCM_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !isfinite(scale)) return ZGCM_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return ZGCM_ERR_INVALID_ARG;
+    if (causal == 0) return ZGCM_ERR_UNSUPPORTED;  // the pages describe causal layers only
+    if (D != kD) return ZGCM_ERR_UNSUPPORTED;
+    if ((long double)B * S * Hq * D >= (long double)(1ULL << 40)) return ZGCM_ERR_UNSUPPORTED;
+    return ZGCM_OK;
+}
+
+void fill_layer(LayerParams& L, const void* q, const void* k, const void* v, const void* g,
+                const float* gamma_q, const float* gamma_k, int B, int S, int Hq, int Hkv,
+                int rope_dims, double rope_base, int window, float eps, float scale) {
+    L.q = static_cast<const bf16*>(q);
+    L.k = static_cast<const bf16*>(k);
+    L.v = static_cast<const bf16*>(v);
+    L.g = static_cast<const bf16*>(g);
+    L.gamma_q = gamma_q;
+    L.gamma_k = gamma_k;
+    L.B = B; L.S = S; L.Hq = Hq; L.Hkv = Hkv; L.G = Hq / Hkv;
+    L.rope_half = rope_dims / 2;
+    L.W = window;
+    L.eps = eps;
+    L.scale = scale;
+    L.scale_log2 = scale * kLog2e;
+    for (int t = 0; t < kMaxHalf; ++t)
+        L.theta[t] = t < L.rope_half ? pow(rope_base, -2.0 * (double)t / (double)rope_dims) : 0.0;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct BwdWorkspace {
+    size_t delta, dA, dq_acc, dgk, dgq, total;
+    int n_k_parts;
+    long long n_q_parts;
+};
+
+BwdWorkspace bwd_layout(int B, int S, int Hq, int Hkv) {
+    BwdWorkspace w;
+    const size_t rows = (size_t)B * S * Hq;
+    w.n_k_parts = bwd_mma_n_k_parts(B, S, Hkv);
+    w.n_q_parts = bwd_mma_n_q_parts(B, S, Hq);
+    size_t off = 0;
+    w.delta = off; off = align256(off + rows * sizeof(float));
+    w.dA = off;    off = align256(off + rows * kD * sizeof(bf16));
+    w.dq_acc = off; off = align256(off + rows * kD * sizeof(float));
+    w.dgk = off;   off = align256(off + (size_t)w.n_k_parts * kD * sizeof(float));
+    w.dgq = off;   off = align256(off + (size_t)w.n_q_parts * kD * sizeof(float));
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* zgcm_status_string(int status) {
+    switch (status) {
+        case ZGCM_OK: return "ZGCM_OK";
+        case ZGCM_ERR_INVALID_ARG: return "ZGCM_ERR_INVALID_ARG: invalid argument";
+        case ZGCM_ERR_UNSUPPORTED: return "ZGCM_ERR_UNSUPPORTED: valid but unsupported configuration";
+        case ZGCM_ERR_ALIGNMENT: return "ZGCM_ERR_ALIGNMENT: tensor pointer not 16-byte aligned";
+        case ZGCM_ERR_WORKSPACE: return "ZGCM_ERR_WORKSPACE: workspace missing or too small";
+        case ZGCM_ERR_CUDA: return "ZGCM_ERR_CUDA: CUDA runtime or launch failure";
+        case ZGCM_ERR_TIMEOUT: return "ZGCM_ERR_TIMEOUT: bounded device wait expired";
+        default: return "unknown zgcm_status";
+    }
+}
+
+int zgcm_attn_fwd(const void* q, const void* k, const void* v, const void* g,
+                  const float* gamma_q, const float* gamma_k,
+                  int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                  double rope_base, int window, int causal, float eps, float scale,
+                  void* out, float* lse, void* cuda_stream) {
+    int st = check_shape(B, S, Hq, Hkv, D, rope_dims, rope_base, window, causal, eps, scale);
+    if (st != ZGCM_OK) return st;
+    if ((long long)B * S == 0) return ZGCM_OK;
+    const void* ptrs[] = {q, k, v, g, gamma_q, gamma_k, out, lse};
+    for (const void* p : ptrs)
+        if (!p) return ZGCM_ERR_INVALID_ARG;
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return ZGCM_ERR_ALIGNMENT;
+    FwdParams p;
+    fill_layer(p.L, q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, rope_dims, rope_base, window, eps, scale);
+    p.out = static_cast<bf16*>(out);
+    p.lse = lse;
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    return launch_fwd_mma(p, stream) == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
+}
+
+size_t zgcm_attn_bwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int window) {
+    if (check_shape(B, S, Hq, Hkv, D, 0, 1.0, window, 1, 0.f, 1.f) != ZGCM_OK) return 0;
+    if ((long long)B * S == 0) return 0;
+    return bwd_layout(B, S, Hq, Hkv).total;
+}
+
+int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void* g,
+                        const float* gamma_q, const float* gamma_k,
+                        const void* out, const float* lse, const void* dout,
+                        int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                        double rope_base, int window, int causal, float eps, float scale,
+                        void* dq, void* dk, void* dv, void* dg,
+                        float* dgamma_q, float* dgamma_k,
+                        void* workspace, size_t workspace_bytes, void* cuda_stream,
+                        void* ev_main_begin, void* ev_main_end) {
+    int st = check_shape(B, S, Hq, Hkv, D, rope_dims, rope_base, window, causal, eps, scale);
+    if (st != ZGCM_OK) return st;
+    if (!dgamma_q || !dgamma_k) return ZGCM_ERR_INVALID_ARG;
+    if (!aligned16(dgamma_q) || !aligned16(dgamma_k)) return ZGCM_ERR_ALIGNMENT;
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    if ((long long)B * S == 0) {
+        if (cudaMemsetAsync(dgamma_q, 0, kD * sizeof(float), stream) != cudaSuccess) return ZGCM_ERR_CUDA;
+        if (cudaMemsetAsync(dgamma_k, 0, kD * sizeof(float), stream) != cudaSuccess) return ZGCM_ERR_CUDA;
+        return ZGCM_OK;
+    }
+    const void* ptrs[] = {q, k, v, g, gamma_q, gamma_k, out, lse, dout, dq, dk, dv, dg};
+    for (const void* p : ptrs)
+        if (!p) return ZGCM_ERR_INVALID_ARG;
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return ZGCM_ERR_ALIGNMENT;
+    const BwdWorkspace w = bwd_layout(B, S, Hq, Hkv);
+    if (!workspace || workspace_bytes < w.total) return ZGCM_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ZGCM_ERR_ALIGNMENT;
+    if (w.n_q_parts > 0x7fffffffLL) return ZGCM_ERR_UNSUPPORTED;
+
+    BwdParams p;
+    fill_layer(p.L, q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, rope_dims, rope_base, window, eps, scale);
+    p.out = static_cast<const bf16*>(out);
+    p.lse = lse;
+    p.dout = static_cast<const bf16*>(dout);
+    p.dq = static_cast<bf16*>(dq);
+    p.dk = static_cast<bf16*>(dk);
+    p.dv = static_cast<bf16*>(dv);
+    p.dg = static_cast<bf16*>(dg);
+    p.dgamma_q = dgamma_q;
+    p.dgamma_k = dgamma_k;
+    char* ws = static_cast<char*>(workspace);
+    p.delta = reinterpret_cast<float*>(ws + w.delta);
+    p.dA = reinterpret_cast<bf16*>(ws + w.dA);
+    p.dq_acc = reinterpret_cast<float*>(ws + w.dq_acc);
+    p.dgk_part = reinterpret_cast<float*>(ws + w.dgk);
+    p.dgq_part = reinterpret_cast<float*>(ws + w.dgq);
+    p.n_k_parts = w.n_k_parts;
+    p.n_q_parts = (int)w.n_q_parts;
+    return launch_bwd_mma(p, stream, static_cast<cudaEvent_t>(ev_main_begin),
+                          static_cast<cudaEvent_t>(ev_main_end)) == cudaSuccess
+               ? ZGCM_OK
+               : ZGCM_ERR_CUDA;
+}
+
+int zgcm_attn_bwd(const void* q, const void* k, const void* v, const void* g,
+                  const float* gamma_q, const float* gamma_k,
+                  const void* out, const float* lse, const void* dout,
+                  int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                  double rope_base, int window, int causal, float eps, float scale,
+                  void* dq, void* dk, void* dv, void* dg,
+                  float* dgamma_q, float* dgamma_k,
+                  void* workspace, size_t workspace_bytes, void* cuda_stream) {
+    return zgcm_attn_bwd_timed(q, k, v, g, gamma_q, gamma_k, out, lse, dout, B, S, Hq, Hkv, D,
+                               rope_dims, rope_base, window, causal, eps, scale, dq, dk, dv, dg,
+                               dgamma_q, dgamma_k, workspace, workspace_bytes, cuda_stream,
+                               nullptr, nullptr);
+}
+
+}  // extern "C"

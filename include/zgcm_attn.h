@@ -113,6 +113,22 @@ int zgcm_attn_bwd(const void* q, const void* k, const void* v, const void* g,
                   float* dgamma_q, float* dgamma_k,
                   void* workspace, size_t workspace_bytes, void* cuda_stream);
 
+/*
+ * Measurement variant of zgcm_attn_bwd: the same work on the same stream, and in addition
+ * records ev_main_begin / ev_main_end (cudaEvent_t created by the caller) immediately
+ * before and after the backward's main kernel (the key-major pass that forms dK, dV and
+ * the dQ accumulation), so that kernel can be timed on its own.  Either event may be NULL.
+ */
+int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void* g,
+                        const float* gamma_q, const float* gamma_k,
+                        const void* out, const float* lse, const void* dout,
+                        int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                        double rope_base, int window, int causal, float eps, float scale,
+                        void* dq, void* dk, void* dv, void* dg,
+                        float* dgamma_q, float* dgamma_k,
+                        void* workspace, size_t workspace_bytes, void* cuda_stream,
+                        void* ev_main_begin, void* ev_main_end);
+
 #ifdef __cplusplus
 }
 #endif

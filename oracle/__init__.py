@@ -99,6 +99,10 @@ class Problem:
                           B, S, Hq, Hkv, D, int(rope_dims), int(window), float(rope_base),
                           float(eps), float(scale))
 
+    def set_window(self, window: int):
+        """Reuse the upcast inputs for another window size."""
+        self.c.W = int(window)
+
     def _rows(self, rows):
         if rows is None:
             return None, self.shape[0] * self.shape[1]

@@ -1,0 +1,111 @@
+"""C-ABI library: loads, exports every declared symbol, and rejects bad arguments on the
+host before any launch.  CPU only: no call here reaches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import global_attention_b200 as ga
+from global_attention_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return ga.load()
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(zgcm_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert {"zgcm_attn_fwd", "zgcm_attn_bwd", "zgcm_attn_bwd_workspace_size",
+            "zgcm_status_string"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+        getattr(lib, n)  # resolves through dlsym
+
+
+def test_status_strings(lib):
+    for st in (0, -1, -2, -3, -4, -5, -6):
+        assert ga.zgcm_status_string(st).startswith("ZGCM_")
+    assert "unknown" in ga.zgcm_status_string(12345)
+
+
+# fake, 256-byte aligned, never dereferenced: every call below fails validation first
+P = 0x7F0000000000
+ARGS = dict(B=1, S=64, Hq=32, Hkv=8, D=128, rope_dims=42, rope_base=10000.0, window=128, causal=1,
+            eps=1e-6, scale=0.0883883)
+
+
+def _fwd(lib, ptrs=None, **kw):
+    a = dict(ARGS, **kw)
+    p = ptrs or [P + 256 * i for i in range(8)]
+    vp = ctypes.c_void_p
+    return lib.zgcm_attn_fwd(*(vp(x) for x in p[:6]), a["B"], a["S"], a["Hq"], a["Hkv"], a["D"],
+                             a["rope_dims"], a["rope_base"], a["window"], a["causal"], a["eps"],
+                             a["scale"], vp(p[6]), vp(p[7]), None)
+
+
+def _bwd(lib, ws_bytes, ws=P + 256 * 40, **kw):
+    a = dict(ARGS, **kw)
+    vp = ctypes.c_void_p
+    p = [vp(P + 256 * i) for i in range(15)]
+    return lib.zgcm_attn_bwd(*p[:9], a["B"], a["S"], a["Hq"], a["Hkv"], a["D"], a["rope_dims"],
+                             a["rope_base"], a["window"], a["causal"], a["eps"], a["scale"],
+                             *p[9:15], vp(ws), ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=64), -2), (dict(causal=0), -2), (dict(causal=2), -1), (dict(Hq=30), -1),
+    (dict(window=0), -1), (dict(rope_dims=41), -1), (dict(rope_dims=130), -1),
+    (dict(eps=-1.0), -1), (dict(scale=0.0), -1), (dict(scale=float("nan")), -1),
+    (dict(B=-1), -1), (dict(S=-5), -1), (dict(Hkv=0), -1), (dict(rope_base=0.0), -1),
+])
+def test_fwd_rejects_bad_arguments(lib, kw, status):
+    assert _fwd(lib, **kw) == status
+
+
+def test_fwd_pointer_checks(lib):
+    good = [P + 256 * i for i in range(8)]
+    for i in range(8):
+        p = list(good); p[i] = 0
+        assert _fwd(lib, ptrs=p) == -1
+        p = list(good); p[i] = good[i] + 8
+        assert _fwd(lib, ptrs=p) == -3
+
+
+def test_bwd_workspace_checks(lib):
+    need = lib.zgcm_attn_bwd_workspace_size(1, 64, 32, 8, 128, 128)
+    assert need > 0
+    assert _bwd(lib, need - 1) == -4
+    assert _bwd(lib, need, ws=0) == -4
+    assert _bwd(lib, need, ws=P + 256 * 40 + 16) == -3
+    assert _bwd(lib, need, D=100) == -2
+
+
+def test_workspace_size_query(lib):
+    ws = lambda *a: lib.zgcm_attn_bwd_workspace_size(*a)
+    assert ws(0, 64, 32, 8, 128, 128) == 0
+    assert ws(1, 0, 32, 8, 128, 128) == 0
+    assert ws(1, 64, 32, 8, 64, 128) == 0   # unsupported D -> 0
+    assert ws(4, 16384, 32, 8, 128, 128) > ws(1, 16384, 32, 8, 128, 128) > ws(1, 1024, 32, 8, 128, 128)
+    assert ws(1, 1024, 32, 8, 128, 128) % 256 == 0
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(ga, "_lib", None)
+    monkeypatch.setattr(ga, "LIB_PATH", "/nonexistent/libzgcm_attn.so")
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        ga.load()

@@ -1,0 +1,188 @@
+"""GPU vs fp64 oracle, element by element, through the C ABI (needs a B200).
+
+Small and ragged shapes are compared in full (every output element); the full-size
+workloads of the layer (16K SWA fwd/bwd, 64K global fwd+bwd, 256K SWA and global fwd)
+are compared on sampled rows the oracle computes one by one, plus properties that hold
+at any size.
+"""
+import numpy as np
+import pytest
+import torch
+
+import global_attention_b200 as ga
+import oracle
+from global_attention_b200.synth import make_inputs, sample_query_rows
+from tests.parity_util import (assert_bf16_close, assert_dgamma_close, assert_lse_close, f64)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    ga.load()
+    oracle.build()
+
+
+def _to_dev(t):
+    return {k: v.cuda() for k, v in t.items()}
+
+
+def _gpu_fwd(d, **kw):
+    out, lse = ga.zgcm_attn_fwd(d["q"], d["k"], d["v"], d["g"], d["gamma_q"], d["gamma_k"], **kw)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def _gpu_bwd(d, out, lse, **kw):
+    gr = ga.zgcm_attn_bwd(d["q"], d["k"], d["v"], d["g"], d["gamma_q"], d["gamma_k"], out, lse,
+                          d["dout"], **kw)
+    torch.cuda.synchronize()
+    return gr
+
+
+def _problem(t, **kw):
+    return oracle.Problem(t["q"], t["k"], t["v"], t["g"], t["gamma_q"], t["gamma_k"], **kw)
+
+
+SMALL = [
+    # B, S, Hq, Hkv, W, rope_dims, base
+    (1, 1024, 32, 8, 128, 42, 1e4),      # the tiny SWA workload of the layer
+    (2, 1000, 32, 8, 128, 42, 1e4),      # ragged tail, two sequences
+    (1, 129, 32, 8, 128, 42, 1e4),       # one tile + one row
+    (1, 1, 32, 8, 128, 42, 1e4),         # single token
+    (1, 300, 8, 8, 1, 42, 1e4),          # self-only window, no GQA sharing
+    (1, 333, 4, 1, 2, 128, 1e7),         # two-key window, full rotation, 10M base
+    (1, 777, 32, 8, 777, 42, 1e4),       # global layer (W = S), ragged
+    (1, 500, 16, 4, 10**6, 0, 1e4),      # global, W >> S, no rotation
+    (3, 260, 32, 8, 200, 42, 1e4),       # window between one and two tiles
+]
+
+
+@pytest.mark.parametrize("B,S,Hq,Hkv,W,R,base", SMALL)
+def test_small_full_compare(B, S, Hq, Hkv, W, R, base):
+    t = make_inputs(B, S, Hq=Hq, Hkv=Hkv, seed=B * 7 + S + W % 97, with_dout=True)
+    kw = dict(window=W, rope_dims=R, rope_base=base)
+    d = _to_dev(t)
+    out, lse = _gpu_fwd(d, **kw)
+    P = _problem(t, **kw)
+    ref_out, ref_lse = P.forward()
+    assert_bf16_close("out", out, ref_out)
+    assert_lse_close("lse", lse, ref_lse)
+    gr = _gpu_bwd(d, out, lse, **kw)
+    ref = P.backward(t["dout"])
+    for n in ("dq", "dk", "dv", "dg"):
+        assert_bf16_close(n, gr[n], ref[n])
+    assert_dgamma_close("dgamma_q", gr["dgamma_q"], ref["dgamma_q"])
+    assert_dgamma_close("dgamma_k", gr["dgamma_k"], ref["dgamma_k"])
+
+
+def test_empty_problem():
+    for B, S in ((0, 16), (2, 0)):
+        t = make_inputs(max(B, 1), max(S, 1), with_dout=True)
+        d = {k: (v[:B, :S].contiguous().cuda() if v.dim() == 4 else v.cuda()) for k, v in t.items()}
+        out, lse = _gpu_fwd(d)
+        assert out.numel() == 0 and lse.numel() == 0
+        gr = _gpu_bwd(d, out, lse)
+        assert torch.all(gr["dgamma_q"] == 0) and torch.all(gr["dgamma_k"] == 0)
+
+
+def test_gate_limits_and_nan():
+    t = make_inputs(1, 256, seed=3, with_dout=True)
+    g = t["g"].clone()
+    g[0, :, 0, :] = float("inf")
+    g[0, :, 1, :] = float("-inf")
+    g[0, 17, 2, 5] = float("nan")
+    t["g"] = g
+    d = _to_dev(t)
+    out, lse = _gpu_fwd(d)
+    ref_out, _ = _problem(t).forward()
+    o = f64(out)
+    assert np.isnan(o[0, 17, 2, 5]) and np.isnan(ref_out[0, 17, 2, 5])
+    mask = np.ones(o.shape, bool)
+    mask[0, 17, 2, 5] = False
+    assert_bf16_close("out(g=+-inf)", o[mask], ref_out[mask])
+    assert np.all(o[0, :, 1, :] == 0.0)
+
+
+def test_forward_bitwise_repeatable():
+    t = make_inputs(2, 2048, seed=5)
+    d = _to_dev(t)
+    o1, l1 = _gpu_fwd(d)
+    o2, l2 = _gpu_fwd(d)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def _sampled_fwd_bwd(B, S, W, n_random, k_rows, check_bwd=True, seed=0, edge=256):
+    t = make_inputs(B, S, seed=seed, with_dout=check_bwd)
+    d = _to_dev(t)
+    out, lse = _gpu_fwd(d, window=W)
+    gr = _gpu_bwd(d, out, lse, window=W) if check_bwd else None
+    P = _problem(t, window=W)
+    rows = sample_query_rows(B, S, n_random=n_random, edge=edge, seed=seed)
+    b, i = rows // S, rows % S
+    ref_out, ref_lse = P.forward(rows)
+    assert_bf16_close("out[rows]", f64(out)[b, i], ref_out)
+    assert_lse_close("lse[rows]", f64(lse)[b, :, i], ref_lse)
+    if not check_bwd:
+        return
+    dq, dg = P.backward_qrows(t["dout"], rows)
+    assert_bf16_close("dq[rows]", f64(gr["dq"])[b, i], dq)
+    assert_bf16_close("dg[rows]", f64(gr["dg"])[b, i], dg)
+    kb, ki = k_rows // S, k_rows % S
+    dk, dv = P.backward_krows(t["dout"], k_rows)
+    assert_bf16_close("dk[rows]", f64(gr["dk"])[kb, ki], dk)
+    assert_bf16_close("dv[rows]", f64(gr["dv"])[kb, ki], dv)
+    # any-size properties: sum_j dv_j = sum_{h in group, i} dout_i * sigmoid(g_i)
+    G = t["q"].shape[2] // t["k"].shape[2]
+    dA = (d["dout"].double() * torch.sigmoid(d["g"].double()))
+    rhs = dA.view(B, S, -1, G, 128).sum(dim=(1, 3))
+    lhs = gr["dv"].double().sum(dim=1)
+    assert_bf16_close("sum_j dv", lhs, rhs, atol=2e-2 * float(rhs.abs().max()) + 2e-2)
+    # gamma_q . dgamma_q = gamma_k . dgamma_k (scores are invariant to q_hat*c, k_hat/c)
+    a = float((gr["dgamma_q"].double() * d["gamma_q"].double()).sum())
+    c = float((gr["dgamma_k"].double() * d["gamma_k"].double()).sum())
+    assert abs(a - c) <= 5e-3 * max(abs(a), abs(c)) + 1e-3, (a, c)
+
+
+def test_swa_16k_forward_backward():
+    """B=4, S=16384, W=128: forward and backward on sampled rows + properties."""
+    B, S = 4, 16384
+    rng = np.random.default_rng(1)
+    k_rows = np.unique(np.concatenate([np.arange(0, 64), np.arange(S * B - 64, S * B),
+                                       rng.integers(0, B * S, 128)]))
+    _sampled_fwd_bwd(B, S, 128, n_random=512, k_rows=k_rows)
+
+
+def test_global_64k_forward_backward():
+    """Global layer: B=1, S=65536, W=S, sampled rows (rows late in the sequence cost the
+    oracle O(S) each, so fewer of them) + properties."""
+    S = 65536
+    k_rows = np.arange(S - 48, S)
+    _sampled_fwd_bwd(1, S, S, n_random=24, k_rows=k_rows, edge=12)
+
+
+def test_256k_swa_and_global_forward():
+    import psutil
+    if psutil.virtual_memory().available < 96e9:
+        pytest.skip("needs ~40 GB of host RAM for the fp64 oracle arrays at S=262144")
+    S = 262144
+    t = make_inputs(1, S, seed=0)
+    d = _to_dev(t)
+    P = _problem(t, window=128)
+    rows = sample_query_rows(1, S, n_random=256, edge=256, seed=0)
+    out, lse = _gpu_fwd(d, window=128)
+    ro, rl = P.forward(rows)
+    assert_bf16_close("swa out[rows]", f64(out)[0, rows], ro)
+    assert_lse_close("swa lse[rows]", f64(lse)[0, :, rows], rl)
+    del out, lse
+    out, lse = _gpu_fwd(d, window=S)
+    grows = np.unique(np.concatenate([np.arange(0, 64), np.arange(S - 3, S),
+                                      np.random.default_rng(2).integers(0, S, 5)]))
+    P.set_window(S)
+    ro, rl = P.forward(grows)
+    assert_bf16_close("global out[rows]", f64(out)[0, grows], ro)
+    assert_lse_close("global lse[rows]", f64(lse)[0, :, grows], rl)
