@@ -60,12 +60,21 @@ def work(B, S, W, bwd):
     fwd_flops = 4 * D * npair
     bwd_bytes = 4 * qb + 2 * kb + lse + 2 * qb + 2 * kb  # read q,k,v,g,out,dout,lse; write dq,dk,dv,dg
     bwd_flops = 10 * D * npair
-    # main backward kernel of this build: reads q, k, v, dA (bf16), lse, Delta;
-    # writes dk, dv and the fp32 dQ~ accumulation (each counted once)
-    main_bytes = qb + 2 * kb + qb + 2 * lse + 2 * kb + tok * HQ * D * 4
+    # per kernel of this build: (algorithmic bytes = each input read once and each output
+    # written once at its stored type, masked FLOPs of the products the kernel's job needs)
+    kernels = {
+        "fwd_mma_kernel": (fwd_bytes, fwd_flops),
+        "fwd_tc_kernel": (fwd_bytes, fwd_flops),
+        # dout, out, g -> dg, dA
+        "bwd_pre_kernel": (5 * qb, 0),
+        # q, k, v, dA, lse -> dq, Delta ; S, dP, dQ
+        "bwd_dq_kernel": (qb + 2 * kb + qb + lse + qb + lse, 6 * D * npair),
+        # q, k, v, dA, lse, Delta -> dk, dv ; S, dP, dV, dK
+        "bwd_main_kernel": (qb + 2 * kb + qb + 2 * lse + 2 * kb, 8 * D * npair),
+    }
     return dict(tokens=tok, npair=npair, fwd_bytes=fwd_bytes, fwd_flops=fwd_flops,
                 bwd_bytes=bwd_bytes if bwd else 0, bwd_flops=bwd_flops if bwd else 0,
-                main_bytes=main_bytes, main_flops=bwd_flops)
+                kernels=kernels)
 
 
 def load_peaks():
@@ -251,8 +260,9 @@ def main():
 
     ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(args.steps)]
-    ev_m = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
+    bwd_names = ga.zgcm_attn_bwd_kernel_names(Sw, W) if bwd else []
+    ev_m = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in bwd_names] for _ in range(args.steps)]
 
     def step(i=None, src=d):
         if i is not None:
@@ -264,7 +274,7 @@ def main():
         if bwd:
             ga.zgcm_attn_bwd(src["q"], src["k"], src["v"], src["g"], src["gamma_q"], src["gamma_k"],
                              out, lse, src["dout"], window=W, grads=grads, workspace=ws, stream=stream,
-                             main_events=None if i is None else ev_m[i])
+                             kernel_events=None if i is None else ev_m[i])
 
     for _ in range(args.warmup):
         step()
@@ -285,7 +295,10 @@ def main():
         dist.barrier()
     ms = t0.elapsed_time(t1)
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_f)
-    main_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_m) if bwd else 0.0
+    fwd_name = ga.zgcm_attn_fwd_kernel_name(Bw, Sw, HQ, HKV, 42, W)
+    kern_ms = {fwd_name: fwd_ms}
+    for k, n in enumerate(bwd_names):
+        kern_ms[n] = statistics.mean(ev_m[i][k][0].elapsed_time(ev_m[i][k][1]) for i in range(args.steps))
     if world > 1:
         tt = torch.tensor([ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -335,11 +348,9 @@ def main():
     step_bytes = wk["fwd_bytes"] + wk["bwd_bytes"]
     step_flops = wk["fwd_flops"] + wk["bwd_flops"]
     t_roof = max(step_bytes / (peaks["hbm_gbs"] * 1e9), step_flops / (peaks["bf16_tflops"] * 1e12))
-    kern = {"fwd_mma_kernel": (fwd_ms, wk["fwd_bytes"], wk["fwd_flops"], "global_attention_b200/csrc/fwd_mma.cu")}
-    if bwd:
-        kern["bwd_main_kernel"] = (main_ms, wk["main_bytes"], wk["main_flops"], "global_attention_b200/csrc/bwd_mma.cu")
+    kern = {n: (ms_, *wk["kernels"][n]) for n, ms_ in kern_ms.items() if n in wk["kernels"]}
     name = max(kern, key=lambda k: kern[k][0])
-    kms, kbytes, kflops, _ = kern[name]
+    kms, kbytes, kflops = kern[name]
     t_hbm = kbytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = kflops / (peaks["bf16_tflops_sustained"] * 1e12)
     if t_hbm >= t_tc:
@@ -350,7 +361,7 @@ def main():
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = traffic_for(name, args.workload)
     roof.update({"kernel": name, "kernel_ms": kms, "algorithmic_bytes": kbytes, "flops": kflops,
-                 "peak_source": peak_src, "other_kernels_ms": {k: v[0] for k, v in kern.items() if k != name}})
+                 "peak_source": peak_src, "kernels_ms": kern_ms})
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -362,7 +373,7 @@ def main():
                "sample": f"{Bc}x{Sc} tokens, window {Wc}, fwd{'+bwd' if bwd else ''} in fp64 "
                          f"({secs:.1f} s); same heads/window as the workload"}
 
-    launches_per_step = 1 + (5 if bwd else 0)   # fwd; pre, main, dq, 2 x d_gamma reduce
+    launches_per_step = 1 + len(bwd_names)     # fwd + every backward kernel
     rec = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",

@@ -49,8 +49,14 @@ def load() -> ctypes.CDLL:
         lib.zgcm_attn_bwd.argtypes = ([vp] * 9 + [i] * 6 + [d, i, i, f, f] + [vp] * 7 +
                                       [ctypes.c_size_t, vp])
         lib.zgcm_attn_bwd.restype = i
-        lib.zgcm_attn_bwd_timed.argtypes = lib.zgcm_attn_bwd.argtypes + [vp, vp]
+        lib.zgcm_attn_bwd_timed.argtypes = lib.zgcm_attn_bwd.argtypes + [ctypes.POINTER(vp), i]
         lib.zgcm_attn_bwd_timed.restype = i
+        lib.zgcm_attn_bwd_kernel_name.argtypes = [i, i, i]
+        lib.zgcm_attn_bwd_kernel_name.restype = ctypes.c_char_p
+        lib.zgcm_attn_fwd_kernel_name.argtypes = [i, i, i, i, i, i]
+        lib.zgcm_attn_fwd_kernel_name.restype = ctypes.c_char_p
+        lib.zgcm_attn_device_error.argtypes = []
+        lib.zgcm_attn_device_error.restype = i
         _lib = lib
     return _lib
 
@@ -107,13 +113,36 @@ def zgcm_attn_bwd_workspace_size(B, S, Hq, Hkv, D=128, window=128) -> int:
     return int(load().zgcm_attn_bwd_workspace_size(int(B), int(S), int(Hq), int(Hkv), int(D), int(window)))
 
 
+def zgcm_attn_fwd_kernel_name(B, S, Hq, Hkv, rope_dims=42, window=128) -> str:
+    """Name of the kernel zgcm_attn_fwd launches for this configuration."""
+    return load().zgcm_attn_fwd_kernel_name(int(B), int(S), int(Hq), int(Hkv), int(rope_dims),
+                                            int(window)).decode()
+
+
+def zgcm_attn_device_error() -> int:
+    """ZGCM_OK, or ZGCM_ERR_TIMEOUT if a bounded device wait expired since the last call."""
+    return int(load().zgcm_attn_device_error())
+
+
+def zgcm_attn_bwd_kernel_names(S, window):
+    """Names of the kernels zgcm_attn_bwd launches, in order."""
+    names, i = [], 0
+    while True:
+        n = load().zgcm_attn_bwd_kernel_name(i, int(S), int(window))
+        if n is None:
+            return names
+        names.append(n.decode())
+        i += 1
+
+
 def zgcm_attn_bwd(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dims=42, rope_base=10000.0,
                   window=128, causal=1, eps=1e-6, scale=None, grads=None, workspace=None, stream=None,
-                  main_events=None):
+                  kernel_events=None):
     """Gated window-attention backward.  Returns dict dq, dk, dv, dg (bf16) and dgamma_q,
     dgamma_k (fp32 [D]).  `grads` may supply preallocated outputs, `workspace` a uint8
-    CUDA tensor of at least zgcm_attn_bwd_workspace_size(...) bytes.  `main_events`, a pair
-    of torch.cuda.Event, brackets the main kernel (zgcm_attn_bwd_timed)."""
+    CUDA tensor of at least zgcm_attn_bwd_workspace_size(...) bytes.  `kernel_events`, a list
+    of (begin, end) torch.cuda.Event pairs, brackets the backward's kernels in launch order
+    (zgcm_attn_bwd_timed; names from zgcm_attn_bwd_kernel_names)."""
     import torch
     B, S, Hq, D = q.shape
     Hkv = k.shape[2]
@@ -136,11 +165,12 @@ def zgcm_attn_bwd(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dims=42,
             _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]), _ptr(grads["dg"]),
             _ptr(grads["dgamma_q"]), _ptr(grads["dgamma_k"]), _ptr(workspace),
             workspace.numel(), _stream(stream))
-    if main_events is None:
+    if kernel_events is None:
         st = load().zgcm_attn_bwd(*args)
     else:
-        ev = [ctypes.c_void_p(e.cuda_event) for e in main_events]
-        st = load().zgcm_attn_bwd_timed(*args, *ev)
+        flat = [ctypes.c_void_p(e.cuda_event) for pair in kernel_events for e in pair]
+        arr = (ctypes.c_void_p * max(1, len(flat)))(*flat)
+        st = load().zgcm_attn_bwd_timed(*args, arr, len(kernel_events))
     if st != ZGCM_OK:
         raise ZgcmError(st, "zgcm_attn_bwd")
     return grads

@@ -3,14 +3,29 @@
 // ZGCM-1 layer (definition and page citations in common.cuh).
 //
 // Kernels, in launch order:
-//   bwd_pre     per (b, s, h) row: Delta = sum_d dout*out; dg = dout*out*(1-sigmoid(g));
-//               dA = dout*sigmoid(g)   (out = sigmoid(g)*A, so neither needs A itself)
+//   bwd_pre     per (b, s, h) row: dg = dout*out*(1-sigmoid(g)); dA = dout*sigmoid(g)
+//               (out = sigmoid(g)*A, so neither needs the pre-gate A itself).  dA is kept
+//               as a pair of bf16 values hi + lo (hi = bf16(dA), lo = bf16(dA - hi)), and
+//               every product with dA is taken as hi-product + lo-product: with dA rounded
+//               to one bf16 the worst dk element near the sequence start was off by ~1.5x
+//               the final bf16 rounding.
+//   bwd_dq      per (b, query head, 64-query tile), two passes over the key tiles its window
+//               reaches: pass 1 forms Delta = sum_j P dP (P = exp(S - lse), dP = dA V^T);
+//               pass 2 forms dS = P (dP - Delta) and dQ~ = scale dS K~.  Epilogue: dq =
+//               RMSNorm/RoPE backward of dQ~, d_gamma_q partials; Delta saved for bwd_main.
+//               Delta is formed from the same P and dP the kernels use, not from the bf16
+//               `out`: rounding out and dA separately made Delta inconsistent with dP and
+//               roughly doubled the worst-case gradient error.  (A one-pass form,
+//               dQ~ = sum_j P dP k~_j - Delta sum_j P k~_j, cancels badly where the softmax
+//               is peaked and dS ~ 0, e.g. a one-key window.)
 //   bwd_main    per (b, KV head, 64-key tile), over the Hq/Hkv query heads of the group and
 //               every 64-query tile whose window reaches the keys:
 //                 P^T = exp(S^T - lse), dV += P^T dA, dP^T = V dA^T, dS^T = P^T (dP^T - Delta),
-//                 dK~ += dS^T Q~, dQ~ += dS K~ (fp32 atomics into the workspace);
-//               epilogue: dk = RMSNorm/RoPE backward of scale*dK~, dv, d_gamma_k partials
-//   bwd_dq      per row: dq = RMSNorm/RoPE backward of scale*dQ~, d_gamma_q partials
+//                 dK~ += dS^T Q~;  epilogue: dk = RMSNorm/RoPE backward of scale*dK~, dv,
+//                 d_gamma_k partials.  P is split hi + lo like dA for the dV product
+//                 (P_hi dA_hi + P_hi dA_lo + P_lo dA_hi): the largest dv entries sit where
+//                 few keys share the softmax, and a single bf16 P left them short of the
+//                 bf16 output rounding.
 //   dgamma      fixed-order sum of the partials (deterministic)
 #include "common.cuh"
 
@@ -39,21 +54,19 @@ __global__ void __launch_bounds__(PRE_WARPS * 32) bwd_pre_kernel(const __grid_co
         a = unpack_bf16(gr.x); b = unpack_bf16(gr.y);
         g[0] = a.x; g[1] = a.y; g[2] = b.x; g[3] = b.y;
     }
-    float delta = 0.f, dgv[4], dav[4];
+    float dgv[4], dav[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         float sg = sigmoidf_(g[e]);
-        delta += d[e] * o[e];
         dgv[e] = d[e] * o[e] * (1.f - sg);
         dav[e] = d[e] * sg;
     }
-    delta = warp_sum(delta);
     *reinterpret_cast<uint2*>(p.dg + off) = make_uint2(pack_bf16(dgv[0], dgv[1]), pack_bf16(dgv[2], dgv[3]));
-    *reinterpret_cast<uint2*>(p.dA + off) = make_uint2(pack_bf16(dav[0], dav[1]), pack_bf16(dav[2], dav[3]));
-    if (lane == 0) {
-        const long long h = row % L.Hq, bs = row / L.Hq, s = bs % L.S, b = bs / L.S;
-        p.delta[((size_t)b * L.Hq + h) * L.S + s] = delta;
-    }
+    const uint32_t h01 = pack_bf16(dav[0], dav[1]), h23 = pack_bf16(dav[2], dav[3]);
+    const float2 r01 = unpack_bf16(h01), r23 = unpack_bf16(h23);
+    *reinterpret_cast<uint2*>(p.dA + off) = make_uint2(h01, h23);
+    *reinterpret_cast<uint2*>(p.dA_lo + off) =
+        make_uint2(pack_bf16(dav[0] - r01.x, dav[1] - r01.y), pack_bf16(dav[2] - r23.x, dav[3] - r23.y));
 }
 
 // =====================================================================  bwd_main
@@ -67,17 +80,13 @@ struct BwdMmaSmem {
     bf16 V[BM_KEYS * kD];
     bf16 Q[BM_Q * kD];        // Q~ of the current query tile
     bf16 dA[BM_Q * kD];
-    bf16 dS[BM_KEYS * BM_Q];  // [key][query], 128-byte rows, chunk ^= row & 7
+    bf16 dAl[BM_Q * kD];      // low part of dA
     float lse2[BM_Q];         // lse * log2(e)
     float delta[BM_Q];
     float ybuf[BM_THREADS / 32][kD];
     float gq[kD], gk[kD];
     float dgk[BM_THREADS / 32][kD];
 };
-
-__device__ __forceinline__ uint32_t ds_off(int row, int chunk) {
-    return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
-}
 
 __device__ __forceinline__ void bm_store_row(bf16* tile, int row, const float y[4]) {
     const int lane = threadIdx.x & 31;
@@ -157,8 +166,9 @@ __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_co
                 int c = tid + BM_THREADS * i;
                 int row = c >> 4, ch = c & 15, pos = q0 + row;
                 bool ok = pos < L.S;
-                const bf16* src = p.dA + ((size_t)(b * (size_t)L.S + (ok ? pos : 0)) * L.Hq + h) * kD + ch * 8;
-                cp_async16(smem_u32(reinterpret_cast<char*>(sm.dA) + tile_off(row, ch)), src, ok);
+                const size_t go = ((size_t)(b * (size_t)L.S + (ok ? pos : 0)) * L.Hq + h) * kD + ch * 8;
+                cp_async16(smem_u32(reinterpret_cast<char*>(sm.dA) + tile_off(row, ch)), p.dA + go, ok);
+                cp_async16(smem_u32(reinterpret_cast<char*>(sm.dAl) + tile_off(row, ch)), p.dA_lo + go, ok);
             }
             cp_async_commit();
             if (tid < BM_Q) {
@@ -188,7 +198,8 @@ __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_co
 
             // warp-level skip: keys [kw0, kw0+15] are seen by queries [kw0, kw0+15+W-1]
             const bool live = kw0 < L.S && q0 <= kw0 + 15 + L.W - 1 && q0 + BM_Q - 1 >= kw0;
-            const uint32_t kb = smem_u32(sm.K), vb = smem_u32(sm.V), qb = smem_u32(sm.Q), db = smem_u32(sm.dA);
+            const uint32_t kb = smem_u32(sm.K), vb = smem_u32(sm.V), qb = smem_u32(sm.Q), db = smem_u32(sm.dA),
+                           dlb = smem_u32(sm.dAl);
             if (live) {
                 float st[8][4], dpt[8][4];
 #pragma unroll
@@ -211,6 +222,9 @@ __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_co
                         ldmatrix_x4(b0, b1, b2, b3, db + tile_off(rr, cc));
                         mma_bf16(dpt[2 * np], av, b0, b1);
                         mma_bf16(dpt[2 * np + 1], av, b2, b3);
+                        ldmatrix_x4(b0, b1, b2, b3, dlb + tile_off(rr, cc));
+                        mma_bf16(dpt[2 * np], av, b0, b1);
+                        mma_bf16(dpt[2 * np + 1], av, b2, b3);
                     }
                 }
                 // P^T = exp2(S^T*scale*log2e - lse2), masked; dS^T = P^T (dP^T - Delta)
@@ -230,11 +244,14 @@ __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_co
                 // dV += P^T dA ; dK~ += dS^T Q~   (A from registers, B via ldmatrix.trans)
 #pragma unroll
                 for (int kq = 0; kq < 4; ++kq) {
-                    uint32_t ap[4], as[4];
-                    ap[0] = pack_bf16(st[2 * kq][0], st[2 * kq][1]);
-                    ap[1] = pack_bf16(st[2 * kq][2], st[2 * kq][3]);
-                    ap[2] = pack_bf16(st[2 * kq + 1][0], st[2 * kq + 1][1]);
-                    ap[3] = pack_bf16(st[2 * kq + 1][2], st[2 * kq + 1][3]);
+                    uint32_t ap[4], apl[4], as[4];
+                    const float* pf[4] = {&st[2 * kq][0], &st[2 * kq][2], &st[2 * kq + 1][0], &st[2 * kq + 1][2]};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        ap[u] = pack_bf16(pf[u][0], pf[u][1]);
+                        const float2 hi = unpack_bf16(ap[u]);
+                        apl[u] = pack_bf16(pf[u][0] - hi.x, pf[u][1] - hi.y);
+                    }
                     as[0] = pack_bf16(dpt[2 * kq][0], dpt[2 * kq][1]);
                     as[1] = pack_bf16(dpt[2 * kq][2], dpt[2 * kq][3]);
                     as[2] = pack_bf16(dpt[2 * kq + 1][0], dpt[2 * kq + 1][1]);
@@ -246,63 +263,14 @@ __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_co
                         ldmatrix_x4_trans(b0, b1, b2, b3, db + tile_off(rr, cc));
                         mma_bf16(dv[2 * dn], ap, b0, b1);
                         mma_bf16(dv[2 * dn + 1], ap, b2, b3);
+                        mma_bf16(dv[2 * dn], apl, b0, b1);
+                        mma_bf16(dv[2 * dn + 1], apl, b2, b3);
+                        ldmatrix_x4_trans(b0, b1, b2, b3, dlb + tile_off(rr, cc));
+                        mma_bf16(dv[2 * dn], ap, b0, b1);
+                        mma_bf16(dv[2 * dn + 1], ap, b2, b3);
                         ldmatrix_x4_trans(b0, b1, b2, b3, qb + tile_off(rr, cc));
                         mma_bf16(dk[2 * dn], as, b0, b1);
                         mma_bf16(dk[2 * dn + 1], as, b2, b3);
-                    }
-                    // dS^T to shared memory ([key][query], bf16) for the dQ product
-                    char* dsb = reinterpret_cast<char*>(sm.dS);
-                    const int kr0 = warp * 16 + (lane >> 2), kr1 = kr0 + 8;
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int nt = 2 * kq + half;
-                        const int ql = nt * 8 + 2 * (lane & 3);
-                        *reinterpret_cast<uint32_t*>(dsb + ds_off(kr0, ql >> 3) + (ql & 7) * 2) = as[2 * half];
-                        *reinterpret_cast<uint32_t*>(dsb + ds_off(kr1, ql >> 3) + (ql & 7) * 2) = as[2 * half + 1];
-                    }
-                }
-            } else {
-                // zero this warp's dS^T rows so the dQ product reads no stale values
-                char* dsb = reinterpret_cast<char*>(sm.dS);
-                for (int c = lane; c < 16 * 8; c += 32) {
-                    int row = warp * 16 + (c >> 3), ch = c & 7;
-                    *reinterpret_cast<uint4*>(dsb + ds_off(row, ch)) = make_uint4(0u, 0u, 0u, 0u);
-                }
-            }
-            __syncthreads();
-            // dQ~ (64 queries x 128) += dS (64 x 64 keys) K~ (64 x 128); warp w: queries 16w..16w+15,
-            // in four 32-column slices to bound the live accumulator registers
-            const int qr0 = q0 + warp * 16 + (lane >> 2), qr1 = qr0 + 8;
-            const uint32_t dsb = smem_u32(sm.dS);
-            if (q0 + warp * 16 < L.S) {
-#pragma unroll
-                for (int dc = 0; dc < 4; ++dc) {
-                    float acc[4][4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        uint32_t a[4];
-                        ldmatrix_x4_trans(a[0], a[1], a[2], a[3],
-                                          dsb + ds_off(16 * kk + (lane & 7) + (lane >> 4) * 8, 2 * warp + ((lane >> 3) & 1)));
-#pragma unroll
-                        for (int dn = 0; dn < 2; ++dn) {
-                            uint32_t b0, b1, b2, b3;
-                            ldmatrix_x4_trans(b0, b1, b2, b3,
-                                              kb + tile_off(16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8, 4 * dc + 2 * dn + (lane >> 4)));
-                            mma_bf16(acc[2 * dn], a, b0, b1);
-                            mma_bf16(acc[2 * dn + 1], a, b2, b3);
-                        }
-                    }
-#pragma unroll
-                    for (int nt = 0; nt < 4; ++nt) {
-                        const int col = 32 * dc + 8 * nt + 2 * (lane & 3);
-                        if (qr0 < L.S)
-                            atomicAdd(reinterpret_cast<float2*>(p.dq_acc + ((size_t)(b * (size_t)L.S + qr0) * L.Hq + h) * kD + col),
-                                      make_float2(acc[nt][0], acc[nt][1]));
-                        if (qr1 < L.S)
-                            atomicAdd(reinterpret_cast<float2*>(p.dq_acc + ((size_t)(b * (size_t)L.S + qr1) * L.Hq + h) * kD + col),
-                                      make_float2(acc[nt][2], acc[nt][3]));
                     }
                 }
             }
@@ -319,7 +287,7 @@ __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_co
             *reinterpret_cast<uint32_t*>(p.dv + ((size_t)(b * (size_t)L.S + j1) * L.Hkv + kvh) * kD + col) = pack_bf16(dv[nt][2], dv[nt][3]);
     }
     __syncthreads();
-    float* stage = reinterpret_cast<float*>(sm.Q);  // Q + dA = 32 KB = [64][128] fp32
+    float* stage = reinterpret_cast<float*>(sm.Q);  // Q + dA = 32 KB = [64][128] fp32 (dAl follows)
     {
         const int rr0 = warp * 16 + (lane >> 2), rr1 = rr0 + 8;
 #pragma unroll
@@ -353,36 +321,250 @@ __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_co
 
 // =====================================================================  bwd_dq
 
-constexpr int DQ_WARPS = 8;
-constexpr int DQ_ROWS_PER_WARP = 32;
+constexpr int DQ_BM = 64;       // query rows per CTA (4 warps x 16)
+constexpr int DQ_BN = 64;       // keys per tile
+constexpr int DQ_THREADS = 128;
 
-__global__ void __launch_bounds__(DQ_WARPS * 32) bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+struct BwdDqSmem {
+    bf16 Q[DQ_BM * kD];         // Q~ (normalised + rotated), swizzled rows
+    bf16 dA[DQ_BM * kD];
+    bf16 dAl[DQ_BM * kD];       // low part of dA
+    bf16 K[2][DQ_BN * kD];      // K~
+    bf16 V[2][DQ_BN * kD];
+    float lse2[DQ_BM];
+    float ybuf[DQ_THREADS / 32][kD];
+    float gq[kD], gk[kD];
+    float dgq[DQ_THREADS / 32][kD];
+};
+static_assert(DQ_BM * kD * 4 <= sizeof(bf16) * 4 * DQ_BN * kD, "dQ staging fits in the K/V buffers");
+
+// K~ prologue (16 rows per warp) + V via cp.async for the key tile at kbase.
+__device__ __forceinline__ void dq_load_kv(const LayerParams& L, BwdDqSmem& sm, int buf, int b, int kvh,
+                                           int kbase) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        int c = tid + DQ_THREADS * i;
+        int row = c >> 4, ch = c & 15, pos = kbase + row;
+        bool ok = pos < L.S;
+        const bf16* src = L.v + ((size_t)(b * (size_t)L.S + (ok ? pos : 0)) * L.Hkv + kvh) * kD + ch * 8;
+        cp_async16(smem_u32(reinterpret_cast<char*>(sm.V[buf]) + tile_off(row, ch)), src, ok);
+    }
+    cp_async_commit();
+    uint2 raw[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        int pos = kbase + warp * 16 + r;
+        raw[r] = pos < L.S ? load_row4(L.k + ((size_t)(b * (size_t)L.S + pos) * L.Hkv + kvh) * kD)
+                           : make_uint2(0u, 0u);
+    }
+    const float g4[4] = {sm.gk[4 * lane], sm.gk[4 * lane + 1], sm.gk[4 * lane + 2], sm.gk[4 * lane + 3]};
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        int row = warp * 16 + r, pos = kbase + row;
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+        if (pos < L.S) prologue_row(raw[r], g4, L, pos, sm.ybuf[warp], y);
+        bm_store_row(sm.K[buf], row, y);
+    }
+}
+
+__global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_constant__ BwdParams p) {
     const LayerParams& L = p.L;
-    __shared__ float ybuf[DQ_WARPS][kD];
-    __shared__ float dgq[DQ_WARPS][kD];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long nrows = (long long)L.B * L.S * L.Hq;
-    const float g4[4] = {L.gamma_q[4 * lane], L.gamma_q[4 * lane + 1], L.gamma_q[4 * lane + 2], L.gamma_q[4 * lane + 3]};
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    BwdDqSmem& sm = *reinterpret_cast<BwdDqSmem*>(smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    const int nqt = (L.S + DQ_BM - 1) / DQ_BM;
+    int bid = blockIdx.x;
+    const int b = bid / (nqt * L.Hq);
+    bid -= b * nqt * L.Hq;
+    const int h = bid / nqt;
+    int qt = bid - h * nqt;
+    if (L.W >= L.S) qt = nqt - 1 - qt;  // full causal: longest rows first
+    const int kvh = h / L.G;
+    const int q0 = qt * DQ_BM;
+
+    if (tid < kD) {
+        sm.gq[tid] = L.gamma_q[tid];
+        sm.gk[tid] = L.gamma_k[tid];
+    }
+    // dA tile
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        int c = tid + DQ_THREADS * i;
+        int row = c >> 4, ch = c & 15, pos = q0 + row;
+        bool ok = pos < L.S;
+        const size_t go = ((size_t)(b * (size_t)L.S + (ok ? pos : 0)) * L.Hq + h) * kD + ch * 8;
+        cp_async16(smem_u32(reinterpret_cast<char*>(sm.dA) + tile_off(row, ch)), p.dA + go, ok);
+        cp_async16(smem_u32(reinterpret_cast<char*>(sm.dAl) + tile_off(row, ch)), p.dA_lo + go, ok);
+    }
+    cp_async_commit();
+    if (tid < DQ_BM) {
+        int pos = q0 + tid;
+        sm.lse2[tid] = pos < L.S ? p.lse[((size_t)b * L.Hq + h) * L.S + pos] * kLog2e : INFINITY;
+    }
+    __syncthreads();
+    const float gq4[4] = {sm.gq[4 * lane], sm.gq[4 * lane + 1], sm.gq[4 * lane + 2], sm.gq[4 * lane + 3]};
+    {
+        uint2 raw[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            int pos = q0 + warp * 16 + r;
+            raw[r] = pos < L.S ? load_row4(L.q + ((size_t)(b * (size_t)L.S + pos) * L.Hq + h) * kD)
+                               : make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            int row = warp * 16 + r, pos = q0 + row;
+            float y[4] = {0.f, 0.f, 0.f, 0.f};
+            if (pos < L.S) prologue_row(raw[r], gq4, L, pos, sm.ybuf[warp], y);
+            bm_store_row(sm.Q, row, y);
+        }
+    }
+
+    const int klo = max(0, q0 - L.W + 1);
+    const int khi = min(L.S - 1, q0 + DQ_BM - 1);
+    const int kt_lo = klo / DQ_BN, kt_hi = khi / DQ_BN;
+    const int wq0 = q0 + warp * 16;
+    const int r0 = wq0 + (lane >> 2), r1 = r0 + 8;
+    const int lr0 = warp * 16 + (lane >> 2), lr1 = lr0 + 8;
+
+    float dq[16][4];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dq[i][e] = 0.f;
+    float ds0 = 0.f, ds1 = 0.f;  // Delta of rows r0, r1 (this thread's columns during pass 1)
+    const int ntiles = kt_hi - kt_lo + 1;
+
+    dq_load_kv(L, sm, 0, b, kvh, kt_lo * DQ_BN);
+    for (int it = 0; it < 2 * ntiles; ++it) {
+        const int pass = it >= ntiles ? 1 : 0;
+        const int kt = kt_lo + (it - pass * ntiles);
+        const int buf = it & 1;
+        cp_async_wait<0>();
+        __syncthreads();
+        if (it + 1 < 2 * ntiles) {
+            const int nkt = kt_lo + ((it + 1) % ntiles);
+            dq_load_kv(L, sm, buf ^ 1, b, kvh, nkt * DQ_BN);
+        }
+        if (pass == 1 && it == ntiles) {
+            // Delta complete: sum over the quad of lanes holding each row
+            ds0 += __shfl_xor_sync(0xffffffffu, ds0, 1);
+            ds0 += __shfl_xor_sync(0xffffffffu, ds0, 2);
+            ds1 += __shfl_xor_sync(0xffffffffu, ds1, 1);
+            ds1 += __shfl_xor_sync(0xffffffffu, ds1, 2);
+        }
+        const int kbase = kt * DQ_BN;
+        const bool live = wq0 < L.S && kbase <= wq0 + 15 && kbase + DQ_BN - 1 >= wq0 - L.W + 1;
+        if (!live) continue;
+        const uint32_t qs = smem_u32(sm.Q), das = smem_u32(sm.dA), dls = smem_u32(sm.dAl),
+                       ks = smem_u32(sm.K[buf]), vs = smem_u32(sm.V[buf]);
+        float s[8][4], dp[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[i][e] = dp[i][e] = 0.f;
+        // S = Q~ K~^T and dP = dA V^T  (16 queries x 64 keys per warp)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            uint32_t aq[4], ad[4], al[4];
+            ldmatrix_x4(aq[0], aq[1], aq[2], aq[3], qs + tile_off(warp * 16 + (lane & 15), 2 * kk + (lane >> 4)));
+            ldmatrix_x4(ad[0], ad[1], ad[2], ad[3], das + tile_off(warp * 16 + (lane & 15), 2 * kk + (lane >> 4)));
+            ldmatrix_x4(al[0], al[1], al[2], al[3], dls + tile_off(warp * 16 + (lane & 15), 2 * kk + (lane >> 4)));
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t b0, b1, b2, b3;
+                const int rr = np * 16 + (lane >> 4) * 8 + (lane & 7), cc = 2 * kk + ((lane >> 3) & 1);
+                ldmatrix_x4(b0, b1, b2, b3, ks + tile_off(rr, cc));
+                mma_bf16(s[2 * np], aq, b0, b1);
+                mma_bf16(s[2 * np + 1], aq, b2, b3);
+                ldmatrix_x4(b0, b1, b2, b3, vs + tile_off(rr, cc));
+                mma_bf16(dp[2 * np], ad, b0, b1);
+                mma_bf16(dp[2 * np + 1], ad, b2, b3);
+                mma_bf16(dp[2 * np], al, b0, b1);
+                mma_bf16(dp[2 * np + 1], al, b2, b3);
+            }
+        }
+        const float l0 = sm.lse2[lr0], l1 = sm.lse2[lr1];
+        if (pass == 0) {
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    int j = kbase + nt * 8 + 2 * (lane & 3) + (e & 1);
+                    int i = e < 2 ? r0 : r1;
+                    bool vis = j <= i && j > i - L.W && j < L.S && i < L.S;
+                    float pv = vis ? exp2f(s[nt][e] * L.scale_log2 - (e < 2 ? l0 : l1)) : 0.f;
+                    if (e < 2) ds0 += pv * dp[nt][e]; else ds1 += pv * dp[nt][e];
+                }
+            }
+            continue;
+        }
+        // pass 1: dS = P (dP - Delta), dQ~ += dS K~  (A from registers, B = K~ via ldmatrix.trans)
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                int j = kbase + nt * 8 + 2 * (lane & 3) + (e & 1);
+                int i = e < 2 ? r0 : r1;
+                bool vis = j <= i && j > i - L.W && j < L.S && i < L.S;
+                float pv = vis ? exp2f(s[nt][e] * L.scale_log2 - (e < 2 ? l0 : l1)) : 0.f;
+                dp[nt][e] = pv * (dp[nt][e] - (e < 2 ? ds0 : ds1));
+            }
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t aw[4];
+            aw[0] = pack_bf16(dp[2 * kk][0], dp[2 * kk][1]);
+            aw[1] = pack_bf16(dp[2 * kk][2], dp[2 * kk][3]);
+            aw[2] = pack_bf16(dp[2 * kk + 1][0], dp[2 * kk + 1][1]);
+            aw[3] = pack_bf16(dp[2 * kk + 1][2], dp[2 * kk + 1][3]);
+#pragma unroll
+            for (int dn = 0; dn < 8; ++dn) {
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4_trans(b0, b1, b2, b3,
+                                  ks + tile_off(16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * dn + (lane >> 4)));
+                mma_bf16(dq[2 * dn], aw, b0, b1);
+                mma_bf16(dq[2 * dn + 1], aw, b2, b3);
+            }
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    if (ntiles == 0) { ds0 = ds1 = 0.f; }
+
+    if ((lane & 3) == 0) {
+        if (r0 < L.S) p.delta[((size_t)b * L.Hq + h) * L.S + r0] = ds0;
+        if (r1 < L.S) p.delta[((size_t)b * L.Hq + h) * L.S + r1] = ds1;
+    }
+    // dQ~ (scaled) -> fp32 staging [64][128] in the K/V buffers
+    float* stage = reinterpret_cast<float*>(sm.K[0]);
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+        const int col = nt * 8 + 2 * (lane & 3);
+        *reinterpret_cast<float2*>(stage + lr0 * kD + col) = make_float2(L.scale * dq[nt][0], L.scale * dq[nt][1]);
+        *reinterpret_cast<float2*>(stage + lr1 * kD + col) = make_float2(L.scale * dq[nt][2], L.scale * dq[nt][3]);
+    }
+    __syncthreads();
     float dgacc[4] = {0.f, 0.f, 0.f, 0.f};
-    const long long first = ((long long)blockIdx.x * DQ_WARPS + warp) * DQ_ROWS_PER_WARP;
-    for (int r = 0; r < DQ_ROWS_PER_WARP; ++r) {
-        const long long row = first + r;
-        if (row >= nrows) break;
-        const int pos = (int)((row / L.Hq) % L.S);
-        const size_t off = (size_t)row * kD;
+    for (int r = 0; r < 16; ++r) {
+        const int row = warp * 16 + r, pos = q0 + row;
+        if (pos >= L.S) break;
+        const size_t off = ((size_t)(b * (size_t)L.S + pos) * L.Hq + h) * kD;
         uint2 raw = load_row4(L.q + off);
-        float4 a = *reinterpret_cast<const float4*>(p.dq_acc + off + 4 * lane);
-        float dy[4] = {a.x * L.scale, a.y * L.scale, a.z * L.scale, a.w * L.scale}, dx[4];
-        prologue_row_backward(raw, g4, L, pos, ybuf[warp], dy, dx, dgacc);
+        float4 d4 = *reinterpret_cast<const float4*>(stage + row * kD + 4 * lane);
+        float dy[4] = {d4.x, d4.y, d4.z, d4.w}, dx[4];
+        prologue_row_backward(raw, gq4, L, pos, sm.ybuf[warp], dy, dx, dgacc);
         *reinterpret_cast<uint2*>(p.dq + off + 4 * lane) = make_uint2(pack_bf16(dx[0], dx[1]), pack_bf16(dx[2], dx[3]));
     }
-    *reinterpret_cast<float4*>(&dgq[warp][4 * lane]) = make_float4(dgacc[0], dgacc[1], dgacc[2], dgacc[3]);
+    *reinterpret_cast<float4*>(&sm.dgq[warp][4 * lane]) = make_float4(dgacc[0], dgacc[1], dgacc[2], dgacc[3]);
     __syncthreads();
-    if (threadIdx.x < kD) {
-        float s = 0.f;
+    if (tid < kD) {
+        float t = 0.f;
 #pragma unroll
-        for (int w = 0; w < DQ_WARPS; ++w) s += dgq[w][threadIdx.x];
-        p.dgq_part[(size_t)blockIdx.x * kD + threadIdx.x] = s;
+        for (int w = 0; w < DQ_THREADS / 32; ++w) t += sm.dgq[w][tid];
+        p.dgq_part[(size_t)blockIdx.x * kD + tid] = t;
     }
 }
 
@@ -410,29 +592,54 @@ __global__ void __launch_bounds__(1024) dgamma_reduce_kernel(const float* __rest
 
 int bwd_mma_n_k_parts(int B, int S, int Hkv) { return ((S + BM_KEYS - 1) / BM_KEYS) * Hkv * B; }
 long long bwd_mma_n_q_parts(int B, int S, int Hq) {
-    const long long rows = (long long)B * S * Hq, per = (long long)DQ_WARPS * DQ_ROWS_PER_WARP;
-    return (rows + per - 1) / per;
+    return (long long)((S + DQ_BM - 1) / DQ_BM) * Hq * B;
 }
 
-cudaError_t launch_bwd_mma(const BwdParams& p, cudaStream_t stream, cudaEvent_t ev0, cudaEvent_t ev1) {
+extern const char* const kBwdMmaKernelNames[] = {"bwd_pre_kernel", "bwd_dq_kernel", "bwd_main_kernel",
+                                          "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"};
+extern const int kBwdMmaKernelCount = 5;
+
+namespace {
+// records events[2i] before / events[2i+1] after kernel i when i < n_pairs
+struct KernelEvents {
+    void* const* ev;
+    int n;
+    cudaStream_t s;
+    cudaError_t before(int i) const {
+        return (i < n) ? cudaEventRecord(static_cast<cudaEvent_t>(ev[2 * i]), s) : cudaSuccess;
+    }
+    cudaError_t after(int i) const {
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        return (i < n) ? cudaEventRecord(static_cast<cudaEvent_t>(ev[2 * i + 1]), s) : cudaSuccess;
+    }
+};
+}  // namespace
+
+cudaError_t launch_bwd_mma(const BwdParams& p, cudaStream_t stream, void* const* events, int n_pairs) {
     const LayerParams& L = p.L;
+    const KernelEvents ke{events, n_pairs, stream};
     const long long nrows = (long long)L.B * L.S * L.Hq;
-    cudaError_t e = cudaMemsetAsync(p.dq_acc, 0, (size_t)nrows * kD * sizeof(float), stream);
+    const size_t smem_dq = sizeof(BwdDqSmem), smem_main = sizeof(BwdMmaSmem);
+    cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dq);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_main);
     if (e != cudaSuccess) return e;
+    if ((e = ke.before(0)) != cudaSuccess) return e;
     bwd_pre_kernel<<<(unsigned)((nrows + PRE_WARPS - 1) / PRE_WARPS), PRE_WARPS * 32, 0, stream>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const size_t smem = sizeof(BwdMmaSmem);
-    e = cudaFuncSetAttribute(bwd_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    if (ev0 && (e = cudaEventRecord(ev0, stream)) != cudaSuccess) return e;
-    bwd_main_kernel<<<(unsigned)p.n_k_parts, BM_THREADS, smem, stream>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (ev1 && (e = cudaEventRecord(ev1, stream)) != cudaSuccess) return e;
-    bwd_dq_kernel<<<(unsigned)p.n_q_parts, DQ_WARPS * 32, 0, stream>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = ke.after(0)) != cudaSuccess) return e;
+    if ((e = ke.before(1)) != cudaSuccess) return e;
+    bwd_dq_kernel<<<(unsigned)p.n_q_parts, DQ_THREADS, smem_dq, stream>>>(p);
+    if ((e = ke.after(1)) != cudaSuccess) return e;
+    if ((e = ke.before(2)) != cudaSuccess) return e;
+    bwd_main_kernel<<<(unsigned)p.n_k_parts, BM_THREADS, smem_main, stream>>>(p);
+    if ((e = ke.after(2)) != cudaSuccess) return e;
+    if ((e = ke.before(3)) != cudaSuccess) return e;
     dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.dgk_part, p.n_k_parts, p.dgamma_k);
+    if ((e = ke.after(3)) != cudaSuccess) return e;
+    if ((e = ke.before(4)) != cudaSuccess) return e;
     dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.dgq_part, p.n_q_parts, p.dgamma_q);
-    return cudaGetLastError();
+    return ke.after(4);
 }
 
 }  // namespace zgcm

@@ -55,9 +55,9 @@ struct BwdParams {
     float* dgamma_q;    // [D]
     float* dgamma_k;    // [D]
     // workspace views
-    float* delta;       // [B,Hq,S]   rowsum(dout * out)
-    bf16* dA;           // [B,S,Hq,D] dout * sigmoid(g)
-    float* dq_acc;      // [B,S,Hq,D] fp32 gradient w.r.t. rotated q (unscaled)
+    float* delta;       // [B,Hq,S]   sum_j P_ij dP_ij (formed by the dq kernel)
+    bf16* dA;           // [B,S,Hq,D] dout * sigmoid(g), rounded to bf16 ("hi")
+    bf16* dA_lo;        // [B,S,Hq,D] dout * sigmoid(g) - hi, rounded to bf16
     float* dgk_part;    // [n_k_parts, D]
     float* dgq_part;    // [n_q_parts, D]
     int n_k_parts, n_q_parts;

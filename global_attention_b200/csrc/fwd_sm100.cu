@@ -1,0 +1,581 @@
+// fwd_sm100.cu — gated sliding-window attention forward on tcgen05 / TMEM / TMA (sm_100a).
+//
+// Layer (ZGCM-1; page citations in common.cuh): out = sigmoid(g) * softmax_window(q~ k~^T) v,
+// with q~, k~ the RMS-normalised (gamma) and partially rotated q, k, window i-W < j <= i.
+// This kernel takes windows W <= 128 (the 27 sliding layers use W = 128) and 42 rotated
+// dims; other shapes run on the warp-MMA kernel (fwd_mma.cu).
+//
+// Work decomposition: a "step" is (batch b, KV head, 128-query block qb) with all Hq/Hkv
+// query heads of the group.  With W <= 128 the window of block qb lies inside key tiles
+// qb-1 and qb, so consecutive steps of one (b, KV head) chain share a tile: a persistent
+// CTA sweeps a contiguous range of steps and loads ONE new K/V tile per step into a 2-slot
+// ring.  K~ and Q~ are normalised/rotated in place in shared memory (TMA-loaded raw,
+// 128-byte swizzle = the UMMA K-major canonical layout).
+//
+// Per head m (TMEM: S/P columns [0,256), O double buffer [256,384) and [384,512)):
+//   S   = Q~ [K~_slot0; K~_slot1]^T          tcgen05.mma M=128 N=256 K=128, A,B in smem
+//   P   = exp2(S*scale*log2e - max)          softmax warpgroup, thread = query row, fp32,
+//                                            written back as bf16 over the front of S
+//   O   = P [V_slot0; V_slot1]               tcgen05.mma M=128 N=128 K=256, A in TMEM,
+//                                            B (V, d-contiguous) MN-major in smem
+//   out = sigmoid(g) * O / l                 epilogue, 16-byte global loads/stores
+//
+// Warp roles (384 threads): w0 TMA K/V, w1 MMA issue + TMEM owner, w2 TMA Q, w3 idle,
+// w4-7 softmax, w8-11 prologue (K~, Q~ in place) + gate epilogue.  Every wait is bounded;
+// on expiry the CTA records the site, drains, frees TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include "sm100.cuh"
+
+namespace zgcm {
+using namespace sm100;
+
+constexpr int TF_BM = 128;
+constexpr int TF_BN = 128;
+constexpr int TF_THREADS = 384;
+constexpr int TF_HALF = 21;              // rotated pairs (rope_dims = 42)
+constexpr uint32_t TF_TILE_BYTES = TF_BN * kD * 2;   // one 128 x 128 bf16 tile
+constexpr uint32_t TF_HALF_BYTES = TF_BN * 64 * 2;   // one 128-row x 64-col half: 16 KB
+constexpr uint32_t TF_RING_HALF = 2 * TF_HALF_BYTES; // one d-half of the 2-slot ring: 32 KB
+
+struct FwdTcParams {
+    CUtensorMap tm_q;   // {D, Hq, S, B}, box {64, 1, 128, 1}, 128B swizzle
+    CUtensorMap tm_k;   // {D, Hkv, S, B}
+    CUtensorMap tm_v;
+    LayerParams L;
+    bf16* out;
+    float* lse;
+    int* err;           // device error word: site of an expired wait (0 = none)
+    int total_steps;    // B * Hkv * ceil(S / 128)
+};
+
+enum Bar {
+    B_KFULL = 0, B_KREADY = 2, B_KEMPTY = 4, B_VFULL = 6, B_VEMPTY = 8,
+    B_QFULL = 10, B_QREADY = 12, B_QEMPTY = 14,
+    B_SFULL = 16, B_PFULL = 17,
+    B_OFULL = 18, B_OEMPTY = 20, B_LFULL = 22, B_LEMPTY = 24,
+    B_DONE = 26, B_COUNT = 27
+};
+
+struct FwdTcSmem {
+    // ring of two K (resp. V) tiles, split by d-half so the 256 rows of a half are
+    // contiguous: K[h] holds rows slot0(0..127), slot1(128..255) of dims 64h..64h+63
+    alignas(1024) unsigned char K[2][TF_RING_HALF];
+    alignas(1024) unsigned char V[2][TF_RING_HALF];
+    alignas(1024) unsigned char Q[2][2][TF_HALF_BYTES];  // [buffer][d-half]
+    float2 cs[TF_HALF][TF_BM];   // (cos, sin) of pair t at row r's position; thread r's column
+    float gq[kD], gk[kD];
+    float rowinv[2][TF_BM];
+    uint64_t bar[B_COUNT];
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct StepInfo {
+    int b, kvh, qb;
+    bool fresh;        // first step of a chain in this CTA: load the previous tile too
+    bool release_cur;  // the next step does not reuse this step's current tile
+};
+
+__device__ __forceinline__ StepInfo decode_step(const LayerParams& L, int t, int t_begin, int t_end) {
+    const int nqb = (L.S + TF_BM - 1) / TF_BM;
+    StepInfo s;
+    const int chain = t / nqb;
+    s.qb = t - chain * nqb;
+    s.b = chain / L.Hkv;
+    s.kvh = chain - s.b * L.Hkv;
+    s.fresh = (t == t_begin) || (s.qb == 0);
+    s.release_cur = (t + 1 >= t_end) || (s.qb + 1 == nqb);
+    return s;
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float fast_tanh(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// ------------------------------------------------------------------ prologue (one row per thread)
+
+// cos/sin of the TF_HALF rotation angles at `pos`, into column r of the table
+__device__ __forceinline__ void tf_angles(const LayerParams& L, int pos, float2 (*cs)[TF_BM], int r) {
+#pragma unroll
+    for (int t = 0; t < TF_HALF; ++t) {
+        float c, s;
+        rope_cs(L.theta[t], pos, c, s);
+        cs[t][r] = make_float2(c, s);
+    }
+}
+
+// Row `r` of a 128-row tile stored as two 16 KB d-halves (h0, h1), 128-byte swizzled:
+// normalise (RMS, gamma), rotate pairs (t, t+21) for t < 21, write back bf16 in place.
+// Rows outside the sequence are zero-filled by TMA and stay zero.
+__device__ __forceinline__ void tf_prologue_row(unsigned char* h0, unsigned char* h1, int r, const float* gamma,
+                                                const LayerParams& L, const float2 (*cs)[TF_BM]) {
+    // chunk ch (8 dims, 16 bytes) of the row: half ch / 8, swizzled position (ch % 8) ^ (r % 8)
+    auto chunk = [&](int ch) -> uint4* {
+        unsigned char* hb = ch < 8 ? h0 : h1;
+        return reinterpret_cast<uint4*>(hb + (uint32_t)r * 128u + (uint32_t)(((ch & 7) ^ (r & 7)) << 4));
+    };
+    float ss = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 16; ++ch) {
+        const uint4 u = *chunk(ch);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float2 f = unpack_bf16(w[e]);
+            ss = fmaf(f.x, f.x, ss);
+            ss = fmaf(f.y, f.y, ss);
+        }
+    }
+    // a zero row (outside the sequence, zero-filled by TMA) stays zero even with eps = 0
+    const float rinv = ss > 0.f ? rsqrtf(ss * (1.0f / kD) + L.eps) : 0.f;
+    // dims 0..47 (chunks 0..5): normalise, rotate the first 42
+    float y[48];
+#pragma unroll
+    for (int ch = 0; ch < 6; ++ch) {
+        const uint4 u = *chunk(ch);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float2 f = unpack_bf16(w[e]);
+            const int d = ch * 8 + 2 * e;
+            y[d] = (f.x * rinv) * gamma[d];
+            y[d + 1] = (f.y * rinv) * gamma[d + 1];
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < TF_HALF; ++t) {
+        const float a = y[t], bb = y[t + TF_HALF];
+        const float2 w = cs[t][r];
+        y[t] = a * w.x - bb * w.y;
+        y[t + TF_HALF] = bb * w.x + a * w.y;
+    }
+#pragma unroll
+    for (int ch = 0; ch < 6; ++ch) {
+        uint4 o;
+        o.x = pack_bf16(y[ch * 8 + 0], y[ch * 8 + 1]);
+        o.y = pack_bf16(y[ch * 8 + 2], y[ch * 8 + 3]);
+        o.z = pack_bf16(y[ch * 8 + 4], y[ch * 8 + 5]);
+        o.w = pack_bf16(y[ch * 8 + 6], y[ch * 8 + 7]);
+        *chunk(ch) = o;
+    }
+    // dims 48..127: normalise only
+#pragma unroll
+    for (int ch = 6; ch < 16; ++ch) {
+        const uint4 u = *chunk(ch);
+        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float2 f = unpack_bf16(w[e]);
+            const int d = ch * 8 + 2 * e;
+            w[e] = pack_bf16((f.x * rinv) * gamma[d], (f.y * rinv) * gamma[d + 1]);
+        }
+        *chunk(ch) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+// ------------------------------------------------------------------ the kernel
+
+__global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_constant__ FwdTcParams p) {
+    const LayerParams& L = p.L;
+    extern __shared__ unsigned char smem_raw[];
+    FwdTcSmem& sm = *reinterpret_cast<FwdTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    volatile int* abort = &sm.abort;
+
+    const int G = L.G;
+    const int t_begin = (int)(((long long)blockIdx.x * p.total_steps) / gridDim.x);
+    const int t_end = (int)(((long long)(blockIdx.x + 1) * p.total_steps) / gridDim.x);
+
+    if (tid == 0) {
+        sm.abort = 0;
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.bar[B_KFULL + i], 1);
+            mbar_init(&sm.bar[B_KREADY + i], 128);
+            mbar_init(&sm.bar[B_KEMPTY + i], 1);
+            mbar_init(&sm.bar[B_VFULL + i], 1);
+            mbar_init(&sm.bar[B_VEMPTY + i], 1);
+            mbar_init(&sm.bar[B_QFULL + i], 1);
+            mbar_init(&sm.bar[B_QREADY + i], 128);
+            mbar_init(&sm.bar[B_QEMPTY + i], 1);
+            mbar_init(&sm.bar[B_OFULL + i], 1);
+            mbar_init(&sm.bar[B_OEMPTY + i], 128);
+            mbar_init(&sm.bar[B_LFULL + i], 128);
+            mbar_init(&sm.bar[B_LEMPTY + i], 128);
+        }
+        mbar_init(&sm.bar[B_SFULL], 1);
+        mbar_init(&sm.bar[B_PFULL], 128);
+        mbar_init(&sm.bar[B_DONE], 1);
+        fence_barrier_init();
+    }
+    if (tid < kD) {
+        sm.gq[tid] = L.gamma_q[tid];
+        sm.gk[tid] = L.gamma_k[tid];
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&p.tm_q);
+        prefetch_tmap(&p.tm_k);
+        prefetch_tmap(&p.tm_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t TM_S = tmem, TM_P = tmem, TM_O0 = tmem + 256;
+
+    if (warp == 0) {
+        // ================================================ K / V producer
+        if (lane == 0) {
+            int n_next = 0;
+            int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};  // last tile issued per slot
+            auto load_tile = [&](int n, int b, int kvh, int kt) -> bool {
+                const int slot = n & 1;
+                if (n >= 2 && !mbar_wait(&sm.bar[B_KEMPTY + slot], ((n >> 1) - 1) & 1, abort, 1)) return false;
+                mbar_expect_tx(&sm.bar[B_KFULL + slot], TF_TILE_BYTES);
+                tma_load_4d(sm.K[0] + slot * TF_HALF_BYTES, &p.tm_k, &sm.bar[B_KFULL + slot], 0, kvh, kt * TF_BN, b);
+                tma_load_4d(sm.K[1] + slot * TF_HALF_BYTES, &p.tm_k, &sm.bar[B_KFULL + slot], 64, kvh, kt * TF_BN, b);
+                last_k[slot] = n;
+                if (n >= 2 && !mbar_wait(&sm.bar[B_VEMPTY + slot], ((n >> 1) - 1) & 1, abort, 2)) return false;
+                mbar_expect_tx(&sm.bar[B_VFULL + slot], TF_TILE_BYTES);
+                tma_load_4d(sm.V[0] + slot * TF_HALF_BYTES, &p.tm_v, &sm.bar[B_VFULL + slot], 0, kvh, kt * TF_BN, b);
+                tma_load_4d(sm.V[1] + slot * TF_HALF_BYTES, &p.tm_v, &sm.bar[B_VFULL + slot], 64, kvh, kt * TF_BN, b);
+                last_v[slot] = n;
+                return true;
+            };
+            for (int t = t_begin; t < t_end && !*abort; ++t) {
+                const StepInfo st = decode_step(L, t, t_begin, t_end);
+                if (st.fresh && !load_tile(n_next++, st.b, st.kvh, st.qb - 1)) break;
+                if (!load_tile(n_next++, st.b, st.kvh, st.qb)) break;
+            }
+            // every copy issued must have landed before the CTA exits (matters after an abort)
+            for (int slot = 0; slot < 2; ++slot) {
+                if (last_k[slot] >= 0) mbar_wait_drain(&sm.bar[B_KFULL + slot], (last_k[slot] >> 1) & 1);
+                if (last_v[slot] >= 0) mbar_wait_drain(&sm.bar[B_VFULL + slot], (last_v[slot] >> 1) & 1);
+            }
+        }
+    } else if (warp == 2) {
+        // ================================================ Q producer
+        if (lane == 0) {
+            int m = 0;
+            int last_q[2] = {-1, -1};
+            for (int t = t_begin; t < t_end && !*abort; ++t) {
+                const StepInfo st = decode_step(L, t, t_begin, t_end);
+                for (int h = 0; h < G; ++h, ++m) {
+                    const int buf = m & 1;
+                    if (m >= 2 && !mbar_wait(&sm.bar[B_QEMPTY + buf], ((m >> 1) - 1) & 1, abort, 3)) break;
+                    mbar_expect_tx(&sm.bar[B_QFULL + buf], TF_TILE_BYTES);
+                    const int hg = st.kvh * G + h;
+                    tma_load_4d(sm.Q[buf][0], &p.tm_q, &sm.bar[B_QFULL + buf], 0, hg, st.qb * TF_BM, st.b);
+                    tma_load_4d(sm.Q[buf][1], &p.tm_q, &sm.bar[B_QFULL + buf], 64, hg, st.qb * TF_BM, st.b);
+                    last_q[buf] = m;
+                }
+            }
+            for (int buf = 0; buf < 2; ++buf)
+                if (last_q[buf] >= 0) mbar_wait_drain(&sm.bar[B_QFULL + buf], (last_q[buf] >> 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ================================================ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16(128, 256, false);
+            constexpr uint32_t IDESC_O = idesc_bf16(128, 128, true);
+            const uint32_t q_base = smem_u32(sm.Q[0][0]);
+            const uint32_t k_base = smem_u32(sm.K[0]);
+            const uint32_t v_base = smem_u32(sm.V[0]);
+            int n_next = 0, n_prev = 0, n_cur = 0, m = 0;
+            bool ok = true;
+            for (int t = t_begin; t < t_end && ok; ++t) {
+                const StepInfo st = decode_step(L, t, t_begin, t_end);
+                if (st.fresh) {
+                    n_prev = n_next++;
+                    n_cur = n_next++;
+                    ok = mbar_wait(&sm.bar[B_KREADY + (n_prev & 1)], (n_prev >> 1) & 1, abort, 10) &&
+                         mbar_wait(&sm.bar[B_VFULL + (n_prev & 1)], (n_prev >> 1) & 1, abort, 11);
+                } else {
+                    n_prev = n_cur;
+                    n_cur = n_next++;
+                }
+                ok = ok && mbar_wait(&sm.bar[B_KREADY + (n_cur & 1)], (n_cur >> 1) & 1, abort, 12) &&
+                     mbar_wait(&sm.bar[B_VFULL + (n_cur & 1)], (n_cur >> 1) & 1, abort, 13);
+                for (int h = 0; h < G && ok; ++h, ++m) {
+                    const int buf = m & 1;
+                    if (!(ok = mbar_wait(&sm.bar[B_QREADY + buf], (m >> 1) & 1, abort, 14))) break;
+                    tc_fence_after();
+                    // S = Q~ K~^T over both ring slots (N = 256), K = 128 in 8 steps of 16
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t half = kk >> 2, within = (kk & 3) * 32;
+                        const uint64_t a = sdesc_sw128(q_base + buf * 2 * TF_HALF_BYTES + half * TF_HALF_BYTES + within, 16, 1024);
+                        const uint64_t bdesc = sdesc_sw128(k_base + half * TF_RING_HALF + within, 16, 1024);
+                        mma_ss(TM_S, a, bdesc, IDESC_S, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&sm.bar[B_QEMPTY + buf]);
+                    mma_commit(&sm.bar[B_SFULL]);
+                    if (h == G - 1) {
+                        mma_commit(&sm.bar[B_KEMPTY + (n_prev & 1)]);
+                        if (st.release_cur) mma_commit(&sm.bar[B_KEMPTY + (n_cur & 1)]);
+                    }
+                    if (!(ok = mbar_wait(&sm.bar[B_PFULL], m & 1, abort, 15))) break;
+                    if (m >= 2 && !(ok = mbar_wait(&sm.bar[B_OEMPTY + buf], ((m >> 1) - 1) & 1, abort, 16))) break;
+                    tc_fence_after();
+                    // O = P V: P bf16 in TMEM (16 keys = 8 columns per step), V MN-major
+#pragma unroll
+                    for (int kk = 0; kk < 16; ++kk) {
+                        const uint64_t bdesc = sdesc_sw128(v_base + kk * 16 * 128, TF_RING_HALF, 1024);
+                        mma_ts(TM_O0 + buf * 128, TM_P + kk * 8, bdesc, IDESC_O, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&sm.bar[B_OFULL + buf]);
+                    if (h == G - 1) {
+                        mma_commit(&sm.bar[B_VEMPTY + (n_prev & 1)]);
+                        if (st.release_cur) mma_commit(&sm.bar[B_VEMPTY + (n_cur & 1)]);
+                    }
+                }
+            }
+            // every MMA issued must complete before TMEM is released
+            mma_commit(&sm.bar[B_DONE]);
+            mbar_wait(&sm.bar[B_DONE], 0, abort, 17);
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ================================================ softmax (thread = query row)
+        const int r = tid - 128, wq = warp - 4;
+        const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+        int n_next = 0, n_prev = 0, n_cur = 0, m = 0;
+        for (int t = t_begin; t < t_end; ++t) {
+            const StepInfo st = decode_step(L, t, t_begin, t_end);
+            if (st.fresh) { n_prev = n_next++; n_cur = n_next++; } else { n_prev = n_cur; n_cur = n_next++; }
+            const int q0 = st.qb * TF_BM, i = q0 + r;
+            // key position of ring column c: slot (c >> 7) holds tile qb (cur) or qb-1 (prev)
+            const int slot_cur = n_cur & 1;
+            const int base0 = (slot_cur == 0 ? q0 : q0 - TF_BN), base1 = (slot_cur == 1 ? q0 : q0 - TF_BN);
+            const int imin = q0 + 32 * wq, imax = imin + 31;
+            bool stop = false;
+            for (int h = 0; h < G; ++h, ++m) {
+                if (!mbar_wait(&sm.bar[B_SFULL], m & 1, abort, 20)) { stop = true; break; }
+                tc_fence_after();
+                float mx = -INFINITY;
+#pragma unroll 1
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const int kp0 = (c8 < 4 ? base0 : base1) + (c8 & 3) * 32;
+                    const bool live = imin < L.S && kp0 <= imax && kp0 + 31 > imin - L.W && kp0 + 31 >= 0 && kp0 < L.S;
+                    if (!live) continue;
+                    uint32_t v[32];
+                    tmem_ld32(TM_S + lane_off + 32 * c8, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = kp0 + e;
+                        const bool vis = j <= i && j > i - L.W && j >= 0 && j < L.S;
+                        if (vis) mx = fmaxf(mx, __uint_as_float(v[e]));
+                    }
+                }
+                const float mu = (mx == -INFINITY) ? 0.f : mx * L.scale_log2;
+                float l = 0.f;
+#pragma unroll 1
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const int kp0 = (c8 < 4 ? base0 : base1) + (c8 & 3) * 32;
+                    const bool live = imin < L.S && kp0 <= imax && kp0 + 31 > imin - L.W && kp0 + 31 >= 0 && kp0 < L.S;
+                    uint32_t pk[16];
+                    if (live) {
+                        uint32_t v[32];
+                        tmem_ld32(TM_S + lane_off + 32 * c8, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const int j = kp0 + e;
+                            const bool v0 = j <= i && j > i - L.W && j >= 0 && j < L.S;
+                            const bool v1 = j + 1 <= i && j + 1 > i - L.W && j + 1 >= 0 && j + 1 < L.S;
+                            const float p0 = v0 ? fast_exp2(__uint_as_float(v[e]) * L.scale_log2 - mu) : 0.f;
+                            const float p1 = v1 ? fast_exp2(__uint_as_float(v[e + 1]) * L.scale_log2 - mu) : 0.f;
+                            l += p0 + p1;
+                            pk[e >> 1] = pack_bf16(p0, p1);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    }
+                    tmem_st16(TM_P + lane_off + 16 * c8, pk);
+                }
+                tmem_wait_st();
+                const int hg = st.kvh * G + h;
+                if (i < L.S) p.lse[((size_t)st.b * L.Hq + hg) * L.S + i] = (mu + __log2f(l)) * kLn2;
+                if (m >= 2 && !mbar_wait(&sm.bar[B_LEMPTY + (m & 1)], ((m >> 1) - 1) & 1, abort, 21)) { stop = true; break; }
+                sm.rowinv[m & 1][r] = 1.f / l;
+                mbar_arrive(&sm.bar[B_LFULL + (m & 1)]);
+                tc_fence_before();
+                mbar_arrive(&sm.bar[B_PFULL]);
+            }
+            if (stop) break;
+        }
+    } else if (warp >= 8) {
+        // ================================================ prologue (K~, Q~ in place) + gate epilogue
+        const int r = tid - 256, wq = warp - 8;
+        const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+        int n_next = 0, m = 0, me = 0;
+        int pend_b[2] = {0, 0}, pend_h[2] = {0, 0}, pend_q[2] = {0, 0};
+        bool ok = true;
+
+        auto epilogue = [&](int e) -> bool {
+            const int buf = e & 1;
+            const int b = pend_b[buf], hg = pend_h[buf], i = pend_q[buf] * TF_BM + r;
+            const bool valid = i < L.S;
+            const size_t off = ((size_t)(b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hg) * kD;
+            if (!mbar_wait(&sm.bar[B_OFULL + buf], (e >> 1) & 1, abort, 30)) return false;
+            if (!mbar_wait(&sm.bar[B_LFULL + buf], (e >> 1) & 1, abort, 31)) return false;
+            const float inv = sm.rowinv[buf][r];
+            mbar_arrive(&sm.bar[B_LEMPTY + buf]);
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint4 gr[4];
+                if (valid) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) gr[q4] = __ldg(reinterpret_cast<const uint4*>(L.g + off + 32 * c) + q4);
+                }
+                uint32_t v[32];
+                tmem_ld32(TM_O0 + buf * 128 + lane_off + 32 * c, v);
+                tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const uint4 g4 = gr[q4];
+                        const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
+                        uint32_t ow[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const float2 gf = unpack_bf16(gw[e2]);
+                            // sigmoid(x) = 0.5 + 0.5 tanh(x / 2)
+                            const float s0 = fmaf(0.5f, fast_tanh(0.5f * gf.x), 0.5f);
+                            const float s1 = fmaf(0.5f, fast_tanh(0.5f * gf.y), 0.5f);
+                            const int col = 8 * q4 + 2 * e2;
+                            ow[e2] = pack_bf16(s0 * (__uint_as_float(v[col]) * inv), s1 * (__uint_as_float(v[col + 1]) * inv));
+                        }
+                        *reinterpret_cast<uint4*>(p.out + off + 32 * c + 8 * q4) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&sm.bar[B_OEMPTY + buf]);
+            return true;
+        };
+        auto prologue_k = [&](int n, int pos0) -> bool {
+            const int slot = n & 1;
+            if (!mbar_wait(&sm.bar[B_KFULL + slot], (n >> 1) & 1, abort, 32)) return false;
+            tf_angles(L, pos0 + r, sm.cs, r);
+            tf_prologue_row(sm.K[0] + slot * TF_HALF_BYTES, sm.K[1] + slot * TF_HALF_BYTES, r, sm.gk, L, sm.cs);
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.bar[B_KREADY + slot]);
+            return true;
+        };
+
+        for (int t = t_begin; t < t_end && ok; ++t) {
+            const StepInfo st = decode_step(L, t, t_begin, t_end);
+            const int q0 = st.qb * TF_BM;
+            if (st.fresh) ok = prologue_k(n_next++, q0 - TF_BN);
+            ok = ok && prologue_k(n_next++, q0);
+            if (!ok) break;
+            // the current K tile was rotated at q0 + r: the table already holds these angles
+            for (int h = 0; h < G; ++h, ++m) {
+                const int buf = m & 1;
+                if (!(ok = mbar_wait(&sm.bar[B_QFULL + buf], (m >> 1) & 1, abort, 33))) break;
+                tf_prologue_row(sm.Q[buf][0], sm.Q[buf][1], r, sm.gq, L, sm.cs);
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.bar[B_QREADY + buf]);
+                pend_b[buf] = st.b;
+                pend_h[buf] = st.kvh * G + h;
+                pend_q[buf] = st.qb;
+                if (m >= 1) {
+                    if (!(ok = epilogue(me))) break;
+                    ++me;
+                }
+            }
+        }
+        while (ok && me < m) {
+            if (!(ok = epilogue(me))) break;
+            ++me;
+        }
+    }
+
+    // ------------------------------------------------ teardown
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+    if (tid == 0 && sm.abort && p.err) atomicExch(p.err, sm.abort);
+}
+
+// ------------------------------------------------------------------ host side
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 4-D bf16 map {D, H, S, B} (innermost first), box {64, 1, 128, 1}, 128-byte swizzle
+bool make_map(CUtensorMap* map, const void* base, int H, int S, int B) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)S * H * kD * 2};
+    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool fwd_tc_supported(const LayerParams& L) {
+    return L.W <= TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1 && get_encode() != nullptr;
+}
+
+size_t fwd_tc_smem_bytes() { return sizeof(FwdTcSmem) + 1024; }
+
+cudaError_t launch_fwd_tc(const FwdParams& fp, int* err_word, cudaStream_t stream) {
+    FwdTcParams p;
+    p.L = fp.L;
+    p.out = fp.out;
+    p.lse = fp.lse;
+    p.err = err_word;
+    const int nqb = (fp.L.S + TF_BM - 1) / TF_BM;
+    const long long total = (long long)fp.L.B * fp.L.Hkv * nqb;
+    if (total > 0x7fffffffLL) return cudaErrorInvalidValue;
+    p.total_steps = (int)total;
+    if (!make_map(&p.tm_q, fp.L.q, fp.L.Hq, fp.L.S, fp.L.B) || !make_map(&p.tm_k, fp.L.k, fp.L.Hkv, fp.L.S, fp.L.B) ||
+        !make_map(&p.tm_v, fp.L.v, fp.L.Hkv, fp.L.S, fp.L.B))
+        return cudaErrorInvalidValue;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const size_t smem = fwd_tc_smem_bytes();
+    e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)(total < sms ? total : sms);
+    fwd_tc_kernel<<<grid, TF_THREADS, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace zgcm

@@ -3,20 +3,41 @@
 // .cu files of this directory.
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #include "../../include/zgcm_attn.h"
 #include "common.cuh"
 
 namespace zgcm {
 cudaError_t launch_fwd_mma(const FwdParams& p, cudaStream_t stream);
-cudaError_t launch_bwd_mma(const BwdParams& p, cudaStream_t stream, cudaEvent_t ev0, cudaEvent_t ev1);
+cudaError_t launch_fwd_tc(const FwdParams& p, int* err_word, cudaStream_t stream);
+bool fwd_tc_supported(const LayerParams& L);
+cudaError_t launch_bwd_mma(const BwdParams& p, cudaStream_t stream, void* const* events, int n_pairs);
+extern const char* const kBwdMmaKernelNames[];
+extern const int kBwdMmaKernelCount;
 int bwd_mma_n_k_parts(int B, int S, int Hkv);
 long long bwd_mma_n_q_parts(int B, int S, int Hq);
 }  // namespace zgcm
 
 using namespace zgcm;
 
+// Site of the last bounded device wait that expired (0 = none); read and cleared by
+// zgcm_attn_device_error().  Written only on a failure path.
+__device__ int zgcm_device_error_word;
+
 namespace {
+
+int* device_error_word() {
+    void* ptr = nullptr;
+    return cudaGetSymbolAddress(&ptr, zgcm_device_error_word) == cudaSuccess ? static_cast<int*>(ptr) : nullptr;
+}
+
+// Kernel choice: the tcgen05 sliding-window kernel where it applies, unless the caller
+// asks for the warp-MMA kernels with ZGCM_FORCE_MMA=1 (used to test both paths).
+bool force_mma() {
+    const char* e = getenv("ZGCM_FORCE_MMA");
+    return e && e[0] == '1';
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -59,7 +80,7 @@ void fill_layer(LayerParams& L, const void* q, const void* k, const void* v, con
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct BwdWorkspace {
-    size_t delta, dA, dq_acc, dgk, dgq, total;
+    size_t delta, dA, dA_lo, dgk, dgq, total;
     int n_k_parts;
     long long n_q_parts;
 };
@@ -72,7 +93,7 @@ BwdWorkspace bwd_layout(int B, int S, int Hq, int Hkv) {
     size_t off = 0;
     w.delta = off; off = align256(off + rows * sizeof(float));
     w.dA = off;    off = align256(off + rows * kD * sizeof(bf16));
-    w.dq_acc = off; off = align256(off + rows * kD * sizeof(float));
+    w.dA_lo = off; off = align256(off + rows * kD * sizeof(bf16));
     w.dgk = off;   off = align256(off + (size_t)w.n_k_parts * kD * sizeof(float));
     w.dgq = off;   off = align256(off + (size_t)w.n_q_parts * kD * sizeof(float));
     w.total = off;
@@ -114,7 +135,25 @@ int zgcm_attn_fwd(const void* q, const void* k, const void* v, const void* g,
     p.out = static_cast<bf16*>(out);
     p.lse = lse;
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-    return launch_fwd_mma(p, stream) == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
+    cudaError_t e;
+    if (!force_mma() && fwd_tc_supported(p.L))
+        e = launch_fwd_tc(p, device_error_word(), stream);
+    else
+        e = launch_fwd_mma(p, stream);
+    return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
+}
+
+int zgcm_attn_device_error(void) {
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, zgcm_device_error_word, sizeof(int)) != cudaSuccess) return ZGCM_ERR_CUDA;
+    if (v != 0 && cudaMemcpyToSymbol(zgcm_device_error_word, &zero, sizeof(int)) != cudaSuccess) return ZGCM_ERR_CUDA;
+    return v == 0 ? ZGCM_OK : ZGCM_ERR_TIMEOUT;
+}
+
+const char* zgcm_attn_fwd_kernel_name(int B, int S, int Hq, int Hkv, int rope_dims, int window) {
+    LayerParams L{};
+    L.B = B; L.S = S; L.Hq = Hq; L.Hkv = Hkv; L.rope_half = rope_dims / 2; L.W = window;
+    return (!force_mma() && fwd_tc_supported(L)) ? "fwd_tc_kernel" : "fwd_mma_kernel";
 }
 
 size_t zgcm_attn_bwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int window) {
@@ -131,7 +170,7 @@ int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void*
                         void* dq, void* dk, void* dv, void* dg,
                         float* dgamma_q, float* dgamma_k,
                         void* workspace, size_t workspace_bytes, void* cuda_stream,
-                        void* ev_main_begin, void* ev_main_end) {
+                        void* const* events, int n_pairs) {
     int st = check_shape(B, S, Hq, Hkv, D, rope_dims, rope_base, window, causal, eps, scale);
     if (st != ZGCM_OK) return st;
     if (!dgamma_q || !dgamma_k) return ZGCM_ERR_INVALID_ARG;
@@ -166,15 +205,18 @@ int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void*
     char* ws = static_cast<char*>(workspace);
     p.delta = reinterpret_cast<float*>(ws + w.delta);
     p.dA = reinterpret_cast<bf16*>(ws + w.dA);
-    p.dq_acc = reinterpret_cast<float*>(ws + w.dq_acc);
+    p.dA_lo = reinterpret_cast<bf16*>(ws + w.dA_lo);
     p.dgk_part = reinterpret_cast<float*>(ws + w.dgk);
     p.dgq_part = reinterpret_cast<float*>(ws + w.dgq);
     p.n_k_parts = w.n_k_parts;
     p.n_q_parts = (int)w.n_q_parts;
-    return launch_bwd_mma(p, stream, static_cast<cudaEvent_t>(ev_main_begin),
-                          static_cast<cudaEvent_t>(ev_main_end)) == cudaSuccess
-               ? ZGCM_OK
-               : ZGCM_ERR_CUDA;
+    if (n_pairs < 0 || (n_pairs > 0 && !events)) return ZGCM_ERR_INVALID_ARG;
+    return launch_bwd_mma(p, stream, events, n_pairs) == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
+}
+
+const char* zgcm_attn_bwd_kernel_name(int i, int S, int window) {
+    (void)S; (void)window;
+    return (i >= 0 && i < kBwdMmaKernelCount) ? kBwdMmaKernelNames[i] : nullptr;
 }
 
 int zgcm_attn_bwd(const void* q, const void* k, const void* v, const void* g,
@@ -188,7 +230,7 @@ int zgcm_attn_bwd(const void* q, const void* k, const void* v, const void* g,
     return zgcm_attn_bwd_timed(q, k, v, g, gamma_q, gamma_k, out, lse, dout, B, S, Hq, Hkv, D,
                                rope_dims, rope_base, window, causal, eps, scale, dq, dk, dv, dg,
                                dgamma_q, dgamma_k, workspace, workspace_bytes, cuda_stream,
-                               nullptr, nullptr);
+                               nullptr, 0);
 }
 
 }  // extern "C"

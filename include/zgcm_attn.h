@@ -115,9 +115,10 @@ int zgcm_attn_bwd(const void* q, const void* k, const void* v, const void* g,
 
 /*
  * Measurement variant of zgcm_attn_bwd: the same work on the same stream, and in addition
- * records ev_main_begin / ev_main_end (cudaEvent_t created by the caller) immediately
- * before and after the backward's main kernel (the key-major pass that forms dK, dV and
- * the dQ accumulation), so that kernel can be timed on its own.  Either event may be NULL.
+ * records events[2i] / events[2i+1] (cudaEvent_t created by the caller) immediately before
+ * and after the i-th kernel the backward launches, for i < n_pairs, so each kernel can be
+ * timed on its own.  zgcm_attn_bwd_kernel_name(i) names kernel i (NULL past the last).
+ * n_pairs may be 0 (then `events` may be NULL).
  */
 int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void* g,
                         const float* gamma_q, const float* gamma_k,
@@ -127,7 +128,26 @@ int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void*
                         void* dq, void* dk, void* dv, void* dg,
                         float* dgamma_q, float* dgamma_k,
                         void* workspace, size_t workspace_bytes, void* cuda_stream,
-                        void* ev_main_begin, void* ev_main_end);
+                        void* const* events, int n_pairs);
+
+/*
+ * Kernel zgcm_attn_fwd launches for this configuration (static string): "fwd_tc_kernel"
+ * (tcgen05/TMEM/TMA, sliding windows up to 128 with 42 rotated dims) or "fwd_mma_kernel".
+ * Setting the environment variable ZGCM_FORCE_MMA=1 selects the warp-MMA kernels.
+ */
+const char* zgcm_attn_fwd_kernel_name(int B, int S, int Hq, int Hkv, int rope_dims, int window);
+
+/*
+ * Device-side failure check.  Every wait inside the kernels is bounded; when one expires
+ * the kernel records where, releases what it holds and returns early (its outputs are then
+ * undefined).  This call synchronises the device, returns ZGCM_ERR_TIMEOUT if such a
+ * record exists (and clears it), ZGCM_OK otherwise.
+ */
+int zgcm_attn_device_error(void);
+
+/* Name of the i-th kernel zgcm_attn_bwd launches for this window/sequence configuration
+ * (static string), or NULL when i is past the last one. */
+const char* zgcm_attn_bwd_kernel_name(int i, int S, int window);
 
 #ifdef __cplusplus
 }

@@ -78,6 +78,26 @@ def test_small_full_compare(B, S, Hq, Hkv, W, R, base):
     assert_dgamma_close("dgamma_k", gr["dgamma_k"], ref["dgamma_k"])
 
 
+@pytest.mark.parametrize("B,S,W", [(1, 1024, 128), (2, 1000, 128), (1, 129, 7), (3, 260, 1), (1, 1, 128),
+                                   (2, 384, 100)])
+def test_forward_both_kernel_paths(B, S, W, monkeypatch):
+    """The tcgen05 sliding-window kernel (default for W <= 128, 42 rotated dims) and the
+    warp-MMA kernel (forced) both match the oracle on the same inputs."""
+    t = make_inputs(B, S, seed=100 + S + W)
+    d = _to_dev(t)
+    ref_out, ref_lse = _problem(t, window=W).forward()
+    monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
+    assert ga.zgcm_attn_fwd_kernel_name(B, S, 32, 8, 42, W) == "fwd_tc_kernel"
+    out_tc, lse_tc = _gpu_fwd(d, window=W)
+    assert ga.zgcm_attn_device_error() == 0
+    monkeypatch.setenv("ZGCM_FORCE_MMA", "1")
+    assert ga.zgcm_attn_fwd_kernel_name(B, S, 32, 8, 42, W) == "fwd_mma_kernel"
+    out_mma, lse_mma = _gpu_fwd(d, window=W)
+    for name, o, l in (("tc", out_tc, lse_tc), ("mma", out_mma, lse_mma)):
+        assert_bf16_close(f"out[{name}]", o, ref_out)
+        assert_lse_close(f"lse[{name}]", l, ref_lse)
+
+
 def test_empty_problem():
     for B, S in ((0, 16), (2, 0)):
         t = make_inputs(max(B, 1), max(S, 1), with_dout=True)
