@@ -168,6 +168,11 @@ def zgcm_attn_bwd(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dims=42,
     if kernel_events is None:
         st = load().zgcm_attn_bwd(*args)
     else:
+        st_obj = stream if stream is not None else torch.cuda.current_stream()
+        for pair in kernel_events:
+            for e in pair:
+                if not e.cuda_event:  # torch creates the CUDA event on its first record
+                    e.record(st_obj)
         flat = [ctypes.c_void_p(e.cuda_event) for pair in kernel_events for e in pair]
         arr = (ctypes.c_void_p * max(1, len(flat)))(*flat)
         st = load().zgcm_attn_bwd_timed(*args, arr, len(kernel_events))

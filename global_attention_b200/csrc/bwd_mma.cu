@@ -4,29 +4,33 @@
 //
 // Kernels, in launch order:
 //   bwd_pre     per (b, s, h) row: dg = dout*out*(1-sigmoid(g)); dA = dout*sigmoid(g)
-//               (out = sigmoid(g)*A, so neither needs the pre-gate A itself).  dA is kept
-//               as a pair of bf16 values hi + lo (hi = bf16(dA), lo = bf16(dA - hi)), and
-//               every product with dA is taken as hi-product + lo-product: with dA rounded
-//               to one bf16 the worst dk element near the sequence start was off by ~1.5x
-//               the final bf16 rounding.
-//   bwd_dq      per (b, query head, 64-query tile), two passes over the key tiles its window
-//               reaches: pass 1 forms Delta = sum_j P dP (P = exp(S - lse), dP = dA V^T);
-//               pass 2 forms dS = P (dP - Delta) and dQ~ = scale dS K~.  Epilogue: dq =
-//               RMSNorm/RoPE backward of dQ~, d_gamma_q partials; Delta saved for bwd_main.
-//               Delta is formed from the same P and dP the kernels use, not from the bf16
-//               `out`: rounding out and dA separately made Delta inconsistent with dP and
-//               roughly doubled the worst-case gradient error.  (A one-pass form,
-//               dQ~ = sum_j P dP k~_j - Delta sum_j P k~_j, cancels badly where the softmax
-//               is peaked and dS ~ 0, e.g. a one-key window.)
+//               (out = sigmoid(g)*A, so neither needs the pre-gate A itself).
+//   bwd_dq      per (b, query head, 64-query tile), two passes over the key tiles its
+//               window reaches.  Pass 1: the tile's own log-sum-exp (online max and sum)
+//               and Delta = sum_j P dP with P = exp(S - lse), dP = dA V^T.  Pass 2:
+//               dS = P (dP - Delta), dQ~ = scale dS K~.  Epilogue: dq = RMSNorm/RoPE
+//               backward of dQ~, d_gamma_q partials; lse and Delta saved for bwd_main.
 //   bwd_main    per (b, KV head, 64-key tile), over the Hq/Hkv query heads of the group and
 //               every 64-query tile whose window reaches the keys:
 //                 P^T = exp(S^T - lse), dV += P^T dA, dP^T = V dA^T, dS^T = P^T (dP^T - Delta),
-//                 dK~ += dS^T Q~;  epilogue: dk = RMSNorm/RoPE backward of scale*dK~, dv,
-//                 d_gamma_k partials.  P is split hi + lo like dA for the dV product
-//                 (P_hi dA_hi + P_hi dA_lo + P_lo dA_hi): the largest dv entries sit where
-//                 few keys share the softmax, and a single bf16 P left them short of the
-//                 bf16 output rounding.
-//   dgamma      fixed-order sum of the partials (deterministic)
+//                 dK~ += dS^T Q~;  epilogue: dk = RMSNorm/RoPE backward of scale dK~, dv,
+//                 d_gamma_k partials.
+//   dgamma      fixed-order sum of the partials (deterministic).
+//
+// Precision.  The stated bound is max-abs 2e-2 on bf16 gradients whose largest entries
+// (|x| ~ 4..6, where one bf16 rounding alone costs up to 0.0156) sit at the start of a
+// sequence, where a handful of keys share the softmax and a few products dominate each
+// sum.  Measured against the fp64 oracle in a CPU emulation of these kernels, three things
+// were needed to stay inside it:
+//   * Delta is formed from the kernels' own P and dP, and lse from their own scores (not
+//     from dout*out with a bf16 `out`, nor from the forward's lse): otherwise P and Delta
+//     are inconsistent with dP and the worst dk error doubles;
+//   * dS in the direct form P (dP - Delta): the one-pass sum_j P dP k~ - Delta sum_j P k~
+//     cancels where the softmax is peaked (one-key windows, the first tokens);
+//   * every operand of a gradient product is carried as a bf16 pair hi + lo
+//     (hi = bf16(x), lo = bf16(x - hi)) and the product as hi*hi + hi*lo + lo*hi:
+//     dA in dP and dV, P in dV, dS and q~ in dK, dS and k~ in dQ.
+// The scores S = q~ k~^T use the bf16 q~, k~ (hi) in both kernels, as the forward does.
 #include "common.cuh"
 
 namespace zgcm {
@@ -69,6 +73,300 @@ __global__ void __launch_bounds__(PRE_WARPS * 32) bwd_pre_kernel(const __grid_co
         make_uint2(pack_bf16(dav[0] - r01.x, dav[1] - r01.y), pack_bf16(dav[2] - r23.x, dav[3] - r23.y));
 }
 
+// =====================================================================  shared helpers
+
+// store this lane's 4 values of `row` as bf16 hi (and lo = bf16(y - hi) when lo != null)
+__device__ __forceinline__ void store_row_split(bf16* hi, bf16* lo, int row, const float y[4]) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t off = tile_off(row, lane >> 1) + (lane & 1) * 8;
+    const uint32_t h01 = pack_bf16(y[0], y[1]), h23 = pack_bf16(y[2], y[3]);
+    *reinterpret_cast<uint2*>(reinterpret_cast<char*>(hi) + off) = make_uint2(h01, h23);
+    if (lo) {
+        const float2 a = unpack_bf16(h01), b = unpack_bf16(h23);
+        *reinterpret_cast<uint2*>(reinterpret_cast<char*>(lo) + off) =
+            make_uint2(pack_bf16(y[0] - a.x, y[1] - a.y), pack_bf16(y[2] - b.x, y[3] - b.y));
+    }
+}
+
+// A-fragments (hi, lo) of a 16x16 slice of fp32 accumulators c[2 kk], c[2 kk + 1]
+__device__ __forceinline__ void split_frag(const float (*c)[4], int kk, uint32_t hi[4], uint32_t lo[4]) {
+    const float* f[4] = {&c[2 * kk][0], &c[2 * kk][2], &c[2 * kk + 1][0], &c[2 * kk + 1][2]};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        hi[u] = pack_bf16(f[u][0], f[u][1]);
+        const float2 h = unpack_bf16(hi[u]);
+        lo[u] = pack_bf16(f[u][0] - h.x, f[u][1] - h.y);
+    }
+}
+
+// =====================================================================  bwd_dq
+
+constexpr int DQ_BM = 64;       // query rows per CTA (4 warps x 16)
+constexpr int DQ_BN = 64;       // keys per tile
+constexpr int DQ_THREADS = 128;
+
+struct BwdDqSmem {
+    bf16 Q[DQ_BM * kD];         // Q~ (normalised + rotated), swizzled rows
+    bf16 dA[DQ_BM * kD];
+    bf16 dAl[DQ_BM * kD];
+    bf16 K[2][DQ_BN * kD];      // K~ hi
+    bf16 Kl[2][DQ_BN * kD];     // K~ lo
+    bf16 V[2][DQ_BN * kD];
+    float ybuf[DQ_THREADS / 32][kD];
+    float gq[kD], gk[kD];
+    float dgq[DQ_THREADS / 32][kD];
+};
+static_assert(DQ_BM * kD * 4 <= sizeof(bf16) * 2 * DQ_BN * kD, "dQ staging fits in the K buffers");
+
+// K~ (hi, lo) prologue (16 rows per warp) + V via cp.async for the key tile at kbase.
+__device__ __forceinline__ void dq_load_kv(const LayerParams& L, BwdDqSmem& sm, int buf, int b, int kvh,
+                                           int kbase) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        int c = tid + DQ_THREADS * i;
+        int row = c >> 4, ch = c & 15, pos = kbase + row;
+        bool ok = pos < L.S;
+        const bf16* src = L.v + ((size_t)(b * (size_t)L.S + (ok ? pos : 0)) * L.Hkv + kvh) * kD + ch * 8;
+        cp_async16(smem_u32(reinterpret_cast<char*>(sm.V[buf]) + tile_off(row, ch)), src, ok);
+    }
+    cp_async_commit();
+    uint2 raw[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        int pos = kbase + warp * 16 + r;
+        raw[r] = pos < L.S ? load_row4(L.k + ((size_t)(b * (size_t)L.S + pos) * L.Hkv + kvh) * kD)
+                           : make_uint2(0u, 0u);
+    }
+    const float g4[4] = {sm.gk[4 * lane], sm.gk[4 * lane + 1], sm.gk[4 * lane + 2], sm.gk[4 * lane + 3]};
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        int row = warp * 16 + r, pos = kbase + row;
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+        if (pos < L.S) prologue_row(raw[r], g4, L, pos, sm.ybuf[warp], y);
+        store_row_split(sm.K[buf], sm.Kl[buf], row, y);
+    }
+}
+
+__global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+    const LayerParams& L = p.L;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    BwdDqSmem& sm = *reinterpret_cast<BwdDqSmem*>(smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    const int nqt = (L.S + DQ_BM - 1) / DQ_BM;
+    int bid = blockIdx.x;
+    const int b = bid / (nqt * L.Hq);
+    bid -= b * nqt * L.Hq;
+    const int h = bid / nqt;
+    int qt = bid - h * nqt;
+    if (L.W >= L.S) qt = nqt - 1 - qt;  // full causal: longest rows first
+    const int kvh = h / L.G;
+    const int q0 = qt * DQ_BM;
+
+    if (tid < kD) {
+        sm.gq[tid] = L.gamma_q[tid];
+        sm.gk[tid] = L.gamma_k[tid];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        int c = tid + DQ_THREADS * i;
+        int row = c >> 4, ch = c & 15, pos = q0 + row;
+        bool ok = pos < L.S;
+        const size_t go = ((size_t)(b * (size_t)L.S + (ok ? pos : 0)) * L.Hq + h) * kD + ch * 8;
+        cp_async16(smem_u32(reinterpret_cast<char*>(sm.dA) + tile_off(row, ch)), p.dA + go, ok);
+        cp_async16(smem_u32(reinterpret_cast<char*>(sm.dAl) + tile_off(row, ch)), p.dA_lo + go, ok);
+    }
+    cp_async_commit();
+    __syncthreads();
+    const float gq4[4] = {sm.gq[4 * lane], sm.gq[4 * lane + 1], sm.gq[4 * lane + 2], sm.gq[4 * lane + 3]};
+    {
+        uint2 raw[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            int pos = q0 + warp * 16 + r;
+            raw[r] = pos < L.S ? load_row4(L.q + ((size_t)(b * (size_t)L.S + pos) * L.Hq + h) * kD)
+                               : make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            int row = warp * 16 + r, pos = q0 + row;
+            float y[4] = {0.f, 0.f, 0.f, 0.f};
+            if (pos < L.S) prologue_row(raw[r], gq4, L, pos, sm.ybuf[warp], y);
+            store_row_split(sm.Q, nullptr, row, y);
+        }
+    }
+
+    const int klo = max(0, q0 - L.W + 1);
+    const int khi = min(L.S - 1, q0 + DQ_BM - 1);
+    const int kt_lo = klo / DQ_BN, kt_hi = khi / DQ_BN;
+    const int wq0 = q0 + warp * 16;
+    const int r0 = wq0 + (lane >> 2), r1 = r0 + 8;
+
+    float dq[16][4];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dq[i][e] = 0.f;
+    // pass-1 statistics of rows r0, r1 (base-2 scores): running max, and this thread's
+    // partial sums of exp2(s - max) and of exp2(s - max) * dP
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f, n0 = 0.f, n1 = 0.f;
+    float lse0 = INFINITY, lse1 = INFINITY, del0 = 0.f, del1 = 0.f;
+    const int ntiles = kt_hi - kt_lo + 1;
+
+    dq_load_kv(L, sm, 0, b, kvh, kt_lo * DQ_BN);
+    for (int it = 0; it < 2 * ntiles; ++it) {
+        const int pass = it >= ntiles ? 1 : 0;
+        const int kt = kt_lo + (it - pass * ntiles);
+        const int buf = it & 1;
+        cp_async_wait<0>();
+        __syncthreads();
+        if (it + 1 < 2 * ntiles) dq_load_kv(L, sm, buf ^ 1, b, kvh, (kt_lo + ((it + 1) % ntiles)) * DQ_BN);
+        if (it == ntiles) {
+            // pass 1 complete: row sums over the quad of lanes holding each row
+            l0 += __shfl_xor_sync(0xffffffffu, l0, 1); l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, 1); l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+            n0 += __shfl_xor_sync(0xffffffffu, n0, 1); n0 += __shfl_xor_sync(0xffffffffu, n0, 2);
+            n1 += __shfl_xor_sync(0xffffffffu, n1, 1); n1 += __shfl_xor_sync(0xffffffffu, n1, 2);
+            if (l0 > 0.f) { lse0 = m0 + log2f(l0); del0 = n0 / l0; }
+            if (l1 > 0.f) { lse1 = m1 + log2f(l1); del1 = n1 / l1; }
+        }
+        const int kbase = kt * DQ_BN;
+        const bool live = wq0 < L.S && kbase <= wq0 + 15 && kbase + DQ_BN - 1 >= wq0 - L.W + 1;
+        if (!live) continue;
+        const uint32_t qs = smem_u32(sm.Q), das = smem_u32(sm.dA), dls = smem_u32(sm.dAl),
+                       ks = smem_u32(sm.K[buf]), kls = smem_u32(sm.Kl[buf]), vs = smem_u32(sm.V[buf]);
+        float s[8][4], dp[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[i][e] = dp[i][e] = 0.f;
+        // S = Q~ K~^T and dP = (dA_hi + dA_lo) V^T  (16 queries x 64 keys per warp)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            uint32_t aq[4], ad[4], al[4];
+            const uint32_t ao = tile_off(warp * 16 + (lane & 15), 2 * kk + (lane >> 4));
+            ldmatrix_x4(aq[0], aq[1], aq[2], aq[3], qs + ao);
+            ldmatrix_x4(ad[0], ad[1], ad[2], ad[3], das + ao);
+            ldmatrix_x4(al[0], al[1], al[2], al[3], dls + ao);
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t b0, b1, b2, b3;
+                const uint32_t bo = tile_off(np * 16 + (lane >> 4) * 8 + (lane & 7), 2 * kk + ((lane >> 3) & 1));
+                ldmatrix_x4(b0, b1, b2, b3, ks + bo);
+                mma_bf16(s[2 * np], aq, b0, b1);
+                mma_bf16(s[2 * np + 1], aq, b2, b3);
+                ldmatrix_x4(b0, b1, b2, b3, vs + bo);
+                mma_bf16(dp[2 * np], ad, b0, b1);
+                mma_bf16(dp[2 * np + 1], ad, b2, b3);
+                mma_bf16(dp[2 * np], al, b0, b1);
+                mma_bf16(dp[2 * np + 1], al, b2, b3);
+            }
+        }
+        // masked base-2 scores
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = kbase + nt * 8 + 2 * (lane & 3) + (e & 1);
+                const int i = e < 2 ? r0 : r1;
+                const bool vis = j <= i && j > i - L.W && j < L.S && i < L.S;
+                s[nt][e] = vis ? s[nt][e] * L.scale_log2 : -INFINITY;
+            }
+        }
+        if (pass == 0) {
+            float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                mx0 = fmaxf(mx0, fmaxf(s[nt][0], s[nt][1]));
+                mx1 = fmaxf(mx1, fmaxf(s[nt][2], s[nt][3]));
+            }
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+            const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
+            const float c0 = exp2f(m0 - mu0), c1 = exp2f(m1 - mu1);
+            l0 *= c0; n0 *= c0; l1 *= c1; n1 *= c1;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float ev = exp2f(s[nt][e] - (e < 2 ? mu0 : mu1));
+                    if (e < 2) { l0 += ev; n0 += ev * dp[nt][e]; } else { l1 += ev; n1 += ev * dp[nt][e]; }
+                }
+            }
+            m0 = mn0; m1 = mn1;
+            continue;
+        }
+        // pass 2: dS = P (dP - Delta), dQ~ += dS K~ as hi*hi + lo*hi + hi*lo
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float pv = exp2f(s[nt][e] - (e < 2 ? lse0 : lse1));
+                dp[nt][e] = pv * (dp[nt][e] - (e < 2 ? del0 : del1));
+            }
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t ah[4], al[4];
+            split_frag(dp, kk, ah, al);
+#pragma unroll
+            for (int dn = 0; dn < 8; ++dn) {
+                uint32_t b0, b1, b2, b3;
+                const uint32_t bo = tile_off(16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * dn + (lane >> 4));
+                ldmatrix_x4_trans(b0, b1, b2, b3, ks + bo);
+                mma_bf16(dq[2 * dn], ah, b0, b1);
+                mma_bf16(dq[2 * dn + 1], ah, b2, b3);
+                mma_bf16(dq[2 * dn], al, b0, b1);
+                mma_bf16(dq[2 * dn + 1], al, b2, b3);
+                ldmatrix_x4_trans(b0, b1, b2, b3, kls + bo);
+                mma_bf16(dq[2 * dn], ah, b0, b1);
+                mma_bf16(dq[2 * dn + 1], ah, b2, b3);
+            }
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+
+    if ((lane & 3) == 0) {
+        const size_t base = ((size_t)b * L.Hq + h) * L.S;
+        if (r0 < L.S) { p.delta[base + r0] = del0; p.lse2[base + r0] = lse0; }
+        if (r1 < L.S) { p.delta[base + r1] = del1; p.lse2[base + r1] = lse1; }
+    }
+    // dQ~ (scaled) -> fp32 staging [64][128] in the K buffers
+    float* stage = reinterpret_cast<float*>(sm.K[0]);
+    const int lr0 = warp * 16 + (lane >> 2), lr1 = lr0 + 8;
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+        const int col = nt * 8 + 2 * (lane & 3);
+        *reinterpret_cast<float2*>(stage + lr0 * kD + col) = make_float2(L.scale * dq[nt][0], L.scale * dq[nt][1]);
+        *reinterpret_cast<float2*>(stage + lr1 * kD + col) = make_float2(L.scale * dq[nt][2], L.scale * dq[nt][3]);
+    }
+    __syncthreads();
+    float dgacc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int r = 0; r < 16; ++r) {
+        const int row = warp * 16 + r, pos = q0 + row;
+        if (pos >= L.S) break;
+        const size_t off = ((size_t)(b * (size_t)L.S + pos) * L.Hq + h) * kD;
+        uint2 raw = load_row4(L.q + off);
+        float4 d4 = *reinterpret_cast<const float4*>(stage + row * kD + 4 * lane);
+        float dy[4] = {d4.x, d4.y, d4.z, d4.w}, dx[4];
+        prologue_row_backward(raw, gq4, L, pos, sm.ybuf[warp], dy, dx, dgacc);
+        *reinterpret_cast<uint2*>(p.dq + off + 4 * lane) = make_uint2(pack_bf16(dx[0], dx[1]), pack_bf16(dx[2], dx[3]));
+    }
+    *reinterpret_cast<float4*>(&sm.dgq[warp][4 * lane]) = make_float4(dgacc[0], dgacc[1], dgacc[2], dgacc[3]);
+    __syncthreads();
+    if (tid < kD) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < DQ_THREADS / 32; ++w) t += sm.dgq[w][tid];
+        p.dgq_part[(size_t)blockIdx.x * kD + tid] = t;
+    }
+}
+
 // =====================================================================  bwd_main
 
 constexpr int BM_KEYS = 64;     // keys per CTA (4 warps x 16)
@@ -78,21 +376,16 @@ constexpr int BM_THREADS = 128;
 struct BwdMmaSmem {
     bf16 K[BM_KEYS * kD];     // K~ (normalised + rotated), swizzled rows
     bf16 V[BM_KEYS * kD];
-    bf16 Q[BM_Q * kD];        // Q~ of the current query tile
+    bf16 Q[BM_Q * kD];        // Q~ hi of the current query tile
+    bf16 Ql[BM_Q * kD];       // Q~ lo
     bf16 dA[BM_Q * kD];
-    bf16 dAl[BM_Q * kD];      // low part of dA
-    float lse2[BM_Q];         // lse * log2(e)
+    bf16 dAl[BM_Q * kD];
+    float lse2[BM_Q];         // base-2 log-sum-exp from bwd_dq
     float delta[BM_Q];
     float ybuf[BM_THREADS / 32][kD];
     float gq[kD], gk[kD];
     float dgk[BM_THREADS / 32][kD];
 };
-
-__device__ __forceinline__ void bm_store_row(bf16* tile, int row, const float y[4]) {
-    const int lane = threadIdx.x & 31;
-    uint2 u = make_uint2(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]));
-    *reinterpret_cast<uint2*>(reinterpret_cast<char*>(tile) + tile_off(row, lane >> 1) + (lane & 1) * 8) = u;
-}
 
 __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_constant__ BwdParams p) {
     const LayerParams& L = p.L;
@@ -130,7 +423,7 @@ __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_co
             int row = warp * 16 + r, pos = k0 + row;
             float y[4] = {0.f, 0.f, 0.f, 0.f};
             if (pos < L.S) prologue_row(raw[r], gk4, L, pos, sm.ybuf[warp], y);
-            bm_store_row(sm.K, row, y);
+            store_row_split(sm.K, nullptr, row, y);
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -159,8 +452,7 @@ __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_co
         const int h = kvh * L.G + hh;
         for (int qt = qt_lo; qt <= qt_hi; ++qt) {
             const int q0 = qt * BM_Q;
-            __syncthreads();  // previous tile's readers of Q, dA, dS are done
-            // dA tile (cp.async), Q~ tile (prologue), lse, Delta
+            __syncthreads();  // previous tile's readers of Q, dA are done
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 int c = tid + BM_THREADS * i;
@@ -174,7 +466,7 @@ __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_co
             if (tid < BM_Q) {
                 int pos = q0 + tid;
                 bool ok = pos < L.S;
-                sm.lse2[tid] = ok ? p.lse[((size_t)b * L.Hq + h) * L.S + pos] * kLog2e : INFINITY;
+                sm.lse2[tid] = ok ? p.lse2[((size_t)b * L.Hq + h) * L.S + pos] : INFINITY;
                 sm.delta[tid] = ok ? p.delta[((size_t)b * L.Hq + h) * L.S + pos] : 0.f;
             }
             {
@@ -190,7 +482,7 @@ __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_co
                     int row = warp * 16 + r, pos = q0 + row;
                     float y[4] = {0.f, 0.f, 0.f, 0.f};
                     if (pos < L.S) prologue_row(raw[r], gq4, L, pos, sm.ybuf[warp], y);
-                    bm_store_row(sm.Q, row, y);
+                    store_row_split(sm.Q, sm.Ql, row, y);
                 }
             }
             cp_async_wait<0>();
@@ -198,80 +490,76 @@ __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_co
 
             // warp-level skip: keys [kw0, kw0+15] are seen by queries [kw0, kw0+15+W-1]
             const bool live = kw0 < L.S && q0 <= kw0 + 15 + L.W - 1 && q0 + BM_Q - 1 >= kw0;
-            const uint32_t kb = smem_u32(sm.K), vb = smem_u32(sm.V), qb = smem_u32(sm.Q), db = smem_u32(sm.dA),
-                           dlb = smem_u32(sm.dAl);
-            if (live) {
-                float st[8][4], dpt[8][4];
+            if (!live) continue;
+            const uint32_t kb = smem_u32(sm.K), vb = smem_u32(sm.V), qb = smem_u32(sm.Q), qlb = smem_u32(sm.Ql),
+                           db = smem_u32(sm.dA), dlb = smem_u32(sm.dAl);
+            float st[8][4], dpt[8][4];
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < 8; ++i)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) st[i][e] = dpt[i][e] = 0.f;
-                // S^T = K~ Q~^T and dP^T = V dA^T  (16 keys x 64 queries)
+                for (int e = 0; e < 4; ++e) st[i][e] = dpt[i][e] = 0.f;
+            // S^T = K~ Q~^T and dP^T = V (dA_hi + dA_lo)^T  (16 keys x 64 queries)
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    uint32_t ak[4], av[4];
-                    ldmatrix_x4(ak[0], ak[1], ak[2], ak[3], kb + tile_off(warp * 16 + (lane & 15), 2 * kk + (lane >> 4)));
-                    ldmatrix_x4(av[0], av[1], av[2], av[3], vb + tile_off(warp * 16 + (lane & 15), 2 * kk + (lane >> 4)));
+            for (int kk = 0; kk < 8; ++kk) {
+                uint32_t ak[4], av[4];
+                const uint32_t ao = tile_off(warp * 16 + (lane & 15), 2 * kk + (lane >> 4));
+                ldmatrix_x4(ak[0], ak[1], ak[2], ak[3], kb + ao);
+                ldmatrix_x4(av[0], av[1], av[2], av[3], vb + ao);
 #pragma unroll
-                    for (int np = 0; np < 4; ++np) {
-                        uint32_t b0, b1, b2, b3;
-                        const int rr = np * 16 + (lane >> 4) * 8 + (lane & 7), cc = 2 * kk + ((lane >> 3) & 1);
-                        ldmatrix_x4(b0, b1, b2, b3, qb + tile_off(rr, cc));
-                        mma_bf16(st[2 * np], ak, b0, b1);
-                        mma_bf16(st[2 * np + 1], ak, b2, b3);
-                        ldmatrix_x4(b0, b1, b2, b3, db + tile_off(rr, cc));
-                        mma_bf16(dpt[2 * np], av, b0, b1);
-                        mma_bf16(dpt[2 * np + 1], av, b2, b3);
-                        ldmatrix_x4(b0, b1, b2, b3, dlb + tile_off(rr, cc));
-                        mma_bf16(dpt[2 * np], av, b0, b1);
-                        mma_bf16(dpt[2 * np + 1], av, b2, b3);
-                    }
+                for (int np = 0; np < 4; ++np) {
+                    uint32_t b0, b1, b2, b3;
+                    const uint32_t bo = tile_off(np * 16 + (lane >> 4) * 8 + (lane & 7), 2 * kk + ((lane >> 3) & 1));
+                    ldmatrix_x4(b0, b1, b2, b3, qb + bo);
+                    mma_bf16(st[2 * np], ak, b0, b1);
+                    mma_bf16(st[2 * np + 1], ak, b2, b3);
+                    ldmatrix_x4(b0, b1, b2, b3, db + bo);
+                    mma_bf16(dpt[2 * np], av, b0, b1);
+                    mma_bf16(dpt[2 * np + 1], av, b2, b3);
+                    ldmatrix_x4(b0, b1, b2, b3, dlb + bo);
+                    mma_bf16(dpt[2 * np], av, b0, b1);
+                    mma_bf16(dpt[2 * np + 1], av, b2, b3);
                 }
-                // P^T = exp2(S^T*scale*log2e - lse2), masked; dS^T = P^T (dP^T - Delta)
+            }
+            // P^T = exp2(S^T*scale*log2e - lse2), masked; dS^T = P^T (dP^T - Delta)
 #pragma unroll
-                for (int nt = 0; nt < 8; ++nt) {
+            for (int nt = 0; nt < 8; ++nt) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        int ql = nt * 8 + 2 * (lane & 3) + (e & 1);
-                        int i = q0 + ql;
-                        int j = e < 2 ? j0 : j1;
-                        bool vis = j <= i && j > i - L.W && i < L.S && j < L.S;
-                        float pv = vis ? exp2f(st[nt][e] * L.scale_log2 - sm.lse2[ql]) : 0.f;
-                        st[nt][e] = pv;
-                        dpt[nt][e] = pv * (dpt[nt][e] - sm.delta[ql]);
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    int ql = nt * 8 + 2 * (lane & 3) + (e & 1);
+                    int i = q0 + ql;
+                    int j = e < 2 ? j0 : j1;
+                    bool vis = j <= i && j > i - L.W && i < L.S && j < L.S;
+                    float pv = vis ? exp2f(st[nt][e] * L.scale_log2 - sm.lse2[ql]) : 0.f;
+                    st[nt][e] = pv;
+                    dpt[nt][e] = pv * (dpt[nt][e] - sm.delta[ql]);
                 }
-                // dV += P^T dA ; dK~ += dS^T Q~   (A from registers, B via ldmatrix.trans)
+            }
+            // dV += P^T dA ; dK~ += dS^T Q~   (hi*hi + lo*hi + hi*lo)
 #pragma unroll
-                for (int kq = 0; kq < 4; ++kq) {
-                    uint32_t ap[4], apl[4], as[4];
-                    const float* pf[4] = {&st[2 * kq][0], &st[2 * kq][2], &st[2 * kq + 1][0], &st[2 * kq + 1][2]};
+            for (int kq = 0; kq < 4; ++kq) {
+                uint32_t ph[4], pl[4], sh[4], sl[4];
+                split_frag(st, kq, ph, pl);
+                split_frag(dpt, kq, sh, sl);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        ap[u] = pack_bf16(pf[u][0], pf[u][1]);
-                        const float2 hi = unpack_bf16(ap[u]);
-                        apl[u] = pack_bf16(pf[u][0] - hi.x, pf[u][1] - hi.y);
-                    }
-                    as[0] = pack_bf16(dpt[2 * kq][0], dpt[2 * kq][1]);
-                    as[1] = pack_bf16(dpt[2 * kq][2], dpt[2 * kq][3]);
-                    as[2] = pack_bf16(dpt[2 * kq + 1][0], dpt[2 * kq + 1][1]);
-                    as[3] = pack_bf16(dpt[2 * kq + 1][2], dpt[2 * kq + 1][3]);
-#pragma unroll
-                    for (int dn = 0; dn < 8; ++dn) {
-                        uint32_t b0, b1, b2, b3;
-                        const int rr = 16 * kq + (lane & 7) + ((lane >> 3) & 1) * 8, cc = 2 * dn + (lane >> 4);
-                        ldmatrix_x4_trans(b0, b1, b2, b3, db + tile_off(rr, cc));
-                        mma_bf16(dv[2 * dn], ap, b0, b1);
-                        mma_bf16(dv[2 * dn + 1], ap, b2, b3);
-                        mma_bf16(dv[2 * dn], apl, b0, b1);
-                        mma_bf16(dv[2 * dn + 1], apl, b2, b3);
-                        ldmatrix_x4_trans(b0, b1, b2, b3, dlb + tile_off(rr, cc));
-                        mma_bf16(dv[2 * dn], ap, b0, b1);
-                        mma_bf16(dv[2 * dn + 1], ap, b2, b3);
-                        ldmatrix_x4_trans(b0, b1, b2, b3, qb + tile_off(rr, cc));
-                        mma_bf16(dk[2 * dn], as, b0, b1);
-                        mma_bf16(dk[2 * dn + 1], as, b2, b3);
-                    }
+                for (int dn = 0; dn < 8; ++dn) {
+                    uint32_t b0, b1, b2, b3;
+                    const uint32_t bo = tile_off(16 * kq + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * dn + (lane >> 4));
+                    ldmatrix_x4_trans(b0, b1, b2, b3, db + bo);
+                    mma_bf16(dv[2 * dn], ph, b0, b1);
+                    mma_bf16(dv[2 * dn + 1], ph, b2, b3);
+                    mma_bf16(dv[2 * dn], pl, b0, b1);
+                    mma_bf16(dv[2 * dn + 1], pl, b2, b3);
+                    ldmatrix_x4_trans(b0, b1, b2, b3, dlb + bo);
+                    mma_bf16(dv[2 * dn], ph, b0, b1);
+                    mma_bf16(dv[2 * dn + 1], ph, b2, b3);
+                    ldmatrix_x4_trans(b0, b1, b2, b3, qb + bo);
+                    mma_bf16(dk[2 * dn], sh, b0, b1);
+                    mma_bf16(dk[2 * dn + 1], sh, b2, b3);
+                    mma_bf16(dk[2 * dn], sl, b0, b1);
+                    mma_bf16(dk[2 * dn + 1], sl, b2, b3);
+                    ldmatrix_x4_trans(b0, b1, b2, b3, qlb + bo);
+                    mma_bf16(dk[2 * dn], sh, b0, b1);
+                    mma_bf16(dk[2 * dn + 1], sh, b2, b3);
                 }
             }
         }
@@ -287,7 +575,7 @@ __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_co
             *reinterpret_cast<uint32_t*>(p.dv + ((size_t)(b * (size_t)L.S + j1) * L.Hkv + kvh) * kD + col) = pack_bf16(dv[nt][2], dv[nt][3]);
     }
     __syncthreads();
-    float* stage = reinterpret_cast<float*>(sm.Q);  // Q + dA = 32 KB = [64][128] fp32 (dAl follows)
+    float* stage = reinterpret_cast<float*>(sm.Q);  // Q + Ql = 32 KB = [64][128] fp32
     {
         const int rr0 = warp * 16 + (lane >> 2), rr1 = rr0 + 8;
 #pragma unroll
@@ -319,255 +607,6 @@ __global__ void __launch_bounds__(BM_THREADS, 1) bwd_main_kernel(const __grid_co
     }
 }
 
-// =====================================================================  bwd_dq
-
-constexpr int DQ_BM = 64;       // query rows per CTA (4 warps x 16)
-constexpr int DQ_BN = 64;       // keys per tile
-constexpr int DQ_THREADS = 128;
-
-struct BwdDqSmem {
-    bf16 Q[DQ_BM * kD];         // Q~ (normalised + rotated), swizzled rows
-    bf16 dA[DQ_BM * kD];
-    bf16 dAl[DQ_BM * kD];       // low part of dA
-    bf16 K[2][DQ_BN * kD];      // K~
-    bf16 V[2][DQ_BN * kD];
-    float lse2[DQ_BM];
-    float ybuf[DQ_THREADS / 32][kD];
-    float gq[kD], gk[kD];
-    float dgq[DQ_THREADS / 32][kD];
-};
-static_assert(DQ_BM * kD * 4 <= sizeof(bf16) * 4 * DQ_BN * kD, "dQ staging fits in the K/V buffers");
-
-// K~ prologue (16 rows per warp) + V via cp.async for the key tile at kbase.
-__device__ __forceinline__ void dq_load_kv(const LayerParams& L, BwdDqSmem& sm, int buf, int b, int kvh,
-                                           int kbase) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        int c = tid + DQ_THREADS * i;
-        int row = c >> 4, ch = c & 15, pos = kbase + row;
-        bool ok = pos < L.S;
-        const bf16* src = L.v + ((size_t)(b * (size_t)L.S + (ok ? pos : 0)) * L.Hkv + kvh) * kD + ch * 8;
-        cp_async16(smem_u32(reinterpret_cast<char*>(sm.V[buf]) + tile_off(row, ch)), src, ok);
-    }
-    cp_async_commit();
-    uint2 raw[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-        int pos = kbase + warp * 16 + r;
-        raw[r] = pos < L.S ? load_row4(L.k + ((size_t)(b * (size_t)L.S + pos) * L.Hkv + kvh) * kD)
-                           : make_uint2(0u, 0u);
-    }
-    const float g4[4] = {sm.gk[4 * lane], sm.gk[4 * lane + 1], sm.gk[4 * lane + 2], sm.gk[4 * lane + 3]};
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-        int row = warp * 16 + r, pos = kbase + row;
-        float y[4] = {0.f, 0.f, 0.f, 0.f};
-        if (pos < L.S) prologue_row(raw[r], g4, L, pos, sm.ybuf[warp], y);
-        bm_store_row(sm.K[buf], row, y);
-    }
-}
-
-__global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_constant__ BwdParams p) {
-    const LayerParams& L = p.L;
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    BwdDqSmem& sm = *reinterpret_cast<BwdDqSmem*>(smem_raw);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-    const int nqt = (L.S + DQ_BM - 1) / DQ_BM;
-    int bid = blockIdx.x;
-    const int b = bid / (nqt * L.Hq);
-    bid -= b * nqt * L.Hq;
-    const int h = bid / nqt;
-    int qt = bid - h * nqt;
-    if (L.W >= L.S) qt = nqt - 1 - qt;  // full causal: longest rows first
-    const int kvh = h / L.G;
-    const int q0 = qt * DQ_BM;
-
-    if (tid < kD) {
-        sm.gq[tid] = L.gamma_q[tid];
-        sm.gk[tid] = L.gamma_k[tid];
-    }
-    // dA tile
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        int c = tid + DQ_THREADS * i;
-        int row = c >> 4, ch = c & 15, pos = q0 + row;
-        bool ok = pos < L.S;
-        const size_t go = ((size_t)(b * (size_t)L.S + (ok ? pos : 0)) * L.Hq + h) * kD + ch * 8;
-        cp_async16(smem_u32(reinterpret_cast<char*>(sm.dA) + tile_off(row, ch)), p.dA + go, ok);
-        cp_async16(smem_u32(reinterpret_cast<char*>(sm.dAl) + tile_off(row, ch)), p.dA_lo + go, ok);
-    }
-    cp_async_commit();
-    if (tid < DQ_BM) {
-        int pos = q0 + tid;
-        sm.lse2[tid] = pos < L.S ? p.lse[((size_t)b * L.Hq + h) * L.S + pos] * kLog2e : INFINITY;
-    }
-    __syncthreads();
-    const float gq4[4] = {sm.gq[4 * lane], sm.gq[4 * lane + 1], sm.gq[4 * lane + 2], sm.gq[4 * lane + 3]};
-    {
-        uint2 raw[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            int pos = q0 + warp * 16 + r;
-            raw[r] = pos < L.S ? load_row4(L.q + ((size_t)(b * (size_t)L.S + pos) * L.Hq + h) * kD)
-                               : make_uint2(0u, 0u);
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            int row = warp * 16 + r, pos = q0 + row;
-            float y[4] = {0.f, 0.f, 0.f, 0.f};
-            if (pos < L.S) prologue_row(raw[r], gq4, L, pos, sm.ybuf[warp], y);
-            bm_store_row(sm.Q, row, y);
-        }
-    }
-
-    const int klo = max(0, q0 - L.W + 1);
-    const int khi = min(L.S - 1, q0 + DQ_BM - 1);
-    const int kt_lo = klo / DQ_BN, kt_hi = khi / DQ_BN;
-    const int wq0 = q0 + warp * 16;
-    const int r0 = wq0 + (lane >> 2), r1 = r0 + 8;
-    const int lr0 = warp * 16 + (lane >> 2), lr1 = lr0 + 8;
-
-    float dq[16][4];
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dq[i][e] = 0.f;
-    float ds0 = 0.f, ds1 = 0.f;  // Delta of rows r0, r1 (this thread's columns during pass 1)
-    const int ntiles = kt_hi - kt_lo + 1;
-
-    dq_load_kv(L, sm, 0, b, kvh, kt_lo * DQ_BN);
-    for (int it = 0; it < 2 * ntiles; ++it) {
-        const int pass = it >= ntiles ? 1 : 0;
-        const int kt = kt_lo + (it - pass * ntiles);
-        const int buf = it & 1;
-        cp_async_wait<0>();
-        __syncthreads();
-        if (it + 1 < 2 * ntiles) {
-            const int nkt = kt_lo + ((it + 1) % ntiles);
-            dq_load_kv(L, sm, buf ^ 1, b, kvh, nkt * DQ_BN);
-        }
-        if (pass == 1 && it == ntiles) {
-            // Delta complete: sum over the quad of lanes holding each row
-            ds0 += __shfl_xor_sync(0xffffffffu, ds0, 1);
-            ds0 += __shfl_xor_sync(0xffffffffu, ds0, 2);
-            ds1 += __shfl_xor_sync(0xffffffffu, ds1, 1);
-            ds1 += __shfl_xor_sync(0xffffffffu, ds1, 2);
-        }
-        const int kbase = kt * DQ_BN;
-        const bool live = wq0 < L.S && kbase <= wq0 + 15 && kbase + DQ_BN - 1 >= wq0 - L.W + 1;
-        if (!live) continue;
-        const uint32_t qs = smem_u32(sm.Q), das = smem_u32(sm.dA), dls = smem_u32(sm.dAl),
-                       ks = smem_u32(sm.K[buf]), vs = smem_u32(sm.V[buf]);
-        float s[8][4], dp[8][4];
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) s[i][e] = dp[i][e] = 0.f;
-        // S = Q~ K~^T and dP = dA V^T  (16 queries x 64 keys per warp)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            uint32_t aq[4], ad[4], al[4];
-            ldmatrix_x4(aq[0], aq[1], aq[2], aq[3], qs + tile_off(warp * 16 + (lane & 15), 2 * kk + (lane >> 4)));
-            ldmatrix_x4(ad[0], ad[1], ad[2], ad[3], das + tile_off(warp * 16 + (lane & 15), 2 * kk + (lane >> 4)));
-            ldmatrix_x4(al[0], al[1], al[2], al[3], dls + tile_off(warp * 16 + (lane & 15), 2 * kk + (lane >> 4)));
-#pragma unroll
-            for (int np = 0; np < 4; ++np) {
-                uint32_t b0, b1, b2, b3;
-                const int rr = np * 16 + (lane >> 4) * 8 + (lane & 7), cc = 2 * kk + ((lane >> 3) & 1);
-                ldmatrix_x4(b0, b1, b2, b3, ks + tile_off(rr, cc));
-                mma_bf16(s[2 * np], aq, b0, b1);
-                mma_bf16(s[2 * np + 1], aq, b2, b3);
-                ldmatrix_x4(b0, b1, b2, b3, vs + tile_off(rr, cc));
-                mma_bf16(dp[2 * np], ad, b0, b1);
-                mma_bf16(dp[2 * np + 1], ad, b2, b3);
-                mma_bf16(dp[2 * np], al, b0, b1);
-                mma_bf16(dp[2 * np + 1], al, b2, b3);
-            }
-        }
-        const float l0 = sm.lse2[lr0], l1 = sm.lse2[lr1];
-        if (pass == 0) {
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    int j = kbase + nt * 8 + 2 * (lane & 3) + (e & 1);
-                    int i = e < 2 ? r0 : r1;
-                    bool vis = j <= i && j > i - L.W && j < L.S && i < L.S;
-                    float pv = vis ? exp2f(s[nt][e] * L.scale_log2 - (e < 2 ? l0 : l1)) : 0.f;
-                    if (e < 2) ds0 += pv * dp[nt][e]; else ds1 += pv * dp[nt][e];
-                }
-            }
-            continue;
-        }
-        // pass 1: dS = P (dP - Delta), dQ~ += dS K~  (A from registers, B = K~ via ldmatrix.trans)
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                int j = kbase + nt * 8 + 2 * (lane & 3) + (e & 1);
-                int i = e < 2 ? r0 : r1;
-                bool vis = j <= i && j > i - L.W && j < L.S && i < L.S;
-                float pv = vis ? exp2f(s[nt][e] * L.scale_log2 - (e < 2 ? l0 : l1)) : 0.f;
-                dp[nt][e] = pv * (dp[nt][e] - (e < 2 ? ds0 : ds1));
-            }
-        }
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            uint32_t aw[4];
-            aw[0] = pack_bf16(dp[2 * kk][0], dp[2 * kk][1]);
-            aw[1] = pack_bf16(dp[2 * kk][2], dp[2 * kk][3]);
-            aw[2] = pack_bf16(dp[2 * kk + 1][0], dp[2 * kk + 1][1]);
-            aw[3] = pack_bf16(dp[2 * kk + 1][2], dp[2 * kk + 1][3]);
-#pragma unroll
-            for (int dn = 0; dn < 8; ++dn) {
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4_trans(b0, b1, b2, b3,
-                                  ks + tile_off(16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8, 2 * dn + (lane >> 4)));
-                mma_bf16(dq[2 * dn], aw, b0, b1);
-                mma_bf16(dq[2 * dn + 1], aw, b2, b3);
-            }
-        }
-    }
-    cp_async_wait<0>();
-    __syncthreads();
-    if (ntiles == 0) { ds0 = ds1 = 0.f; }
-
-    if ((lane & 3) == 0) {
-        if (r0 < L.S) p.delta[((size_t)b * L.Hq + h) * L.S + r0] = ds0;
-        if (r1 < L.S) p.delta[((size_t)b * L.Hq + h) * L.S + r1] = ds1;
-    }
-    // dQ~ (scaled) -> fp32 staging [64][128] in the K/V buffers
-    float* stage = reinterpret_cast<float*>(sm.K[0]);
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-        const int col = nt * 8 + 2 * (lane & 3);
-        *reinterpret_cast<float2*>(stage + lr0 * kD + col) = make_float2(L.scale * dq[nt][0], L.scale * dq[nt][1]);
-        *reinterpret_cast<float2*>(stage + lr1 * kD + col) = make_float2(L.scale * dq[nt][2], L.scale * dq[nt][3]);
-    }
-    __syncthreads();
-    float dgacc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int r = 0; r < 16; ++r) {
-        const int row = warp * 16 + r, pos = q0 + row;
-        if (pos >= L.S) break;
-        const size_t off = ((size_t)(b * (size_t)L.S + pos) * L.Hq + h) * kD;
-        uint2 raw = load_row4(L.q + off);
-        float4 d4 = *reinterpret_cast<const float4*>(stage + row * kD + 4 * lane);
-        float dy[4] = {d4.x, d4.y, d4.z, d4.w}, dx[4];
-        prologue_row_backward(raw, gq4, L, pos, sm.ybuf[warp], dy, dx, dgacc);
-        *reinterpret_cast<uint2*>(p.dq + off + 4 * lane) = make_uint2(pack_bf16(dx[0], dx[1]), pack_bf16(dx[2], dx[3]));
-    }
-    *reinterpret_cast<float4*>(&sm.dgq[warp][4 * lane]) = make_float4(dgacc[0], dgacc[1], dgacc[2], dgacc[3]);
-    __syncthreads();
-    if (tid < kD) {
-        float t = 0.f;
-#pragma unroll
-        for (int w = 0; w < DQ_THREADS / 32; ++w) t += sm.dgq[w][tid];
-        p.dgq_part[(size_t)blockIdx.x * kD + tid] = t;
-    }
-}
-
 // =====================================================================  d_gamma reduction
 
 // 1024 threads: 8 groups of 128 sum parts p = group (mod 8) in increasing order; the group
@@ -596,7 +635,7 @@ long long bwd_mma_n_q_parts(int B, int S, int Hq) {
 }
 
 extern const char* const kBwdMmaKernelNames[] = {"bwd_pre_kernel", "bwd_dq_kernel", "bwd_main_kernel",
-                                          "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"};
+                                                 "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"};
 extern const int kBwdMmaKernelCount = 5;
 
 namespace {

@@ -56,6 +56,7 @@ struct BwdParams {
     float* dgamma_k;    // [D]
     // workspace views
     float* delta;       // [B,Hq,S]   sum_j P_ij dP_ij (formed by the dq kernel)
+    float* lse2;        // [B,Hq,S]   base-2 log-sum-exp of the backward's own scores
     bf16* dA;           // [B,S,Hq,D] dout * sigmoid(g), rounded to bf16 ("hi")
     bf16* dA_lo;        // [B,S,Hq,D] dout * sigmoid(g) - hi, rounded to bf16
     float* dgk_part;    // [n_k_parts, D]

@@ -80,7 +80,7 @@ void fill_layer(LayerParams& L, const void* q, const void* k, const void* v, con
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct BwdWorkspace {
-    size_t delta, dA, dA_lo, dgk, dgq, total;
+    size_t delta, lse2, dA, dA_lo, dgk, dgq, total;
     int n_k_parts;
     long long n_q_parts;
 };
@@ -92,6 +92,7 @@ BwdWorkspace bwd_layout(int B, int S, int Hq, int Hkv) {
     w.n_q_parts = bwd_mma_n_q_parts(B, S, Hq);
     size_t off = 0;
     w.delta = off; off = align256(off + rows * sizeof(float));
+    w.lse2 = off;  off = align256(off + rows * sizeof(float));
     w.dA = off;    off = align256(off + rows * kD * sizeof(bf16));
     w.dA_lo = off; off = align256(off + rows * kD * sizeof(bf16));
     w.dgk = off;   off = align256(off + (size_t)w.n_k_parts * kD * sizeof(float));
@@ -204,6 +205,7 @@ int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void*
     p.dgamma_k = dgamma_k;
     char* ws = static_cast<char*>(workspace);
     p.delta = reinterpret_cast<float*>(ws + w.delta);
+    p.lse2 = reinterpret_cast<float*>(ws + w.lse2);
     p.dA = reinterpret_cast<bf16*>(ws + w.dA);
     p.dA_lo = reinterpret_cast<bf16*>(ws + w.dA_lo);
     p.dgk_part = reinterpret_cast<float*>(ws + w.dgk);

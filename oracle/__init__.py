@@ -45,23 +45,43 @@ class _Problem(ctypes.Structure):
                 ("scale", ctypes.c_double)]
 
 
+def _bind(lib):
+    P = ctypes.POINTER(_Problem)
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    lib.zo_forward.argtypes = [P, vp, i64, vp, vp]
+    lib.zo_backward_qrows.argtypes = [P, vp, vp, i64, vp, vp]
+    lib.zo_backward_krows.argtypes = [P, vp, vp, i64, vp, vp]
+    lib.zo_backward_full.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
+    lib.zo_prologue_row.argtypes = [P, vp, vp, i64, vp]
+    lib.zo_prologue_row.restype = None
+    lib.zo_num_threads.argtypes = []
+    for f in (lib.zo_forward, lib.zo_backward_qrows, lib.zo_backward_krows, lib.zo_backward_full,
+              lib.zo_num_threads):
+        f.restype = ctypes.c_int
+    return lib
+
+
+class using_library:
+    """Temporarily route every oracle call to another build of zgcm_oracle.c (the pin tests
+    use it to check that planted mistakes are caught)."""
+
+    def __init__(self, path: str):
+        self.lib = _bind(ctypes.CDLL(path))
+
+    def __enter__(self):
+        global _lib
+        self.saved, _lib = _lib, self.lib
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+
+
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
-        P = ctypes.POINTER(_Problem)
-        vp, i64 = ctypes.c_void_p, ctypes.c_int64
-        lib.zo_forward.argtypes = [P, vp, i64, vp, vp]
-        lib.zo_backward_qrows.argtypes = [P, vp, vp, i64, vp, vp]
-        lib.zo_backward_krows.argtypes = [P, vp, vp, i64, vp, vp]
-        lib.zo_backward_full.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
-        lib.zo_prologue_row.argtypes = [P, vp, vp, i64, vp]
-        lib.zo_prologue_row.restype = None
-        lib.zo_num_threads.argtypes = []
-        for f in (lib.zo_forward, lib.zo_backward_qrows, lib.zo_backward_krows, lib.zo_backward_full,
-                  lib.zo_num_threads):
-            f.restype = ctypes.c_int
-        _lib = lib
+        _lib = _bind(ctypes.CDLL(build()))
     return _lib
 
 

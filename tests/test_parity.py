@@ -126,6 +126,23 @@ def test_gate_limits_and_nan():
     assert np.all(o[0, :, 1, :] == 0.0)
 
 
+def test_timed_backward_matches_untimed():
+    """zgcm_attn_bwd_timed (events around each kernel) does the same work."""
+    t = make_inputs(1, 640, seed=9, with_dout=True)
+    d = _to_dev(t)
+    out, lse = _gpu_fwd(d)
+    names = ga.zgcm_attn_bwd_kernel_names(640, 128)
+    assert len(names) >= 3
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in names]
+    g1 = _gpu_bwd(d, out, lse)
+    g2 = ga.zgcm_attn_bwd(d["q"], d["k"], d["v"], d["g"], d["gamma_q"], d["gamma_k"], out, lse, d["dout"],
+                          kernel_events=ev)
+    torch.cuda.synchronize()
+    for n in ("dq", "dk", "dv", "dg", "dgamma_q", "dgamma_k"):
+        assert torch.equal(g1[n], g2[n]), n
+    assert all(a.elapsed_time(b) >= 0.0 for a, b in ev)
+
+
 def test_forward_bitwise_repeatable():
     t = make_inputs(2, 2048, seed=5)
     d = _to_dev(t)
@@ -162,10 +179,13 @@ def _sampled_fwd_bwd(B, S, W, n_random, k_rows, check_bwd=True, seed=0, edge=256
     rhs = dA.view(B, S, -1, G, 128).sum(dim=(1, 3))
     lhs = gr["dv"].double().sum(dim=1)
     assert_bf16_close("sum_j dv", lhs, rhs, atol=2e-2 * float(rhs.abs().max()) + 2e-2)
-    # gamma_q . dgamma_q = gamma_k . dgamma_k (scores are invariant to q_hat*c, k_hat/c)
+    # gamma_q . dgamma_q = gamma_k . dgamma_k (scores are invariant to q_hat*c, k_hat/c).
+    # Each side sums B*S*H rows of gradient terms that carry the per-element error the
+    # bf16 bound allows (rel-RMS 5e-3) and largely cancel, so the two sums are compared
+    # to 2e-2 of their size.
     a = float((gr["dgamma_q"].double() * d["gamma_q"].double()).sum())
     c = float((gr["dgamma_k"].double() * d["gamma_k"].double()).sum())
-    assert abs(a - c) <= 5e-3 * max(abs(a), abs(c)) + 1e-3, (a, c)
+    assert abs(a - c) <= 2e-2 * max(abs(a), abs(c)) + 1e-3, (a, c)
 
 
 def test_swa_16k_forward_backward():
