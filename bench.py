@@ -38,6 +38,8 @@ WORKLOADS = {
     "swa256k_fwd": (1, 262144, 128, False),
     "global256k_fwd": (1, 262144, 262144, False),
     "tiny_fwd": (1, 1024, 128, False),
+    "swa16k_b1_fwd": (1, 16384, 128, False),
+    "swa16k_b1": (1, 16384, 128, True),
 }
 HQ, HKV, D = 32, 8, 128
 
