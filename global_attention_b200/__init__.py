@@ -57,6 +57,8 @@ def load() -> ctypes.CDLL:
         lib.zgcm_attn_fwd_kernel_name.restype = ctypes.c_char_p
         lib.zgcm_attn_device_error.argtypes = []
         lib.zgcm_attn_device_error.restype = i
+        lib.zgcm_attn_bwd_noalloc.argtypes = [vp] * 9 + [i] * 6 + [d, i, i, f, f] + [vp] * 7
+        lib.zgcm_attn_bwd_noalloc.restype = i
         _lib = lib
     return _lib
 
@@ -178,4 +180,29 @@ def zgcm_attn_bwd(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dims=42,
         st = load().zgcm_attn_bwd_timed(*args, arr, len(kernel_events))
     if st != ZGCM_OK:
         raise ZgcmError(st, "zgcm_attn_bwd")
+    return grads
+
+
+def zgcm_attn_bwd_noalloc(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dims=42, rope_base=10000.0,
+                          window=128, causal=1, eps=1e-6, scale=None, grads=None, stream=None):
+    """zgcm_attn_bwd without a workspace: for callers that cannot allocate device memory,
+    the library's fixed 64 MiB per-device scratch array is used instead (problems needing
+    more raise ZgcmError with ZGCM_ERR_TOO_LARGE).  Calls that overlap on the GPU race."""
+    import torch
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if grads is None:
+        grads = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+                     dg=torch.empty_like(g),
+                     dgamma_q=torch.empty(D, dtype=torch.float32, device=q.device),
+                     dgamma_k=torch.empty(D, dtype=torch.float32, device=q.device))
+    st = load().zgcm_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma_q), _ptr(gamma_k),
+                                      _ptr(out), _ptr(lse), _ptr(dout), B, S, Hq, Hkv, D, int(rope_dims),
+                                      float(rope_base), int(window), int(causal), float(eps), float(scale),
+                                      _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]), _ptr(grads["dg"]),
+                                      _ptr(grads["dgamma_q"]), _ptr(grads["dgamma_k"]), _stream(stream))
+    if st != ZGCM_OK:
+        raise ZgcmError(st, "zgcm_attn_bwd_noalloc")
     return grads

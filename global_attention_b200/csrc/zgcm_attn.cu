@@ -114,6 +114,8 @@ const char* zgcm_status_string(int status) {
         case ZGCM_ERR_WORKSPACE: return "ZGCM_ERR_WORKSPACE: workspace missing or too small";
         case ZGCM_ERR_CUDA: return "ZGCM_ERR_CUDA: CUDA runtime or launch failure";
         case ZGCM_ERR_TIMEOUT: return "ZGCM_ERR_TIMEOUT: bounded device wait expired";
+        case ZGCM_ERR_TOO_LARGE:
+            return "ZGCM_ERR_TOO_LARGE: problem needs more than the 64 MiB scratch of zgcm_attn_bwd_noalloc";
         default: return "unknown zgcm_status";
     }
 }

@@ -56,7 +56,8 @@ typedef enum {
     ZGCM_ERR_ALIGNMENT = -3,   /* a tensor pointer is not 16-byte aligned                 */
     ZGCM_ERR_WORKSPACE = -4,   /* workspace null or smaller than the size query returns  */
     ZGCM_ERR_CUDA = -5,        /* a CUDA runtime call or a kernel launch failed          */
-    ZGCM_ERR_TIMEOUT = -6      /* reserved: a bounded device-side wait gave up           */
+    ZGCM_ERR_TIMEOUT = -6,     /* a bounded device-side wait gave up                     */
+    ZGCM_ERR_TOO_LARGE = -7    /* problem needs more scratch than zgcm_attn_bwd_noalloc has */
 } zgcm_status;
 
 /* Human-readable name of a zgcm_status value (static string, never NULL). */
@@ -129,6 +130,30 @@ int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void*
                         float* dgamma_q, float* dgamma_k,
                         void* workspace, size_t workspace_bytes, void* cuda_stream,
                         void* const* events, int n_pairs);
+
+/*
+ * zgcm_attn_bwd for callers that cannot allocate device memory.  (No counterpart in the
+ * paper: this is an interface convenience of this library.)  A process that has reserved
+ * the GPU's memory for its own pool, or a plugin given no allocator, cannot provide the
+ * workspace zgcm_attn_bwd asks for, and cudaMalloc/cudaFree may synchronise the device.
+ * This variant takes the same arguments minus the workspace and uses a fixed 64 MiB
+ * scratch array that lives in the library's device image on every GPU that loads the
+ * library, until the process exits.  It allocates nothing.
+ *
+ * Limit: problems whose zgcm_attn_bwd_workspace_size exceeds 64 MiB (about 4K tokens
+ * at 32 query heads) return ZGCM_ERR_TOO_LARGE before anything runs.
+ * The first call on a device looks up the array's device address (once per device).
+ * All calls on a device share the array, which keeps the last call's contents; every
+ * scratch word is written before it is read, so nothing needs clearing.  Calls whose
+ * executions overlap on the GPU (other streams, other host threads) race on it.
+ */
+int zgcm_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* g,
+                          const float* gamma_q, const float* gamma_k,
+                          const void* out, const float* lse, const void* dout,
+                          int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                          double rope_base, int window, int causal, float eps, float scale,
+                          void* dq, void* dk, void* dv, void* dg,
+                          float* dgamma_q, float* dgamma_k, void* cuda_stream);
 
 /*
  * Kernel zgcm_attn_fwd launches for this configuration (static string): "fwd_tc_kernel"
