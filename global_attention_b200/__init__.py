@@ -51,7 +51,7 @@ def load() -> ctypes.CDLL:
         lib.zgcm_attn_bwd.restype = i
         lib.zgcm_attn_bwd_timed.argtypes = lib.zgcm_attn_bwd.argtypes + [ctypes.POINTER(vp), i]
         lib.zgcm_attn_bwd_timed.restype = i
-        lib.zgcm_attn_bwd_kernel_name.argtypes = [i, i, i]
+        lib.zgcm_attn_bwd_kernel_name.argtypes = [i, i, i, i]
         lib.zgcm_attn_bwd_kernel_name.restype = ctypes.c_char_p
         lib.zgcm_attn_fwd_kernel_name.argtypes = [i, i, i, i, i, i]
         lib.zgcm_attn_fwd_kernel_name.restype = ctypes.c_char_p
@@ -126,11 +126,11 @@ def zgcm_attn_device_error() -> int:
     return int(load().zgcm_attn_device_error())
 
 
-def zgcm_attn_bwd_kernel_names(S, window):
+def zgcm_attn_bwd_kernel_names(S, window, rope_dims=42):
     """Names of the kernels zgcm_attn_bwd launches, in order."""
     names, i = [], 0
     while True:
-        n = load().zgcm_attn_bwd_kernel_name(i, int(S), int(window))
+        n = load().zgcm_attn_bwd_kernel_name(i, int(S), int(rope_dims), int(window))
         if n is None:
             return names
         names.append(n.decode())

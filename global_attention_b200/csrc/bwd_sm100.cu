@@ -1,0 +1,1099 @@
+// bwd_sm100.cu — gated sliding-window attention backward on tcgen05 / TMEM / TMA (sm_100a).
+//
+// Exact gradients of L = sum(dout * out) for the ZGCM-1 layer (definition and page
+// citations in common.cuh), for windows W <= 128 and 42 rotated dims; other shapes run on
+// the warp-MMA kernels (bwd_mma.cu).  Two kernels:
+//
+//   bwd_q_tc   query-major sweep over (b, KV head, 128-query block) steps, all query heads
+//              of the group per step, key tiles qb-1 and qb in a 2-slot ring (as the forward).
+//              Per head: S = Q~ K~^T and dP = dA V^T (both M=128 N=256 into TMEM), then one
+//              warpgroup per row forms the log-sum-exp, Delta = sum_j P dP and dS = P(dP-Delta)
+//              from its own scores, dQ~ = dS K~ (M=128 N=128 K=256, dS from TMEM), and an
+//              epilogue warpgroup applies the RoPE / RMSNorm backward and writes dq.  The gate
+//              preprocessing is fused into its prologue: dA = dout*sigmoid(g) and
+//              dg = dout*out*(1-sigmoid(g)).  Writes lse, Delta and max|dout| per row.
+//   bwd_kv_tc  key-major: persistent CTAs over (b, KV head, 128-key tile) units; per unit the
+//              Hq/Hkv heads x the two query blocks that see the tile:
+//              S^T = K~ Q~^T, dP^T = V dA^T, P^T and dS^T from the saved lse and Delta,
+//              dV += P^T dA and dK~ += dS^T Q~ accumulated in TMEM; epilogue writes dv and dk
+//              (RoPE / RMSNorm backward).
+//
+// Numerics.  Every product runs as kind::f16 with fp16 operands (11-bit significand) and
+// fp32 accumulation; each operand is brought into fp16 range by an exact power-of-two scale
+// that the product lets factor out: q~, k~ are RMS-normalised (one scale from gamma); dA
+// and dS rows of the query-major products; V and dS^T rows of the key-major products; dA in
+// dV by one scale per unit (a sum over query rows).  Scales are undone in fp32.  Measured
+// in a CPU emulation against the fp64 oracle this keeps every gradient within the bf16
+// output rounding of the reference (single bf16 operands did not).
+#include <cudaTypedefs.h>
+
+#include "tc_rows.cuh"
+
+namespace zgcm {
+using namespace sm100;
+
+constexpr int TB_THREADS = 512;
+constexpr int TB_MAX_GRID = 1024;  // partial-sum slots reserved in the workspace
+
+struct BwdTcParams {
+    CUtensorMap tm_q;   // {D, Hq, S, B}, box {64, 1, 128, 1}, 128B swizzle
+    CUtensorMap tm_k;
+    CUtensorMap tm_v;
+    BwdParams P;
+    float* domax;       // [B,Hq,S] max |dout| of each row (bound on |dA|)
+    int* err;
+    int total;          // steps (query-major) or units (key-major)
+};
+
+// Power of two that keeps the fp16 q~, k~ in range: |y_d| <= sqrt(D) max|gamma|.  Every
+// CTA of both kernels derives the same value from gamma_q, gamma_k in shared memory.
+__device__ __forceinline__ float qk_fp16_scale(const float* gq, const float* gk) {
+    float gmax = 0.f;
+    for (int d = 0; d < kD; ++d) gmax = fmaxf(gmax, fmaxf(fabsf(gq[d]), fabsf(gk[d])));
+    const float bound = gmax * sqrtf((float)kD);
+    return (bound > 16384.f && isfinite(bound)) ? ldexpf(1.0f, 13 - ilogbf(bound)) : 1.0f;
+}
+
+// power-of-two exponent e with |x| * 2^e in [2^13, 2^14); 0 for x == 0 or non-finite
+__device__ __forceinline__ int fit_exp(float x) {
+    if (!(x > 0.f) || !isfinite(x)) return 0;
+    int e = 13 - ilogbf(x);
+    return max(-120, min(120, e));
+}
+
+// 32 lanes x 16 consecutive 32-bit columns load
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// Sum of v[e] over the 32 lanes of the warp for e = 0..31, delivered as: lane L returns the
+// total of index L (recursive halving; 31 shuffles).
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[32]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int k = 16; k >= 1; k >>= 1) {
+        const bool upper = (lane & k) != 0;
+#pragma unroll
+        for (int j = 0; j < k; ++j) {
+            const float send = upper ? v[j] : v[j + k];
+            const float keep = upper ? v[j + k] : v[j];
+            v[j] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+        }
+    }
+    return v[0];
+}
+
+// swizzled 16-byte chunk ch (0..15, 8 values each) of row r in a two-half 128-row tile
+__device__ __forceinline__ uint4* tile_chunk(unsigned char* h0, unsigned char* h1, int r, int ch) {
+    unsigned char* hb = ch < 8 ? h0 : h1;
+    return reinterpret_cast<uint4*>(hb + (uint32_t)r * 128u + (uint32_t)(((ch & 7) ^ (r & 7)) << 4));
+}
+
+// RoPE / RMSNorm backward of one row held by one thread: dq~ (fp32, 128 columns of TMEM at
+// `taddr`, times `f`) -> dx (bf16, to `dst`), adding dy * xhat of the row into this warp's
+// d_gamma slice `dgam` (warp-transposed sums: lane L owns one dimension per 32-wide block,
+// so the slice is updated in a fixed order and the result is reproducible).  `x` is the raw row
+// in global memory; `valid` masks rows past the sequence (they still join the collectives).
+__device__ __forceinline__ void row_rope_rms_backward(uint32_t taddr, float f, const bf16* x, bf16* dst,
+                                                      bool valid, int pos, const float* gamma, float* dgam,
+                                                      const LayerParams& L) {
+    const int lane = threadIdx.x & 31;
+    const uint4* xr = reinterpret_cast<const uint4*>(x);
+    float ss = 0.f;
+    if (valid) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const uint4 u = __ldg(xr + c);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 t = unpack_bf16(w[e]);
+                ss = fmaf(t.x, t.x, fmaf(t.y, t.y, ss));
+            }
+        }
+    }
+    const float rinv = ss > 0.f ? rsqrtf(ss * (1.0f / kD) + L.eps) : 0.f;
+    float mdot = 0.f;
+    // two passes: (A) mean of dy*gamma*xhat and d_gamma, (B) dx
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll 1
+        for (int blk = 0; blk < 2; ++blk) {  // dims [64 blk, 64 blk + 64)
+            float dy[64];
+            {
+                uint32_t a[32], b2[32];
+                tmem_ld32(taddr + 64 * blk, a);
+                tmem_ld32(taddr + 64 * blk + 32, b2);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    dy[e] = __uint_as_float(a[e]) * f;
+                    dy[32 + e] = __uint_as_float(b2[e]) * f;
+                }
+            }
+            if (blk == 0) {
+                // transpose of the rotation of pairs (t, t + 21)
+#pragma unroll
+                for (int t = 0; t < TF_HALF; ++t) {
+                    float c, s;
+                    rope_cs(L.theta[t], pos, c, s);
+                    const float d1 = dy[t], d2 = dy[t + TF_HALF];
+                    dy[t] = d1 * c + d2 * s;
+                    dy[t + TF_HALF] = d2 * c - d1 * s;
+                }
+            }
+            if (pass == 0) {
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float v[32];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint4 u = make_uint4(0u, 0u, 0u, 0u);
+                        if (valid) u = __ldg(xr + 8 * blk + 4 * half + c);
+                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 t = unpack_bf16(w[e]);
+                            const int d = 32 * half + 8 * c + 2 * e;
+                            const float x0 = t.x * rinv, x1 = t.y * rinv;
+                            mdot = fmaf(dy[d] * gamma[64 * blk + d], x0, mdot);
+                            mdot = fmaf(dy[d + 1] * gamma[64 * blk + d + 1], x1, mdot);
+                            v[8 * c + 2 * e] = valid ? dy[d] * x0 : 0.f;
+                            v[8 * c + 2 * e + 1] = valid ? dy[d + 1] * x1 : 0.f;
+                        }
+                    }
+                    const float tot = warp_transpose_sum(v);
+                    dgam[64 * blk + 32 * half + lane] += tot;
+                }
+            } else if (valid) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 u = __ldg(xr + 8 * blk + c);
+                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 t = unpack_bf16(w[e]);
+                        const int d = 8 * c + 2 * e;
+                        const float a0 = (dy[d] * gamma[64 * blk + d] - t.x * rinv * mdot) * rinv;
+                        const float a1 = (dy[d + 1] * gamma[64 * blk + d + 1] - t.y * rinv * mdot) * rinv;
+                        o[e] = pack_bf16(a0, a1);
+                    }
+                    reinterpret_cast<uint4*>(dst)[8 * blk + c] = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+        }
+        if (pass == 0) mdot *= (1.0f / kD);
+    }
+}
+
+// =====================================================================  query-major kernel
+
+enum QBar {
+    QB_KFULL = 0, QB_KREADY = 2, QB_KEMPTY = 4, QB_VFULL = 6, QB_VREADY = 8, QB_VEMPTY = 10,
+    QB_QFULL = 12, QB_QREADY = 13, QB_QEMPTY = 14, QB_DAEMPTY = 15,
+    QB_SFULL = 16, QB_DSFULL = 17, QB_DQFULL = 18, QB_DQEMPTY = 19, QB_DONE = 20, QB_COUNT = 21
+};
+
+struct BwdQTcSmem {
+    alignas(1024) unsigned char K[2][TF_RING_HALF];    // K~ fp16, 2-slot ring split by d-half
+    alignas(1024) unsigned char V[2][TF_RING_HALF];    // V fp16, row-scaled
+    alignas(1024) unsigned char Q[2][TF_HALF_BYTES];   // raw q -> Q~ fp16 in place
+    alignas(1024) unsigned char dA[2][TF_HALF_BYTES];  // dA fp16, row-scaled
+    float2 cs[TF_HALF][TF_BM];
+    float gq[kD], gk[kD];
+    float vinv[4][TF_BN];    // 2^-e of each V row, by tile number % 4
+    float dainv[2][TF_BM];   // 2^-e of each dA row, by head number % 2
+    float dsinv[TF_BM];      // 2^-e of each dS row of the current head
+    float dgq[4][kD];        // this CTA's d_gamma_q, one slice per epilogue warp
+    uint64_t bar[QB_COUNT];
+    uint32_t tmem_base;
+    int abort;
+};
+
+// In-place fp16 conversion of row r of a raw bf16 V tile, scaled so max|v| lands in
+// [2^13, 2^14); returns 2^-e (and the row's 2-norm in *norm if wanted).
+__device__ __forceinline__ float v_row_to_f16(unsigned char* h0, unsigned char* h1, int r, float* norm) {
+    float mx = 0.f, ss = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 16; ++ch) {
+        const uint4 u = *tile_chunk(h0, h1, r, ch);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 t = unpack_bf16(w[e]);
+            mx = fmaxf(mx, fmaxf(fabsf(t.x), fabsf(t.y)));
+            ss = fmaf(t.x, t.x, fmaf(t.y, t.y, ss));
+        }
+    }
+    const int e = fit_exp(mx);
+    const float sc = ldexpf(1.0f, e);
+#pragma unroll
+    for (int ch = 0; ch < 16; ++ch) {
+        uint4* pc = tile_chunk(h0, h1, r, ch);
+        const uint4 u = *pc;
+        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 t = unpack_bf16(w[k]);
+            w[k] = pack2<true>(t.x * sc, t.y * sc);
+        }
+        *pc = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (norm) *norm = sqrtf(ss);
+    return ldexpf(1.0f, -e);
+}
+
+__global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_constant__ BwdTcParams p) {
+    const LayerParams& L = p.P.L;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    BwdQTcSmem& sm = *reinterpret_cast<BwdQTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    volatile int* abort = &sm.abort;
+    const int G = L.G;
+    const int t_begin = (int)(((long long)blockIdx.x * p.total) / gridDim.x);
+    const int t_end = (int)(((long long)(blockIdx.x + 1) * p.total) / gridDim.x);
+
+    if (tid == 0) {
+        sm.abort = 0;
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.bar[QB_KFULL + i], 1);
+            mbar_init(&sm.bar[QB_KREADY + i], 128);
+            mbar_init(&sm.bar[QB_KEMPTY + i], 1);
+            mbar_init(&sm.bar[QB_VFULL + i], 1);
+            mbar_init(&sm.bar[QB_VREADY + i], 128);
+            mbar_init(&sm.bar[QB_VEMPTY + i], 1);
+        }
+        mbar_init(&sm.bar[QB_QFULL], 1);
+        mbar_init(&sm.bar[QB_QREADY], 128);
+        mbar_init(&sm.bar[QB_QEMPTY], 1);
+        mbar_init(&sm.bar[QB_DAEMPTY], 1);
+        mbar_init(&sm.bar[QB_SFULL], 1);
+        mbar_init(&sm.bar[QB_DSFULL], 128);
+        mbar_init(&sm.bar[QB_DQFULL], 1);
+        mbar_init(&sm.bar[QB_DQEMPTY], 128);
+        mbar_init(&sm.bar[QB_DONE], 1);
+        fence_barrier_init();
+    }
+    if (tid < kD) {
+        sm.gq[tid] = L.gamma_q[tid];
+        sm.gk[tid] = L.gamma_k[tid];
+        for (int w = 0; w < 4; ++w) sm.dgq[w][tid] = 0.f;
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&p.tm_q);
+        prefetch_tmap(&p.tm_k);
+        prefetch_tmap(&p.tm_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t TM_S = tmem, TM_DP = tmem + 256, TM_DS = tmem, TM_DQ = tmem + 128;
+    const float oscale = qk_fp16_scale(sm.gq, sm.gk);
+    const float c2 = L.scale_log2 / (oscale * oscale);
+
+    if (warp == 0) {
+        // ================================================ K / V producer
+        if (lane == 0) {
+            int n_next = 0;
+            int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
+            auto load_tile = [&](int n, int b, int kvh, int kt) -> bool {
+                const int slot = n & 1;
+                if (n >= 2 && !mbar_wait(&sm.bar[QB_KEMPTY + slot], ((n >> 1) - 1) & 1, abort, 101)) return false;
+                mbar_expect_tx(&sm.bar[QB_KFULL + slot], TF_TILE_BYTES);
+                tma_load_4d(sm.K[0] + slot * TF_HALF_BYTES, &p.tm_k, &sm.bar[QB_KFULL + slot], 0, kvh, kt * TF_BN, b);
+                tma_load_4d(sm.K[1] + slot * TF_HALF_BYTES, &p.tm_k, &sm.bar[QB_KFULL + slot], 64, kvh, kt * TF_BN, b);
+                last_k[slot] = n;
+                if (n >= 2 && !mbar_wait(&sm.bar[QB_VEMPTY + slot], ((n >> 1) - 1) & 1, abort, 102)) return false;
+                mbar_expect_tx(&sm.bar[QB_VFULL + slot], TF_TILE_BYTES);
+                tma_load_4d(sm.V[0] + slot * TF_HALF_BYTES, &p.tm_v, &sm.bar[QB_VFULL + slot], 0, kvh, kt * TF_BN, b);
+                tma_load_4d(sm.V[1] + slot * TF_HALF_BYTES, &p.tm_v, &sm.bar[QB_VFULL + slot], 64, kvh, kt * TF_BN, b);
+                last_v[slot] = n;
+                return true;
+            };
+            for (int t = t_begin; t < t_end && !*abort; ++t) {
+                const StepInfo st = decode_step(L, t, t_begin, t_end);
+                if (st.fresh && !load_tile(n_next++, st.b, st.kvh, st.qb - 1)) break;
+                if (!load_tile(n_next++, st.b, st.kvh, st.qb)) break;
+            }
+            for (int slot = 0; slot < 2; ++slot) {
+                if (last_k[slot] >= 0) mbar_wait_drain(&sm.bar[QB_KFULL + slot], (last_k[slot] >> 1) & 1);
+                if (last_v[slot] >= 0) mbar_wait_drain(&sm.bar[QB_VFULL + slot], (last_v[slot] >> 1) & 1);
+            }
+        }
+    } else if (warp == 2) {
+        // ================================================ Q producer (single buffer)
+        if (lane == 0) {
+            int m = 0, last = -1;
+            for (int t = t_begin; t < t_end && !*abort; ++t) {
+                const StepInfo st = decode_step(L, t, t_begin, t_end);
+                for (int h = 0; h < G; ++h, ++m) {
+                    if (m >= 1 && !mbar_wait(&sm.bar[QB_QEMPTY], (m - 1) & 1, abort, 103)) break;
+                    mbar_expect_tx(&sm.bar[QB_QFULL], TF_TILE_BYTES);
+                    const int hg = st.kvh * G + h;
+                    tma_load_4d(sm.Q[0], &p.tm_q, &sm.bar[QB_QFULL], 0, hg, st.qb * TF_BM, st.b);
+                    tma_load_4d(sm.Q[1], &p.tm_q, &sm.bar[QB_QFULL], 64, hg, st.qb * TF_BM, st.b);
+                    last = m;
+                }
+            }
+            if (last >= 0) mbar_wait_drain(&sm.bar[QB_QFULL], last & 1);
+        }
+    } else if (warp == 1) {
+        // ================================================ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_N256 = idesc_f16(128, 256, false);
+            constexpr uint32_t IDESC_DQ = idesc_f16(128, 128, true);
+            const uint32_t q_base = smem_u32(sm.Q[0]), da_base = smem_u32(sm.dA[0]);
+            const uint32_t k_base = smem_u32(sm.K[0]), v_base = smem_u32(sm.V[0]);
+            int n_next = 0, n_prev = 0, n_cur = 0, m = 0;
+            bool ok = true;
+            for (int t = t_begin; t < t_end && ok; ++t) {
+                const StepInfo st = decode_step(L, t, t_begin, t_end);
+                if (st.fresh) {
+                    n_prev = n_next++;
+                    n_cur = n_next++;
+                    ok = mbar_wait(&sm.bar[QB_KREADY + (n_prev & 1)], (n_prev >> 1) & 1, abort, 110) &&
+                         mbar_wait(&sm.bar[QB_VREADY + (n_prev & 1)], (n_prev >> 1) & 1, abort, 111);
+                } else {
+                    n_prev = n_cur;
+                    n_cur = n_next++;
+                }
+                ok = ok && mbar_wait(&sm.bar[QB_KREADY + (n_cur & 1)], (n_cur >> 1) & 1, abort, 112) &&
+                     mbar_wait(&sm.bar[QB_VREADY + (n_cur & 1)], (n_cur >> 1) & 1, abort, 113);
+                for (int h = 0; h < G && ok; ++h, ++m) {
+                    if (!(ok = mbar_wait(&sm.bar[QB_QREADY], m & 1, abort, 114))) break;
+                    if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_DQEMPTY], (m - 1) & 1, abort, 115))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t half = kk >> 2, within = (kk & 3) * 32;
+                        const uint64_t aq = sdesc_sw128(q_base + half * TF_HALF_BYTES + within, 16, 1024);
+                        const uint64_t bk = sdesc_sw128(k_base + half * TF_RING_HALF + within, 16, 1024);
+                        mma_ss(TM_S, aq, bk, IDESC_N256, kk > 0 ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t half = kk >> 2, within = (kk & 3) * 32;
+                        const uint64_t ad = sdesc_sw128(da_base + half * TF_HALF_BYTES + within, 16, 1024);
+                        const uint64_t bv = sdesc_sw128(v_base + half * TF_RING_HALF + within, 16, 1024);
+                        mma_ss(TM_DP, ad, bv, IDESC_N256, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&sm.bar[QB_QEMPTY]);
+                    mma_commit(&sm.bar[QB_DAEMPTY]);
+                    mma_commit(&sm.bar[QB_SFULL]);
+                    if (h == G - 1) {
+                        mma_commit(&sm.bar[QB_VEMPTY + (n_prev & 1)]);
+                        if (st.release_cur) mma_commit(&sm.bar[QB_VEMPTY + (n_cur & 1)]);
+                    }
+                    if (!(ok = mbar_wait(&sm.bar[QB_DSFULL], m & 1, abort, 116))) break;
+                    tc_fence_after();
+                    // dQ~ = dS K~ : dS fp16 in TMEM (16 keys = 8 columns per step), K~ MN-major
+#pragma unroll
+                    for (int kk = 0; kk < 16; ++kk) {
+                        const uint64_t bk = sdesc_sw128(k_base + kk * 16 * 128, TF_RING_HALF, 1024);
+                        mma_ts(TM_DQ, TM_DS + kk * 8, bk, IDESC_DQ, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&sm.bar[QB_DQFULL]);
+                    if (h == G - 1) {
+                        mma_commit(&sm.bar[QB_KEMPTY + (n_prev & 1)]);
+                        if (st.release_cur) mma_commit(&sm.bar[QB_KEMPTY + (n_cur & 1)]);
+                    }
+                }
+            }
+            mma_commit(&sm.bar[QB_DONE]);
+            mbar_wait(&sm.bar[QB_DONE], 0, abort, 117);
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ================================================ lse, Delta, dS (thread = query row)
+        const int r = tid - 128, wq = warp - 4;
+        const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+        int n_next = 0, n_prev = 0, n_cur = 0, m = 0;
+        for (int t = t_begin; t < t_end; ++t) {
+            const StepInfo st = decode_step(L, t, t_begin, t_end);
+            if (st.fresh) { n_prev = n_next++; n_cur = n_next++; } else { n_prev = n_cur; n_cur = n_next++; }
+            const int q0 = st.qb * TF_BM, i = q0 + r;
+            const int slot_cur = n_cur & 1;
+            const int base0 = (slot_cur == 0 ? q0 : q0 - TF_BN), base1 = (slot_cur == 1 ? q0 : q0 - TF_BN);
+            const float* vin0 = sm.vinv[((slot_cur == 0) ? n_cur : n_prev) & 3];
+            const float* vin1 = sm.vinv[((slot_cur == 1) ? n_cur : n_prev) & 3];
+            const int imin = q0 + 32 * wq, imax = imin + 31;
+            bool stop = false;
+            for (int h = 0; h < G; ++h, ++m) {
+                if (!mbar_wait(&sm.bar[QB_SFULL], m & 1, abort, 120)) { stop = true; break; }
+                tc_fence_after();
+                const float dai = sm.dainv[m & 1][r];
+                float mx = -INFINITY;
+#pragma unroll 1
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const int kp0 = (c8 < 4 ? base0 : base1) + (c8 & 3) * 32;
+                    const bool live = imin < L.S && kp0 <= imax && kp0 + 31 > imin - L.W && kp0 + 31 >= 0 && kp0 < L.S;
+                    if (!live) continue;
+                    uint32_t v[32];
+                    tmem_ld32(TM_S + lane_off + 32 * c8, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = kp0 + e;
+                        if (j <= i && j > i - L.W && j >= 0 && j < L.S) mx = fmaxf(mx, __uint_as_float(v[e]));
+                    }
+                }
+                const float mu = (mx == -INFINITY) ? 0.f : mx * c2;
+                float l = 0.f, num = 0.f, mxdp = 0.f;
+#pragma unroll 1
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const int kp0 = (c8 < 4 ? base0 : base1) + (c8 & 3) * 32;
+                    const bool live = imin < L.S && kp0 <= imax && kp0 + 31 > imin - L.W && kp0 + 31 >= 0 && kp0 < L.S;
+                    if (!live) continue;
+                    const float* vin = (c8 < 4 ? vin0 : vin1) + (c8 & 3) * 32;
+                    uint32_t sv[32], dv[32];
+                    tmem_ld32(TM_S + lane_off + 32 * c8, sv);
+                    tmem_ld32(TM_DP + lane_off + 32 * c8, dv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = kp0 + e;
+                        if (j <= i && j > i - L.W && j >= 0 && j < L.S) {
+                            const float ev = fast_exp2(__uint_as_float(sv[e]) * c2 - mu);
+                            const float dp = __uint_as_float(dv[e]) * dai * vin[e];
+                            l += ev;
+                            num = fmaf(ev, dp, num);
+                            mxdp = fmaxf(mxdp, fabsf(dp));
+                        }
+                    }
+                }
+                const float lse2 = l > 0.f ? mu + log2f(l) : INFINITY;
+                const float delta = l > 0.f ? num / l : 0.f;
+                const int es = fit_exp(mxdp + fabsf(delta));
+                const float dsc = ldexpf(1.0f, es);
+#pragma unroll 1
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const int kp0 = (c8 < 4 ? base0 : base1) + (c8 & 3) * 32;
+                    const bool live = imin < L.S && kp0 <= imax && kp0 + 31 > imin - L.W && kp0 + 31 >= 0 && kp0 < L.S;
+                    uint32_t pk[16];
+                    if (live) {
+                        const float* vin = (c8 < 4 ? vin0 : vin1) + (c8 & 3) * 32;
+                        uint32_t sv[32], dv[32];
+                        tmem_ld32(TM_S + lane_off + 32 * c8, sv);
+                        tmem_ld32(TM_DP + lane_off + 32 * c8, dv);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            float ds2[2];
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const int j = kp0 + e + u;
+                                const bool vis = j <= i && j > i - L.W && j >= 0 && j < L.S;
+                                const float pv = vis ? fast_exp2(__uint_as_float(sv[e + u]) * c2 - lse2) : 0.f;
+                                const float dp = __uint_as_float(dv[e + u]) * dai * vin[e + u];
+                                ds2[u] = pv * (dp - delta) * dsc;
+                            }
+                            pk[e >> 1] = pack2<true>(ds2[0], ds2[1]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    }
+                    tmem_st16(TM_DS + lane_off + 16 * c8, pk);
+                }
+                tmem_wait_st();
+                const int hg = st.kvh * G + h;
+                if (i < L.S) {
+                    const size_t ro = ((size_t)st.b * L.Hq + hg) * L.S + i;
+                    p.P.lse2[ro] = lse2;
+                    p.P.delta[ro] = delta;
+                }
+                sm.dsinv[r] = 1.0f / dsc;
+                tc_fence_before();
+                mbar_arrive(&sm.bar[QB_DSFULL]);
+            }
+            if (stop) break;
+        }
+    } else if (warp >= 8 && warp < 12) {
+        // ================================================ prologue: K~, V, Q~ (fp16, in place), dA, dg
+        const int r = tid - 256;
+        int n_next = 0, m = 0;
+        bool ok = true;
+        auto prologue_kv = [&](int n, int pos0) -> bool {
+            const int slot = n & 1;
+            if (!mbar_wait(&sm.bar[QB_KFULL + slot], (n >> 1) & 1, abort, 130)) return false;
+            tf_angles(L, pos0 + r, sm.cs, r);
+            tf_prologue_row<true>(sm.K[0] + slot * TF_HALF_BYTES, sm.K[1] + slot * TF_HALF_BYTES, r, sm.gk, L,
+                                  sm.cs, oscale);
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.bar[QB_KREADY + slot]);
+            if (!mbar_wait(&sm.bar[QB_VFULL + slot], (n >> 1) & 1, abort, 131)) return false;
+            sm.vinv[n & 3][r] = v_row_to_f16(sm.V[0] + slot * TF_HALF_BYTES, sm.V[1] + slot * TF_HALF_BYTES, r, nullptr);
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.bar[QB_VREADY + slot]);
+            return true;
+        };
+        for (int t = t_begin; t < t_end && ok; ++t) {
+            const StepInfo st = decode_step(L, t, t_begin, t_end);
+            const int q0 = st.qb * TF_BM, i = q0 + r;
+            const bool valid = i < L.S;
+            if (st.fresh) ok = prologue_kv(n_next++, q0 - TF_BN);
+            ok = ok && prologue_kv(n_next++, q0);
+            if (!ok) break;
+            for (int h = 0; h < G; ++h, ++m) {
+                if (!(ok = mbar_wait(&sm.bar[QB_QFULL], m & 1, abort, 132))) break;
+                tf_prologue_row<true>(sm.Q[0], sm.Q[1], r, sm.gq, L, sm.cs, oscale);
+                if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_DAEMPTY], (m - 1) & 1, abort, 133))) break;
+                // dA = dout * sigmoid(g) (row-scaled fp16), dg = dout * out * (1 - sigmoid(g))
+                const int hg = st.kvh * G + h;
+                const size_t off = ((size_t)(st.b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hg) * kD;
+                const uint4* dor = reinterpret_cast<const uint4*>(p.P.dout + off);
+                const uint4* gr = reinterpret_cast<const uint4*>(L.g + off);
+                const uint4* outr = reinterpret_cast<const uint4*>(p.P.out + off);
+                float mx = 0.f;
+                if (valid) {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const uint4 u = __ldg(dor + c);
+                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 t2 = unpack_bf16(w[e]);
+                            mx = fmaxf(mx, fmaxf(fabsf(t2.x), fabsf(t2.y)));
+                        }
+                    }
+                }
+                const int ea = fit_exp(mx);
+                const float sc = ldexpf(1.0f, ea);
+#pragma unroll 2
+                for (int c = 0; c < 16; ++c) {
+                    uint32_t da[4] = {0u, 0u, 0u, 0u};
+                    if (valid) {
+                        const uint4 ud = __ldg(dor + c), ug = __ldg(gr + c), uo = __ldg(outr + c);
+                        const uint32_t wd[4] = {ud.x, ud.y, ud.z, ud.w}, wg[4] = {ug.x, ug.y, ug.z, ug.w},
+                                       wo[4] = {uo.x, uo.y, uo.z, uo.w};
+                        uint32_t dgw[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 fd = unpack_bf16(wd[e]), fg = unpack_bf16(wg[e]), fo = unpack_bf16(wo[e]);
+                            const float s0 = sigmoidf_(fg.x), s1 = sigmoidf_(fg.y);
+                            da[e] = pack2<true>(fd.x * s0 * sc, fd.y * s1 * sc);
+                            dgw[e] = pack_bf16(fd.x * fo.x * (1.f - s0), fd.y * fo.y * (1.f - s1));
+                        }
+                        reinterpret_cast<uint4*>(p.P.dg + off)[c] = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
+                    }
+                    *tile_chunk(sm.dA[0], sm.dA[1], r, c) = make_uint4(da[0], da[1], da[2], da[3]);
+                }
+                if (valid) p.domax[((size_t)st.b * L.Hq + hg) * L.S + i] = mx;
+                sm.dainv[m & 1][r] = 1.0f / sc;
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.bar[QB_QREADY]);
+            }
+        }
+    } else if (warp >= 12) {
+        // ================================================ dq epilogue (thread = query row)
+        const int r = tid - 384, wq = warp - 12;
+        const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+        int m = 0;
+        bool ok = true;
+        for (int t = t_begin; t < t_end && ok; ++t) {
+            const StepInfo st = decode_step(L, t, t_begin, t_end);
+            const int i = st.qb * TF_BM + r;
+            const bool valid = i < L.S;
+            for (int h = 0; h < G; ++h, ++m) {
+                if (!(ok = mbar_wait(&sm.bar[QB_DQFULL], m & 1, abort, 140))) break;
+                tc_fence_after();
+                const float f = L.scale * sm.dsinv[r] / oscale;
+                const int hg = st.kvh * G + h;
+                const size_t off = ((size_t)(st.b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hg) * kD;
+                row_rope_rms_backward(TM_DQ + lane_off, f, L.q + off, p.P.dq + off, valid, i, sm.gq, sm.dgq[wq], L);
+                tc_fence_before();
+                mbar_arrive(&sm.bar[QB_DQEMPTY]);
+            }
+        }
+    }
+
+    // ------------------------------------------------ teardown
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+    if (tid < kD)
+        p.P.dgq_part[(size_t)blockIdx.x * kD + tid] = (sm.dgq[0][tid] + sm.dgq[1][tid]) + (sm.dgq[2][tid] + sm.dgq[3][tid]);
+    if (tid == 0 && sm.abort && p.err) atomicExch(p.err, sm.abort);
+}
+
+// =====================================================================  key-major kernel
+
+enum KBar {
+    KB_KVFULL = 0, KB_KVREADY = 1, KB_KVEMPTY = 2,
+    KB_QFULL = 3, KB_QREADY = 5, KB_QEMPTY = 7,
+    KB_SFULL = 9, KB_PFULL = 10, KB_DVKFULL = 11, KB_DVKEMPTY = 12, KB_DONE = 13, KB_COUNT = 14
+};
+
+struct BwdKTcSmem {
+    alignas(1024) unsigned char K[2][TF_HALF_BYTES];      // K~ fp16 of the unit's key tile
+    alignas(1024) unsigned char V[2][TF_HALF_BYTES];      // V fp16, row-scaled
+    alignas(1024) unsigned char Q[2][2][TF_HALF_BYTES];   // [buffer][half] raw q -> Q~ fp16
+    alignas(1024) unsigned char dA[2][2][TF_HALF_BYTES];  // [buffer][half] dA fp16, unit scale
+    float2 cs[TF_HALF][TF_BM];
+    float gq[kD], gk[kD];
+    float lse2[2][TF_BM];    // per query column of the buffer
+    float delta[2][TF_BM];
+    float vinv[TF_BN];       // 2^-e of each V row of the current unit
+    float dsc[2][TF_BN];     // 2^e of each dS^T row, by unit parity
+    float dainv[2];          // 2^-E of dA, by unit parity
+    float red[2][4];         // per-warp maxima for the unit statistics
+    float dgk[4][kD];        // this CTA's d_gamma_k, one slice per epilogue warp
+    uint64_t bar[KB_COUNT];
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct UnitInfo {
+    int b, kvh, kt, nit;   // nit = iterations: heads x query blocks that see the key tile
+};
+__device__ __forceinline__ UnitInfo decode_unit(const LayerParams& L, int u) {
+    const int nkb = (L.S + TF_BN - 1) / TF_BN;
+    UnitInfo x;
+    const int chain = u / nkb;
+    x.kt = u - chain * nkb;
+    x.b = chain / L.Hkv;
+    x.kvh = chain - x.b * L.Hkv;
+    x.nit = L.G * ((x.kt + 1 < nkb) ? 2 : 1);
+    return x;
+}
+// iteration it of a unit: query block kt + it / G, head it % G
+__device__ __forceinline__ void decode_iter(const LayerParams& L, const UnitInfo& x, int it, int& qb, int& hg) {
+    qb = x.kt + it / L.G;
+    hg = x.kvh * L.G + it % L.G;
+}
+
+__global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_constant__ BwdTcParams p) {
+    const LayerParams& L = p.P.L;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    BwdKTcSmem& sm = *reinterpret_cast<BwdKTcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    volatile int* abort = &sm.abort;
+    const int u_begin = (int)(((long long)blockIdx.x * p.total) / gridDim.x);
+    const int u_end = (int)(((long long)(blockIdx.x + 1) * p.total) / gridDim.x);
+
+    if (tid == 0) {
+        sm.abort = 0;
+        mbar_init(&sm.bar[KB_KVFULL], 1);
+        mbar_init(&sm.bar[KB_KVREADY], 128);
+        mbar_init(&sm.bar[KB_KVEMPTY], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.bar[KB_QFULL + i], 1);
+            mbar_init(&sm.bar[KB_QREADY + i], 128);
+            mbar_init(&sm.bar[KB_QEMPTY + i], 1);
+        }
+        mbar_init(&sm.bar[KB_SFULL], 1);
+        mbar_init(&sm.bar[KB_PFULL], 128);
+        mbar_init(&sm.bar[KB_DVKFULL], 1);
+        mbar_init(&sm.bar[KB_DVKEMPTY], 128);
+        mbar_init(&sm.bar[KB_DONE], 1);
+        fence_barrier_init();
+    }
+    if (tid < kD) {
+        sm.gq[tid] = L.gamma_q[tid];
+        sm.gk[tid] = L.gamma_k[tid];
+        for (int w = 0; w < 4; ++w) sm.dgk[w][tid] = 0.f;
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&p.tm_q);
+        prefetch_tmap(&p.tm_k);
+        prefetch_tmap(&p.tm_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t TM_S = tmem, TM_DP = tmem + 128, TM_P = tmem, TM_DS = tmem + 128, TM_DV = tmem + 256,
+                   TM_DK = tmem + 384;
+    const float oscale = qk_fp16_scale(sm.gq, sm.gk);
+    const float c2 = L.scale_log2 / (oscale * oscale);
+
+    if (warp == 0) {
+        // ================================================ TMA producer: K, V per unit; Q per iteration
+        if (lane == 0) {
+            int it_all = 0, last_q[2] = {-1, -1}, uu = 0;
+            for (int u = u_begin; u < u_end && !*abort; ++u, ++uu) {
+                const UnitInfo x = decode_unit(L, u);
+                if (uu >= 1 && !mbar_wait(&sm.bar[KB_KVEMPTY], (uu - 1) & 1, abort, 201)) break;
+                mbar_expect_tx(&sm.bar[KB_KVFULL], 2 * TF_TILE_BYTES);
+                tma_load_4d(sm.K[0], &p.tm_k, &sm.bar[KB_KVFULL], 0, x.kvh, x.kt * TF_BN, x.b);
+                tma_load_4d(sm.K[1], &p.tm_k, &sm.bar[KB_KVFULL], 64, x.kvh, x.kt * TF_BN, x.b);
+                tma_load_4d(sm.V[0], &p.tm_v, &sm.bar[KB_KVFULL], 0, x.kvh, x.kt * TF_BN, x.b);
+                tma_load_4d(sm.V[1], &p.tm_v, &sm.bar[KB_KVFULL], 64, x.kvh, x.kt * TF_BN, x.b);
+                bool ok = true;
+                for (int it = 0; it < x.nit; ++it, ++it_all) {
+                    const int buf = it_all & 1;
+                    if (it_all >= 2 && !(ok = mbar_wait(&sm.bar[KB_QEMPTY + buf], ((it_all >> 1) - 1) & 1, abort, 202))) break;
+                    int qb, hg;
+                    decode_iter(L, x, it, qb, hg);
+                    mbar_expect_tx(&sm.bar[KB_QFULL + buf], TF_TILE_BYTES);
+                    tma_load_4d(sm.Q[buf][0], &p.tm_q, &sm.bar[KB_QFULL + buf], 0, hg, qb * TF_BM, x.b);
+                    tma_load_4d(sm.Q[buf][1], &p.tm_q, &sm.bar[KB_QFULL + buf], 64, hg, qb * TF_BM, x.b);
+                    last_q[buf] = it_all;
+                }
+                if (!ok) break;
+            }
+            if (uu >= 1) mbar_wait_drain(&sm.bar[KB_KVFULL], (uu - 1) & 1);
+            for (int buf = 0; buf < 2; ++buf)
+                if (last_q[buf] >= 0) mbar_wait_drain(&sm.bar[KB_QFULL + buf], (last_q[buf] >> 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ================================================ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_KM = idesc_f16(128, 128, false);
+            constexpr uint32_t IDESC_MN = idesc_f16(128, 128, true);
+            const uint32_t k_base = smem_u32(sm.K[0]), v_base = smem_u32(sm.V[0]);
+            const uint32_t q_base = smem_u32(sm.Q[0][0]), da_base = smem_u32(sm.dA[0][0]);
+            int it_all = 0, uu = 0;
+            bool ok = true;
+            for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
+                const UnitInfo x = decode_unit(L, u);
+                if (!(ok = mbar_wait(&sm.bar[KB_KVREADY], uu & 1, abort, 210))) break;
+                for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
+                    const int buf = it_all & 1;
+                    const uint32_t qb_addr = q_base + buf * 2 * TF_HALF_BYTES, da_addr = da_base + buf * 2 * TF_HALF_BYTES;
+                    if (!(ok = mbar_wait(&sm.bar[KB_QREADY + buf], (it_all >> 1) & 1, abort, 211))) break;
+                    tc_fence_after();
+                    // S^T = K~ Q~^T, dP^T = V dA^T   (M = keys, N = queries, K = d)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t half = kk >> 2, within = (kk & 3) * 32;
+                        mma_ss(TM_S, sdesc_sw128(k_base + half * TF_HALF_BYTES + within, 16, 1024),
+                               sdesc_sw128(qb_addr + half * TF_HALF_BYTES + within, 16, 1024), IDESC_KM, kk > 0 ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t half = kk >> 2, within = (kk & 3) * 32;
+                        mma_ss(TM_DP, sdesc_sw128(v_base + half * TF_HALF_BYTES + within, 16, 1024),
+                               sdesc_sw128(da_addr + half * TF_HALF_BYTES + within, 16, 1024), IDESC_KM, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&sm.bar[KB_SFULL]);
+                    if (!(ok = mbar_wait(&sm.bar[KB_PFULL], it_all & 1, abort, 212))) break;
+                    if (it == 0 && uu >= 1 && !(ok = mbar_wait(&sm.bar[KB_DVKEMPTY], (uu - 1) & 1, abort, 213))) break;
+                    tc_fence_after();
+                    // dV += P^T dA ; dK~ += dS^T Q~  (A from TMEM: 16 queries = 8 columns per step;
+                    // B = dA / Q~ MN-major: N = d, K = queries)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t bda = sdesc_sw128(da_addr + kk * 16 * 128, TF_HALF_BYTES, 1024);
+                        mma_ts(TM_DV, TM_P + kk * 8, bda, IDESC_MN, (it > 0 || kk > 0) ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t bq = sdesc_sw128(qb_addr + kk * 16 * 128, TF_HALF_BYTES, 1024);
+                        mma_ts(TM_DK, TM_DS + kk * 8, bq, IDESC_MN, (it > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&sm.bar[KB_QEMPTY + buf]);
+                }
+                if (!ok) break;
+                mma_commit(&sm.bar[KB_DVKFULL]);
+                mma_commit(&sm.bar[KB_KVEMPTY]);
+            }
+            mma_commit(&sm.bar[KB_DONE]);
+            mbar_wait(&sm.bar[KB_DONE], 0, abort, 214);
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ================================================ P^T, dS^T (thread = key row)
+        const int r = tid - 128, wq = warp - 4;
+        const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+        int it_all = 0, uu = 0;
+        bool ok = true;
+        for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
+            const UnitInfo x = decode_unit(L, u);
+            const int j = x.kt * TF_BN + r;
+            if (!(ok = mbar_wait(&sm.bar[KB_KVREADY], uu & 1, abort, 220))) break;
+            const float vin = sm.vinv[r] * sm.dainv[uu & 1];  // undoes the V-row and dA scales of dP^T
+            const float dsc = sm.dsc[uu & 1][r];
+            for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
+                const int buf = it_all & 1;
+                int qb, hg;
+                decode_iter(L, x, it, qb, hg);
+                const int q0 = qb * TF_BM;
+                if (!(ok = mbar_wait(&sm.bar[KB_QREADY + buf], (it_all >> 1) & 1, abort, 221))) break;
+                if (!(ok = mbar_wait(&sm.bar[KB_SFULL], it_all & 1, abort, 222))) break;
+                tc_fence_after();
+                const int jmin = x.kt * TF_BN + 32 * wq, jmax = jmin + 31;
+#pragma unroll 1
+                for (int c8 = 0; c8 < 4; ++c8) {
+                    const int i0 = q0 + 32 * c8;  // queries of this chunk: i0 .. i0+31
+                    const bool live = jmin < L.S && i0 < L.S && i0 + 31 >= jmin && i0 <= jmax + L.W - 1;
+                    uint32_t pp[16], dd[16];
+                    if (live) {
+                        uint32_t sv[32], dv[32];
+                        tmem_ld32(TM_S + lane_off + 32 * c8, sv);
+                        tmem_ld32(TM_DP + lane_off + 32 * c8, dv);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            float pv2[2], ds2[2];
+#pragma unroll
+                            for (int w2 = 0; w2 < 2; ++w2) {
+                                const int ql = 32 * c8 + e + w2, i = q0 + ql;
+                                const bool vis = j <= i && j > i - L.W && i < L.S && j < L.S;
+                                const float pv = vis ? fast_exp2(__uint_as_float(sv[e + w2]) * c2 - sm.lse2[buf][ql]) : 0.f;
+                                const float dp = __uint_as_float(dv[e + w2]) * vin;
+                                pv2[w2] = pv;
+                                ds2[w2] = pv * (dp - sm.delta[buf][ql]) * dsc;
+                            }
+                            pp[e >> 1] = pack2<true>(pv2[0], pv2[1]);
+                            dd[e >> 1] = pack2<true>(ds2[0], ds2[1]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pp[e] = dd[e] = 0u;
+                    }
+                    tmem_st16(TM_P + lane_off + 16 * c8, pp);
+                    tmem_st16(TM_DS + lane_off + 16 * c8, dd);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&sm.bar[KB_PFULL]);
+            }
+        }
+    } else if (warp >= 8 && warp < 12) {
+        // ================================================ prologue: K~, V (per unit), Q~ and dA (per iteration)
+        const int r = tid - 256, wq = warp - 8;
+        int it_all = 0, uu = 0;
+        bool ok = true;
+        for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
+            const UnitInfo x = decode_unit(L, u);
+            if (!(ok = mbar_wait(&sm.bar[KB_KVFULL], uu & 1, abort, 230))) break;
+            // unit statistics: max |dout| and max |Delta| over the rows this unit reads
+            float domx = 0.f, dlmx = 0.f;
+            for (int it = 0; it < x.nit; ++it) {
+                int qb, hg;
+                decode_iter(L, x, it, qb, hg);
+                const int i = qb * TF_BM + r;
+                if (i < L.S) {
+                    const size_t ro = ((size_t)x.b * L.Hq + hg) * L.S + i;
+                    domx = fmaxf(domx, p.domax[ro]);
+                    dlmx = fmaxf(dlmx, fabsf(p.P.delta[ro]));
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                domx = fmaxf(domx, __shfl_xor_sync(0xffffffffu, domx, o));
+                dlmx = fmaxf(dlmx, __shfl_xor_sync(0xffffffffu, dlmx, o));
+            }
+            if (lane == 0) {
+                sm.red[0][wq] = domx;
+                sm.red[1][wq] = dlmx;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            domx = fmaxf(fmaxf(sm.red[0][0], sm.red[0][1]), fmaxf(sm.red[0][2], sm.red[0][3]));
+            dlmx = fmaxf(fmaxf(sm.red[1][0], sm.red[1][1]), fmaxf(sm.red[1][2], sm.red[1][3]));
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            const int E = fit_exp(domx);
+            const float dsc_a = ldexpf(1.0f, E);
+            // K~ (fp16) and V (fp16, row-scaled) of the unit's key tile
+            tf_angles(L, x.kt * TF_BN + r, sm.cs, r);
+            tf_prologue_row<true>(sm.K[0], sm.K[1], r, sm.gk, L, sm.cs, oscale);
+            float vnorm = 0.f;
+            sm.vinv[r] = v_row_to_f16(sm.V[0], sm.V[1], r, &vnorm);
+            // dS^T row scale: |dS_ji| <= |v_j| |dA_i| + |Delta_i| <= |v_j| sqrt(D) max|dout| + max|Delta|
+            sm.dsc[uu & 1][r] = ldexpf(1.0f, fit_exp(vnorm * sqrtf((float)kD) * domx + dlmx));
+            if (r == 0) sm.dainv[uu & 1] = 1.0f / dsc_a;
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.bar[KB_KVREADY]);
+            int cur_qb = -1;
+            for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
+                const int buf = it_all & 1;
+                int qb, hg;
+                decode_iter(L, x, it, qb, hg);
+                const int i = qb * TF_BM + r;
+                const bool valid = i < L.S;
+                if (!(ok = mbar_wait(&sm.bar[KB_QFULL + buf], (it_all >> 1) & 1, abort, 231))) break;
+                if (qb != cur_qb) {
+                    tf_angles(L, i, sm.cs, r);
+                    cur_qb = qb;
+                }
+                tf_prologue_row<true>(sm.Q[buf][0], sm.Q[buf][1], r, sm.gq, L, sm.cs, oscale);
+                // dA row (unit-uniform scale) for query row i of head hg
+                const size_t off = ((size_t)(x.b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hg) * kD;
+                const uint4* dor = reinterpret_cast<const uint4*>(p.P.dout + off);
+                const uint4* gr = reinterpret_cast<const uint4*>(L.g + off);
+#pragma unroll 2
+                for (int c = 0; c < 16; ++c) {
+                    uint32_t da[4] = {0u, 0u, 0u, 0u};
+                    if (valid) {
+                        const uint4 ud = __ldg(dor + c), ug = __ldg(gr + c);
+                        const uint32_t wd[4] = {ud.x, ud.y, ud.z, ud.w}, wg[4] = {ug.x, ug.y, ug.z, ug.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 fd = unpack_bf16(wd[e]), fg = unpack_bf16(wg[e]);
+                            da[e] = pack2<true>(fd.x * sigmoidf_(fg.x) * dsc_a, fd.y * sigmoidf_(fg.y) * dsc_a);
+                        }
+                    }
+                    *tile_chunk(sm.dA[buf][0], sm.dA[buf][1], r, c) = make_uint4(da[0], da[1], da[2], da[3]);
+                }
+                const size_t ro = ((size_t)x.b * L.Hq + hg) * L.S + (valid ? i : 0);
+                sm.lse2[buf][r] = valid ? p.P.lse2[ro] : INFINITY;
+                sm.delta[buf][r] = valid ? p.P.delta[ro] : 0.f;
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.bar[KB_QREADY + buf]);
+            }
+        }
+    } else if (warp >= 12) {
+        // ================================================ dv, dk epilogue (thread = key row)
+        const int r = tid - 384, wq = warp - 12;
+        const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+        int uu = 0;
+        for (int u = u_begin; u < u_end; ++u, ++uu) {
+            const UnitInfo x = decode_unit(L, u);
+            const int j = x.kt * TF_BN + r;
+            const bool valid = j < L.S;
+            if (!mbar_wait(&sm.bar[KB_DVKFULL], uu & 1, abort, 240)) break;
+            tc_fence_after();
+            const size_t off = ((size_t)(x.b * (size_t)L.S + (valid ? j : 0)) * L.Hkv + x.kvh) * kD;
+            const float dvf = sm.dainv[uu & 1];
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                tmem_ld32(TM_DV + lane_off + 32 * c, v);
+                tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint32_t o[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            o[e] = pack_bf16(__uint_as_float(v[8 * q4 + 2 * e]) * dvf,
+                                             __uint_as_float(v[8 * q4 + 2 * e + 1]) * dvf);
+                        reinterpret_cast<uint4*>(p.P.dv + off)[4 * c + q4] = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                }
+            }
+            const float f = L.scale / (sm.dsc[uu & 1][r] * oscale);
+            row_rope_rms_backward(TM_DK + lane_off, f, L.k + off, p.P.dk + off, valid, j, sm.gk, sm.dgk[wq], L);
+            tc_fence_before();
+            mbar_arrive(&sm.bar[KB_DVKEMPTY]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+    if (tid < kD)
+        p.P.dgk_part[(size_t)blockIdx.x * kD + tid] = (sm.dgk[0][tid] + sm.dgk[1][tid]) + (sm.dgk[2][tid] + sm.dgk[3][tid]);
+    if (tid == 0 && sm.abort && p.err) atomicExch(p.err, sm.abort);
+}
+
+// =====================================================================  host side
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_b() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+bool make_map_b(CUtensorMap* map, const void* base, int H, int S, int B) {
+    auto enc = get_encode_b();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)S * H * kD * 2};
+    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern const char* const kBwdTcKernelNames[] = {"bwd_q_tc_kernel", "bwd_kv_tc_kernel", "dgamma_reduce_kernel(k)",
+                                                "dgamma_reduce_kernel(q)"};
+extern const int kBwdTcKernelCount = 4;
+
+__global__ void dgamma_reduce_kernel(const float* __restrict__ parts, int n, float* __restrict__ out);
+
+bool bwd_tc_supported(const LayerParams& L) {
+    return L.W <= TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1 && get_encode_b() != nullptr;
+}
+
+// workspace of the tcgen05 backward: lse2, delta, domax [B,Hq,S] fp32; 2 x partials
+size_t bwd_tc_workspace_bytes(int B, int S, int Hq) {
+    const size_t rows = (size_t)B * S * Hq;
+    auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
+    return 3 * a(rows * sizeof(float)) + 2 * a((size_t)TB_MAX_GRID * kD * sizeof(float));
+}
+
+cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, cudaStream_t stream,
+                          void* const* events, int n_pairs) {
+    BwdTcParams p;
+    p.P = bp;
+    const LayerParams& L = bp.L;
+    const size_t rows = (size_t)L.B * L.S * L.Hq;
+    auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
+    char* ws = static_cast<char*>(workspace);
+    p.P.lse2 = reinterpret_cast<float*>(ws);
+    p.P.delta = reinterpret_cast<float*>(ws + a(rows * 4));
+    p.domax = reinterpret_cast<float*>(ws + 2 * a(rows * 4));
+    p.P.dgq_part = reinterpret_cast<float*>(ws + 3 * a(rows * 4));
+    p.P.dgk_part = reinterpret_cast<float*>(ws + 3 * a(rows * 4) + a((size_t)TB_MAX_GRID * kD * 4));
+    p.err = err_word;
+    if (!make_map_b(&p.tm_q, L.q, L.Hq, L.S, L.B) || !make_map_b(&p.tm_k, L.k, L.Hkv, L.S, L.B) ||
+        !make_map_b(&p.tm_v, L.v, L.Hkv, L.S, L.B))
+        return cudaErrorInvalidValue;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    sms = sms < TB_MAX_GRID ? sms : TB_MAX_GRID;
+    const size_t smem_q = sizeof(BwdQTcSmem) + 1024, smem_k = sizeof(BwdKTcSmem) + 1024;
+    if ((e = cudaFuncSetAttribute(bwd_q_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_q)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(bwd_kv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_k)) != cudaSuccess)
+        return e;
+    // events[2i] / events[2i+1] bracket kernel i (i < n_pairs)
+    auto before = [&](int i) -> cudaError_t {
+        return i < n_pairs ? cudaEventRecord(static_cast<cudaEvent_t>(events[2 * i]), stream) : cudaSuccess;
+    };
+    auto after = [&](int i) -> cudaError_t {
+        cudaError_t le = cudaGetLastError();
+        if (le != cudaSuccess) return le;
+        return i < n_pairs ? cudaEventRecord(static_cast<cudaEvent_t>(events[2 * i + 1]), stream) : cudaSuccess;
+    };
+    const int nqb = (L.S + TF_BM - 1) / TF_BM;
+    const long long steps = (long long)L.B * L.Hkv * nqb;  // query-major steps = key-major units
+    if (steps > 0x7fffffffLL) return cudaErrorInvalidValue;
+    p.total = (int)steps;
+    const int grid = (int)(steps < sms ? steps : sms);
+    if ((e = before(0)) != cudaSuccess) return e;
+    bwd_q_tc_kernel<<<grid, TB_THREADS, smem_q, stream>>>(p);
+    if ((e = after(0)) != cudaSuccess) return e;
+    if ((e = before(1)) != cudaSuccess) return e;
+    bwd_kv_tc_kernel<<<grid, TB_THREADS, smem_k, stream>>>(p);
+    if ((e = after(1)) != cudaSuccess) return e;
+    if ((e = before(2)) != cudaSuccess) return e;
+    dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgk_part, grid, bp.dgamma_k);
+    if ((e = after(2)) != cudaSuccess) return e;
+    if ((e = before(3)) != cudaSuccess) return e;
+    dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgq_part, grid, bp.dgamma_q);
+    return after(3);
+}
+
+}  // namespace zgcm

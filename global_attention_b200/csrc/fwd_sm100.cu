@@ -20,23 +20,18 @@
 //                                            B (V, d-contiguous) MN-major in smem
 //   out = sigmoid(g) * O / l                 epilogue, 16-byte global loads/stores
 //
-// Warp roles (384 threads): w0 TMA K/V, w1 MMA issue + TMEM owner, w2 TMA Q, w3 idle,
-// w4-7 softmax, w8-11 prologue (K~, Q~ in place) + gate epilogue.  Every wait is bounded;
+// Warp roles (512 threads): w0 TMA K/V, w1 MMA issue + TMEM owner, w2 TMA Q, w3 idle,
+// w4-7 softmax, w8-11 prologue (K~, Q~ in place), w12-15 gate epilogue.  Every wait is bounded;
 // on expiry the CTA records the site, drains, frees TMEM and returns.
 #include <cudaTypedefs.h>
 
 #include "sm100.cuh"
+#include "tc_rows.cuh"
 
 namespace zgcm {
 using namespace sm100;
 
-constexpr int TF_BM = 128;
-constexpr int TF_BN = 128;
-constexpr int TF_THREADS = 384;
-constexpr int TF_HALF = 21;              // rotated pairs (rope_dims = 42)
-constexpr uint32_t TF_TILE_BYTES = TF_BN * kD * 2;   // one 128 x 128 bf16 tile
-constexpr uint32_t TF_HALF_BYTES = TF_BN * 64 * 2;   // one 128-row x 64-col half: 16 KB
-constexpr uint32_t TF_RING_HALF = 2 * TF_HALF_BYTES; // one d-half of the 2-slot ring: 32 KB
+constexpr int TF_THREADS = 512;
 
 struct FwdTcParams {
     CUtensorMap tm_q;   // {D, Hq, S, B}, box {64, 1, 128, 1}, 128B swizzle
@@ -70,116 +65,6 @@ struct FwdTcSmem {
     uint32_t tmem_base;
     int abort;
 };
-
-struct StepInfo {
-    int b, kvh, qb;
-    bool fresh;        // first step of a chain in this CTA: load the previous tile too
-    bool release_cur;  // the next step does not reuse this step's current tile
-};
-
-__device__ __forceinline__ StepInfo decode_step(const LayerParams& L, int t, int t_begin, int t_end) {
-    const int nqb = (L.S + TF_BM - 1) / TF_BM;
-    StepInfo s;
-    const int chain = t / nqb;
-    s.qb = t - chain * nqb;
-    s.b = chain / L.Hkv;
-    s.kvh = chain - s.b * L.Hkv;
-    s.fresh = (t == t_begin) || (s.qb == 0);
-    s.release_cur = (t + 1 >= t_end) || (s.qb + 1 == nqb);
-    return s;
-}
-
-__device__ __forceinline__ float fast_exp2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-__device__ __forceinline__ float fast_tanh(float x) {
-    float y;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// ------------------------------------------------------------------ prologue (one row per thread)
-
-// cos/sin of the TF_HALF rotation angles at `pos`, into column r of the table
-__device__ __forceinline__ void tf_angles(const LayerParams& L, int pos, float2 (*cs)[TF_BM], int r) {
-#pragma unroll
-    for (int t = 0; t < TF_HALF; ++t) {
-        float c, s;
-        rope_cs(L.theta[t], pos, c, s);
-        cs[t][r] = make_float2(c, s);
-    }
-}
-
-// Row `r` of a 128-row tile stored as two 16 KB d-halves (h0, h1), 128-byte swizzled:
-// normalise (RMS, gamma), rotate pairs (t, t+21) for t < 21, write back bf16 in place.
-// Rows outside the sequence are zero-filled by TMA and stay zero.
-__device__ __forceinline__ void tf_prologue_row(unsigned char* h0, unsigned char* h1, int r, const float* gamma,
-                                                const LayerParams& L, const float2 (*cs)[TF_BM]) {
-    // chunk ch (8 dims, 16 bytes) of the row: half ch / 8, swizzled position (ch % 8) ^ (r % 8)
-    auto chunk = [&](int ch) -> uint4* {
-        unsigned char* hb = ch < 8 ? h0 : h1;
-        return reinterpret_cast<uint4*>(hb + (uint32_t)r * 128u + (uint32_t)(((ch & 7) ^ (r & 7)) << 4));
-    };
-    float ss = 0.f;
-#pragma unroll
-    for (int ch = 0; ch < 16; ++ch) {
-        const uint4 u = *chunk(ch);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float2 f = unpack_bf16(w[e]);
-            ss = fmaf(f.x, f.x, ss);
-            ss = fmaf(f.y, f.y, ss);
-        }
-    }
-    // a zero row (outside the sequence, zero-filled by TMA) stays zero even with eps = 0
-    const float rinv = ss > 0.f ? rsqrtf(ss * (1.0f / kD) + L.eps) : 0.f;
-    // dims 0..47 (chunks 0..5): normalise, rotate the first 42
-    float y[48];
-#pragma unroll
-    for (int ch = 0; ch < 6; ++ch) {
-        const uint4 u = *chunk(ch);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float2 f = unpack_bf16(w[e]);
-            const int d = ch * 8 + 2 * e;
-            y[d] = (f.x * rinv) * gamma[d];
-            y[d + 1] = (f.y * rinv) * gamma[d + 1];
-        }
-    }
-#pragma unroll
-    for (int t = 0; t < TF_HALF; ++t) {
-        const float a = y[t], bb = y[t + TF_HALF];
-        const float2 w = cs[t][r];
-        y[t] = a * w.x - bb * w.y;
-        y[t + TF_HALF] = bb * w.x + a * w.y;
-    }
-#pragma unroll
-    for (int ch = 0; ch < 6; ++ch) {
-        uint4 o;
-        o.x = pack_bf16(y[ch * 8 + 0], y[ch * 8 + 1]);
-        o.y = pack_bf16(y[ch * 8 + 2], y[ch * 8 + 3]);
-        o.z = pack_bf16(y[ch * 8 + 4], y[ch * 8 + 5]);
-        o.w = pack_bf16(y[ch * 8 + 6], y[ch * 8 + 7]);
-        *chunk(ch) = o;
-    }
-    // dims 48..127: normalise only
-#pragma unroll
-    for (int ch = 6; ch < 16; ++ch) {
-        const uint4 u = *chunk(ch);
-        uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float2 f = unpack_bf16(w[e]);
-            const int d = ch * 8 + 2 * e;
-            w[e] = pack_bf16((f.x * rinv) * gamma[d], (f.y * rinv) * gamma[d + 1]);
-        }
-        *chunk(ch) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
 
 // ------------------------------------------------------------------ the kernel
 
@@ -416,57 +301,11 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
             }
             if (stop) break;
         }
-    } else if (warp >= 8) {
-        // ================================================ prologue (K~, Q~ in place) + gate epilogue
-        const int r = tid - 256, wq = warp - 8;
-        const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
-        int n_next = 0, m = 0, me = 0;
-        int pend_b[2] = {0, 0}, pend_h[2] = {0, 0}, pend_q[2] = {0, 0};
+    } else if (warp >= 8 && warp < 12) {
+        // ================================================ prologue: K~, Q~ normalised + rotated in place
+        const int r = tid - 256;
+        int n_next = 0, m = 0;
         bool ok = true;
-
-        auto epilogue = [&](int e) -> bool {
-            const int buf = e & 1;
-            const int b = pend_b[buf], hg = pend_h[buf], i = pend_q[buf] * TF_BM + r;
-            const bool valid = i < L.S;
-            const size_t off = ((size_t)(b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hg) * kD;
-            if (!mbar_wait(&sm.bar[B_OFULL + buf], (e >> 1) & 1, abort, 30)) return false;
-            if (!mbar_wait(&sm.bar[B_LFULL + buf], (e >> 1) & 1, abort, 31)) return false;
-            const float inv = sm.rowinv[buf][r];
-            mbar_arrive(&sm.bar[B_LEMPTY + buf]);
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint4 gr[4];
-                if (valid) {
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) gr[q4] = __ldg(reinterpret_cast<const uint4*>(L.g + off + 32 * c) + q4);
-                }
-                uint32_t v[32];
-                tmem_ld32(TM_O0 + buf * 128 + lane_off + 32 * c, v);
-                tmem_wait_ld();
-                if (valid) {
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const uint4 g4 = gr[q4];
-                        const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
-                        uint32_t ow[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const float2 gf = unpack_bf16(gw[e2]);
-                            // sigmoid(x) = 0.5 + 0.5 tanh(x / 2)
-                            const float s0 = fmaf(0.5f, fast_tanh(0.5f * gf.x), 0.5f);
-                            const float s1 = fmaf(0.5f, fast_tanh(0.5f * gf.y), 0.5f);
-                            const int col = 8 * q4 + 2 * e2;
-                            ow[e2] = pack_bf16(s0 * (__uint_as_float(v[col]) * inv), s1 * (__uint_as_float(v[col + 1]) * inv));
-                        }
-                        *reinterpret_cast<uint4*>(p.out + off + 32 * c + 8 * q4) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                    }
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(&sm.bar[B_OEMPTY + buf]);
-            return true;
-        };
         auto prologue_k = [&](int n, int pos0) -> bool {
             const int slot = n & 1;
             if (!mbar_wait(&sm.bar[B_KFULL + slot], (n >> 1) & 1, abort, 32)) return false;
@@ -476,7 +315,6 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
             mbar_arrive(&sm.bar[B_KREADY + slot]);
             return true;
         };
-
         for (int t = t_begin; t < t_end && ok; ++t) {
             const StepInfo st = decode_step(L, t, t_begin, t_end);
             const int q0 = st.qb * TF_BM;
@@ -490,18 +328,61 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
                 tf_prologue_row(sm.Q[buf][0], sm.Q[buf][1], r, sm.gq, L, sm.cs);
                 fence_proxy_async_smem();
                 mbar_arrive(&sm.bar[B_QREADY + buf]);
-                pend_b[buf] = st.b;
-                pend_h[buf] = st.kvh * G + h;
-                pend_q[buf] = st.qb;
-                if (m >= 1) {
-                    if (!(ok = epilogue(me))) break;
-                    ++me;
-                }
             }
         }
-        while (ok && me < m) {
-            if (!(ok = epilogue(me))) break;
-            ++me;
+    } else if (warp >= 12) {
+        // ================================================ gate epilogue: out = sigmoid(g) * O / l
+        // A warpgroup of its own, so the gate loads of head m are in flight while it waits
+        // for head m's P.V to finish.
+        const int r = tid - 384, wq = warp - 12;
+        const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+        int e = 0;
+        bool ok = true;
+        for (int t = t_begin; t < t_end && ok; ++t) {
+            const StepInfo st = decode_step(L, t, t_begin, t_end);
+            const int i = st.qb * TF_BM + r;
+            const bool valid = i < L.S;
+            for (int h = 0; h < G; ++h, ++e) {
+                const int buf = e & 1, hg = st.kvh * G + h;
+                const size_t off = ((size_t)(st.b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hg) * kD;
+                uint4 gr[16];
+                if (valid) {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) gr[c] = __ldg(reinterpret_cast<const uint4*>(L.g + off) + c);
+                }
+                if (!(ok = mbar_wait(&sm.bar[B_OFULL + buf], (e >> 1) & 1, abort, 30))) break;
+                if (!(ok = mbar_wait(&sm.bar[B_LFULL + buf], (e >> 1) & 1, abort, 31))) break;
+                const float inv = sm.rowinv[buf][r];
+                mbar_arrive(&sm.bar[B_LEMPTY + buf]);
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(TM_O0 + buf * 128 + lane_off + 32 * c, v);
+                    tmem_wait_ld();
+                    if (valid) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const uint4 g4 = gr[4 * c + q4];
+                            const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
+                            uint32_t ow[4];
+#pragma unroll
+                            for (int e2 = 0; e2 < 4; ++e2) {
+                                const float2 gf = unpack_bf16(gw[e2]);
+                                // sigmoid(x) = 0.5 + 0.5 tanh(x / 2)
+                                const float s0 = fmaf(0.5f, fast_tanh(0.5f * gf.x), 0.5f);
+                                const float s1 = fmaf(0.5f, fast_tanh(0.5f * gf.y), 0.5f);
+                                const int col = 8 * q4 + 2 * e2;
+                                ow[e2] = pack_bf16(s0 * (__uint_as_float(v[col]) * inv),
+                                                   s1 * (__uint_as_float(v[col + 1]) * inv));
+                            }
+                            *reinterpret_cast<uint4*>(p.out + off + 32 * c + 8 * q4) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.bar[B_OEMPTY + buf]);
+            }
         }
     }
 

@@ -15,6 +15,12 @@ bool fwd_tc_supported(const LayerParams& L);
 cudaError_t launch_bwd_mma(const BwdParams& p, cudaStream_t stream, void* const* events, int n_pairs);
 extern const char* const kBwdMmaKernelNames[];
 extern const int kBwdMmaKernelCount;
+cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, cudaStream_t stream,
+                          void* const* events, int n_pairs);
+bool bwd_tc_supported(const LayerParams& L);
+size_t bwd_tc_workspace_bytes(int B, int S, int Hq);
+extern const char* const kBwdTcKernelNames[];
+extern const int kBwdTcKernelCount;
 int bwd_mma_n_k_parts(int B, int S, int Hkv);
 long long bwd_mma_n_q_parts(int B, int S, int Hq);
 }  // namespace zgcm
@@ -162,7 +168,9 @@ const char* zgcm_attn_fwd_kernel_name(int B, int S, int Hq, int Hkv, int rope_di
 size_t zgcm_attn_bwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int window) {
     if (check_shape(B, S, Hq, Hkv, D, 0, 1.0, window, 1, 0.f, 1.f) != ZGCM_OK) return 0;
     if ((long long)B * S == 0) return 0;
-    return bwd_layout(B, S, Hq, Hkv).total;
+    // enough for either backward (the kernel choice also depends on rope_dims)
+    const size_t a = bwd_layout(B, S, Hq, Hkv).total, b = bwd_tc_workspace_bytes(B, S, Hq);
+    return a > b ? a : b;
 }
 
 int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void* g,
@@ -190,7 +198,8 @@ int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void*
     for (const void* p : ptrs)
         if (!aligned16(p)) return ZGCM_ERR_ALIGNMENT;
     const BwdWorkspace w = bwd_layout(B, S, Hq, Hkv);
-    if (!workspace || workspace_bytes < w.total) return ZGCM_ERR_WORKSPACE;
+    const size_t need = zgcm_attn_bwd_workspace_size(B, S, Hq, Hkv, D, window);
+    if (!workspace || workspace_bytes < need) return ZGCM_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ZGCM_ERR_ALIGNMENT;
     if (w.n_q_parts > 0x7fffffffLL) return ZGCM_ERR_UNSUPPORTED;
 
@@ -215,12 +224,21 @@ int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void*
     p.n_k_parts = w.n_k_parts;
     p.n_q_parts = (int)w.n_q_parts;
     if (n_pairs < 0 || (n_pairs > 0 && !events)) return ZGCM_ERR_INVALID_ARG;
-    return launch_bwd_mma(p, stream, events, n_pairs) == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
+    cudaError_t e;
+    if (!force_mma() && bwd_tc_supported(p.L))
+        e = launch_bwd_tc(p, workspace, device_error_word(), stream, events, n_pairs);
+    else
+        e = launch_bwd_mma(p, stream, events, n_pairs);
+    return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
 }
 
-const char* zgcm_attn_bwd_kernel_name(int i, int S, int window) {
-    (void)S; (void)window;
-    return (i >= 0 && i < kBwdMmaKernelCount) ? kBwdMmaKernelNames[i] : nullptr;
+const char* zgcm_attn_bwd_kernel_name(int i, int S, int rope_dims, int window) {
+    LayerParams L{};
+    L.B = 1; L.S = S; L.rope_half = rope_dims / 2; L.W = window;
+    const bool tc = !force_mma() && S >= 1 && bwd_tc_supported(L);
+    const char* const* names = tc ? kBwdTcKernelNames : kBwdMmaKernelNames;
+    const int n = tc ? kBwdTcKernelCount : kBwdMmaKernelCount;
+    return (i >= 0 && i < n) ? names[i] : nullptr;
 }
 
 int zgcm_attn_bwd(const void* q, const void* k, const void* v, const void* g,

@@ -170,9 +170,11 @@ const char* zgcm_attn_fwd_kernel_name(int B, int S, int Hq, int Hkv, int rope_di
  */
 int zgcm_attn_device_error(void);
 
-/* Name of the i-th kernel zgcm_attn_bwd launches for this window/sequence configuration
- * (static string), or NULL when i is past the last one. */
-const char* zgcm_attn_bwd_kernel_name(int i, int S, int window);
+/* Name of the i-th kernel zgcm_attn_bwd launches for this configuration (static string),
+ * or NULL when i is past the last one.  Windows up to 128 with 42 rotated dims run the
+ * tcgen05 pair (bwd_q_tc_kernel, bwd_kv_tc_kernel); other shapes, or ZGCM_FORCE_MMA=1, the
+ * warp-MMA kernels. */
+const char* zgcm_attn_bwd_kernel_name(int i, int S, int rope_dims, int window);
 
 #ifdef __cplusplus
 }

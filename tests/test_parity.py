@@ -98,6 +98,28 @@ def test_forward_both_kernel_paths(B, S, W, monkeypatch):
         assert_lse_close(f"lse[{name}]", l, ref_lse)
 
 
+@pytest.mark.parametrize("B,S,W", [(1, 1024, 128), (2, 1000, 128), (1, 129, 7), (3, 260, 1), (1, 1, 128),
+                                   (2, 384, 100)])
+def test_backward_both_kernel_paths(B, S, W, monkeypatch):
+    """The tcgen05 backward pair (default for W <= 128, 42 rotated dims) and the warp-MMA
+    backward (forced) both match the oracle's gradients on the same inputs."""
+    t = make_inputs(B, S, seed=200 + S + W, with_dout=True)
+    d = _to_dev(t)
+    ref = _problem(t, window=W).backward(t["dout"])
+    monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
+    assert ga.zgcm_attn_bwd_kernel_names(S, W)[:2] == ["bwd_q_tc_kernel", "bwd_kv_tc_kernel"]
+    out, lse = _gpu_fwd(d, window=W)
+    got_tc = _gpu_bwd(d, out, lse, window=W)
+    assert ga.zgcm_attn_device_error() == 0
+    monkeypatch.setenv("ZGCM_FORCE_MMA", "1")
+    got_mma = _gpu_bwd(d, out, lse, window=W)
+    for name, gr in (("tc", got_tc), ("mma", got_mma)):
+        for n in ("dq", "dk", "dv", "dg"):
+            assert_bf16_close(f"{n}[{name}]", gr[n], ref[n])
+        assert_dgamma_close(f"dgamma_q[{name}]", gr["dgamma_q"], ref["dgamma_q"])
+        assert_dgamma_close(f"dgamma_k[{name}]", gr["dgamma_k"], ref["dgamma_k"])
+
+
 def test_empty_problem():
     for B, S in ((0, 16), (2, 0)):
         t = make_inputs(max(B, 1), max(S, 1), with_dout=True)
