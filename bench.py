@@ -73,10 +73,12 @@ def work(B, S, W, bwd):
         "bwd_dq_kernel": (qb + 2 * kb + qb + lse + qb + lse, 6 * D * npair),
         # q, k, v, dA, lse, Delta -> dk, dv ; S, dP, dV, dK
         "bwd_main_kernel": (qb + 2 * kb + qb + 2 * lse + 2 * kb, 8 * D * npair),
-        # tcgen05 pair: q, k, v, dout, g, out -> dq, dg (+ per-row lse, Delta, max|dout|) ;
-        # S, dP, dQ  |  q, k, v, dout, g, row stats -> dk, dv ; S, dP, dV, dK
-        "bwd_q_tc_kernel": (qb + 2 * kb + 3 * qb + 2 * qb + 3 * lse, 6 * D * npair),
-        "bwd_kv_tc_kernel": (qb + 2 * kb + 2 * qb + 3 * lse + 2 * kb, 8 * D * npair),
+        # tcgen05 backward: gate pass dout, g, out -> dg, dA16 (fp16), 2^-e and max|dout| per row;
+        # q, k, v, dA16, 2^-e -> dq, lse, Delta ; S, dP, dQ  |
+        # q, k, v, dA16, 4 row stats -> dk, dv ; S, dP, dV, dK
+        "bwd_gate_kernel": (5 * qb + 2 * lse, 0),
+        "bwd_q_tc_kernel": (qb + 2 * kb + qb + qb + 3 * lse, 6 * D * npair),
+        "bwd_kv_tc_kernel": (qb + 2 * kb + qb + 4 * lse + 2 * kb, 8 * D * npair),
     }
     return dict(tokens=tok, npair=npair, fwd_bytes=fwd_bytes, fwd_flops=fwd_flops,
                 bwd_bytes=bwd_bytes if bwd else 0, bwd_flops=bwd_flops if bwd else 0,

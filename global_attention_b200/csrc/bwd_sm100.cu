@@ -2,16 +2,18 @@
 //
 // Exact gradients of L = sum(dout * out) for the ZGCM-1 layer (definition and page
 // citations in common.cuh), for windows W <= 128 and 42 rotated dims; other shapes run on
-// the warp-MMA kernels (bwd_mma.cu).  Two kernels:
+// the warp-MMA kernels (bwd_mma.cu).  Three kernels:
 //
+//   bwd_gate   streaming pass over dout, g, out (coalesced, 16 lanes per row): the gate
+//              backward dg = dout*out*(1-sigmoid(g)), and dA = dout*sigmoid(g) stored as fp16
+//              scaled by a power of two per row (2^-e and max|dout| saved per row).
 //   bwd_q_tc   query-major sweep over (b, KV head, 128-query block) steps, all query heads
 //              of the group per step, key tiles qb-1 and qb in a 2-slot ring (as the forward).
 //              Per head: S = Q~ K~^T and dP = dA V^T (both M=128 N=256 into TMEM), then one
 //              warpgroup per row forms the log-sum-exp, Delta = sum_j P dP and dS = P(dP-Delta)
 //              from its own scores, dQ~ = dS K~ (M=128 N=128 K=256, dS from TMEM), and an
-//              epilogue warpgroup applies the RoPE / RMSNorm backward and writes dq.  The gate
-//              preprocessing is fused into its prologue: dA = dout*sigmoid(g) and
-//              dg = dout*out*(1-sigmoid(g)).  Writes lse, Delta and max|dout| per row.
+//              epilogue warpgroup applies the RoPE / RMSNorm backward and writes dq.  Writes
+//              lse and Delta per row.
 //   bwd_kv_tc  key-major: persistent CTAs over (b, KV head, 128-key tile) units; per unit the
 //              Hq/Hkv heads x the two query blocks that see the tile:
 //              S^T = K~ Q~^T, dP^T = V dA^T, P^T and dS^T from the saved lse and Delta,
@@ -21,10 +23,11 @@
 // Numerics.  Every product runs as kind::f16 with fp16 operands (11-bit significand) and
 // fp32 accumulation; each operand is brought into fp16 range by an exact power-of-two scale
 // that the product lets factor out: q~, k~ are RMS-normalised (one scale from gamma); dA
-// and dS rows of the query-major products; V and dS^T rows of the key-major products; dA in
-// dV by one scale per unit (a sum over query rows).  Scales are undone in fp32.  Measured
-// in a CPU emulation against the fp64 oracle this keeps every gradient within the bf16
-// output rounding of the reference (single bf16 operands did not).
+// rows (undone per row in dP, per column in dP^T); dS rows of the query-major products; V and
+// dS^T rows of the key-major products; in dV = P^T dA the dA row scales are moved onto the
+// columns of P^T relative to one scale per unit (a sum over query rows).  Scales are undone
+// in fp32.  Measured in a CPU emulation against the fp64 oracle this keeps every gradient
+// within the bf16 output rounding of the reference (single bf16 operands did not).
 #include <cudaTypedefs.h>
 
 #include "tc_rows.cuh"
@@ -39,7 +42,10 @@ struct BwdTcParams {
     CUtensorMap tm_q;   // {D, Hq, S, B}, box {64, 1, 128, 1}, 128B swizzle
     CUtensorMap tm_k;
     CUtensorMap tm_v;
+    CUtensorMap tm_da;  // dA16, fp16, same geometry as tm_q
     BwdParams P;
+    const __half* da16; // [B,S,Hq,D] dA * 2^e (e per row)
+    float* dainv;       // [B,Hq,S] 2^-e of each dA row (0 for an all-zero row)
     float* domax;       // [B,Hq,S] max |dout| of each row (bound on |dA|)
     int* err;
     int total;          // steps (query-major) or units (key-major)
@@ -59,6 +65,84 @@ __device__ __forceinline__ int fit_exp(float x) {
     if (!(x > 0.f) || !isfinite(x)) return 0;
     int e = 13 - ilogbf(x);
     return max(-120, min(120, e));
+}
+
+// =====================================================================  gate backward pass
+
+constexpr int GATE_THREADS = 256;
+constexpr int GATE_UNROLL = 4;  // rows in flight per half-warp
+
+// Sigmoid gate backward of out = sigmoid(g) * A (the gated-attention page, output gate):
+//   dA = dout * sigmoid(g)  -> da16 = fp16(dA * 2^e), e = fit_exp(max|dout| of the row)
+//   dg = dout * A * sigmoid'(g) = dout * out * (1 - sigmoid(g))
+// One half-warp per row of D = 128 (16 lanes x 8 values, fully coalesced), GATE_UNROLL rows
+// per half-warp in flight; every loop bound is warp-uniform so the row-max shuffles see all
+// 32 lanes.  dainv = 2^-e (0 when the row of dout is all zero: its dA row is zero and must
+// not be rescaled), domax = max|dout|, both [B,Hq,S].
+__global__ void __launch_bounds__(GATE_THREADS, 2) bwd_gate_kernel(const bf16* __restrict__ dout,
+                                                                const bf16* __restrict__ g,
+                                                                const bf16* __restrict__ out,
+                                                                bf16* __restrict__ dg, __half* __restrict__ da16,
+                                                                float* __restrict__ dainv,
+                                                                float* __restrict__ domax, long long rows, int S,
+                                                                int Hq) {
+    const int lane = threadIdx.x & 31, sub = lane & 15;
+    const long long warp0 = ((long long)blockIdx.x * GATE_THREADS + threadIdx.x) >> 5;
+    const long long nwarps = ((long long)gridDim.x * GATE_THREADS) >> 5;
+    const long long stride = 2 * nwarps;  // rows between the k-th rows of consecutive unroll slots
+    for (long long base = 2 * warp0; base < rows; base += GATE_UNROLL * stride) {
+        uint4 ud[GATE_UNROLL], ug[GATE_UNROLL], uo[GATE_UNROLL];
+#pragma unroll
+        for (int k = 0; k < GATE_UNROLL; ++k) {
+            const long long r = base + k * stride + (lane >> 4);
+            ud[k] = ug[k] = uo[k] = make_uint4(0u, 0u, 0u, 0u);
+            if (r < rows) {
+                const size_t o = (size_t)r * (kD / 8) + sub;
+                ud[k] = __ldg(reinterpret_cast<const uint4*>(dout) + o);
+                ug[k] = __ldg(reinterpret_cast<const uint4*>(g) + o);
+                uo[k] = __ldg(reinterpret_cast<const uint4*>(out) + o);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < GATE_UNROLL; ++k) {
+            const long long r = base + k * stride + (lane >> 4);
+            const uint32_t wd[4] = {ud[k].x, ud[k].y, ud[k].z, ud[k].w};
+            const uint32_t wg[4] = {ug[k].x, ug[k].y, ug[k].z, ug[k].w};
+            const uint32_t wo[4] = {uo[k].x, uo[k].y, uo[k].z, uo[k].w};
+            float mx = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 fd = unpack_bf16(wd[e]);
+                mx = fmaxf(mx, fmaxf(fabsf(fd.x), fabsf(fd.y)));
+            }
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const int ea = fit_exp(mx);
+            const float sc = ldexpf(1.0f, ea);
+            uint32_t da[4], dgw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 fd = unpack_bf16(wd[e]), fg = unpack_bf16(wg[e]), fo = unpack_bf16(wo[e]);
+                const float s0 = sigmoidf_(fg.x), s1 = sigmoidf_(fg.y);
+                da[e] = pack2<true>(fd.x * s0 * sc, fd.y * s1 * sc);
+                dgw[e] = pack_bf16(fd.x * fo.x * (1.f - s0), fd.y * fo.y * (1.f - s1));
+            }
+            if (r < rows) {
+                const size_t o = (size_t)r * (kD / 8) + sub;
+                reinterpret_cast<uint4*>(da16)[o] = make_uint4(da[0], da[1], da[2], da[3]);
+                reinterpret_cast<uint4*>(dg)[o] = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
+                if (sub == 0) {
+                    // row r = (b*S + s)*Hq + h  ->  [B,Hq,S] index (b*Hq + h)*S + s
+                    const long long sh = (long long)S * Hq;
+                    const long long b = r / sh, rem = r - b * sh;
+                    const long long s = rem / Hq, h = rem - s * Hq;
+                    const size_t ro = (size_t)(b * Hq + h) * S + s;
+                    dainv[ro] = mx > 0.f ? 1.0f / sc : 0.f;
+                    domax[ro] = mx;
+                }
+            }
+        }
+    }
 }
 
 // 32 lanes x 16 consecutive 32-bit columns load
@@ -196,18 +280,17 @@ __device__ __forceinline__ void row_rope_rms_backward(uint32_t taddr, float f, c
 enum QBar {
     QB_KFULL = 0, QB_KREADY = 2, QB_KEMPTY = 4, QB_VFULL = 6, QB_VREADY = 8, QB_VEMPTY = 10,
     QB_QFULL = 12, QB_QREADY = 13, QB_QEMPTY = 14, QB_DAEMPTY = 15,
-    QB_SFULL = 16, QB_DSFULL = 17, QB_DQFULL = 18, QB_DQEMPTY = 19, QB_DONE = 20, QB_COUNT = 21
+    QB_SFULL = 16, QB_DSFULL = 17, QB_DQFULL = 18, QB_DQEMPTY = 19, QB_DONE = 20, QB_DAFULL = 21, QB_COUNT = 22
 };
 
 struct BwdQTcSmem {
     alignas(1024) unsigned char K[2][TF_RING_HALF];    // K~ fp16, 2-slot ring split by d-half
     alignas(1024) unsigned char V[2][TF_RING_HALF];    // V fp16, row-scaled
     alignas(1024) unsigned char Q[2][TF_HALF_BYTES];   // raw q -> Q~ fp16 in place
-    alignas(1024) unsigned char dA[2][TF_HALF_BYTES];  // dA fp16, row-scaled
+    alignas(1024) unsigned char dA[2][TF_HALF_BYTES];  // dA fp16, row-scaled (TMA from the gate pass)
     float2 cs[TF_HALF][TF_BM];
     float gq[kD], gk[kD];
     float vinv[4][TF_BN];    // 2^-e of each V row, by tile number % 4
-    float dainv[2][TF_BM];   // 2^-e of each dA row, by head number % 2
     float dsinv[TF_BM];      // 2^-e of each dS row of the current head
     float dgq[4][kD];        // this CTA's d_gamma_q, one slice per epilogue warp
     uint64_t bar[QB_COUNT];
@@ -272,6 +355,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
         mbar_init(&sm.bar[QB_QREADY], 128);
         mbar_init(&sm.bar[QB_QEMPTY], 1);
         mbar_init(&sm.bar[QB_DAEMPTY], 1);
+        mbar_init(&sm.bar[QB_DAFULL], 1);
         mbar_init(&sm.bar[QB_SFULL], 1);
         mbar_init(&sm.bar[QB_DSFULL], 128);
         mbar_init(&sm.bar[QB_DQFULL], 1);
@@ -292,6 +376,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
         prefetch_tmap(&p.tm_q);
         prefetch_tmap(&p.tm_k);
         prefetch_tmap(&p.tm_v);
+        prefetch_tmap(&p.tm_da);
     }
     tc_fence_before();
     __syncthreads();
@@ -331,21 +416,28 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             }
         }
     } else if (warp == 2) {
-        // ================================================ Q producer (single buffer)
+        // ================================================ Q and dA producer (single buffers)
         if (lane == 0) {
-            int m = 0, last = -1;
-            for (int t = t_begin; t < t_end && !*abort; ++t) {
+            int m = 0, last = -1, last_da = -1;
+            bool ok = true;
+            for (int t = t_begin; t < t_end && ok && !*abort; ++t) {
                 const StepInfo st = decode_step(L, t, t_begin, t_end);
                 for (int h = 0; h < G; ++h, ++m) {
-                    if (m >= 1 && !mbar_wait(&sm.bar[QB_QEMPTY], (m - 1) & 1, abort, 103)) break;
-                    mbar_expect_tx(&sm.bar[QB_QFULL], TF_TILE_BYTES);
                     const int hg = st.kvh * G + h;
+                    if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_QEMPTY], (m - 1) & 1, abort, 103))) break;
+                    mbar_expect_tx(&sm.bar[QB_QFULL], TF_TILE_BYTES);
                     tma_load_4d(sm.Q[0], &p.tm_q, &sm.bar[QB_QFULL], 0, hg, st.qb * TF_BM, st.b);
                     tma_load_4d(sm.Q[1], &p.tm_q, &sm.bar[QB_QFULL], 64, hg, st.qb * TF_BM, st.b);
                     last = m;
+                    if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_DAEMPTY], (m - 1) & 1, abort, 104))) break;
+                    mbar_expect_tx(&sm.bar[QB_DAFULL], TF_TILE_BYTES);
+                    tma_load_4d(sm.dA[0], &p.tm_da, &sm.bar[QB_DAFULL], 0, hg, st.qb * TF_BM, st.b);
+                    tma_load_4d(sm.dA[1], &p.tm_da, &sm.bar[QB_DAFULL], 64, hg, st.qb * TF_BM, st.b);
+                    last_da = m;
                 }
             }
             if (last >= 0) mbar_wait_drain(&sm.bar[QB_QFULL], last & 1);
+            if (last_da >= 0) mbar_wait_drain(&sm.bar[QB_DAFULL], last_da & 1);
         }
     } else if (warp == 1) {
         // ================================================ MMA issuer
@@ -371,6 +463,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                      mbar_wait(&sm.bar[QB_VREADY + (n_cur & 1)], (n_cur >> 1) & 1, abort, 113);
                 for (int h = 0; h < G && ok; ++h, ++m) {
                     if (!(ok = mbar_wait(&sm.bar[QB_QREADY], m & 1, abort, 114))) break;
+                    if (!(ok = mbar_wait(&sm.bar[QB_DAFULL], m & 1, abort, 118))) break;
                     if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_DQEMPTY], (m - 1) & 1, abort, 115))) break;
                     tc_fence_after();
 #pragma unroll
@@ -428,9 +521,11 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             const int imin = q0 + 32 * wq, imax = imin + 31;
             bool stop = false;
             for (int h = 0; h < G; ++h, ++m) {
+                const int hg = st.kvh * G + h;
+                const size_t ro = ((size_t)st.b * L.Hq + hg) * L.S + (i < L.S ? i : 0);
+                const float dai = i < L.S ? p.dainv[ro] : 0.f;  // undoes the dA row scale
                 if (!mbar_wait(&sm.bar[QB_SFULL], m & 1, abort, 120)) { stop = true; break; }
                 tc_fence_after();
-                const float dai = sm.dainv[m & 1][r];
                 float mx = -INFINITY;
 #pragma unroll 1
                 for (int c8 = 0; c8 < 8; ++c8) {
@@ -505,9 +600,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                     tmem_st16(TM_DS + lane_off + 16 * c8, pk);
                 }
                 tmem_wait_st();
-                const int hg = st.kvh * G + h;
                 if (i < L.S) {
-                    const size_t ro = ((size_t)st.b * L.Hq + hg) * L.S + i;
                     p.P.lse2[ro] = lse2;
                     p.P.delta[ro] = delta;
                 }
@@ -518,7 +611,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             if (stop) break;
         }
     } else if (warp >= 8 && warp < 12) {
-        // ================================================ prologue: K~, V, Q~ (fp16, in place), dA, dg
+        // ================================================ prologue: K~, V, Q~ (fp16, in place)
         const int r = tid - 256;
         int n_next = 0, m = 0;
         bool ok = true;
@@ -538,57 +631,13 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
         };
         for (int t = t_begin; t < t_end && ok; ++t) {
             const StepInfo st = decode_step(L, t, t_begin, t_end);
-            const int q0 = st.qb * TF_BM, i = q0 + r;
-            const bool valid = i < L.S;
+            const int q0 = st.qb * TF_BM;
             if (st.fresh) ok = prologue_kv(n_next++, q0 - TF_BN);
             ok = ok && prologue_kv(n_next++, q0);
             if (!ok) break;
             for (int h = 0; h < G; ++h, ++m) {
                 if (!(ok = mbar_wait(&sm.bar[QB_QFULL], m & 1, abort, 132))) break;
                 tf_prologue_row<true>(sm.Q[0], sm.Q[1], r, sm.gq, L, sm.cs, oscale);
-                if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_DAEMPTY], (m - 1) & 1, abort, 133))) break;
-                // dA = dout * sigmoid(g) (row-scaled fp16), dg = dout * out * (1 - sigmoid(g))
-                const int hg = st.kvh * G + h;
-                const size_t off = ((size_t)(st.b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hg) * kD;
-                const uint4* dor = reinterpret_cast<const uint4*>(p.P.dout + off);
-                const uint4* gr = reinterpret_cast<const uint4*>(L.g + off);
-                const uint4* outr = reinterpret_cast<const uint4*>(p.P.out + off);
-                float mx = 0.f;
-                if (valid) {
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const uint4 u = __ldg(dor + c);
-                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 t2 = unpack_bf16(w[e]);
-                            mx = fmaxf(mx, fmaxf(fabsf(t2.x), fabsf(t2.y)));
-                        }
-                    }
-                }
-                const int ea = fit_exp(mx);
-                const float sc = ldexpf(1.0f, ea);
-#pragma unroll 2
-                for (int c = 0; c < 16; ++c) {
-                    uint32_t da[4] = {0u, 0u, 0u, 0u};
-                    if (valid) {
-                        const uint4 ud = __ldg(dor + c), ug = __ldg(gr + c), uo = __ldg(outr + c);
-                        const uint32_t wd[4] = {ud.x, ud.y, ud.z, ud.w}, wg[4] = {ug.x, ug.y, ug.z, ug.w},
-                                       wo[4] = {uo.x, uo.y, uo.z, uo.w};
-                        uint32_t dgw[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 fd = unpack_bf16(wd[e]), fg = unpack_bf16(wg[e]), fo = unpack_bf16(wo[e]);
-                            const float s0 = sigmoidf_(fg.x), s1 = sigmoidf_(fg.y);
-                            da[e] = pack2<true>(fd.x * s0 * sc, fd.y * s1 * sc);
-                            dgw[e] = pack_bf16(fd.x * fo.x * (1.f - s0), fd.y * fo.y * (1.f - s1));
-                        }
-                        reinterpret_cast<uint4*>(p.P.dg + off)[c] = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
-                    }
-                    *tile_chunk(sm.dA[0], sm.dA[1], r, c) = make_uint4(da[0], da[1], da[2], da[3]);
-                }
-                if (valid) p.domax[((size_t)st.b * L.Hq + hg) * L.S + i] = mx;
-                sm.dainv[m & 1][r] = 1.0f / sc;
                 fence_proxy_async_smem();
                 mbar_arrive(&sm.bar[QB_QREADY]);
             }
@@ -638,14 +687,15 @@ struct BwdKTcSmem {
     alignas(1024) unsigned char K[2][TF_HALF_BYTES];      // K~ fp16 of the unit's key tile
     alignas(1024) unsigned char V[2][TF_HALF_BYTES];      // V fp16, row-scaled
     alignas(1024) unsigned char Q[2][2][TF_HALF_BYTES];   // [buffer][half] raw q -> Q~ fp16
-    alignas(1024) unsigned char dA[2][2][TF_HALF_BYTES];  // [buffer][half] dA fp16, unit scale
+    alignas(1024) unsigned char dA[2][2][TF_HALF_BYTES];  // [buffer][half] dA fp16, row-scaled (TMA)
     float2 cs[TF_HALF][TF_BM];
     float gq[kD], gk[kD];
     float lse2[2][TF_BM];    // per query column of the buffer
     float delta[2][TF_BM];
+    float dcol[2][TF_BM];    // 2^-e of the dA row of each query column
     float vinv[TF_BN];       // 2^-e of each V row of the current unit
     float dsc[2][TF_BN];     // 2^e of each dS^T row, by unit parity
-    float dainv[2];          // 2^-E of dA, by unit parity
+    float uinv[2];           // 2^-E, E = the unit's smallest dA row exponent, by unit parity
     float red[2][4];         // per-warp maxima for the unit statistics
     float dgk[4][kD];        // this CTA's d_gamma_k, one slice per epilogue warp
     uint64_t bar[KB_COUNT];
@@ -711,6 +761,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
         prefetch_tmap(&p.tm_q);
         prefetch_tmap(&p.tm_k);
         prefetch_tmap(&p.tm_v);
+        prefetch_tmap(&p.tm_da);
     }
     tc_fence_before();
     __syncthreads();
@@ -739,9 +790,11 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                     if (it_all >= 2 && !(ok = mbar_wait(&sm.bar[KB_QEMPTY + buf], ((it_all >> 1) - 1) & 1, abort, 202))) break;
                     int qb, hg;
                     decode_iter(L, x, it, qb, hg);
-                    mbar_expect_tx(&sm.bar[KB_QFULL + buf], TF_TILE_BYTES);
+                    mbar_expect_tx(&sm.bar[KB_QFULL + buf], 2 * TF_TILE_BYTES);
                     tma_load_4d(sm.Q[buf][0], &p.tm_q, &sm.bar[KB_QFULL + buf], 0, hg, qb * TF_BM, x.b);
                     tma_load_4d(sm.Q[buf][1], &p.tm_q, &sm.bar[KB_QFULL + buf], 64, hg, qb * TF_BM, x.b);
+                    tma_load_4d(sm.dA[buf][0], &p.tm_da, &sm.bar[KB_QFULL + buf], 0, hg, qb * TF_BM, x.b);
+                    tma_load_4d(sm.dA[buf][1], &p.tm_da, &sm.bar[KB_QFULL + buf], 64, hg, qb * TF_BM, x.b);
                     last_q[buf] = it_all;
                 }
                 if (!ok) break;
@@ -815,7 +868,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             const UnitInfo x = decode_unit(L, u);
             const int j = x.kt * TF_BN + r;
             if (!(ok = mbar_wait(&sm.bar[KB_KVREADY], uu & 1, abort, 220))) break;
-            const float vin = sm.vinv[r] * sm.dainv[uu & 1];  // undoes the V-row and dA scales of dP^T
+            const float vin = sm.vinv[r];        // undoes the V-row scale of dP^T
+            const float su = 1.0f / sm.uinv[uu & 1];  // 2^E: P^T columns carry 2^(E - e_i)
             const float dsc = sm.dsc[uu & 1][r];
             for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
                 const int buf = it_all & 1;
@@ -844,8 +898,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                                 const int ql = 32 * c8 + e + w2, i = q0 + ql;
                                 const bool vis = j <= i && j > i - L.W && i < L.S && j < L.S;
                                 const float pv = vis ? fast_exp2(__uint_as_float(sv[e + w2]) * c2 - sm.lse2[buf][ql]) : 0.f;
-                                const float dp = __uint_as_float(dv[e + w2]) * vin;
-                                pv2[w2] = pv;
+                                const float dcl = sm.dcol[buf][ql];
+                                const float dp = __uint_as_float(dv[e + w2]) * vin * dcl;
+                                pv2[w2] = pv * (dcl * su);
                                 ds2[w2] = pv * (dp - sm.delta[buf][ql]) * dsc;
                             }
                             pp[e >> 1] = pack2<true>(pv2[0], pv2[1]);
@@ -896,8 +951,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             domx = fmaxf(fmaxf(sm.red[0][0], sm.red[0][1]), fmaxf(sm.red[0][2], sm.red[0][3]));
             dlmx = fmaxf(fmaxf(sm.red[1][0], sm.red[1][1]), fmaxf(sm.red[1][2], sm.red[1][3]));
             asm volatile("bar.sync 1, 128;" ::: "memory");
+            // E = fit_exp(max domax) is the smallest row exponent of dA in the unit, so every
+            // column factor 2^(E - e_i) of P^T is <= 1
             const int E = fit_exp(domx);
-            const float dsc_a = ldexpf(1.0f, E);
             // K~ (fp16) and V (fp16, row-scaled) of the unit's key tile
             tf_angles(L, x.kt * TF_BN + r, sm.cs, r);
             tf_prologue_row<true>(sm.K[0], sm.K[1], r, sm.gk, L, sm.cs, oscale);
@@ -905,7 +961,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             sm.vinv[r] = v_row_to_f16(sm.V[0], sm.V[1], r, &vnorm);
             // dS^T row scale: |dS_ji| <= |v_j| |dA_i| + |Delta_i| <= |v_j| sqrt(D) max|dout| + max|Delta|
             sm.dsc[uu & 1][r] = ldexpf(1.0f, fit_exp(vnorm * sqrtf((float)kD) * domx + dlmx));
-            if (r == 0) sm.dainv[uu & 1] = 1.0f / dsc_a;
+            if (r == 0) sm.uinv[uu & 1] = ldexpf(1.0f, -E);
             fence_proxy_async_smem();
             mbar_arrive(&sm.bar[KB_KVREADY]);
             int cur_qb = -1;
@@ -921,27 +977,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                     cur_qb = qb;
                 }
                 tf_prologue_row<true>(sm.Q[buf][0], sm.Q[buf][1], r, sm.gq, L, sm.cs, oscale);
-                // dA row (unit-uniform scale) for query row i of head hg
-                const size_t off = ((size_t)(x.b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hg) * kD;
-                const uint4* dor = reinterpret_cast<const uint4*>(p.P.dout + off);
-                const uint4* gr = reinterpret_cast<const uint4*>(L.g + off);
-#pragma unroll 2
-                for (int c = 0; c < 16; ++c) {
-                    uint32_t da[4] = {0u, 0u, 0u, 0u};
-                    if (valid) {
-                        const uint4 ud = __ldg(dor + c), ug = __ldg(gr + c);
-                        const uint32_t wd[4] = {ud.x, ud.y, ud.z, ud.w}, wg[4] = {ug.x, ug.y, ug.z, ug.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 fd = unpack_bf16(wd[e]), fg = unpack_bf16(wg[e]);
-                            da[e] = pack2<true>(fd.x * sigmoidf_(fg.x) * dsc_a, fd.y * sigmoidf_(fg.y) * dsc_a);
-                        }
-                    }
-                    *tile_chunk(sm.dA[buf][0], sm.dA[buf][1], r, c) = make_uint4(da[0], da[1], da[2], da[3]);
-                }
                 const size_t ro = ((size_t)x.b * L.Hq + hg) * L.S + (valid ? i : 0);
                 sm.lse2[buf][r] = valid ? p.P.lse2[ro] : INFINITY;
                 sm.delta[buf][r] = valid ? p.P.delta[ro] : 0.f;
+                sm.dcol[buf][r] = valid ? p.dainv[ro] : 0.f;
                 fence_proxy_async_smem();
                 mbar_arrive(&sm.bar[KB_QREADY + buf]);
             }
@@ -958,7 +997,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             if (!mbar_wait(&sm.bar[KB_DVKFULL], uu & 1, abort, 240)) break;
             tc_fence_after();
             const size_t off = ((size_t)(x.b * (size_t)L.S + (valid ? j : 0)) * L.Hkv + x.kvh) * kD;
-            const float dvf = sm.dainv[uu & 1];
+            const float dvf = sm.uinv[uu & 1];
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 uint32_t v[32];
@@ -1010,23 +1049,24 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_b() {
     return fn;
 }
 
-bool make_map_b(CUtensorMap* map, const void* base, int H, int S, int B) {
+bool make_map_b(CUtensorMap* map, const void* base, int H, int S, int B,
+                CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     auto enc = get_encode_b();
     if (!enc) return false;
     cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)S * H * kD * 2};
     cuuint32_t box[4] = {64, 1, 128, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+    return enc(map, dtype, 4, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
-extern const char* const kBwdTcKernelNames[] = {"bwd_q_tc_kernel", "bwd_kv_tc_kernel", "dgamma_reduce_kernel(k)",
-                                                "dgamma_reduce_kernel(q)"};
-extern const int kBwdTcKernelCount = 4;
+extern const char* const kBwdTcKernelNames[] = {"bwd_gate_kernel", "bwd_q_tc_kernel", "bwd_kv_tc_kernel",
+                                                "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"};
+extern const int kBwdTcKernelCount = 5;
 
 __global__ void dgamma_reduce_kernel(const float* __restrict__ parts, int n, float* __restrict__ out);
 
@@ -1034,11 +1074,13 @@ bool bwd_tc_supported(const LayerParams& L) {
     return L.W <= TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1 && get_encode_b() != nullptr;
 }
 
-// workspace of the tcgen05 backward: lse2, delta, domax [B,Hq,S] fp32; 2 x partials
+// workspace of the tcgen05 backward: lse2, delta, domax, dainv [B,Hq,S] fp32; dA16
+// [B,S,Hq,D] fp16; 2 x d_gamma partials
 size_t bwd_tc_workspace_bytes(int B, int S, int Hq) {
     const size_t rows = (size_t)B * S * Hq;
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
-    return 3 * a(rows * sizeof(float)) + 2 * a((size_t)TB_MAX_GRID * kD * sizeof(float));
+    return 4 * a(rows * sizeof(float)) + a(rows * kD * sizeof(__half)) +
+           2 * a((size_t)TB_MAX_GRID * kD * sizeof(float));
 }
 
 cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, cudaStream_t stream,
@@ -1049,14 +1091,24 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     const size_t rows = (size_t)L.B * L.S * L.Hq;
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
     char* ws = static_cast<char*>(workspace);
-    p.P.lse2 = reinterpret_cast<float*>(ws);
-    p.P.delta = reinterpret_cast<float*>(ws + a(rows * 4));
-    p.domax = reinterpret_cast<float*>(ws + 2 * a(rows * 4));
-    p.P.dgq_part = reinterpret_cast<float*>(ws + 3 * a(rows * 4));
-    p.P.dgk_part = reinterpret_cast<float*>(ws + 3 * a(rows * 4) + a((size_t)TB_MAX_GRID * kD * 4));
+    size_t off = 0;
+    auto take = [&](size_t bytes) -> char* {
+        char* q = ws + off;
+        off += a(bytes);
+        return q;
+    };
+    p.P.lse2 = reinterpret_cast<float*>(take(rows * 4));
+    p.P.delta = reinterpret_cast<float*>(take(rows * 4));
+    p.domax = reinterpret_cast<float*>(take(rows * 4));
+    p.dainv = reinterpret_cast<float*>(take(rows * 4));
+    __half* da16 = reinterpret_cast<__half*>(take(rows * kD * sizeof(__half)));
+    p.da16 = da16;
+    p.P.dgq_part = reinterpret_cast<float*>(take((size_t)TB_MAX_GRID * kD * 4));
+    p.P.dgk_part = reinterpret_cast<float*>(take((size_t)TB_MAX_GRID * kD * 4));
     p.err = err_word;
     if (!make_map_b(&p.tm_q, L.q, L.Hq, L.S, L.B) || !make_map_b(&p.tm_k, L.k, L.Hkv, L.S, L.B) ||
-        !make_map_b(&p.tm_v, L.v, L.Hkv, L.S, L.B))
+        !make_map_b(&p.tm_v, L.v, L.Hkv, L.S, L.B) ||
+        !make_map_b(&p.tm_da, da16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1082,18 +1134,26 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     if (steps > 0x7fffffffLL) return cudaErrorInvalidValue;
     p.total = (int)steps;
     const int grid = (int)(steps < sms ? steps : sms);
+    // gate pass: 2 resident blocks of 256 threads per SM, each half-warp GATE_UNROLL rows at a time
+    const long long half_warps = ((long long)rows + GATE_UNROLL - 1) / GATE_UNROLL;
+    const long long gate_need = (half_warps * 16 + GATE_THREADS - 1) / GATE_THREADS;
+    const int gate_grid = (int)(gate_need < 2LL * sms ? gate_need : 2LL * sms);
     if ((e = before(0)) != cudaSuccess) return e;
-    bwd_q_tc_kernel<<<grid, TB_THREADS, smem_q, stream>>>(p);
+    bwd_gate_kernel<<<gate_grid, GATE_THREADS, 0, stream>>>(bp.dout, L.g, bp.out, bp.dg, da16, p.dainv, p.domax,
+                                                            (long long)rows, L.S, L.Hq);
     if ((e = after(0)) != cudaSuccess) return e;
     if ((e = before(1)) != cudaSuccess) return e;
-    bwd_kv_tc_kernel<<<grid, TB_THREADS, smem_k, stream>>>(p);
+    bwd_q_tc_kernel<<<grid, TB_THREADS, smem_q, stream>>>(p);
     if ((e = after(1)) != cudaSuccess) return e;
     if ((e = before(2)) != cudaSuccess) return e;
-    dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgk_part, grid, bp.dgamma_k);
+    bwd_kv_tc_kernel<<<grid, TB_THREADS, smem_k, stream>>>(p);
     if ((e = after(2)) != cudaSuccess) return e;
     if ((e = before(3)) != cudaSuccess) return e;
+    dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgk_part, grid, bp.dgamma_k);
+    if ((e = after(3)) != cudaSuccess) return e;
+    if ((e = before(4)) != cudaSuccess) return e;
     dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgq_part, grid, bp.dgamma_q);
-    return after(3);
+    return after(4);
 }
 
 }  // namespace zgcm
