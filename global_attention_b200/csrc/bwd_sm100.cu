@@ -155,8 +155,8 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 
 // Sum of v[e] over the 32 lanes of the warp for e = 0..31, delivered as: lane L returns the
-// total of index L (recursive halving; 31 shuffles).
-__device__ __forceinline__ float warp_transpose_sum(float (&v)[32]) {
+// total of index L (recursive halving; 31 shuffles).  v is clobbered.
+__device__ __forceinline__ float warp_transpose_sum(float* v) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int k = 16; k >= 1; k >>= 1) {
@@ -177,101 +177,156 @@ __device__ __forceinline__ uint4* tile_chunk(unsigned char* h0, unsigned char* h
     return reinterpret_cast<uint4*>(hb + (uint32_t)r * 128u + (uint32_t)(((ch & 7) ^ (r & 7)) << 4));
 }
 
-// RoPE / RMSNorm backward of one row held by one thread: dq~ (fp32, 128 columns of TMEM at
-// `taddr`, times `f`) -> dx (bf16, to `dst`), adding dy * xhat of the row into this warp's
-// d_gamma slice `dgam` (warp-transposed sums: lane L owns one dimension per 32-wide block,
-// so the slice is updated in a fixed order and the result is reproducible).  `x` is the raw row
-// in global memory; `valid` masks rows past the sequence (they still join the collectives).
-__device__ __forceinline__ void row_rope_rms_backward(uint32_t taddr, float f, const bf16* x, bf16* dst,
-                                                      bool valid, int pos, const float* gamma, float* dgam,
-                                                      const LayerParams& L) {
+// RoPE / RMSNorm backward of one row held by one thread, one pass over the row:
+//   dy = R^T (f * dq~)       (128 fp32 columns of TMEM at `taddr`; R rotates pairs (t, t+21) at `pos`)
+//   dx = (dy * gamma - xhat * mdot) * rinv,   xhat = x * rinv,   d_gamma += dy * xhat
+// The caller supplies rinv = 1/sqrt(mean x^2 + eps) (from the prologue) and
+// mdot = mean_d(dy_d gamma_d xhat_d).  Because R is orthogonal and q~ = R(gamma * xhat),
+// mdot = (q~ . dq~) / D, which the softmax warps form as a row sum of dS * S; so the raw row
+// x (global memory) is read once, here.  d_gamma goes into this warp's slice `dgam` through
+// warp-transposed sums (lane L owns one dimension per 32-wide block: a fixed summation order,
+// reproducible).  `valid` masks rows past the sequence (they still join the collectives).
+__device__ __forceinline__ void row_rope_rms_backward(uint32_t taddr, float f, float mdot, float rinv,
+                                                      const bf16* x, bf16* dst, bool valid, int pos,
+                                                      const float* gamma, float* dgam, const LayerParams& L) {
     const int lane = threadIdx.x & 31;
     const uint4* xr = reinterpret_cast<const uint4*>(x);
-    float ss = 0.f;
-    if (valid) {
+    uint4* dr = reinterpret_cast<uint4*>(dst);
+#pragma unroll 1
+    for (int blk = 0; blk < 2; ++blk) {  // dims [64 blk, 64 blk + 64)
+        uint4 xv[8];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            const uint4 u = __ldg(xr + c);
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        for (int c = 0; c < 8; ++c) xv[c] = valid ? __ldg(xr + 8 * blk + c) : make_uint4(0u, 0u, 0u, 0u);
+        float dy[64];
+        tmem_ld32f(taddr + 64 * blk, dy);
+        tmem_ld32f(taddr + 64 * blk + 32, dy + 32);
+        tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 t = unpack_bf16(w[e]);
-                ss = fmaf(t.x, t.x, fmaf(t.y, t.y, ss));
+        for (int e = 0; e < 64; ++e) dy[e] *= f;
+        if (blk == 0) {
+            // transpose of the rotation of pairs (t, t + 21)
+#pragma unroll
+            for (int t = 0; t < TF_HALF; ++t) {
+                float c, s;
+                rope_cs(L.theta[t], pos, c, s);
+                const float d1 = dy[t], d2 = dy[t + TF_HALF];
+                dy[t] = d1 * c + d2 * s;
+                dy[t + TF_HALF] = d2 * c - d1 * s;
+            }
+        }
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float* v = dy + 32 * half;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint4 u = xv[4 * half + c];
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                uint32_t o[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 t = unpack_bf16(w[e]);
+                    const int d = 8 * c + 2 * e, gd = 64 * blk + 32 * half + d;
+                    const float x0 = t.x * rinv, x1 = t.y * rinv;
+                    o[e] = pack_bf16((v[d] * gamma[gd] - x0 * mdot) * rinv, (v[d + 1] * gamma[gd + 1] - x1 * mdot) * rinv);
+                    v[d] *= x0;
+                    v[d + 1] *= x1;
+                }
+                if (valid) dr[8 * blk + 4 * half + c] = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+            const float tot = warp_transpose_sum(v);
+            dgam[64 * blk + 32 * half + lane] += tot;
+        }
+    }
+}
+
+// visibility of key j to query i: the causal window max(0, i-W+1) <= j <= i inside the
+// sequence (always true for a chunk known to be fully visible)
+template <bool FULL>
+__device__ __forceinline__ bool visible(int i, int j, const LayerParams& L) {
+    return FULL || (j <= i && j > i - L.W && j >= 0 && j < L.S);
+}
+
+// Query-major statistics over one 32-key chunk of a row: l += 2^(s c2 - mu),
+// num += 2^(s c2 - mu) dP, mxdp = max |dP|, with dP = dv * dai * vin (dA row and V row scales
+// undone).
+template <bool FULL>
+__device__ __forceinline__ void q_stats_chunk(const float* sv, const float* dv, const float* vin, float dai,
+                                              float c2, float mu, int i, int kp0, const LayerParams& L,
+                                              float& l, float& num, float& mxdp) {
+#pragma unroll
+    for (int e4 = 0; e4 < 8; ++e4) {
+        const float4 vi = *reinterpret_cast<const float4*>(vin + 4 * e4);
+        const float vv[4] = {vi.x, vi.y, vi.z, vi.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = 4 * e4 + u;
+            if (visible<FULL>(i, kp0 + e, L)) {
+                const float ev = fast_exp2(fmaf(sv[e], c2, -mu));
+                const float dp = dv[e] * dai * vv[u];
+                l += ev;
+                num = fmaf(ev, dp, num);
+                mxdp = fmaxf(mxdp, fabsf(dp));
             }
         }
     }
-    const float rinv = ss > 0.f ? rsqrtf(ss * (1.0f / kD) + L.eps) : 0.f;
-    float mdot = 0.f;
-    // two passes: (A) mean of dy*gamma*xhat and d_gamma, (B) dx
-#pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {
-#pragma unroll 1
-        for (int blk = 0; blk < 2; ++blk) {  // dims [64 blk, 64 blk + 64)
-            float dy[64];
-            {
-                uint32_t a[32], b2[32];
-                tmem_ld32(taddr + 64 * blk, a);
-                tmem_ld32(taddr + 64 * blk + 32, b2);
-                tmem_wait_ld();
+}
+
+// Query-major dS over one 32-key chunk: dS = P (dP - Delta) * dsc packed to fp16 pairs, and
+// macc += dS S (unscaled dS; the RMSNorm backward's row term).
+template <bool FULL>
+__device__ __forceinline__ void q_ds_chunk(const float* sv, const float* dv, const float* vin, float dai,
+                                           float c2, float lse2, float delta, float dsc, int i, int kp0,
+                                           const LayerParams& L, uint32_t (&pk)[16], float& macc) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    dy[e] = __uint_as_float(a[e]) * f;
-                    dy[32 + e] = __uint_as_float(b2[e]) * f;
-                }
-            }
-            if (blk == 0) {
-                // transpose of the rotation of pairs (t, t + 21)
+    for (int e4 = 0; e4 < 8; ++e4) {
+        const float4 vi = *reinterpret_cast<const float4*>(vin + 4 * e4);
+        const float vv[4] = {vi.x, vi.y, vi.z, vi.w};
+        float ds[4];
 #pragma unroll
-                for (int t = 0; t < TF_HALF; ++t) {
-                    float c, s;
-                    rope_cs(L.theta[t], pos, c, s);
-                    const float d1 = dy[t], d2 = dy[t + TF_HALF];
-                    dy[t] = d1 * c + d2 * s;
-                    dy[t + TF_HALF] = d2 * c - d1 * s;
-                }
-            }
-            if (pass == 0) {
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float v[32];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint4 u = make_uint4(0u, 0u, 0u, 0u);
-                        if (valid) u = __ldg(xr + 8 * blk + 4 * half + c);
-                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 t = unpack_bf16(w[e]);
-                            const int d = 32 * half + 8 * c + 2 * e;
-                            const float x0 = t.x * rinv, x1 = t.y * rinv;
-                            mdot = fmaf(dy[d] * gamma[64 * blk + d], x0, mdot);
-                            mdot = fmaf(dy[d + 1] * gamma[64 * blk + d + 1], x1, mdot);
-                            v[8 * c + 2 * e] = valid ? dy[d] * x0 : 0.f;
-                            v[8 * c + 2 * e + 1] = valid ? dy[d + 1] * x1 : 0.f;
-                        }
-                    }
-                    const float tot = warp_transpose_sum(v);
-                    dgam[64 * blk + 32 * half + lane] += tot;
-                }
-            } else if (valid) {
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 u = __ldg(xr + 8 * blk + c);
-                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-                    uint32_t o[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 t = unpack_bf16(w[e]);
-                        const int d = 8 * c + 2 * e;
-                        const float a0 = (dy[d] * gamma[64 * blk + d] - t.x * rinv * mdot) * rinv;
-                        const float a1 = (dy[d + 1] * gamma[64 * blk + d + 1] - t.y * rinv * mdot) * rinv;
-                        o[e] = pack_bf16(a0, a1);
-                    }
-                    reinterpret_cast<uint4*>(dst)[8 * blk + c] = make_uint4(o[0], o[1], o[2], o[3]);
-                }
-            }
+        for (int u = 0; u < 4; ++u) {
+            const int e = 4 * e4 + u;
+            const float pv = visible<FULL>(i, kp0 + e, L) ? fast_exp2(fmaf(sv[e], c2, -lse2)) : 0.f;
+            const float dp = dv[e] * dai * vv[u];
+            const float d = pv * (dp - delta);
+            macc = fmaf(d, sv[e], macc);
+            ds[u] = d * dsc;
         }
-        if (pass == 0) mdot *= (1.0f / kD);
+        pk[2 * e4] = pack2<true>(ds[0], ds[1]);
+        pk[2 * e4 + 1] = pack2<true>(ds[2], ds[3]);
+    }
+}
+
+// Key-major chunk: one key row j against 32 query columns i0.. (S^T, dP^T from TMEM; per
+// column lse, Delta and dA row scale 2^-e_i from shared memory):
+//   P^T = 2^(s c2 - lse) (visible pairs), dP^T = dv * vin * 2^-e_i,
+//   P^T for dV carries 2^(E - e_i) (su = 2^E), dS^T = P^T (dP^T - Delta) * dsc,
+//   kacc += dS^T S^T (unscaled dS^T; dk's RMSNorm row term).
+template <bool FULL>
+__device__ __forceinline__ void kv_chunk(const float* sv, const float* dv, const float* lse2c, const float* deltac,
+                                         const float* dcolc, float vin, float su, float dsc, float c2, int j, int i0,
+                                         const LayerParams& L, uint32_t (&pp)[16], uint32_t (&dd)[16], float& kacc) {
+#pragma unroll
+    for (int e4 = 0; e4 < 8; ++e4) {
+        const float4 ls = *reinterpret_cast<const float4*>(lse2c + 4 * e4);
+        const float4 dl = *reinterpret_cast<const float4*>(deltac + 4 * e4);
+        const float4 dc = *reinterpret_cast<const float4*>(dcolc + 4 * e4);
+        const float lsv[4] = {ls.x, ls.y, ls.z, ls.w}, dlv[4] = {dl.x, dl.y, dl.z, dl.w}, dcv[4] = {dc.x, dc.y, dc.z, dc.w};
+        float p4[4], d4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = 4 * e4 + u, i = i0 + e;
+            const bool vis = FULL || (j <= i && j > i - L.W && i < L.S && j < L.S);
+            const float pv = vis ? fast_exp2(fmaf(sv[e], c2, -lsv[u])) : 0.f;
+            const float dp = dv[e] * vin * dcv[u];
+            const float d = pv * (dp - dlv[u]);
+            kacc = fmaf(d, sv[e], kacc);
+            p4[u] = pv * (dcv[u] * su);
+            d4[u] = d * dsc;
+        }
+        pp[2 * e4] = pack2<true>(p4[0], p4[1]);
+        pp[2 * e4 + 1] = pack2<true>(p4[2], p4[3]);
+        dd[2 * e4] = pack2<true>(d4[0], d4[1]);
+        dd[2 * e4 + 1] = pack2<true>(d4[2], d4[3]);
     }
 }
 
@@ -280,7 +335,8 @@ __device__ __forceinline__ void row_rope_rms_backward(uint32_t taddr, float f, c
 enum QBar {
     QB_KFULL = 0, QB_KREADY = 2, QB_KEMPTY = 4, QB_VFULL = 6, QB_VREADY = 8, QB_VEMPTY = 10,
     QB_QFULL = 12, QB_QREADY = 13, QB_QEMPTY = 14, QB_DAEMPTY = 15,
-    QB_SFULL = 16, QB_DSFULL = 17, QB_DQFULL = 18, QB_DQEMPTY = 19, QB_DONE = 20, QB_DAFULL = 21, QB_COUNT = 22
+    QB_SFULL = 16, QB_DSFULL = 17, QB_DQFULL = 18, QB_DQEMPTY = 19, QB_DONE = 20, QB_DAFULL = 21,
+    QB_DPFULL = 22, QB_COUNT = 23
 };
 
 struct BwdQTcSmem {
@@ -291,7 +347,9 @@ struct BwdQTcSmem {
     float2 cs[TF_HALF][TF_BM];
     float gq[kD], gk[kD];
     float vinv[4][TF_BN];    // 2^-e of each V row, by tile number % 4
-    float dsinv[TF_BM];      // 2^-e of each dS row of the current head
+    float dsinv[2][TF_BM];   // 2^-e of each dS row, by head number % 2
+    float mdot[2][TF_BM];    // mean(dy gamma xhat) of each row (RMSNorm backward), by head % 2
+    float qrinv[4][TF_BM];   // inverse RMS of each raw q row, by head number % 4
     float dgq[4][kD];        // this CTA's d_gamma_q, one slice per epilogue warp
     uint64_t bar[QB_COUNT];
     uint32_t tmem_base;
@@ -357,6 +415,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
         mbar_init(&sm.bar[QB_DAEMPTY], 1);
         mbar_init(&sm.bar[QB_DAFULL], 1);
         mbar_init(&sm.bar[QB_SFULL], 1);
+        mbar_init(&sm.bar[QB_DPFULL], 1);
         mbar_init(&sm.bar[QB_DSFULL], 128);
         mbar_init(&sm.bar[QB_DQFULL], 1);
         mbar_init(&sm.bar[QB_DQEMPTY], 128);
@@ -382,9 +441,15 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t TM_S = tmem, TM_DP = tmem + 256, TM_DS = tmem, TM_DQ = tmem + 128;
+    // TMEM ping-pong over two 256-column halves, by head number m:
+    //   S(m) -> half m%2, dP(m) -> the other half; dS(m) (fp16) over the first 128 columns of
+    //   S(m) and dQ(m) in the last 128.  So S(m+1) can be issued as soon as dQ(m) is, while the
+    //   epilogue still reads dQ(m); only dP(m+1) waits for that epilogue.
+    auto tm_half = [&](int m) -> uint32_t { return tmem + 256u * (uint32_t)(m & 1); };
     const float oscale = qk_fp16_scale(sm.gq, sm.gk);
     const float c2 = L.scale_log2 / (oscale * oscale);
+    // mdot = scale / (D oscale^2) * sum_j dS_ij S_ij  (S as accumulated in TMEM)
+    const float mdot_f = c2 * kLn2 / (float)kD;
 
     if (warp == 0) {
         // ================================================ K / V producer
@@ -462,38 +527,44 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                 ok = ok && mbar_wait(&sm.bar[QB_KREADY + (n_cur & 1)], (n_cur >> 1) & 1, abort, 112) &&
                      mbar_wait(&sm.bar[QB_VREADY + (n_cur & 1)], (n_cur >> 1) & 1, abort, 113);
                 for (int h = 0; h < G && ok; ++h, ++m) {
+                    const uint32_t tA = tm_half(m), tB = tm_half(m + 1);
                     if (!(ok = mbar_wait(&sm.bar[QB_QREADY], m & 1, abort, 114))) break;
+                    tc_fence_after();
+                    // S = Q~ K~^T -> tA  (its columns were last read by the softmax of head m-1,
+                    // as dP, and by the epilogue of head m-2, both waited for already)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t half = kk >> 2, within = (kk & 3) * 32;
+                        const uint64_t aq = sdesc_sw128(q_base + half * TF_HALF_BYTES + within, 16, 1024);
+                        const uint64_t bk = sdesc_sw128(k_base + half * TF_RING_HALF + within, 16, 1024);
+                        mma_ss(tA, aq, bk, IDESC_N256, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&sm.bar[QB_QEMPTY]);
+                    mma_commit(&sm.bar[QB_SFULL]);
+                    // dP = dA V^T -> tB, once the epilogue of head m-1 has read dQ(m-1) there
                     if (!(ok = mbar_wait(&sm.bar[QB_DAFULL], m & 1, abort, 118))) break;
                     if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_DQEMPTY], (m - 1) & 1, abort, 115))) break;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t half = kk >> 2, within = (kk & 3) * 32;
-                        const uint64_t aq = sdesc_sw128(q_base + half * TF_HALF_BYTES + within, 16, 1024);
-                        const uint64_t bk = sdesc_sw128(k_base + half * TF_RING_HALF + within, 16, 1024);
-                        mma_ss(TM_S, aq, bk, IDESC_N256, kk > 0 ? 1u : 0u);
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t half = kk >> 2, within = (kk & 3) * 32;
                         const uint64_t ad = sdesc_sw128(da_base + half * TF_HALF_BYTES + within, 16, 1024);
                         const uint64_t bv = sdesc_sw128(v_base + half * TF_RING_HALF + within, 16, 1024);
-                        mma_ss(TM_DP, ad, bv, IDESC_N256, kk > 0 ? 1u : 0u);
+                        mma_ss(tB, ad, bv, IDESC_N256, kk > 0 ? 1u : 0u);
                     }
-                    mma_commit(&sm.bar[QB_QEMPTY]);
                     mma_commit(&sm.bar[QB_DAEMPTY]);
-                    mma_commit(&sm.bar[QB_SFULL]);
+                    mma_commit(&sm.bar[QB_DPFULL]);
                     if (h == G - 1) {
                         mma_commit(&sm.bar[QB_VEMPTY + (n_prev & 1)]);
                         if (st.release_cur) mma_commit(&sm.bar[QB_VEMPTY + (n_cur & 1)]);
                     }
                     if (!(ok = mbar_wait(&sm.bar[QB_DSFULL], m & 1, abort, 116))) break;
                     tc_fence_after();
-                    // dQ~ = dS K~ : dS fp16 in TMEM (16 keys = 8 columns per step), K~ MN-major
+                    // dQ~ = dS K~ -> tA + 128 : dS fp16 in tA (16 keys = 8 columns per step), K~ MN-major
 #pragma unroll
                     for (int kk = 0; kk < 16; ++kk) {
                         const uint64_t bk = sdesc_sw128(k_base + kk * 16 * 128, TF_RING_HALF, 1024);
-                        mma_ts(TM_DQ, TM_DS + kk * 8, bk, IDESC_DQ, kk > 0 ? 1u : 0u);
+                        mma_ts(tA + 128, tA + kk * 8, bk, IDESC_DQ, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(&sm.bar[QB_DQFULL]);
                     if (h == G - 1) {
@@ -519,92 +590,93 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             const float* vin0 = sm.vinv[((slot_cur == 0) ? n_cur : n_prev) & 3];
             const float* vin1 = sm.vinv[((slot_cur == 1) ? n_cur : n_prev) & 3];
             const int imin = q0 + 32 * wq, imax = imin + 31;
+            // chunk c8 (32 keys from kp0) against this warp's 32 rows: live = some pair visible,
+            // full = every pair visible (warp-uniform; masks skipped)
+            auto chunk_kp0 = [&](int c8) { return (c8 < 4 ? base0 : base1) + (c8 & 3) * 32; };
+            auto chunk_live = [&](int kp0) {
+                return imin < L.S && kp0 <= imax && kp0 + 31 > imin - L.W && kp0 + 31 >= 0 && kp0 < L.S;
+            };
+            auto chunk_full = [&](int kp0) {
+                return kp0 + 31 <= imin && kp0 > imax - L.W && kp0 >= 0 && kp0 + 31 < L.S;
+            };
             bool stop = false;
             for (int h = 0; h < G; ++h, ++m) {
                 const int hg = st.kvh * G + h;
                 const size_t ro = ((size_t)st.b * L.Hq + hg) * L.S + (i < L.S ? i : 0);
                 const float dai = i < L.S ? p.dainv[ro] : 0.f;  // undoes the dA row scale
+                const uint32_t tS = tm_half(m) + lane_off, tP = tm_half(m + 1) + lane_off;
                 if (!mbar_wait(&sm.bar[QB_SFULL], m & 1, abort, 120)) { stop = true; break; }
                 tc_fence_after();
+                // pass 1 (S only, may overlap the previous head's epilogue): row maximum
                 float mx = -INFINITY;
 #pragma unroll 1
                 for (int c8 = 0; c8 < 8; ++c8) {
-                    const int kp0 = (c8 < 4 ? base0 : base1) + (c8 & 3) * 32;
-                    const bool live = imin < L.S && kp0 <= imax && kp0 + 31 > imin - L.W && kp0 + 31 >= 0 && kp0 < L.S;
-                    if (!live) continue;
-                    uint32_t v[32];
-                    tmem_ld32(TM_S + lane_off + 32 * c8, v);
+                    const int kp0 = chunk_kp0(c8);
+                    if (!chunk_live(kp0)) continue;
+                    float sv[32];
+                    tmem_ld32f(tS + 32 * c8, sv);
                     tmem_wait_ld();
+                    if (chunk_full(kp0)) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int j = kp0 + e;
-                        if (j <= i && j > i - L.W && j >= 0 && j < L.S) mx = fmaxf(mx, __uint_as_float(v[e]));
+                        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, sv[e]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (visible<false>(i, kp0 + e, L)) mx = fmaxf(mx, sv[e]);
                     }
                 }
                 const float mu = (mx == -INFINITY) ? 0.f : mx * c2;
+                if (!mbar_wait(&sm.bar[QB_DPFULL], m & 1, abort, 121)) { stop = true; break; }
+                tc_fence_after();
+                // pass 2: l = sum 2^(s c2 - mu), Delta = sum P dP, max |dP|
                 float l = 0.f, num = 0.f, mxdp = 0.f;
 #pragma unroll 1
                 for (int c8 = 0; c8 < 8; ++c8) {
-                    const int kp0 = (c8 < 4 ? base0 : base1) + (c8 & 3) * 32;
-                    const bool live = imin < L.S && kp0 <= imax && kp0 + 31 > imin - L.W && kp0 + 31 >= 0 && kp0 < L.S;
-                    if (!live) continue;
+                    const int kp0 = chunk_kp0(c8);
+                    if (!chunk_live(kp0)) continue;
                     const float* vin = (c8 < 4 ? vin0 : vin1) + (c8 & 3) * 32;
-                    uint32_t sv[32], dv[32];
-                    tmem_ld32(TM_S + lane_off + 32 * c8, sv);
-                    tmem_ld32(TM_DP + lane_off + 32 * c8, dv);
+                    float sv[32], dv[32];
+                    tmem_ld32f(tS + 32 * c8, sv);
+                    tmem_ld32f(tP + 32 * c8, dv);
                     tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int j = kp0 + e;
-                        if (j <= i && j > i - L.W && j >= 0 && j < L.S) {
-                            const float ev = fast_exp2(__uint_as_float(sv[e]) * c2 - mu);
-                            const float dp = __uint_as_float(dv[e]) * dai * vin[e];
-                            l += ev;
-                            num = fmaf(ev, dp, num);
-                            mxdp = fmaxf(mxdp, fabsf(dp));
-                        }
-                    }
+                    if (chunk_full(kp0))
+                        q_stats_chunk<true>(sv, dv, vin, dai, c2, mu, i, kp0, L, l, num, mxdp);
+                    else
+                        q_stats_chunk<false>(sv, dv, vin, dai, c2, mu, i, kp0, L, l, num, mxdp);
                 }
                 const float lse2 = l > 0.f ? mu + log2f(l) : INFINITY;
                 const float delta = l > 0.f ? num / l : 0.f;
                 const int es = fit_exp(mxdp + fabsf(delta));
                 const float dsc = ldexpf(1.0f, es);
+                // pass 3: dS = P (dP - Delta), row-scaled fp16 over the first 128 columns of S
+                float macc = 0.f;
 #pragma unroll 1
                 for (int c8 = 0; c8 < 8; ++c8) {
-                    const int kp0 = (c8 < 4 ? base0 : base1) + (c8 & 3) * 32;
-                    const bool live = imin < L.S && kp0 <= imax && kp0 + 31 > imin - L.W && kp0 + 31 >= 0 && kp0 < L.S;
+                    const int kp0 = chunk_kp0(c8);
                     uint32_t pk[16];
-                    if (live) {
+                    if (chunk_live(kp0)) {
                         const float* vin = (c8 < 4 ? vin0 : vin1) + (c8 & 3) * 32;
-                        uint32_t sv[32], dv[32];
-                        tmem_ld32(TM_S + lane_off + 32 * c8, sv);
-                        tmem_ld32(TM_DP + lane_off + 32 * c8, dv);
+                        float sv[32], dv[32];
+                        tmem_ld32f(tS + 32 * c8, sv);
+                        tmem_ld32f(tP + 32 * c8, dv);
                         tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            float ds2[2];
-#pragma unroll
-                            for (int u = 0; u < 2; ++u) {
-                                const int j = kp0 + e + u;
-                                const bool vis = j <= i && j > i - L.W && j >= 0 && j < L.S;
-                                const float pv = vis ? fast_exp2(__uint_as_float(sv[e + u]) * c2 - lse2) : 0.f;
-                                const float dp = __uint_as_float(dv[e + u]) * dai * vin[e + u];
-                                ds2[u] = pv * (dp - delta) * dsc;
-                            }
-                            pk[e >> 1] = pack2<true>(ds2[0], ds2[1]);
-                        }
+                        if (chunk_full(kp0))
+                            q_ds_chunk<true>(sv, dv, vin, dai, c2, lse2, delta, dsc, i, kp0, L, pk, macc);
+                        else
+                            q_ds_chunk<false>(sv, dv, vin, dai, c2, lse2, delta, dsc, i, kp0, L, pk, macc);
                     } else {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) pk[e] = 0u;
                     }
-                    tmem_st16(TM_DS + lane_off + 16 * c8, pk);
+                    tmem_st16(tS + 16 * c8, pk);
                 }
                 tmem_wait_st();
                 if (i < L.S) {
                     p.P.lse2[ro] = lse2;
                     p.P.delta[ro] = delta;
                 }
-                sm.dsinv[r] = 1.0f / dsc;
+                sm.dsinv[m & 1][r] = 1.0f / dsc;
+                sm.mdot[m & 1][r] = macc * mdot_f;
                 tc_fence_before();
                 mbar_arrive(&sm.bar[QB_DSFULL]);
             }
@@ -637,7 +709,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             if (!ok) break;
             for (int h = 0; h < G; ++h, ++m) {
                 if (!(ok = mbar_wait(&sm.bar[QB_QFULL], m & 1, abort, 132))) break;
-                tf_prologue_row<true>(sm.Q[0], sm.Q[1], r, sm.gq, L, sm.cs, oscale);
+                sm.qrinv[m & 3][r] = tf_prologue_row<true>(sm.Q[0], sm.Q[1], r, sm.gq, L, sm.cs, oscale);
                 fence_proxy_async_smem();
                 mbar_arrive(&sm.bar[QB_QREADY]);
             }
@@ -655,10 +727,11 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             for (int h = 0; h < G; ++h, ++m) {
                 if (!(ok = mbar_wait(&sm.bar[QB_DQFULL], m & 1, abort, 140))) break;
                 tc_fence_after();
-                const float f = L.scale * sm.dsinv[r] / oscale;
+                const float f = L.scale * sm.dsinv[m & 1][r] / oscale;
                 const int hg = st.kvh * G + h;
                 const size_t off = ((size_t)(st.b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hg) * kD;
-                row_rope_rms_backward(TM_DQ + lane_off, f, L.q + off, p.P.dq + off, valid, i, sm.gq, sm.dgq[wq], L);
+                row_rope_rms_backward(tm_half(m) + 128 + lane_off, f, sm.mdot[m & 1][r], sm.qrinv[m & 3][r], L.q + off,
+                                      p.P.dq + off, valid, i, sm.gq, sm.dgq[wq], L);
                 tc_fence_before();
                 mbar_arrive(&sm.bar[QB_DQEMPTY]);
             }
@@ -696,6 +769,8 @@ struct BwdKTcSmem {
     float vinv[TF_BN];       // 2^-e of each V row of the current unit
     float dsc[2][TF_BN];     // 2^e of each dS^T row, by unit parity
     float uinv[2];           // 2^-E, E = the unit's smallest dA row exponent, by unit parity
+    float kmdot[2][TF_BN];   // mean(dy gamma xhat) of each key row (RMSNorm backward), by unit parity
+    float krinv[2][TF_BN];   // inverse RMS of each raw k row, by unit parity
     float red[2][4];         // per-warp maxima for the unit statistics
     float dgk[4][kD];        // this CTA's d_gamma_k, one slice per epilogue warp
     uint64_t bar[KB_COUNT];
@@ -771,6 +846,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                    TM_DK = tmem + 384;
     const float oscale = qk_fp16_scale(sm.gq, sm.gk);
     const float c2 = L.scale_log2 / (oscale * oscale);
+    const float mdot_f = c2 * kLn2 / (float)kD;  // scale / (D oscale^2)
 
     if (warp == 0) {
         // ================================================ TMA producer: K, V per unit; Q per iteration
@@ -871,6 +947,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             const float vin = sm.vinv[r];        // undoes the V-row scale of dP^T
             const float su = 1.0f / sm.uinv[uu & 1];  // 2^E: P^T columns carry 2^(E - e_i)
             const float dsc = sm.dsc[uu & 1][r];
+            float kacc = 0.f;  // sum over the unit of dS^T S^T (unscaled dS^T): dk's RMSNorm row term
             for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
                 const int buf = it_all & 1;
                 int qb, hg;
@@ -884,28 +961,20 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 for (int c8 = 0; c8 < 4; ++c8) {
                     const int i0 = q0 + 32 * c8;  // queries of this chunk: i0 .. i0+31
                     const bool live = jmin < L.S && i0 < L.S && i0 + 31 >= jmin && i0 <= jmax + L.W - 1;
+                    const bool full = jmax <= i0 && jmin > i0 + 31 - L.W && i0 + 31 < L.S && jmax < L.S;
                     uint32_t pp[16], dd[16];
                     if (live) {
-                        uint32_t sv[32], dv[32];
-                        tmem_ld32(TM_S + lane_off + 32 * c8, sv);
-                        tmem_ld32(TM_DP + lane_off + 32 * c8, dv);
+                        float sv[32], dv[32];
+                        tmem_ld32f(TM_S + lane_off + 32 * c8, sv);
+                        tmem_ld32f(TM_DP + lane_off + 32 * c8, dv);
                         tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            float pv2[2], ds2[2];
-#pragma unroll
-                            for (int w2 = 0; w2 < 2; ++w2) {
-                                const int ql = 32 * c8 + e + w2, i = q0 + ql;
-                                const bool vis = j <= i && j > i - L.W && i < L.S && j < L.S;
-                                const float pv = vis ? fast_exp2(__uint_as_float(sv[e + w2]) * c2 - sm.lse2[buf][ql]) : 0.f;
-                                const float dcl = sm.dcol[buf][ql];
-                                const float dp = __uint_as_float(dv[e + w2]) * vin * dcl;
-                                pv2[w2] = pv * (dcl * su);
-                                ds2[w2] = pv * (dp - sm.delta[buf][ql]) * dsc;
-                            }
-                            pp[e >> 1] = pack2<true>(pv2[0], pv2[1]);
-                            dd[e >> 1] = pack2<true>(ds2[0], ds2[1]);
-                        }
+                        const int ql0 = 32 * c8;
+                        if (full)
+                            kv_chunk<true>(sv, dv, sm.lse2[buf] + ql0, sm.delta[buf] + ql0, sm.dcol[buf] + ql0, vin, su,
+                                           dsc, c2, j, i0, L, pp, dd, kacc);
+                        else
+                            kv_chunk<false>(sv, dv, sm.lse2[buf] + ql0, sm.delta[buf] + ql0, sm.dcol[buf] + ql0, vin, su,
+                                            dsc, c2, j, i0, L, pp, dd, kacc);
                     } else {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) pp[e] = dd[e] = 0u;
@@ -913,6 +982,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                     tmem_st16(TM_P + lane_off + 16 * c8, pp);
                     tmem_st16(TM_DS + lane_off + 16 * c8, dd);
                 }
+                if (it == x.nit - 1) sm.kmdot[uu & 1][r] = kacc * mdot_f;
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.bar[KB_PFULL]);
@@ -956,7 +1026,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             const int E = fit_exp(domx);
             // K~ (fp16) and V (fp16, row-scaled) of the unit's key tile
             tf_angles(L, x.kt * TF_BN + r, sm.cs, r);
-            tf_prologue_row<true>(sm.K[0], sm.K[1], r, sm.gk, L, sm.cs, oscale);
+            sm.krinv[uu & 1][r] = tf_prologue_row<true>(sm.K[0], sm.K[1], r, sm.gk, L, sm.cs, oscale);
             float vnorm = 0.f;
             sm.vinv[r] = v_row_to_f16(sm.V[0], sm.V[1], r, &vnorm);
             // dS^T row scale: |dS_ji| <= |v_j| |dA_i| + |Delta_i| <= |v_j| sqrt(D) max|dout| + max|Delta|
@@ -1016,7 +1086,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 }
             }
             const float f = L.scale / (sm.dsc[uu & 1][r] * oscale);
-            row_rope_rms_backward(TM_DK + lane_off, f, L.k + off, p.P.dk + off, valid, j, sm.gk, sm.dgk[wq], L);
+            row_rope_rms_backward(TM_DK + lane_off, f, sm.kmdot[uu & 1][r], sm.krinv[uu & 1][r], L.k + off, p.P.dk + off,
+                                  valid, j, sm.gk, sm.dgk[wq], L);
             tc_fence_before();
             mbar_arrive(&sm.bar[KB_DVKEMPTY]);
         }

@@ -49,7 +49,7 @@ __device__ __forceinline__ float fast_tanh(float x) {
 
 // cos/sin of the TF_HALF rotation angles at `pos`, into column r of the table
 __device__ __forceinline__ void tf_angles(const LayerParams& L, int pos, float2 (*cs)[TF_BM], int r) {
-#pragma unroll
+#pragma unroll 1  // rolled: unrolled, the fp64 angle products of all 21 pairs stay live and spill
     for (int t = 0; t < TF_HALF; ++t) {
         float c, s;
         rope_cs(L.theta[t], pos, c, s);
@@ -60,7 +60,8 @@ __device__ __forceinline__ void tf_angles(const LayerParams& L, int pos, float2 
 // Row `r` of a 128-row tile stored as two 16 KB d-halves (h0, h1), 128-byte swizzled:
 // normalise (RMS, gamma), rotate pairs (t, t+21) for t < 21, multiply by `oscale` (a power
 // of two, 1 unless the fp16 range needs it) and write back in place as bf16 (F16 = false)
-// or fp16.  Rows outside the sequence are zero-filled by TMA and stay zero.
+// or fp16.  Rows outside the sequence are zero-filled by TMA and stay zero.  Returns the
+// row's inverse RMS (the backward's epilogue reuses it).
 template <bool F16>
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
     if constexpr (F16) {
@@ -72,7 +73,7 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 }
 
 template <bool F16 = false>
-__device__ __forceinline__ void tf_prologue_row(unsigned char* h0, unsigned char* h1, int r, const float* gamma,
+__device__ __forceinline__ float tf_prologue_row(unsigned char* h0, unsigned char* h1, int r, const float* gamma,
                                                 const LayerParams& L, const float2 (*cs)[TF_BM],
                                                 float oscale = 1.0f) {
     // chunk ch (8 dims, 16 bytes) of the row: half ch / 8, swizzled position (ch % 8) ^ (r % 8)
@@ -93,7 +94,8 @@ __device__ __forceinline__ void tf_prologue_row(unsigned char* h0, unsigned char
         }
     }
     // a zero row (outside the sequence, zero-filled by TMA) stays zero even with eps = 0
-    const float rinv = ss > 0.f ? rsqrtf(ss * (1.0f / kD) + L.eps) * oscale : 0.f;
+    const float rinv1 = ss > 0.f ? rsqrtf(ss * (1.0f / kD) + L.eps) : 0.f;
+    const float rinv = rinv1 * oscale;
     // dims 0..47 (chunks 0..5): normalise, rotate the first 42
     float y[48];
 #pragma unroll
@@ -137,6 +139,7 @@ __device__ __forceinline__ void tf_prologue_row(unsigned char* h0, unsigned char
         }
         *chunk(ch) = make_uint4(w[0], w[1], w[2], w[3]);
     }
+    return rinv1;  // 1 / sqrt(mean x^2 + eps) of the row (0 for a zero row)
 }
 
 
