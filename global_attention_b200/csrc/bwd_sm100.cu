@@ -51,15 +51,6 @@ struct BwdTcParams {
     int total;          // steps (query-major) or units (key-major)
 };
 
-// Power of two that keeps the fp16 q~, k~ in range: |y_d| <= sqrt(D) max|gamma|.  Every
-// CTA of both kernels derives the same value from gamma_q, gamma_k in shared memory.
-__device__ __forceinline__ float qk_fp16_scale(const float* gq, const float* gk) {
-    float gmax = 0.f;
-    for (int d = 0; d < kD; ++d) gmax = fmaxf(gmax, fmaxf(fabsf(gq[d]), fabsf(gk[d])));
-    const float bound = gmax * sqrtf((float)kD);
-    return (bound > 16384.f && isfinite(bound)) ? ldexpf(1.0f, 13 - ilogbf(bound)) : 1.0f;
-}
-
 // power-of-two exponent e with |x| * 2^e in [2^13, 2^14); 0 for x == 0 or non-finite
 __device__ __forceinline__ int fit_exp(float x) {
     if (!(x > 0.f) || !isfinite(x)) return 0;
@@ -177,68 +168,6 @@ __device__ __forceinline__ uint4* tile_chunk(unsigned char* h0, unsigned char* h
     return reinterpret_cast<uint4*>(hb + (uint32_t)r * 128u + (uint32_t)(((ch & 7) ^ (r & 7)) << 4));
 }
 
-// RoPE / RMSNorm backward of one row held by one thread, one pass over the row:
-//   dy = R^T (f * dq~)       (128 fp32 columns of TMEM at `taddr`; R rotates pairs (t, t+21) at `pos`)
-//   dx = (dy * gamma - xhat * mdot) * rinv,   xhat = x * rinv,   d_gamma += dy * xhat
-// The caller supplies rinv = 1/sqrt(mean x^2 + eps) (from the prologue) and
-// mdot = mean_d(dy_d gamma_d xhat_d).  Because R is orthogonal and q~ = R(gamma * xhat),
-// mdot = (q~ . dq~) / D, which the softmax warps form as a row sum of dS * S; so the raw row
-// x (global memory) is read once, here.  d_gamma goes into this warp's slice `dgam` through
-// warp-transposed sums (lane L owns one dimension per 32-wide block: a fixed summation order,
-// reproducible).  `valid` masks rows past the sequence (they still join the collectives).
-__device__ __forceinline__ void row_rope_rms_backward(uint32_t taddr, float f, float mdot, float rinv,
-                                                      const bf16* x, bf16* dst, bool valid, int pos,
-                                                      const float* gamma, float* dgam, const LayerParams& L) {
-    const int lane = threadIdx.x & 31;
-    const uint4* xr = reinterpret_cast<const uint4*>(x);
-    uint4* dr = reinterpret_cast<uint4*>(dst);
-#pragma unroll 1
-    for (int blk = 0; blk < 2; ++blk) {  // dims [64 blk, 64 blk + 64)
-        uint4 xv[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) xv[c] = valid ? __ldg(xr + 8 * blk + c) : make_uint4(0u, 0u, 0u, 0u);
-        float dy[64];
-        tmem_ld32f(taddr + 64 * blk, dy);
-        tmem_ld32f(taddr + 64 * blk + 32, dy + 32);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 64; ++e) dy[e] *= f;
-        if (blk == 0) {
-            // transpose of the rotation of pairs (t, t + 21)
-#pragma unroll
-            for (int t = 0; t < TF_HALF; ++t) {
-                float c, s;
-                rope_cs(L.theta[t], pos, c, s);
-                const float d1 = dy[t], d2 = dy[t + TF_HALF];
-                dy[t] = d1 * c + d2 * s;
-                dy[t + TF_HALF] = d2 * c - d1 * s;
-            }
-        }
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float* v = dy + 32 * half;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint4 u = xv[4 * half + c];
-                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-                uint32_t o[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 t = unpack_bf16(w[e]);
-                    const int d = 8 * c + 2 * e, gd = 64 * blk + 32 * half + d;
-                    const float x0 = t.x * rinv, x1 = t.y * rinv;
-                    o[e] = pack_bf16((v[d] * gamma[gd] - x0 * mdot) * rinv, (v[d + 1] * gamma[gd + 1] - x1 * mdot) * rinv);
-                    v[d] *= x0;
-                    v[d + 1] *= x1;
-                }
-                if (valid) dr[8 * blk + 4 * half + c] = make_uint4(o[0], o[1], o[2], o[3]);
-            }
-            const float tot = warp_transpose_sum(v);
-            dgam[64 * blk + 32 * half + lane] += tot;
-        }
-    }
-}
-
 // visibility of key j to query i: the causal window max(0, i-W+1) <= j <= i inside the
 // sequence (always true for a chunk known to be fully visible)
 template <bool FULL>
@@ -246,53 +175,25 @@ __device__ __forceinline__ bool visible(int i, int j, const LayerParams& L) {
     return FULL || (j <= i && j > i - L.W && j >= 0 && j < L.S);
 }
 
-// Query-major statistics over one 32-key chunk of a row: l += 2^(s c2 - mu),
-// num += 2^(s c2 - mu) dP, mxdp = max |dP|, with dP = dv * dai * vin (dA row and V row scales
-// undone).
+// Query-major pass over one 32-key chunk of a row (S, dP as accumulated in TMEM):
+//   P = 2^(s c2 - lse2) on visible pairs (0 elsewhere),  P dP with dP = dv * kd (kd undoes
+//   the dA row and V tile scales);  num += P dP,  mpd = max |P dP|,  sa += P dP s,  sb += P s.
+// P and P dP replace s and dv in place (the caller writes them back to TMEM).
 template <bool FULL>
-__device__ __forceinline__ void q_stats_chunk(const float* sv, const float* dv, const float* vin, float dai,
-                                              float c2, float mu, int i, int kp0, const LayerParams& L,
-                                              float& l, float& num, float& mxdp) {
+__device__ __forceinline__ void q_pass1_chunk(float (&sv)[32], float (&dv)[32], float kd, float c2, float lse2, int i,
+                                              int kp0, const LayerParams& L, float& num, float& mpd, float& sa,
+                                              float& sb) {
 #pragma unroll
-    for (int e4 = 0; e4 < 8; ++e4) {
-        const float4 vi = *reinterpret_cast<const float4*>(vin + 4 * e4);
-        const float vv[4] = {vi.x, vi.y, vi.z, vi.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = 4 * e4 + u;
-            if (visible<FULL>(i, kp0 + e, L)) {
-                const float ev = fast_exp2(fmaf(sv[e], c2, -mu));
-                const float dp = dv[e] * dai * vv[u];
-                l += ev;
-                num = fmaf(ev, dp, num);
-                mxdp = fmaxf(mxdp, fabsf(dp));
-            }
-        }
-    }
-}
-
-// Query-major dS over one 32-key chunk: dS = P (dP - Delta) * dsc packed to fp16 pairs, and
-// macc += dS S (unscaled dS; the RMSNorm backward's row term).
-template <bool FULL>
-__device__ __forceinline__ void q_ds_chunk(const float* sv, const float* dv, const float* vin, float dai,
-                                           float c2, float lse2, float delta, float dsc, int i, int kp0,
-                                           const LayerParams& L, uint32_t (&pk)[16], float& macc) {
-#pragma unroll
-    for (int e4 = 0; e4 < 8; ++e4) {
-        const float4 vi = *reinterpret_cast<const float4*>(vin + 4 * e4);
-        const float vv[4] = {vi.x, vi.y, vi.z, vi.w};
-        float ds[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = 4 * e4 + u;
-            const float pv = visible<FULL>(i, kp0 + e, L) ? fast_exp2(fmaf(sv[e], c2, -lse2)) : 0.f;
-            const float dp = dv[e] * dai * vv[u];
-            const float d = pv * (dp - delta);
-            macc = fmaf(d, sv[e], macc);
-            ds[u] = d * dsc;
-        }
-        pk[2 * e4] = pack2<true>(ds[0], ds[1]);
-        pk[2 * e4 + 1] = pack2<true>(ds[2], ds[3]);
+    for (int e = 0; e < 32; ++e) {
+        const float s = sv[e];
+        const float pv = visible<FULL>(i, kp0 + e, L) ? fast_exp2(fmaf(s, c2, -lse2)) : 0.f;
+        const float pd = pv * (dv[e] * kd);
+        num += pd;
+        mpd = fmaxf(mpd, fabsf(pd));
+        sa = fmaf(pd, s, sa);
+        sb = fmaf(pv, s, sb);
+        sv[e] = pv;
+        dv[e] = pd;
     }
 }
 
@@ -330,12 +231,69 @@ __device__ __forceinline__ void kv_chunk(const float* sv, const float* dv, const
     }
 }
 
+// RoPE / RMSNorm backward of one row held by one thread, one pass over the row:
+//   dy = R^T (f * dq~)       (dq~: the row's 128 accumulator columns, copied out of TMEM
+//                             into registers so that the tensor memory is released first;
+//                             R rotates pairs (t, t+21) at `pos`)
+//   dx = (dy * gamma - xhat * mdot) * rinv,   xhat = x * rinv,   d_gamma += dy * xhat
+// The caller supplies rinv = 1/sqrt(mean x^2 + eps) (from the prologue) and
+// mdot = mean_d(dy_d gamma_d xhat_d).  Because R is orthogonal and q~ = R(gamma * xhat),
+// mdot = (q~ . dq~) / D, which the softmax warps form as a row sum of dS * S; so the raw row
+// x (global memory) is read once: its first 64 values prefetched by the caller (xv0), the
+// last 64 here.  d_gamma goes into this warp's slice `dgam` through warp-transposed sums
+// (lane L owns one dimension per 32-wide block: a fixed summation order, reproducible).
+// `valid` masks rows past the sequence (they still join the collectives).
+__device__ __forceinline__ void row_rope_rms_backward_regs(float (&dy)[128], float f, float mdot, float rinv,
+                                                           const uint4 (&xv0)[8], const bf16* x, bf16* dst,
+                                                           bool valid, int pos, const float* gamma, float* dgam,
+                                                           const LayerParams& L) {
+    const int lane = threadIdx.x & 31;
+    const uint4* xr = reinterpret_cast<const uint4*>(x);
+    uint4* dr = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int e = 0; e < 128; ++e) dy[e] *= f;
+    // transpose of the rotation of pairs (t, t + 21)
+#pragma unroll
+    for (int t = 0; t < TF_HALF; ++t) {
+        float c, s;
+        rope_cs(L.theta[t], pos, c, s);
+        const float d1 = dy[t], d2 = dy[t + TF_HALF];
+        dy[t] = d1 * c + d2 * s;
+        dy[t + TF_HALF] = d2 * c - d1 * s;
+    }
+    uint4 xv1[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) xv1[c] = valid ? __ldg(xr + 8 + c) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // dims [32 q, 32 q + 32)
+        float* v = dy + 32 * q;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint4 u = q < 2 ? xv0[4 * q + c] : xv1[4 * (q - 2) + c];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 t = unpack_bf16(w[e]);
+                const int d = 8 * c + 2 * e, gd = 32 * q + d;
+                const float x0 = t.x * rinv, x1 = t.y * rinv;
+                o[e] = pack_bf16((v[d] * gamma[gd] - x0 * mdot) * rinv, (v[d + 1] * gamma[gd + 1] - x1 * mdot) * rinv);
+                v[d] *= x0;
+                v[d + 1] *= x1;
+            }
+            if (valid) dr[4 * q + c] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        const float tot = warp_transpose_sum(v);
+        dgam[32 * q + lane] += tot;
+    }
+}
+
 // =====================================================================  query-major kernel
 
 enum QBar {
     QB_KFULL = 0, QB_KREADY = 2, QB_KEMPTY = 4, QB_VFULL = 6, QB_VREADY = 8, QB_VEMPTY = 10,
     QB_QFULL = 12, QB_QREADY = 13, QB_QEMPTY = 14, QB_DAEMPTY = 15,
-    QB_SFULL = 16, QB_DSFULL = 17, QB_DQFULL = 18, QB_DQEMPTY = 19, QB_DONE = 20, QB_DAFULL = 21,
+    QB_DSFULL = 17, QB_DQFULL = 18, QB_DQEMPTY = 19, QB_DONE = 20, QB_DAFULL = 21,
     QB_DPFULL = 22, QB_COUNT = 23
 };
 
@@ -346,7 +304,8 @@ struct BwdQTcSmem {
     alignas(1024) unsigned char dA[2][TF_HALF_BYTES];  // dA fp16, row-scaled (TMA from the gate pass)
     float2 cs[TF_HALF][TF_BM];
     float gq[kD], gk[kD];
-    float vinv[4][TF_BN];    // 2^-e of each V row, by tile number % 4
+    float vtinv[4];          // 2^-e of each V tile, by tile number % 4
+    float vred[2][4];        // scratch of the V tile maximum, by tile number % 2
     float dsinv[2][TF_BM];   // 2^-e of each dS row, by head number % 2
     float mdot[2][TF_BM];    // mean(dy gamma xhat) of each row (RMSNorm backward), by head % 2
     float qrinv[4][TF_BM];   // inverse RMS of each raw q row, by head number % 4
@@ -356,9 +315,15 @@ struct BwdQTcSmem {
     int abort;
 };
 
-// In-place fp16 conversion of row r of a raw bf16 V tile, scaled so max|v| lands in
-// [2^13, 2^14); returns 2^-e (and the row's 2-norm in *norm if wanted).
-__device__ __forceinline__ float v_row_to_f16(unsigned char* h0, unsigned char* h1, int r, float* norm) {
+// In-place fp16 conversion of a raw bf16 V tile by its 128 owner threads (thread r = row r;
+// the four warps of one warpgroup, named barrier 1), with one power-of-two scale for the whole
+// tile: the tile's max|v| lands in [2^13, 2^14).  (fp16 keeps its relative precision down to
+// 2^-14, so one scale per tile loses nothing against one per row for any realistic spread of
+// row magnitudes, and it makes the dP scale per tile instead of per key.)  Both backward
+// kernels convert the same 128-row tiles the same way, so their fp16 V agree bit for bit.
+// `red`: 4 floats of shared scratch; the caller alternates two so that the next tile does not
+// overwrite values still being read.  Returns 2^-e; the row's 2-norm in *norm if wanted.
+__device__ __forceinline__ float v_tile_to_f16(unsigned char* h0, unsigned char* h1, int r, float* red, float* norm) {
     float mx = 0.f, ss = 0.f;
 #pragma unroll
     for (int ch = 0; ch < 16; ++ch) {
@@ -371,6 +336,11 @@ __device__ __forceinline__ float v_row_to_f16(unsigned char* h0, unsigned char* 
             ss = fmaf(t.x, t.x, fmaf(t.y, t.y, ss));
         }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) red[(r >> 5) & 3] = mx;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
     const int e = fit_exp(mx);
     const float sc = ldexpf(1.0f, e);
 #pragma unroll
@@ -414,7 +384,6 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
         mbar_init(&sm.bar[QB_QEMPTY], 1);
         mbar_init(&sm.bar[QB_DAEMPTY], 1);
         mbar_init(&sm.bar[QB_DAFULL], 1);
-        mbar_init(&sm.bar[QB_SFULL], 1);
         mbar_init(&sm.bar[QB_DPFULL], 1);
         mbar_init(&sm.bar[QB_DSFULL], 128);
         mbar_init(&sm.bar[QB_DQFULL], 1);
@@ -451,133 +420,138 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
     // mdot = scale / (D oscale^2) * sum_j dS_ij S_ij  (S as accumulated in TMEM)
     const float mdot_f = c2 * kLn2 / (float)kD;
 
-    if (warp == 0) {
-        // ================================================ K / V producer
-        if (lane == 0) {
-            int n_next = 0;
-            int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
-            auto load_tile = [&](int n, int b, int kvh, int kt) -> bool {
-                const int slot = n & 1;
-                if (n >= 2 && !mbar_wait(&sm.bar[QB_KEMPTY + slot], ((n >> 1) - 1) & 1, abort, 101)) return false;
-                mbar_expect_tx(&sm.bar[QB_KFULL + slot], TF_TILE_BYTES);
-                tma_load_4d(sm.K[0] + slot * TF_HALF_BYTES, &p.tm_k, &sm.bar[QB_KFULL + slot], 0, kvh, kt * TF_BN, b);
-                tma_load_4d(sm.K[1] + slot * TF_HALF_BYTES, &p.tm_k, &sm.bar[QB_KFULL + slot], 64, kvh, kt * TF_BN, b);
-                last_k[slot] = n;
-                if (n >= 2 && !mbar_wait(&sm.bar[QB_VEMPTY + slot], ((n >> 1) - 1) & 1, abort, 102)) return false;
-                mbar_expect_tx(&sm.bar[QB_VFULL + slot], TF_TILE_BYTES);
-                tma_load_4d(sm.V[0] + slot * TF_HALF_BYTES, &p.tm_v, &sm.bar[QB_VFULL + slot], 0, kvh, kt * TF_BN, b);
-                tma_load_4d(sm.V[1] + slot * TF_HALF_BYTES, &p.tm_v, &sm.bar[QB_VFULL + slot], 64, kvh, kt * TF_BN, b);
-                last_v[slot] = n;
-                return true;
-            };
-            for (int t = t_begin; t < t_end && !*abort; ++t) {
-                const StepInfo st = decode_step(L, t, t_begin, t_end);
-                if (st.fresh && !load_tile(n_next++, st.b, st.kvh, st.qb - 1)) break;
-                if (!load_tile(n_next++, st.b, st.kvh, st.qb)) break;
-            }
-            for (int slot = 0; slot < 2; ++slot) {
-                if (last_k[slot] >= 0) mbar_wait_drain(&sm.bar[QB_KFULL + slot], (last_k[slot] >> 1) & 1);
-                if (last_v[slot] >= 0) mbar_wait_drain(&sm.bar[QB_VFULL + slot], (last_v[slot] >> 1) & 1);
-            }
-        }
-    } else if (warp == 2) {
-        // ================================================ Q and dA producer (single buffers)
-        if (lane == 0) {
-            int m = 0, last = -1, last_da = -1;
-            bool ok = true;
-            for (int t = t_begin; t < t_end && ok && !*abort; ++t) {
-                const StepInfo st = decode_step(L, t, t_begin, t_end);
-                for (int h = 0; h < G; ++h, ++m) {
-                    const int hg = st.kvh * G + h;
-                    if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_QEMPTY], (m - 1) & 1, abort, 103))) break;
-                    mbar_expect_tx(&sm.bar[QB_QFULL], TF_TILE_BYTES);
-                    tma_load_4d(sm.Q[0], &p.tm_q, &sm.bar[QB_QFULL], 0, hg, st.qb * TF_BM, st.b);
-                    tma_load_4d(sm.Q[1], &p.tm_q, &sm.bar[QB_QFULL], 64, hg, st.qb * TF_BM, st.b);
-                    last = m;
-                    if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_DAEMPTY], (m - 1) & 1, abort, 104))) break;
-                    mbar_expect_tx(&sm.bar[QB_DAFULL], TF_TILE_BYTES);
-                    tma_load_4d(sm.dA[0], &p.tm_da, &sm.bar[QB_DAFULL], 0, hg, st.qb * TF_BM, st.b);
-                    tma_load_4d(sm.dA[1], &p.tm_da, &sm.bar[QB_DAFULL], 64, hg, st.qb * TF_BM, st.b);
-                    last_da = m;
+    // Registers by warpgroup (4 x 128 in all, set at the top of each role): TMA / MMA issue
+    // 48, softmax 128, prologue 128, epilogue 208 (it holds a whole dq~ row so that it can
+    // release TMEM before its arithmetic).
+    if (warp < 4) {
+        reg_dealloc<48>();
+        if (warp == 0) {
+            // ================================================ K / V producer
+            if (lane == 0) {
+                int n_next = 0;
+                int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
+                auto load_tile = [&](int n, int b, int kvh, int kt) -> bool {
+                    const int slot = n & 1;
+                    if (n >= 2 && !mbar_wait(&sm.bar[QB_KEMPTY + slot], ((n >> 1) - 1) & 1, abort, 101)) return false;
+                    mbar_expect_tx(&sm.bar[QB_KFULL + slot], TF_TILE_BYTES);
+                    tma_load_4d(sm.K[0] + slot * TF_HALF_BYTES, &p.tm_k, &sm.bar[QB_KFULL + slot], 0, kvh, kt * TF_BN, b);
+                    tma_load_4d(sm.K[1] + slot * TF_HALF_BYTES, &p.tm_k, &sm.bar[QB_KFULL + slot], 64, kvh, kt * TF_BN, b);
+                    last_k[slot] = n;
+                    if (n >= 2 && !mbar_wait(&sm.bar[QB_VEMPTY + slot], ((n >> 1) - 1) & 1, abort, 102)) return false;
+                    mbar_expect_tx(&sm.bar[QB_VFULL + slot], TF_TILE_BYTES);
+                    tma_load_4d(sm.V[0] + slot * TF_HALF_BYTES, &p.tm_v, &sm.bar[QB_VFULL + slot], 0, kvh, kt * TF_BN, b);
+                    tma_load_4d(sm.V[1] + slot * TF_HALF_BYTES, &p.tm_v, &sm.bar[QB_VFULL + slot], 64, kvh, kt * TF_BN, b);
+                    last_v[slot] = n;
+                    return true;
+                };
+                for (int t = t_begin; t < t_end && !*abort; ++t) {
+                    const StepInfo st = decode_step(L, t, t_begin, t_end);
+                    if (st.fresh && !load_tile(n_next++, st.b, st.kvh, st.qb - 1)) break;
+                    if (!load_tile(n_next++, st.b, st.kvh, st.qb)) break;
+                }
+                for (int slot = 0; slot < 2; ++slot) {
+                    if (last_k[slot] >= 0) mbar_wait_drain(&sm.bar[QB_KFULL + slot], (last_k[slot] >> 1) & 1);
+                    if (last_v[slot] >= 0) mbar_wait_drain(&sm.bar[QB_VFULL + slot], (last_v[slot] >> 1) & 1);
                 }
             }
-            if (last >= 0) mbar_wait_drain(&sm.bar[QB_QFULL], last & 1);
-            if (last_da >= 0) mbar_wait_drain(&sm.bar[QB_DAFULL], last_da & 1);
-        }
-    } else if (warp == 1) {
-        // ================================================ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t IDESC_N256 = idesc_f16(128, 256, false);
-            constexpr uint32_t IDESC_DQ = idesc_f16(128, 128, true);
-            const uint32_t q_base = smem_u32(sm.Q[0]), da_base = smem_u32(sm.dA[0]);
-            const uint32_t k_base = smem_u32(sm.K[0]), v_base = smem_u32(sm.V[0]);
-            int n_next = 0, n_prev = 0, n_cur = 0, m = 0;
-            bool ok = true;
-            for (int t = t_begin; t < t_end && ok; ++t) {
-                const StepInfo st = decode_step(L, t, t_begin, t_end);
-                if (st.fresh) {
-                    n_prev = n_next++;
-                    n_cur = n_next++;
-                    ok = mbar_wait(&sm.bar[QB_KREADY + (n_prev & 1)], (n_prev >> 1) & 1, abort, 110) &&
-                         mbar_wait(&sm.bar[QB_VREADY + (n_prev & 1)], (n_prev >> 1) & 1, abort, 111);
-                } else {
-                    n_prev = n_cur;
-                    n_cur = n_next++;
-                }
-                ok = ok && mbar_wait(&sm.bar[QB_KREADY + (n_cur & 1)], (n_cur >> 1) & 1, abort, 112) &&
-                     mbar_wait(&sm.bar[QB_VREADY + (n_cur & 1)], (n_cur >> 1) & 1, abort, 113);
-                for (int h = 0; h < G && ok; ++h, ++m) {
-                    const uint32_t tA = tm_half(m), tB = tm_half(m + 1);
-                    if (!(ok = mbar_wait(&sm.bar[QB_QREADY], m & 1, abort, 114))) break;
-                    tc_fence_after();
-                    // S = Q~ K~^T -> tA  (its columns were last read by the softmax of head m-1,
-                    // as dP, and by the epilogue of head m-2, both waited for already)
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t half = kk >> 2, within = (kk & 3) * 32;
-                        const uint64_t aq = sdesc_sw128(q_base + half * TF_HALF_BYTES + within, 16, 1024);
-                        const uint64_t bk = sdesc_sw128(k_base + half * TF_RING_HALF + within, 16, 1024);
-                        mma_ss(tA, aq, bk, IDESC_N256, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&sm.bar[QB_QEMPTY]);
-                    mma_commit(&sm.bar[QB_SFULL]);
-                    // dP = dA V^T -> tB, once the epilogue of head m-1 has read dQ(m-1) there
-                    if (!(ok = mbar_wait(&sm.bar[QB_DAFULL], m & 1, abort, 118))) break;
-                    if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_DQEMPTY], (m - 1) & 1, abort, 115))) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t half = kk >> 2, within = (kk & 3) * 32;
-                        const uint64_t ad = sdesc_sw128(da_base + half * TF_HALF_BYTES + within, 16, 1024);
-                        const uint64_t bv = sdesc_sw128(v_base + half * TF_RING_HALF + within, 16, 1024);
-                        mma_ss(tB, ad, bv, IDESC_N256, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&sm.bar[QB_DAEMPTY]);
-                    mma_commit(&sm.bar[QB_DPFULL]);
-                    if (h == G - 1) {
-                        mma_commit(&sm.bar[QB_VEMPTY + (n_prev & 1)]);
-                        if (st.release_cur) mma_commit(&sm.bar[QB_VEMPTY + (n_cur & 1)]);
-                    }
-                    if (!(ok = mbar_wait(&sm.bar[QB_DSFULL], m & 1, abort, 116))) break;
-                    tc_fence_after();
-                    // dQ~ = dS K~ -> tA + 128 : dS fp16 in tA (16 keys = 8 columns per step), K~ MN-major
-#pragma unroll
-                    for (int kk = 0; kk < 16; ++kk) {
-                        const uint64_t bk = sdesc_sw128(k_base + kk * 16 * 128, TF_RING_HALF, 1024);
-                        mma_ts(tA + 128, tA + kk * 8, bk, IDESC_DQ, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&sm.bar[QB_DQFULL]);
-                    if (h == G - 1) {
-                        mma_commit(&sm.bar[QB_KEMPTY + (n_prev & 1)]);
-                        if (st.release_cur) mma_commit(&sm.bar[QB_KEMPTY + (n_cur & 1)]);
+        } else if (warp == 2) {
+            // ================================================ Q and dA producer (single buffers)
+            if (lane == 0) {
+                int m = 0, last = -1, last_da = -1;
+                bool ok = true;
+                for (int t = t_begin; t < t_end && ok && !*abort; ++t) {
+                    const StepInfo st = decode_step(L, t, t_begin, t_end);
+                    for (int h = 0; h < G; ++h, ++m) {
+                        const int hg = st.kvh * G + h;
+                        if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_QEMPTY], (m - 1) & 1, abort, 103))) break;
+                        mbar_expect_tx(&sm.bar[QB_QFULL], TF_TILE_BYTES);
+                        tma_load_4d(sm.Q[0], &p.tm_q, &sm.bar[QB_QFULL], 0, hg, st.qb * TF_BM, st.b);
+                        tma_load_4d(sm.Q[1], &p.tm_q, &sm.bar[QB_QFULL], 64, hg, st.qb * TF_BM, st.b);
+                        last = m;
+                        if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_DAEMPTY], (m - 1) & 1, abort, 104))) break;
+                        mbar_expect_tx(&sm.bar[QB_DAFULL], TF_TILE_BYTES);
+                        tma_load_4d(sm.dA[0], &p.tm_da, &sm.bar[QB_DAFULL], 0, hg, st.qb * TF_BM, st.b);
+                        tma_load_4d(sm.dA[1], &p.tm_da, &sm.bar[QB_DAFULL], 64, hg, st.qb * TF_BM, st.b);
+                        last_da = m;
                     }
                 }
+                if (last >= 0) mbar_wait_drain(&sm.bar[QB_QFULL], last & 1);
+                if (last_da >= 0) mbar_wait_drain(&sm.bar[QB_DAFULL], last_da & 1);
             }
-            mma_commit(&sm.bar[QB_DONE]);
-            mbar_wait(&sm.bar[QB_DONE], 0, abort, 117);
+        } else if (warp == 1) {
+            // ================================================ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t IDESC_N256 = idesc_f16(128, 256, false);
+                constexpr uint32_t IDESC_DQ = idesc_f16(128, 128, true);
+                const uint32_t q_base = smem_u32(sm.Q[0]), da_base = smem_u32(sm.dA[0]);
+                const uint32_t k_base = smem_u32(sm.K[0]), v_base = smem_u32(sm.V[0]);
+                int n_next = 0, n_prev = 0, n_cur = 0, m = 0;
+                bool ok = true;
+                for (int t = t_begin; t < t_end && ok; ++t) {
+                    const StepInfo st = decode_step(L, t, t_begin, t_end);
+                    if (st.fresh) {
+                        n_prev = n_next++;
+                        n_cur = n_next++;
+                        ok = mbar_wait(&sm.bar[QB_KREADY + (n_prev & 1)], (n_prev >> 1) & 1, abort, 110) &&
+                             mbar_wait(&sm.bar[QB_VREADY + (n_prev & 1)], (n_prev >> 1) & 1, abort, 111);
+                    } else {
+                        n_prev = n_cur;
+                        n_cur = n_next++;
+                    }
+                    ok = ok && mbar_wait(&sm.bar[QB_KREADY + (n_cur & 1)], (n_cur >> 1) & 1, abort, 112) &&
+                         mbar_wait(&sm.bar[QB_VREADY + (n_cur & 1)], (n_cur >> 1) & 1, abort, 113);
+                    for (int h = 0; h < G && ok; ++h, ++m) {
+                        const uint32_t tA = tm_half(m), tB = tm_half(m + 1);
+                        if (!(ok = mbar_wait(&sm.bar[QB_QREADY], m & 1, abort, 114))) break;
+                        tc_fence_after();
+                        // S = Q~ K~^T -> tA  (its columns were last read by the softmax of head m-1,
+                        // as dP, and by the epilogue of head m-2, both waited for already)
+    #pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t half = kk >> 2, within = (kk & 3) * 32;
+                            const uint64_t aq = sdesc_sw128(q_base + half * TF_HALF_BYTES + within, 16, 1024);
+                            const uint64_t bk = sdesc_sw128(k_base + half * TF_RING_HALF + within, 16, 1024);
+                            mma_ss(tA, aq, bk, IDESC_N256, kk > 0 ? 1u : 0u);
+                        }
+                        mma_commit(&sm.bar[QB_QEMPTY]);
+                        // dP = dA V^T -> tB, once the epilogue of head m-1 has read dQ(m-1) there
+                        if (!(ok = mbar_wait(&sm.bar[QB_DAFULL], m & 1, abort, 118))) break;
+                        if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_DQEMPTY], (m - 1) & 1, abort, 115))) break;
+                        tc_fence_after();
+    #pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t half = kk >> 2, within = (kk & 3) * 32;
+                            const uint64_t ad = sdesc_sw128(da_base + half * TF_HALF_BYTES + within, 16, 1024);
+                            const uint64_t bv = sdesc_sw128(v_base + half * TF_RING_HALF + within, 16, 1024);
+                            mma_ss(tB, ad, bv, IDESC_N256, kk > 0 ? 1u : 0u);
+                        }
+                        mma_commit(&sm.bar[QB_DAEMPTY]);
+                        mma_commit(&sm.bar[QB_DPFULL]);
+                        if (h == G - 1) {
+                            mma_commit(&sm.bar[QB_VEMPTY + (n_prev & 1)]);
+                            if (st.release_cur) mma_commit(&sm.bar[QB_VEMPTY + (n_cur & 1)]);
+                        }
+                        if (!(ok = mbar_wait(&sm.bar[QB_DSFULL], m & 1, abort, 116))) break;
+                        tc_fence_after();
+                        // dQ~ = dS K~ -> tA + 128 : dS fp16 in tA (16 keys = 8 columns per step), K~ MN-major
+    #pragma unroll
+                        for (int kk = 0; kk < 16; ++kk) {
+                            const uint64_t bk = sdesc_sw128(k_base + kk * 16 * 128, TF_RING_HALF, 1024);
+                            mma_ts(tA + 128, tA + kk * 8, bk, IDESC_DQ, kk > 0 ? 1u : 0u);
+                        }
+                        mma_commit(&sm.bar[QB_DQFULL]);
+                        if (h == G - 1) {
+                            mma_commit(&sm.bar[QB_KEMPTY + (n_prev & 1)]);
+                            if (st.release_cur) mma_commit(&sm.bar[QB_KEMPTY + (n_cur & 1)]);
+                        }
+                    }
+                }
+                mma_commit(&sm.bar[QB_DONE]);
+                mbar_wait(&sm.bar[QB_DONE], 0, abort, 117);
+            }
         }
     } else if (warp >= 4 && warp < 8) {
-        // ================================================ lse, Delta, dS (thread = query row)
+        // ================================================ Delta, dS (thread = query row)
         const int r = tid - 128, wq = warp - 4;
         const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
         int n_next = 0, n_prev = 0, n_cur = 0, m = 0;
@@ -587,8 +561,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             const int q0 = st.qb * TF_BM, i = q0 + r;
             const int slot_cur = n_cur & 1;
             const int base0 = (slot_cur == 0 ? q0 : q0 - TF_BN), base1 = (slot_cur == 1 ? q0 : q0 - TF_BN);
-            const float* vin0 = sm.vinv[((slot_cur == 0) ? n_cur : n_prev) & 3];
-            const float* vin1 = sm.vinv[((slot_cur == 1) ? n_cur : n_prev) & 3];
+            const int tile0 = (slot_cur == 0) ? n_cur : n_prev, tile1 = (slot_cur == 1) ? n_cur : n_prev;
             const int imin = q0 + 32 * wq, imax = imin + 31;
             // chunk c8 (32 keys from kp0) against this warp's 32 rows: live = some pair visible,
             // full = every pair visible (warp-uniform; masks skipped)
@@ -603,67 +576,49 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             for (int h = 0; h < G; ++h, ++m) {
                 const int hg = st.kvh * G + h;
                 const size_t ro = ((size_t)st.b * L.Hq + hg) * L.S + (i < L.S ? i : 0);
+                // the forward's log-sum-exp (base 2): its scores are these, bit for bit
+                const float lse2 = i < L.S ? p.P.lse[ro] * kLog2e : INFINITY;
                 const float dai = i < L.S ? p.dainv[ro] : 0.f;  // undoes the dA row scale
                 const uint32_t tS = tm_half(m) + lane_off, tP = tm_half(m + 1) + lane_off;
-                if (!mbar_wait(&sm.bar[QB_SFULL], m & 1, abort, 120)) { stop = true; break; }
-                tc_fence_after();
-                // pass 1 (S only, may overlap the previous head's epilogue): row maximum
-                float mx = -INFINITY;
-#pragma unroll 1
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    const int kp0 = chunk_kp0(c8);
-                    if (!chunk_live(kp0)) continue;
-                    float sv[32];
-                    tmem_ld32f(tS + 32 * c8, sv);
-                    tmem_wait_ld();
-                    if (chunk_full(kp0)) {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, sv[e]);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (visible<false>(i, kp0 + e, L)) mx = fmaxf(mx, sv[e]);
-                    }
-                }
-                const float mu = (mx == -INFINITY) ? 0.f : mx * c2;
                 if (!mbar_wait(&sm.bar[QB_DPFULL], m & 1, abort, 121)) { stop = true; break; }
                 tc_fence_after();
-                // pass 2: l = sum 2^(s c2 - mu), Delta = sum P dP, max |dP|
-                float l = 0.f, num = 0.f, mxdp = 0.f;
+                const float kd0 = dai * sm.vtinv[tile0 & 3], kd1 = dai * sm.vtinv[tile1 & 3];
+                // pass 1: P = 2^(S c2 - lse), P dP (written back over S and dP), Delta = sum P dP,
+                // max |P dP|, and the RMSNorm backward's row sums  a = sum P dP S,  b = sum P S
+                float num = 0.f, mpd = 0.f, sa = 0.f, sb = 0.f;
 #pragma unroll 1
                 for (int c8 = 0; c8 < 8; ++c8) {
                     const int kp0 = chunk_kp0(c8);
                     if (!chunk_live(kp0)) continue;
-                    const float* vin = (c8 < 4 ? vin0 : vin1) + (c8 & 3) * 32;
                     float sv[32], dv[32];
                     tmem_ld32f(tS + 32 * c8, sv);
                     tmem_ld32f(tP + 32 * c8, dv);
                     tmem_wait_ld();
+                    const float kd = c8 < 4 ? kd0 : kd1;
                     if (chunk_full(kp0))
-                        q_stats_chunk<true>(sv, dv, vin, dai, c2, mu, i, kp0, L, l, num, mxdp);
+                        q_pass1_chunk<true>(sv, dv, kd, c2, lse2, i, kp0, L, num, mpd, sa, sb);
                     else
-                        q_stats_chunk<false>(sv, dv, vin, dai, c2, mu, i, kp0, L, l, num, mxdp);
+                        q_pass1_chunk<false>(sv, dv, kd, c2, lse2, i, kp0, L, num, mpd, sa, sb);
+                    tmem_st32f(tS + 32 * c8, sv);
+                    tmem_st32f(tP + 32 * c8, dv);
                 }
-                const float lse2 = l > 0.f ? mu + log2f(l) : INFINITY;
-                const float delta = l > 0.f ? num / l : 0.f;
-                const int es = fit_exp(mxdp + fabsf(delta));
-                const float dsc = ldexpf(1.0f, es);
-                // pass 3: dS = P (dP - Delta), row-scaled fp16 over the first 128 columns of S
-                float macc = 0.f;
+                tmem_wait_st();
+                const float delta = num;
+                // |dS| = |P dP - P Delta| <= max |P dP| + |Delta|
+                const float dsc = ldexpf(1.0f, fit_exp(mpd + fabsf(delta)));
+                // pass 2: dS = (P dP - P Delta) dsc, fp16, over the first 128 columns of S
 #pragma unroll 1
                 for (int c8 = 0; c8 < 8; ++c8) {
                     const int kp0 = chunk_kp0(c8);
                     uint32_t pk[16];
                     if (chunk_live(kp0)) {
-                        const float* vin = (c8 < 4 ? vin0 : vin1) + (c8 & 3) * 32;
-                        float sv[32], dv[32];
-                        tmem_ld32f(tS + 32 * c8, sv);
-                        tmem_ld32f(tP + 32 * c8, dv);
+                        float pv[32], pd[32];
+                        tmem_ld32f(tS + 32 * c8, pv);
+                        tmem_ld32f(tP + 32 * c8, pd);
                         tmem_wait_ld();
-                        if (chunk_full(kp0))
-                            q_ds_chunk<true>(sv, dv, vin, dai, c2, lse2, delta, dsc, i, kp0, L, pk, macc);
-                        else
-                            q_ds_chunk<false>(sv, dv, vin, dai, c2, lse2, delta, dsc, i, kp0, L, pk, macc);
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2)
+                            pk[e >> 1] = pack2<true>(fmaf(-delta, pv[e], pd[e]) * dsc, fmaf(-delta, pv[e + 1], pd[e + 1]) * dsc);
                     } else {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) pk[e] = 0u;
@@ -671,12 +626,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                     tmem_st16(tS + 16 * c8, pk);
                 }
                 tmem_wait_st();
-                if (i < L.S) {
-                    p.P.lse2[ro] = lse2;
-                    p.P.delta[ro] = delta;
-                }
+                if (i < L.S) p.P.delta[ro] = delta;
                 sm.dsinv[m & 1][r] = 1.0f / dsc;
-                sm.mdot[m & 1][r] = macc * mdot_f;
+                sm.mdot[m & 1][r] = fmaf(-delta, sb, sa) * mdot_f;  // sum dS S = a - Delta b
                 tc_fence_before();
                 mbar_arrive(&sm.bar[QB_DSFULL]);
             }
@@ -696,7 +648,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             fence_proxy_async_smem();
             mbar_arrive(&sm.bar[QB_KREADY + slot]);
             if (!mbar_wait(&sm.bar[QB_VFULL + slot], (n >> 1) & 1, abort, 131)) return false;
-            sm.vinv[n & 3][r] = v_row_to_f16(sm.V[0] + slot * TF_HALF_BYTES, sm.V[1] + slot * TF_HALF_BYTES, r, nullptr);
+            const float vt = v_tile_to_f16(sm.V[0] + slot * TF_HALF_BYTES, sm.V[1] + slot * TF_HALF_BYTES, r,
+                                           sm.vred[n & 1], nullptr);
+            if (r == 0) sm.vtinv[n & 3] = vt;
             fence_proxy_async_smem();
             mbar_arrive(&sm.bar[QB_VREADY + slot]);
             return true;
@@ -715,6 +669,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             }
         }
     } else if (warp >= 12) {
+        reg_alloc<208>();
         // ================================================ dq epilogue (thread = query row)
         const int r = tid - 384, wq = warp - 12;
         const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
@@ -725,15 +680,26 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             const int i = st.qb * TF_BM + r;
             const bool valid = i < L.S;
             for (int h = 0; h < G; ++h, ++m) {
-                if (!(ok = mbar_wait(&sm.bar[QB_DQFULL], m & 1, abort, 140))) break;
-                tc_fence_after();
-                const float f = L.scale * sm.dsinv[m & 1][r] / oscale;
                 const int hg = st.kvh * G + h;
                 const size_t off = ((size_t)(st.b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hg) * kD;
-                row_rope_rms_backward(tm_half(m) + 128 + lane_off, f, sm.mdot[m & 1][r], sm.qrinv[m & 3][r], L.q + off,
-                                      p.P.dq + off, valid, i, sm.gq, sm.dgq[wq], L);
+                uint4 xv0[8];  // first half of the raw q row, in flight during the wait
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    xv0[c] = valid ? __ldg(reinterpret_cast<const uint4*>(L.q + off) + c) : make_uint4(0u, 0u, 0u, 0u);
+                if (!(ok = mbar_wait(&sm.bar[QB_DQFULL], m & 1, abort, 140))) break;
+                tc_fence_after();
+                float dy[128];
+                const uint32_t tq = tm_half(m) + 128 + lane_off;
+                tmem_ld32f(tq, dy);
+                tmem_ld32f(tq + 32, dy + 32);
+                tmem_ld32f(tq + 64, dy + 64);
+                tmem_ld32f(tq + 96, dy + 96);
+                tmem_wait_ld();
+                const float f = L.scale * sm.dsinv[m & 1][r] / oscale;
+                const float mdot = sm.mdot[m & 1][r], rinv = sm.qrinv[m & 3][r];
                 tc_fence_before();
-                mbar_arrive(&sm.bar[QB_DQEMPTY]);
+                mbar_arrive(&sm.bar[QB_DQEMPTY]);  // dQ(m) is in registers: TMEM free for dP(m+1)
+                row_rope_rms_backward_regs(dy, f, mdot, rinv, xv0, L.q + off, p.P.dq + off, valid, i, sm.gq, sm.dgq[wq], L);
             }
         }
     }
@@ -766,7 +732,8 @@ struct BwdKTcSmem {
     float lse2[2][TF_BM];    // per query column of the buffer
     float delta[2][TF_BM];
     float dcol[2][TF_BM];    // 2^-e of the dA row of each query column
-    float vinv[TF_BN];       // 2^-e of each V row of the current unit
+    float vtinv[2];          // 2^-e of the unit's V tile, by unit parity
+    float vred[2][4];        // scratch of the V tile maximum, by unit parity
     float dsc[2][TF_BN];     // 2^e of each dS^T row, by unit parity
     float uinv[2];           // 2^-E, E = the unit's smallest dA row exponent, by unit parity
     float kmdot[2][TF_BN];   // mean(dy gamma xhat) of each key row (RMSNorm backward), by unit parity
@@ -848,91 +815,103 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
     const float c2 = L.scale_log2 / (oscale * oscale);
     const float mdot_f = c2 * kLn2 / (float)kD;  // scale / (D oscale^2)
 
-    if (warp == 0) {
-        // ================================================ TMA producer: K, V per unit; Q per iteration
-        if (lane == 0) {
-            int it_all = 0, last_q[2] = {-1, -1}, uu = 0;
-            for (int u = u_begin; u < u_end && !*abort; ++u, ++uu) {
-                const UnitInfo x = decode_unit(L, u);
-                if (uu >= 1 && !mbar_wait(&sm.bar[KB_KVEMPTY], (uu - 1) & 1, abort, 201)) break;
-                mbar_expect_tx(&sm.bar[KB_KVFULL], 2 * TF_TILE_BYTES);
-                tma_load_4d(sm.K[0], &p.tm_k, &sm.bar[KB_KVFULL], 0, x.kvh, x.kt * TF_BN, x.b);
-                tma_load_4d(sm.K[1], &p.tm_k, &sm.bar[KB_KVFULL], 64, x.kvh, x.kt * TF_BN, x.b);
-                tma_load_4d(sm.V[0], &p.tm_v, &sm.bar[KB_KVFULL], 0, x.kvh, x.kt * TF_BN, x.b);
-                tma_load_4d(sm.V[1], &p.tm_v, &sm.bar[KB_KVFULL], 64, x.kvh, x.kt * TF_BN, x.b);
+    // Registers by warpgroup (4 x 128 in all, set at the top of each role): TMA / MMA issue
+    // 48, softmax 128, prologue 128, epilogue 208 (it holds a whole dk~ row so that it can
+    // release TMEM before its arithmetic).
+    if (warp < 4) {
+        reg_dealloc<48>();
+        if (warp == 0) {
+            // ================================================ TMA producer: K, V per unit; Q, dA per iteration
+            if (lane == 0) {
+                int it_all = 0, last_q[2] = {-1, -1}, uu = 0;
+                auto load_kv = [&](const UnitInfo& x) {
+                    mbar_expect_tx(&sm.bar[KB_KVFULL], 2 * TF_TILE_BYTES);
+                    tma_load_4d(sm.K[0], &p.tm_k, &sm.bar[KB_KVFULL], 0, x.kvh, x.kt * TF_BN, x.b);
+                    tma_load_4d(sm.K[1], &p.tm_k, &sm.bar[KB_KVFULL], 64, x.kvh, x.kt * TF_BN, x.b);
+                    tma_load_4d(sm.V[0], &p.tm_v, &sm.bar[KB_KVFULL], 0, x.kvh, x.kt * TF_BN, x.b);
+                    tma_load_4d(sm.V[1], &p.tm_v, &sm.bar[KB_KVFULL], 64, x.kvh, x.kt * TF_BN, x.b);
+                };
                 bool ok = true;
-                for (int it = 0; it < x.nit; ++it, ++it_all) {
-                    const int buf = it_all & 1;
-                    if (it_all >= 2 && !(ok = mbar_wait(&sm.bar[KB_QEMPTY + buf], ((it_all >> 1) - 1) & 1, abort, 202))) break;
-                    int qb, hg;
-                    decode_iter(L, x, it, qb, hg);
-                    mbar_expect_tx(&sm.bar[KB_QFULL + buf], 2 * TF_TILE_BYTES);
-                    tma_load_4d(sm.Q[buf][0], &p.tm_q, &sm.bar[KB_QFULL + buf], 0, hg, qb * TF_BM, x.b);
-                    tma_load_4d(sm.Q[buf][1], &p.tm_q, &sm.bar[KB_QFULL + buf], 64, hg, qb * TF_BM, x.b);
-                    tma_load_4d(sm.dA[buf][0], &p.tm_da, &sm.bar[KB_QFULL + buf], 0, hg, qb * TF_BM, x.b);
-                    tma_load_4d(sm.dA[buf][1], &p.tm_da, &sm.bar[KB_QFULL + buf], 64, hg, qb * TF_BM, x.b);
-                    last_q[buf] = it_all;
+                for (int u = u_begin; u < u_end && ok && !*abort; ++u, ++uu) {
+                    const UnitInfo x = decode_unit(L, u);
+                    for (int it = 0; it < x.nit; ++it, ++it_all) {
+                        const int buf = it_all & 1;
+                        if (it_all >= 2 && !(ok = mbar_wait(&sm.bar[KB_QEMPTY + buf], ((it_all >> 1) - 1) & 1, abort, 202))) break;
+                        int qb, hg;
+                        decode_iter(L, x, it, qb, hg);
+                        mbar_expect_tx(&sm.bar[KB_QFULL + buf], 2 * TF_TILE_BYTES);
+                        tma_load_4d(sm.Q[buf][0], &p.tm_q, &sm.bar[KB_QFULL + buf], 0, hg, qb * TF_BM, x.b);
+                        tma_load_4d(sm.Q[buf][1], &p.tm_q, &sm.bar[KB_QFULL + buf], 64, hg, qb * TF_BM, x.b);
+                        tma_load_4d(sm.dA[buf][0], &p.tm_da, &sm.bar[KB_QFULL + buf], 0, hg, qb * TF_BM, x.b);
+                        tma_load_4d(sm.dA[buf][1], &p.tm_da, &sm.bar[KB_QFULL + buf], 64, hg, qb * TF_BM, x.b);
+                        last_q[buf] = it_all;
+                        if (it == 0) {
+                            // K, V of the unit once the previous unit's products are done; the
+                            // unit's first query tile went out before, as soon as its buffer was free
+                            if (uu >= 1 && !(ok = mbar_wait(&sm.bar[KB_KVEMPTY], (uu - 1) & 1, abort, 201))) break;
+                            load_kv(x);
+                        }
+                    }
                 }
-                if (!ok) break;
+                if (uu >= 1) mbar_wait_drain(&sm.bar[KB_KVFULL], (uu - 1) & 1);
+                for (int buf = 0; buf < 2; ++buf)
+                    if (last_q[buf] >= 0) mbar_wait_drain(&sm.bar[KB_QFULL + buf], (last_q[buf] >> 1) & 1);
             }
-            if (uu >= 1) mbar_wait_drain(&sm.bar[KB_KVFULL], (uu - 1) & 1);
-            for (int buf = 0; buf < 2; ++buf)
-                if (last_q[buf] >= 0) mbar_wait_drain(&sm.bar[KB_QFULL + buf], (last_q[buf] >> 1) & 1);
-        }
-    } else if (warp == 1) {
-        // ================================================ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t IDESC_KM = idesc_f16(128, 128, false);
-            constexpr uint32_t IDESC_MN = idesc_f16(128, 128, true);
-            const uint32_t k_base = smem_u32(sm.K[0]), v_base = smem_u32(sm.V[0]);
-            const uint32_t q_base = smem_u32(sm.Q[0][0]), da_base = smem_u32(sm.dA[0][0]);
-            int it_all = 0, uu = 0;
-            bool ok = true;
-            for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
-                const UnitInfo x = decode_unit(L, u);
-                if (!(ok = mbar_wait(&sm.bar[KB_KVREADY], uu & 1, abort, 210))) break;
-                for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
-                    const int buf = it_all & 1;
-                    const uint32_t qb_addr = q_base + buf * 2 * TF_HALF_BYTES, da_addr = da_base + buf * 2 * TF_HALF_BYTES;
-                    if (!(ok = mbar_wait(&sm.bar[KB_QREADY + buf], (it_all >> 1) & 1, abort, 211))) break;
-                    tc_fence_after();
-                    // S^T = K~ Q~^T, dP^T = V dA^T   (M = keys, N = queries, K = d)
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t half = kk >> 2, within = (kk & 3) * 32;
-                        mma_ss(TM_S, sdesc_sw128(k_base + half * TF_HALF_BYTES + within, 16, 1024),
-                               sdesc_sw128(qb_addr + half * TF_HALF_BYTES + within, 16, 1024), IDESC_KM, kk > 0 ? 1u : 0u);
+        } else if (warp == 1) {
+            // ================================================ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t IDESC_KM = idesc_f16(128, 128, false);
+                constexpr uint32_t IDESC_MN = idesc_f16(128, 128, true);
+                const uint32_t k_base = smem_u32(sm.K[0]), v_base = smem_u32(sm.V[0]);
+                const uint32_t q_base = smem_u32(sm.Q[0][0]), da_base = smem_u32(sm.dA[0][0]);
+                int it_all = 0, uu = 0;
+                bool ok = true;
+                for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
+                    const UnitInfo x = decode_unit(L, u);
+                    if (!(ok = mbar_wait(&sm.bar[KB_KVREADY], uu & 1, abort, 210))) break;
+                    for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
+                        const int buf = it_all & 1;
+                        const uint32_t qb_addr = q_base + buf * 2 * TF_HALF_BYTES, da_addr = da_base + buf * 2 * TF_HALF_BYTES;
+                        if (!(ok = mbar_wait(&sm.bar[KB_QREADY + buf], (it_all >> 1) & 1, abort, 211))) break;
+                        tc_fence_after();
+                        // S^T = K~ Q~^T, dP^T = V dA^T   (M = keys, N = queries, K = d)
+    #pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t half = kk >> 2, within = (kk & 3) * 32;
+                            mma_ss(TM_S, sdesc_sw128(k_base + half * TF_HALF_BYTES + within, 16, 1024),
+                                   sdesc_sw128(qb_addr + half * TF_HALF_BYTES + within, 16, 1024), IDESC_KM, kk > 0 ? 1u : 0u);
+                        }
+    #pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t half = kk >> 2, within = (kk & 3) * 32;
+                            mma_ss(TM_DP, sdesc_sw128(v_base + half * TF_HALF_BYTES + within, 16, 1024),
+                                   sdesc_sw128(da_addr + half * TF_HALF_BYTES + within, 16, 1024), IDESC_KM, kk > 0 ? 1u : 0u);
+                        }
+                        mma_commit(&sm.bar[KB_SFULL]);
+                        if (!(ok = mbar_wait(&sm.bar[KB_PFULL], it_all & 1, abort, 212))) break;
+                        if (it == 0 && uu >= 1 && !(ok = mbar_wait(&sm.bar[KB_DVKEMPTY], (uu - 1) & 1, abort, 213))) break;
+                        tc_fence_after();
+                        // dV += P^T dA ; dK~ += dS^T Q~  (A from TMEM: 16 queries = 8 columns per step;
+                        // B = dA / Q~ MN-major: N = d, K = queries)
+    #pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t bda = sdesc_sw128(da_addr + kk * 16 * 128, TF_HALF_BYTES, 1024);
+                            mma_ts(TM_DV, TM_P + kk * 8, bda, IDESC_MN, (it > 0 || kk > 0) ? 1u : 0u);
+                        }
+    #pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t bq = sdesc_sw128(qb_addr + kk * 16 * 128, TF_HALF_BYTES, 1024);
+                            mma_ts(TM_DK, TM_DS + kk * 8, bq, IDESC_MN, (it > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit(&sm.bar[KB_QEMPTY + buf]);
                     }
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t half = kk >> 2, within = (kk & 3) * 32;
-                        mma_ss(TM_DP, sdesc_sw128(v_base + half * TF_HALF_BYTES + within, 16, 1024),
-                               sdesc_sw128(da_addr + half * TF_HALF_BYTES + within, 16, 1024), IDESC_KM, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&sm.bar[KB_SFULL]);
-                    if (!(ok = mbar_wait(&sm.bar[KB_PFULL], it_all & 1, abort, 212))) break;
-                    if (it == 0 && uu >= 1 && !(ok = mbar_wait(&sm.bar[KB_DVKEMPTY], (uu - 1) & 1, abort, 213))) break;
-                    tc_fence_after();
-                    // dV += P^T dA ; dK~ += dS^T Q~  (A from TMEM: 16 queries = 8 columns per step;
-                    // B = dA / Q~ MN-major: N = d, K = queries)
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t bda = sdesc_sw128(da_addr + kk * 16 * 128, TF_HALF_BYTES, 1024);
-                        mma_ts(TM_DV, TM_P + kk * 8, bda, IDESC_MN, (it > 0 || kk > 0) ? 1u : 0u);
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t bq = sdesc_sw128(qb_addr + kk * 16 * 128, TF_HALF_BYTES, 1024);
-                        mma_ts(TM_DK, TM_DS + kk * 8, bq, IDESC_MN, (it > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    mma_commit(&sm.bar[KB_QEMPTY + buf]);
+                    if (!ok) break;
+                    mma_commit(&sm.bar[KB_DVKFULL]);
+                    mma_commit(&sm.bar[KB_KVEMPTY]);
                 }
-                if (!ok) break;
-                mma_commit(&sm.bar[KB_DVKFULL]);
-                mma_commit(&sm.bar[KB_KVEMPTY]);
+                mma_commit(&sm.bar[KB_DONE]);
+                mbar_wait(&sm.bar[KB_DONE], 0, abort, 214);
             }
-            mma_commit(&sm.bar[KB_DONE]);
-            mbar_wait(&sm.bar[KB_DONE], 0, abort, 214);
         }
     } else if (warp >= 4 && warp < 8) {
         // ================================================ P^T, dS^T (thread = key row)
@@ -944,7 +923,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             const UnitInfo x = decode_unit(L, u);
             const int j = x.kt * TF_BN + r;
             if (!(ok = mbar_wait(&sm.bar[KB_KVREADY], uu & 1, abort, 220))) break;
-            const float vin = sm.vinv[r];        // undoes the V-row scale of dP^T
+            const float vin = sm.vtinv[uu & 1];  // undoes the V tile scale of dP^T
             const float su = 1.0f / sm.uinv[uu & 1];  // 2^E: P^T columns carry 2^(E - e_i)
             const float dsc = sm.dsc[uu & 1][r];
             float kacc = 0.f;  // sum over the unit of dS^T S^T (unscaled dS^T): dk's RMSNorm row term
@@ -989,15 +968,16 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             }
         }
     } else if (warp >= 8 && warp < 12) {
-        // ================================================ prologue: K~, V (per unit), Q~ and dA (per iteration)
+        // ================================================ prologue: K~, V (per unit), Q~ (per iteration)
         const int r = tid - 256, wq = warp - 8;
         int it_all = 0, uu = 0;
         bool ok = true;
         for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
             const UnitInfo x = decode_unit(L, u);
-            if (!(ok = mbar_wait(&sm.bar[KB_KVFULL], uu & 1, abort, 230))) break;
-            // unit statistics: max |dout| and max |Delta| over the rows this unit reads
+            // unit statistics, max |dout| and max |Delta| over the rows this unit reads (global
+            // loads only: issued before any tile wait)
             float domx = 0.f, dlmx = 0.f;
+#pragma unroll 4
             for (int it = 0; it < x.nit; ++it) {
                 int qb, hg;
                 decode_iter(L, x, it, qb, hg);
@@ -1024,17 +1004,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             // E = fit_exp(max domax) is the smallest row exponent of dA in the unit, so every
             // column factor 2^(E - e_i) of P^T is <= 1
             const int E = fit_exp(domx);
-            // K~ (fp16) and V (fp16, row-scaled) of the unit's key tile
+            // angles of the key tile's positions, which are also those of the query block of the
+            // first G iterations (qb = kt)
             tf_angles(L, x.kt * TF_BN + r, sm.cs, r);
-            sm.krinv[uu & 1][r] = tf_prologue_row<true>(sm.K[0], sm.K[1], r, sm.gk, L, sm.cs, oscale);
-            float vnorm = 0.f;
-            sm.vinv[r] = v_row_to_f16(sm.V[0], sm.V[1], r, &vnorm);
-            // dS^T row scale: |dS_ji| <= |v_j| |dA_i| + |Delta_i| <= |v_j| sqrt(D) max|dout| + max|Delta|
-            sm.dsc[uu & 1][r] = ldexpf(1.0f, fit_exp(vnorm * sqrtf((float)kD) * domx + dlmx));
-            if (r == 0) sm.uinv[uu & 1] = ldexpf(1.0f, -E);
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.bar[KB_KVREADY]);
-            int cur_qb = -1;
+            int cur_qb = x.kt;
             for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
                 const int buf = it_all & 1;
                 int qb, hg;
@@ -1048,14 +1021,31 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 }
                 tf_prologue_row<true>(sm.Q[buf][0], sm.Q[buf][1], r, sm.gq, L, sm.cs, oscale);
                 const size_t ro = ((size_t)x.b * L.Hq + hg) * L.S + (valid ? i : 0);
-                sm.lse2[buf][r] = valid ? p.P.lse2[ro] : INFINITY;
+                sm.lse2[buf][r] = valid ? p.P.lse[ro] * kLog2e : INFINITY;  // the forward's, base 2
                 sm.delta[buf][r] = valid ? p.P.delta[ro] : 0.f;
                 sm.dcol[buf][r] = valid ? p.dainv[ro] : 0.f;
                 fence_proxy_async_smem();
                 mbar_arrive(&sm.bar[KB_QREADY + buf]);
+                if (it == 0) {
+                    // K~ (fp16) and V (fp16, row-scaled) of the unit's key tile, after the first
+                    // query tile: that one was loaded during the previous unit, K and V only once
+                    // its products were done
+                    if (!(ok = mbar_wait(&sm.bar[KB_KVFULL], uu & 1, abort, 230))) break;
+                    sm.krinv[uu & 1][r] = tf_prologue_row<true>(sm.K[0], sm.K[1], r, sm.gk, L, sm.cs, oscale);
+                    float vnorm = 0.f;
+                    const float vt = v_tile_to_f16(sm.V[0], sm.V[1], r, sm.vred[uu & 1], &vnorm);
+                    if (r == 0) sm.vtinv[uu & 1] = vt;
+                    // dS^T row scale: |dS_ji| <= |v_j| |dA_i| + |Delta_i| <= |v_j| sqrt(D) max|dout| + max|Delta|
+                    // (vnorm is the raw row's norm: the bound is taken before any fp16 scaling)
+                    sm.dsc[uu & 1][r] = ldexpf(1.0f, fit_exp(vnorm * sqrtf((float)kD) * domx + dlmx));
+                    if (r == 0) sm.uinv[uu & 1] = ldexpf(1.0f, -E);
+                    fence_proxy_async_smem();
+                    mbar_arrive(&sm.bar[KB_KVREADY]);
+                }
             }
         }
     } else if (warp >= 12) {
+        reg_alloc<208>();
         // ================================================ dv, dk epilogue (thread = key row)
         const int r = tid - 384, wq = warp - 12;
         const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
@@ -1064,32 +1054,40 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             const UnitInfo x = decode_unit(L, u);
             const int j = x.kt * TF_BN + r;
             const bool valid = j < L.S;
+            const size_t off = ((size_t)(x.b * (size_t)L.S + (valid ? j : 0)) * L.Hkv + x.kvh) * kD;
+            uint4 xv0[8];  // first half of the raw k row, in flight during the wait
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                xv0[c] = valid ? __ldg(reinterpret_cast<const uint4*>(L.k + off) + c) : make_uint4(0u, 0u, 0u, 0u);
             if (!mbar_wait(&sm.bar[KB_DVKFULL], uu & 1, abort, 240)) break;
             tc_fence_after();
-            const size_t off = ((size_t)(x.b * (size_t)L.S + (valid ? j : 0)) * L.Hkv + x.kvh) * kD;
             const float dvf = sm.uinv[uu & 1];
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
-                uint32_t v[32];
-                tmem_ld32(TM_DV + lane_off + 32 * c, v);
+                float v[32];
+                tmem_ld32f(TM_DV + lane_off + 32 * c, v);
                 tmem_wait_ld();
                 if (valid) {
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         uint32_t o[4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            o[e] = pack_bf16(__uint_as_float(v[8 * q4 + 2 * e]) * dvf,
-                                             __uint_as_float(v[8 * q4 + 2 * e + 1]) * dvf);
+                        for (int e = 0; e < 4; ++e) o[e] = pack_bf16(v[8 * q4 + 2 * e] * dvf, v[8 * q4 + 2 * e + 1] * dvf);
                         reinterpret_cast<uint4*>(p.P.dv + off)[4 * c + q4] = make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 }
             }
+            float dy[128];
+            tmem_ld32f(TM_DK + lane_off, dy);
+            tmem_ld32f(TM_DK + lane_off + 32, dy + 32);
+            tmem_ld32f(TM_DK + lane_off + 64, dy + 64);
+            tmem_ld32f(TM_DK + lane_off + 96, dy + 96);
+            tmem_wait_ld();
             const float f = L.scale / (sm.dsc[uu & 1][r] * oscale);
-            row_rope_rms_backward(TM_DK + lane_off, f, sm.kmdot[uu & 1][r], sm.krinv[uu & 1][r], L.k + off, p.P.dk + off,
-                                  valid, j, sm.gk, sm.dgk[wq], L);
+            const float mdot = sm.kmdot[uu & 1][r], rinv = sm.krinv[uu & 1][r];
             tc_fence_before();
-            mbar_arrive(&sm.bar[KB_DVKEMPTY]);
+            mbar_arrive(&sm.bar[KB_DVKEMPTY]);  // dV, dK of the unit are out of TMEM
+            row_rope_rms_backward_regs(dy, f, mdot, rinv, xv0, L.k + off, p.P.dk + off, valid, j, sm.gk, sm.dgk[wq], L);
         }
     }
 
@@ -1145,12 +1143,12 @@ bool bwd_tc_supported(const LayerParams& L) {
     return L.W <= TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1 && get_encode_b() != nullptr;
 }
 
-// workspace of the tcgen05 backward: lse2, delta, domax, dainv [B,Hq,S] fp32; dA16
+// workspace of the tcgen05 backward: delta, domax, dainv [B,Hq,S] fp32; dA16
 // [B,S,Hq,D] fp16; 2 x d_gamma partials
 size_t bwd_tc_workspace_bytes(int B, int S, int Hq) {
     const size_t rows = (size_t)B * S * Hq;
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
-    return 4 * a(rows * sizeof(float)) + a(rows * kD * sizeof(__half)) +
+    return 3 * a(rows * sizeof(float)) + a(rows * kD * sizeof(__half)) +
            2 * a((size_t)TB_MAX_GRID * kD * sizeof(float));
 }
 
@@ -1168,7 +1166,7 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
         off += a(bytes);
         return q;
     };
-    p.P.lse2 = reinterpret_cast<float*>(take(rows * 4));
+    p.P.lse2 = nullptr;  // P is formed from the forward's lse
     p.P.delta = reinterpret_cast<float*>(take(rows * 4));
     p.domax = reinterpret_cast<float*>(take(rows * 4));
     p.dainv = reinterpret_cast<float*>(take(rows * 4));

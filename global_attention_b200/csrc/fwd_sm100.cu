@@ -10,10 +10,13 @@
 // qb-1 and qb, so consecutive steps of one (b, KV head) chain share a tile: a persistent
 // CTA sweeps a contiguous range of steps and loads ONE new K/V tile per step into a 2-slot
 // ring.  K~ and Q~ are normalised/rotated in place in shared memory (TMA-loaded raw,
-// 128-byte swizzle = the UMMA K-major canonical layout).
+// 128-byte swizzle = the UMMA K-major canonical layout) and stored as fp16 times a power of
+// two (qk_fp16_scale) that keeps them in range.
 //
 // Per head m (TMEM: S/P columns [0,256), O double buffer [256,384) and [384,512)):
 //   S   = Q~ [K~_slot0; K~_slot1]^T          tcgen05.mma M=128 N=256 K=128, A,B in smem
+//                                            (fp16 q~, k~, the backward's operands, so the
+//                                            backward recomputes these scores bit for bit)
 //   P   = exp2(S*scale*log2e - max)          softmax warpgroup, thread = query row, fp32,
 //                                            written back as bf16 over the front of S
 //   O   = P [V_slot0; V_slot1]               tcgen05.mma M=128 N=128 K=256, A in TMEM,
@@ -118,6 +121,8 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const uint32_t TM_S = tmem, TM_P = tmem, TM_O0 = tmem + 256;
+    const float oscale = qk_fp16_scale(sm.gq, sm.gk);
+    const float c2 = L.scale_log2 / (oscale * oscale);  // S holds oscale^2 q~.k~
 
     if (warp == 0) {
         // ================================================ K / V producer
@@ -172,7 +177,7 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
     } else if (warp == 1) {
         // ================================================ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t IDESC_S = idesc_bf16(128, 256, false);
+            constexpr uint32_t IDESC_S = idesc_f16(128, 256, false);
             constexpr uint32_t IDESC_O = idesc_bf16(128, 128, true);
             const uint32_t q_base = smem_u32(sm.Q[0][0]);
             const uint32_t k_base = smem_u32(sm.K[0]);
@@ -263,7 +268,7 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
                         if (vis) mx = fmaxf(mx, __uint_as_float(v[e]));
                     }
                 }
-                const float mu = (mx == -INFINITY) ? 0.f : mx * L.scale_log2;
+                const float mu = (mx == -INFINITY) ? 0.f : mx * c2;
                 float l = 0.f;
 #pragma unroll 1
                 for (int c8 = 0; c8 < 8; ++c8) {
@@ -279,8 +284,8 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
                             const int j = kp0 + e;
                             const bool v0 = j <= i && j > i - L.W && j >= 0 && j < L.S;
                             const bool v1 = j + 1 <= i && j + 1 > i - L.W && j + 1 >= 0 && j + 1 < L.S;
-                            const float p0 = v0 ? fast_exp2(__uint_as_float(v[e]) * L.scale_log2 - mu) : 0.f;
-                            const float p1 = v1 ? fast_exp2(__uint_as_float(v[e + 1]) * L.scale_log2 - mu) : 0.f;
+                            const float p0 = v0 ? fast_exp2(__uint_as_float(v[e]) * c2 - mu) : 0.f;
+                            const float p1 = v1 ? fast_exp2(__uint_as_float(v[e + 1]) * c2 - mu) : 0.f;
                             l += p0 + p1;
                             pk[e >> 1] = pack_bf16(p0, p1);
                         }
@@ -310,7 +315,8 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
             const int slot = n & 1;
             if (!mbar_wait(&sm.bar[B_KFULL + slot], (n >> 1) & 1, abort, 32)) return false;
             tf_angles(L, pos0 + r, sm.cs, r);
-            tf_prologue_row(sm.K[0] + slot * TF_HALF_BYTES, sm.K[1] + slot * TF_HALF_BYTES, r, sm.gk, L, sm.cs);
+            tf_prologue_row<true>(sm.K[0] + slot * TF_HALF_BYTES, sm.K[1] + slot * TF_HALF_BYTES, r, sm.gk, L, sm.cs,
+                                  oscale);
             fence_proxy_async_smem();
             mbar_arrive(&sm.bar[B_KREADY + slot]);
             return true;
@@ -325,7 +331,7 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
             for (int h = 0; h < G; ++h, ++m) {
                 const int buf = m & 1;
                 if (!(ok = mbar_wait(&sm.bar[B_QFULL + buf], (m >> 1) & 1, abort, 33))) break;
-                tf_prologue_row(sm.Q[buf][0], sm.Q[buf][1], r, sm.gq, L, sm.cs);
+                tf_prologue_row<true>(sm.Q[buf][0], sm.Q[buf][1], r, sm.gq, L, sm.cs, oscale);
                 fence_proxy_async_smem();
                 mbar_arrive(&sm.bar[B_QREADY + buf]);
             }

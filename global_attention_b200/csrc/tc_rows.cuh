@@ -45,6 +45,16 @@ __device__ __forceinline__ float fast_tanh(float x) {
     return y;
 }
 
+// Power of two that keeps the fp16 q~, k~ in range: |y_d| <= sqrt(D) max|gamma|.  Every CTA
+// of the forward and of both backward kernels derives the same value from gamma_q, gamma_k
+// in shared memory, so all of them form bit-identical fp16 q~, k~ and scores.
+__device__ __forceinline__ float qk_fp16_scale(const float* gq, const float* gk) {
+    float gmax = 0.f;
+    for (int d = 0; d < kD; ++d) gmax = fmaxf(gmax, fmaxf(fabsf(gq[d]), fabsf(gk[d])));
+    const float bound = gmax * sqrtf((float)kD);
+    return (bound > 16384.f && isfinite(bound)) ? ldexpf(1.0f, 13 - ilogbf(bound)) : 1.0f;
+}
+
 // ------------------------------------------------------------------ prologue (one row per thread)
 
 // cos/sin of the TF_HALF rotation angles at `pos`, into column r of the table
