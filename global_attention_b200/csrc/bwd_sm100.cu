@@ -43,10 +43,15 @@ struct BwdTcParams {
     CUtensorMap tm_k;
     CUtensorMap tm_v;
     CUtensorMap tm_da;  // dA16, fp16, same geometry as tm_q
+    CUtensorMap tm_k16; // K~ fp16 (normalised, rotated, times the q~/k~ scale), geometry of tm_k
+    CUtensorMap tm_v16; // V fp16 times 2^e per 128-row tile, geometry of tm_v
     BwdParams P;
     const __half* da16; // [B,S,Hq,D] dA * 2^e (e per row)
     float* dainv;       // [B,Hq,S] 2^-e of each dA row (0 for an all-zero row)
     float* domax;       // [B,Hq,S] max |dout| of each row (bound on |dA|)
+    float* krinv;       // [B,Hkv,S] inverse RMS of each raw k row
+    float* vnorm;       // [B,Hkv,S] 2-norm of each raw v row
+    float* vtinv;       // [B,Hkv,ceil(S/128)] 2^-e of each V tile
     int* err;
     int total;          // steps (query-major) or units (key-major)
 };
@@ -291,7 +296,7 @@ __device__ __forceinline__ void row_rope_rms_backward_regs(float (&dy)[128], flo
 // =====================================================================  query-major kernel
 
 enum QBar {
-    QB_KFULL = 0, QB_KREADY = 2, QB_KEMPTY = 4, QB_VFULL = 6, QB_VREADY = 8, QB_VEMPTY = 10,
+    QB_KFULL = 0, QB_KEMPTY = 4, QB_VFULL = 6, QB_VEMPTY = 10,
     QB_QFULL = 12, QB_QREADY = 13, QB_QEMPTY = 14, QB_DAEMPTY = 15,
     QB_DSFULL = 17, QB_DQFULL = 18, QB_DQEMPTY = 19, QB_DONE = 20, QB_DAFULL = 21,
     QB_DPFULL = 22, QB_COUNT = 23
@@ -304,8 +309,6 @@ struct BwdQTcSmem {
     alignas(1024) unsigned char dA[2][TF_HALF_BYTES];  // dA fp16, row-scaled (TMA from the gate pass)
     float2 cs[TF_HALF][TF_BM];
     float gq[kD], gk[kD];
-    float vtinv[4];          // 2^-e of each V tile, by tile number % 4
-    float vred[2][4];        // scratch of the V tile maximum, by tile number % 2
     float dsinv[2][TF_BM];   // 2^-e of each dS row, by head number % 2
     float mdot[2][TF_BM];    // mean(dy gamma xhat) of each row (RMSNorm backward), by head % 2
     float qrinv[4][TF_BM];   // inverse RMS of each raw q row, by head number % 4
@@ -359,6 +362,81 @@ __device__ __forceinline__ float v_tile_to_f16(unsigned char* h0, unsigned char*
     return ldexpf(1.0f, -e);
 }
 
+// =====================================================================  K / V preparation
+
+constexpr int KP_THREADS = 128;
+
+struct KvPrepSmem {
+    alignas(1024) unsigned char K[2][TF_HALF_BYTES];  // raw k -> K~ fp16 in place
+    alignas(1024) unsigned char V[2][TF_HALF_BYTES];  // raw v -> fp16 in place
+    float2 cs[TF_HALF][TF_BM];
+    float gq[kD], gk[kD];
+    float vred[4];
+    uint64_t bar;
+};
+
+// One CTA per 128-key tile (b, KV head, kt): K~ = fp16(RoPE(gamma_k * k / rms) * oscale) and
+// V * 2^e (one e per tile) into the workspace, with the same device functions the query-major
+// and key-major kernels once applied in their prologues, so every kernel sees the same bits.
+// Also saves each row's inverse RMS (RMSNorm backward of dk) and raw norm of v (dS^T scale).
+// The conversion used to sit on the critical path of both kernels at every new tile.
+__global__ void __launch_bounds__(KP_THREADS) bwd_kv_prep_kernel(const __grid_constant__ BwdTcParams p) {
+    const LayerParams& L = p.P.L;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    KvPrepSmem& sm = *reinterpret_cast<KvPrepSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int r = threadIdx.x;
+    const int nkt = (L.S + TF_BN - 1) / TF_BN;
+    const int kt = blockIdx.x % nkt, chain = blockIdx.x / nkt;
+    const int kvh = chain % L.Hkv, b = chain / L.Hkv;
+    volatile int abort = 0;
+    if (r == 0) {
+        mbar_init(&sm.bar, 1);
+        fence_barrier_init();
+    }
+    sm.gq[r] = L.gamma_q[r];
+    sm.gk[r] = L.gamma_k[r];
+    __syncthreads();
+    if (r == 0) {
+        mbar_expect_tx(&sm.bar, 2 * TF_TILE_BYTES);
+        tma_load_4d(sm.K[0], &p.tm_k, &sm.bar, 0, kvh, kt * TF_BN, b);
+        tma_load_4d(sm.K[1], &p.tm_k, &sm.bar, 64, kvh, kt * TF_BN, b);
+        tma_load_4d(sm.V[0], &p.tm_v, &sm.bar, 0, kvh, kt * TF_BN, b);
+        tma_load_4d(sm.V[1], &p.tm_v, &sm.bar, 64, kvh, kt * TF_BN, b);
+    }
+    const int j = kt * TF_BN + r;
+    tf_angles(L, j, sm.cs, r);
+    const float oscale = qk_fp16_scale(sm.gq, sm.gk);
+    // one decision for the whole CTA (the V conversion below has a CTA-wide barrier)
+    const bool ok = __syncthreads_and(mbar_wait(&sm.bar, 0, &abort, 250)) != 0;
+    if (ok) {
+        const float krinv = tf_prologue_row<true>(sm.K[0], sm.K[1], r, sm.gk, L, sm.cs, oscale);
+        float vn = 0.f;
+        const float vt = v_tile_to_f16(sm.V[0], sm.V[1], r, sm.vred, &vn);
+        if (j < L.S) {
+            const size_t ro = ((size_t)b * L.Hkv + kvh) * L.S + j;
+            p.krinv[ro] = krinv;
+            p.vnorm[ro] = vn;
+        }
+        if (r == 0) p.vtinv[(size_t)chain * nkt + kt] = vt;
+        fence_proxy_async_smem();
+    } else if (r == 0) {
+        mbar_wait_drain(&sm.bar, 0);  // the loads must land before the CTA exits
+    }
+    __syncthreads();
+    if (r == 0) {
+        if (ok) {
+            tma_store_4d(&p.tm_k16, sm.K[0], 0, kvh, kt * TF_BN, b);
+            tma_store_4d(&p.tm_k16, sm.K[1], 64, kvh, kt * TF_BN, b);
+            tma_store_4d(&p.tm_v16, sm.V[0], 0, kvh, kt * TF_BN, b);
+            tma_store_4d(&p.tm_v16, sm.V[1], 64, kvh, kt * TF_BN, b);
+            tma_store_commit();
+            tma_store_wait_read();
+        } else if (p.err) {
+            atomicExch(p.err, 250);
+        }
+    }
+}
+
 __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_constant__ BwdTcParams p) {
     const LayerParams& L = p.P.L;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -373,10 +451,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
         sm.abort = 0;
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.bar[QB_KFULL + i], 1);
-            mbar_init(&sm.bar[QB_KREADY + i], 128);
             mbar_init(&sm.bar[QB_KEMPTY + i], 1);
             mbar_init(&sm.bar[QB_VFULL + i], 1);
-            mbar_init(&sm.bar[QB_VREADY + i], 128);
             mbar_init(&sm.bar[QB_VEMPTY + i], 1);
         }
         mbar_init(&sm.bar[QB_QFULL], 1);
@@ -405,6 +481,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
         prefetch_tmap(&p.tm_k);
         prefetch_tmap(&p.tm_v);
         prefetch_tmap(&p.tm_da);
+        prefetch_tmap(&p.tm_k16);
+        prefetch_tmap(&p.tm_v16);
     }
     tc_fence_before();
     __syncthreads();
@@ -434,13 +512,13 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                     const int slot = n & 1;
                     if (n >= 2 && !mbar_wait(&sm.bar[QB_KEMPTY + slot], ((n >> 1) - 1) & 1, abort, 101)) return false;
                     mbar_expect_tx(&sm.bar[QB_KFULL + slot], TF_TILE_BYTES);
-                    tma_load_4d(sm.K[0] + slot * TF_HALF_BYTES, &p.tm_k, &sm.bar[QB_KFULL + slot], 0, kvh, kt * TF_BN, b);
-                    tma_load_4d(sm.K[1] + slot * TF_HALF_BYTES, &p.tm_k, &sm.bar[QB_KFULL + slot], 64, kvh, kt * TF_BN, b);
+                    tma_load_4d(sm.K[0] + slot * TF_HALF_BYTES, &p.tm_k16, &sm.bar[QB_KFULL + slot], 0, kvh, kt * TF_BN, b);
+                    tma_load_4d(sm.K[1] + slot * TF_HALF_BYTES, &p.tm_k16, &sm.bar[QB_KFULL + slot], 64, kvh, kt * TF_BN, b);
                     last_k[slot] = n;
                     if (n >= 2 && !mbar_wait(&sm.bar[QB_VEMPTY + slot], ((n >> 1) - 1) & 1, abort, 102)) return false;
                     mbar_expect_tx(&sm.bar[QB_VFULL + slot], TF_TILE_BYTES);
-                    tma_load_4d(sm.V[0] + slot * TF_HALF_BYTES, &p.tm_v, &sm.bar[QB_VFULL + slot], 0, kvh, kt * TF_BN, b);
-                    tma_load_4d(sm.V[1] + slot * TF_HALF_BYTES, &p.tm_v, &sm.bar[QB_VFULL + slot], 64, kvh, kt * TF_BN, b);
+                    tma_load_4d(sm.V[0] + slot * TF_HALF_BYTES, &p.tm_v16, &sm.bar[QB_VFULL + slot], 0, kvh, kt * TF_BN, b);
+                    tma_load_4d(sm.V[1] + slot * TF_HALF_BYTES, &p.tm_v16, &sm.bar[QB_VFULL + slot], 64, kvh, kt * TF_BN, b);
                     last_v[slot] = n;
                     return true;
                 };
@@ -492,14 +570,14 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                     if (st.fresh) {
                         n_prev = n_next++;
                         n_cur = n_next++;
-                        ok = mbar_wait(&sm.bar[QB_KREADY + (n_prev & 1)], (n_prev >> 1) & 1, abort, 110) &&
-                             mbar_wait(&sm.bar[QB_VREADY + (n_prev & 1)], (n_prev >> 1) & 1, abort, 111);
+                        ok = mbar_wait(&sm.bar[QB_KFULL + (n_prev & 1)], (n_prev >> 1) & 1, abort, 110) &&
+                             mbar_wait(&sm.bar[QB_VFULL + (n_prev & 1)], (n_prev >> 1) & 1, abort, 111);
                     } else {
                         n_prev = n_cur;
                         n_cur = n_next++;
                     }
-                    ok = ok && mbar_wait(&sm.bar[QB_KREADY + (n_cur & 1)], (n_cur >> 1) & 1, abort, 112) &&
-                         mbar_wait(&sm.bar[QB_VREADY + (n_cur & 1)], (n_cur >> 1) & 1, abort, 113);
+                    ok = ok && mbar_wait(&sm.bar[QB_KFULL + (n_cur & 1)], (n_cur >> 1) & 1, abort, 112) &&
+                         mbar_wait(&sm.bar[QB_VFULL + (n_cur & 1)], (n_cur >> 1) & 1, abort, 113);
                     for (int h = 0; h < G && ok; ++h, ++m) {
                         const uint32_t tA = tm_half(m), tB = tm_half(m + 1);
                         if (!(ok = mbar_wait(&sm.bar[QB_QREADY], m & 1, abort, 114))) break;
@@ -553,6 +631,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
     } else if (warp >= 4 && warp < 8) {
         // ================================================ Delta, dS (thread = query row)
         const int r = tid - 128, wq = warp - 4;
+        const int nkt = (L.S + TF_BN - 1) / TF_BN;
         const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
         int n_next = 0, n_prev = 0, n_cur = 0, m = 0;
         for (int t = t_begin; t < t_end; ++t) {
@@ -561,7 +640,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             const int q0 = st.qb * TF_BM, i = q0 + r;
             const int slot_cur = n_cur & 1;
             const int base0 = (slot_cur == 0 ? q0 : q0 - TF_BN), base1 = (slot_cur == 1 ? q0 : q0 - TF_BN);
-            const int tile0 = (slot_cur == 0) ? n_cur : n_prev, tile1 = (slot_cur == 1) ? n_cur : n_prev;
+            // V tile scales of the two ring slots (a tile before the sequence start holds no key)
+            const float* vtrow = p.vtinv + ((size_t)st.b * L.Hkv + st.kvh) * nkt;
+            const float vt0 = base0 >= 0 ? vtrow[base0 / TF_BN] : 0.f, vt1 = base1 >= 0 ? vtrow[base1 / TF_BN] : 0.f;
             const int imin = q0 + 32 * wq, imax = imin + 31;
             // chunk c8 (32 keys from kp0) against this warp's 32 rows: live = some pair visible,
             // full = every pair visible (warp-uniform; masks skipped)
@@ -582,7 +663,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                 const uint32_t tS = tm_half(m) + lane_off, tP = tm_half(m + 1) + lane_off;
                 if (!mbar_wait(&sm.bar[QB_DPFULL], m & 1, abort, 121)) { stop = true; break; }
                 tc_fence_after();
-                const float kd0 = dai * sm.vtinv[tile0 & 3], kd1 = dai * sm.vtinv[tile1 & 3];
+                const float kd0 = dai * vt0, kd1 = dai * vt1;
                 // pass 1: P = 2^(S c2 - lse), P dP (written back over S and dP), Delta = sum P dP,
                 // max |P dP|, and the RMSNorm backward's row sums  a = sum P dP S,  b = sum P S
                 float num = 0.f, mpd = 0.f, sa = 0.f, sb = 0.f;
@@ -635,32 +716,13 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             if (stop) break;
         }
     } else if (warp >= 8 && warp < 12) {
-        // ================================================ prologue: K~, V, Q~ (fp16, in place)
+        // ================================================ prologue: Q~ (fp16, in place)
         const int r = tid - 256;
-        int n_next = 0, m = 0;
+        int m = 0;
         bool ok = true;
-        auto prologue_kv = [&](int n, int pos0) -> bool {
-            const int slot = n & 1;
-            if (!mbar_wait(&sm.bar[QB_KFULL + slot], (n >> 1) & 1, abort, 130)) return false;
-            tf_angles(L, pos0 + r, sm.cs, r);
-            tf_prologue_row<true>(sm.K[0] + slot * TF_HALF_BYTES, sm.K[1] + slot * TF_HALF_BYTES, r, sm.gk, L,
-                                  sm.cs, oscale);
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.bar[QB_KREADY + slot]);
-            if (!mbar_wait(&sm.bar[QB_VFULL + slot], (n >> 1) & 1, abort, 131)) return false;
-            const float vt = v_tile_to_f16(sm.V[0] + slot * TF_HALF_BYTES, sm.V[1] + slot * TF_HALF_BYTES, r,
-                                           sm.vred[n & 1], nullptr);
-            if (r == 0) sm.vtinv[n & 3] = vt;
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.bar[QB_VREADY + slot]);
-            return true;
-        };
         for (int t = t_begin; t < t_end && ok; ++t) {
             const StepInfo st = decode_step(L, t, t_begin, t_end);
-            const int q0 = st.qb * TF_BM;
-            if (st.fresh) ok = prologue_kv(n_next++, q0 - TF_BN);
-            ok = ok && prologue_kv(n_next++, q0);
-            if (!ok) break;
+            tf_angles(L, st.qb * TF_BM + r, sm.cs, r);  // the step's query positions
             for (int h = 0; h < G; ++h, ++m) {
                 if (!(ok = mbar_wait(&sm.bar[QB_QFULL], m & 1, abort, 132))) break;
                 sm.qrinv[m & 3][r] = tf_prologue_row<true>(sm.Q[0], sm.Q[1], r, sm.gq, L, sm.cs, oscale);
@@ -732,12 +794,12 @@ struct BwdKTcSmem {
     float lse2[2][TF_BM];    // per query column of the buffer
     float delta[2][TF_BM];
     float dcol[2][TF_BM];    // 2^-e of the dA row of each query column
-    float vtinv[2];          // 2^-e of the unit's V tile, by unit parity
-    float vred[2][4];        // scratch of the V tile maximum, by unit parity
-    float dsc[2][TF_BN];     // 2^e of each dS^T row, by unit parity
-    float uinv[2];           // 2^-E, E = the unit's smallest dA row exponent, by unit parity
+    float vtinv[4];          // 2^-e of the unit's V tile, by unit number % 4
+    float dsc[4][TF_BN];     // 2^e of each dS^T row, by unit number % 4
+    // 4 deep: the prologue writes a unit's scales at its start, while the epilogue of an earlier
+    // unit may still read its own (with one query head per KV head a unit has two iterations)
+    float uinv[4];           // 2^-E, E = the unit's smallest dA row exponent, by unit number % 4
     float kmdot[2][TF_BN];   // mean(dy gamma xhat) of each key row (RMSNorm backward), by unit parity
-    float krinv[2][TF_BN];   // inverse RMS of each raw k row, by unit parity
     float red[2][4];         // per-warp maxima for the unit statistics
     float dgk[4][kD];        // this CTA's d_gamma_k, one slice per epilogue warp
     uint64_t bar[KB_COUNT];
@@ -804,6 +866,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
         prefetch_tmap(&p.tm_k);
         prefetch_tmap(&p.tm_v);
         prefetch_tmap(&p.tm_da);
+        prefetch_tmap(&p.tm_k16);
+        prefetch_tmap(&p.tm_v16);
     }
     tc_fence_before();
     __syncthreads();
@@ -826,10 +890,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 int it_all = 0, last_q[2] = {-1, -1}, uu = 0;
                 auto load_kv = [&](const UnitInfo& x) {
                     mbar_expect_tx(&sm.bar[KB_KVFULL], 2 * TF_TILE_BYTES);
-                    tma_load_4d(sm.K[0], &p.tm_k, &sm.bar[KB_KVFULL], 0, x.kvh, x.kt * TF_BN, x.b);
-                    tma_load_4d(sm.K[1], &p.tm_k, &sm.bar[KB_KVFULL], 64, x.kvh, x.kt * TF_BN, x.b);
-                    tma_load_4d(sm.V[0], &p.tm_v, &sm.bar[KB_KVFULL], 0, x.kvh, x.kt * TF_BN, x.b);
-                    tma_load_4d(sm.V[1], &p.tm_v, &sm.bar[KB_KVFULL], 64, x.kvh, x.kt * TF_BN, x.b);
+                    tma_load_4d(sm.K[0], &p.tm_k16, &sm.bar[KB_KVFULL], 0, x.kvh, x.kt * TF_BN, x.b);
+                    tma_load_4d(sm.K[1], &p.tm_k16, &sm.bar[KB_KVFULL], 64, x.kvh, x.kt * TF_BN, x.b);
+                    tma_load_4d(sm.V[0], &p.tm_v16, &sm.bar[KB_KVFULL], 0, x.kvh, x.kt * TF_BN, x.b);
+                    tma_load_4d(sm.V[1], &p.tm_v16, &sm.bar[KB_KVFULL], 64, x.kvh, x.kt * TF_BN, x.b);
                 };
                 bool ok = true;
                 for (int u = u_begin; u < u_end && ok && !*abort; ++u, ++uu) {
@@ -868,7 +932,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 bool ok = true;
                 for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
                     const UnitInfo x = decode_unit(L, u);
-                    if (!(ok = mbar_wait(&sm.bar[KB_KVREADY], uu & 1, abort, 210))) break;
+                    if (!(ok = mbar_wait(&sm.bar[KB_KVFULL], uu & 1, abort, 210))) break;
                     for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
                         const int buf = it_all & 1;
                         const uint32_t qb_addr = q_base + buf * 2 * TF_HALF_BYTES, da_addr = da_base + buf * 2 * TF_HALF_BYTES;
@@ -923,9 +987,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             const UnitInfo x = decode_unit(L, u);
             const int j = x.kt * TF_BN + r;
             if (!(ok = mbar_wait(&sm.bar[KB_KVREADY], uu & 1, abort, 220))) break;
-            const float vin = sm.vtinv[uu & 1];  // undoes the V tile scale of dP^T
-            const float su = 1.0f / sm.uinv[uu & 1];  // 2^E: P^T columns carry 2^(E - e_i)
-            const float dsc = sm.dsc[uu & 1][r];
+            const float vin = sm.vtinv[uu & 3];  // undoes the V tile scale of dP^T
+            const float su = 1.0f / sm.uinv[uu & 3];  // 2^E: P^T columns carry 2^(E - e_i)
+            const float dsc = sm.dsc[uu & 3][r];
             float kacc = 0.f;  // sum over the unit of dS^T S^T (unscaled dS^T): dk's RMSNorm row term
             for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
                 const int buf = it_all & 1;
@@ -1004,6 +1068,18 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             // E = fit_exp(max domax) is the smallest row exponent of dA in the unit, so every
             // column factor 2^(E - e_i) of P^T is <= 1
             const int E = fit_exp(domx);
+            {
+                // unit scales for the softmax warps: V tile (prepared), dS^T rows, dA columns
+                const int j = x.kt * TF_BN + r, nkt = (L.S + TF_BN - 1) / TF_BN;
+                const float vnorm = j < L.S ? p.vnorm[((size_t)x.b * L.Hkv + x.kvh) * L.S + j] : 0.f;
+                // dS^T row scale: |dS_ji| <= |v_j| |dA_i| + |Delta_i| <= |v_j| sqrt(D) max|dout| + max|Delta|
+                sm.dsc[uu & 3][r] = ldexpf(1.0f, fit_exp(vnorm * sqrtf((float)kD) * domx + dlmx));
+                if (r == 0) {
+                    sm.uinv[uu & 3] = ldexpf(1.0f, -E);
+                    sm.vtinv[uu & 3] = p.vtinv[((size_t)x.b * L.Hkv + x.kvh) * nkt + x.kt];
+                }
+                mbar_arrive(&sm.bar[KB_KVREADY]);
+            }
             // angles of the key tile's positions, which are also those of the query block of the
             // first G iterations (qb = kt)
             tf_angles(L, x.kt * TF_BN + r, sm.cs, r);
@@ -1026,22 +1102,6 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 sm.dcol[buf][r] = valid ? p.dainv[ro] : 0.f;
                 fence_proxy_async_smem();
                 mbar_arrive(&sm.bar[KB_QREADY + buf]);
-                if (it == 0) {
-                    // K~ (fp16) and V (fp16, row-scaled) of the unit's key tile, after the first
-                    // query tile: that one was loaded during the previous unit, K and V only once
-                    // its products were done
-                    if (!(ok = mbar_wait(&sm.bar[KB_KVFULL], uu & 1, abort, 230))) break;
-                    sm.krinv[uu & 1][r] = tf_prologue_row<true>(sm.K[0], sm.K[1], r, sm.gk, L, sm.cs, oscale);
-                    float vnorm = 0.f;
-                    const float vt = v_tile_to_f16(sm.V[0], sm.V[1], r, sm.vred[uu & 1], &vnorm);
-                    if (r == 0) sm.vtinv[uu & 1] = vt;
-                    // dS^T row scale: |dS_ji| <= |v_j| |dA_i| + |Delta_i| <= |v_j| sqrt(D) max|dout| + max|Delta|
-                    // (vnorm is the raw row's norm: the bound is taken before any fp16 scaling)
-                    sm.dsc[uu & 1][r] = ldexpf(1.0f, fit_exp(vnorm * sqrtf((float)kD) * domx + dlmx));
-                    if (r == 0) sm.uinv[uu & 1] = ldexpf(1.0f, -E);
-                    fence_proxy_async_smem();
-                    mbar_arrive(&sm.bar[KB_KVREADY]);
-                }
             }
         }
     } else if (warp >= 12) {
@@ -1061,7 +1121,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 xv0[c] = valid ? __ldg(reinterpret_cast<const uint4*>(L.k + off) + c) : make_uint4(0u, 0u, 0u, 0u);
             if (!mbar_wait(&sm.bar[KB_DVKFULL], uu & 1, abort, 240)) break;
             tc_fence_after();
-            const float dvf = sm.uinv[uu & 1];
+            const float dvf = sm.uinv[uu & 3];
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 float v[32];
@@ -1083,8 +1143,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             tmem_ld32f(TM_DK + lane_off + 64, dy + 64);
             tmem_ld32f(TM_DK + lane_off + 96, dy + 96);
             tmem_wait_ld();
-            const float f = L.scale / (sm.dsc[uu & 1][r] * oscale);
-            const float mdot = sm.kmdot[uu & 1][r], rinv = sm.krinv[uu & 1][r];
+            const float f = L.scale / (sm.dsc[uu & 3][r] * oscale);
+            const float mdot = sm.kmdot[uu & 1][r];
+            const float rinv = valid ? p.krinv[((size_t)x.b * L.Hkv + x.kvh) * L.S + j] : 0.f;
             tc_fence_before();
             mbar_arrive(&sm.bar[KB_DVKEMPTY]);  // dV, dK of the unit are out of TMEM
             row_rope_rms_backward_regs(dy, f, mdot, rinv, xv0, L.k + off, p.P.dk + off, valid, j, sm.gk, sm.dgk[wq], L);
@@ -1133,9 +1194,10 @@ bool make_map_b(CUtensorMap* map, const void* base, int H, int S, int B,
 
 }  // namespace
 
-extern const char* const kBwdTcKernelNames[] = {"bwd_gate_kernel", "bwd_q_tc_kernel", "bwd_kv_tc_kernel",
+extern const char* const kBwdTcKernelNames[] = {"bwd_gate_kernel",         "bwd_kv_prep_kernel",
+                                                "bwd_q_tc_kernel",         "bwd_kv_tc_kernel",
                                                 "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"};
-extern const int kBwdTcKernelCount = 5;
+extern const int kBwdTcKernelCount = 6;
 
 __global__ void dgamma_reduce_kernel(const float* __restrict__ parts, int n, float* __restrict__ out);
 
@@ -1143,13 +1205,15 @@ bool bwd_tc_supported(const LayerParams& L) {
     return L.W <= TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1 && get_encode_b() != nullptr;
 }
 
-// workspace of the tcgen05 backward: delta, domax, dainv [B,Hq,S] fp32; dA16
-// [B,S,Hq,D] fp16; 2 x d_gamma partials
-size_t bwd_tc_workspace_bytes(int B, int S, int Hq) {
-    const size_t rows = (size_t)B * S * Hq;
+// workspace of the tcgen05 backward: delta, domax, dainv [B,Hq,S] fp32; dA16 [B,S,Hq,D]
+// fp16; K~16, V16 [B,S,Hkv,D] fp16; krinv, vnorm [B,Hkv,S] fp32; vtinv per V tile; 2 x
+// d_gamma partials
+size_t bwd_tc_workspace_bytes(int B, int S, int Hq, int Hkv) {
+    const size_t rows = (size_t)B * S * Hq, krows = (size_t)B * S * Hkv;
+    const size_t tiles = (size_t)B * Hkv * ((S + TF_BN - 1) / TF_BN);
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
-    return 3 * a(rows * sizeof(float)) + a(rows * kD * sizeof(__half)) +
-           2 * a((size_t)TB_MAX_GRID * kD * sizeof(float));
+    return 3 * a(rows * sizeof(float)) + a(rows * kD * sizeof(__half)) + 2 * a(krows * kD * sizeof(__half)) +
+           2 * a(krows * sizeof(float)) + a(tiles * sizeof(float)) + 2 * a((size_t)TB_MAX_GRID * kD * sizeof(float));
 }
 
 cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, cudaStream_t stream,
@@ -1172,12 +1236,21 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     p.dainv = reinterpret_cast<float*>(take(rows * 4));
     __half* da16 = reinterpret_cast<__half*>(take(rows * kD * sizeof(__half)));
     p.da16 = da16;
+    const size_t krows = (size_t)L.B * L.S * L.Hkv;
+    const int nkt = (L.S + TF_BN - 1) / TF_BN;
+    void* k16 = take(krows * kD * sizeof(__half));
+    void* v16 = take(krows * kD * sizeof(__half));
+    p.krinv = reinterpret_cast<float*>(take(krows * 4));
+    p.vnorm = reinterpret_cast<float*>(take(krows * 4));
+    p.vtinv = reinterpret_cast<float*>(take((size_t)L.B * L.Hkv * nkt * 4));
     p.P.dgq_part = reinterpret_cast<float*>(take((size_t)TB_MAX_GRID * kD * 4));
     p.P.dgk_part = reinterpret_cast<float*>(take((size_t)TB_MAX_GRID * kD * 4));
     p.err = err_word;
     if (!make_map_b(&p.tm_q, L.q, L.Hq, L.S, L.B) || !make_map_b(&p.tm_k, L.k, L.Hkv, L.S, L.B) ||
         !make_map_b(&p.tm_v, L.v, L.Hkv, L.S, L.B) ||
-        !make_map_b(&p.tm_da, da16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        !make_map_b(&p.tm_da, da16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+        !make_map_b(&p.tm_k16, k16, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+        !make_map_b(&p.tm_v16, v16, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1207,22 +1280,31 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     const long long half_warps = ((long long)rows + GATE_UNROLL - 1) / GATE_UNROLL;
     const long long gate_need = (half_warps * 16 + GATE_THREADS - 1) / GATE_THREADS;
     const int gate_grid = (int)(gate_need < 2LL * sms ? gate_need : 2LL * sms);
+    const size_t smem_p = sizeof(KvPrepSmem) + 1024;
+    if ((e = cudaFuncSetAttribute(bwd_kv_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p)) !=
+        cudaSuccess)
+        return e;
+    const long long kv_tiles = (long long)L.B * L.Hkv * nkt;
+    if (kv_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
     if ((e = before(0)) != cudaSuccess) return e;
     bwd_gate_kernel<<<gate_grid, GATE_THREADS, 0, stream>>>(bp.dout, L.g, bp.out, bp.dg, da16, p.dainv, p.domax,
                                                             (long long)rows, L.S, L.Hq);
     if ((e = after(0)) != cudaSuccess) return e;
     if ((e = before(1)) != cudaSuccess) return e;
-    bwd_q_tc_kernel<<<grid, TB_THREADS, smem_q, stream>>>(p);
+    bwd_kv_prep_kernel<<<(int)kv_tiles, KP_THREADS, smem_p, stream>>>(p);
     if ((e = after(1)) != cudaSuccess) return e;
     if ((e = before(2)) != cudaSuccess) return e;
-    bwd_kv_tc_kernel<<<grid, TB_THREADS, smem_k, stream>>>(p);
+    bwd_q_tc_kernel<<<grid, TB_THREADS, smem_q, stream>>>(p);
     if ((e = after(2)) != cudaSuccess) return e;
     if ((e = before(3)) != cudaSuccess) return e;
-    dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgk_part, grid, bp.dgamma_k);
+    bwd_kv_tc_kernel<<<grid, TB_THREADS, smem_k, stream>>>(p);
     if ((e = after(3)) != cudaSuccess) return e;
     if ((e = before(4)) != cudaSuccess) return e;
+    dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgk_part, grid, bp.dgamma_k);
+    if ((e = after(4)) != cudaSuccess) return e;
+    if ((e = before(5)) != cudaSuccess) return e;
     dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgq_part, grid, bp.dgamma_q);
-    return after(4);
+    return after(5);
 }
 
 }  // namespace zgcm

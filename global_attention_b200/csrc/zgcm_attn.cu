@@ -18,7 +18,7 @@ extern const int kBwdMmaKernelCount;
 cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, cudaStream_t stream,
                           void* const* events, int n_pairs);
 bool bwd_tc_supported(const LayerParams& L);
-size_t bwd_tc_workspace_bytes(int B, int S, int Hq);
+size_t bwd_tc_workspace_bytes(int B, int S, int Hq, int Hkv);
 extern const char* const kBwdTcKernelNames[];
 extern const int kBwdTcKernelCount;
 int bwd_mma_n_k_parts(int B, int S, int Hkv);
@@ -169,7 +169,7 @@ size_t zgcm_attn_bwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int wi
     if (check_shape(B, S, Hq, Hkv, D, 0, 1.0, window, 1, 0.f, 1.f) != ZGCM_OK) return 0;
     if ((long long)B * S == 0) return 0;
     // enough for either backward (the kernel choice also depends on rope_dims)
-    const size_t a = bwd_layout(B, S, Hq, Hkv).total, b = bwd_tc_workspace_bytes(B, S, Hq);
+    const size_t a = bwd_layout(B, S, Hq, Hkv).total, b = bwd_tc_workspace_bytes(B, S, Hq, Hkv);
     return a > b ? a : b;
 }
 

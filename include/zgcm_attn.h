@@ -96,7 +96,10 @@ size_t zgcm_attn_bwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int wi
  * q, k, v, g, gamma_q and gamma_k.
  *
  * In : the forward's inputs and arguments, its outputs `out` (bf16) and `lse` (fp32),
- *      and dout bf16 [B,S,Hq,D].
+ *      and dout bf16 [B,S,Hq,D].  The backward forms the softmax probabilities from `lse`
+ *      as exp(s_ij - lse_i), so `lse` must be the one zgcm_attn_fwd returned for these
+ *      inputs: the tcgen05 kernels recompute the forward's scores bit for bit, and a
+ *      log-sum-exp from elsewhere leaves the probabilities of a row summing to other than 1.
  * Out: dq, dg bf16 [B,S,Hq,D] — gradients w.r.t. the RAW q (before RMSNorm) and the gate
  *      logits; dk, dv bf16 [B,S,Hkv,D] — summed over the Hq/Hkv query heads that share
  *      each KV head; dgamma_q, dgamma_k fp32 [D] — overwritten (not accumulated).
@@ -172,8 +175,9 @@ int zgcm_attn_device_error(void);
 
 /* Name of the i-th kernel zgcm_attn_bwd launches for this configuration (static string),
  * or NULL when i is past the last one.  Windows up to 128 with 42 rotated dims run the
- * gate pass and the tcgen05 pair (bwd_gate_kernel, bwd_q_tc_kernel, bwd_kv_tc_kernel, then
- * the two d_gamma reductions); other shapes, or ZGCM_FORCE_MMA=1, the warp-MMA kernels. */
+ * gate pass, the K/V preparation and the tcgen05 pair (bwd_gate_kernel, bwd_kv_prep_kernel,
+ * bwd_q_tc_kernel, bwd_kv_tc_kernel, then the two d_gamma reductions); other shapes, or
+ * ZGCM_FORCE_MMA=1, the warp-MMA kernels. */
 const char* zgcm_attn_bwd_kernel_name(int i, int S, int rope_dims, int window);
 
 #ifdef __cplusplus
