@@ -173,29 +173,33 @@ __device__ __forceinline__ uint4* tile_chunk(unsigned char* h0, unsigned char* h
     return reinterpret_cast<uint4*>(hb + (uint32_t)r * 128u + (uint32_t)(((ch & 7) ^ (r & 7)) << 4));
 }
 
-// visibility of key j to query i: the causal window max(0, i-W+1) <= j <= i inside the
-// sequence (always true for a chunk known to be fully visible)
-template <bool FULL>
-__device__ __forceinline__ bool visible(int i, int j, const LayerParams& L) {
-    return FULL || (j <= i && j > i - L.W && j >= 0 && j < L.S);
+// Bits lo..hi of a 32-bit word, clamped to 0..31 (0 when the range is empty): the visible
+// positions of a 32-wide chunk for one thread's row.  A bit test and a select per element
+// replace the window comparisons, which compiled to divergent branches around the exp2.
+__device__ __forceinline__ uint32_t bit_range(int lo, int hi) {
+    lo = max(lo, 0);
+    hi = min(hi, 31);
+    if (lo > hi) return 0u;
+    return (0xffffffffu >> (31 - hi)) & (0xffffffffu << lo);
 }
 
-// Query-major pass over one 32-key chunk of a row (S, dP as accumulated in TMEM):
-//   P = 2^(s c2 - lse2) on visible pairs (0 elsewhere),  P dP with dP = dv * kd (kd undoes
-//   the dA row and V tile scales);  num += P dP,  mpd = max |P dP|,  sa += P dP s,  sb += P s.
-// P and P dP replace s and dv in place (the caller writes them back to TMEM).
+// Query-major pass over one 32-key chunk of a row (S, dP as accumulated in TMEM), with
+// vm = the visible keys of the chunk (ignored when FULL: all visible):
+//   P = 2^(s c2 - lse2) on visible keys (0 elsewhere) and P dv, dv = dP before the chunk's
+//   scale kd (the caller applies kd to the chunk sums): cnum += P dv, cmpd = max |P dv|,
+//   csa += P dv s, sb += P s.  P and P dv replace s and dv in place (written back to TMEM).
 template <bool FULL>
-__device__ __forceinline__ void q_pass1_chunk(float (&sv)[32], float (&dv)[32], float kd, float c2, float lse2, int i,
-                                              int kp0, const LayerParams& L, float& num, float& mpd, float& sa,
-                                              float& sb) {
+__device__ __forceinline__ void q_pass1_chunk(float (&sv)[32], float (&dv)[32], uint32_t vm, float c2, float lse2,
+                                              float& cnum, float& cmpd, float& csa, float& sb) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
         const float s = sv[e];
-        const float pv = visible<FULL>(i, kp0 + e, L) ? fast_exp2(fmaf(s, c2, -lse2)) : 0.f;
-        const float pd = pv * (dv[e] * kd);
-        num += pd;
-        mpd = fmaxf(mpd, fabsf(pd));
-        sa = fmaf(pd, s, sa);
+        float pv = fast_exp2(fmaf(s, c2, -lse2));
+        if (!FULL) pv = ((vm >> e) & 1u) ? pv : 0.f;  // (a masked score may overflow: selected away)
+        const float pd = pv * dv[e];
+        cnum += pd;
+        cmpd = fmaxf(cmpd, fabsf(pd));
+        csa = fmaf(pd, s, csa);
         sb = fmaf(pv, s, sb);
         sv[e] = pv;
         dv[e] = pd;
@@ -203,14 +207,15 @@ __device__ __forceinline__ void q_pass1_chunk(float (&sv)[32], float (&dv)[32], 
 }
 
 // Key-major chunk: one key row j against 32 query columns i0.. (S^T, dP^T from TMEM; per
-// column lse, Delta and dA row scale 2^-e_i from shared memory):
+// column lse, Delta and dA row scale 2^-e_i from shared memory; vm = the visible columns,
+// ignored when FULL):
 //   P^T = 2^(s c2 - lse) (visible pairs), dP^T = dv * vin * 2^-e_i,
 //   P^T for dV carries 2^(E - e_i) (su = 2^E), dS^T = P^T (dP^T - Delta) * dsc,
 //   kacc += dS^T S^T (unscaled dS^T; dk's RMSNorm row term).
 template <bool FULL>
 __device__ __forceinline__ void kv_chunk(const float* sv, const float* dv, const float* lse2c, const float* deltac,
-                                         const float* dcolc, float vin, float su, float dsc, float c2, int j, int i0,
-                                         const LayerParams& L, uint32_t (&pp)[16], uint32_t (&dd)[16], float& kacc) {
+                                         const float* dcolc, uint32_t vm, float vin, float su, float dsc, float c2,
+                                         uint32_t (&pp)[16], uint32_t (&dd)[16], float& kacc) {
 #pragma unroll
     for (int e4 = 0; e4 < 8; ++e4) {
         const float4 ls = *reinterpret_cast<const float4*>(lse2c + 4 * e4);
@@ -220,9 +225,9 @@ __device__ __forceinline__ void kv_chunk(const float* sv, const float* dv, const
         float p4[4], d4[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const int e = 4 * e4 + u, i = i0 + e;
-            const bool vis = FULL || (j <= i && j > i - L.W && i < L.S && j < L.S);
-            const float pv = vis ? fast_exp2(fmaf(sv[e], c2, -lsv[u])) : 0.f;
+            const int e = 4 * e4 + u;
+            float pv = fast_exp2(fmaf(sv[e], c2, -lsv[u]));
+            if (!FULL) pv = ((vm >> e) & 1u) ? pv : 0.f;
             const float dp = dv[e] * vin * dcv[u];
             const float d = pv * (dp - dlv[u]);
             kacc = fmaf(d, sv[e], kacc);
@@ -499,10 +504,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
     const float mdot_f = c2 * kLn2 / (float)kD;
 
     // Registers by warpgroup (4 x 128 in all, set at the top of each role): TMA / MMA issue
-    // 48, softmax 128, prologue 128, epilogue 208 (it holds a whole dq~ row so that it can
-    // release TMEM before its arithmetic).
+    // 64, softmax 128, prologue 128, epilogue 192 (it holds a whole dq~ row so that it can
+    // release TMEM before its arithmetic).  Fewer for the issue warps made them spill.
     if (warp < 4) {
-        reg_dealloc<48>();
+        reg_dealloc<64>();
         if (warp == 0) {
             // ================================================ K / V producer
             if (lane == 0) {
@@ -667,6 +672,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                 // pass 1: P = 2^(S c2 - lse), P dP (written back over S and dP), Delta = sum P dP,
                 // max |P dP|, and the RMSNorm backward's row sums  a = sum P dP S,  b = sum P S
                 float num = 0.f, mpd = 0.f, sa = 0.f, sb = 0.f;
+                const int klo = max(i - L.W + 1, 0), khi = min(i, L.S - 1);  // this row's visible keys
 #pragma unroll 1
                 for (int c8 = 0; c8 < 8; ++c8) {
                     const int kp0 = chunk_kp0(c8);
@@ -675,11 +681,15 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                     tmem_ld32f(tS + 32 * c8, sv);
                     tmem_ld32f(tP + 32 * c8, dv);
                     tmem_wait_ld();
-                    const float kd = c8 < 4 ? kd0 : kd1;
+                    float cnum = 0.f, cmpd = 0.f, csa = 0.f;
                     if (chunk_full(kp0))
-                        q_pass1_chunk<true>(sv, dv, kd, c2, lse2, i, kp0, L, num, mpd, sa, sb);
+                        q_pass1_chunk<true>(sv, dv, 0u, c2, lse2, cnum, cmpd, csa, sb);
                     else
-                        q_pass1_chunk<false>(sv, dv, kd, c2, lse2, i, kp0, L, num, mpd, sa, sb);
+                        q_pass1_chunk<false>(sv, dv, bit_range(klo - kp0, khi - kp0), c2, lse2, cnum, cmpd, csa, sb);
+                    const float kd = c8 < 4 ? kd0 : kd1;  // dP = dv * kd on this key tile
+                    num = fmaf(kd, cnum, num);
+                    mpd = fmaxf(mpd, fabsf(kd) * cmpd);
+                    sa = fmaf(kd, csa, sa);
                     tmem_st32f(tS + 32 * c8, sv);
                     tmem_st32f(tP + 32 * c8, dv);
                 }
@@ -697,9 +707,11 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                         tmem_ld32f(tS + 32 * c8, pv);
                         tmem_ld32f(tP + 32 * c8, pd);
                         tmem_wait_ld();
+                        // pd holds P dv: dS dsc = P dv (kd dsc) - P (Delta dsc)
+                        const float ka = (c8 < 4 ? kd0 : kd1) * dsc, kb = -delta * dsc;
 #pragma unroll
                         for (int e = 0; e < 32; e += 2)
-                            pk[e >> 1] = pack2<true>(fmaf(-delta, pv[e], pd[e]) * dsc, fmaf(-delta, pv[e + 1], pd[e + 1]) * dsc);
+                            pk[e >> 1] = pack2<true>(fmaf(pd[e], ka, pv[e] * kb), fmaf(pd[e + 1], ka, pv[e + 1] * kb));
                     } else {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) pk[e] = 0u;
@@ -731,7 +743,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             }
         }
     } else if (warp >= 12) {
-        reg_alloc<208>();
+        reg_alloc<192>();
         // ================================================ dq epilogue (thread = query row)
         const int r = tid - 384, wq = warp - 12;
         const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
@@ -880,10 +892,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
     const float mdot_f = c2 * kLn2 / (float)kD;  // scale / (D oscale^2)
 
     // Registers by warpgroup (4 x 128 in all, set at the top of each role): TMA / MMA issue
-    // 48, softmax 128, prologue 128, epilogue 208 (it holds a whole dk~ row so that it can
+    // 64, softmax 128, prologue 128, epilogue 192 (it holds a whole dk~ row so that it can
     // release TMEM before its arithmetic).
     if (warp < 4) {
-        reg_dealloc<48>();
+        reg_dealloc<64>();
         if (warp == 0) {
             // ================================================ TMA producer: K, V per unit; Q, dA per iteration
             if (lane == 0) {
@@ -1012,12 +1024,15 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                         tmem_ld32f(TM_DP + lane_off + 32 * c8, dv);
                         tmem_wait_ld();
                         const int ql0 = 32 * c8;
-                        if (full)
-                            kv_chunk<true>(sv, dv, sm.lse2[buf] + ql0, sm.delta[buf] + ql0, sm.dcol[buf] + ql0, vin, su,
-                                           dsc, c2, j, i0, L, pp, dd, kacc);
-                        else
-                            kv_chunk<false>(sv, dv, sm.lse2[buf] + ql0, sm.delta[buf] + ql0, sm.dcol[buf] + ql0, vin, su,
-                                            dsc, c2, j, i0, L, pp, dd, kacc);
+                        if (full) {
+                            kv_chunk<true>(sv, dv, sm.lse2[buf] + ql0, sm.delta[buf] + ql0, sm.dcol[buf] + ql0, 0u, vin,
+                                           su, dsc, c2, pp, dd, kacc);
+                        } else {
+                            // queries that see key j: j <= i <= min(j + W - 1, S - 1)
+                            const uint32_t vm = j < L.S ? bit_range(j - i0, min(j + L.W - 1, L.S - 1) - i0) : 0u;
+                            kv_chunk<false>(sv, dv, sm.lse2[buf] + ql0, sm.delta[buf] + ql0, sm.dcol[buf] + ql0, vm, vin,
+                                            su, dsc, c2, pp, dd, kacc);
+                        }
                     } else {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) pp[e] = dd[e] = 0u;
@@ -1105,7 +1120,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             }
         }
     } else if (warp >= 12) {
-        reg_alloc<208>();
+        reg_alloc<192>();
         // ================================================ dv, dk epilogue (thread = key row)
         const int r = tid - 384, wq = warp - 12;
         const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
