@@ -173,16 +173,6 @@ __device__ __forceinline__ uint4* tile_chunk(unsigned char* h0, unsigned char* h
     return reinterpret_cast<uint4*>(hb + (uint32_t)r * 128u + (uint32_t)(((ch & 7) ^ (r & 7)) << 4));
 }
 
-// Bits lo..hi of a 32-bit word, clamped to 0..31 (0 when the range is empty): the visible
-// positions of a 32-wide chunk for one thread's row.  A bit test and a select per element
-// replace the window comparisons, which compiled to divergent branches around the exp2.
-__device__ __forceinline__ uint32_t bit_range(int lo, int hi) {
-    lo = max(lo, 0);
-    hi = min(hi, 31);
-    if (lo > hi) return 0u;
-    return (0xffffffffu >> (31 - hi)) & (0xffffffffu << lo);
-}
-
 // Query-major pass over one 32-key chunk of a row (S, dP as accumulated in TMEM), with
 // vm = the visible keys of the chunk (ignored when FULL: all visible):
 //   P = 2^(s c2 - lse2) on visible keys (0 elsewhere) and P dv, dv = dP before the chunk's
@@ -791,7 +781,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
 // =====================================================================  key-major kernel
 
 enum KBar {
-    KB_KVFULL = 0, KB_KVREADY = 1, KB_KVEMPTY = 2,
+    KB_KVFULL = 0, KB_KVEMPTY = 2,
     KB_QFULL = 3, KB_QREADY = 5, KB_QEMPTY = 7,
     KB_SFULL = 9, KB_PFULL = 10, KB_DVKFULL = 11, KB_DVKEMPTY = 12, KB_DONE = 13, KB_COUNT = 14
 };
@@ -850,7 +840,6 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
     if (tid == 0) {
         sm.abort = 0;
         mbar_init(&sm.bar[KB_KVFULL], 1);
-        mbar_init(&sm.bar[KB_KVREADY], 128);
         mbar_init(&sm.bar[KB_KVEMPTY], 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.bar[KB_QFULL + i], 1);
@@ -998,10 +987,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
         for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
             const UnitInfo x = decode_unit(L, u);
             const int j = x.kt * TF_BN + r;
-            if (!(ok = mbar_wait(&sm.bar[KB_KVREADY], uu & 1, abort, 220))) break;
-            const float vin = sm.vtinv[uu & 3];  // undoes the V tile scale of dP^T
-            const float su = 1.0f / sm.uinv[uu & 3];  // 2^E: P^T columns carry 2^(E - e_i)
-            const float dsc = sm.dsc[uu & 3][r];
+            float vin = 0.f, su = 0.f, dsc = 0.f;
             float kacc = 0.f;  // sum over the unit of dS^T S^T (unscaled dS^T): dk's RMSNorm row term
             for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
                 const int buf = it_all & 1;
@@ -1009,6 +995,12 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 decode_iter(L, x, it, qb, hg);
                 const int q0 = qb * TF_BM;
                 if (!(ok = mbar_wait(&sm.bar[KB_QREADY + buf], (it_all >> 1) & 1, abort, 221))) break;
+                if (it == 0) {
+                    // the unit's scales, written by the prologue before this query tile's barrier
+                    vin = sm.vtinv[uu & 3];        // undoes the V tile scale of dP^T
+                    su = 1.0f / sm.uinv[uu & 3];   // 2^E: P^T columns carry 2^(E - e_i)
+                    dsc = sm.dsc[uu & 3][r];
+                }
                 if (!(ok = mbar_wait(&sm.bar[KB_SFULL], it_all & 1, abort, 222))) break;
                 tc_fence_after();
                 const int jmin = x.kt * TF_BN + 32 * wq, jmax = jmin + 31;
@@ -1047,14 +1039,14 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             }
         }
     } else if (warp >= 8 && warp < 12) {
-        // ================================================ prologue: K~, V (per unit), Q~ (per iteration)
+        // ================================================ prologue: unit scales, Q~ (per iteration)
         const int r = tid - 256, wq = warp - 8;
         int it_all = 0, uu = 0;
         bool ok = true;
-        for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
-            const UnitInfo x = decode_unit(L, u);
-            // unit statistics, max |dout| and max |Delta| over the rows this unit reads (global
-            // loads only: issued before any tile wait)
+        // Scales of unit x into ring slot `slot`: max |dout| and max |Delta| over the rows the
+        // unit reads (global loads only), the dA scale E, the dS^T row scales and the V tile
+        // scale.  Computed during the previous unit's last iteration, off the unit boundary.
+        auto unit_scales = [&](const UnitInfo& x, int slot) {
             float domx = 0.f, dlmx = 0.f;
 #pragma unroll 4
             for (int it = 0; it < x.nit; ++it) {
@@ -1083,22 +1075,19 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             // E = fit_exp(max domax) is the smallest row exponent of dA in the unit, so every
             // column factor 2^(E - e_i) of P^T is <= 1
             const int E = fit_exp(domx);
-            {
-                // unit scales for the softmax warps: V tile (prepared), dS^T rows, dA columns
-                const int j = x.kt * TF_BN + r, nkt = (L.S + TF_BN - 1) / TF_BN;
-                const float vnorm = j < L.S ? p.vnorm[((size_t)x.b * L.Hkv + x.kvh) * L.S + j] : 0.f;
-                // dS^T row scale: |dS_ji| <= |v_j| |dA_i| + |Delta_i| <= |v_j| sqrt(D) max|dout| + max|Delta|
-                sm.dsc[uu & 3][r] = ldexpf(1.0f, fit_exp(vnorm * sqrtf((float)kD) * domx + dlmx));
-                if (r == 0) {
-                    sm.uinv[uu & 3] = ldexpf(1.0f, -E);
-                    sm.vtinv[uu & 3] = p.vtinv[((size_t)x.b * L.Hkv + x.kvh) * nkt + x.kt];
-                }
-                mbar_arrive(&sm.bar[KB_KVREADY]);
+            const int j = x.kt * TF_BN + r, nkt = (L.S + TF_BN - 1) / TF_BN;
+            const float vnorm = j < L.S ? p.vnorm[((size_t)x.b * L.Hkv + x.kvh) * L.S + j] : 0.f;
+            // dS^T row scale: |dS_ji| <= |v_j| |dA_i| + |Delta_i| <= |v_j| sqrt(D) max|dout| + max|Delta|
+            sm.dsc[slot][r] = ldexpf(1.0f, fit_exp(vnorm * sqrtf((float)kD) * domx + dlmx));
+            if (r == 0) {
+                sm.uinv[slot] = ldexpf(1.0f, -E);
+                sm.vtinv[slot] = p.vtinv[((size_t)x.b * L.Hkv + x.kvh) * nkt + x.kt];
             }
-            // angles of the key tile's positions, which are also those of the query block of the
-            // first G iterations (qb = kt)
-            tf_angles(L, x.kt * TF_BN + r, sm.cs, r);
-            int cur_qb = x.kt;
+        };
+        if (u_begin < u_end) unit_scales(decode_unit(L, u_begin), 0);
+        int cur_qb = -1;  // query block whose positions the angle table holds
+        for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
+            const UnitInfo x = decode_unit(L, u);
             for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
                 const int buf = it_all & 1;
                 int qb, hg;
@@ -1117,6 +1106,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 sm.dcol[buf][r] = valid ? p.dainv[ro] : 0.f;
                 fence_proxy_async_smem();
                 mbar_arrive(&sm.bar[KB_QREADY + buf]);
+                if (it == x.nit - 1 && u + 1 < u_end) unit_scales(decode_unit(L, u + 1), (uu + 1) & 3);
             }
         }
     } else if (warp >= 12) {

@@ -252,20 +252,27 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
             for (int h = 0; h < G; ++h, ++m) {
                 if (!mbar_wait(&sm.bar[B_SFULL], m & 1, abort, 20)) { stop = true; break; }
                 tc_fence_after();
+                // this row's visible keys; a chunk fully visible to the warp's 32 rows needs no mask
+                const int klo = max(i - L.W + 1, 0), khi = min(i, L.S - 1);
+                auto chunk_full = [&](int kp0) {
+                    return kp0 + 31 <= imin && kp0 > imax - L.W && kp0 >= 0 && kp0 + 31 < L.S;
+                };
                 float mx = -INFINITY;
 #pragma unroll 1
                 for (int c8 = 0; c8 < 8; ++c8) {
                     const int kp0 = (c8 < 4 ? base0 : base1) + (c8 & 3) * 32;
                     const bool live = imin < L.S && kp0 <= imax && kp0 + 31 > imin - L.W && kp0 + 31 >= 0 && kp0 < L.S;
                     if (!live) continue;
-                    uint32_t v[32];
-                    tmem_ld32(TM_S + lane_off + 32 * c8, v);
+                    float v[32];
+                    tmem_ld32f(TM_S + lane_off + 32 * c8, v);
                     tmem_wait_ld();
+                    if (chunk_full(kp0)) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int j = kp0 + e;
-                        const bool vis = j <= i && j > i - L.W && j >= 0 && j < L.S;
-                        if (vis) mx = fmaxf(mx, __uint_as_float(v[e]));
+                        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
+                    } else {
+                        const uint32_t vm = bit_range(klo - kp0, khi - kp0);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, ((vm >> e) & 1u) ? v[e] : -INFINITY);
                     }
                 }
                 const float mu = (mx == -INFINITY) ? 0.f : mx * c2;
@@ -276,16 +283,15 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
                     const bool live = imin < L.S && kp0 <= imax && kp0 + 31 > imin - L.W && kp0 + 31 >= 0 && kp0 < L.S;
                     uint32_t pk[16];
                     if (live) {
-                        uint32_t v[32];
-                        tmem_ld32(TM_S + lane_off + 32 * c8, v);
+                        float v[32];
+                        tmem_ld32f(TM_S + lane_off + 32 * c8, v);
                         tmem_wait_ld();
+                        const uint32_t vm = chunk_full(kp0) ? 0xffffffffu : bit_range(klo - kp0, khi - kp0);
 #pragma unroll
                         for (int e = 0; e < 32; e += 2) {
-                            const int j = kp0 + e;
-                            const bool v0 = j <= i && j > i - L.W && j >= 0 && j < L.S;
-                            const bool v1 = j + 1 <= i && j + 1 > i - L.W && j + 1 >= 0 && j + 1 < L.S;
-                            const float p0 = v0 ? fast_exp2(__uint_as_float(v[e]) * c2 - mu) : 0.f;
-                            const float p1 = v1 ? fast_exp2(__uint_as_float(v[e + 1]) * c2 - mu) : 0.f;
+                            float p0 = fast_exp2(v[e] * c2 - mu), p1 = fast_exp2(v[e + 1] * c2 - mu);
+                            p0 = ((vm >> e) & 1u) ? p0 : 0.f;  // (a masked score may overflow: selected away)
+                            p1 = ((vm >> (e + 1)) & 1u) ? p1 : 0.f;
                             l += p0 + p1;
                             pk[e >> 1] = pack_bf16(p0, p1);
                         }

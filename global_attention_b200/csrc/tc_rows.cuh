@@ -55,6 +55,16 @@ __device__ __forceinline__ float qk_fp16_scale(const float* gq, const float* gk)
     return (bound > 16384.f && isfinite(bound)) ? ldexpf(1.0f, 13 - ilogbf(bound)) : 1.0f;
 }
 
+// Bits lo..hi of a 32-bit word, clamped to 0..31 (0 when the range is empty): the visible
+// positions of a 32-wide chunk for one thread's row.  A bit test and a select per element
+// replace the window comparisons, which compiled to divergent branches around the exp2.
+__device__ __forceinline__ uint32_t bit_range(int lo, int hi) {
+    lo = max(lo, 0);
+    hi = min(hi, 31);
+    if (lo > hi) return 0u;
+    return (0xffffffffu >> (31 - hi)) & (0xffffffffu << lo);
+}
+
 // ------------------------------------------------------------------ prologue (one row per thread)
 
 // cos/sin of the TF_HALF rotation angles at `pos`, into column r of the table
