@@ -1047,16 +1047,31 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
         // unit reads (global loads only), the dA scale E, the dS^T row scales and the V tile
         // scale.  Computed during the previous unit's last iteration, off the unit boundary.
         auto unit_scales = [&](const UnitInfo& x, int slot) {
+            // every global load of the unit's statistics is issued before any is used (one
+            // round trip instead of one per dependent batch)
+            const int j = x.kt * TF_BN + r, nkt = (L.S + TF_BN - 1) / TF_BN;
+            const float vnorm = j < L.S ? p.vnorm[((size_t)x.b * L.Hkv + x.kvh) * L.S + j] : 0.f;
+            const float vtile = p.vtinv[((size_t)x.b * L.Hkv + x.kvh) * nkt + x.kt];
             float domx = 0.f, dlmx = 0.f;
-#pragma unroll 4
-            for (int it = 0; it < x.nit; ++it) {
-                int qb, hg;
-                decode_iter(L, x, it, qb, hg);
-                const int i = qb * TF_BM + r;
-                if (i < L.S) {
-                    const size_t ro = ((size_t)x.b * L.Hq + hg) * L.S + i;
-                    domx = fmaxf(domx, p.domax[ro]);
-                    dlmx = fmaxf(dlmx, fabsf(p.P.delta[ro]));
+            for (int it0 = 0; it0 < x.nit; it0 += 8) {
+                float dm[8], dl[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    dm[k] = 0.f;
+                    dl[k] = 0.f;
+                    int qb, hg;
+                    decode_iter(L, x, it0 + k, qb, hg);
+                    const int i = qb * TF_BM + r;
+                    if (it0 + k < x.nit && i < L.S) {
+                        const size_t ro = ((size_t)x.b * L.Hq + hg) * L.S + i;
+                        dm[k] = p.domax[ro];
+                        dl[k] = p.P.delta[ro];
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    domx = fmaxf(domx, dm[k]);
+                    dlmx = fmaxf(dlmx, fabsf(dl[k]));
                 }
             }
 #pragma unroll
@@ -1075,13 +1090,11 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             // E = fit_exp(max domax) is the smallest row exponent of dA in the unit, so every
             // column factor 2^(E - e_i) of P^T is <= 1
             const int E = fit_exp(domx);
-            const int j = x.kt * TF_BN + r, nkt = (L.S + TF_BN - 1) / TF_BN;
-            const float vnorm = j < L.S ? p.vnorm[((size_t)x.b * L.Hkv + x.kvh) * L.S + j] : 0.f;
             // dS^T row scale: |dS_ji| <= |v_j| |dA_i| + |Delta_i| <= |v_j| sqrt(D) max|dout| + max|Delta|
             sm.dsc[slot][r] = ldexpf(1.0f, fit_exp(vnorm * sqrtf((float)kD) * domx + dlmx));
             if (r == 0) {
                 sm.uinv[slot] = ldexpf(1.0f, -E);
-                sm.vtinv[slot] = p.vtinv[((size_t)x.b * L.Hkv + x.kvh) * nkt + x.kt];
+                sm.vtinv[slot] = vtile;
             }
         };
         if (u_begin < u_end) unit_scales(decode_unit(L, u_begin), 0);
