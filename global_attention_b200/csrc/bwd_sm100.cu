@@ -45,11 +45,13 @@ struct BwdTcParams {
     CUtensorMap tm_da;  // dA16, fp16, same geometry as tm_q
     CUtensorMap tm_k16; // K~ fp16 (normalised, rotated, times the q~/k~ scale), geometry of tm_k
     CUtensorMap tm_v16; // V fp16 times 2^e per 128-row tile, geometry of tm_v
+    CUtensorMap tm_q16; // Q~ fp16 (normalised, rotated, times the q~/k~ scale), geometry of tm_q
     BwdParams P;
     const __half* da16; // [B,S,Hq,D] dA * 2^e (e per row)
     float* dainv;       // [B,Hq,S] 2^-e of each dA row (0 for an all-zero row)
     float* domax;       // [B,Hq,S] max |dout| of each row (bound on |dA|)
     float* krinv;       // [B,Hkv,S] inverse RMS of each raw k row
+    float* qrinv;       // [B,Hq,S] inverse RMS of each raw q row
     float* vnorm;       // [B,Hkv,S] 2-norm of each raw v row
     float* vtinv;       // [B,Hkv,ceil(S/128)] 2^-e of each V tile
     int* err;
@@ -292,7 +294,7 @@ __device__ __forceinline__ void row_rope_rms_backward_regs(float (&dy)[128], flo
 
 enum QBar {
     QB_KFULL = 0, QB_KEMPTY = 4, QB_VFULL = 6, QB_VEMPTY = 10,
-    QB_QFULL = 12, QB_QREADY = 13, QB_QEMPTY = 14, QB_DAEMPTY = 15,
+    QB_QFULL = 12, QB_QEMPTY = 14, QB_DAEMPTY = 15,
     QB_DSFULL = 17, QB_DQFULL = 18, QB_DQEMPTY = 19, QB_DONE = 20, QB_DAFULL = 21,
     QB_DPFULL = 22, QB_COUNT = 23
 };
@@ -300,13 +302,11 @@ enum QBar {
 struct BwdQTcSmem {
     alignas(1024) unsigned char K[2][TF_RING_HALF];    // K~ fp16, 2-slot ring split by d-half
     alignas(1024) unsigned char V[2][TF_RING_HALF];    // V fp16, row-scaled
-    alignas(1024) unsigned char Q[2][TF_HALF_BYTES];   // raw q -> Q~ fp16 in place
+    alignas(1024) unsigned char Q[2][TF_HALF_BYTES];   // Q~ fp16 (from the preparation kernel)
     alignas(1024) unsigned char dA[2][TF_HALF_BYTES];  // dA fp16, row-scaled (TMA from the gate pass)
-    float2 cs[TF_HALF][TF_BM];
     float gq[kD], gk[kD];
     float dsinv[2][TF_BM];   // 2^-e of each dS row, by head number % 2
     float mdot[2][TF_BM];    // mean(dy gamma xhat) of each row (RMSNorm backward), by head % 2
-    float qrinv[4][TF_BM];   // inverse RMS of each raw q row, by head number % 4
     float dgq[4][kD];        // this CTA's d_gamma_q, one slice per epilogue warp
     uint64_t bar[QB_COUNT];
     uint32_t tmem_base;
@@ -357,12 +357,12 @@ __device__ __forceinline__ float v_tile_to_f16(unsigned char* h0, unsigned char*
     return ldexpf(1.0f, -e);
 }
 
-// =====================================================================  K / V preparation
+// =====================================================================  Q / K / V preparation
 
 constexpr int KP_THREADS = 128;
 
-struct KvPrepSmem {
-    alignas(1024) unsigned char K[2][TF_HALF_BYTES];  // raw k -> K~ fp16 in place
+struct PrepSmem {
+    alignas(1024) unsigned char X[2][TF_HALF_BYTES];  // raw k or q -> K~ / Q~ fp16 in place
     alignas(1024) unsigned char V[2][TF_HALF_BYTES];  // raw v -> fp16 in place
     float2 cs[TF_HALF][TF_BM];
     float gq[kD], gk[kD];
@@ -370,19 +370,25 @@ struct KvPrepSmem {
     uint64_t bar;
 };
 
-// One CTA per 128-key tile (b, KV head, kt): K~ = fp16(RoPE(gamma_k * k / rms) * oscale) and
-// V * 2^e (one e per tile) into the workspace, with the same device functions the query-major
-// and key-major kernels once applied in their prologues, so every kernel sees the same bits.
-// Also saves each row's inverse RMS (RMSNorm backward of dk) and raw norm of v (dS^T scale).
-// The conversion used to sit on the critical path of both kernels at every new tile.
-__global__ void __launch_bounds__(KP_THREADS) bwd_kv_prep_kernel(const __grid_constant__ BwdTcParams p) {
+// One CTA per 128-row tile: the first B*Hkv*ceil(S/128) blocks take a key tile (b, KV head,
+// kt), the rest a query tile (b, query head, qb).  K~ = fp16(RoPE(gamma_k * k / rms) * oscale)
+// and V * 2^e (one e per tile), or Q~ likewise from q and gamma_q, go to the workspace; the
+// in-place conversion is the one the kernels once ran in their prologues (same device
+// functions, same bits).  Also saved: each row's inverse RMS (RMSNorm backward of dq, dk),
+// the raw norm of each v row (dS^T scale) and the V tile scale.  The conversions used to sit
+// on the critical path of both tcgen05 kernels.
+__global__ void __launch_bounds__(KP_THREADS) bwd_prep_kernel(const __grid_constant__ BwdTcParams p) {
     const LayerParams& L = p.P.L;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    KvPrepSmem& sm = *reinterpret_cast<KvPrepSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    PrepSmem& sm = *reinterpret_cast<PrepSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int r = threadIdx.x;
-    const int nkt = (L.S + TF_BN - 1) / TF_BN;
-    const int kt = blockIdx.x % nkt, chain = blockIdx.x / nkt;
-    const int kvh = chain % L.Hkv, b = chain / L.Hkv;
+    const int nt = (L.S + TF_BN - 1) / TF_BN;
+    const int n_k_tiles = L.B * L.Hkv * nt;
+    const bool is_k = (int)blockIdx.x < n_k_tiles;
+    const int tile = is_k ? (int)blockIdx.x : (int)blockIdx.x - n_k_tiles;
+    const int H = is_k ? L.Hkv : L.Hq;
+    const int t = tile % nt, chain = tile / nt;
+    const int h = chain % H, b = chain / H;
     volatile int abort = 0;
     if (r == 0) {
         mbar_init(&sm.bar, 1);
@@ -392,27 +398,34 @@ __global__ void __launch_bounds__(KP_THREADS) bwd_kv_prep_kernel(const __grid_co
     sm.gk[r] = L.gamma_k[r];
     __syncthreads();
     if (r == 0) {
-        mbar_expect_tx(&sm.bar, 2 * TF_TILE_BYTES);
-        tma_load_4d(sm.K[0], &p.tm_k, &sm.bar, 0, kvh, kt * TF_BN, b);
-        tma_load_4d(sm.K[1], &p.tm_k, &sm.bar, 64, kvh, kt * TF_BN, b);
-        tma_load_4d(sm.V[0], &p.tm_v, &sm.bar, 0, kvh, kt * TF_BN, b);
-        tma_load_4d(sm.V[1], &p.tm_v, &sm.bar, 64, kvh, kt * TF_BN, b);
+        const CUtensorMap* src = is_k ? &p.tm_k : &p.tm_q;
+        mbar_expect_tx(&sm.bar, (is_k ? 2 : 1) * TF_TILE_BYTES);
+        tma_load_4d(sm.X[0], src, &sm.bar, 0, h, t * TF_BN, b);
+        tma_load_4d(sm.X[1], src, &sm.bar, 64, h, t * TF_BN, b);
+        if (is_k) {
+            tma_load_4d(sm.V[0], &p.tm_v, &sm.bar, 0, h, t * TF_BN, b);
+            tma_load_4d(sm.V[1], &p.tm_v, &sm.bar, 64, h, t * TF_BN, b);
+        }
     }
-    const int j = kt * TF_BN + r;
-    tf_angles(L, j, sm.cs, r);
+    const int pos = t * TF_BN + r;
+    tf_angles(L, pos, sm.cs, r);
     const float oscale = qk_fp16_scale(sm.gq, sm.gk);
     // one decision for the whole CTA (the V conversion below has a CTA-wide barrier)
     const bool ok = __syncthreads_and(mbar_wait(&sm.bar, 0, &abort, 250)) != 0;
     if (ok) {
-        const float krinv = tf_prologue_row<true>(sm.K[0], sm.K[1], r, sm.gk, L, sm.cs, oscale);
-        float vn = 0.f;
-        const float vt = v_tile_to_f16(sm.V[0], sm.V[1], r, sm.vred, &vn);
-        if (j < L.S) {
-            const size_t ro = ((size_t)b * L.Hkv + kvh) * L.S + j;
-            p.krinv[ro] = krinv;
-            p.vnorm[ro] = vn;
+        const float rinv = tf_prologue_row<true>(sm.X[0], sm.X[1], r, is_k ? sm.gk : sm.gq, L, sm.cs, oscale);
+        const size_t ro = ((size_t)b * H + h) * L.S + pos;
+        if (is_k) {
+            float vn = 0.f;
+            const float vt = v_tile_to_f16(sm.V[0], sm.V[1], r, sm.vred, &vn);
+            if (pos < L.S) {
+                p.krinv[ro] = rinv;
+                p.vnorm[ro] = vn;
+            }
+            if (r == 0) p.vtinv[(size_t)chain * nt + t] = vt;
+        } else if (pos < L.S) {
+            p.qrinv[ro] = rinv;
         }
-        if (r == 0) p.vtinv[(size_t)chain * nkt + kt] = vt;
         fence_proxy_async_smem();
     } else if (r == 0) {
         mbar_wait_drain(&sm.bar, 0);  // the loads must land before the CTA exits
@@ -420,10 +433,13 @@ __global__ void __launch_bounds__(KP_THREADS) bwd_kv_prep_kernel(const __grid_co
     __syncthreads();
     if (r == 0) {
         if (ok) {
-            tma_store_4d(&p.tm_k16, sm.K[0], 0, kvh, kt * TF_BN, b);
-            tma_store_4d(&p.tm_k16, sm.K[1], 64, kvh, kt * TF_BN, b);
-            tma_store_4d(&p.tm_v16, sm.V[0], 0, kvh, kt * TF_BN, b);
-            tma_store_4d(&p.tm_v16, sm.V[1], 64, kvh, kt * TF_BN, b);
+            const CUtensorMap* dst = is_k ? &p.tm_k16 : &p.tm_q16;
+            tma_store_4d(dst, sm.X[0], 0, h, t * TF_BN, b);
+            tma_store_4d(dst, sm.X[1], 64, h, t * TF_BN, b);
+            if (is_k) {
+                tma_store_4d(&p.tm_v16, sm.V[0], 0, h, t * TF_BN, b);
+                tma_store_4d(&p.tm_v16, sm.V[1], 64, h, t * TF_BN, b);
+            }
             tma_store_commit();
             tma_store_wait_read();
         } else if (p.err) {
@@ -451,7 +467,6 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             mbar_init(&sm.bar[QB_VEMPTY + i], 1);
         }
         mbar_init(&sm.bar[QB_QFULL], 1);
-        mbar_init(&sm.bar[QB_QREADY], 128);
         mbar_init(&sm.bar[QB_QEMPTY], 1);
         mbar_init(&sm.bar[QB_DAEMPTY], 1);
         mbar_init(&sm.bar[QB_DAFULL], 1);
@@ -478,6 +493,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
         prefetch_tmap(&p.tm_da);
         prefetch_tmap(&p.tm_k16);
         prefetch_tmap(&p.tm_v16);
+        prefetch_tmap(&p.tm_q16);
     }
     tc_fence_before();
     __syncthreads();
@@ -494,10 +510,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
     const float mdot_f = c2 * kLn2 / (float)kD;
 
     // Registers by warpgroup (4 x 128 in all, set at the top of each role): TMA / MMA issue
-    // 64, softmax 128, prologue 128, epilogue 192 (it holds a whole dq~ row so that it can
-    // release TMEM before its arithmetic).  Fewer for the issue warps made them spill.
+    // 72, softmax 176, idle 24, epilogue 240 (it holds a whole dq~ row so that it can release
+    // TMEM before its arithmetic).  This split is the one without spills.
     if (warp < 4) {
-        reg_dealloc<64>();
+        reg_dealloc<72>();
         if (warp == 0) {
             // ================================================ K / V producer
             if (lane == 0) {
@@ -538,8 +554,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                         const int hg = st.kvh * G + h;
                         if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_QEMPTY], (m - 1) & 1, abort, 103))) break;
                         mbar_expect_tx(&sm.bar[QB_QFULL], TF_TILE_BYTES);
-                        tma_load_4d(sm.Q[0], &p.tm_q, &sm.bar[QB_QFULL], 0, hg, st.qb * TF_BM, st.b);
-                        tma_load_4d(sm.Q[1], &p.tm_q, &sm.bar[QB_QFULL], 64, hg, st.qb * TF_BM, st.b);
+                        tma_load_4d(sm.Q[0], &p.tm_q16, &sm.bar[QB_QFULL], 0, hg, st.qb * TF_BM, st.b);
+                        tma_load_4d(sm.Q[1], &p.tm_q16, &sm.bar[QB_QFULL], 64, hg, st.qb * TF_BM, st.b);
                         last = m;
                         if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_DAEMPTY], (m - 1) & 1, abort, 104))) break;
                         mbar_expect_tx(&sm.bar[QB_DAFULL], TF_TILE_BYTES);
@@ -575,7 +591,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                          mbar_wait(&sm.bar[QB_VFULL + (n_cur & 1)], (n_cur >> 1) & 1, abort, 113);
                     for (int h = 0; h < G && ok; ++h, ++m) {
                         const uint32_t tA = tm_half(m), tB = tm_half(m + 1);
-                        if (!(ok = mbar_wait(&sm.bar[QB_QREADY], m & 1, abort, 114))) break;
+                        if (!(ok = mbar_wait(&sm.bar[QB_QFULL], m & 1, abort, 114))) break;
                         tc_fence_after();
                         // S = Q~ K~^T -> tA  (its columns were last read by the softmax of head m-1,
                         // as dP, and by the epilogue of head m-2, both waited for already)
@@ -624,14 +640,16 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             }
         }
     } else if (warp >= 4 && warp < 8) {
+        reg_alloc<176>();
         // ================================================ Delta, dS (thread = query row)
         const int r = tid - 128, wq = warp - 4;
         const int nkt = (L.S + TF_BN - 1) / TF_BN;
         const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
-        int n_next = 0, n_prev = 0, n_cur = 0, m = 0;
+        int n_next = 0, n_cur = 0, m = 0;
         for (int t = t_begin; t < t_end; ++t) {
             const StepInfo st = decode_step(L, t, t_begin, t_end);
-            if (st.fresh) { n_prev = n_next++; n_cur = n_next++; } else { n_prev = n_cur; n_cur = n_next++; }
+            if (st.fresh) n_next++;  // the previous tile takes a ring slot of its own
+            n_cur = n_next++;
             const int q0 = st.qb * TF_BM, i = q0 + r;
             const int slot_cur = n_cur & 1;
             const int base0 = (slot_cur == 0 ? q0 : q0 - TF_BN), base1 = (slot_cur == 1 ? q0 : q0 - TF_BN);
@@ -718,22 +736,11 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             if (stop) break;
         }
     } else if (warp >= 8 && warp < 12) {
-        // ================================================ prologue: Q~ (fp16, in place)
-        const int r = tid - 256;
-        int m = 0;
-        bool ok = true;
-        for (int t = t_begin; t < t_end && ok; ++t) {
-            const StepInfo st = decode_step(L, t, t_begin, t_end);
-            tf_angles(L, st.qb * TF_BM + r, sm.cs, r);  // the step's query positions
-            for (int h = 0; h < G; ++h, ++m) {
-                if (!(ok = mbar_wait(&sm.bar[QB_QFULL], m & 1, abort, 132))) break;
-                sm.qrinv[m & 3][r] = tf_prologue_row<true>(sm.Q[0], sm.Q[1], r, sm.gq, L, sm.cs, oscale);
-                fence_proxy_async_smem();
-                mbar_arrive(&sm.bar[QB_QREADY]);
-            }
-        }
+        // (no prologue: Q~, K~ and V arrive converted from the preparation kernel; the
+        // warpgroup only hands its registers to the others)
+        reg_dealloc<24>();
     } else if (warp >= 12) {
-        reg_alloc<192>();
+        reg_alloc<240>();
         // ================================================ dq epilogue (thread = query row)
         const int r = tid - 384, wq = warp - 12;
         const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
@@ -746,6 +753,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             for (int h = 0; h < G; ++h, ++m) {
                 const int hg = st.kvh * G + h;
                 const size_t off = ((size_t)(st.b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hg) * kD;
+                const float rinv = valid ? p.qrinv[((size_t)st.b * L.Hq + hg) * L.S + i] : 0.f;
                 uint4 xv0[8];  // first half of the raw q row, in flight during the wait
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
@@ -760,7 +768,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                 tmem_ld32f(tq + 96, dy + 96);
                 tmem_wait_ld();
                 const float f = L.scale * sm.dsinv[m & 1][r] / oscale;
-                const float mdot = sm.mdot[m & 1][r], rinv = sm.qrinv[m & 3][r];
+                const float mdot = sm.mdot[m & 1][r];
                 tc_fence_before();
                 mbar_arrive(&sm.bar[QB_DQEMPTY]);  // dQ(m) is in registers: TMEM free for dP(m+1)
                 row_rope_rms_backward_regs(dy, f, mdot, rinv, xv0, L.q + off, p.P.dq + off, valid, i, sm.gq, sm.dgq[wq], L);
@@ -783,15 +791,15 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
 enum KBar {
     KB_KVFULL = 0, KB_KVEMPTY = 2,
     KB_QFULL = 3, KB_QREADY = 5, KB_QEMPTY = 7,
-    KB_SFULL = 9, KB_PFULL = 10, KB_DVKFULL = 11, KB_DVKEMPTY = 12, KB_DONE = 13, KB_COUNT = 14
+    KB_SFULL = 9, KB_PFULL = 11,  // by 64-query half (TMEM buffer)
+    KB_DVKFULL = 13, KB_DVKEMPTY = 14, KB_DONE = 15, KB_COUNT = 16
 };
 
 struct BwdKTcSmem {
     alignas(1024) unsigned char K[2][TF_HALF_BYTES];      // K~ fp16 of the unit's key tile
     alignas(1024) unsigned char V[2][TF_HALF_BYTES];      // V fp16, row-scaled
-    alignas(1024) unsigned char Q[2][2][TF_HALF_BYTES];   // [buffer][half] raw q -> Q~ fp16
+    alignas(1024) unsigned char Q[2][2][TF_HALF_BYTES];   // [buffer][half] Q~ fp16 (prepared)
     alignas(1024) unsigned char dA[2][2][TF_HALF_BYTES];  // [buffer][half] dA fp16, row-scaled (TMA)
-    float2 cs[TF_HALF][TF_BM];
     float gq[kD], gk[kD];
     float lse2[2][TF_BM];    // per query column of the buffer
     float delta[2][TF_BM];
@@ -846,8 +854,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             mbar_init(&sm.bar[KB_QREADY + i], 128);
             mbar_init(&sm.bar[KB_QEMPTY + i], 1);
         }
-        mbar_init(&sm.bar[KB_SFULL], 1);
-        mbar_init(&sm.bar[KB_PFULL], 128);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.bar[KB_SFULL + i], 1);
+            mbar_init(&sm.bar[KB_PFULL + i], 128);
+        }
         mbar_init(&sm.bar[KB_DVKFULL], 1);
         mbar_init(&sm.bar[KB_DVKEMPTY], 128);
         mbar_init(&sm.bar[KB_DONE], 1);
@@ -869,12 +879,16 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
         prefetch_tmap(&p.tm_da);
         prefetch_tmap(&p.tm_k16);
         prefetch_tmap(&p.tm_v16);
+        prefetch_tmap(&p.tm_q16);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t TM_S = tmem, TM_DP = tmem + 128, TM_P = tmem, TM_DS = tmem + 128, TM_DV = tmem + 256,
+    // TMEM: two 128-column buffers, one per 64-query half of an iteration: S^T in columns
+    // [0,64) and dP^T in [64,128) of the buffer, P^T and dS^T (fp16) over their first 32;
+    // dV and dK accumulators in [256,384) and [384,512).
+    const uint32_t TM_DV = tmem + 256,
                    TM_DK = tmem + 384;
     const float oscale = qk_fp16_scale(sm.gq, sm.gk);
     const float c2 = L.scale_log2 / (oscale * oscale);
@@ -905,8 +919,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                         int qb, hg;
                         decode_iter(L, x, it, qb, hg);
                         mbar_expect_tx(&sm.bar[KB_QFULL + buf], 2 * TF_TILE_BYTES);
-                        tma_load_4d(sm.Q[buf][0], &p.tm_q, &sm.bar[KB_QFULL + buf], 0, hg, qb * TF_BM, x.b);
-                        tma_load_4d(sm.Q[buf][1], &p.tm_q, &sm.bar[KB_QFULL + buf], 64, hg, qb * TF_BM, x.b);
+                        tma_load_4d(sm.Q[buf][0], &p.tm_q16, &sm.bar[KB_QFULL + buf], 0, hg, qb * TF_BM, x.b);
+                        tma_load_4d(sm.Q[buf][1], &p.tm_q16, &sm.bar[KB_QFULL + buf], 64, hg, qb * TF_BM, x.b);
                         tma_load_4d(sm.dA[buf][0], &p.tm_da, &sm.bar[KB_QFULL + buf], 0, hg, qb * TF_BM, x.b);
                         tma_load_4d(sm.dA[buf][1], &p.tm_da, &sm.bar[KB_QFULL + buf], 64, hg, qb * TF_BM, x.b);
                         last_q[buf] = it_all;
@@ -924,55 +938,98 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             }
         } else if (warp == 1) {
             // ================================================ MMA issuer
+            // Per 64-query half h (sweep order: unit, iteration, half), into TMEM buffer h % 2:
+            //   S(h):   S^T = K~ Q~_h^T, dP^T = V dA_h^T      (M = 128 keys, N = 64, K = d)
+            //   DVK(h): dV += P^T_h dA_h, dK~ += dS^T_h Q~_h  (K = 64 queries)
+            // issued as S(0) S(1) DVK(0) S(2) DVK(1) S(3) ...: the softmax of half h+1 runs while
+            // the tensor core does DVK(h) and S(h+2).
             if (lane == 0) {
-                constexpr uint32_t IDESC_KM = idesc_f16(128, 128, false);
+                constexpr uint32_t IDESC_S = idesc_f16(128, 64, false);
                 constexpr uint32_t IDESC_MN = idesc_f16(128, 128, true);
                 const uint32_t k_base = smem_u32(sm.K[0]), v_base = smem_u32(sm.V[0]);
                 const uint32_t q_base = smem_u32(sm.Q[0][0]), da_base = smem_u32(sm.dA[0][0]);
-                int it_all = 0, uu = 0;
-                bool ok = true;
-                for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
-                    const UnitInfo x = decode_unit(L, u);
-                    if (!(ok = mbar_wait(&sm.bar[KB_KVFULL], uu & 1, abort, 210))) break;
-                    for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
-                        const int buf = it_all & 1;
-                        const uint32_t qb_addr = q_base + buf * 2 * TF_HALF_BYTES, da_addr = da_base + buf * 2 * TF_HALF_BYTES;
-                        if (!(ok = mbar_wait(&sm.bar[KB_QREADY + buf], (it_all >> 1) & 1, abort, 211))) break;
-                        tc_fence_after();
-                        // S^T = K~ Q~^T, dP^T = V dA^T   (M = keys, N = queries, K = d)
-    #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t half = kk >> 2, within = (kk & 3) * 32;
-                            mma_ss(TM_S, sdesc_sw128(k_base + half * TF_HALF_BYTES + within, 16, 1024),
-                                   sdesc_sw128(qb_addr + half * TF_HALF_BYTES + within, 16, 1024), IDESC_KM, kk > 0 ? 1u : 0u);
-                        }
-    #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t half = kk >> 2, within = (kk & 3) * 32;
-                            mma_ss(TM_DP, sdesc_sw128(v_base + half * TF_HALF_BYTES + within, 16, 1024),
-                                   sdesc_sw128(da_addr + half * TF_HALF_BYTES + within, 16, 1024), IDESC_KM, kk > 0 ? 1u : 0u);
-                        }
-                        mma_commit(&sm.bar[KB_SFULL]);
-                        if (!(ok = mbar_wait(&sm.bar[KB_PFULL], it_all & 1, abort, 212))) break;
-                        if (it == 0 && uu >= 1 && !(ok = mbar_wait(&sm.bar[KB_DVKEMPTY], (uu - 1) & 1, abort, 213))) break;
-                        tc_fence_after();
-                        // dV += P^T dA ; dK~ += dS^T Q~  (A from TMEM: 16 queries = 8 columns per step;
-                        // B = dA / Q~ MN-major: N = d, K = queries)
-    #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint64_t bda = sdesc_sw128(da_addr + kk * 16 * 128, TF_HALF_BYTES, 1024);
-                            mma_ts(TM_DV, TM_P + kk * 8, bda, IDESC_MN, (it > 0 || kk > 0) ? 1u : 0u);
-                        }
-    #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint64_t bq = sdesc_sw128(qb_addr + kk * 16 * 128, TF_HALF_BYTES, 1024);
-                            mma_ts(TM_DK, TM_DS + kk * 8, bq, IDESC_MN, (it > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        mma_commit(&sm.bar[KB_QEMPTY + buf]);
+                struct Cursor {
+                    int u, uu, it, it_all, half;
+                    UnitInfo x;
+                    bool valid;
+                };
+                auto cur_first = [&]() {
+                    Cursor c{u_begin, 0, 0, 0, 0, UnitInfo{}, u_begin < u_end};
+                    if (c.valid) c.x = decode_unit(L, c.u);
+                    return c;
+                };
+                auto cur_next = [&](Cursor& c) {
+                    if (++c.half < 2) return;
+                    c.half = 0;
+                    ++c.it_all;
+                    if (++c.it < c.x.nit) return;
+                    c.it = 0;
+                    ++c.uu;
+                    if (++c.u < u_end) c.x = decode_unit(L, c.u);
+                    else c.valid = false;
+                };
+                auto last_of_unit = [](const Cursor& c) { return c.half == 1 && c.it == c.x.nit - 1; };
+                auto issue_s = [&](const Cursor& c) -> bool {
+                    const int buf = c.it_all & 1;
+                    if (c.it == 0 && c.half == 0 && !mbar_wait(&sm.bar[KB_KVFULL], c.uu & 1, abort, 210)) return false;
+                    if (c.half == 0 && !mbar_wait(&sm.bar[KB_QFULL + buf], (c.it_all >> 1) & 1, abort, 211)) return false;
+                    tc_fence_after();
+                    const uint32_t tX = tmem + 128u * (uint32_t)c.half;
+                    const uint32_t rows = (uint32_t)c.half * 64u * 128u;  // first query row of the half
+                    const uint32_t qa = q_base + buf * 2 * TF_HALF_BYTES + rows, da = da_base + buf * 2 * TF_HALF_BYTES + rows;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t dh = kk >> 2, within = (kk & 3) * 32;
+                        mma_ss(tX, sdesc_sw128(k_base + dh * TF_HALF_BYTES + within, 16, 1024),
+                               sdesc_sw128(qa + dh * TF_HALF_BYTES + within, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
                     }
-                    if (!ok) break;
-                    mma_commit(&sm.bar[KB_DVKFULL]);
-                    mma_commit(&sm.bar[KB_KVEMPTY]);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t dh = kk >> 2, within = (kk & 3) * 32;
+                        mma_ss(tX + 64, sdesc_sw128(v_base + dh * TF_HALF_BYTES + within, 16, 1024),
+                               sdesc_sw128(da + dh * TF_HALF_BYTES + within, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&sm.bar[KB_SFULL + c.half]);
+                    if (last_of_unit(c)) mma_commit(&sm.bar[KB_KVEMPTY]);  // K, V read for the last time
+                    return true;
+                };
+                auto issue_dvk = [&](const Cursor& c) -> bool {
+                    const int buf = c.it_all & 1;
+                    if (!mbar_wait(&sm.bar[KB_PFULL + c.half], c.it_all & 1, abort, 212)) return false;
+                    if (c.it == 0 && c.half == 0 && c.uu >= 1 &&
+                        !mbar_wait(&sm.bar[KB_DVKEMPTY], (c.uu - 1) & 1, abort, 213))
+                        return false;
+                    tc_fence_after();
+                    const uint32_t tX = tmem + 128u * (uint32_t)c.half;
+                    const uint32_t rows = (uint32_t)c.half * 64u * 128u;
+                    const uint32_t qa = q_base + buf * 2 * TF_HALF_BYTES + rows, da = da_base + buf * 2 * TF_HALF_BYTES + rows;
+                    const bool first = c.it == 0 && c.half == 0;
+                    // A from TMEM (16 queries = 8 columns per step); B = dA / Q~ MN-major (N = d)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(TM_DV, tX + kk * 8, sdesc_sw128(da + kk * 16 * 128, TF_HALF_BYTES, 1024), IDESC_MN,
+                               (!first || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(TM_DK, tX + 64 + kk * 8, sdesc_sw128(qa + kk * 16 * 128, TF_HALF_BYTES, 1024), IDESC_MN,
+                               (!first || kk > 0) ? 1u : 0u);
+                    if (c.half == 1) mma_commit(&sm.bar[KB_QEMPTY + buf]);
+                    if (last_of_unit(c)) mma_commit(&sm.bar[KB_DVKFULL]);
+                    return true;
+                };
+                Cursor cs_ = cur_first(), cd = cur_first();
+                bool ok = true;
+                for (int n = 0; n < 2 && ok && cs_.valid; ++n) {
+                    ok = issue_s(cs_);
+                    cur_next(cs_);
+                }
+                while (ok && cd.valid) {
+                    ok = issue_dvk(cd);
+                    if (ok && cs_.valid) {
+                        ok = issue_s(cs_);
+                        cur_next(cs_);
+                    }
+                    cur_next(cd);
                 }
                 mma_commit(&sm.bar[KB_DONE]);
                 mbar_wait(&sm.bar[KB_DONE], 0, abort, 214);
@@ -1001,45 +1058,48 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                     su = 1.0f / sm.uinv[uu & 3];   // 2^E: P^T columns carry 2^(E - e_i)
                     dsc = sm.dsc[uu & 3][r];
                 }
-                if (!(ok = mbar_wait(&sm.bar[KB_SFULL], it_all & 1, abort, 222))) break;
-                tc_fence_after();
                 const int jmin = x.kt * TF_BN + 32 * wq, jmax = jmin + 31;
+                for (int half = 0; half < 2 && ok; ++half) {
+                    // 64-query half in TMEM buffer `half`: S^T at columns [0,64), dP^T at [64,128)
+                    if (!(ok = mbar_wait(&sm.bar[KB_SFULL + half], it_all & 1, abort, 222))) break;
+                    tc_fence_after();
+                    const uint32_t tX = tmem + 128u * (uint32_t)half + lane_off;
 #pragma unroll 1
-                for (int c8 = 0; c8 < 4; ++c8) {
-                    const int i0 = q0 + 32 * c8;  // queries of this chunk: i0 .. i0+31
-                    const bool live = jmin < L.S && i0 < L.S && i0 + 31 >= jmin && i0 <= jmax + L.W - 1;
-                    const bool full = jmax <= i0 && jmin > i0 + 31 - L.W && i0 + 31 < L.S && jmax < L.S;
-                    uint32_t pp[16], dd[16];
-                    if (live) {
-                        float sv[32], dv[32];
-                        tmem_ld32f(TM_S + lane_off + 32 * c8, sv);
-                        tmem_ld32f(TM_DP + lane_off + 32 * c8, dv);
-                        tmem_wait_ld();
-                        const int ql0 = 32 * c8;
-                        if (full) {
-                            kv_chunk<true>(sv, dv, sm.lse2[buf] + ql0, sm.delta[buf] + ql0, sm.dcol[buf] + ql0, 0u, vin,
-                                           su, dsc, c2, pp, dd, kacc);
+                    for (int c8 = 0; c8 < 2; ++c8) {
+                        const int ql0 = 64 * half + 32 * c8, i0 = q0 + ql0;  // queries i0 .. i0+31
+                        const bool live = jmin < L.S && i0 < L.S && i0 + 31 >= jmin && i0 <= jmax + L.W - 1;
+                        const bool full = jmax <= i0 && jmin > i0 + 31 - L.W && i0 + 31 < L.S && jmax < L.S;
+                        uint32_t pp[16], dd[16];
+                        if (live) {
+                            float sv[32], dv[32];
+                            tmem_ld32f(tX + 32 * c8, sv);
+                            tmem_ld32f(tX + 64 + 32 * c8, dv);
+                            tmem_wait_ld();
+                            if (full) {
+                                kv_chunk<true>(sv, dv, sm.lse2[buf] + ql0, sm.delta[buf] + ql0, sm.dcol[buf] + ql0, 0u,
+                                               vin, su, dsc, c2, pp, dd, kacc);
+                            } else {
+                                // queries that see key j: j <= i <= min(j + W - 1, S - 1)
+                                const uint32_t vm = j < L.S ? bit_range(j - i0, min(j + L.W - 1, L.S - 1) - i0) : 0u;
+                                kv_chunk<false>(sv, dv, sm.lse2[buf] + ql0, sm.delta[buf] + ql0, sm.dcol[buf] + ql0, vm,
+                                                vin, su, dsc, c2, pp, dd, kacc);
+                            }
                         } else {
-                            // queries that see key j: j <= i <= min(j + W - 1, S - 1)
-                            const uint32_t vm = j < L.S ? bit_range(j - i0, min(j + L.W - 1, L.S - 1) - i0) : 0u;
-                            kv_chunk<false>(sv, dv, sm.lse2[buf] + ql0, sm.delta[buf] + ql0, sm.dcol[buf] + ql0, vm, vin,
-                                            su, dsc, c2, pp, dd, kacc);
-                        }
-                    } else {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) pp[e] = dd[e] = 0u;
+                            for (int e = 0; e < 16; ++e) pp[e] = dd[e] = 0u;
+                        }
+                        tmem_st16(tX + 16 * c8, pp);       // P^T over S^T (already read)
+                        tmem_st16(tX + 64 + 16 * c8, dd);  // dS^T over dP^T
                     }
-                    tmem_st16(TM_P + lane_off + 16 * c8, pp);
-                    tmem_st16(TM_DS + lane_off + 16 * c8, dd);
+                    if (half == 1 && it == x.nit - 1) sm.kmdot[uu & 1][r] = kacc * mdot_f;
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&sm.bar[KB_PFULL + half]);
                 }
-                if (it == x.nit - 1) sm.kmdot[uu & 1][r] = kacc * mdot_f;
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&sm.bar[KB_PFULL]);
             }
         }
     } else if (warp >= 8 && warp < 12) {
-        // ================================================ prologue: unit scales, Q~ (per iteration)
+        // ================================================ prologue: unit scales, per-column values
         const int r = tid - 256, wq = warp - 8;
         int it_all = 0, uu = 0;
         bool ok = true;
@@ -1098,7 +1158,6 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             }
         };
         if (u_begin < u_end) unit_scales(decode_unit(L, u_begin), 0);
-        int cur_qb = -1;  // query block whose positions the angle table holds
         for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
             const UnitInfo x = decode_unit(L, u);
             for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
@@ -1107,17 +1166,13 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 decode_iter(L, x, it, qb, hg);
                 const int i = qb * TF_BM + r;
                 const bool valid = i < L.S;
+                // (the wait keeps these per-column values from overwriting those of iteration
+                // it - 2 before its products are done: the buffer's tiles land only after that)
                 if (!(ok = mbar_wait(&sm.bar[KB_QFULL + buf], (it_all >> 1) & 1, abort, 231))) break;
-                if (qb != cur_qb) {
-                    tf_angles(L, i, sm.cs, r);
-                    cur_qb = qb;
-                }
-                tf_prologue_row<true>(sm.Q[buf][0], sm.Q[buf][1], r, sm.gq, L, sm.cs, oscale);
                 const size_t ro = ((size_t)x.b * L.Hq + hg) * L.S + (valid ? i : 0);
                 sm.lse2[buf][r] = valid ? p.P.lse[ro] * kLog2e : INFINITY;  // the forward's, base 2
                 sm.delta[buf][r] = valid ? p.P.delta[ro] : 0.f;
                 sm.dcol[buf][r] = valid ? p.dainv[ro] : 0.f;
-                fence_proxy_async_smem();
                 mbar_arrive(&sm.bar[KB_QREADY + buf]);
                 if (it == x.nit - 1 && u + 1 < u_end) unit_scales(decode_unit(L, u + 1), (uu + 1) & 3);
             }
@@ -1212,7 +1267,7 @@ bool make_map_b(CUtensorMap* map, const void* base, int H, int S, int B,
 
 }  // namespace
 
-extern const char* const kBwdTcKernelNames[] = {"bwd_gate_kernel",         "bwd_kv_prep_kernel",
+extern const char* const kBwdTcKernelNames[] = {"bwd_gate_kernel",         "bwd_prep_kernel",
                                                 "bwd_q_tc_kernel",         "bwd_kv_tc_kernel",
                                                 "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"};
 extern const int kBwdTcKernelCount = 6;
@@ -1223,14 +1278,14 @@ bool bwd_tc_supported(const LayerParams& L) {
     return L.W <= TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1 && get_encode_b() != nullptr;
 }
 
-// workspace of the tcgen05 backward: delta, domax, dainv [B,Hq,S] fp32; dA16 [B,S,Hq,D]
-// fp16; K~16, V16 [B,S,Hkv,D] fp16; krinv, vnorm [B,Hkv,S] fp32; vtinv per V tile; 2 x
-// d_gamma partials
+// workspace of the tcgen05 backward: delta, domax, dainv, qrinv [B,Hq,S] fp32; dA16, Q~16
+// [B,S,Hq,D] fp16; K~16, V16 [B,S,Hkv,D] fp16; krinv, vnorm [B,Hkv,S] fp32; vtinv per V
+// tile; 2 x d_gamma partials
 size_t bwd_tc_workspace_bytes(int B, int S, int Hq, int Hkv) {
     const size_t rows = (size_t)B * S * Hq, krows = (size_t)B * S * Hkv;
     const size_t tiles = (size_t)B * Hkv * ((S + TF_BN - 1) / TF_BN);
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
-    return 3 * a(rows * sizeof(float)) + a(rows * kD * sizeof(__half)) + 2 * a(krows * kD * sizeof(__half)) +
+    return 4 * a(rows * sizeof(float)) + 2 * a(rows * kD * sizeof(__half)) + 2 * a(krows * kD * sizeof(__half)) +
            2 * a(krows * sizeof(float)) + a(tiles * sizeof(float)) + 2 * a((size_t)TB_MAX_GRID * kD * sizeof(float));
 }
 
@@ -1254,6 +1309,8 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     p.dainv = reinterpret_cast<float*>(take(rows * 4));
     __half* da16 = reinterpret_cast<__half*>(take(rows * kD * sizeof(__half)));
     p.da16 = da16;
+    void* q16 = take(rows * kD * sizeof(__half));
+    p.qrinv = reinterpret_cast<float*>(take(rows * 4));
     const size_t krows = (size_t)L.B * L.S * L.Hkv;
     const int nkt = (L.S + TF_BN - 1) / TF_BN;
     void* k16 = take(krows * kD * sizeof(__half));
@@ -1268,7 +1325,8 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
         !make_map_b(&p.tm_v, L.v, L.Hkv, L.S, L.B) ||
         !make_map_b(&p.tm_da, da16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
         !make_map_b(&p.tm_k16, k16, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-        !make_map_b(&p.tm_v16, v16, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        !make_map_b(&p.tm_v16, v16, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+        !make_map_b(&p.tm_q16, q16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1298,18 +1356,18 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     const long long half_warps = ((long long)rows + GATE_UNROLL - 1) / GATE_UNROLL;
     const long long gate_need = (half_warps * 16 + GATE_THREADS - 1) / GATE_THREADS;
     const int gate_grid = (int)(gate_need < 2LL * sms ? gate_need : 2LL * sms);
-    const size_t smem_p = sizeof(KvPrepSmem) + 1024;
-    if ((e = cudaFuncSetAttribute(bwd_kv_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p)) !=
+    const size_t smem_p = sizeof(PrepSmem) + 1024;
+    if ((e = cudaFuncSetAttribute(bwd_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p)) !=
         cudaSuccess)
         return e;
-    const long long kv_tiles = (long long)L.B * L.Hkv * nkt;
-    if (kv_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const long long prep_tiles = (long long)L.B * (L.Hkv + L.Hq) * nkt;  // key tiles, then query tiles
+    if (prep_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
     if ((e = before(0)) != cudaSuccess) return e;
     bwd_gate_kernel<<<gate_grid, GATE_THREADS, 0, stream>>>(bp.dout, L.g, bp.out, bp.dg, da16, p.dainv, p.domax,
                                                             (long long)rows, L.S, L.Hq);
     if ((e = after(0)) != cudaSuccess) return e;
     if ((e = before(1)) != cudaSuccess) return e;
-    bwd_kv_prep_kernel<<<(int)kv_tiles, KP_THREADS, smem_p, stream>>>(p);
+    bwd_prep_kernel<<<(int)prep_tiles, KP_THREADS, smem_p, stream>>>(p);
     if ((e = after(1)) != cudaSuccess) return e;
     if ((e = before(2)) != cudaSuccess) return e;
     bwd_q_tc_kernel<<<grid, TB_THREADS, smem_q, stream>>>(p);
