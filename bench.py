@@ -77,8 +77,9 @@ def work(B, S, W, bwd):
         # q, k, v, dA16, 2^-e -> dq, lse, Delta ; S, dP, dQ  |
         # q, k, v, dA16, 4 row stats -> dk, dv ; S, dP, dV, dK
         "bwd_gate_kernel": (5 * qb + 2 * lse, 0),
-        # q, k, v -> Q~, K~, V fp16 (+ per-row inverse RMS, v norm, per-tile V scale)
-        "bwd_prep_kernel": (2 * qb + 4 * kb + qb // D + kb // D, 0),
+        # k, v -> K~, V fp16 (+ per-row inverse RMS and v norm, per-tile V scale); q -> Q~ fp16
+        "bwd_prep_kv_kernel": (4 * kb + kb // D, 0),
+        "bwd_prep_q_kernel": (2 * qb + qb // (2 * D), 0),
         "bwd_q_tc_kernel": (qb + 2 * kb + qb + qb + 3 * lse, 6 * D * npair),
         "bwd_kv_tc_kernel": (qb + 2 * kb + qb + 4 * lse + 2 * kb, 8 * D * npair),
     }

@@ -361,33 +361,32 @@ __device__ __forceinline__ float v_tile_to_f16(unsigned char* h0, unsigned char*
 
 constexpr int KP_THREADS = 128;
 
+template <bool IS_K>
 struct PrepSmem {
-    alignas(1024) unsigned char X[2][TF_HALF_BYTES];  // raw k or q -> K~ / Q~ fp16 in place
-    alignas(1024) unsigned char V[2][TF_HALF_BYTES];  // raw v -> fp16 in place
-    float2 cs[TF_HALF][TF_BM];
+    alignas(1024) unsigned char X[2][TF_HALF_BYTES];                 // raw k or q -> K~ / Q~ in place
+    alignas(1024) unsigned char V[IS_K ? 2 : 1][IS_K ? TF_HALF_BYTES : 16];  // raw v -> fp16 in place
     float gq[kD], gk[kD];
     float vred[4];
     uint64_t bar;
 };
 
-// One CTA per 128-row tile: the first B*Hkv*ceil(S/128) blocks take a key tile (b, KV head,
-// kt), the rest a query tile (b, query head, qb).  K~ = fp16(RoPE(gamma_k * k / rms) * oscale)
-// and V * 2^e (one e per tile), or Q~ likewise from q and gamma_q, go to the workspace; the
-// in-place conversion is the one the kernels once ran in their prologues (same device
-// functions, same bits).  Also saved: each row's inverse RMS (RMSNorm backward of dq, dk),
-// the raw norm of each v row (dS^T scale) and the V tile scale.  The conversions used to sit
-// on the critical path of both tcgen05 kernels.
-__global__ void __launch_bounds__(KP_THREADS) bwd_prep_kernel(const __grid_constant__ BwdTcParams p) {
+// One CTA per 128-row tile (b, head, t): a key tile (IS_K: K~ and V) or a query tile (Q~).
+// K~ = fp16(RoPE(gamma_k * k / rms) * oscale) and V * 2^e (one e per tile), or Q~ likewise
+// from q and gamma_q, go to the workspace; the in-place conversion is the one the kernels
+// once ran in their prologues (same device functions and angle values, same bits; the
+// angles sit in registers here).  Also saved: each row's inverse RMS (RMSNorm backward of dq,
+// dk), the raw norm of each v row (dS^T scale) and the V tile scale.  Several CTAs per SM keep
+// tile loads, conversions and stores of different tiles in flight.
+template <bool IS_K>
+__device__ __forceinline__ void prep_tile(const BwdTcParams& p) {
     const LayerParams& L = p.P.L;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    PrepSmem& sm = *reinterpret_cast<PrepSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    PrepSmem<IS_K>& sm =
+        *reinterpret_cast<PrepSmem<IS_K>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int r = threadIdx.x;
     const int nt = (L.S + TF_BN - 1) / TF_BN;
-    const int n_k_tiles = L.B * L.Hkv * nt;
-    const bool is_k = (int)blockIdx.x < n_k_tiles;
-    const int tile = is_k ? (int)blockIdx.x : (int)blockIdx.x - n_k_tiles;
-    const int H = is_k ? L.Hkv : L.Hq;
-    const int t = tile % nt, chain = tile / nt;
+    const int H = IS_K ? L.Hkv : L.Hq;
+    const int t = (int)blockIdx.x % nt, chain = (int)blockIdx.x / nt;
     const int h = chain % H, b = chain / H;
     volatile int abort = 0;
     if (r == 0) {
@@ -398,24 +397,27 @@ __global__ void __launch_bounds__(KP_THREADS) bwd_prep_kernel(const __grid_const
     sm.gk[r] = L.gamma_k[r];
     __syncthreads();
     if (r == 0) {
-        const CUtensorMap* src = is_k ? &p.tm_k : &p.tm_q;
-        mbar_expect_tx(&sm.bar, (is_k ? 2 : 1) * TF_TILE_BYTES);
+        const CUtensorMap* src = IS_K ? &p.tm_k : &p.tm_q;
+        mbar_expect_tx(&sm.bar, (IS_K ? 2 : 1) * TF_TILE_BYTES);
         tma_load_4d(sm.X[0], src, &sm.bar, 0, h, t * TF_BN, b);
         tma_load_4d(sm.X[1], src, &sm.bar, 64, h, t * TF_BN, b);
-        if (is_k) {
+        if constexpr (IS_K) {
             tma_load_4d(sm.V[0], &p.tm_v, &sm.bar, 0, h, t * TF_BN, b);
             tma_load_4d(sm.V[1], &p.tm_v, &sm.bar, 64, h, t * TF_BN, b);
         }
     }
     const int pos = t * TF_BN + r;
-    tf_angles(L, pos, sm.cs, r);
+    float2 csr[TF_HALF];  // (cos, sin) of the rotated pairs at this row's position
+#pragma unroll
+    for (int q = 0; q < TF_HALF; ++q) rope_cs(L.theta[q], pos, csr[q].x, csr[q].y);
     const float oscale = qk_fp16_scale(sm.gq, sm.gk);
     // one decision for the whole CTA (the V conversion below has a CTA-wide barrier)
     const bool ok = __syncthreads_and(mbar_wait(&sm.bar, 0, &abort, 250)) != 0;
     if (ok) {
-        const float rinv = tf_prologue_row<true>(sm.X[0], sm.X[1], r, is_k ? sm.gk : sm.gq, L, sm.cs, oscale);
+        const float rinv = tf_prologue_row_at<true>(sm.X[0], sm.X[1], r, IS_K ? sm.gk : sm.gq, L,
+                                                    [&](int q) { return csr[q]; }, oscale);
         const size_t ro = ((size_t)b * H + h) * L.S + pos;
-        if (is_k) {
+        if constexpr (IS_K) {
             float vn = 0.f;
             const float vt = v_tile_to_f16(sm.V[0], sm.V[1], r, sm.vred, &vn);
             if (pos < L.S) {
@@ -423,8 +425,8 @@ __global__ void __launch_bounds__(KP_THREADS) bwd_prep_kernel(const __grid_const
                 p.vnorm[ro] = vn;
             }
             if (r == 0) p.vtinv[(size_t)chain * nt + t] = vt;
-        } else if (pos < L.S) {
-            p.qrinv[ro] = rinv;
+        } else {
+            if (pos < L.S) p.qrinv[ro] = rinv;
         }
         fence_proxy_async_smem();
     } else if (r == 0) {
@@ -433,10 +435,10 @@ __global__ void __launch_bounds__(KP_THREADS) bwd_prep_kernel(const __grid_const
     __syncthreads();
     if (r == 0) {
         if (ok) {
-            const CUtensorMap* dst = is_k ? &p.tm_k16 : &p.tm_q16;
+            const CUtensorMap* dst = IS_K ? &p.tm_k16 : &p.tm_q16;
             tma_store_4d(dst, sm.X[0], 0, h, t * TF_BN, b);
             tma_store_4d(dst, sm.X[1], 64, h, t * TF_BN, b);
-            if (is_k) {
+            if constexpr (IS_K) {
                 tma_store_4d(&p.tm_v16, sm.V[0], 0, h, t * TF_BN, b);
                 tma_store_4d(&p.tm_v16, sm.V[1], 64, h, t * TF_BN, b);
             }
@@ -446,6 +448,13 @@ __global__ void __launch_bounds__(KP_THREADS) bwd_prep_kernel(const __grid_const
             atomicExch(p.err, 250);
         }
     }
+}
+
+__global__ void __launch_bounds__(KP_THREADS, 3) bwd_prep_kv_kernel(const __grid_constant__ BwdTcParams p) {
+    prep_tile<true>(p);
+}
+__global__ void __launch_bounds__(KP_THREADS, 4) bwd_prep_q_kernel(const __grid_constant__ BwdTcParams p) {
+    prep_tile<false>(p);
 }
 
 __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_constant__ BwdTcParams p) {
@@ -1267,10 +1276,11 @@ bool make_map_b(CUtensorMap* map, const void* base, int H, int S, int B,
 
 }  // namespace
 
-extern const char* const kBwdTcKernelNames[] = {"bwd_gate_kernel",         "bwd_prep_kernel",
-                                                "bwd_q_tc_kernel",         "bwd_kv_tc_kernel",
-                                                "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"};
-extern const int kBwdTcKernelCount = 6;
+extern const char* const kBwdTcKernelNames[] = {"bwd_gate_kernel",         "bwd_prep_kv_kernel",
+                                                "bwd_prep_q_kernel",       "bwd_q_tc_kernel",
+                                                "bwd_kv_tc_kernel",        "dgamma_reduce_kernel(k)",
+                                                "dgamma_reduce_kernel(q)"};
+extern const int kBwdTcKernelCount = 7;
 
 __global__ void dgamma_reduce_kernel(const float* __restrict__ parts, int n, float* __restrict__ out);
 
@@ -1356,31 +1366,38 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     const long long half_warps = ((long long)rows + GATE_UNROLL - 1) / GATE_UNROLL;
     const long long gate_need = (half_warps * 16 + GATE_THREADS - 1) / GATE_THREADS;
     const int gate_grid = (int)(gate_need < 2LL * sms ? gate_need : 2LL * sms);
-    const size_t smem_p = sizeof(PrepSmem) + 1024;
-    if ((e = cudaFuncSetAttribute(bwd_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p)) !=
+    const size_t smem_pk = sizeof(PrepSmem<true>) + 1024, smem_pq = sizeof(PrepSmem<false>) + 1024;
+    if ((e = cudaFuncSetAttribute(bwd_prep_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_pk)) !=
         cudaSuccess)
         return e;
-    const long long prep_tiles = (long long)L.B * (L.Hkv + L.Hq) * nkt;  // key tiles, then query tiles
-    if (prep_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
-    if ((e = before(0)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(bwd_prep_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_pq)) !=
+        cudaSuccess)
+        return e;
+    const long long k_tiles = (long long)L.B * L.Hkv * nkt, q_tiles = (long long)L.B * L.Hq * nkt;
+    if (q_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+    int i = 0;
+    if ((e = before(i)) != cudaSuccess) return e;
     bwd_gate_kernel<<<gate_grid, GATE_THREADS, 0, stream>>>(bp.dout, L.g, bp.out, bp.dg, da16, p.dainv, p.domax,
                                                             (long long)rows, L.S, L.Hq);
-    if ((e = after(0)) != cudaSuccess) return e;
-    if ((e = before(1)) != cudaSuccess) return e;
-    bwd_prep_kernel<<<(int)prep_tiles, KP_THREADS, smem_p, stream>>>(p);
-    if ((e = after(1)) != cudaSuccess) return e;
-    if ((e = before(2)) != cudaSuccess) return e;
+    if ((e = after(i++)) != cudaSuccess) return e;
+    if ((e = before(i)) != cudaSuccess) return e;
+    bwd_prep_kv_kernel<<<(int)k_tiles, KP_THREADS, smem_pk, stream>>>(p);
+    if ((e = after(i++)) != cudaSuccess) return e;
+    if ((e = before(i)) != cudaSuccess) return e;
+    bwd_prep_q_kernel<<<(int)q_tiles, KP_THREADS, smem_pq, stream>>>(p);
+    if ((e = after(i++)) != cudaSuccess) return e;
+    if ((e = before(i)) != cudaSuccess) return e;
     bwd_q_tc_kernel<<<grid, TB_THREADS, smem_q, stream>>>(p);
-    if ((e = after(2)) != cudaSuccess) return e;
-    if ((e = before(3)) != cudaSuccess) return e;
+    if ((e = after(i++)) != cudaSuccess) return e;
+    if ((e = before(i)) != cudaSuccess) return e;
     bwd_kv_tc_kernel<<<grid, TB_THREADS, smem_k, stream>>>(p);
-    if ((e = after(3)) != cudaSuccess) return e;
-    if ((e = before(4)) != cudaSuccess) return e;
+    if ((e = after(i++)) != cudaSuccess) return e;
+    if ((e = before(i)) != cudaSuccess) return e;
     dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgk_part, grid, bp.dgamma_k);
-    if ((e = after(4)) != cudaSuccess) return e;
-    if ((e = before(5)) != cudaSuccess) return e;
+    if ((e = after(i++)) != cudaSuccess) return e;
+    if ((e = before(i)) != cudaSuccess) return e;
     dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgq_part, grid, bp.dgamma_q);
-    return after(5);
+    return after(i);
 }
 
 }  // namespace zgcm

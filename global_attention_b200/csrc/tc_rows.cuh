@@ -92,10 +92,11 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     }
 }
 
-template <bool F16 = false>
-__device__ __forceinline__ float tf_prologue_row(unsigned char* h0, unsigned char* h1, int r, const float* gamma,
-                                                const LayerParams& L, const float2 (*cs)[TF_BM],
-                                                float oscale = 1.0f) {
+// cs_at(t) gives (cos, sin) of pair t at the row's position: from the shared table
+// (tf_prologue_row) or from registers (the preparation kernel).  Same values, same bits.
+template <bool F16, class CsAt>
+__device__ __forceinline__ float tf_prologue_row_at(unsigned char* h0, unsigned char* h1, int r, const float* gamma,
+                                                   const LayerParams& L, CsAt cs_at, float oscale) {
     // chunk ch (8 dims, 16 bytes) of the row: half ch / 8, swizzled position (ch % 8) ^ (r % 8)
     auto chunk = [&](int ch) -> uint4* {
         unsigned char* hb = ch < 8 ? h0 : h1;
@@ -133,7 +134,7 @@ __device__ __forceinline__ float tf_prologue_row(unsigned char* h0, unsigned cha
 #pragma unroll
     for (int t = 0; t < TF_HALF; ++t) {
         const float a = y[t], bb = y[t + TF_HALF];
-        const float2 w = cs[t][r];
+        const float2 w = cs_at(t);
         y[t] = a * w.x - bb * w.y;
         y[t + TF_HALF] = bb * w.x + a * w.y;
     }
@@ -160,6 +161,13 @@ __device__ __forceinline__ float tf_prologue_row(unsigned char* h0, unsigned cha
         *chunk(ch) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     return rinv1;  // 1 / sqrt(mean x^2 + eps) of the row (0 for a zero row)
+}
+
+template <bool F16 = false>
+__device__ __forceinline__ float tf_prologue_row(unsigned char* h0, unsigned char* h1, int r, const float* gamma,
+                                                const LayerParams& L, const float2 (*cs)[TF_BM],
+                                                float oscale = 1.0f) {
+    return tf_prologue_row_at<F16>(h0, h1, r, gamma, L, [&](int t) { return cs[t][r]; }, oscale);
 }
 
 
