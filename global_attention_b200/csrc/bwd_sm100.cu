@@ -130,11 +130,20 @@ __global__ void __launch_bounds__(GATE_THREADS, 2) bwd_gate_kernel(const bf16* _
                 reinterpret_cast<uint4*>(da16)[o] = make_uint4(da[0], da[1], da[2], da[3]);
                 reinterpret_cast<uint4*>(dg)[o] = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
                 if (sub == 0) {
-                    // row r = (b*S + s)*Hq + h  ->  [B,Hq,S] index (b*Hq + h)*S + s
-                    const long long sh = (long long)S * Hq;
-                    const long long b = r / sh, rem = r - b * sh;
-                    const long long s = rem / Hq, h = rem - s * Hq;
-                    const size_t ro = (size_t)(b * Hq + h) * S + s;
+                    // row r = (b*S + s)*Hq + h  ->  [B,Hq,S] index (b*Hq + h)*S + s (32-bit
+                    // division where the row count allows: the 64-bit one is a long sequence)
+                    size_t ro;
+                    if (rows <= 0xffffffffLL) {
+                        const uint32_t ru = (uint32_t)r, sh = (uint32_t)S * (uint32_t)Hq;
+                        const uint32_t b = ru / sh, rem = ru - b * sh;
+                        const uint32_t s = rem / (uint32_t)Hq, h = rem - s * (uint32_t)Hq;
+                        ro = ((size_t)b * Hq + h) * S + s;
+                    } else {
+                        const long long sh = (long long)S * Hq;
+                        const long long b = r / sh, rem = r - b * sh;
+                        const long long s = rem / Hq, h = rem - s * Hq;
+                        ro = (size_t)(b * Hq + h) * S + s;
+                    }
                     dainv[ro] = mx > 0.f ? 1.0f / sc : 0.f;
                     domax[ro] = mx;
                 }
