@@ -74,14 +74,14 @@ def work(B, S, W, bwd):
         # q, k, v, dA, lse, Delta -> dk, dv ; S, dP, dV, dK
         "bwd_main_kernel": (qb + 2 * kb + qb + 2 * lse + 2 * kb, 8 * D * npair),
         # tcgen05 backward: gate pass dout, g, out -> dg, dA16 (fp16), 2^-e and max|dout| per row;
-        # q, k, v, dA16, 2^-e -> dq, lse, Delta ; S, dP, dQ  |
-        # q, k, v, dA16, 4 row stats -> dk, dv ; S, dP, dV, dK
+        # Q~16, K~16, V16, dA16, lse, 2^-e, raw q (RMSNorm backward) -> dq, Delta ; S, dP, dQ  |
+        # Q~16, K~16, V16, dA16, lse, Delta, 2^-e, max|dout|, raw k -> dk, dv ; S, dP, dV, dK
         "bwd_gate_kernel": (5 * qb + 2 * lse, 0),
         # k, v -> K~, V fp16 (+ per-row inverse RMS and v norm, per-tile V scale); q -> Q~ fp16
         "bwd_prep_kv_kernel": (4 * kb + kb // D, 0),
         "bwd_prep_q_kernel": (2 * qb + qb // (2 * D), 0),
-        "bwd_q_tc_kernel": (qb + 2 * kb + qb + qb + 3 * lse, 6 * D * npair),
-        "bwd_kv_tc_kernel": (qb + 2 * kb + qb + 4 * lse + 2 * kb, 8 * D * npair),
+        "bwd_q_tc_kernel": (4 * qb + 2 * kb + 3 * lse, 6 * D * npair),
+        "bwd_kv_tc_kernel": (2 * qb + 5 * kb + 4 * lse, 8 * D * npair),
     }
     return dict(tokens=tok, npair=npair, fwd_bytes=fwd_bytes, fwd_flops=fwd_flops,
                 bwd_bytes=bwd_bytes if bwd else 0, bwd_flops=bwd_flops if bwd else 0,
