@@ -46,17 +46,28 @@ struct BwdTcParams {
     CUtensorMap tm_k16; // K~ fp16 (normalised, rotated, times the q~/k~ scale), geometry of tm_k
     CUtensorMap tm_v16; // V fp16 times 2^e per 128-row tile, geometry of tm_v
     CUtensorMap tm_q16; // Q~ fp16 (normalised, rotated, times the q~/k~ scale), geometry of tm_q
+    CUtensorMap tm_q16h;  // the same with 64-row boxes (key-major kernel, one 64-query half)
+    CUtensorMap tm_dah;   // dA16 with 64-row boxes
+    CUtensorMap tm_lse;   // lse2p, Delta, 2^-e of the dA rows: fp32 {Spad, Hq, B}, box {64, 1, 1}
+    CUtensorMap tm_delta;
+    CUtensorMap tm_dainv;
     BwdParams P;
     const __half* da16; // [B,S,Hq,D] dA * 2^e (e per row)
-    float* dainv;       // [B,Hq,S] 2^-e of each dA row (0 for an all-zero row)
-    float* domax;       // [B,Hq,S] max |dout| of each row (bound on |dA|)
+    float* dainv;       // [B,Hq,Spad] 2^-e of each dA row (0 for an all-zero row and past S)
+    float* domax;       // [B,Hq,Spad] max |dout| of each row (bound on |dA|)
     float* krinv;       // [B,Hkv,S] inverse RMS of each raw k row
     float* qrinv;       // [B,Hq,S] inverse RMS of each raw q row
+    float* lse2p;       // [B,Hq,Spad] the forward's lse in base 2 (+inf past S), for TMA
     float* vnorm;       // [B,Hkv,S] 2-norm of each raw v row
     float* vtinv;       // [B,Hkv,ceil(S/128)] 2^-e of each V tile
     int* err;
     int total;          // steps (query-major) or units (key-major)
 };
+
+// Row stride of the backward's per-row arrays [B, Hq, Spad]: the sequence rounded up to 64,
+// so that a 64-row run starts on a 256-byte boundary and the arrays can be TMA tensors (a
+// global stride must be a multiple of 16 bytes).  Entries past S hold neutral values.
+__host__ __device__ __forceinline__ int row_stride(int S) { return (S + 63) & ~63; }
 
 // power-of-two exponent e with |x| * 2^e in [2^13, 2^14); 0 for x == 0 or non-finite
 __device__ __forceinline__ int fit_exp(float x) {
@@ -76,7 +87,8 @@ constexpr int GATE_UNROLL = 4;  // rows in flight per half-warp
 // One half-warp per row of D = 128 (16 lanes x 8 values, fully coalesced), GATE_UNROLL rows
 // per half-warp in flight; every loop bound is warp-uniform so the row-max shuffles see all
 // 32 lanes.  dainv = 2^-e (0 when the row of dout is all zero: its dA row is zero and must
-// not be rescaled), domax = max|dout|, both [B,Hq,S].
+// not be rescaled), domax = max|dout|, both [B,Hq,Spad] (row_stride; the query-major kernel
+// fills the entries past S).
 __global__ void __launch_bounds__(GATE_THREADS, 2) bwd_gate_kernel(const bf16* __restrict__ dout,
                                                                 const bf16* __restrict__ g,
                                                                 const bf16* __restrict__ out,
@@ -137,12 +149,12 @@ __global__ void __launch_bounds__(GATE_THREADS, 2) bwd_gate_kernel(const bf16* _
                         const uint32_t ru = (uint32_t)r, sh = (uint32_t)S * (uint32_t)Hq;
                         const uint32_t b = ru / sh, rem = ru - b * sh;
                         const uint32_t s = rem / (uint32_t)Hq, h = rem - s * (uint32_t)Hq;
-                        ro = ((size_t)b * Hq + h) * S + s;
+                        ro = ((size_t)b * Hq + h) * row_stride(S) + s;
                     } else {
                         const long long sh = (long long)S * Hq;
                         const long long b = r / sh, rem = r - b * sh;
                         const long long s = rem / Hq, h = rem - s * Hq;
-                        ro = (size_t)(b * Hq + h) * S + s;
+                        ro = (size_t)(b * Hq + h) * row_stride(S) + s;
                     }
                     dainv[ro] = mx > 0.f ? 1.0f / sc : 0.f;
                     domax[ro] = mx;
@@ -208,8 +220,8 @@ __device__ __forceinline__ void q_pass1_chunk(float (&sv)[32], float (&dv)[32], 
 }
 
 // Key-major chunk: one key row j against 32 query columns i0.. (S^T, dP^T from TMEM; per
-// column lse, Delta and dA row scale 2^-e_i from shared memory; vm = the visible columns,
-// ignored when FULL):
+// column lse (base 2), Delta and dA row scale 2^-e_i from shared memory; vm = the visible
+// columns, ignored when FULL):
 //   P^T = 2^(s c2 - lse) (visible pairs), dP^T = dv * vin * 2^-e_i,
 //   P^T for dV carries 2^(E - e_i) (su = 2^E), dS^T = P^T (dP^T - Delta) * dsc,
 //   kacc += dS^T S^T (unscaled dS^T; dk's RMSNorm row term).
@@ -228,7 +240,7 @@ __device__ __forceinline__ void kv_chunk(const float* sv, const float* dv, const
         for (int u = 0; u < 4; ++u) {
             const int e = 4 * e4 + u;
             float pv = fast_exp2(fmaf(sv[e], c2, -lsv[u]));
-            if (!FULL) pv = ((vm >> e) & 1u) ? pv : 0.f;
+            if (!FULL) pv = ((vm >> e) & 1u) ? pv : 0.f;  // (columns past the sequence: masked)
             const float dp = dv[e] * vin * dcv[u];
             const float d = pv * (dp - dlv[u]);
             kacc = fmaf(d, sv[e], kacc);
@@ -661,7 +673,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
         reg_alloc<176>();
         // ================================================ Delta, dS (thread = query row)
         const int r = tid - 128, wq = warp - 4;
-        const int nkt = (L.S + TF_BN - 1) / TF_BN;
+        const int nkt = (L.S + TF_BN - 1) / TF_BN, Spad = row_stride(L.S);
         const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
         int n_next = 0, n_cur = 0, m = 0;
         for (int t = t_begin; t < t_end; ++t) {
@@ -688,9 +700,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             for (int h = 0; h < G; ++h, ++m) {
                 const int hg = st.kvh * G + h;
                 const size_t ro = ((size_t)st.b * L.Hq + hg) * L.S + (i < L.S ? i : 0);
+                const size_t rp = ((size_t)st.b * L.Hq + hg) * Spad + i;  // padded row arrays
                 // the forward's log-sum-exp (base 2): its scores are these, bit for bit
                 const float lse2 = i < L.S ? p.P.lse[ro] * kLog2e : INFINITY;
-                const float dai = i < L.S ? p.dainv[ro] : 0.f;  // undoes the dA row scale
+                const float dai = i < L.S ? p.dainv[rp] : 0.f;  // undoes the dA row scale
                 const uint32_t tS = tm_half(m) + lane_off, tP = tm_half(m + 1) + lane_off;
                 if (!mbar_wait(&sm.bar[QB_DPFULL], m & 1, abort, 121)) { stop = true; break; }
                 tc_fence_after();
@@ -745,7 +758,13 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                     tmem_st16(tS + 16 * c8, pk);
                 }
                 tmem_wait_st();
-                if (i < L.S) p.P.delta[ro] = delta;
+                if (i < Spad) {
+                    // Delta and the base-2 lse per row for the key-major kernel; past S the
+                    // neutral values (P = 0 there, and the dA scale 0)
+                    p.P.delta[rp] = i < L.S ? delta : 0.f;
+                    p.lse2p[rp] = lse2;
+                    if (i >= L.S) p.dainv[rp] = 0.f;
+                }
                 sm.dsinv[m & 1][r] = 1.0f / dsc;
                 sm.mdot[m & 1][r] = fmaf(-delta, sb, sa) * mdot_f;  // sum dS S = a - Delta b
                 tc_fence_before();
@@ -806,29 +825,39 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
 
 // =====================================================================  key-major kernel
 
+constexpr int KV_SLOTS = 4;                      // Q~ / dA ring depth, in 64-query halves
+constexpr uint32_t KV_SLOT_HALF = 64u * 128u;   // 64 rows x 128 bytes: one d-half of a slot
+
 enum KBar {
     KB_KVFULL = 0, KB_KVEMPTY = 2,
-    KB_QFULL = 3, KB_QREADY = 5, KB_QEMPTY = 7,
-    KB_SFULL = 9, KB_PFULL = 11,  // by 64-query half (TMEM buffer)
-    KB_DVKFULL = 13, KB_DVKEMPTY = 14, KB_DONE = 15, KB_COUNT = 16
+    KB_QFULL = 3, KB_QEMPTY = 11,  // by ring slot (KV_SLOTS each)
+    KB_SFULL = 15, KB_PFULL = 17,                 // by TMEM buffer (2 each)
+    KB_DVKFULL = 19, KB_DVKEMPTY = 20, KB_DONE = 21, KB_RED = 22,
+    KB_STATS = 23,  // a unit's scales are in shared memory; by unit number % 2
+    KB_COUNT = 25
 };
 
 struct BwdKTcSmem {
     alignas(1024) unsigned char K[2][TF_HALF_BYTES];      // K~ fp16 of the unit's key tile
     alignas(1024) unsigned char V[2][TF_HALF_BYTES];      // V fp16, row-scaled
-    alignas(1024) unsigned char Q[2][2][TF_HALF_BYTES];   // [buffer][half] Q~ fp16 (prepared)
-    alignas(1024) unsigned char dA[2][2][TF_HALF_BYTES];  // [buffer][half] dA fp16, row-scaled (TMA)
+    // ring of KV_SLOTS slots, one per 64-query half: Q~ and dA rows of the half, each as two
+    // d-halves of 64 rows x 128 bytes (the SW128 layout of a 64-row TMA box)
+    alignas(1024) unsigned char Q[KV_SLOTS][2][KV_SLOT_HALF];
+    alignas(1024) unsigned char dA[KV_SLOTS][2][KV_SLOT_HALF];
     float gq[kD], gk[kD];
-    float lse2[2][TF_BM];    // per query column of the buffer
-    float delta[2][TF_BM];
-    float dcol[2][TF_BM];    // 2^-e of the dA row of each query column
+    // per query column of the slot, loaded by TMA with the slot's rows (neutral values past
+    // the sequence end, where every pair is masked): the forward's lse in base 2, Delta, 2^-e
+    // of the dA row
+    alignas(128) float lsec[KV_SLOTS][64];
+    alignas(128) float delta[KV_SLOTS][64];
+    alignas(128) float dcol[KV_SLOTS][64];
     float vtinv[4];          // 2^-e of the unit's V tile, by unit number % 4
     float dsc[4][TF_BN];     // 2^e of each dS^T row, by unit number % 4
     // 4 deep: the prologue writes a unit's scales at its start, while the epilogue of an earlier
     // unit may still read its own (with one query head per KV head a unit has two iterations)
     float uinv[4];           // 2^-E, E = the unit's smallest dA row exponent, by unit number % 4
     float kmdot[2][TF_BN];   // mean(dy gamma xhat) of each key row (RMSNorm backward), by unit parity
-    float red[2][4];         // per-warp maxima for the unit statistics
+    float red[2][2][4];      // per-warp maxima for the unit statistics, by call parity
     float dgk[4][kD];        // this CTA's d_gamma_k, one slice per epilogue warp
     uint64_t bar[KB_COUNT];
     uint32_t tmem_base;
@@ -867,9 +896,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
         sm.abort = 0;
         mbar_init(&sm.bar[KB_KVFULL], 1);
         mbar_init(&sm.bar[KB_KVEMPTY], 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < KV_SLOTS; ++i) {
             mbar_init(&sm.bar[KB_QFULL + i], 1);
-            mbar_init(&sm.bar[KB_QREADY + i], 128);
             mbar_init(&sm.bar[KB_QEMPTY + i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -879,6 +907,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
         mbar_init(&sm.bar[KB_DVKFULL], 1);
         mbar_init(&sm.bar[KB_DVKEMPTY], 128);
         mbar_init(&sm.bar[KB_DONE], 1);
+        mbar_init(&sm.bar[KB_RED], 4);  // one arrival per epilogue warp
+        mbar_init(&sm.bar[KB_STATS], 128);
+        mbar_init(&sm.bar[KB_STATS + 1], 128);
         fence_barrier_init();
     }
     if (tid < kD) {
@@ -918,9 +949,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
     if (warp < 4) {
         reg_dealloc<64>();
         if (warp == 0) {
-            // ================================================ TMA producer: K, V per unit; Q, dA per iteration
+            // ================================================ TMA producer: K, V per unit; Q~, dA per 64-query half
             if (lane == 0) {
-                int it_all = 0, last_q[2] = {-1, -1}, uu = 0;
+                int hs = 0, uu = 0, last_q[KV_SLOTS];
+                for (int i = 0; i < KV_SLOTS; ++i) last_q[i] = -1;
                 auto load_kv = [&](const UnitInfo& x) {
                     mbar_expect_tx(&sm.bar[KB_KVFULL], 2 * TF_TILE_BYTES);
                     tma_load_4d(sm.K[0], &p.tm_k16, &sm.bar[KB_KVFULL], 0, x.kvh, x.kt * TF_BN, x.b);
@@ -931,28 +963,36 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 bool ok = true;
                 for (int u = u_begin; u < u_end && ok && !*abort; ++u, ++uu) {
                     const UnitInfo x = decode_unit(L, u);
-                    for (int it = 0; it < x.nit; ++it, ++it_all) {
-                        const int buf = it_all & 1;
-                        if (it_all >= 2 && !(ok = mbar_wait(&sm.bar[KB_QEMPTY + buf], ((it_all >> 1) - 1) & 1, abort, 202))) break;
+                    for (int it = 0; it < x.nit && ok; ++it) {
                         int qb, hg;
                         decode_iter(L, x, it, qb, hg);
-                        mbar_expect_tx(&sm.bar[KB_QFULL + buf], 2 * TF_TILE_BYTES);
-                        tma_load_4d(sm.Q[buf][0], &p.tm_q16, &sm.bar[KB_QFULL + buf], 0, hg, qb * TF_BM, x.b);
-                        tma_load_4d(sm.Q[buf][1], &p.tm_q16, &sm.bar[KB_QFULL + buf], 64, hg, qb * TF_BM, x.b);
-                        tma_load_4d(sm.dA[buf][0], &p.tm_da, &sm.bar[KB_QFULL + buf], 0, hg, qb * TF_BM, x.b);
-                        tma_load_4d(sm.dA[buf][1], &p.tm_da, &sm.bar[KB_QFULL + buf], 64, hg, qb * TF_BM, x.b);
-                        last_q[buf] = it_all;
-                        if (it == 0) {
-                            // K, V of the unit once the previous unit's products are done; the
-                            // unit's first query tile went out before, as soon as its buffer was free
-                            if (uu >= 1 && !(ok = mbar_wait(&sm.bar[KB_KVEMPTY], (uu - 1) & 1, abort, 201))) break;
-                            load_kv(x);
+                        for (int half = 0; half < 2; ++half, ++hs) {
+                            const int slot = hs % KV_SLOTS;
+                            if (hs >= KV_SLOTS &&
+                                !(ok = mbar_wait(&sm.bar[KB_QEMPTY + slot], ((hs / KV_SLOTS) - 1) & 1, abort, 202)))
+                                break;
+                            const int row = qb * TF_BM + 64 * half;
+                            mbar_expect_tx(&sm.bar[KB_QFULL + slot], 4 * KV_SLOT_HALF + 3 * 64 * 4);
+                            tma_load_3d(sm.lsec[slot], &p.tm_lse, &sm.bar[KB_QFULL + slot], row, hg, x.b);  // base-2 lse
+                            tma_load_3d(sm.delta[slot], &p.tm_delta, &sm.bar[KB_QFULL + slot], row, hg, x.b);
+                            tma_load_3d(sm.dcol[slot], &p.tm_dainv, &sm.bar[KB_QFULL + slot], row, hg, x.b);
+                            tma_load_4d(sm.Q[slot][0], &p.tm_q16h, &sm.bar[KB_QFULL + slot], 0, hg, row, x.b);
+                            tma_load_4d(sm.Q[slot][1], &p.tm_q16h, &sm.bar[KB_QFULL + slot], 64, hg, row, x.b);
+                            tma_load_4d(sm.dA[slot][0], &p.tm_dah, &sm.bar[KB_QFULL + slot], 0, hg, row, x.b);
+                            tma_load_4d(sm.dA[slot][1], &p.tm_dah, &sm.bar[KB_QFULL + slot], 64, hg, row, x.b);
+                            last_q[slot] = hs;
+                            if (it == 0 && half == 0) {
+                                // K, V of the unit once the previous unit's products are done; the
+                                // unit's first query half went out before, as soon as its slot was free
+                                if (uu >= 1 && !(ok = mbar_wait(&sm.bar[KB_KVEMPTY], (uu - 1) & 1, abort, 201))) break;
+                                load_kv(x);
+                            }
                         }
                     }
                 }
                 if (uu >= 1) mbar_wait_drain(&sm.bar[KB_KVFULL], (uu - 1) & 1);
-                for (int buf = 0; buf < 2; ++buf)
-                    if (last_q[buf] >= 0) mbar_wait_drain(&sm.bar[KB_QFULL + buf], (last_q[buf] >> 1) & 1);
+                for (int i = 0; i < KV_SLOTS; ++i)
+                    if (last_q[i] >= 0) mbar_wait_drain(&sm.bar[KB_QFULL + i], (last_q[i] / KV_SLOTS) & 1);
             }
         } else if (warp == 1) {
             // ================================================ MMA issuer
@@ -988,50 +1028,50 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 };
                 auto last_of_unit = [](const Cursor& c) { return c.half == 1 && c.it == c.x.nit - 1; };
                 auto issue_s = [&](const Cursor& c) -> bool {
-                    const int buf = c.it_all & 1;
+                    const int hs = 2 * c.it_all + c.half, slot = hs % KV_SLOTS;
                     if (c.it == 0 && c.half == 0 && !mbar_wait(&sm.bar[KB_KVFULL], c.uu & 1, abort, 210)) return false;
-                    if (c.half == 0 && !mbar_wait(&sm.bar[KB_QFULL + buf], (c.it_all >> 1) & 1, abort, 211)) return false;
+                    if (!mbar_wait(&sm.bar[KB_QFULL + slot], (hs / KV_SLOTS) & 1, abort, 211)) return false;
                     tc_fence_after();
                     const uint32_t tX = tmem + 128u * (uint32_t)c.half;
-                    const uint32_t rows = (uint32_t)c.half * 64u * 128u;  // first query row of the half
-                    const uint32_t qa = q_base + buf * 2 * TF_HALF_BYTES + rows, da = da_base + buf * 2 * TF_HALF_BYTES + rows;
+                    const uint32_t qa = q_base + (uint32_t)slot * 2u * KV_SLOT_HALF;
+                    const uint32_t da = da_base + (uint32_t)slot * 2u * KV_SLOT_HALF;
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t dh = kk >> 2, within = (kk & 3) * 32;
                         mma_ss(tX, sdesc_sw128(k_base + dh * TF_HALF_BYTES + within, 16, 1024),
-                               sdesc_sw128(qa + dh * TF_HALF_BYTES + within, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+                               sdesc_sw128(qa + dh * KV_SLOT_HALF + within, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
                     }
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t dh = kk >> 2, within = (kk & 3) * 32;
                         mma_ss(tX + 64, sdesc_sw128(v_base + dh * TF_HALF_BYTES + within, 16, 1024),
-                               sdesc_sw128(da + dh * TF_HALF_BYTES + within, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+                               sdesc_sw128(da + dh * KV_SLOT_HALF + within, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(&sm.bar[KB_SFULL + c.half]);
                     if (last_of_unit(c)) mma_commit(&sm.bar[KB_KVEMPTY]);  // K, V read for the last time
                     return true;
                 };
                 auto issue_dvk = [&](const Cursor& c) -> bool {
-                    const int buf = c.it_all & 1;
+                    const int hs = 2 * c.it_all + c.half, slot = hs % KV_SLOTS;
                     if (!mbar_wait(&sm.bar[KB_PFULL + c.half], c.it_all & 1, abort, 212)) return false;
                     if (c.it == 0 && c.half == 0 && c.uu >= 1 &&
                         !mbar_wait(&sm.bar[KB_DVKEMPTY], (c.uu - 1) & 1, abort, 213))
                         return false;
                     tc_fence_after();
                     const uint32_t tX = tmem + 128u * (uint32_t)c.half;
-                    const uint32_t rows = (uint32_t)c.half * 64u * 128u;
-                    const uint32_t qa = q_base + buf * 2 * TF_HALF_BYTES + rows, da = da_base + buf * 2 * TF_HALF_BYTES + rows;
+                    const uint32_t qa = q_base + (uint32_t)slot * 2u * KV_SLOT_HALF;
+                    const uint32_t da = da_base + (uint32_t)slot * 2u * KV_SLOT_HALF;
                     const bool first = c.it == 0 && c.half == 0;
                     // A from TMEM (16 queries = 8 columns per step); B = dA / Q~ MN-major (N = d)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(TM_DV, tX + kk * 8, sdesc_sw128(da + kk * 16 * 128, TF_HALF_BYTES, 1024), IDESC_MN,
+                        mma_ts(TM_DV, tX + kk * 8, sdesc_sw128(da + kk * 16 * 128, KV_SLOT_HALF, 1024), IDESC_MN,
                                (!first || kk > 0) ? 1u : 0u);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(TM_DK, tX + 64 + kk * 8, sdesc_sw128(qa + kk * 16 * 128, TF_HALF_BYTES, 1024), IDESC_MN,
+                        mma_ts(TM_DK, tX + 64 + kk * 8, sdesc_sw128(qa + kk * 16 * 128, KV_SLOT_HALF, 1024), IDESC_MN,
                                (!first || kk > 0) ? 1u : 0u);
-                    if (c.half == 1) mma_commit(&sm.bar[KB_QEMPTY + buf]);
+                    mma_commit(&sm.bar[KB_QEMPTY + slot]);  // the half's Q~ and dA rows were read for the last time
                     if (last_of_unit(c)) mma_commit(&sm.bar[KB_DVKFULL]);
                     return true;
                 };
@@ -1065,26 +1105,26 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             float vin = 0.f, su = 0.f, dsc = 0.f;
             float kacc = 0.f;  // sum over the unit of dS^T S^T (unscaled dS^T): dk's RMSNorm row term
             for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
-                const int buf = it_all & 1;
                 int qb, hg;
                 decode_iter(L, x, it, qb, hg);
                 const int q0 = qb * TF_BM;
-                if (!(ok = mbar_wait(&sm.bar[KB_QREADY + buf], (it_all >> 1) & 1, abort, 221))) break;
-                if (it == 0) {
-                    // the unit's scales, written by the prologue before this query tile's barrier
-                    vin = sm.vtinv[uu & 3];        // undoes the V tile scale of dP^T
-                    su = 1.0f / sm.uinv[uu & 3];   // 2^E: P^T columns carry 2^(E - e_i)
-                    dsc = sm.dsc[uu & 3][r];
-                }
                 const int jmin = x.kt * TF_BN + 32 * wq, jmax = jmin + 31;
                 for (int half = 0; half < 2 && ok; ++half) {
-                    // 64-query half in TMEM buffer `half`: S^T at columns [0,64), dP^T at [64,128)
+                    const int hs = 2 * it_all + half, slot = hs % KV_SLOTS;
+                    if (it == 0 && half == 0) {
+                        if (!(ok = mbar_wait(&sm.bar[KB_STATS + (uu & 1)], (uu >> 1) & 1, abort, 223))) break;
+                        vin = sm.vtinv[uu & 3];        // undoes the V tile scale of dP^T
+                        su = 1.0f / sm.uinv[uu & 3];   // 2^E: P^T columns carry 2^(E - e_i)
+                        dsc = sm.dsc[uu & 3][r];
+                    }
+                    // 64-query half in TMEM buffer `half`: S^T at columns [0,64), dP^T at [64,128);
+                    // its S MMA waited for the slot's TMA, per-column values included
                     if (!(ok = mbar_wait(&sm.bar[KB_SFULL + half], it_all & 1, abort, 222))) break;
                     tc_fence_after();
                     const uint32_t tX = tmem + 128u * (uint32_t)half + lane_off;
 #pragma unroll 1
                     for (int c8 = 0; c8 < 2; ++c8) {
-                        const int ql0 = 64 * half + 32 * c8, i0 = q0 + ql0;  // queries i0 .. i0+31
+                        const int ql0 = 32 * c8, i0 = q0 + 64 * half + ql0;  // queries i0 .. i0+31
                         const bool live = jmin < L.S && i0 < L.S && i0 + 31 >= jmin && i0 <= jmax + L.W - 1;
                         const bool full = jmax <= i0 && jmin > i0 + 31 - L.W && i0 + 31 < L.S && jmax < L.S;
                         uint32_t pp[16], dd[16];
@@ -1094,12 +1134,12 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                             tmem_ld32f(tX + 64 + 32 * c8, dv);
                             tmem_wait_ld();
                             if (full) {
-                                kv_chunk<true>(sv, dv, sm.lse2[buf] + ql0, sm.delta[buf] + ql0, sm.dcol[buf] + ql0, 0u,
+                                kv_chunk<true>(sv, dv, sm.lsec[slot] + ql0, sm.delta[slot] + ql0, sm.dcol[slot] + ql0, 0u,
                                                vin, su, dsc, c2, pp, dd, kacc);
                             } else {
                                 // queries that see key j: j <= i <= min(j + W - 1, S - 1)
                                 const uint32_t vm = j < L.S ? bit_range(j - i0, min(j + L.W - 1, L.S - 1) - i0) : 0u;
-                                kv_chunk<false>(sv, dv, sm.lse2[buf] + ql0, sm.delta[buf] + ql0, sm.dcol[buf] + ql0, vm,
+                                kv_chunk<false>(sv, dv, sm.lsec[slot] + ql0, sm.delta[slot] + ql0, sm.dcol[slot] + ql0, vm,
                                                 vin, su, dsc, c2, pp, dd, kacc);
                             }
                         } else {
@@ -1117,14 +1157,20 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             }
         }
     } else if (warp >= 8 && warp < 12) {
-        // ================================================ prologue: unit scales, per-column values
-        const int r = tid - 256, wq = warp - 8;
-        int it_all = 0, uu = 0;
-        bool ok = true;
+        // (no prologue: the slots' per-column values arrive by TMA with their rows)
+    } else if (warp >= 12) {
+        reg_alloc<192>();
+        // ================================================ unit scales; dv, dk epilogue (thread = key row)
+        const int r = tid - 384, wq = warp - 12;
+        const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+        int uu = 0;
         // Scales of unit x into ring slot `slot`: max |dout| and max |Delta| over the rows the
         // unit reads (global loads only), the dA scale E, the dS^T row scales and the V tile
-        // scale.  Computed during the previous unit's last iteration, off the unit boundary.
-        auto unit_scales = [&](const UnitInfo& x, int slot) {
+        // scale.  This warpgroup is otherwise idle during a unit: it computes the next unit's
+        // scales right after the previous unit's epilogue, and hands them to the softmax
+        // through KB_STATS (two barriers alternating by unit, so neither runs a phase ahead).
+        int n_red = 0;
+        auto unit_scales = [&](const UnitInfo& x, int slot) -> bool {
             // every global load of the unit's statistics is issued before any is used (one
             // round trip instead of one per dependent batch)
             const int j = x.kt * TF_BN + r, nkt = (L.S + TF_BN - 1) / TF_BN;
@@ -1141,9 +1187,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                     decode_iter(L, x, it0 + k, qb, hg);
                     const int i = qb * TF_BM + r;
                     if (it0 + k < x.nit && i < L.S) {
-                        const size_t ro = ((size_t)x.b * L.Hq + hg) * L.S + i;
-                        dm[k] = p.domax[ro];
-                        dl[k] = p.P.delta[ro];
+                        const size_t rp = ((size_t)x.b * L.Hq + hg) * row_stride(L.S) + i;
+                        dm[k] = p.domax[rp];
+                        dl[k] = p.P.delta[rp];
                     }
                 }
 #pragma unroll
@@ -1157,14 +1203,18 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 domx = fmaxf(domx, __shfl_xor_sync(0xffffffffu, domx, o));
                 dlmx = fmaxf(dlmx, __shfl_xor_sync(0xffffffffu, dlmx, o));
             }
+            // across the 4 warps through an mbarrier (a bounded wait: a named barrier would hang
+            // if some thread had given up earlier); the scratch alternates by call parity
+            float(*rr)[4] = sm.red[n_red & 1];
             if (lane == 0) {
-                sm.red[0][wq] = domx;
-                sm.red[1][wq] = dlmx;
+                rr[0][wq] = domx;
+                rr[1][wq] = dlmx;
+                mbar_arrive(&sm.bar[KB_RED]);
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            domx = fmaxf(fmaxf(sm.red[0][0], sm.red[0][1]), fmaxf(sm.red[0][2], sm.red[0][3]));
-            dlmx = fmaxf(fmaxf(sm.red[1][0], sm.red[1][1]), fmaxf(sm.red[1][2], sm.red[1][3]));
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (!mbar_wait(&sm.bar[KB_RED], n_red & 1, abort, 232)) return false;
+            ++n_red;
+            domx = fmaxf(fmaxf(rr[0][0], rr[0][1]), fmaxf(rr[0][2], rr[0][3]));
+            dlmx = fmaxf(fmaxf(rr[1][0], rr[1][1]), fmaxf(rr[1][2], rr[1][3]));
             // E = fit_exp(max domax) is the smallest row exponent of dA in the unit, so every
             // column factor 2^(E - e_i) of P^T is <= 1
             const int E = fit_exp(domx);
@@ -1174,34 +1224,15 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 sm.uinv[slot] = ldexpf(1.0f, -E);
                 sm.vtinv[slot] = vtile;
             }
+            return true;
         };
-        if (u_begin < u_end) unit_scales(decode_unit(L, u_begin), 0);
+        bool ok = true;
+        if (u_begin < u_end && (ok = unit_scales(decode_unit(L, u_begin), 0))) mbar_arrive(&sm.bar[KB_STATS]);
         for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
-            const UnitInfo x = decode_unit(L, u);
-            for (int it = 0; it < x.nit && ok; ++it, ++it_all) {
-                const int buf = it_all & 1;
-                int qb, hg;
-                decode_iter(L, x, it, qb, hg);
-                const int i = qb * TF_BM + r;
-                const bool valid = i < L.S;
-                // (the wait keeps these per-column values from overwriting those of iteration
-                // it - 2 before its products are done: the buffer's tiles land only after that)
-                if (!(ok = mbar_wait(&sm.bar[KB_QFULL + buf], (it_all >> 1) & 1, abort, 231))) break;
-                const size_t ro = ((size_t)x.b * L.Hq + hg) * L.S + (valid ? i : 0);
-                sm.lse2[buf][r] = valid ? p.P.lse[ro] * kLog2e : INFINITY;  // the forward's, base 2
-                sm.delta[buf][r] = valid ? p.P.delta[ro] : 0.f;
-                sm.dcol[buf][r] = valid ? p.dainv[ro] : 0.f;
-                mbar_arrive(&sm.bar[KB_QREADY + buf]);
-                if (it == x.nit - 1 && u + 1 < u_end) unit_scales(decode_unit(L, u + 1), (uu + 1) & 3);
+            if (u + 1 < u_end) {
+                if (!(ok = unit_scales(decode_unit(L, u + 1), (uu + 1) & 3))) break;
+                mbar_arrive(&sm.bar[KB_STATS + ((uu + 1) & 1)]);
             }
-        }
-    } else if (warp >= 12) {
-        reg_alloc<192>();
-        // ================================================ dv, dk epilogue (thread = key row)
-        const int r = tid - 384, wq = warp - 12;
-        const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
-        int uu = 0;
-        for (int u = u_begin; u < u_end; ++u, ++uu) {
             const UnitInfo x = decode_unit(L, u);
             const int j = x.kt * TF_BN + r;
             const bool valid = j < L.S;
@@ -1271,15 +1302,28 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_b() {
 }
 
 bool make_map_b(CUtensorMap* map, const void* base, int H, int S, int B,
-                CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+                CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, int box_rows = 128) {
     auto enc = get_encode_b();
     if (!enc) return false;
     cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)S * H * kD * 2};
-    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(map, dtype, 4, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D fp32 map {Spad, H, B} of a padded per-row array, box {64, 1, 1}, no swizzle
+bool make_map_rows(CUtensorMap* map, const float* base, int H, int Spad, int B) {
+    auto enc = get_encode_b();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)Spad, (cuuint64_t)H, (cuuint64_t)B};
+    cuuint64_t strides[2] = {(cuuint64_t)Spad * 4, (cuuint64_t)H * Spad * 4};
+    cuuint32_t box[3] = {64, 1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1297,15 +1341,18 @@ bool bwd_tc_supported(const LayerParams& L) {
     return L.W <= TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1 && get_encode_b() != nullptr;
 }
 
-// workspace of the tcgen05 backward: delta, domax, dainv, qrinv [B,Hq,S] fp32; dA16, Q~16
+// workspace of the tcgen05 backward: delta, domax, dainv, lse2p [B,Hq,Spad] and qrinv
+// [B,Hq,S] fp32; dA16, Q~16
 // [B,S,Hq,D] fp16; K~16, V16 [B,S,Hkv,D] fp16; krinv, vnorm [B,Hkv,S] fp32; vtinv per V
 // tile; 2 x d_gamma partials
 size_t bwd_tc_workspace_bytes(int B, int S, int Hq, int Hkv) {
     const size_t rows = (size_t)B * S * Hq, krows = (size_t)B * S * Hkv;
+    const size_t prows = (size_t)B * Hq * row_stride(S);  // padded row arrays
     const size_t tiles = (size_t)B * Hkv * ((S + TF_BN - 1) / TF_BN);
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
-    return 4 * a(rows * sizeof(float)) + 2 * a(rows * kD * sizeof(__half)) + 2 * a(krows * kD * sizeof(__half)) +
-           2 * a(krows * sizeof(float)) + a(tiles * sizeof(float)) + 2 * a((size_t)TB_MAX_GRID * kD * sizeof(float));
+    return 4 * a(prows * sizeof(float)) + a(rows * sizeof(float)) + 2 * a(rows * kD * sizeof(__half)) +
+           2 * a(krows * kD * sizeof(__half)) + 2 * a(krows * sizeof(float)) + a(tiles * sizeof(float)) +
+           2 * a((size_t)TB_MAX_GRID * kD * sizeof(float));
 }
 
 cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, cudaStream_t stream,
@@ -1323,9 +1370,12 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
         return q;
     };
     p.P.lse2 = nullptr;  // P is formed from the forward's lse
-    p.P.delta = reinterpret_cast<float*>(take(rows * 4));
-    p.domax = reinterpret_cast<float*>(take(rows * 4));
-    p.dainv = reinterpret_cast<float*>(take(rows * 4));
+    const int Spad = row_stride(L.S);
+    const size_t prows = (size_t)L.B * L.Hq * Spad;
+    p.P.delta = reinterpret_cast<float*>(take(prows * 4));
+    p.domax = reinterpret_cast<float*>(take(prows * 4));
+    p.dainv = reinterpret_cast<float*>(take(prows * 4));
+    p.lse2p = reinterpret_cast<float*>(take(prows * 4));
     __half* da16 = reinterpret_cast<__half*>(take(rows * kD * sizeof(__half)));
     p.da16 = da16;
     void* q16 = take(rows * kD * sizeof(__half));
@@ -1345,7 +1395,11 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
         !make_map_b(&p.tm_da, da16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
         !make_map_b(&p.tm_k16, k16, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
         !make_map_b(&p.tm_v16, v16, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-        !make_map_b(&p.tm_q16, q16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        !make_map_b(&p.tm_q16, q16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+        !make_map_b(&p.tm_q16h, q16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 64) ||
+        !make_map_b(&p.tm_dah, da16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 64) ||
+        !make_map_rows(&p.tm_lse, p.lse2p, L.Hq, Spad, L.B) || !make_map_rows(&p.tm_delta, p.P.delta, L.Hq, Spad, L.B) ||
+        !make_map_rows(&p.tm_dainv, p.dainv, L.Hq, Spad, L.B))
         return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
