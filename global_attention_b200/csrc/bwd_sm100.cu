@@ -856,7 +856,8 @@ struct BwdKTcSmem {
     // 4 deep: the prologue writes a unit's scales at its start, while the epilogue of an earlier
     // unit may still read its own (with one query head per KV head a unit has two iterations)
     float uinv[4];           // 2^-E, E = the unit's smallest dA row exponent, by unit number % 4
-    float kmdot[2][TF_BN];   // mean(dy gamma xhat) of each key row (RMSNorm backward), by unit parity
+    float kmdot[2][2][TF_BN];  // mean(dy gamma xhat) of each key row (RMSNorm backward): the two
+                               // softmax warpgroups' shares, by unit parity
     float red[2][2][4];      // per-warp maxima for the unit statistics, by call parity
     float dgk[4][kD];        // this CTA's d_gamma_k, one slice per epilogue warp
     uint64_t bar[KB_COUNT];
@@ -944,8 +945,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
     const float mdot_f = c2 * kLn2 / (float)kD;  // scale / (D oscale^2)
 
     // Registers by warpgroup (4 x 128 in all, set at the top of each role): TMA / MMA issue
-    // 64, softmax 128, prologue 128, epilogue 192 (it holds a whole dk~ row so that it can
-    // release TMEM before its arithmetic).
+    // 64, the two softmax warpgroups 128 each, epilogue 192 (it holds a whole dk~ row so that
+    // it can release TMEM before its arithmetic).
     if (warp < 4) {
         reg_dealloc<64>();
         if (warp == 0) {
@@ -1093,9 +1094,11 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 mbar_wait(&sm.bar[KB_DONE], 0, abort, 214);
             }
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= 4 && warp < 12) {
         // ================================================ P^T, dS^T (thread = key row)
-        const int r = tid - 128, wq = warp - 4;
+        // Two warpgroups: warps 4-7 take the first 64-query half of every iteration (TMEM
+        // buffer 0), warps 8-11 the second (buffer 1), so the halves' softmax runs in parallel.
+        const int r = (tid - 128) & 127, wq = warp & 3, my_half = warp >= 8 ? 1 : 0;
         const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
         int it_all = 0, uu = 0;
         bool ok = true;
@@ -1109,9 +1112,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 decode_iter(L, x, it, qb, hg);
                 const int q0 = qb * TF_BM;
                 const int jmin = x.kt * TF_BN + 32 * wq, jmax = jmin + 31;
-                for (int half = 0; half < 2 && ok; ++half) {
+                for (int half = my_half; half == my_half && ok; ++half) {
                     const int hs = 2 * it_all + half, slot = hs % KV_SLOTS;
-                    if (it == 0 && half == 0) {
+                    if (it == 0) {
                         if (!(ok = mbar_wait(&sm.bar[KB_STATS + (uu & 1)], (uu >> 1) & 1, abort, 223))) break;
                         vin = sm.vtinv[uu & 3];        // undoes the V tile scale of dP^T
                         su = 1.0f / sm.uinv[uu & 3];   // 2^E: P^T columns carry 2^(E - e_i)
@@ -1149,15 +1152,13 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                         tmem_st16(tX + 16 * c8, pp);       // P^T over S^T (already read)
                         tmem_st16(tX + 64 + 16 * c8, dd);  // dS^T over dP^T
                     }
-                    if (half == 1 && it == x.nit - 1) sm.kmdot[uu & 1][r] = kacc * mdot_f;
+                    if (it == x.nit - 1) sm.kmdot[my_half][uu & 1][r] = kacc * mdot_f;  // the epilogue adds both
                     tmem_wait_st();
                     tc_fence_before();
                     mbar_arrive(&sm.bar[KB_PFULL + half]);
                 }
             }
         }
-    } else if (warp >= 8 && warp < 12) {
-        // (no prologue: the slots' per-column values arrive by TMA with their rows)
     } else if (warp >= 12) {
         reg_alloc<192>();
         // ================================================ unit scales; dv, dk epilogue (thread = key row)
@@ -1266,7 +1267,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             tmem_ld32f(TM_DK + lane_off + 96, dy + 96);
             tmem_wait_ld();
             const float f = L.scale / (sm.dsc[uu & 3][r] * oscale);
-            const float mdot = sm.kmdot[uu & 1][r];
+            const float mdot = sm.kmdot[0][uu & 1][r] + sm.kmdot[1][uu & 1][r];
             const float rinv = valid ? p.krinv[((size_t)x.b * L.Hkv + x.kvh) * L.S + j] : 0.f;
             tc_fence_before();
             mbar_arrive(&sm.bar[KB_DVKEMPTY]);  // dV, dK of the unit are out of TMEM
