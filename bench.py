@@ -44,6 +44,38 @@ WORKLOADS = {
 HQ, HKV, D = 32, 8, 128
 
 
+# ---------------------------------------------------------------- ranks (one process per GPU)
+#
+# Sequences are independent problems, so the ranks share no data: each draws its own batch
+# (seed = rank) and the only cross-rank traffic is the timing reduction below.
+
+def rank_env():
+    """(world, rank, local_rank) from the launcher's environment (1, 0, 0 without one)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's synthetic batch: distinct per rank, the same on every run."""
+    return rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Largest value of x over all ranks (every rank receives it); x itself when world == 1."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's step time."""
+    return tokens_per_rank * world / (ms_per_step / 1e3)
+
+
 def pairs(S: int, W: int) -> int:
     """Visible (i, j) pairs per (batch, head): sum_i min(i+1, W)."""
     if W >= S:
@@ -189,7 +221,7 @@ def cpu_sample_shape(Bw, Sw, W):
 
 def run_reference(args):
     """--impl reference: the fp64 CPU oracle as it stands, each step a bounded sample."""
-    rank = int(os.environ.get("RANK", "0"))
+    _, rank, _ = rank_env()
     if rank != 0:
         return 0
     import oracle
@@ -240,9 +272,7 @@ def main():
     import global_attention_b200 as ga
     from global_attention_b200.synth import make_inputs
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device"}))
         return 1
@@ -255,7 +285,7 @@ def main():
 
     Bw, Sw, W, bwd = WORKLOADS[args.workload]
     wk = work(Bw, Sw, W, bwd)
-    t = make_inputs(Bw, Sw, seed=rank, with_dout=bwd)
+    t = make_inputs(Bw, Sw, seed=rank_seed(rank), with_dout=bwd)
     host = {k: v.pin_memory() for k, v in t.items()}
     d = {k: v.to(dev) for k, v in host.items()}
     stream = torch.cuda.current_stream()
@@ -310,10 +340,7 @@ def main():
     kern_ms = {fwd_name: fwd_ms}
     for k, n in enumerate(bwd_names):
         kern_ms[n] = statistics.mean(ev_m[i][k][0].elapsed_time(ev_m[i][k][1]) for i in range(args.steps))
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, world, dev)
     ms_step = ms / args.steps
 
     # ---- end to end through the public API: pinned host inputs -> HBM -> fwd+bwd -> host
@@ -342,10 +369,8 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
     if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
         dist.barrier()
 
     if rank != 0:
@@ -354,7 +379,7 @@ def main():
 
     peaks, peak_src = load_peaks()
     tokens_step = wk["tokens"] * world
-    value = tokens_step / (ms_step / 1e3)
+    value = job_throughput(wk["tokens"], world, ms_step)
     # roofline of the whole step and of the dominant kernel
     step_bytes = wk["fwd_bytes"] + wk["bwd_bytes"]
     step_flops = wk["fwd_flops"] + wk["bwd_flops"]
@@ -398,7 +423,7 @@ def main():
         "roofline_step_ms": t_roof * 1e3,
         "roofline": roof,
         "cpu_baseline": cpu,
-        "e2e": {"value": tokens_step / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_throughput(wk["tokens"], world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
