@@ -40,7 +40,11 @@ WORKLOADS = {
     "tiny_fwd": (1, 1024, 128, False),
     "swa16k_b1_fwd": (1, 16384, 128, False),
     "swa16k_b1": (1, 16384, 128, True),
+    # one sliding (W=128) and one global (W=S) layer on the same inputs, reported with the
+    # 5:1 sliding:global weighted time per layer of the model's layer pattern
+    "mix256k_fwd": (1, 262144, 128, False),
 }
+LAYER_MIX = {"mix256k_fwd": ((128, 5), (None, 1))}   # (window or None = global, weight)
 HQ, HKV, D = 32, 8, 128
 
 
@@ -99,6 +103,8 @@ def work(B, S, W, bwd):
     kernels = {
         "fwd_mma_kernel": (fwd_bytes, fwd_flops),
         "fwd_tc_kernel": (fwd_bytes, fwd_flops),
+        # wide-window / global forward: q, K~16 (fp16), v, g -> out, lse (K~ prepared from k first)
+        "fwd_glob_tc_kernel": (fwd_bytes, fwd_flops),
         # dout, out, g -> dg, dA
         "bwd_pre_kernel": (5 * qb, 0),
         # q, k, v, dA, lse -> dq, Delta ; S, dP, dQ
@@ -211,6 +217,12 @@ def cpu_oracle_run(B, S, W, bwd, seed=0):
     return time.perf_counter() - t0
 
 
+def pair_scaled(secs, B, S, W, S_full, W_full):
+    """Seconds per token of the (S_full, W_full) layer from an oracle run over B x S tokens with
+    window W: the oracle's work is proportional to the visible (query, key) pairs."""
+    return secs / (B * pairs(S, W)) * pairs(S_full, W_full) / S_full
+
+
 def cpu_sample_shape(Bw, Sw, W):
     """A bounded sample of the workload for the oracle: same heads and window, fewer and
     shorter sequences (window work per token is the same once past the first W tokens)."""
@@ -227,14 +239,22 @@ def run_reference(args):
     import oracle
     oracle.build()
     Bw, Sw, W, bwd = WORKLOADS[args.workload]
-    B, S, Wc = (1, 512, 512) if W >= Sw else (1, 1024, W)
+    # one sample per layer of the step: (B, S, window) with every layer's window kept
+    shapes = [(1, 512, 512) if lw >= Sw else (1, 1024, lw) for lw, _ in layers_of(args.workload)]
+
+    def one(seed=0):   # seconds per token of a whole step
+        return sum(pair_scaled(cpu_oracle_run(B, S, Wc, bwd, seed=seed), B, S, Wc, Sw, lw)
+                   for (B, S, Wc), (lw, _) in zip(shapes, layers_of(args.workload)))
+
     for _ in range(args.warmup):
-        cpu_oracle_run(B, S, Wc, bwd)
-    times = [cpu_oracle_run(B, S, Wc, bwd, seed=i) for i in range(args.steps)]
-    ms = 1e3 * sum(times) / len(times)
-    val = B * S / (ms / 1e3)
+        one()
+    spt = sum(one(seed=i) for i in range(args.steps)) / args.steps
+    val = 1.0 / spt
+    ms = 1e3 * Bw * Sw * spt          # the workload's step at this rate
     cores = oracle.num_threads()
-    sample = f"{B}x{S} tokens per step, window {Wc}, fwd{'+bwd' if bwd else ''}, fp64, {cores} threads"
+    sample = "; ".join(f"{B}x{S} tokens, window {Wc}" for B, S, Wc in shapes)
+    sample += (f" per step, fwd{'+bwd' if bwd else ''}, fp64, {cores} threads; time per visible (query, key) "
+               "pair scaled to the workload's pairs per token")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -246,8 +266,20 @@ def run_reference(args):
     return 0
 
 
+def layers_of(w):
+    """[(window, weight)] of the layers one step of workload w runs."""
+    B, S, W, bwd = WORKLOADS[w]
+    if w in LAYER_MIX:
+        return [(S if lw is None else lw, wt) for lw, wt in LAYER_MIX[w]]
+    return [(W, 1)]
+
+
 def workload_name(w):
     B, S, W, bwd = WORKLOADS[w]
+    if w in LAYER_MIX:
+        mix = ":".join(str(wt) for _, wt in LAYER_MIX[w])
+        return (f"gated sliding W={W} + global (full causal) attention fwd on the same inputs, {mix} layer mix, "
+                f"B={B} S={S} Hq={HQ} Hkv={HKV} D={D}")
     kind = "global (full causal)" if W >= S else f"sliding window W={W}"
     return f"gated {kind} attention {'fwd+bwd' if bwd else 'fwd'}, B={B} S={S} Hq={HQ} Hkv={HKV} D={D}"
 
@@ -284,7 +316,10 @@ def main():
     ga.load()
 
     Bw, Sw, W, bwd = WORKLOADS[args.workload]
-    wk = work(Bw, Sw, W, bwd)
+    layers = layers_of(args.workload)
+    wks = [work(Bw, Sw, lw, bwd) for lw, _ in layers]
+    wk = {k: sum(x[k] for x in wks) for k in ("fwd_bytes", "fwd_flops", "bwd_bytes", "bwd_flops")}
+    wk["tokens"] = Bw * Sw
     t = make_inputs(Bw, Sw, seed=rank_seed(rank), with_dout=bwd)
     host = {k: v.pin_memory() for k, v in t.items()}
     d = {k: v.to(dev) for k, v in host.items()}
@@ -299,23 +334,30 @@ def main():
         ws = torch.empty(max(256, ga.zgcm_attn_bwd_workspace_size(Bw, Sw, HQ, HKV, D, W)),
                          dtype=torch.uint8, device=dev)
 
-    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
-    bwd_names = ga.zgcm_attn_bwd_kernel_names(Sw, W) if bwd else []
-    ev_m = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in bwd_names] for _ in range(args.steps)]
+    def pair():
+        return (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+
+    # per layer: the forward's events, and one event pair per backward kernel
+    ev_f = [[pair() for _ in layers] for _ in range(args.steps)]
+    bwd_names = [ga.zgcm_attn_bwd_kernel_names(Sw, lw) if bwd else [] for lw, _ in layers]
+    ev_m = [[[pair() for _ in names] for names in bwd_names] for _ in range(args.steps)]
+
+    # forward scratch (normalised keys of the wide-window kernel), allocated once
+    fws = [None if n == 0 else torch.empty(n, dtype=torch.uint8, device=dev)
+           for n in (ga.zgcm_attn_fwd_workspace_size(Bw, Sw, HQ, HKV, D, 42, lw) for lw, _ in layers)]
 
     def step(i=None, src=d):
-        if i is not None:
-            ev_f[i][0].record(stream)
-        ga.zgcm_attn_fwd(src["q"], src["k"], src["v"], src["g"], src["gamma_q"], src["gamma_k"],
-                         window=W, out=out, lse=lse, stream=stream)
-        if i is not None:
-            ev_f[i][1].record(stream)
-        if bwd:
-            ga.zgcm_attn_bwd(src["q"], src["k"], src["v"], src["g"], src["gamma_q"], src["gamma_k"],
-                             out, lse, src["dout"], window=W, grads=grads, workspace=ws, stream=stream,
-                             kernel_events=None if i is None else ev_m[i])
+        for li, (lw, _) in enumerate(layers):
+            if i is not None:
+                ev_f[i][li][0].record(stream)
+            ga.zgcm_attn_fwd(src["q"], src["k"], src["v"], src["g"], src["gamma_q"], src["gamma_k"],
+                             window=lw, out=out, lse=lse, workspace=fws[li], stream=stream)
+            if i is not None:
+                ev_f[i][li][1].record(stream)
+            if bwd:
+                ga.zgcm_attn_bwd(src["q"], src["k"], src["v"], src["g"], src["gamma_q"], src["gamma_k"],
+                                 out, lse, src["dout"], window=lw, grads=grads, workspace=ws, stream=stream,
+                                 kernel_events=None if i is None else ev_m[i][li])
 
     for _ in range(args.warmup):
         step()
@@ -335,11 +377,21 @@ def main():
     if world > 1:
         dist.barrier()
     ms = t0.elapsed_time(t1)
-    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_f)
-    fwd_name = ga.zgcm_attn_fwd_kernel_name(Bw, Sw, HQ, HKV, 42, W)
-    kern_ms = {fwd_name: fwd_ms}
-    for k, n in enumerate(bwd_names):
-        kern_ms[n] = statistics.mean(ev_m[i][k][0].elapsed_time(ev_m[i][k][1]) for i in range(args.steps))
+    # per kernel and layer: (mean ms, algorithmic bytes, flops); the key names the kernel, and
+    # the layer's window when the step runs more than one layer
+    kern, layer_ms = {}, []
+    for li, (lw, _) in enumerate(layers):
+        tag = "" if len(layers) == 1 else f" (W={lw})"
+        fwd_name = ga.zgcm_attn_fwd_kernel_name(Bw, Sw, HQ, HKV, 42, lw)
+        fms = statistics.mean(ev_f[i][li][0].elapsed_time(ev_f[i][li][1]) for i in range(args.steps))
+        kern[fwd_name + tag] = (fms, *wks[li]["kernels"].get(fwd_name, (0, 0)))
+        lms = fms
+        for k, n in enumerate(bwd_names[li]):
+            kms_ = statistics.mean(ev_m[i][li][k][0].elapsed_time(ev_m[i][li][k][1]) for i in range(args.steps))
+            kern[n + tag] = (kms_, *wks[li]["kernels"].get(n, (0, 0)))
+            lms += kms_
+        layer_ms.append(lms)
+    kern_ms = {n: v[0] for n, v in kern.items()}
     ms = max_over_ranks(ms, world, dev)
     ms_step = ms / args.steps
 
@@ -384,7 +436,7 @@ def main():
     step_bytes = wk["fwd_bytes"] + wk["bwd_bytes"]
     step_flops = wk["fwd_flops"] + wk["bwd_flops"]
     t_roof = max(step_bytes / (peaks["hbm_gbs"] * 1e9), step_flops / (peaks["bf16_tflops"] * 1e12))
-    kern = {n: (ms_, *wk["kernels"][n]) for n, ms_ in kern_ms.items() if n in wk["kernels"]}
+    kern = {n: v for n, v in kern.items() if v[1] or v[2]}
     name = max(kern, key=lambda k: kern[k][0])
     kms, kbytes, kflops = kern[name]
     t_hbm = kbytes / (peaks["hbm_gbs"] * 1e9)
@@ -395,7 +447,7 @@ def main():
         roof = {"bound": "tensor", "achieved": kflops / (kms / 1e3) / 1e12,
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = traffic_for(name, args.workload)
+    roof["traffic"] = traffic_for(name.split(" (W=")[0], args.workload)
     roof.update({"kernel": name, "kernel_ms": kms, "algorithmic_bytes": kbytes, "flops": kflops,
                  "peak_source": peak_src, "kernels_ms": kern_ms})
 
@@ -403,13 +455,22 @@ def main():
     if world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        Bc, Sc, Wc = cpu_sample_shape(Bw, Sw, W)
-        secs = cpu_oracle_run(Bc, Sc, Wc, bwd)
-        cpu = {"value": Bc * Sc / secs, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-               "sample": f"{Bc}x{Sc} tokens, window {Wc}, fwd{'+bwd' if bwd else ''} in fp64 "
-                         f"({secs:.1f} s); same heads/window as the workload"}
+        # seconds per token of each layer of the step, each on its own bounded sample
+        spt, parts = 0.0, []
+        for lw, _ in layers:
+            Bc, Sc, Wc = cpu_sample_shape(Bw, Sw, lw)
+            secs = cpu_oracle_run(Bc, Sc, Wc, bwd)
+            spt += pair_scaled(secs, Bc, Sc, Wc, Sw, lw)
+            parts.append(f"{Bc}x{Sc} tokens, window {Wc}, fwd{'+bwd' if bwd else ''} in fp64 ({secs:.1f} s)")
+        cpu = {"value": 1.0 / spt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+               "sample": "; ".join(parts) + "; same heads as the workload, time per visible (query, key) "
+                         "pair scaled to the workload's pairs per token"}
 
-    launches_per_step = 1 + len(bwd_names)     # fwd + every backward kernel
+    # per layer: the forward's kernels (the wide-window forward runs a key preparation kernel
+    # first) + every backward kernel
+    fwd_launches = [2 if ga.zgcm_attn_fwd_kernel_name(Bw, Sw, HQ, HKV, 42, lw) == "fwd_glob_tc_kernel" else 1
+                    for lw, _ in layers]
+    launches_per_step = sum(f + len(n) for f, n in zip(fwd_launches, bwd_names))
     rec = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -428,6 +489,12 @@ def main():
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
+    if len(layers) > 1:
+        wsum = sum(wt for _, wt in layers)
+        mix_ms = sum(wt * t for (_, wt), t in zip(layers, layer_ms)) / wsum
+        rec["layer_mix"] = {"layers": [{"window": lw, "weight": wt, "ms": t} for (lw, wt), t in zip(layers, layer_ms)],
+                            "weighted_ms_per_layer": mix_ms,
+                            "weighted_tokens_per_s": wk["tokens"] / (mix_ms / 1e3)}
     print(json.dumps(rec))
     if world > 1:
         dist.destroy_process_group()

@@ -44,6 +44,10 @@ def load() -> ctypes.CDLL:
         lib.zgcm_status_string.restype = ctypes.c_char_p
         lib.zgcm_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, d, i, i, f, f, vp, vp, vp]
         lib.zgcm_attn_fwd.restype = i
+        lib.zgcm_attn_fwd_ws.argtypes = lib.zgcm_attn_fwd.argtypes[:-1] + [vp, ctypes.c_size_t, vp]
+        lib.zgcm_attn_fwd_ws.restype = i
+        lib.zgcm_attn_fwd_workspace_size.argtypes = [i, i, i, i, i, i, i]
+        lib.zgcm_attn_fwd_workspace_size.restype = ctypes.c_size_t
         lib.zgcm_attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
         lib.zgcm_attn_bwd_workspace_size.restype = ctypes.c_size_t
         lib.zgcm_attn_bwd.argtypes = ([vp] * 9 + [i] * 6 + [d, i, i, f, f] + [vp] * 7 +
@@ -86,9 +90,17 @@ def _check(t, name, dtype, ndim):
         raise TypeError(f"{name} must be a contiguous {dtype} tensor of rank {ndim}")
 
 
+def zgcm_attn_fwd_workspace_size(B, S, Hq, Hkv, D=128, rope_dims=42, window=128) -> int:
+    """Bytes of device scratch the forward needs (0 for windows up to 128)."""
+    return int(load().zgcm_attn_fwd_workspace_size(int(B), int(S), int(Hq), int(Hkv), int(D), int(rope_dims),
+                                                   int(window)))
+
+
 def zgcm_attn_fwd(q, k, v, g, gamma_q, gamma_k, *, rope_dims=42, rope_base=10000.0, window=128,
-                  causal=1, eps=1e-6, scale=None, out=None, lse=None, stream=None):
-    """Gated window-attention forward.  Returns (out bf16 [B,S,Hq,D], lse fp32 [B,Hq,S])."""
+                  causal=1, eps=1e-6, scale=None, out=None, lse=None, workspace=None, stream=None):
+    """Gated window-attention forward.  Returns (out bf16 [B,S,Hq,D], lse fp32 [B,Hq,S]).
+    `workspace`: a uint8 device tensor of at least zgcm_attn_fwd_workspace_size bytes, or None
+    to allocate it here when the configuration needs one."""
     import torch
     for n, t in (("q", q), ("k", k), ("v", v), ("g", g)):
         _check(t, n, torch.bfloat16, 4)
@@ -102,10 +114,14 @@ def zgcm_attn_fwd(q, k, v, g, gamma_q, gamma_k, *, rope_dims=42, rope_base=10000
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
-    st = load().zgcm_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma_q), _ptr(gamma_k),
-                              B, S, Hq, Hkv, D, int(rope_dims), float(rope_base), int(window),
-                              int(causal), float(eps), float(scale), _ptr(out), _ptr(lse),
-                              _stream(stream))
+    need = zgcm_attn_fwd_workspace_size(B, S, Hq, Hkv, D, rope_dims, window)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel())
+    st = load().zgcm_attn_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma_q), _ptr(gamma_k),
+                                 B, S, Hq, Hkv, D, int(rope_dims), float(rope_base), int(window),
+                                 int(causal), float(eps), float(scale), _ptr(out), _ptr(lse),
+                                 ws_ptr, ws_bytes, _stream(stream))
     if st != ZGCM_OK:
         raise ZgcmError(st, "zgcm_attn_fwd")
     return out, lse

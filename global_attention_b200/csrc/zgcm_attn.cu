@@ -12,6 +12,9 @@ namespace zgcm {
 cudaError_t launch_fwd_mma(const FwdParams& p, cudaStream_t stream);
 cudaError_t launch_fwd_tc(const FwdParams& p, int* err_word, cudaStream_t stream);
 bool fwd_tc_supported(const LayerParams& L);
+cudaError_t launch_fwd_glob_tc(const FwdParams& p, void* workspace, int* err_word, cudaStream_t stream);
+bool fwd_glob_supported(const LayerParams& L);
+size_t fwd_glob_workspace_bytes(int B, int S, int Hkv);
 cudaError_t launch_bwd_mma(const BwdParams& p, cudaStream_t stream, void* const* events, int n_pairs);
 extern const char* const kBwdMmaKernelNames[];
 extern const int kBwdMmaKernelCount;
@@ -46,6 +49,24 @@ bool force_mma() {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Forward kernel for a layer: the sliding-window tcgen05 kernel (W <= 128), the wide-window /
+// global tcgen05 pair (W > 128), else (or with ZGCM_FORCE_MMA=1) the warp-MMA kernel.
+enum class FwdPath { TC, GLOB, MMA };
+
+FwdPath fwd_path(const LayerParams& L) {
+    if (force_mma()) return FwdPath::MMA;
+    if (fwd_tc_supported(L)) return FwdPath::TC;
+    if (fwd_glob_supported(L)) return FwdPath::GLOB;
+    return FwdPath::MMA;
+}
+
+LayerParams shape_only(int B, int S, int Hq, int Hkv, int rope_dims, int window) {
+    LayerParams L{};
+    L.B = B; L.S = S; L.Hq = Hq; L.Hkv = Hkv; L.G = Hkv > 0 ? Hq / Hkv : 0;
+    L.rope_half = rope_dims / 2; L.W = window;
+    return L;
+}
 
 // Checks shared by forward and backward.  Returns ZGCM_OK or the first failing status.
 int check_shape(int B, int S, int Hq, int Hkv, int D, int rope_dims, double rope_base, int window,
@@ -126,11 +147,19 @@ const char* zgcm_status_string(int status) {
     }
 }
 
-int zgcm_attn_fwd(const void* q, const void* k, const void* v, const void* g,
-                  const float* gamma_q, const float* gamma_k,
-                  int B, int S, int Hq, int Hkv, int D, int rope_dims,
-                  double rope_base, int window, int causal, float eps, float scale,
-                  void* out, float* lse, void* cuda_stream) {
+size_t zgcm_attn_fwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int rope_dims, int window) {
+    if (check_shape(B, S, Hq, Hkv, D, rope_dims, 1.0, window, 1, 0.f, 1.f) != ZGCM_OK) return 0;
+    if ((long long)B * S == 0) return 0;
+    return fwd_path(shape_only(B, S, Hq, Hkv, rope_dims, window)) == FwdPath::GLOB
+               ? align256(fwd_glob_workspace_bytes(B, S, Hkv))
+               : 0;
+}
+
+int zgcm_attn_fwd_ws(const void* q, const void* k, const void* v, const void* g,
+                     const float* gamma_q, const float* gamma_k,
+                     int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                     double rope_base, int window, int causal, float eps, float scale,
+                     void* out, float* lse, void* workspace, size_t workspace_bytes, void* cuda_stream) {
     int st = check_shape(B, S, Hq, Hkv, D, rope_dims, rope_base, window, causal, eps, scale);
     if (st != ZGCM_OK) return st;
     if ((long long)B * S == 0) return ZGCM_OK;
@@ -139,16 +168,42 @@ int zgcm_attn_fwd(const void* q, const void* k, const void* v, const void* g,
         if (!p) return ZGCM_ERR_INVALID_ARG;
     for (const void* p : ptrs)
         if (!aligned16(p)) return ZGCM_ERR_ALIGNMENT;
+    const size_t need = zgcm_attn_fwd_workspace_size(B, S, Hq, Hkv, D, rope_dims, window);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need) return ZGCM_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ZGCM_ERR_ALIGNMENT;
+    }
     FwdParams p;
     fill_layer(p.L, q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, rope_dims, rope_base, window, eps, scale);
     p.out = static_cast<bf16*>(out);
     p.lse = lse;
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     cudaError_t e;
-    if (!force_mma() && fwd_tc_supported(p.L))
-        e = launch_fwd_tc(p, device_error_word(), stream);
-    else
-        e = launch_fwd_mma(p, stream);
+    switch (fwd_path(p.L)) {
+        case FwdPath::TC: e = launch_fwd_tc(p, device_error_word(), stream); break;
+        case FwdPath::GLOB: e = launch_fwd_glob_tc(p, workspace, device_error_word(), stream); break;
+        default: e = launch_fwd_mma(p, stream); break;
+    }
+    return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
+}
+
+int zgcm_attn_fwd(const void* q, const void* k, const void* v, const void* g,
+                  const float* gamma_q, const float* gamma_k,
+                  int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                  double rope_base, int window, int causal, float eps, float scale,
+                  void* out, float* lse, void* cuda_stream) {
+    const size_t need = zgcm_attn_fwd_workspace_size(B, S, Hq, Hkv, D, rope_dims, window);
+    if (need == 0)
+        return zgcm_attn_fwd_ws(q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, D, rope_dims, rope_base, window,
+                                causal, eps, scale, out, lse, nullptr, 0, cuda_stream);
+    // stream-ordered scratch: taken from and returned to the device's default memory pool
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    void* ws = nullptr;
+    if (cudaMallocAsync(&ws, need, stream) != cudaSuccess) return ZGCM_ERR_CUDA;
+    const int st = zgcm_attn_fwd_ws(q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, D, rope_dims, rope_base,
+                                    window, causal, eps, scale, out, lse, ws, need, cuda_stream);
+    const cudaError_t e = cudaFreeAsync(ws, stream);
+    if (st != ZGCM_OK) return st;
     return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
 }
 
@@ -160,9 +215,11 @@ int zgcm_attn_device_error(void) {
 }
 
 const char* zgcm_attn_fwd_kernel_name(int B, int S, int Hq, int Hkv, int rope_dims, int window) {
-    LayerParams L{};
-    L.B = B; L.S = S; L.Hq = Hq; L.Hkv = Hkv; L.rope_half = rope_dims / 2; L.W = window;
-    return (!force_mma() && fwd_tc_supported(L)) ? "fwd_tc_kernel" : "fwd_mma_kernel";
+    switch (fwd_path(shape_only(B, S, Hq, Hkv, rope_dims, window))) {
+        case FwdPath::TC: return "fwd_tc_kernel";
+        case FwdPath::GLOB: return "fwd_glob_tc_kernel";
+        default: return "fwd_mma_kernel";
+    }
 }
 
 size_t zgcm_attn_bwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int window) {

@@ -27,8 +27,10 @@
  *     unless stated: q, g, out, dout, dq, dg are [B, S, Hq, D]; k, v, dk, dv are
  *     [B, S, Hkv, D]; lse is fp32 [B, Hq, S]; gamma_q, gamma_k, dgamma_q, dgamma_k are
  *     fp32 [D].  Every pointer must be 16-byte aligned (ZGCM_ERR_ALIGNMENT otherwise).
- *   - Ownership: the caller owns every buffer.  The library never allocates device memory
- *     and keeps no state between calls.
+ *   - Ownership: the caller owns every buffer.  The library keeps no state between calls
+ *     and allocates no device memory, with one exception: zgcm_attn_fwd on a window wider
+ *     than 128 takes its scratch from the device's stream-ordered pool (see there);
+ *     zgcm_attn_fwd_ws is the same call with caller-owned scratch.
  *   - Streams: every call is asynchronous on `cuda_stream` (a cudaStream_t, NULL = legacy
  *     default stream) and never synchronises the device.
  *   - Errors: arguments are checked on the host before anything is launched; a failed
@@ -78,12 +80,36 @@ const char* zgcm_status_string(int status);
  * In : q, g bf16 [B,S,Hq,D]; k, v bf16 [B,S,Hkv,D]; gamma_q, gamma_k fp32 [D].
  * Out: out bf16 [B,S,Hq,D] (rounded once, to nearest even); lse fp32 [B,Hq,S].
  * out/lse must not alias any input.
+ * Windows wider than 128 (the global layer, window >= S, among them) need device scratch
+ * for the normalised keys (zgcm_attn_fwd_workspace_size bytes): this call takes it with
+ * cudaMallocAsync on `cuda_stream` and returns it with cudaFreeAsync after the kernels,
+ * so it never synchronises; callers that manage memory themselves use zgcm_attn_fwd_ws.
  */
 int zgcm_attn_fwd(const void* q, const void* k, const void* v, const void* g,
                   const float* gamma_q, const float* gamma_k,
                   int B, int S, int Hq, int Hkv, int D, int rope_dims,
                   double rope_base, int window, int causal, float eps, float scale,
                   void* out, float* lse, void* cuda_stream);
+
+/*
+ * Bytes of device scratch the forward needs for this configuration: 0 for windows up to
+ * 128 (the sliding layers), B*S*Hkv*D*2 rounded up to 256 for wider windows with 42
+ * rotated dims and an even Hq/Hkv (the fp16 normalised, rotated keys, written by the
+ * forward's preparation kernel and read by its attention kernel).  0 for invalid arguments.
+ */
+size_t zgcm_attn_fwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int rope_dims, int window);
+
+/*
+ * zgcm_attn_fwd with caller-owned scratch: workspace must hold at least
+ * zgcm_attn_fwd_workspace_size(...) bytes, 256-byte aligned (may be NULL when that is 0),
+ * contents on entry irrelevant, not used by a concurrent call.  ZGCM_ERR_WORKSPACE if it
+ * is missing or too small.
+ */
+int zgcm_attn_fwd_ws(const void* q, const void* k, const void* v, const void* g,
+                     const float* gamma_q, const float* gamma_k,
+                     int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                     double rope_base, int window, int causal, float eps, float scale,
+                     void* out, float* lse, void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
  * Bytes of device workspace zgcm_attn_bwd needs for this problem (0 for an empty one).
@@ -159,9 +185,12 @@ int zgcm_attn_bwd_noalloc(const void* q, const void* k, const void* v, const voi
                           float* dgamma_q, float* dgamma_k, void* cuda_stream);
 
 /*
- * Kernel zgcm_attn_fwd launches for this configuration (static string): "fwd_tc_kernel"
- * (tcgen05/TMEM/TMA, sliding windows up to 128 with 42 rotated dims) or "fwd_mma_kernel".
- * Setting the environment variable ZGCM_FORCE_MMA=1 selects the warp-MMA kernels.
+ * Main kernel zgcm_attn_fwd launches for this configuration (static string):
+ * "fwd_tc_kernel" (tcgen05/TMEM/TMA, sliding windows up to 128 with 42 rotated dims),
+ * "fwd_glob_tc_kernel" (tcgen05, wider windows and the global layer, with 42 rotated dims
+ * and an even Hq/Hkv; preceded by the key preparation kernel fwd_prep_k_kernel) or
+ * "fwd_mma_kernel" (warp MMA, every other shape).  Setting the environment variable
+ * ZGCM_FORCE_MMA=1 selects the warp-MMA kernels.
  */
 const char* zgcm_attn_fwd_kernel_name(int B, int S, int Hq, int Hkv, int rope_dims, int window);
 

@@ -109,3 +109,40 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(ga, "LIB_PATH", "/nonexistent/libzgcm_attn.so")
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         ga.load()
+
+
+def _fwd_ws(lib, ws, ws_bytes, **kw):
+    a = dict(ARGS, **kw)
+    vp = ctypes.c_void_p
+    p = [vp(P + 256 * i) for i in range(8)]
+    return lib.zgcm_attn_fwd_ws(*p[:6], a["B"], a["S"], a["Hq"], a["Hkv"], a["D"], a["rope_dims"],
+                                a["rope_base"], a["window"], a["causal"], a["eps"], a["scale"],
+                                p[6], p[7], vp(ws), ws_bytes, None)
+
+
+def test_fwd_workspace_size_query(lib):
+    ws = lambda *a: lib.zgcm_attn_fwd_workspace_size(*a)
+    # sliding windows up to one key tile need none
+    assert ws(4, 16384, 32, 8, 128, 42, 128) == 0
+    assert ws(1, 1024, 32, 8, 128, 42, 7) == 0
+    # wider windows and the global layer: the fp16 normalised keys, [B, S, Hkv, D]
+    for B, S, W in ((1, 65536, 65536), (2, 1000, 300), (1, 1, 10**6), (3, 777, 129)):
+        n = B * S * 8 * 128 * 2
+        assert ws(B, S, 32, 8, 128, 42, W) == (n + 255) // 256 * 256
+    # the warp-MMA kernel takes the rest (no rotation, odd group size) and needs none
+    assert ws(1, 1024, 32, 8, 128, 0, 1024) == 0
+    assert ws(1, 1024, 24, 8, 128, 42, 1024) == 0
+    # invalid or empty -> 0
+    assert ws(1, 1024, 32, 8, 64, 42, 1024) == 0
+    assert ws(0, 1024, 32, 8, 128, 42, 1024) == 0
+    assert ws(1, 1024, 30, 8, 128, 42, 1024) == 0
+
+
+def test_fwd_ws_checks(lib):
+    need = lib.zgcm_attn_fwd_workspace_size(1, 640, 32, 8, 128, 42, 640)
+    assert need > 0
+    assert _fwd_ws(lib, P + 256 * 40, need - 1, S=640, window=640) == -4
+    assert _fwd_ws(lib, 0, need, S=640, window=640) == -4
+    assert _fwd_ws(lib, P + 256 * 40 + 16, need, S=640, window=640) == -3
+    assert _fwd_ws(lib, P + 256 * 40, need, S=640, window=640, D=96) == -2
+    assert _fwd_ws(lib, P + 256 * 40, need, S=640, window=0) == -1

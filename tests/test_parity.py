@@ -98,6 +98,33 @@ def test_forward_both_kernel_paths(B, S, W, monkeypatch):
         assert_lse_close(f"lse[{name}]", l, ref_lse)
 
 
+@pytest.mark.parametrize("B,S,W", [(1, 777, 777), (2, 1000, 10**6), (1, 129, 129), (1, 1, 4096),
+                                   (3, 260, 200), (1, 1300, 300), (2, 640, 129), (1, 2048, 2048)])
+def test_forward_wide_window_kernel(B, S, W, monkeypatch):
+    """Windows wider than one key tile (the global layer W >= S among them) run the tcgen05
+    wide-window forward; it matches the oracle and the forced warp-MMA kernel's tolerance."""
+    t = make_inputs(B, S, seed=300 + S + W % 1000)
+    d = _to_dev(t)
+    ref_out, ref_lse = _problem(t, window=W).forward()
+    monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
+    assert ga.zgcm_attn_fwd_kernel_name(B, S, 32, 8, 42, W) == "fwd_glob_tc_kernel"
+    out, lse = _gpu_fwd(d, window=W)
+    assert ga.zgcm_attn_device_error() == 0
+    assert_bf16_close("out", out, ref_out)
+    assert_lse_close("lse", lse, ref_lse)
+    # the same call through the plain C entry (scratch from the stream-ordered pool)
+    import ctypes
+    lib = ga.load()
+    out2, lse2 = torch.empty_like(out), torch.empty_like(lse)
+    vp = lambda x: ctypes.c_void_p(x.data_ptr())
+    st = lib.zgcm_attn_fwd(vp(d["q"]), vp(d["k"]), vp(d["v"]), vp(d["g"]), vp(d["gamma_q"]), vp(d["gamma_k"]),
+                           B, S, 32, 8, 128, 42, 10000.0, W, 1, 1e-6, 128 ** -0.5, vp(out2), vp(lse2),
+                           ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert st == 0
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
 @pytest.mark.parametrize("B,S,W", [(1, 1024, 128), (2, 1000, 128), (1, 129, 7), (3, 260, 1), (1, 1, 128),
                                    (2, 384, 100)])
 def test_backward_both_kernel_paths(B, S, W, monkeypatch):
