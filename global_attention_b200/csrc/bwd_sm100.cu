@@ -28,53 +28,9 @@
 // columns of P^T relative to one scale per unit (a sum over query rows).  Scales are undone
 // in fp32.  Measured in a CPU emulation against the fp64 oracle this keeps every gradient
 // within the bf16 output rounding of the reference (single bf16 operands did not).
-#include <cudaTypedefs.h>
-
-#include "tc_rows.cuh"
+#include "bwd_tc.cuh"
 
 namespace zgcm {
-using namespace sm100;
-
-constexpr int TB_THREADS = 512;
-constexpr int TB_MAX_GRID = 1024;  // partial-sum slots reserved in the workspace
-
-struct BwdTcParams {
-    CUtensorMap tm_q;   // {D, Hq, S, B}, box {64, 1, 128, 1}, 128B swizzle
-    CUtensorMap tm_k;
-    CUtensorMap tm_v;
-    CUtensorMap tm_da;  // dA16, fp16, same geometry as tm_q
-    CUtensorMap tm_k16; // K~ fp16 (normalised, rotated, times the q~/k~ scale), geometry of tm_k
-    CUtensorMap tm_v16; // V fp16 times 2^e per 128-row tile, geometry of tm_v
-    CUtensorMap tm_q16; // Q~ fp16 (normalised, rotated, times the q~/k~ scale), geometry of tm_q
-    CUtensorMap tm_q16h;  // the same with 64-row boxes (key-major kernel, one 64-query half)
-    CUtensorMap tm_dah;   // dA16 with 64-row boxes
-    CUtensorMap tm_lse;   // lse2p, Delta, 2^-e of the dA rows: fp32 {Spad, Hq, B}, box {64, 1, 1}
-    CUtensorMap tm_delta;
-    CUtensorMap tm_dainv;
-    BwdParams P;
-    const __half* da16; // [B,S,Hq,D] dA * 2^e (e per row)
-    float* dainv;       // [B,Hq,Spad] 2^-e of each dA row (0 for an all-zero row and past S)
-    float* domax;       // [B,Hq,Spad] max |dout| of each row (bound on |dA|)
-    float* krinv;       // [B,Hkv,S] inverse RMS of each raw k row
-    float* qrinv;       // [B,Hq,S] inverse RMS of each raw q row
-    float* lse2p;       // [B,Hq,Spad] the forward's lse in base 2 (+inf past S), for TMA
-    float* vnorm;       // [B,Hkv,S] 2-norm of each raw v row
-    float* vtinv;       // [B,Hkv,ceil(S/128)] 2^-e of each V tile
-    int* err;
-    int total;          // steps (query-major) or units (key-major)
-};
-
-// Row stride of the backward's per-row arrays [B, Hq, Spad]: the sequence rounded up to 64,
-// so that a 64-row run starts on a 256-byte boundary and the arrays can be TMA tensors (a
-// global stride must be a multiple of 16 bytes).  Entries past S hold neutral values.
-__host__ __device__ __forceinline__ int row_stride(int S) { return (S + 63) & ~63; }
-
-// power-of-two exponent e with |x| * 2^e in [2^13, 2^14); 0 for x == 0 or non-finite
-__device__ __forceinline__ int fit_exp(float x) {
-    if (!(x > 0.f) || !isfinite(x)) return 0;
-    int e = 13 - ilogbf(x);
-    return max(-120, min(120, e));
-}
 
 // =====================================================================  gate backward pass
 
@@ -88,13 +44,17 @@ constexpr int GATE_UNROLL = 4;  // rows in flight per half-warp
 // per half-warp in flight; every loop bound is warp-uniform so the row-max shuffles see all
 // 32 lanes.  dainv = 2^-e (0 when the row of dout is all zero: its dA row is zero and must
 // not be rescaled), domax = max|dout|, both [B,Hq,Spad] (row_stride; the query-major kernel
-// fills the entries past S).
+// fills the entries past S).  With DELTA (wide windows) also Delta = sum_d dout*out
+// per row, [B,Hq,Spad]: the row sum of dA * A (A = out / sigmoid(g)), which the wide-window
+// query-major kernel needs before its first key tile.
+template <bool DELTA>
 __global__ void __launch_bounds__(GATE_THREADS, 2) bwd_gate_kernel(const bf16* __restrict__ dout,
                                                                 const bf16* __restrict__ g,
                                                                 const bf16* __restrict__ out,
                                                                 bf16* __restrict__ dg, __half* __restrict__ da16,
                                                                 float* __restrict__ dainv,
-                                                                float* __restrict__ domax, long long rows, int S,
+                                                                float* __restrict__ domax,
+                                                                float* __restrict__ delta, long long rows, int S,
                                                                 int Hq) {
     const int lane = threadIdx.x & 31, sub = lane & 15;
     const long long warp0 = ((long long)blockIdx.x * GATE_THREADS + threadIdx.x) >> 5;
@@ -130,12 +90,18 @@ __global__ void __launch_bounds__(GATE_THREADS, 2) bwd_gate_kernel(const bf16* _
             const int ea = fit_exp(mx);
             const float sc = ldexpf(1.0f, ea);
             uint32_t da[4], dgw[4];
+            float dsum = 0.f;  // sum_d dout out = sum_d dA A  (Delta of the wide-window backward)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 fd = unpack_bf16(wd[e]), fg = unpack_bf16(wg[e]), fo = unpack_bf16(wo[e]);
                 const float s0 = sigmoidf_(fg.x), s1 = sigmoidf_(fg.y);
                 da[e] = pack2<true>(fd.x * s0 * sc, fd.y * s1 * sc);
                 dgw[e] = pack_bf16(fd.x * fo.x * (1.f - s0), fd.y * fo.y * (1.f - s1));
+                if constexpr (DELTA) dsum = fmaf(fd.x, fo.x, fmaf(fd.y, fo.y, dsum));
+            }
+            if constexpr (DELTA) {
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
             }
             if (r < rows) {
                 const size_t o = (size_t)r * (kD / 8) + sub;
@@ -158,42 +124,11 @@ __global__ void __launch_bounds__(GATE_THREADS, 2) bwd_gate_kernel(const bf16* _
                     }
                     dainv[ro] = mx > 0.f ? 1.0f / sc : 0.f;
                     domax[ro] = mx;
+                    if constexpr (DELTA) delta[ro] = dsum;
                 }
             }
         }
     }
-}
-
-// 32 lanes x 16 consecutive 32-bit columns load
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
-
-// Sum of v[e] over the 32 lanes of the warp for e = 0..31, delivered as: lane L returns the
-// total of index L (recursive halving; 31 shuffles).  v is clobbered.
-__device__ __forceinline__ float warp_transpose_sum(float* v) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int k = 16; k >= 1; k >>= 1) {
-        const bool upper = (lane & k) != 0;
-#pragma unroll
-        for (int j = 0; j < k; ++j) {
-            const float send = upper ? v[j] : v[j + k];
-            const float keep = upper ? v[j + k] : v[j];
-            v[j] = keep + __shfl_xor_sync(0xffffffffu, send, k);
-        }
-    }
-    return v[0];
-}
-
-// swizzled 16-byte chunk ch (0..15, 8 values each) of row r in a two-half 128-row tile
-__device__ __forceinline__ uint4* tile_chunk(unsigned char* h0, unsigned char* h1, int r, int ch) {
-    unsigned char* hb = ch < 8 ? h0 : h1;
-    return reinterpret_cast<uint4*>(hb + (uint32_t)r * 128u + (uint32_t)(((ch & 7) ^ (r & 7)) << 4));
 }
 
 // Query-major pass over one 32-key chunk of a row (S, dP as accumulated in TMEM), with
@@ -251,63 +186,6 @@ __device__ __forceinline__ void kv_chunk(const float* sv, const float* dv, const
         pp[2 * e4 + 1] = pack2<true>(p4[2], p4[3]);
         dd[2 * e4] = pack2<true>(d4[0], d4[1]);
         dd[2 * e4 + 1] = pack2<true>(d4[2], d4[3]);
-    }
-}
-
-// RoPE / RMSNorm backward of one row held by one thread, one pass over the row:
-//   dy = R^T (f * dq~)       (dq~: the row's 128 accumulator columns, copied out of TMEM
-//                             into registers so that the tensor memory is released first;
-//                             R rotates pairs (t, t+21) at `pos`)
-//   dx = (dy * gamma - xhat * mdot) * rinv,   xhat = x * rinv,   d_gamma += dy * xhat
-// The caller supplies rinv = 1/sqrt(mean x^2 + eps) (from the prologue) and
-// mdot = mean_d(dy_d gamma_d xhat_d).  Because R is orthogonal and q~ = R(gamma * xhat),
-// mdot = (q~ . dq~) / D, which the softmax warps form as a row sum of dS * S; so the raw row
-// x (global memory) is read once: its first 64 values prefetched by the caller (xv0), the
-// last 64 here.  d_gamma goes into this warp's slice `dgam` through warp-transposed sums
-// (lane L owns one dimension per 32-wide block: a fixed summation order, reproducible).
-// `valid` masks rows past the sequence (they still join the collectives).
-__device__ __forceinline__ void row_rope_rms_backward_regs(float (&dy)[128], float f, float mdot, float rinv,
-                                                           const uint4 (&xv0)[8], const bf16* x, bf16* dst,
-                                                           bool valid, int pos, const float* gamma, float* dgam,
-                                                           const LayerParams& L) {
-    const int lane = threadIdx.x & 31;
-    const uint4* xr = reinterpret_cast<const uint4*>(x);
-    uint4* dr = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-    for (int e = 0; e < 128; ++e) dy[e] *= f;
-    // transpose of the rotation of pairs (t, t + 21)
-#pragma unroll
-    for (int t = 0; t < TF_HALF; ++t) {
-        float c, s;
-        rope_cs(L.theta[t], pos, c, s);
-        const float d1 = dy[t], d2 = dy[t + TF_HALF];
-        dy[t] = d1 * c + d2 * s;
-        dy[t + TF_HALF] = d2 * c - d1 * s;
-    }
-    uint4 xv1[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) xv1[c] = valid ? __ldg(xr + 8 + c) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {  // dims [32 q, 32 q + 32)
-        float* v = dy + 32 * q;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const uint4 u = q < 2 ? xv0[4 * q + c] : xv1[4 * (q - 2) + c];
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-            uint32_t o[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 t = unpack_bf16(w[e]);
-                const int d = 8 * c + 2 * e, gd = 32 * q + d;
-                const float x0 = t.x * rinv, x1 = t.y * rinv;
-                o[e] = pack_bf16((v[d] * gamma[gd] - x0 * mdot) * rinv, (v[d + 1] * gamma[gd + 1] - x1 * mdot) * rinv);
-                v[d] *= x0;
-                v[d + 1] *= x1;
-            }
-            if (valid) dr[4 * q + c] = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-        const float tot = warp_transpose_sum(v);
-        dgam[32 * q + lane] += tot;
     }
 }
 
@@ -868,14 +746,30 @@ struct BwdKTcSmem {
 struct UnitInfo {
     int b, kvh, kt, nit;   // nit = iterations: heads x query blocks that see the key tile
 };
-__device__ __forceinline__ UnitInfo decode_unit(const LayerParams& L, int u) {
+// Unit u: key tile kt of (b, KV head).  Sliding windows (W <= 128) sweep the units of a chain
+// in order (u = chain * tiles + kt), and query blocks kt and kt + 1 see the tile; wide windows
+// run one unit per CTA, heaviest (first tiles) first (u = kt * chains + chain), and the
+// query blocks that see tile kt run from kt to the block of the last query whose window
+// reaches the tile's last key, kt*128 + 127 + W - 1.
+__device__ __forceinline__ UnitInfo decode_unit(const LayerParams& L, int u, bool wide) {
     const int nkb = (L.S + TF_BN - 1) / TF_BN;
     UnitInfo x;
-    const int chain = u / nkb;
-    x.kt = u - chain * nkb;
+    int chain;
+    if (wide) {
+        const int chains = L.B * L.Hkv;
+        x.kt = u / chains;
+        chain = u - x.kt * chains;
+        // W <= S here (the launcher clamps it), so the sum stays in range
+        const int last_q = x.kt * TF_BN + TF_BN - 1 + L.W - 1;
+        const int qb_hi = min(nkb - 1, last_q / TF_BM);
+        x.nit = L.G * (qb_hi - x.kt + 1);
+    } else {
+        chain = u / nkb;
+        x.kt = u - chain * nkb;
+        x.nit = L.G * ((x.kt + 1 < nkb) ? 2 : 1);  // W <= 128: blocks kt and kt + 1
+    }
     x.b = chain / L.Hkv;
     x.kvh = chain - x.b * L.Hkv;
-    x.nit = L.G * ((x.kt + 1 < nkb) ? 2 : 1);
     return x;
 }
 // iteration it of a unit: query block kt + it / G, head it % G
@@ -884,6 +778,7 @@ __device__ __forceinline__ void decode_iter(const LayerParams& L, const UnitInfo
     hg = x.kvh * L.G + it % L.G;
 }
 
+template <bool WIDE>
 __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_constant__ BwdTcParams p) {
     const LayerParams& L = p.P.L;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -963,7 +858,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 };
                 bool ok = true;
                 for (int u = u_begin; u < u_end && ok && !*abort; ++u, ++uu) {
-                    const UnitInfo x = decode_unit(L, u);
+                    const UnitInfo x = decode_unit(L, u, WIDE);
                     for (int it = 0; it < x.nit && ok; ++it) {
                         int qb, hg;
                         decode_iter(L, x, it, qb, hg);
@@ -1014,7 +909,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 };
                 auto cur_first = [&]() {
                     Cursor c{u_begin, 0, 0, 0, 0, UnitInfo{}, u_begin < u_end};
-                    if (c.valid) c.x = decode_unit(L, c.u);
+                    if (c.valid) c.x = decode_unit(L, c.u, WIDE);
                     return c;
                 };
                 auto cur_next = [&](Cursor& c) {
@@ -1024,7 +919,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                     if (++c.it < c.x.nit) return;
                     c.it = 0;
                     ++c.uu;
-                    if (++c.u < u_end) c.x = decode_unit(L, c.u);
+                    if (++c.u < u_end) c.x = decode_unit(L, c.u, WIDE);
                     else c.valid = false;
                 };
                 auto last_of_unit = [](const Cursor& c) { return c.half == 1 && c.it == c.x.nit - 1; };
@@ -1103,7 +998,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
         int it_all = 0, uu = 0;
         bool ok = true;
         for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
-            const UnitInfo x = decode_unit(L, u);
+            const UnitInfo x = decode_unit(L, u, WIDE);
             const int j = x.kt * TF_BN + r;
             float vin = 0.f, su = 0.f, dsc = 0.f;
             float kacc = 0.f;  // sum over the unit of dS^T S^T (unscaled dS^T): dk's RMSNorm row term
@@ -1178,7 +1073,15 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             const float vnorm = j < L.S ? p.vnorm[((size_t)x.b * L.Hkv + x.kvh) * L.S + j] : 0.f;
             const float vtile = p.vtinv[((size_t)x.b * L.Hkv + x.kvh) * nkt + x.kt];
             float domx = 0.f, dlmx = 0.f;
-            for (int it0 = 0; it0 < x.nit; it0 += 8) {
+            if constexpr (WIDE) {
+                // per-tile maxima over the query blocks kt .. kt + nit/G - 1 (bwd_tile_stats_kernel)
+                const size_t nst = (size_t)L.B * L.Hkv * nkt, base = ((size_t)x.b * L.Hkv + x.kvh) * nkt;
+                for (int t = x.kt + r; t < x.kt + x.nit / L.G; t += TF_BN) {
+                    domx = fmaxf(domx, p.tstat[base + t]);
+                    dlmx = fmaxf(dlmx, p.tstat[nst + base + t]);
+                }
+            }
+            for (int it0 = 0; !WIDE && it0 < x.nit; it0 += 8) {
                 float dm[8], dl[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
@@ -1228,13 +1131,13 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             return true;
         };
         bool ok = true;
-        if (u_begin < u_end && (ok = unit_scales(decode_unit(L, u_begin), 0))) mbar_arrive(&sm.bar[KB_STATS]);
+        if (u_begin < u_end && (ok = unit_scales(decode_unit(L, u_begin, WIDE), 0))) mbar_arrive(&sm.bar[KB_STATS]);
         for (int u = u_begin; u < u_end && ok; ++u, ++uu) {
             if (u + 1 < u_end) {
-                if (!(ok = unit_scales(decode_unit(L, u + 1), (uu + 1) & 3))) break;
+                if (!(ok = unit_scales(decode_unit(L, u + 1, WIDE), (uu + 1) & 3))) break;
                 mbar_arrive(&sm.bar[KB_STATS + ((uu + 1) & 1)]);
             }
-            const UnitInfo x = decode_unit(L, u);
+            const UnitInfo x = decode_unit(L, u, WIDE);
             const int j = x.kt * TF_BN + r;
             const bool valid = j < L.S;
             const size_t off = ((size_t)(x.b * (size_t)L.S + (valid ? j : 0)) * L.Hkv + x.kvh) * kD;
@@ -1335,6 +1238,11 @@ extern const char* const kBwdTcKernelNames[] = {"bwd_gate_kernel",         "bwd_
                                                 "bwd_kv_tc_kernel",        "dgamma_reduce_kernel(k)",
                                                 "dgamma_reduce_kernel(q)"};
 extern const int kBwdTcKernelCount = 7;
+extern const char* const kBwdWideKernelNames[] = {"bwd_gate_kernel",       "bwd_prep_kv_kernel",
+                                                  "bwd_prep_q_kernel",     "bwd_tile_stats_kernel",
+                                                  "bwd_q_glob_kernel",     "bwd_kv_tc_kernel",
+                                                  "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"};
+extern const int kBwdWideKernelCount = 8;
 
 __global__ void dgamma_reduce_kernel(const float* __restrict__ parts, int n, float* __restrict__ out);
 
@@ -1342,10 +1250,25 @@ bool bwd_tc_supported(const LayerParams& L) {
     return L.W <= TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1 && get_encode_b() != nullptr;
 }
 
+// Windows wider than one tile (the global layer among them), 42 rotated dims.  A shape test
+// only: without the driver's tensor-map encoder the launch fails (ZGCM_ERR_CUDA).
+bool bwd_wide_supported(const LayerParams& L) {
+    return L.W > TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1;
+}
+
+namespace {
+// d_gamma partial-sum slots: the persistent sliding-window kernels use at most TB_MAX_GRID
+// CTAs, the wide-window ones one CTA per unit (at most B*Hq*ceil(S/128))
+size_t dgamma_slots(int B, int S, int Hq) {
+    const size_t units = (size_t)B * Hq * ((S + TF_BM - 1) / TF_BM);
+    return units > (size_t)TB_MAX_GRID ? units : (size_t)TB_MAX_GRID;
+}
+}  // namespace
+
 // workspace of the tcgen05 backward: delta, domax, dainv, lse2p [B,Hq,Spad] and qrinv
 // [B,Hq,S] fp32; dA16, Q~16
 // [B,S,Hq,D] fp16; K~16, V16 [B,S,Hkv,D] fp16; krinv, vnorm [B,Hkv,S] fp32; vtinv per V
-// tile; 2 x d_gamma partials
+// tile; per-tile maxima (wide windows); 2 x d_gamma partials
 size_t bwd_tc_workspace_bytes(int B, int S, int Hq, int Hkv) {
     const size_t rows = (size_t)B * S * Hq, krows = (size_t)B * S * Hkv;
     const size_t prows = (size_t)B * Hq * row_stride(S);  // padded row arrays
@@ -1353,14 +1276,17 @@ size_t bwd_tc_workspace_bytes(int B, int S, int Hq, int Hkv) {
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
     return 4 * a(prows * sizeof(float)) + a(rows * sizeof(float)) + 2 * a(rows * kD * sizeof(__half)) +
            2 * a(krows * kD * sizeof(__half)) + 2 * a(krows * sizeof(float)) + a(tiles * sizeof(float)) +
-           2 * a((size_t)TB_MAX_GRID * kD * sizeof(float));
+           a(3 * tiles * sizeof(float)) + 2 * a(dgamma_slots(B, S, Hq) * kD * sizeof(float));
 }
 
 cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, cudaStream_t stream,
                           void* const* events, int n_pairs) {
     BwdTcParams p;
     p.P = bp;
-    const LayerParams& L = bp.L;
+    // a window of S or more is the full causal one: clamped so that window arithmetic
+    // (j + W - 1) stays in range
+    if (p.P.L.W > p.P.L.S) p.P.L.W = p.P.L.S;
+    const LayerParams& L = p.P.L;
     const size_t rows = (size_t)L.B * L.S * L.Hq;
     auto a = [](size_t x) { return (x + 255) & ~size_t(255); };
     char* ws = static_cast<char*>(workspace);
@@ -1388,9 +1314,13 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     p.krinv = reinterpret_cast<float*>(take(krows * 4));
     p.vnorm = reinterpret_cast<float*>(take(krows * 4));
     p.vtinv = reinterpret_cast<float*>(take((size_t)L.B * L.Hkv * nkt * 4));
-    p.P.dgq_part = reinterpret_cast<float*>(take((size_t)TB_MAX_GRID * kD * 4));
-    p.P.dgk_part = reinterpret_cast<float*>(take((size_t)TB_MAX_GRID * kD * 4));
+    p.tstat = reinterpret_cast<float*>(take(3 * (size_t)L.B * L.Hkv * nkt * 4));
+    const size_t slots = dgamma_slots(L.B, L.S, L.Hq);
+    p.P.dgq_part = reinterpret_cast<float*>(take(slots * kD * 4));
+    p.P.dgk_part = reinterpret_cast<float*>(take(slots * kD * 4));
     p.err = err_word;
+    const bool wide = bp.L.W > TF_BN;  // as the kernel-name query decides: on the window given
+    p.wide = wide ? 1 : 0;
     if (!make_map_b(&p.tm_q, L.q, L.Hq, L.S, L.B) || !make_map_b(&p.tm_k, L.k, L.Hkv, L.S, L.B) ||
         !make_map_b(&p.tm_v, L.v, L.Hkv, L.S, L.B) ||
         !make_map_b(&p.tm_da, da16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
@@ -1410,7 +1340,11 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     const size_t smem_q = sizeof(BwdQTcSmem) + 1024, smem_k = sizeof(BwdKTcSmem) + 1024;
     if ((e = cudaFuncSetAttribute(bwd_q_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_q)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(bwd_kv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_k)) != cudaSuccess)
+    if ((e = cudaFuncSetAttribute(bwd_kv_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_k)) !=
+        cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(bwd_kv_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_k)) !=
+        cudaSuccess)
         return e;
     // events[2i] / events[2i+1] bracket kernel i (i < n_pairs)
     auto before = [&](int i) -> cudaError_t {
@@ -1441,8 +1375,12 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     if (q_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
     int i = 0;
     if ((e = before(i)) != cudaSuccess) return e;
-    bwd_gate_kernel<<<gate_grid, GATE_THREADS, 0, stream>>>(bp.dout, L.g, bp.out, bp.dg, da16, p.dainv, p.domax,
-                                                            (long long)rows, L.S, L.Hq);
+    if (wide)
+        bwd_gate_kernel<true><<<gate_grid, GATE_THREADS, 0, stream>>>(bp.dout, L.g, bp.out, bp.dg, da16, p.dainv,
+                                                                      p.domax, p.P.delta, (long long)rows, L.S, L.Hq);
+    else
+        bwd_gate_kernel<false><<<gate_grid, GATE_THREADS, 0, stream>>>(bp.dout, L.g, bp.out, bp.dg, da16, p.dainv,
+                                                                       p.domax, nullptr, (long long)rows, L.S, L.Hq);
     if ((e = after(i++)) != cudaSuccess) return e;
     if ((e = before(i)) != cudaSuccess) return e;
     bwd_prep_kv_kernel<<<(int)k_tiles, KP_THREADS, smem_pk, stream>>>(p);
@@ -1450,11 +1388,36 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     if ((e = before(i)) != cudaSuccess) return e;
     bwd_prep_q_kernel<<<(int)q_tiles, KP_THREADS, smem_pq, stream>>>(p);
     if ((e = after(i++)) != cudaSuccess) return e;
+    if (wide) {
+        // per-tile bounds, then the query-major sweep (one CTA per (b, head, block), heaviest
+        // first) and the key-major one (one CTA per (b, KV head, tile), heaviest first)
+        const long long units_q = (long long)L.B * L.Hq * nqb;
+        const size_t smem_g = bwd_q_glob_smem_bytes();
+        if ((e = cudaFuncSetAttribute(bwd_q_glob_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_g)) !=
+            cudaSuccess)
+            return e;
+        if ((e = before(i)) != cudaSuccess) return e;
+        bwd_tile_stats_kernel<<<(int)k_tiles, BTS_THREADS, 0, stream>>>(p);
+        if ((e = after(i++)) != cudaSuccess) return e;
+        if ((e = before(i)) != cudaSuccess) return e;
+        bwd_q_glob_kernel<<<(int)units_q, BQG_THREADS, smem_g, stream>>>(p);
+        if ((e = after(i++)) != cudaSuccess) return e;
+        p.total = (int)k_tiles;
+        if ((e = before(i)) != cudaSuccess) return e;
+        bwd_kv_tc_kernel<true><<<(int)k_tiles, TB_THREADS, smem_k, stream>>>(p);
+        if ((e = after(i++)) != cudaSuccess) return e;
+        if ((e = before(i)) != cudaSuccess) return e;
+        dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgk_part, (int)k_tiles, bp.dgamma_k);
+        if ((e = after(i++)) != cudaSuccess) return e;
+        if ((e = before(i)) != cudaSuccess) return e;
+        dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgq_part, (int)units_q, bp.dgamma_q);
+        return after(i);
+    }
     if ((e = before(i)) != cudaSuccess) return e;
     bwd_q_tc_kernel<<<grid, TB_THREADS, smem_q, stream>>>(p);
     if ((e = after(i++)) != cudaSuccess) return e;
     if ((e = before(i)) != cudaSuccess) return e;
-    bwd_kv_tc_kernel<<<grid, TB_THREADS, smem_k, stream>>>(p);
+    bwd_kv_tc_kernel<false><<<grid, TB_THREADS, smem_k, stream>>>(p);
     if ((e = after(i++)) != cudaSuccess) return e;
     if ((e = before(i)) != cudaSuccess) return e;
     dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgk_part, grid, bp.dgamma_k);

@@ -465,9 +465,11 @@ bool fwd_glob_supported(const LayerParams& L) {
 size_t fwd_glob_workspace_bytes(int B, int S, int Hkv) { return (size_t)B * S * Hkv * kD * 2; }
 
 cudaError_t launch_fwd_glob_tc(const FwdParams& fp, void* workspace, int* err_word, cudaStream_t stream) {
-    const LayerParams& L = fp.L;
     FwdGlobParams p;
-    p.L = L;
+    p.L = fp.L;
+    // a window of S or more is the full causal one: clamped so that window arithmetic stays in range
+    if (p.L.W > p.L.S) p.L.W = p.L.S;
+    const LayerParams& L = p.L;
     p.out = fp.out;
     p.lse = fp.lse;
     p.err = err_word;

@@ -21,6 +21,9 @@ extern const int kBwdMmaKernelCount;
 cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, cudaStream_t stream,
                           void* const* events, int n_pairs);
 bool bwd_tc_supported(const LayerParams& L);
+bool bwd_wide_supported(const LayerParams& L);
+extern const char* const kBwdWideKernelNames[];
+extern const int kBwdWideKernelCount;
 size_t bwd_tc_workspace_bytes(int B, int S, int Hq, int Hkv);
 extern const char* const kBwdTcKernelNames[];
 extern const int kBwdTcKernelCount;
@@ -282,7 +285,7 @@ int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void*
     p.n_q_parts = (int)w.n_q_parts;
     if (n_pairs < 0 || (n_pairs > 0 && !events)) return ZGCM_ERR_INVALID_ARG;
     cudaError_t e;
-    if (!force_mma() && bwd_tc_supported(p.L))
+    if (!force_mma() && (bwd_tc_supported(p.L) || bwd_wide_supported(p.L)))
         e = launch_bwd_tc(p, workspace, device_error_word(), stream, events, n_pairs);
     else
         e = launch_bwd_mma(p, stream, events, n_pairs);
@@ -292,9 +295,15 @@ int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void*
 const char* zgcm_attn_bwd_kernel_name(int i, int S, int rope_dims, int window) {
     LayerParams L{};
     L.B = 1; L.S = S; L.rope_half = rope_dims / 2; L.W = window;
-    const bool tc = !force_mma() && S >= 1 && bwd_tc_supported(L);
-    const char* const* names = tc ? kBwdTcKernelNames : kBwdMmaKernelNames;
-    const int n = tc ? kBwdTcKernelCount : kBwdMmaKernelCount;
+    const char* const* names = kBwdMmaKernelNames;
+    int n = kBwdMmaKernelCount;
+    if (!force_mma() && S >= 1 && bwd_tc_supported(L)) {
+        names = kBwdTcKernelNames;
+        n = kBwdTcKernelCount;
+    } else if (!force_mma() && S >= 1 && bwd_wide_supported(L)) {
+        names = kBwdWideKernelNames;
+        n = kBwdWideKernelCount;
+    }
     return (i >= 0 && i < n) ? names[i] : nullptr;
 }
 

@@ -148,6 +148,28 @@ def test_backward_both_kernel_paths(B, S, W, monkeypatch):
         assert_dgamma_close(f"dgamma_k[{name}]", gr["dgamma_k"], ref["dgamma_k"])
 
 
+@pytest.mark.parametrize("B,S,W", [(1, 777, 777), (2, 1000, 10**6), (1, 129, 129), (1, 1, 4096),
+                                   (3, 260, 200), (1, 1300, 300), (2, 640, 129), (1, 2048, 2048)])
+def test_backward_wide_window_kernels(B, S, W, monkeypatch):
+    """Windows wider than one key tile (the global layer among them) run the tcgen05
+    wide-window backward (tile bounds, query-major dq sweep, key-major dk/dv sweep); every
+    gradient matches the oracle."""
+    t = make_inputs(B, S, seed=400 + S + W % 1000, with_dout=True)
+    d = _to_dev(t)
+    ref = _problem(t, window=W).backward(t["dout"])
+    monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
+    assert ga.zgcm_attn_bwd_kernel_names(S, W) == [
+        "bwd_gate_kernel", "bwd_prep_kv_kernel", "bwd_prep_q_kernel", "bwd_tile_stats_kernel",
+        "bwd_q_glob_kernel", "bwd_kv_tc_kernel", "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"]
+    out, lse = _gpu_fwd(d, window=W)
+    gr = _gpu_bwd(d, out, lse, window=W)
+    assert ga.zgcm_attn_device_error() == 0
+    for n in ("dq", "dk", "dv", "dg"):
+        assert_bf16_close(n, gr[n], ref[n])
+    assert_dgamma_close("dgamma_q", gr["dgamma_q"], ref["dgamma_q"])
+    assert_dgamma_close("dgamma_k", gr["dgamma_k"], ref["dgamma_k"])
+
+
 def test_empty_problem():
     for B, S in ((0, 16), (2, 0)):
         t = make_inputs(max(B, 1), max(S, 1), with_dout=True)
