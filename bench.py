@@ -40,6 +40,7 @@ WORKLOADS = {
     "tiny_fwd": (1, 1024, 128, False),
     "swa16k_b1_fwd": (1, 16384, 128, False),
     "swa16k_b1": (1, 16384, 128, True),
+    "global8k": (1, 8192, 8192, True),      # small global case (profiling captures)
     # one sliding (W=128) and one global (W=S) layer on the same inputs, reported with the
     # 5:1 sliding:global weighted time per layer of the model's layer pattern
     "mix256k_fwd": (1, 262144, 128, False),

@@ -203,10 +203,12 @@ const char* zgcm_attn_fwd_kernel_name(int B, int S, int Hq, int Hkv, int rope_di
 int zgcm_attn_device_error(void);
 
 /* Name of the i-th kernel zgcm_attn_bwd launches for this configuration (static string),
- * or NULL when i is past the last one.  Windows up to 128 with 42 rotated dims run the
+ * or NULL when i is past the last one.  With 42 rotated dims, windows up to 128 run the
  * gate pass, the K/V and Q preparation and the tcgen05 pair (bwd_gate_kernel,
  * bwd_prep_kv_kernel, bwd_prep_q_kernel, bwd_q_tc_kernel, bwd_kv_tc_kernel, then the two
- * d_gamma reductions); other shapes, or ZGCM_FORCE_MMA=1, the warp-MMA kernels. */
+ * d_gamma reductions); wider windows (the global layer among them) the same gate pass and
+ * preparation, then bwd_tile_stats_kernel, bwd_q_glob_kernel, bwd_kv_tc_kernel and the two
+ * reductions; other shapes, or ZGCM_FORCE_MMA=1, the warp-MMA kernels. */
 const char* zgcm_attn_bwd_kernel_name(int i, int S, int rope_dims, int window);
 
 #ifdef __cplusplus
