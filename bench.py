@@ -104,7 +104,7 @@ def work(B, S, W, bwd):
     kernels = {
         "fwd_mma_kernel": (fwd_bytes, fwd_flops),
         "fwd_tc_kernel": (fwd_bytes, fwd_flops),
-        # wide-window / global forward: q, K~16 (fp16), v, g -> out, lse (K~ prepared from k first)
+        # tcgen05 forwards: q, K~16 (fp16, prepared from k by fwd_prep_k_kernel), v, g -> out, lse
         "fwd_glob_tc_kernel": (fwd_bytes, fwd_flops),
         # dout, out, g -> dg, dA
         "bwd_pre_kernel": (5 * qb, 0),
@@ -467,9 +467,9 @@ def main():
                "sample": "; ".join(parts) + "; same heads as the workload, time per visible (query, key) "
                          "pair scaled to the workload's pairs per token"}
 
-    # per layer: the forward's kernels (the wide-window forward runs a key preparation kernel
+    # per layer: the forward's kernels (each tcgen05 forward runs the key preparation kernel
     # first) + every backward kernel
-    fwd_launches = [2 if ga.zgcm_attn_fwd_kernel_name(Bw, Sw, HQ, HKV, 42, lw) == "fwd_glob_tc_kernel" else 1
+    fwd_launches = [1 if ga.zgcm_attn_fwd_kernel_name(Bw, Sw, HQ, HKV, 42, lw) == "fwd_mma_kernel" else 2
                     for lw, _ in layers]
     launches_per_step = sum(f + len(n) for f, n in zip(fwd_launches, bwd_names))
     rec = {

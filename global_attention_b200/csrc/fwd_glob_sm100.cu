@@ -461,7 +461,7 @@ bool fwd_glob_supported(const LayerParams& L) {
     return L.W > TF_BN && L.rope_half == TF_HALF && L.G % 2 == 0 && L.S >= 1 && L.B >= 1;
 }
 
-// K~ fp16 [B, S, Hkv, D]
+// K~ fp16 [B, S, Hkv, D] (both tcgen05 forwards)
 size_t fwd_glob_workspace_bytes(int B, int S, int Hkv) { return (size_t)B * S * Hkv * kD * 2; }
 
 cudaError_t launch_fwd_glob_tc(const FwdParams& fp, void* workspace, int* err_word, cudaStream_t stream) {
@@ -491,6 +491,26 @@ cudaError_t launch_fwd_glob_tc(const FwdParams& fp, void* workspace, int* err_wo
     fwd_prep_k_kernel<<<(int)k_tiles, FP_THREADS, smem_p, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     fwd_glob_tc_kernel<<<(int)units, FG_THREADS, smem_a, stream>>>(p);
+    return cudaGetLastError();
+}
+
+// K~ fp16 of every key tile into `workspace` ([B,S,Hkv,D]) for the sliding-window forward.
+cudaError_t launch_fwd_prep_k(const LayerParams& L, void* workspace, int* err_word, cudaStream_t stream) {
+    FwdGlobParams p;
+    p.L = L;
+    p.out = nullptr;
+    p.lse = nullptr;
+    p.err = err_word;
+    p.units = 0;
+    const long long k_tiles = (long long)L.B * L.Hkv * ((L.S + TF_BN - 1) / TF_BN);
+    if (k_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+    if (!make_map_g(&p.tm_k, L.k, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) ||
+        !make_map_g(&p.tm_k16, workspace, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        return cudaErrorInvalidValue;
+    const size_t smem_p = sizeof(FwdPrepSmem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(fwd_prep_k_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p);
+    if (e != cudaSuccess) return e;
+    fwd_prep_k_kernel<<<(int)k_tiles, FP_THREADS, smem_p, stream>>>(p);
     return cudaGetLastError();
 }
 

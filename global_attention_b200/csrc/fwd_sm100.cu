@@ -9,9 +9,10 @@
 // query heads of the group.  With W <= 128 the window of block qb lies inside key tiles
 // qb-1 and qb, so consecutive steps of one (b, KV head) chain share a tile: a persistent
 // CTA sweeps a contiguous range of steps and loads ONE new K/V tile per step into a 2-slot
-// ring.  K~ and Q~ are normalised/rotated in place in shared memory (TMA-loaded raw,
-// 128-byte swizzle = the UMMA K-major canonical layout) and stored as fp16 times a power of
-// two (qk_fp16_scale) that keeps them in range.
+// ring.  K~ (fp16, normalised and rotated once per tile by fwd_prep_k_kernel into the
+// workspace) arrives by TMA ready to use; Q~ is normalised/rotated in place in shared memory
+// (TMA-loaded raw, 128-byte swizzle = the UMMA K-major canonical layout).  Both are fp16
+// times a power of two (qk_fp16_scale) that keeps them in range.
 //
 // Per head m (TMEM: S/P columns [0,256), O double buffer [256,384) and [384,512)):
 //   S   = Q~ [K~_slot0; K~_slot1]^T          tcgen05.mma M=128 N=256 K=128, A,B in smem
@@ -24,7 +25,7 @@
 //   out = sigmoid(g) * O / l                 epilogue, 16-byte global loads/stores
 //
 // Warp roles (512 threads): w0 TMA K/V, w1 MMA issue + TMEM owner, w2 TMA Q, w3 idle,
-// w4-7 softmax, w8-11 prologue (K~, Q~ in place), w12-15 gate epilogue.  Every wait is bounded;
+// w4-7 softmax, w8-11 prologue (Q~ in place), w12-15 gate epilogue.  Every wait is bounded;
 // on expiry the CTA records the site, drains, frees TMEM and returns.
 #include <cudaTypedefs.h>
 
@@ -38,7 +39,7 @@ constexpr int TF_THREADS = 512;
 
 struct FwdTcParams {
     CUtensorMap tm_q;   // {D, Hq, S, B}, box {64, 1, 128, 1}, 128B swizzle
-    CUtensorMap tm_k;   // {D, Hkv, S, B}
+    CUtensorMap tm_k16; // K~ fp16 {D, Hkv, S, B} (fwd_prep_k_kernel, in the workspace)
     CUtensorMap tm_v;
     LayerParams L;
     bf16* out;
@@ -48,11 +49,11 @@ struct FwdTcParams {
 };
 
 enum Bar {
-    B_KFULL = 0, B_KREADY = 2, B_KEMPTY = 4, B_VFULL = 6, B_VEMPTY = 8,
-    B_QFULL = 10, B_QREADY = 12, B_QEMPTY = 14,
-    B_SFULL = 16, B_PFULL = 17,
-    B_OFULL = 18, B_OEMPTY = 20, B_LFULL = 22, B_LEMPTY = 24,
-    B_DONE = 26, B_COUNT = 27
+    B_KFULL = 0, B_KEMPTY = 2, B_VFULL = 4, B_VEMPTY = 6,
+    B_QFULL = 8, B_QREADY = 10, B_QEMPTY = 12,
+    B_SFULL = 14, B_PFULL = 15,
+    B_OFULL = 16, B_OEMPTY = 18, B_LFULL = 20, B_LEMPTY = 22,
+    B_DONE = 24, B_COUNT = 25
 };
 
 struct FwdTcSmem {
@@ -86,7 +87,6 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
         sm.abort = 0;
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.bar[B_KFULL + i], 1);
-            mbar_init(&sm.bar[B_KREADY + i], 128);
             mbar_init(&sm.bar[B_KEMPTY + i], 1);
             mbar_init(&sm.bar[B_VFULL + i], 1);
             mbar_init(&sm.bar[B_VEMPTY + i], 1);
@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&p.tm_q);
-        prefetch_tmap(&p.tm_k);
+        prefetch_tmap(&p.tm_k16);
         prefetch_tmap(&p.tm_v);
     }
     tc_fence_before();
@@ -133,8 +133,8 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
                 const int slot = n & 1;
                 if (n >= 2 && !mbar_wait(&sm.bar[B_KEMPTY + slot], ((n >> 1) - 1) & 1, abort, 1)) return false;
                 mbar_expect_tx(&sm.bar[B_KFULL + slot], TF_TILE_BYTES);
-                tma_load_4d(sm.K[0] + slot * TF_HALF_BYTES, &p.tm_k, &sm.bar[B_KFULL + slot], 0, kvh, kt * TF_BN, b);
-                tma_load_4d(sm.K[1] + slot * TF_HALF_BYTES, &p.tm_k, &sm.bar[B_KFULL + slot], 64, kvh, kt * TF_BN, b);
+                tma_load_4d(sm.K[0] + slot * TF_HALF_BYTES, &p.tm_k16, &sm.bar[B_KFULL + slot], 0, kvh, kt * TF_BN, b);
+                tma_load_4d(sm.K[1] + slot * TF_HALF_BYTES, &p.tm_k16, &sm.bar[B_KFULL + slot], 64, kvh, kt * TF_BN, b);
                 last_k[slot] = n;
                 if (n >= 2 && !mbar_wait(&sm.bar[B_VEMPTY + slot], ((n >> 1) - 1) & 1, abort, 2)) return false;
                 mbar_expect_tx(&sm.bar[B_VFULL + slot], TF_TILE_BYTES);
@@ -189,13 +189,13 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
                 if (st.fresh) {
                     n_prev = n_next++;
                     n_cur = n_next++;
-                    ok = mbar_wait(&sm.bar[B_KREADY + (n_prev & 1)], (n_prev >> 1) & 1, abort, 10) &&
+                    ok = mbar_wait(&sm.bar[B_KFULL + (n_prev & 1)], (n_prev >> 1) & 1, abort, 10) &&
                          mbar_wait(&sm.bar[B_VFULL + (n_prev & 1)], (n_prev >> 1) & 1, abort, 11);
                 } else {
                     n_prev = n_cur;
                     n_cur = n_next++;
                 }
-                ok = ok && mbar_wait(&sm.bar[B_KREADY + (n_cur & 1)], (n_cur >> 1) & 1, abort, 12) &&
+                ok = ok && mbar_wait(&sm.bar[B_KFULL + (n_cur & 1)], (n_cur >> 1) & 1, abort, 12) &&
                      mbar_wait(&sm.bar[B_VFULL + (n_cur & 1)], (n_cur >> 1) & 1, abort, 13);
                 for (int h = 0; h < G && ok; ++h, ++m) {
                     const int buf = m & 1;
@@ -313,27 +313,14 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
             if (stop) break;
         }
     } else if (warp >= 8 && warp < 12) {
-        // ================================================ prologue: K~, Q~ normalised + rotated in place
+        // ================================================ prologue: Q~ normalised + rotated in place
+        // (K~ arrives converted from the preparation kernel)
         const int r = tid - 256;
-        int n_next = 0, m = 0;
+        int m = 0;
         bool ok = true;
-        auto prologue_k = [&](int n, int pos0) -> bool {
-            const int slot = n & 1;
-            if (!mbar_wait(&sm.bar[B_KFULL + slot], (n >> 1) & 1, abort, 32)) return false;
-            tf_angles(L, pos0 + r, sm.cs, r);
-            tf_prologue_row<true>(sm.K[0] + slot * TF_HALF_BYTES, sm.K[1] + slot * TF_HALF_BYTES, r, sm.gk, L, sm.cs,
-                                  oscale);
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.bar[B_KREADY + slot]);
-            return true;
-        };
         for (int t = t_begin; t < t_end && ok; ++t) {
             const StepInfo st = decode_step(L, t, t_begin, t_end);
-            const int q0 = st.qb * TF_BM;
-            if (st.fresh) ok = prologue_k(n_next++, q0 - TF_BN);
-            ok = ok && prologue_k(n_next++, q0);
-            if (!ok) break;
-            // the current K tile was rotated at q0 + r: the table already holds these angles
+            tf_angles(L, st.qb * TF_BM + r, sm.cs, r);  // this row's angles, shared by the G heads
             for (int h = 0; h < G; ++h, ++m) {
                 const int buf = m & 1;
                 if (!(ok = mbar_wait(&sm.bar[B_QFULL + buf], (m >> 1) & 1, abort, 33))) break;
@@ -424,15 +411,16 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-// 4-D bf16 map {D, H, S, B} (innermost first), box {64, 1, 128, 1}, 128-byte swizzle
-bool make_map(CUtensorMap* map, const void* base, int H, int S, int B) {
+// 4-D 16-bit map {D, H, S, B} (innermost first), box {64, 1, 128, 1}, 128-byte swizzle
+bool make_map(CUtensorMap* map, const void* base, int H, int S, int B,
+              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     auto enc = get_encode();
     if (!enc) return false;
     cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)S * H * kD * 2};
     cuuint32_t box[4] = {64, 1, 128, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = enc(map, dtype, 4, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -440,13 +428,18 @@ bool make_map(CUtensorMap* map, const void* base, int H, int S, int B) {
 
 }  // namespace
 
+// Windows up to one key tile with 42 rotated dims.  A shape test only: without the driver's
+// tensor-map encoder the launch fails (ZGCM_ERR_CUDA).
 bool fwd_tc_supported(const LayerParams& L) {
-    return L.W <= TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1 && get_encode() != nullptr;
+    return L.W <= TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1;
 }
 
 size_t fwd_tc_smem_bytes() { return sizeof(FwdTcSmem) + 1024; }
 
-cudaError_t launch_fwd_tc(const FwdParams& fp, int* err_word, cudaStream_t stream) {
+cudaError_t launch_fwd_prep_k(const LayerParams& L, void* workspace, int* err_word, cudaStream_t stream);
+
+// fwd_prep_k_kernel (K~ into `workspace`, [B,S,Hkv,D] fp16), then the attention kernel
+cudaError_t launch_fwd_tc(const FwdParams& fp, void* workspace, int* err_word, cudaStream_t stream) {
     FwdTcParams p;
     p.L = fp.L;
     p.out = fp.out;
@@ -456,11 +449,14 @@ cudaError_t launch_fwd_tc(const FwdParams& fp, int* err_word, cudaStream_t strea
     const long long total = (long long)fp.L.B * fp.L.Hkv * nqb;
     if (total > 0x7fffffffLL) return cudaErrorInvalidValue;
     p.total_steps = (int)total;
-    if (!make_map(&p.tm_q, fp.L.q, fp.L.Hq, fp.L.S, fp.L.B) || !make_map(&p.tm_k, fp.L.k, fp.L.Hkv, fp.L.S, fp.L.B) ||
+    if (!make_map(&p.tm_q, fp.L.q, fp.L.Hq, fp.L.S, fp.L.B) ||
+        !make_map(&p.tm_k16, workspace, fp.L.Hkv, fp.L.S, fp.L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
         !make_map(&p.tm_v, fp.L.v, fp.L.Hkv, fp.L.S, fp.L.B))
         return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    cudaError_t e = launch_fwd_prep_k(fp.L, workspace, err_word, stream);
+    if (e != cudaSuccess) return e;
+    e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     const size_t smem = fwd_tc_smem_bytes();

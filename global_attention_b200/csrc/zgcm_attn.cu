@@ -10,7 +10,7 @@
 
 namespace zgcm {
 cudaError_t launch_fwd_mma(const FwdParams& p, cudaStream_t stream);
-cudaError_t launch_fwd_tc(const FwdParams& p, int* err_word, cudaStream_t stream);
+cudaError_t launch_fwd_tc(const FwdParams& p, void* workspace, int* err_word, cudaStream_t stream);
 bool fwd_tc_supported(const LayerParams& L);
 cudaError_t launch_fwd_glob_tc(const FwdParams& p, void* workspace, int* err_word, cudaStream_t stream);
 bool fwd_glob_supported(const LayerParams& L);
@@ -153,24 +153,41 @@ const char* zgcm_status_string(int status) {
 size_t zgcm_attn_fwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int rope_dims, int window) {
     if (check_shape(B, S, Hq, Hkv, D, rope_dims, 1.0, window, 1, 0.f, 1.f) != ZGCM_OK) return 0;
     if ((long long)B * S == 0) return 0;
-    return fwd_path(shape_only(B, S, Hq, Hkv, rope_dims, window)) == FwdPath::GLOB
+    // both tcgen05 forwards read K~ (fp16, normalised and rotated once per key tile) from it
+    return fwd_path(shape_only(B, S, Hq, Hkv, rope_dims, window)) != FwdPath::MMA
                ? align256(fwd_glob_workspace_bytes(B, S, Hkv))
                : 0;
 }
+
+}  // extern "C"
+
+namespace {
+// Checks of the forward's arguments other than the workspace (ZGCM_OK or the first failure).
+int fwd_check(const void* q, const void* k, const void* v, const void* g, const float* gamma_q,
+              const float* gamma_k, int B, int S, int Hq, int Hkv, int D, int rope_dims, double rope_base,
+              int window, int causal, float eps, float scale, const void* out, const float* lse) {
+    int st = check_shape(B, S, Hq, Hkv, D, rope_dims, rope_base, window, causal, eps, scale);
+    if (st != ZGCM_OK || (long long)B * S == 0) return st;
+    const void* ptrs[] = {q, k, v, g, gamma_q, gamma_k, out, lse};
+    for (const void* p : ptrs)
+        if (!p) return ZGCM_ERR_INVALID_ARG;
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return ZGCM_ERR_ALIGNMENT;
+    return ZGCM_OK;
+}
+}  // namespace
+
+extern "C" {
 
 int zgcm_attn_fwd_ws(const void* q, const void* k, const void* v, const void* g,
                      const float* gamma_q, const float* gamma_k,
                      int B, int S, int Hq, int Hkv, int D, int rope_dims,
                      double rope_base, int window, int causal, float eps, float scale,
                      void* out, float* lse, void* workspace, size_t workspace_bytes, void* cuda_stream) {
-    int st = check_shape(B, S, Hq, Hkv, D, rope_dims, rope_base, window, causal, eps, scale);
+    int st = fwd_check(q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, D, rope_dims, rope_base, window, causal,
+                       eps, scale, out, lse);
     if (st != ZGCM_OK) return st;
     if ((long long)B * S == 0) return ZGCM_OK;
-    const void* ptrs[] = {q, k, v, g, gamma_q, gamma_k, out, lse};
-    for (const void* p : ptrs)
-        if (!p) return ZGCM_ERR_INVALID_ARG;
-    for (const void* p : ptrs)
-        if (!aligned16(p)) return ZGCM_ERR_ALIGNMENT;
     const size_t need = zgcm_attn_fwd_workspace_size(B, S, Hq, Hkv, D, rope_dims, window);
     if (need > 0) {
         if (!workspace || workspace_bytes < need) return ZGCM_ERR_WORKSPACE;
@@ -183,7 +200,7 @@ int zgcm_attn_fwd_ws(const void* q, const void* k, const void* v, const void* g,
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     cudaError_t e;
     switch (fwd_path(p.L)) {
-        case FwdPath::TC: e = launch_fwd_tc(p, device_error_word(), stream); break;
+        case FwdPath::TC: e = launch_fwd_tc(p, workspace, device_error_word(), stream); break;
         case FwdPath::GLOB: e = launch_fwd_glob_tc(p, workspace, device_error_word(), stream); break;
         default: e = launch_fwd_mma(p, stream); break;
     }
@@ -195,6 +212,9 @@ int zgcm_attn_fwd(const void* q, const void* k, const void* v, const void* g,
                   int B, int S, int Hq, int Hkv, int D, int rope_dims,
                   double rope_base, int window, int causal, float eps, float scale,
                   void* out, float* lse, void* cuda_stream) {
+    const int st0 = fwd_check(q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, D, rope_dims, rope_base, window,
+                              causal, eps, scale, out, lse);
+    if (st0 != ZGCM_OK) return st0;
     const size_t need = zgcm_attn_fwd_workspace_size(B, S, Hq, Hkv, D, rope_dims, window);
     if (need == 0)
         return zgcm_attn_fwd_ws(q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, D, rope_dims, rope_base, window,

@@ -28,9 +28,9 @@
  *     [B, S, Hkv, D]; lse is fp32 [B, Hq, S]; gamma_q, gamma_k, dgamma_q, dgamma_k are
  *     fp32 [D].  Every pointer must be 16-byte aligned (ZGCM_ERR_ALIGNMENT otherwise).
  *   - Ownership: the caller owns every buffer.  The library keeps no state between calls
- *     and allocates no device memory, with one exception: zgcm_attn_fwd on a window wider
- *     than 128 takes its scratch from the device's stream-ordered pool (see there);
- *     zgcm_attn_fwd_ws is the same call with caller-owned scratch.
+ *     and allocates no device memory, with one exception: zgcm_attn_fwd takes its key
+ *     scratch from the device's stream-ordered pool (see there); zgcm_attn_fwd_ws is the
+ *     same call with caller-owned scratch.
  *   - Streams: every call is asynchronous on `cuda_stream` (a cudaStream_t, NULL = legacy
  *     default stream) and never synchronises the device.
  *   - Errors: arguments are checked on the host before anything is launched; a failed
@@ -80,10 +80,10 @@ const char* zgcm_status_string(int status);
  * In : q, g bf16 [B,S,Hq,D]; k, v bf16 [B,S,Hkv,D]; gamma_q, gamma_k fp32 [D].
  * Out: out bf16 [B,S,Hq,D] (rounded once, to nearest even); lse fp32 [B,Hq,S].
  * out/lse must not alias any input.
- * Windows wider than 128 (the global layer, window >= S, among them) need device scratch
- * for the normalised keys (zgcm_attn_fwd_workspace_size bytes): this call takes it with
- * cudaMallocAsync on `cuda_stream` and returns it with cudaFreeAsync after the kernels,
- * so it never synchronises; callers that manage memory themselves use zgcm_attn_fwd_ws.
+ * The tcgen05 kernels need device scratch for the normalised keys
+ * (zgcm_attn_fwd_workspace_size bytes): this call takes it with cudaMallocAsync on
+ * `cuda_stream` and returns it with cudaFreeAsync after the kernels, so it never
+ * synchronises; callers that manage memory themselves use zgcm_attn_fwd_ws.
  */
 int zgcm_attn_fwd(const void* q, const void* k, const void* v, const void* g,
                   const float* gamma_q, const float* gamma_k,
@@ -92,10 +92,11 @@ int zgcm_attn_fwd(const void* q, const void* k, const void* v, const void* g,
                   void* out, float* lse, void* cuda_stream);
 
 /*
- * Bytes of device scratch the forward needs for this configuration: 0 for windows up to
- * 128 (the sliding layers), B*S*Hkv*D*2 rounded up to 256 for wider windows with 42
- * rotated dims and an even Hq/Hkv (the fp16 normalised, rotated keys, written by the
- * forward's preparation kernel and read by its attention kernel).  0 for invalid arguments.
+ * Bytes of device scratch the forward needs for this configuration: B*S*Hkv*D*2 rounded up
+ * to 256 wherever a tcgen05 forward runs (42 rotated dims; any window up to 128, or wider
+ * windows with an even Hq/Hkv): the fp16 normalised, rotated keys, written once per key
+ * tile by the forward's preparation kernel (fwd_prep_k_kernel) and read by its attention
+ * kernel.  0 for the warp-MMA kernel and for invalid arguments.
  */
 size_t zgcm_attn_fwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int rope_dims, int window);
 
@@ -188,7 +189,7 @@ int zgcm_attn_bwd_noalloc(const void* q, const void* k, const void* v, const voi
  * Main kernel zgcm_attn_fwd launches for this configuration (static string):
  * "fwd_tc_kernel" (tcgen05/TMEM/TMA, sliding windows up to 128 with 42 rotated dims),
  * "fwd_glob_tc_kernel" (tcgen05, wider windows and the global layer, with 42 rotated dims
- * and an even Hq/Hkv; preceded by the key preparation kernel fwd_prep_k_kernel) or
+ * and an even Hq/Hkv), each preceded by the key preparation kernel fwd_prep_k_kernel, or
  * "fwd_mma_kernel" (warp MMA, every other shape).  Setting the environment variable
  * ZGCM_FORCE_MMA=1 selects the warp-MMA kernels.
  */

@@ -122,11 +122,10 @@ def _fwd_ws(lib, ws, ws_bytes, **kw):
 
 def test_fwd_workspace_size_query(lib):
     ws = lambda *a: lib.zgcm_attn_fwd_workspace_size(*a)
-    # sliding windows up to one key tile need none
-    assert ws(4, 16384, 32, 8, 128, 42, 128) == 0
-    assert ws(1, 1024, 32, 8, 128, 42, 7) == 0
-    # wider windows and the global layer: the fp16 normalised keys, [B, S, Hkv, D]
-    for B, S, W in ((1, 65536, 65536), (2, 1000, 300), (1, 1, 10**6), (3, 777, 129)):
+    # both tcgen05 forwards (sliding windows and wider ones, the global layer among them) read
+    # the fp16 normalised keys, [B, S, Hkv, D]
+    for B, S, W in ((4, 16384, 128), (1, 1024, 7), (1, 65536, 65536), (2, 1000, 300), (1, 1, 10**6),
+                    (3, 777, 129)):
         n = B * S * 8 * 128 * 2
         assert ws(B, S, 32, 8, 128, 42, W) == (n + 255) // 256 * 256
     # the warp-MMA kernel takes the rest (no rotation, odd group size) and needs none
