@@ -334,9 +334,15 @@ __global__ void __launch_bounds__(FG_THREADS, 1) fwd_glob_tc_kernel(const __grid
                     for (int e = 0; e < 32; ++e) v[32 * c + e] = ((vm >> e) & 1u) ? v[32 * c + e] : -INFINITY;
                 }
             }
-            float mx = v[0];
+            // row max and (below) row sum over 8 and 4 independent partials: a single running
+            // value would make each a chain of dependent instructions as long as the row
+            float mx8[8];
 #pragma unroll
-            for (int e = 1; e < 128; ++e) mx = fmaxf(mx, v[e]);
+            for (int k = 0; k < 8; ++k) mx8[k] = v[k];
+#pragma unroll
+            for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], v[e]);
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             const float mt = mx * c2;   // -inf when the row sees no key of this tile
             const bool raise = mt > m_ref + FG_RESCALE_LOG2;
             const bool warp_raise = __any_sync(0xffffffffu, raise) != 0;
@@ -345,6 +351,7 @@ __global__ void __launch_bounds__(FG_THREADS, 1) fwd_glob_tc_kernel(const __grid
             if (raise) m_ref = mt;
             l *= alpha;
             const float mb = m_ref == -INFINITY ? 0.f : m_ref;
+            float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t pk[16];
@@ -352,11 +359,12 @@ __global__ void __launch_bounds__(FG_THREADS, 1) fwd_glob_tc_kernel(const __grid
                 for (int e = 0; e < 32; e += 2) {
                     const float p0 = fast_exp2(fmaf(v[32 * c + e], c2, -mb));
                     const float p1 = fast_exp2(fmaf(v[32 * c + e + 1], c2, -mb));
-                    l += p0 + p1;
+                    l4[(e >> 1) & 3] += p0 + p1;
                     pk[e >> 1] = pack_bf16(p0, p1);
                 }
                 tmem_st16(TM_S + lane_off + 16 * c, pk);
             }
+            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
             if (warp_raise && n > 0) {
                 // O_x holds PV_x(0..n-1), complete (S_x(n) was issued after PV_x(n-1))
 #pragma unroll 1
