@@ -48,6 +48,11 @@ def load() -> ctypes.CDLL:
         lib.zgcm_attn_fwd_ws.restype = i
         lib.zgcm_attn_fwd_workspace_size.argtypes = [i, i, i, i, i, i, i]
         lib.zgcm_attn_fwd_workspace_size.restype = ctypes.c_size_t
+        lib.zgcm_attn_decode.argtypes = [vp] * 7 + [i] * 5 + [d, i, f, f, vp, vp, i, vp, vp, vp,
+                                                              ctypes.c_size_t, vp]
+        lib.zgcm_attn_decode.restype = i
+        lib.zgcm_attn_decode_workspace_size.argtypes = [i, i, i, i]
+        lib.zgcm_attn_decode_workspace_size.restype = ctypes.c_size_t
         lib.zgcm_attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
         lib.zgcm_attn_bwd_workspace_size.restype = ctypes.c_size_t
         lib.zgcm_attn_bwd.argtypes = ([vp] * 9 + [i] * 6 + [d, i, i, f, f] + [vp] * 7 +
@@ -124,6 +129,40 @@ def zgcm_attn_fwd(q, k, v, g, gamma_q, gamma_k, *, rope_dims=42, rope_base=10000
                                  ws_ptr, ws_bytes, _stream(stream))
     if st != ZGCM_OK:
         raise ZgcmError(st, "zgcm_attn_fwd")
+    return out, lse
+
+
+def zgcm_attn_decode(q, k, v, g, gamma_q, gamma_k, pos, k_cache, v_cache, *, rope_dims=42,
+                     rope_base=10000.0, window=128, eps=1e-6, scale=None, out=None, lse=None,
+                     workspace=None, stream=None):
+    """One decode step: q, g [B,Hq,D] and k, v [B,Hkv,D] bf16 (the new token of each sequence),
+    pos int32 [B] (its position), k_cache fp16 / v_cache bf16 [B,C,Hkv,D] (updated in place).
+    Returns (out bf16 [B,Hq,D], lse fp32 [B,Hq])."""
+    import torch
+    for n, t in (("q", q), ("g", g), ("k", k), ("v", v)):
+        _check(t, n, torch.bfloat16, 3)
+    _check(gamma_q, "gamma_q", torch.float32, 1)
+    _check(gamma_k, "gamma_k", torch.float32, 1)
+    _check(pos, "pos", torch.int32, 1)
+    _check(k_cache, "k_cache", torch.float16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    B, Hq, D = q.shape
+    Hkv, C = k.shape[1], k_cache.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = int(load().zgcm_attn_decode_workspace_size(B, Hq, int(window), C))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = load().zgcm_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos),
+                                 B, Hq, Hkv, D, int(rope_dims), float(rope_base), int(window), float(eps),
+                                 float(scale), _ptr(k_cache), _ptr(v_cache), C, _ptr(out), _ptr(lse),
+                                 _ptr(workspace), workspace.numel(), _stream(stream))
+    if st != ZGCM_OK:
+        raise ZgcmError(st, "zgcm_attn_decode")
     return out, lse
 
 

@@ -14,6 +14,9 @@ cudaError_t launch_fwd_tc(const FwdParams& p, void* workspace, int* err_word, cu
 bool fwd_tc_supported(const LayerParams& L);
 cudaError_t launch_fwd_glob_tc(const FwdParams& p, void* workspace, int* err_word, cudaStream_t stream);
 bool fwd_glob_supported(const LayerParams& L);
+size_t decode_workspace_bytes(int B, int Hq, int window, int C);
+cudaError_t launch_decode(const LayerParams& L, const int* pos, void* k_cache, void* v_cache, int C, void* out,
+                          float* lse, void* workspace, cudaStream_t stream);
 size_t fwd_glob_workspace_bytes(int B, int S, int Hkv);
 cudaError_t launch_bwd_mma(const BwdParams& p, cudaStream_t stream, void* const* events, int n_pairs);
 extern const char* const kBwdMmaKernelNames[];
@@ -227,6 +230,36 @@ int zgcm_attn_fwd(const void* q, const void* k, const void* v, const void* g,
                                     window, causal, eps, scale, out, lse, ws, need, cuda_stream);
     const cudaError_t e = cudaFreeAsync(ws, stream);
     if (st != ZGCM_OK) return st;
+    return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
+}
+
+size_t zgcm_attn_decode_workspace_size(int B, int Hq, int window, int cache_len) {
+    if (B <= 0 || Hq < 1 || window < 1 || cache_len < 1) return 0;
+    return decode_workspace_bytes(B, Hq, window, cache_len);
+}
+
+int zgcm_attn_decode(const void* q, const void* k, const void* v, const void* g,
+                     const float* gamma_q, const float* gamma_k, const int* pos,
+                     int B, int Hq, int Hkv, int D, int rope_dims, double rope_base, int window,
+                     float eps, float scale, void* k_cache, void* v_cache, int cache_len,
+                     void* out, float* lse, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+    int st = check_shape(B, 1, Hq, Hkv, D, rope_dims, rope_base, window, 1, eps, scale);
+    if (st != ZGCM_OK) return st;
+    if (cache_len < 1) return ZGCM_ERR_INVALID_ARG;
+    if (B == 0) return ZGCM_OK;
+    if ((long double)B * cache_len * Hkv * D >= (long double)(1ULL << 40)) return ZGCM_ERR_UNSUPPORTED;
+    const void* ptrs[] = {q, k, v, g, gamma_q, gamma_k, pos, k_cache, v_cache, out, lse};
+    for (const void* p : ptrs)
+        if (!p) return ZGCM_ERR_INVALID_ARG;
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return ZGCM_ERR_ALIGNMENT;
+    const size_t need = zgcm_attn_decode_workspace_size(B, Hq, window, cache_len);
+    if (!workspace || workspace_bytes < need) return ZGCM_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ZGCM_ERR_ALIGNMENT;
+    LayerParams L;
+    fill_layer(L, q, k, v, g, gamma_q, gamma_k, B, 1, Hq, Hkv, rope_dims, rope_base, window, eps, scale);
+    const cudaError_t e = launch_decode(L, static_cast<const int*>(pos), k_cache, v_cache, cache_len, out, lse,
+                                        workspace, static_cast<cudaStream_t>(cuda_stream));
     return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
 }
 

@@ -186,6 +186,43 @@ int zgcm_attn_bwd_noalloc(const void* q, const void* k, const void* v, const voi
                           float* dgamma_q, float* dgamma_k, void* cuda_stream);
 
 /*
+ * One decode step (inference): a single new token per sequence against a KV cache.  The
+ * sliding layers keep a ring of `window` key/value slots per sequence (the constant-size
+ * cache of the ZGCM-1 KV design: 128 tokens per sliding layer, ZGCM-1 summary section
+ * "前置知识"); the global layers keep every token (a growing cache).
+ *
+ * For sequence b at position p = pos[b]: the new key k is RMS-normalised and rotated at p
+ * (as in the forward) and stored with v in cache slot p mod cache_len; then
+ *   out = sigmoid(g) * softmax_j(scale q~ . k~_j) v_j   over j = max(0, p-window+1) .. p,
+ *   lse = log sum_j exp(scale q~ . k~_j),
+ * the forward's row p for the same tokens (each key written by an earlier call).
+ *
+ * In : q, g bf16 [B,Hq,D] and k, v bf16 [B,Hkv,D]: the new token of each sequence (raw,
+ *      before the norm); pos int32 [B], device: the token's position (0-based);
+ *      gamma_q, gamma_k fp32 [D].
+ * Cache (caller-owned, updated in place): k_cache fp16 [B,cache_len,Hkv,D] holds the
+ *      normalised, rotated keys times the power of two the training kernels use for their
+ *      fp16 keys (1 unless max|gamma| sqrt(D) > 16384); v_cache bf16 [B,cache_len,Hkv,D] the
+ *      values.  Position j lives in slot j mod cache_len.  The window's keys must all still
+ *      be there: cache_len >= min(window, p + 1) (a ring of cache_len = window slots for a
+ *      sliding layer; cache_len > the longest position for a global one).  A row whose
+ *      window is longer than the cache gets NaN (out and lse); its cache is not written.
+ * Out: out bf16 [B,Hq,D]; lse fp32 [B,Hq].
+ * workspace: at least zgcm_attn_decode_workspace_size(...) bytes, 16-byte aligned (split
+ *      partial results).  Same checks, errors and stream behaviour as the forward.
+ * Kernels: decode_split_kernel (one CTA per sequence, KV head and split of up to 512 keys),
+ *      then decode_combine_kernel.
+ */
+int zgcm_attn_decode(const void* q, const void* k, const void* v, const void* g,
+                     const float* gamma_q, const float* gamma_k, const int* pos,
+                     int B, int Hq, int Hkv, int D, int rope_dims, double rope_base, int window,
+                     float eps, float scale, void* k_cache, void* v_cache, int cache_len,
+                     void* out, float* lse, void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* Bytes of workspace zgcm_attn_decode needs (0 for invalid arguments or B == 0). */
+size_t zgcm_attn_decode_workspace_size(int B, int Hq, int window, int cache_len);
+
+/*
  * Main kernel zgcm_attn_fwd launches for this configuration (static string):
  * "fwd_tc_kernel" (tcgen05/TMEM/TMA, sliding windows up to 128 with 42 rotated dims),
  * "fwd_glob_tc_kernel" (tcgen05, wider windows and the global layer, with 42 rotated dims

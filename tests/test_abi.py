@@ -145,3 +145,32 @@ def test_fwd_ws_checks(lib):
     assert _fwd_ws(lib, P + 256 * 40 + 16, need, S=640, window=640) == -3
     assert _fwd_ws(lib, P + 256 * 40, need, S=640, window=640, D=96) == -2
     assert _fwd_ws(lib, P + 256 * 40, need, S=640, window=0) == -1
+
+
+def _dec(lib, ws_bytes, ptrs=None, ws=P + 256 * 40, **kw):
+    a = dict(ARGS, **kw)
+    vp = ctypes.c_void_p
+    p = ptrs or [P + 256 * i for i in range(11)]
+    return lib.zgcm_attn_decode(*(vp(x) for x in p[:7]), a["B"], a["Hq"], a["Hkv"], a["D"], a["rope_dims"],
+                                a["rope_base"], a["window"], a["eps"], a["scale"], vp(p[7]), vp(p[8]),
+                                a.get("cache_len", 128), vp(p[9]), vp(p[10]), vp(ws), ws_bytes, None)
+
+
+def test_decode_checks(lib):
+    need = lib.zgcm_attn_decode_workspace_size(1, 32, 128, 128)
+    # one split of up to 512 keys per (sequence, head): max, sum, 2 pad and 128 partial outputs
+    assert need == 1 * 32 * 1 * (4 + 128) * 4
+    assert lib.zgcm_attn_decode_workspace_size(2, 32, 10**6, 65536) == 2 * 32 * 128 * 132 * 4
+    assert lib.zgcm_attn_decode_workspace_size(2, 32, 300, 65536) == 2 * 32 * 1 * 132 * 4
+    assert lib.zgcm_attn_decode_workspace_size(0, 32, 128, 128) == 0
+    assert _dec(lib, need - 1) == -4
+    assert _dec(lib, need, ws=0) == -4
+    assert _dec(lib, need, cache_len=0) == -1
+    assert _dec(lib, need, D=64) == -2
+    assert _dec(lib, need, window=0) == -1
+    good = [P + 256 * i for i in range(11)]
+    for i in range(11):
+        p = list(good); p[i] = 0
+        assert _dec(lib, need, ptrs=p) == -1
+        p = list(good); p[i] = good[i] + 4
+        assert _dec(lib, need, ptrs=p) == -3

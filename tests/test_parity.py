@@ -170,6 +170,62 @@ def test_backward_wide_window_kernels(B, S, W, monkeypatch):
     assert_dgamma_close("dgamma_k", gr["dgamma_k"], ref["dgamma_k"])
 
 
+def _decode_run(t, W, C, offsets=None, rope_dims=42):
+    """Feed each sequence of t token by token through zgcm_attn_decode; sequence b starts
+    offsets[b] calls late (before that it replays its token 0 at position 0, which rewrites the
+    same cache slot with the same values).  Returns out [T, B, Hq, D], lse [T, B, Hq], pos [T, B]."""
+    B, S, Hq, D = t["q"].shape
+    Hkv = t["k"].shape[2]
+    offsets = offsets or [0] * B
+    d = _to_dev(t)
+    kc = torch.zeros((B, C, Hkv, D), dtype=torch.float16, device="cuda")
+    vc = torch.zeros((B, C, Hkv, D), dtype=torch.bfloat16, device="cuda")
+    outs, lses, poss = [], [], []
+    ar = torch.arange(B, device="cuda")
+    for call in range(S + max(offsets)):
+        pos = torch.tensor([min(max(call - o, 0), S - 1) for o in offsets], dtype=torch.int32, device="cuda")
+        pl = pos.long()
+        o, l = ga.zgcm_attn_decode(d["q"][ar, pl].contiguous(), d["k"][ar, pl].contiguous(),
+                                   d["v"][ar, pl].contiguous(), d["g"][ar, pl].contiguous(),
+                                   d["gamma_q"], d["gamma_k"], pos, kc, vc, window=W, rope_dims=rope_dims)
+        outs.append(o.clone()); lses.append(l.clone()); poss.append(pos.cpu())
+    torch.cuda.synchronize()
+    return torch.stack(outs), torch.stack(lses), torch.stack(poss)
+
+
+@pytest.mark.parametrize("B,S,W,C", [(2, 300, 128, 128),     # sliding layer: a ring of W slots
+                                     (1, 700, 700, 768),     # global layer: every token kept, 2 splits
+                                     (3, 200, 50, 64),       # ring larger than the window
+                                     (2, 1100, 10**6, 1100)])  # global, 3 splits of 512 keys
+def test_decode_matches_forward_rows(B, S, W, C):
+    """Decoding a sequence token by token gives, at every step, the forward's row for that
+    position (the oracle's), through the layer's sliding ring cache or its growing one."""
+    t = make_inputs(B, S, seed=500 + S + W % 997)
+    out, lse, pos = _decode_run(t, W, C)
+    ref_out, ref_lse = _problem(t, window=W).forward()
+    # call c decodes position c of every sequence
+    got = f64(out).transpose(1, 0, 2, 3)          # [B, S, Hq, D]
+    assert_bf16_close("decode out", got, ref_out)
+    assert_lse_close("decode lse", f64(lse).transpose(1, 2, 0), ref_lse)
+    assert ga.zgcm_attn_device_error() == 0
+
+
+def test_decode_ragged_positions_and_short_cache():
+    B, S, W = 3, 160, 128
+    t = make_inputs(B, S, seed=77)
+    offsets = [0, 7, 33]
+    out, lse, pos = _decode_run(t, W, W, offsets=offsets)
+    ref_out, ref_lse = _problem(t, window=W).forward()
+    for b, o in enumerate(offsets):
+        calls = np.arange(o, o + S)
+        got = f64(out[calls, b])                  # positions 0..S-1 of sequence b
+        assert_bf16_close(f"decode out[{b}]", got, ref_out[b])
+    # a window longer than the cache: rows past the cache get NaN, earlier ones are exact
+    out2, lse2, _ = _decode_run(make_inputs(1, 100, seed=3), 80, 64)
+    o2 = f64(out2)
+    assert np.isnan(o2[64:]).all() and np.isfinite(o2[:64]).all()
+
+
 def test_empty_problem():
     for B, S in ((0, 16), (2, 0)):
         t = make_inputs(max(B, 1), max(S, 1), with_dout=True)
