@@ -285,18 +285,190 @@ def workload_name(w):
     return f"gated {kind} attention {'fwd+bwd' if bwd else 'fwd'}, B={B} S={S} Hq={HQ} Hkv={HKV} D={D}"
 
 
+# decode: B sequences at context position P, one new token each, per layer (window, cache
+# slots, weight of the layer in the 5:1 sliding:global pattern)
+DECODE_WORKLOADS = {
+    "decode16k": (64, 16383, ((128, 128, 5), (16384, 16384, 1))),
+}
+
+
+def decode_bytes(B, P, W, C):
+    """Algorithmic HBM bytes of one decode call: every visible cached key (fp16) and value
+    (bf16) read once; the new token's q, g, k, v read, out written; its cache slot written."""
+    vis = min(W, C, P + 1)
+    return (B * vis * HKV * D * 4 + B * HQ * D * 2 * 3 + B * HKV * D * 2 * 2 + B * HKV * D * 4
+            + B * HQ * 4)
+
+
+def run_decode(args):
+    """One decode step per layer of the workload: B tokens through zgcm_attn_decode."""
+    import torch
+    import global_attention_b200 as ga
+    world, rank, local = rank_env()
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ga.load()
+    B, P, layers = DECODE_WORKLOADS[args.workload]
+    gen = torch.Generator().manual_seed(1000 + rank)
+    tok = {n: torch.randn((B, h, D), generator=gen).to(torch.bfloat16)
+           for n, h in (("q", HQ), ("k", HKV), ("v", HKV), ("g", HQ))}
+    gam = {n: torch.rand((D,), generator=gen) + 0.5 for n in ("gamma_q", "gamma_k")}
+    host = {n: t.pin_memory() for n, t in {**tok, **gam}.items()}
+    d = {n: t.to(dev) for n, t in host.items()}
+    pos = torch.full((B,), P, dtype=torch.int32, device=dev)
+    caches = []
+    for W, C, _ in layers:
+        # synthetic cache contents of the shape and scale of normalised keys / raw values
+        kc = (torch.randn((B, C, HKV, D), generator=gen) * 1.0).to(torch.float16).to(dev)
+        vc = torch.randn((B, C, HKV, D), generator=gen).to(torch.bfloat16).to(dev)
+        ws = torch.empty(max(16, ga.zgcm_attn_decode_workspace_size(B, HQ, W, C)), dtype=torch.uint8, device=dev)
+        caches.append((kc, vc, ws))
+    out = torch.empty((B, HQ, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, HQ), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call(li, src=d):
+        W, C, _ = layers[li]
+        kc, vc, ws = caches[li]
+        ga.zgcm_attn_decode(src["q"], src["k"], src["v"], src["g"], src["gamma_q"], src["gamma_k"], pos, kc, vc,
+                            window=W, out=out, lse=lse, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        for li in range(len(layers)):
+            call(li)
+    torch.cuda.synchronize()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in layers]
+          for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            for li in range(len(layers)):
+                ev[i][li][0].record(stream)
+                call(li)
+                ev[i][li][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev) / args.steps
+    layer_ms = [statistics.mean(ev[i][li][0].elapsed_time(ev[i][li][1]) for i in range(args.steps))
+                for li in range(len(layers))]
+    # end to end: the new tokens from pinned host memory, the outputs back, every step
+    outs_host = torch.empty_like(out, device="cpu").pin_memory()
+    h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v", "g"))
+    d2h = outs_host.numel() * outs_host.element_size()
+    dst = {n: torch.empty_like(t) for n, t in d.items()}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        for n in ("q", "k", "v", "g"):
+            dst[n].copy_(host[n], non_blocking=True)
+        for n in ("gamma_q", "gamma_k"):
+            dst[n] = d[n]
+        for li in range(len(layers)):
+            call(li, dst)
+            outs_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        if rank != 0:
+            dist.destroy_process_group()
+            return 0
+    peaks, peak_src = load_peaks()
+    # roofline of the heaviest layer's call (HBM-bound: it reads its whole window of cache)
+    li = max(range(len(layers)), key=lambda k: layer_ms[k])
+    W, C, _ = layers[li]
+    nbytes = decode_bytes(B, P, W, C)
+    roof = {"bound": "hbm", "achieved": nbytes / (layer_ms[li] / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "traffic": None, "kernel": f"decode_split_kernel + decode_combine_kernel (W={W})",
+            "kernel_ms": layer_ms[li], "algorithmic_bytes": nbytes, "peak_source": peak_src}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    step_bytes = sum(decode_bytes(B, P, W, C) for W, C, _ in layers)
+    t_roof = step_bytes / (peaks["hbm_gbs"] * 1e9)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = decode_cpu_baseline(P, layers)
+    wsum = sum(wt for _, _, wt in layers)
+    mix_ms = sum(wt * t for (_, _, wt), t in zip(layers, layer_ms)) / wsum
+    rec = {
+        "metric": METRIC, "value": job_throughput(B, world, ms), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) bf16 tokens, N(0,1) fp16 / bf16 cache contents",
+        "config": {"workload": f"gated attention decode, {B} sequences at position {P}, one token each through "
+                               + " + ".join(f"W={W} (cache {C})" for W, C, _ in layers)
+                               + f", Hq={HQ} Hkv={HKV} D={D}",
+                   "global_batch": B * world, "seq_len": P + 1, "parallelism": f"dp{world} (independent sequences)",
+                   "l2": f"caches larger than L2 ({sum(c[0].numel() * 2 + c[1].numel() * 2 for c in caches) / 1e9:.2f} GB)"},
+        "pct_of_roofline": t_roof / (ms / 1e3), "roofline_step_ms": t_roof * 1e3,
+        "roofline": roof, "cpu_baseline": cpu,
+        "e2e": {"value": job_throughput(B, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h * len(layers), "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * len(layers) * args.steps,
+        "clocks": clk.summary(),
+        "layer_mix": {"layers": [{"window": W, "cache": C, "weight": wt, "ms": t}
+                                 for (W, C, wt), t in zip(layers, layer_ms)],
+                      "weighted_ms_per_layer": mix_ms},
+    }
+    print(json.dumps(rec))
+    return 0
+
+
+def decode_cpu_baseline(P, layers):
+    """The oracle's forward rows for a bounded sample: the last row of 2 sequences of P + 1
+    tokens per layer (the row a decode step computes), tokens per second over both layers."""
+    import oracle
+    from global_attention_b200.synth import make_inputs
+    oracle.build()
+    spt, parts = 0.0, []
+    for W, C, _ in layers:
+        t = make_inputs(2, P + 1, seed=7)
+        prob = oracle.Problem(t["q"], t["k"], t["v"], t["g"], t["gamma_q"], t["gamma_k"], window=W)
+        rows = [P, (P + 1) + P]        # flat row index b * S + i
+        t0 = time.perf_counter()
+        prob.forward(rows)
+        secs = time.perf_counter() - t0
+        spt += secs / 2
+        parts.append(f"2 rows at position {P}, window {W}: {secs:.2f} s")
+    return {"value": 1.0 / spt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "; ".join(parts) + " (the oracle's per-row forward, fp64, including its prologue)"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="swa16k")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS), default="swa16k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload in DECODE_WORKLOADS:
+        if args.impl == "reference":
+            _, rank, _ = rank_env()
+            if rank == 0:
+                B, P, layers = DECODE_WORKLOADS[args.workload]
+                cpu = decode_cpu_baseline(P, layers)
+                print(json.dumps({"impl": "reference", "metric": METRIC, "value": cpu["value"], "unit": "tokens/s",
+                                  "n_gpus": args.gpus, "steps": 1, "warmup": 0, "higher_is_better": True,
+                                  "dtype": "f64", "data": "synthetic", "cpu_baseline": cpu,
+                                  "e2e": {"value": cpu["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                                          "d2h_bytes_per_step": 0}}))
+            return 0
+        return run_decode(args)
     if args.impl == "reference":
         return run_reference(args)
 

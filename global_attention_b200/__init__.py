@@ -132,6 +132,11 @@ def zgcm_attn_fwd(q, k, v, g, gamma_q, gamma_k, *, rope_dims=42, rope_base=10000
     return out, lse
 
 
+def zgcm_attn_decode_workspace_size(B, Hq, window, cache_len) -> int:
+    """Bytes of workspace zgcm_attn_decode needs."""
+    return int(load().zgcm_attn_decode_workspace_size(int(B), int(Hq), int(window), int(cache_len)))
+
+
 def zgcm_attn_decode(q, k, v, g, gamma_q, gamma_k, pos, k_cache, v_cache, *, rope_dims=42,
                      rope_base=10000.0, window=128, eps=1e-6, scale=None, out=None, lse=None,
                      workspace=None, stream=None):
@@ -154,7 +159,7 @@ def zgcm_attn_decode(q, k, v, g, gamma_q, gamma_k, pos, k_cache, v_cache, *, rop
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    need = int(load().zgcm_attn_decode_workspace_size(B, Hq, int(window), C))
+    need = zgcm_attn_decode_workspace_size(B, Hq, window, C)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     st = load().zgcm_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos),

@@ -83,48 +83,68 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const __grid_
         prologue_row(load_row4(L.q + ((size_t)b * L.Hq + hq) * kD), gq + 4 * lane, L, pos, ybuf[warp], q4);
         float m = -INFINITY, l = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
         if (fits) {
-            // four keys per iteration: their dot products and butterfly sums are independent
-            // (every lane ends each sum with the same value, so m is warp-uniform)
-            for (int j = j0; j < j1; j += 4) {
-                const int nk = min(4, j1 - j);
-                float d[4], vv[4][4];
+            // eight keys per iteration: all their loads are issued before any is used (a key
+            // past the split's end loads the split's last key and is masked), and their dot
+            // products and butterfly sums are independent (every lane ends each sum with the
+            // same value, so m is warp-uniform).  The cache slot advances with j, wrapping at C.
+            constexpr int KB = 8;
+            const size_t head_off = (size_t)kvh * kD + 4 * lane;
+            const size_t seq_off = (size_t)b * p.C;
+            uint2 kw[KB], vw[KB];
+            // loads of the keys j .. j+KB-1 (slots from `slot`; keys past the split's end load
+            // its last key again, masked below)
+            auto load_batch = [&](int j, int slot) {
+                const int nk = min(KB, j1 - j);
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    d[t] = -INFINITY;
-                    if (t < nk) {
-                        const size_t off = ((size_t)b * p.C + (j + t) % p.C) * kv_row + (size_t)kvh * kD + 4 * lane;
-                        const uint2 kw = *reinterpret_cast<const uint2*>(p.kc + off);
-                        const uint2 vw = *reinterpret_cast<const uint2*>(p.vc + off);
-                        const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kw.x));
-                        const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kw.y));
-                        d[t] = q4[0] * k01.x + q4[1] * k01.y + q4[2] * k23.x + q4[3] * k23.y;
-                        const float2 v01 = unpack_bf16(vw.x), v23 = unpack_bf16(vw.y);
-                        vv[t][0] = v01.x; vv[t][1] = v01.y; vv[t][2] = v23.x; vv[t][3] = v23.y;
-                    } else {
-                        vv[t][0] = vv[t][1] = vv[t][2] = vv[t][3] = 0.f;
-                    }
+                for (int t = 0; t < KB; ++t) {
+                    int sl = slot + min(t, nk - 1);
+                    sl = sl >= p.C ? sl - p.C : sl;
+                    const size_t off = (seq_off + sl) * kv_row + head_off;
+                    kw[t] = *reinterpret_cast<const uint2*>(p.kc + off);
+                    vw[t] = *reinterpret_cast<const uint2*>(p.vc + off);
                 }
+            };
+            int slot = j0 % p.C;
+            if (j0 < j1) load_batch(j0, slot);
+            for (int j = j0; j < j1; j += KB) {
+                const int nk = min(KB, j1 - j);
+                float d[KB], vf[KB][4];
+#pragma unroll
+                for (int t = 0; t < KB; ++t) {
+                    const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kw[t].x));
+                    const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kw[t].y));
+                    d[t] = q4[0] * k01.x + q4[1] * k01.y + q4[2] * k23.x + q4[3] * k23.y;
+                    const float2 v01 = unpack_bf16(vw[t].x), v23 = unpack_bf16(vw[t].y);
+                    vf[t][0] = v01.x; vf[t][1] = v01.y; vf[t][2] = v23.x; vf[t][3] = v23.y;
+                }
+                // the next batch's loads go out while this one is reduced
+                slot += KB;
+                slot = slot >= p.C ? slot - p.C : slot;
+                if (j + KB < j1) load_batch(j + KB, slot);
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) {
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) d[t] += __shfl_xor_sync(0xffffffffu, d[t], off);
+                    for (int t = 0; t < KB; ++t) d[t] += __shfl_xor_sync(0xffffffffu, d[t], off);
                 }
+                float mn = m;
 #pragma unroll
-                for (int t = 0; t < 4; ++t) d[t] = t < nk ? d[t] * c2 : -INFINITY;
-                const float mn = fmaxf(fmaxf(m, fmaxf(d[0], d[1])), fmaxf(d[2], d[3]));
+                for (int t = 0; t < KB; ++t) {
+                    d[t] = t < nk ? d[t] * c2 : -INFINITY;
+                    mn = fmaxf(mn, d[t]);
+                }
                 if (mn > m) {
-                    const float a = exp2f(m - mn);  // 0 from the empty start
+                    const float a = fast_exp2(m - mn);  // 0 from the empty start
                     l *= a;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) o[e] *= a;
                     m = mn;
                 }
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const float pj = exp2f(d[t] - m);   // 0 for the padding keys
+                for (int t = 0; t < KB; ++t) {
+                    const float pj = fast_exp2(d[t] - m);   // 0 for the padding keys
                     l += pj;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) o[e] = fmaf(pj, vv[t][e], o[e]);
+                    for (int e = 0; e < 4; ++e) o[e] = fmaf(pj, vf[t][e], o[e]);
                 }
             }
         } else {
