@@ -168,7 +168,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except OSError:
@@ -229,7 +229,7 @@ def cpu_sample_shape(Bw, Sw, W):
     shorter sequences (window work per token is the same once past the first W tokens)."""
     if W >= Sw:            # global layer: a shorter causal sequence
         return 1, 2048, 2048
-    return 4, 2048, W
+    return 8, 8192, W
 
 
 def run_reference(args):
@@ -447,7 +447,7 @@ def decode_cpu_baseline(P, layers):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS), default="swa16k")
