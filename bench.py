@@ -452,7 +452,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS), default="swa16k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -519,18 +519,19 @@ def main():
     fws = [None if n == 0 else torch.empty(n, dtype=torch.uint8, device=dev)
            for n in (ga.zgcm_attn_fwd_workspace_size(Bw, Sw, HQ, HKV, D, 42, lw) for lw, _ in layers)]
 
-    def step(i=None, src=d):
+    def step(i=None, src=d, dst=None):
+        o = dst or {"out": out, "lse": lse, "grads": grads}
         for li, (lw, _) in enumerate(layers):
             if i is not None:
                 ev_f[i][li][0].record(stream)
             ga.zgcm_attn_fwd(src["q"], src["k"], src["v"], src["g"], src["gamma_q"], src["gamma_k"],
-                             window=lw, out=out, lse=lse, workspace=fws[li], stream=stream)
+                             window=lw, out=o["out"], lse=o["lse"], workspace=fws[li], stream=stream)
             if i is not None:
                 ev_f[i][li][1].record(stream)
             if bwd:
                 ga.zgcm_attn_bwd(src["q"], src["k"], src["v"], src["g"], src["gamma_q"], src["gamma_k"],
-                                 out, lse, src["dout"], window=lw, grads=grads, workspace=ws, stream=stream,
-                                 kernel_events=None if i is None else ev_m[i][li])
+                                 o["out"], o["lse"], src["dout"], window=lw, grads=o["grads"], workspace=ws,
+                                 stream=stream, kernel_events=None if i is None else ev_m[i][li])
 
     for _ in range(args.warmup):
         step()
@@ -568,7 +569,10 @@ def main():
     ms = max_over_ranks(ms, world, dev)
     ms_step = ms / args.steps
 
-    # ---- end to end through the public API: pinned host inputs -> HBM -> fwd+bwd -> host
+    # ---- end to end through the public API: pinned host inputs -> HBM -> fwd+bwd -> host.
+    # Every step uploads its inputs and downloads its results; the copies run on streams of
+    # their own with double-buffered device tensors, so the download of step i overlaps the
+    # upload of step i+1 (the two copy directions are independent) and both overlap compute.
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     outs_host = {"out": torch.empty_like(out, device="cpu").pin_memory(),
                  "lse": torch.empty_like(lse, device="cpu").pin_memory()}
@@ -576,21 +580,41 @@ def main():
         for k, v in grads.items():
             outs_host[k] = torch.empty_like(v, device="cpu").pin_memory()
     d2h = sum(v.numel() * v.element_size() for v in outs_host.values())
-    dst = {k: torch.empty_like(v) for k, v in d.items()}
+    inbuf = [{k: torch.empty_like(v) for k, v in d.items()} for _ in range(2)]
+    outbuf = [{"out": torch.empty_like(out), "lse": torch.empty_like(lse),
+               "grads": {k: torch.empty_like(v) for k, v in grads.items()} if bwd else None} for _ in range(2)]
+    s_up, s_dn = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_up = [torch.cuda.Event() for _ in range(2)]
+    ev_cp = [torch.cuda.Event() for _ in range(2)]
+    ev_dn = [torch.cuda.Event() for _ in range(2)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(args.e2e_steps):
-        for k in dst:
-            dst[k].copy_(host[k], non_blocking=True)
-        step(src=dst)
-        outs_host["out"].copy_(out, non_blocking=True)
-        outs_host["lse"].copy_(lse, non_blocking=True)
-        if bwd:
-            for k, v in grads.items():
-                outs_host[k].copy_(v, non_blocking=True)
+    s_up.wait_event(e0)
+    s_dn.wait_event(e0)
+    for i in range(args.e2e_steps):
+        x = i & 1
+        with torch.cuda.stream(s_up):
+            s_up.wait_event(ev_cp[x])          # step i-2's compute has read inbuf[x]
+            for k in inbuf[x]:
+                inbuf[x][k].copy_(host[k], non_blocking=True)
+            ev_up[x].record(s_up)
+        stream.wait_event(ev_up[x])
+        stream.wait_event(ev_dn[x])            # step i-2's results have left outbuf[x]
+        step(src=inbuf[x], dst=outbuf[x])
+        ev_cp[x].record(stream)
+        with torch.cuda.stream(s_dn):
+            s_dn.wait_event(ev_cp[x])
+            outs_host["out"].copy_(outbuf[x]["out"], non_blocking=True)
+            outs_host["lse"].copy_(outbuf[x]["lse"], non_blocking=True)
+            if bwd:
+                for k, v in outbuf[x]["grads"].items():
+                    outs_host[k].copy_(v, non_blocking=True)
+            ev_dn[x].record(s_dn)
+    for x in range(2):
+        stream.wait_event(ev_dn[x])
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
