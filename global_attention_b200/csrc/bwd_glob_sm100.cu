@@ -100,6 +100,28 @@ struct BwdQGlobSmem {
 static_assert(sizeof(BwdQGlobSmem) + 1024 <= 232448, "beyond the 227 KB of shared memory a CTA can have");
 size_t bwd_q_glob_smem_bytes() { return sizeof(BwdQGlobSmem) + 1024; }
 
+// dS of 32 keys of a row, already times its power-of-two scale dsc (kds = kd dsc, dls =
+// Delta dsc: a power-of-two factor commutes with every rounding, so these are the values
+// (P (dP kd - Delta)) dsc exactly), packed to fp16; ma[] accumulates (dS dsc) S in two
+// partials.  MASK: keys outside the row's window (vm) get P = 0.
+template <bool MASK>
+__device__ __forceinline__ void qg_ds_chunk(const float* sv, const float* dv, uint32_t vm, float c2, float lse2,
+                                            float kds, float dls, float (&ma)[2], uint32_t (&pk)[16]) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        const float s0 = sv[e], s1 = sv[e + 1];
+        float p0 = fast_exp2(fmaf(s0, c2, -lse2)), p1 = fast_exp2(fmaf(s1, c2, -lse2));
+        if (MASK) {
+            p0 = ((vm >> e) & 1u) ? p0 : 0.f;  // (a masked score may overflow: selected away)
+            p1 = ((vm >> (e + 1)) & 1u) ? p1 : 0.f;
+        }
+        const float d0 = p0 * fmaf(dv[e], kds, -dls), d1 = p1 * fmaf(dv[e + 1], kds, -dls);
+        ma[0] = fmaf(d0, s0, ma[0]);
+        ma[1] = fmaf(d1, s1, ma[1]);
+        pk[e >> 1] = pack2<true>(d0, d1);
+    }
+}
+
 __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid_constant__ BwdTcParams p) {
     const LayerParams& L = p.P.L;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -314,7 +336,7 @@ __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid
         const float* vtrow = p.vtinv + ((size_t)b * L.Hkv + kvh) * nkt;
         const int lo = max(i - L.W + 1, 0), hi = i;              // this row's visible keys
         const int rmin = q0 + 32 * wq, rmax = rmin + 31;        // rows of this warp
-        float macc = 0.f;                                        // sum_j dS_ij S_ij (unscaled dS)
+        float macc2[2] = {0.f, 0.f};                             // sum_j (dS_ij dsc) S_ij, two partials
         bool ok = true;
         for (int n = 0; n < N && ok; ++n) {
             const int kc0 = (kt_lo + n) * TF_BN + 64 * hh;       // first key of this half
@@ -355,20 +377,15 @@ __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid
                 delta = valid ? dpart[r] + dpart[TF_BM + r] : 0.f;
                 if (hh == 0 && valid) p.P.delta[rp] = delta;
             }
+            const float kds = kd * dsc, dls = delta * dsc;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                const uint32_t vm = full ? 0xffffffffu : bit_range(lo - (kc0 + 32 * c), hi - (kc0 + 32 * c));
                 uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float s0 = sv[32 * c + e], s1 = sv[32 * c + e + 1];
-                    float p0 = fast_exp2(fmaf(s0, c2, -lse2)), p1 = fast_exp2(fmaf(s1, c2, -lse2));
-                    p0 = ((vm >> e) & 1u) ? p0 : 0.f;  // (a masked score may overflow: selected away)
-                    p1 = ((vm >> (e + 1)) & 1u) ? p1 : 0.f;
-                    const float d0 = p0 * fmaf(dv[32 * c + e], kd, -delta);
-                    const float d1 = p1 * fmaf(dv[32 * c + e + 1], kd, -delta);
-                    macc = fmaf(d0, s0, fmaf(d1, s1, macc));
-                    pk[e >> 1] = pack2<true>(d0 * dsc, d1 * dsc);
+                if (full) {
+                    qg_ds_chunk<false>(sv + 32 * c, dv + 32 * c, 0u, c2, lse2, kds, dls, macc2, pk);
+                } else {
+                    const uint32_t vm = bit_range(lo - (kc0 + 32 * c), hi - (kc0 + 32 * c));
+                    qg_ds_chunk<true>(sv + 32 * c, dv + 32 * c, vm, c2, lse2, kds, dls, macc2, pk);
                 }
                 tmem_st16(tm_s(n) + lane_off + 64 * hh + 16 * c, pk);
             }
@@ -376,6 +393,8 @@ __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid
             tc_fence_before();
             mbar_arrive(&sm.bar[QG_DSFULL]);
         }
+        // sum_j dS_ij S_ij (dsc, a power of two, divides out exactly)
+        const float macc = (macc2[0] + macc2[1]) / dsc;
         if (hh == 1) {
             reinterpret_cast<float*>(sm.V[1][0])[256 + r] = macc;  // mdot_hi
             mbar_arrive(&sm.bar[QG_MDOT]);
