@@ -64,6 +64,8 @@ def load() -> ctypes.CDLL:
         lib.zgcm_attn_bwd_kernel_name.restype = ctypes.c_char_p
         lib.zgcm_attn_fwd_kernel_name.argtypes = [i, i, i, i, i, i]
         lib.zgcm_attn_fwd_kernel_name.restype = ctypes.c_char_p
+        lib.zgcm_attn_selftest_expired_wait.argtypes = [vp]
+        lib.zgcm_attn_selftest_expired_wait.restype = i
         lib.zgcm_attn_device_error.argtypes = []
         lib.zgcm_attn_device_error.restype = i
         lib.zgcm_attn_bwd_noalloc.argtypes = [vp] * 9 + [i] * 6 + [d, i, i, f, f] + [vp] * 7
@@ -179,6 +181,11 @@ def zgcm_attn_fwd_kernel_name(B, S, Hq, Hkv, rope_dims=42, window=128) -> str:
     """Name of the kernel zgcm_attn_fwd launches for this configuration."""
     return load().zgcm_attn_fwd_kernel_name(int(B), int(S), int(Hq), int(Hkv), int(rope_dims),
                                             int(window)).decode()
+
+
+def zgcm_attn_selftest_expired_wait(stream=None) -> int:
+    """Launch the bounded-wait self-test (a wait that expires); see the C header."""
+    return int(load().zgcm_attn_selftest_expired_wait(_stream(stream)))
 
 
 def zgcm_attn_device_error() -> int:

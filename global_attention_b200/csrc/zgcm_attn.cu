@@ -15,6 +15,7 @@ bool fwd_tc_supported(const LayerParams& L);
 cudaError_t launch_fwd_glob_tc(const FwdParams& p, void* workspace, int* err_word, cudaStream_t stream);
 bool fwd_glob_supported(const LayerParams& L);
 size_t decode_workspace_bytes(int B, int Hq, int window, int C);
+cudaError_t launch_selftest_expired_wait(int* err_word, cudaStream_t stream);
 cudaError_t launch_decode(const LayerParams& L, const int* pos, void* k_cache, void* v_cache, int C, void* out,
                           float* lse, void* workspace, cudaStream_t stream);
 size_t fwd_glob_workspace_bytes(int B, int S, int Hkv);
@@ -261,6 +262,12 @@ int zgcm_attn_decode(const void* q, const void* k, const void* v, const void* g,
     const cudaError_t e = launch_decode(L, static_cast<const int*>(pos), k_cache, v_cache, cache_len, out, lse,
                                         workspace, static_cast<cudaStream_t>(cuda_stream));
     return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
+}
+
+int zgcm_attn_selftest_expired_wait(void* cuda_stream) {
+    return launch_selftest_expired_wait(device_error_word(), static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess
+               ? ZGCM_OK
+               : ZGCM_ERR_CUDA;
 }
 
 int zgcm_attn_device_error(void) {

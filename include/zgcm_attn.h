@@ -240,6 +240,14 @@ const char* zgcm_attn_fwd_kernel_name(int B, int S, int Hq, int Hkv, int rope_di
  */
 int zgcm_attn_device_error(void);
 
+/*
+ * Test of the failure path above, without a fault: launches one CTA that waits on a barrier
+ * nothing arrives on.  The bounded wait expires (about a second), the CTA records the site
+ * as the attention kernels would and returns, so the next zgcm_attn_device_error() returns
+ * ZGCM_ERR_TIMEOUT and the context stays usable.  Asynchronous on `cuda_stream`.
+ */
+int zgcm_attn_selftest_expired_wait(void* cuda_stream);
+
 /* Name of the i-th kernel zgcm_attn_bwd launches for this configuration (static string),
  * or NULL when i is past the last one.  With 42 rotated dims, windows up to 128 run the
  * gate pass, the K/V and Q preparation and the tcgen05 pair (bwd_gate_kernel,

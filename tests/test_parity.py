@@ -226,6 +226,25 @@ def test_decode_ragged_positions_and_short_cache():
     assert np.isnan(o2[64:]).all() and np.isfinite(o2[:64]).all()
 
 
+def test_bounded_wait_expires_and_is_reported():
+    """A wait nothing satisfies gives up after its bound, the kernel returns, the host reads
+    ZGCM_ERR_TIMEOUT (once), and the context still computes correct results."""
+    import time
+    assert ga.zgcm_attn_device_error() == 0
+    t0 = time.perf_counter()
+    assert ga.zgcm_attn_selftest_expired_wait() == 0
+    torch.cuda.synchronize()
+    waited = time.perf_counter() - t0
+    assert ga.zgcm_attn_device_error() == -6      # ZGCM_ERR_TIMEOUT
+    assert ga.zgcm_attn_device_error() == 0       # read and cleared
+    assert waited < 60.0
+    t = make_inputs(1, 256, seed=12)
+    d = _to_dev(t)
+    out, lse = _gpu_fwd(d)
+    ref_out, _ = _problem(t).forward()
+    assert_bf16_close("out after the expired wait", out, ref_out)
+
+
 def test_empty_problem():
     for B, S in ((0, 16), (2, 0)):
         t = make_inputs(max(B, 1), max(S, 1), with_dout=True)
