@@ -19,13 +19,16 @@
 //                          the cached (fp16) value like every other key.
 //   decode_combine_kernel  CTA = (b, query head), thread = head dim: merges the splits,
 //                          applies the gate, writes out and lse.
-#include "tc_rows.cuh"
+#include "bwd_tc.cuh"  // warp_transpose_sum
 
 namespace zgcm {
 
 constexpr int DEC_THREADS = 128;        // 4 warps
-constexpr int DEC_KEYS = 512;           // keys per split
-constexpr int DEC_REC = 4 + kD;         // floats per split record: max, sum, 2 pad, O (16-byte aligned)
+constexpr int DEC_WARPS = DEC_THREADS / 32;
+constexpr int DEC_KEYS = 512;           // keys per split (CTA)
+constexpr int DEC_KB = 8;               // keys per batch
+constexpr int DEC_GH = 4;               // query heads per pass: DEC_GH x DEC_KB = 32 scores, one per lane
+constexpr int DEC_REC = 4 + kD;         // floats per partial record: max, sum, 2 pad, O (16-byte aligned)
 
 struct DecodeParams {
     LayerParams L;          // q, k, v, g: the new token ([B,Hq,D] / [B,Hkv,D]); S unused
@@ -34,16 +37,23 @@ struct DecodeParams {
     bf16* vc;               // [B,C,Hkv,D]
     int C;                  // cache slots per sequence
     int nsplit;             // splits of the visible keys (ceil(min(W, C) / DEC_KEYS))
-    float* part;            // [B*Hq*nsplit][DEC_REC]: max (base 2), sum, pad, O (relative to max)
+    float* part;            // [B*Hq][nsplit * DEC_WARPS][DEC_REC]: max (base 2), sum, pad, O (relative to max)
     bf16* out;              // [B,Hq,D]
     float* lse;             // [B,Hq]
 };
 
+// CTA = (b, KV head, split of DEC_KEYS visible keys).  The split's keys go to the 4 warps in
+// batches of 8 (batch i to warp i mod 4); a warp takes all the group's query heads (4 per
+// pass), so every cached row is loaded once per CTA.  Per batch, lane l holds the partial dot
+// products of its 4 head dims for the 4 x 8 (head, key) pairs; one transposed warp sum (31
+// shuffles) leaves the score of pair l = (head l/8, key l%8) in lane l; the heads' max and
+// sum run over their 8 lanes; the O update takes each pair's weight from its lane.  Each
+// warp writes its own partial record (max, sum, O) per head.
 __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const __grid_constant__ DecodeParams p) {
     const LayerParams& L = p.L;
     __shared__ __align__(16) float gq[kD];
     __shared__ __align__(16) float gk[kD];
-    __shared__ __align__(16) float ybuf[4][kD];  // prologue_row's per-warp scratch (float4 stores)
+    __shared__ __align__(16) float ybuf[DEC_WARPS][kD];  // prologue_row's per-warp scratch (float4 stores)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.x / L.Hkv, kvh = blockIdx.x % L.Hkv, s = blockIdx.y;
     gq[tid] = L.gamma_q[tid];
@@ -77,98 +87,112 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const __grid_
     __syncthreads();  // the new cache entry is read below like every other key
 
     const float c2 = L.scale_log2 / oscale;  // q~ (fp32) . (k~ oscale) -> base-2 score
-    for (int h = warp; h < L.G; h += DEC_THREADS / 32) {
-        const int hq = kvh * L.G + h;
-        float q4[4];
-        prologue_row(load_row4(L.q + ((size_t)b * L.Hq + hq) * kD), gq + 4 * lane, L, pos, ybuf[warp], q4);
-        float m = -INFINITY, l = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
-        if (fits) {
-            // eight keys per iteration: all their loads are issued before any is used (a key
-            // past the split's end loads the split's last key and is masked), and their dot
-            // products and butterfly sums are independent (every lane ends each sum with the
-            // same value, so m is warp-uniform).  The cache slot advances with j, wrapping at C.
-            constexpr int KB = 8;
-            const size_t head_off = (size_t)kvh * kD + 4 * lane;
-            const size_t seq_off = (size_t)b * p.C;
-            uint2 kw[KB], vw[KB];
-            // loads of the keys j .. j+KB-1 (slots from `slot`; keys past the split's end load
-            // its last key again, masked below)
-            auto load_batch = [&](int j, int slot) {
-                const int nk = min(KB, j1 - j);
+    const int nb = j1 > j0 ? (j1 - j0 + DEC_KB - 1) / DEC_KB : 0;
+    const int hl = lane >> 3, kl = lane & 7;      // the (head, key) pair of this lane's score
+    const size_t head_off = (size_t)kvh * kD + 4 * lane;
+    for (int hg0 = 0; hg0 < L.G; hg0 += DEC_GH) {
+        const int nh = min(DEC_GH, L.G - hg0);
+        float q[DEC_GH][4];
 #pragma unroll
-                for (int t = 0; t < KB; ++t) {
-                    int sl = slot + min(t, nk - 1);
-                    sl = sl >= p.C ? sl - p.C : sl;
-                    const size_t off = (seq_off + sl) * kv_row + head_off;
-                    kw[t] = *reinterpret_cast<const uint2*>(p.kc + off);
-                    vw[t] = *reinterpret_cast<const uint2*>(p.vc + off);
-                }
-            };
-            int slot = j0 % p.C;
-            if (j0 < j1) load_batch(j0, slot);
-            for (int j = j0; j < j1; j += KB) {
-                const int nk = min(KB, j1 - j);
-                float d[KB], vf[KB][4];
+        for (int h = 0; h < DEC_GH; ++h) {
+            if (h < nh) {
+                prologue_row(load_row4(L.q + ((size_t)b * L.Hq + kvh * L.G + hg0 + h) * kD), gq + 4 * lane, L, pos,
+                             ybuf[warp], q[h]);
+            } else {
+                q[h][0] = q[h][1] = q[h][2] = q[h][3] = 0.f;
+            }
+        }
+        float m[DEC_GH], l[DEC_GH], o[DEC_GH][4];
 #pragma unroll
-                for (int t = 0; t < KB; ++t) {
-                    const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kw[t].x));
-                    const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kw[t].y));
-                    d[t] = q4[0] * k01.x + q4[1] * k01.y + q4[2] * k23.x + q4[3] * k23.y;
-                    const float2 v01 = unpack_bf16(vw[t].x), v23 = unpack_bf16(vw[t].y);
-                    vf[t][0] = v01.x; vf[t][1] = v01.y; vf[t][2] = v23.x; vf[t][3] = v23.y;
-                }
-                // the next batch's loads go out while this one is reduced
-                slot += KB;
-                slot = slot >= p.C ? slot - p.C : slot;
-                if (j + KB < j1) load_batch(j + KB, slot);
+        for (int h = 0; h < DEC_GH; ++h) {
+            m[h] = fits ? -INFINITY : NAN;   // a window longer than the cache: no valid answer
+            l[h] = fits ? 0.f : NAN;
+            o[h][0] = o[h][1] = o[h][2] = o[h][3] = 0.f;
+        }
+        for (int bi = warp; fits && bi < nb; bi += DEC_WARPS) {
+            const int jb = j0 + bi * DEC_KB, nk = min(DEC_KB, j1 - jb);
+            uint2 kw[DEC_KB], vw[DEC_KB];
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
+            for (int t = 0; t < DEC_KB; ++t) {  // keys past the split's end load its last key (masked)
+                const size_t off = ((size_t)b * p.C + (jb + min(t, nk - 1)) % p.C) * kv_row + head_off;
+                kw[t] = *reinterpret_cast<const uint2*>(p.kc + off);
+                vw[t] = *reinterpret_cast<const uint2*>(p.vc + off);
+            }
+            float v[DEC_GH * DEC_KB];  // partial dots, index h * DEC_KB + key
 #pragma unroll
-                    for (int t = 0; t < KB; ++t) d[t] += __shfl_xor_sync(0xffffffffu, d[t], off);
-                }
-                float mn = m;
+            for (int t = 0; t < DEC_KB; ++t) {
+                const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&kw[t].x));
+                const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&kw[t].y));
 #pragma unroll
-                for (int t = 0; t < KB; ++t) {
-                    d[t] = t < nk ? d[t] * c2 : -INFINITY;
-                    mn = fmaxf(mn, d[t]);
-                }
-                if (mn > m) {
-                    const float a = fast_exp2(m - mn);  // 0 from the empty start
-                    l *= a;
+                for (int h = 0; h < DEC_GH; ++h)
+                    v[h * DEC_KB + t] = q[h][0] * k01.x + q[h][1] * k01.y + q[h][2] * k23.x + q[h][3] * k23.y;
+            }
+            const float tot = warp_transpose_sum(v);
+            const float sc = (kl < nk && hl < nh) ? tot * c2 : -INFINITY;
+            // each head's batch maximum over its 8 lanes, then every lane learns all four
+            float gm = sc;
+            gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, 4));
+            gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, 2));
+            gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, 1));
+            float mn[DEC_GH];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) o[e] *= a;
-                    m = mn;
-                }
+            for (int h = 0; h < DEC_GH; ++h) {
+                mn[h] = fmaxf(m[h], __shfl_sync(0xffffffffu, gm, 8 * h));
+                if (mn[h] > m[h]) {   // the same decision on every lane
+                    const float a = fast_exp2(m[h] - mn[h]);  // 0 from the empty start
+                    l[h] *= a;
 #pragma unroll
-                for (int t = 0; t < KB; ++t) {
-                    const float pj = fast_exp2(d[t] - m);   // 0 for the padding keys
-                    l += pj;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) o[e] = fmaf(pj, vf[t][e], o[e]);
+                    for (int e = 0; e < 4; ++e) o[h][e] *= a;
+                    m[h] = mn[h];
                 }
             }
-        } else {
-            m = l = NAN;  // a window longer than the cache: no valid answer
+            const float mh = hl == 0 ? mn[0] : hl == 1 ? mn[1] : hl == 2 ? mn[2] : mn[3];
+            const float pl = sc == -INFINITY ? 0.f : fast_exp2(sc - mh);
+            float gs = pl;
+            gs += __shfl_xor_sync(0xffffffffu, gs, 4);
+            gs += __shfl_xor_sync(0xffffffffu, gs, 2);
+            gs += __shfl_xor_sync(0xffffffffu, gs, 1);
+#pragma unroll
+            for (int h = 0; h < DEC_GH; ++h) l[h] += __shfl_sync(0xffffffffu, gs, 8 * h);
+#pragma unroll
+            for (int t = 0; t < DEC_KB; ++t) {
+                const float2 v01 = unpack_bf16(vw[t].x), v23 = unpack_bf16(vw[t].y);
+#pragma unroll
+                for (int h = 0; h < DEC_GH; ++h) {
+                    const float ph = __shfl_sync(0xffffffffu, pl, 8 * h + t);
+                    o[h][0] = fmaf(ph, v01.x, o[h][0]);
+                    o[h][1] = fmaf(ph, v01.y, o[h][1]);
+                    o[h][2] = fmaf(ph, v23.x, o[h][2]);
+                    o[h][3] = fmaf(ph, v23.y, o[h][3]);
+                }
+            }
         }
-        float* part = p.part + (((size_t)b * L.Hq + hq) * p.nsplit + s) * DEC_REC;
-        if (lane == 0) *reinterpret_cast<float4*>(part) = make_float4(m, l, 0.f, 0.f);
-        *reinterpret_cast<float4*>(part + 4 + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
+        const int nrec = p.nsplit * DEC_WARPS;
+#pragma unroll
+        for (int h = 0; h < DEC_GH; ++h) {
+            if (h >= nh) break;
+            const int hq = kvh * L.G + hg0 + h;
+            float* part = p.part + (((size_t)b * L.Hq + hq) * nrec + s * DEC_WARPS + warp) * DEC_REC;
+            if (lane == 0) *reinterpret_cast<float4*>(part) = make_float4(m[h], l[h], 0.f, 0.f);
+            *reinterpret_cast<float4*>(part + 4 + 4 * lane) = make_float4(o[h][0], o[h][1], o[h][2], o[h][3]);
+        }
     }
 }
 
 __global__ void __launch_bounds__(kD) decode_combine_kernel(const __grid_constant__ DecodeParams p) {
     const LayerParams& L = p.L;
     const int d = threadIdx.x, bh = blockIdx.x;
-    const float* part = p.part + (size_t)bh * p.nsplit * DEC_REC;
+    const int nrec = p.nsplit * DEC_WARPS;
+    const float* part = p.part + (size_t)bh * nrec * DEC_REC;
     float m = -INFINITY;
     bool bad = false;  // a split marked the window as longer than the cache
-    for (int s = 0; s < p.nsplit; ++s) {
+    for (int s = 0; s < nrec; ++s) {
         const float ms = part[s * DEC_REC];
         bad |= isnan(ms);
         m = fmaxf(m, ms);
     }
     float l = 0.f, o = 0.f;
-    for (int s = 0; s < p.nsplit; ++s) {
+    for (int s = 0; s < nrec; ++s) {
         const float* ps = part + s * DEC_REC;
         if (ps[0] == -INFINITY) continue;   // a split past the last key: empty
         const float a = exp2f(ps[0] - m);
@@ -185,7 +209,7 @@ __global__ void __launch_bounds__(kD) decode_combine_kernel(const __grid_constan
 size_t decode_workspace_bytes(int B, int Hq, int window, int C) {
     const int vis = window < C ? window : C;
     const size_t nsplit = (size_t)((vis + DEC_KEYS - 1) / DEC_KEYS);
-    return (size_t)B * Hq * nsplit * DEC_REC * sizeof(float);
+    return (size_t)B * Hq * nsplit * DEC_WARPS * DEC_REC * sizeof(float);
 }
 
 cudaError_t launch_decode(const LayerParams& L, const int* pos, void* k_cache, void* v_cache, int C, void* out,

@@ -158,10 +158,11 @@ def _dec(lib, ws_bytes, ptrs=None, ws=P + 256 * 40, **kw):
 
 def test_decode_checks(lib):
     need = lib.zgcm_attn_decode_workspace_size(1, 32, 128, 128)
-    # one split of up to 512 keys per (sequence, head): max, sum, 2 pad and 128 partial outputs
-    assert need == 1 * 32 * 1 * (4 + 128) * 4
-    assert lib.zgcm_attn_decode_workspace_size(2, 32, 10**6, 65536) == 2 * 32 * 128 * 132 * 4
-    assert lib.zgcm_attn_decode_workspace_size(2, 32, 300, 65536) == 2 * 32 * 1 * 132 * 4
+    # per (sequence, head): 4 records (one per warp) per split of up to 512 keys, each max, sum,
+    # 2 pad and 128 partial outputs
+    assert need == 1 * 32 * 1 * 4 * (4 + 128) * 4
+    assert lib.zgcm_attn_decode_workspace_size(2, 32, 10**6, 65536) == 2 * 32 * 128 * 4 * 132 * 4
+    assert lib.zgcm_attn_decode_workspace_size(2, 32, 300, 65536) == 2 * 32 * 1 * 4 * 132 * 4
     assert lib.zgcm_attn_decode_workspace_size(0, 32, 128, 128) == 0
     assert _dec(lib, need - 1) == -4
     assert _dec(lib, need, ws=0) == -4
