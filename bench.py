@@ -16,6 +16,7 @@ only; a bounded sample of the same workload per step).
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -444,18 +445,56 @@ def decode_cpu_baseline(P, layers):
             "sample": "; ".join(parts) + " (the oracle's per-row forward, fp64, including its prologue)"}
 
 
+def run_probe_ex2(args):
+    """The MUFU exp2 rate of this GPU (the softmax kernels' exponential), at full occupancy
+    and with one warp per SM sub-partition; prints one JSON line."""
+    import torch
+    import global_attention_b200 as ga
+    lib = ga.load()
+    dev = torch.device("cuda", 0)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    stream = torch.cuda.current_stream()
+    res = {}
+    for name, blocks, threads in (("full", sms * 8, 256), ("one_warp_per_smsp", sms, 128)):
+        iters = 4096
+        out = torch.empty(blocks * threads, dtype=torch.float32, device=dev)
+        call = lambda: lib.zgcm_attn_probe_ex2(ctypes.c_void_p(out.data_ptr()), blocks, threads, iters,
+                                               ctypes.c_void_p(stream.cuda_stream))
+        for _ in range(3):
+            assert call() == 0
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) as clk:
+            e0.record(stream)
+            for _ in range(args.steps):
+                assert call() == 0
+            e1.record(stream)
+            torch.cuda.synchronize()
+        secs = e0.elapsed_time(e1) / 1e3 / args.steps
+        n = blocks * threads * iters * 8
+        c = clk.summary()
+        mhz = c["sm_mhz"] or c["sm_max_mhz"] or 1965.0
+        res[name] = {"ex2_per_s": n / secs, "ex2_per_clock_per_sm": n / secs / (sms * mhz * 1e6),
+                     "ms": secs * 1e3, "sm_mhz": mhz}
+    print(json.dumps({"probe": "MUFU ex2.approx.ftz.f32 rate", "sms": sms, **res}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS), default="swa16k")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + ["probe_ex2"],
+                    default="swa16k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=8)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload == "probe_ex2":
+        return run_probe_ex2(args)
     if args.workload in DECODE_WORKLOADS:
         if args.impl == "reference":
             _, rank, _ = rank_env()

@@ -64,6 +64,8 @@ def load() -> ctypes.CDLL:
         lib.zgcm_attn_bwd_kernel_name.restype = ctypes.c_char_p
         lib.zgcm_attn_fwd_kernel_name.argtypes = [i, i, i, i, i, i]
         lib.zgcm_attn_fwd_kernel_name.restype = ctypes.c_char_p
+        lib.zgcm_attn_probe_ex2.argtypes = [vp, i, i, i, vp]
+        lib.zgcm_attn_probe_ex2.restype = i
         lib.zgcm_attn_selftest_expired_wait.argtypes = [vp]
         lib.zgcm_attn_selftest_expired_wait.restype = i
         lib.zgcm_attn_device_error.argtypes = []

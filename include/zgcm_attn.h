@@ -248,6 +248,14 @@ int zgcm_attn_device_error(void);
  */
 int zgcm_attn_selftest_expired_wait(void* cuda_stream);
 
+/*
+ * Diagnostic: runs blocks x threads threads of `iters` rounds of 8 independent exp2 chains
+ * (the MUFU instruction of the softmax kernels), 8 * iters exponentials per thread, and
+ * writes one float per thread to `out` (device, blocks * threads floats).  Timed by the
+ * caller, it measures the exponential rate the softmax kernels are budgeted against.
+ */
+int zgcm_attn_probe_ex2(float* out, int blocks, int threads, int iters, void* cuda_stream);
+
 /* Name of the i-th kernel zgcm_attn_bwd launches for this configuration (static string),
  * or NULL when i is past the last one.  With 42 rotated dims, windows up to 128 run the
  * gate pass, the K/V and Q preparation and the tcgen05 pair (bwd_gate_kernel,
