@@ -65,6 +65,7 @@ struct FwdTcSmem {
     float2 cs[TF_HALF][TF_BM];   // (cos, sin) of pair t at row r's position; thread r's column
     float gq[kD], gk[kD];
     float rowinv[2][TF_BM];
+    float mref;   // bound on |scores| in exp2 units: the softmax's reference when small enough
     uint64_t bar[B_COUNT];
     uint32_t tmem_base;
     int abort;
@@ -110,6 +111,23 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
     if (warp == 1) {
         tmem_alloc(&sm.tmem_base, 512);
         tmem_relinquish();
+    }
+    if (warp == 3) {
+        // Reference of the exponentials: a bound on every score rather than each row's maximum,
+        // which saves a pass over the scores.  An RMS-normalised row has norm at most sqrt(D)
+        // before gamma, and the rotation keeps norms, so |q~.k~| <= D max|gamma_q| max|gamma_k|;
+        // with that as the reference no weight exceeds 1 and none falls below 2^(-2 mref).  Where
+        // the bound is above 60 (far from fp32 / bf16 underflow) the rows take their maximum.
+        float amax_q = 0.f, amax_k = 0.f;
+        for (int d = lane; d < kD; d += 32) {
+            amax_q = fmaxf(amax_q, fabsf(L.gamma_q[d]));
+            amax_k = fmaxf(amax_k, fabsf(L.gamma_k[d]));
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+            amax_q = fmaxf(amax_q, __shfl_xor_sync(0xffffffffu, amax_q, o));
+            amax_k = fmaxf(amax_k, __shfl_xor_sync(0xffffffffu, amax_k, o));
+        }
+        if (lane == 0) sm.mref = fabsf(L.scale_log2) * (float)kD * amax_q * amax_k * 1.001f + 0.25f;
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&p.tm_q);
@@ -257,25 +275,28 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
                 auto chunk_full = [&](int kp0) {
                     return kp0 + 31 <= imin && kp0 > imax - L.W && kp0 >= 0 && kp0 + 31 < L.S;
                 };
-                float mx = -INFINITY;
+                float mu = sm.mref;
+                if (!(mu <= 60.f)) {
+                    float mx = -INFINITY;
 #pragma unroll 1
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    const int kp0 = (c8 < 4 ? base0 : base1) + (c8 & 3) * 32;
-                    const bool live = imin < L.S && kp0 <= imax && kp0 + 31 > imin - L.W && kp0 + 31 >= 0 && kp0 < L.S;
-                    if (!live) continue;
-                    float v[32];
-                    tmem_ld32f(TM_S + lane_off + 32 * c8, v);
-                    tmem_wait_ld();
-                    if (chunk_full(kp0)) {
+                    for (int c8 = 0; c8 < 8; ++c8) {
+                        const int kp0 = (c8 < 4 ? base0 : base1) + (c8 & 3) * 32;
+                        const bool live = imin < L.S && kp0 <= imax && kp0 + 31 > imin - L.W && kp0 + 31 >= 0 && kp0 < L.S;
+                        if (!live) continue;
+                        float v[32];
+                        tmem_ld32f(TM_S + lane_off + 32 * c8, v);
+                        tmem_wait_ld();
+                        if (chunk_full(kp0)) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
-                    } else {
-                        const uint32_t vm = bit_range(klo - kp0, khi - kp0);
+                            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
+                        } else {
+                            const uint32_t vm = bit_range(klo - kp0, khi - kp0);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, ((vm >> e) & 1u) ? v[e] : -INFINITY);
+                            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, ((vm >> e) & 1u) ? v[e] : -INFINITY);
+                        }
                     }
+                    mu = (mx == -INFINITY) ? 0.f : mx * c2;
                 }
-                const float mu = (mx == -INFINITY) ? 0.f : mx * c2;
                 float l = 0.f;
 #pragma unroll 1
                 for (int c8 = 0; c8 < 8; ++c8) {

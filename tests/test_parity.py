@@ -98,6 +98,32 @@ def test_forward_both_kernel_paths(B, S, W, monkeypatch):
         assert_lse_close(f"lse[{name}]", l, ref_lse)
 
 
+@pytest.mark.parametrize("gq_all,spike,B,S,W", [
+    (1.0, 20.0, 1, 1000, 128),     # two large gamma_q entries: bound far above the limit
+    (1.9, None, 2, 700, 128),      # gamma 1.9 everywhere: bound just under the limit (59.2)
+    (2.0, None, 1, 333, 37),       # gamma 2.0 everywhere: just over it (65.6)
+])
+def test_forward_score_bound_fallback(gq_all, spike, B, S, W, monkeypatch):
+    """The sliding-window forward takes its exponentials' reference from a bound on every
+    score, |scale| log2(e) D max|gamma_q| max|gamma_k|, when that bound is at most 60, and
+    from each row's maximum otherwise.  Both sides of the limit, and a bound far above it,
+    match the oracle."""
+    t = make_inputs(B, S, seed=500 + S + W)
+    gq = torch.full((128,), gq_all, dtype=torch.float32)
+    if spike is not None:
+        gq[:2] = spike
+    t["gamma_q"] = gq
+    t["gamma_k"] = torch.full((128,), gq_all, dtype=torch.float32)
+    d = _to_dev(t)
+    ref_out, ref_lse = _problem(t, window=W).forward()
+    monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
+    assert ga.zgcm_attn_fwd_kernel_name(B, S, 32, 8, 42, W) == "fwd_tc_kernel"
+    out, lse = _gpu_fwd(d, window=W)
+    assert ga.zgcm_attn_device_error() == 0
+    assert_bf16_close("out", out, ref_out)
+    assert_lse_close("lse", lse, ref_lse)
+
+
 @pytest.mark.parametrize("B,S,W", [(1, 777, 777), (2, 1000, 10**6), (1, 129, 129), (1, 1, 4096),
                                    (3, 260, 200), (1, 1300, 300), (2, 640, 129), (1, 2048, 2048)])
 def test_forward_wide_window_kernel(B, S, W, monkeypatch):
