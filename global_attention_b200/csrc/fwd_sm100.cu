@@ -303,11 +303,31 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
                     const int kp0 = (c8 < 4 ? base0 : base1) + (c8 & 3) * 32;
                     const bool live = imin < L.S && kp0 <= imax && kp0 + 31 > imin - L.W && kp0 + 31 >= 0 && kp0 < L.S;
                     uint32_t pk[16];
-                    if (live) {
+                    if (live && chunk_full(kp0)) {
+                        // every key visible to the warp's rows: no mask, scores two at a time
                         float v[32];
                         tmem_ld32f(TM_S + lane_off + 32 * c8, v);
                         tmem_wait_ld();
-                        const uint32_t vm = chunk_full(kp0) ? 0xffffffffu : bit_range(klo - kp0, khi - kp0);
+                        const float2 cc = make_float2(c2, c2), nm = make_float2(-mu, -mu);
+                        float2 la = make_float2(0.f, 0.f), lb = la;
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            const float2 xa = ffma2(make_float2(v[e], v[e + 1]), cc, nm);
+                            const float2 xb = ffma2(make_float2(v[e + 2], v[e + 3]), cc, nm);
+                            const float2 pa = make_float2(fast_exp2(xa.x), fast_exp2(xa.y));
+                            const float2 pb = make_float2(fast_exp2(xb.x), fast_exp2(xb.y));
+                            la = fadd2(la, pa);
+                            lb = fadd2(lb, pb);
+                            pk[e >> 1] = pack_bf16(pa.x, pa.y);
+                            pk[(e >> 1) + 1] = pack_bf16(pb.x, pb.y);
+                        }
+                        la = fadd2(la, lb);
+                        l += la.x + la.y;
+                    } else if (live) {
+                        float v[32];
+                        tmem_ld32f(TM_S + lane_off + 32 * c8, v);
+                        tmem_wait_ld();
+                        const uint32_t vm = bit_range(klo - kp0, khi - kp0);
 #pragma unroll
                         for (int e = 0; e < 32; e += 2) {
                             float p0 = fast_exp2(v[e] * c2 - mu), p1 = fast_exp2(v[e + 1] * c2 - mu);
@@ -372,7 +392,8 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
                 }
                 if (!(ok = mbar_wait(&sm.bar[B_OFULL + buf], (e >> 1) & 1, abort, 30))) break;
                 if (!(ok = mbar_wait(&sm.bar[B_LFULL + buf], (e >> 1) & 1, abort, 31))) break;
-                const float inv = sm.rowinv[buf][r];
+                const float hi = 0.5f * sm.rowinv[buf][r];
+                const float2 hinv = make_float2(hi, hi);
                 mbar_arrive(&sm.bar[B_LEMPTY + buf]);
                 tc_fence_after();
 #pragma unroll
@@ -388,13 +409,13 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
                             uint32_t ow[4];
 #pragma unroll
                             for (int e2 = 0; e2 < 4; ++e2) {
-                                const float2 gf = unpack_bf16(gw[e2]);
-                                // sigmoid(x) = 0.5 + 0.5 tanh(x / 2)
-                                const float s0 = fmaf(0.5f, fast_tanh(0.5f * gf.x), 0.5f);
-                                const float s1 = fmaf(0.5f, fast_tanh(0.5f * gf.y), 0.5f);
+                                // sigmoid(x) / l = (0.5 + 0.5 tanh(x / 2)) / l, two columns at a time
+                                const float2 hg = fmul2(unpack_bf16(gw[e2]), make_float2(0.5f, 0.5f));
+                                const float2 th = make_float2(fast_tanh(hg.x), fast_tanh(hg.y));
+                                const float2 sg = ffma2(th, hinv, hinv);
                                 const int col = 8 * q4 + 2 * e2;
-                                ow[e2] = pack_bf16(s0 * (__uint_as_float(v[col]) * inv),
-                                                   s1 * (__uint_as_float(v[col + 1]) * inv));
+                                const float2 o = fmul2(make_float2(__uint_as_float(v[col]), __uint_as_float(v[col + 1])), sg);
+                                ow[e2] = pack_bf16(o.x, o.y);
                             }
                             *reinterpret_cast<uint4*>(p.out + off + 32 * c + 8 * q4) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                         }
