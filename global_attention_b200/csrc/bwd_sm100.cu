@@ -164,29 +164,38 @@ template <bool FULL>
 __device__ __forceinline__ void kv_chunk(const float* sv, const float* dv, const float* lse2c, const float* deltac,
                                          const float* dcolc, uint32_t vm, float vin, float su, float dsc, float c2,
                                          uint32_t (&pp)[16], uint32_t (&dd)[16], float& kacc) {
+    // two query columns per paired fp32 instruction
+    const float2 cc = make_float2(c2, c2), vin2 = make_float2(vin, vin), su2 = make_float2(su, su),
+                 dsc2 = make_float2(dsc, dsc);
+    float2 kacc2 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int e4 = 0; e4 < 8; ++e4) {
         const float4 ls = *reinterpret_cast<const float4*>(lse2c + 4 * e4);
         const float4 dl = *reinterpret_cast<const float4*>(deltac + 4 * e4);
         const float4 dc = *reinterpret_cast<const float4*>(dcolc + 4 * e4);
-        const float lsv[4] = {ls.x, ls.y, ls.z, ls.w}, dlv[4] = {dl.x, dl.y, dl.z, dl.w}, dcv[4] = {dc.x, dc.y, dc.z, dc.w};
-        float p4[4], d4[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = 4 * e4 + u;
-            float pv = fast_exp2(fmaf(sv[e], c2, -lsv[u]));
-            if (!FULL) pv = ((vm >> e) & 1u) ? pv : 0.f;  // (columns past the sequence: masked)
-            const float dp = dv[e] * vin * dcv[u];
-            const float d = pv * (dp - dlv[u]);
-            kacc = fmaf(d, sv[e], kacc);
-            p4[u] = pv * (dcv[u] * su);
-            d4[u] = d * dsc;
+        for (int hf = 0; hf < 2; ++hf) {
+            const int e = 4 * e4 + 2 * hf;
+            const float2 lsp = hf ? make_float2(ls.z, ls.w) : make_float2(ls.x, ls.y);
+            const float2 dlp = hf ? make_float2(dl.z, dl.w) : make_float2(dl.x, dl.y);
+            const float2 dcp = hf ? make_float2(dc.z, dc.w) : make_float2(dc.x, dc.y);
+            const float2 s = make_float2(sv[e], sv[e + 1]);
+            const float2 x = fsub2(fmul2(s, cc), lsp);
+            float2 pv = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            if (!FULL) {  // (columns past the sequence: masked)
+                pv.x = ((vm >> e) & 1u) ? pv.x : 0.f;
+                pv.y = ((vm >> (e + 1)) & 1u) ? pv.y : 0.f;
+            }
+            const float2 dp = fmul2(fmul2(make_float2(dv[e], dv[e + 1]), vin2), dcp);
+            const float2 d = fmul2(pv, fsub2(dp, dlp));
+            kacc2 = ffma2(d, s, kacc2);
+            const float2 p2 = fmul2(pv, fmul2(dcp, su2));
+            const float2 d2 = fmul2(d, dsc2);
+            pp[2 * e4 + hf] = pack2<true>(p2.x, p2.y);
+            dd[2 * e4 + hf] = pack2<true>(d2.x, d2.y);
         }
-        pp[2 * e4] = pack2<true>(p4[0], p4[1]);
-        pp[2 * e4 + 1] = pack2<true>(p4[2], p4[3]);
-        dd[2 * e4] = pack2<true>(d4[0], d4[1]);
-        dd[2 * e4 + 1] = pack2<true>(d4[2], d4[3]);
     }
+    kacc += kacc2.x + kacc2.y;
 }
 
 // =====================================================================  query-major kernel
@@ -626,9 +635,13 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                         tmem_wait_ld();
                         // pd holds P dv: dS dsc = P dv (kd dsc) - P (Delta dsc)
                         const float ka = (c8 < 4 ? kd0 : kd1) * dsc, kb = -delta * dsc;
+                        const float2 ka2 = make_float2(ka, ka), kb2 = make_float2(kb, kb);
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2)
-                            pk[e >> 1] = pack2<true>(fmaf(pd[e], ka, pv[e] * kb), fmaf(pd[e + 1], ka, pv[e + 1] * kb));
+                        for (int e = 0; e < 32; e += 2) {
+                            const float2 t = ffma2(make_float2(pd[e], pd[e + 1]), ka2,
+                                                   fmul2(make_float2(pv[e], pv[e + 1]), kb2));
+                            pk[e >> 1] = pack2<true>(t.x, t.y);
+                        }
                     } else {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) pk[e] = 0u;
