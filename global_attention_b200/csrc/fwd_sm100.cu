@@ -198,8 +198,10 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
             constexpr uint32_t IDESC_S = idesc_f16(128, 256, false);
             constexpr uint32_t IDESC_O = idesc_bf16(128, 128, true);
             const uint32_t q_base = smem_u32(sm.Q[0][0]);
-            const uint32_t k_base = smem_u32(sm.K[0]);
-            const uint32_t v_base = smem_u32(sm.V[0]);
+            // descriptors of each operand's first 16-element step; the others are offsets
+            const uint64_t q_desc0 = sdesc_sw128(q_base, 16, 1024);
+            const uint64_t k_desc0 = sdesc_sw128(smem_u32(sm.K[0]), 16, 1024);
+            const uint64_t v_desc0 = sdesc_sw128(smem_u32(sm.V[0]), TF_RING_HALF, 1024);
             int n_next = 0, n_prev = 0, n_cur = 0, m = 0;
             bool ok = true;
             for (int t = t_begin; t < t_end && ok; ++t) {
@@ -223,8 +225,8 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t half = kk >> 2, within = (kk & 3) * 32;
-                        const uint64_t a = sdesc_sw128(q_base + buf * 2 * TF_HALF_BYTES + half * TF_HALF_BYTES + within, 16, 1024);
-                        const uint64_t bdesc = sdesc_sw128(k_base + half * TF_RING_HALF + within, 16, 1024);
+                        const uint64_t a = sdesc_step(q_desc0, buf * 2 * TF_HALF_BYTES + half * TF_HALF_BYTES + within);
+                        const uint64_t bdesc = sdesc_step(k_desc0, half * TF_RING_HALF + within);
                         mma_ss(TM_S, a, bdesc, IDESC_S, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(&sm.bar[B_QEMPTY + buf]);
@@ -239,7 +241,7 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
                     // O = P V: P bf16 in TMEM (16 keys = 8 columns per step), V MN-major
 #pragma unroll
                     for (int kk = 0; kk < 16; ++kk) {
-                        const uint64_t bdesc = sdesc_sw128(v_base + kk * 16 * 128, TF_RING_HALF, 1024);
+                        const uint64_t bdesc = sdesc_step(v_desc0, kk * 16 * 128);
                         mma_ts(TM_O0 + buf * 128, TM_P + kk * 8, bdesc, IDESC_O, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(&sm.bar[B_OFULL + buf]);

@@ -261,6 +261,16 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo
     return d;
 }
 
+// The descriptor of an address `bytes` further on: the address field is (address >> 4) in the
+// low 14 bits and a CTA's shared memory (< 228 KB) keeps it below 2^14, so the step never
+// carries out of the field and is one 32-bit add on the low word.
+__device__ __forceinline__ uint64_t sdesc_step(uint64_t d, uint32_t bytes) {
+    const uint32_t lo = (uint32_t)d + (bytes >> 4), hi = (uint32_t)(d >> 32);
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+
 // Instruction descriptor for kind::f16: bf16 A and B, fp32 D, dense, no negation.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
     return (1u << 4)                      // D format: f32
