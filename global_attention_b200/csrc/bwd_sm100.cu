@@ -913,8 +913,13 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             if (lane == 0) {
                 constexpr uint32_t IDESC_S = idesc_f16(128, 64, false);
                 constexpr uint32_t IDESC_MN = idesc_f16(128, 128, true);
-                const uint32_t k_base = smem_u32(sm.K[0]), v_base = smem_u32(sm.V[0]);
-                const uint32_t q_base = smem_u32(sm.Q[0][0]), da_base = smem_u32(sm.dA[0][0]);
+                // descriptors of each operand's first step; the others are offsets from them
+                const uint64_t k_d = sdesc_sw128(smem_u32(sm.K[0]), 16, 1024);
+                const uint64_t v_d = sdesc_sw128(smem_u32(sm.V[0]), 16, 1024);
+                const uint64_t q_d = sdesc_sw128(smem_u32(sm.Q[0][0]), 16, 1024);
+                const uint64_t da_d = sdesc_sw128(smem_u32(sm.dA[0][0]), 16, 1024);
+                const uint64_t q_mn = sdesc_sw128(smem_u32(sm.Q[0][0]), KV_SLOT_HALF, 1024);
+                const uint64_t da_mn = sdesc_sw128(smem_u32(sm.dA[0][0]), KV_SLOT_HALF, 1024);
                 struct Cursor {
                     int u, uu, it, it_all, half;
                     UnitInfo x;
@@ -942,19 +947,18 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                     if (!mbar_wait(&sm.bar[KB_QFULL + slot], (hs / KV_SLOTS) & 1, abort, 211)) return false;
                     tc_fence_after();
                     const uint32_t tX = tmem + 128u * (uint32_t)c.half;
-                    const uint32_t qa = q_base + (uint32_t)slot * 2u * KV_SLOT_HALF;
-                    const uint32_t da = da_base + (uint32_t)slot * 2u * KV_SLOT_HALF;
+                    const uint32_t so = (uint32_t)slot * 2u * KV_SLOT_HALF;
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t dh = kk >> 2, within = (kk & 3) * 32;
-                        mma_ss(tX, sdesc_sw128(k_base + dh * TF_HALF_BYTES + within, 16, 1024),
-                               sdesc_sw128(qa + dh * KV_SLOT_HALF + within, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+                        mma_ss(tX, sdesc_step(k_d, dh * TF_HALF_BYTES + within),
+                               sdesc_step(q_d, so + dh * KV_SLOT_HALF + within), IDESC_S, kk > 0 ? 1u : 0u);
                     }
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t dh = kk >> 2, within = (kk & 3) * 32;
-                        mma_ss(tX + 64, sdesc_sw128(v_base + dh * TF_HALF_BYTES + within, 16, 1024),
-                               sdesc_sw128(da + dh * KV_SLOT_HALF + within, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+                        mma_ss(tX + 64, sdesc_step(v_d, dh * TF_HALF_BYTES + within),
+                               sdesc_step(da_d, so + dh * KV_SLOT_HALF + within), IDESC_S, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(&sm.bar[KB_SFULL + c.half]);
                     if (last_of_unit(c)) mma_commit(&sm.bar[KB_KVEMPTY]);  // K, V read for the last time
@@ -968,17 +972,16 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                         return false;
                     tc_fence_after();
                     const uint32_t tX = tmem + 128u * (uint32_t)c.half;
-                    const uint32_t qa = q_base + (uint32_t)slot * 2u * KV_SLOT_HALF;
-                    const uint32_t da = da_base + (uint32_t)slot * 2u * KV_SLOT_HALF;
+                    const uint32_t so = (uint32_t)slot * 2u * KV_SLOT_HALF;
                     const bool first = c.it == 0 && c.half == 0;
                     // A from TMEM (16 queries = 8 columns per step); B = dA / Q~ MN-major (N = d)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(TM_DV, tX + kk * 8, sdesc_sw128(da + kk * 16 * 128, KV_SLOT_HALF, 1024), IDESC_MN,
+                        mma_ts(TM_DV, tX + kk * 8, sdesc_step(da_mn, so + kk * 16 * 128), IDESC_MN,
                                (!first || kk > 0) ? 1u : 0u);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(TM_DK, tX + 64 + kk * 8, sdesc_sw128(qa + kk * 16 * 128, KV_SLOT_HALF, 1024), IDESC_MN,
+                        mma_ts(TM_DK, tX + 64 + kk * 8, sdesc_step(q_mn, so + kk * 16 * 128), IDESC_MN,
                                (!first || kk > 0) ? 1u : 0u);
                     mma_commit(&sm.bar[KB_QEMPTY + slot]);  // the half's Q~ and dA rows were read for the last time
                     if (last_of_unit(c)) mma_commit(&sm.bar[KB_DVKFULL]);
