@@ -89,8 +89,9 @@ def pairs(S: int, W: int) -> int:
     return W * S - W * (W - 1) // 2
 
 
-def work(B, S, W, bwd):
-    """Masked FLOPs and algorithmic HBM bytes of one step (and of each dominant kernel)."""
+def work(B, S, W, bwd, saved=False):
+    """Masked FLOPs and algorithmic HBM bytes of one step (and of each dominant kernel).
+    `saved`: the forward keeps q~, k~ and the rows' inverse RMS for the backward."""
     npair = pairs(S, W) * B * HQ
     tok = B * S
     qb = tok * HQ * D * 2            # q, g, out, dout, dq, dg (bf16 [B,S,Hq,D])
@@ -102,11 +103,13 @@ def work(B, S, W, bwd):
     bwd_flops = 10 * D * npair
     # per kernel of this build: (algorithmic bytes = each input read once and each output
     # written once at its stored type, masked FLOPs of the products the kernel's job needs)
+    # a forward that keeps its activations also writes q~ fp16 and each q and k row's inverse RMS
+    keep = (qb + tok * HQ * 4 + tok * HKV * 4) if saved else 0
     kernels = {
         "fwd_mma_kernel": (fwd_bytes, fwd_flops),
-        "fwd_tc_kernel": (fwd_bytes, fwd_flops),
+        "fwd_tc_kernel": (fwd_bytes + keep, fwd_flops),
         # tcgen05 forwards: q, K~16 (fp16, prepared from k by fwd_prep_k_kernel), v, g -> out, lse
-        "fwd_glob_tc_kernel": (fwd_bytes, fwd_flops),
+        "fwd_glob_tc_kernel": (fwd_bytes + keep, fwd_flops),
         # dout, out, g -> dg, dA
         "bwd_pre_kernel": (5 * qb, 0),
         # q, k, v, dA, lse -> dq, Delta ; S, dP, dQ
@@ -120,6 +123,8 @@ def work(B, S, W, bwd):
         # k, v -> K~, V fp16 (+ per-row inverse RMS and v norm, per-tile V scale); q -> Q~ fp16
         "bwd_prep_kv_kernel": (4 * kb + kb // D, 0),
         "bwd_prep_q_kernel": (2 * qb + qb // (2 * D), 0),
+        # given the forward's q~, k~: v -> V fp16 (+ v norm per row, V scale per tile)
+        "bwd_prep_v_kernel": (2 * kb + kb // (D // 2), 0),
         "bwd_q_tc_kernel": (4 * qb + 2 * kb + 3 * lse, 6 * D * npair),
         "bwd_kv_tc_kernel": (2 * qb + 5 * kb + 4 * lse, 8 * D * npair),
     }
@@ -529,7 +534,9 @@ def main():
 
     Bw, Sw, W, bwd = WORKLOADS[args.workload]
     layers = layers_of(args.workload)
-    wks = [work(Bw, Sw, lw, bwd) for lw, _ in layers]
+    # a training step: the forward keeps q~, k~ and the rows' inverse RMS for its backward
+    keep = [bwd and ga.zgcm_attn_saved_size(Bw, Sw, HQ, HKV, D, 42, lw) > 0 for lw, _ in layers]
+    wks = [work(Bw, Sw, lw, bwd, kp) for (lw, _), kp in zip(layers, keep)]
     wk = {k: sum(x[k] for x in wks) for k in ("fwd_bytes", "fwd_flops", "bwd_bytes", "bwd_flops")}
     wk["tokens"] = Bw * Sw
     t = make_inputs(Bw, Sw, seed=rank_seed(rank), with_dout=bwd)
@@ -551,12 +558,15 @@ def main():
 
     # per layer: the forward's events, and one event pair per backward kernel
     ev_f = [[pair() for _ in layers] for _ in range(args.steps)]
-    bwd_names = [ga.zgcm_attn_bwd_kernel_names(Sw, lw) if bwd else [] for lw, _ in layers]
+    bwd_names = [ga.zgcm_attn_bwd_kernel_names(Sw, lw, saved=kp) if bwd else [] for (lw, _), kp in zip(layers, keep)]
     ev_m = [[[pair() for _ in names] for names in bwd_names] for _ in range(args.steps)]
 
     # forward scratch (normalised keys of the wide-window kernel), allocated once
     fws = [None if n == 0 else torch.empty(n, dtype=torch.uint8, device=dev)
            for n in (ga.zgcm_attn_fwd_workspace_size(Bw, Sw, HQ, HKV, D, 42, lw) for lw, _ in layers)]
+    # the activation store of each layer (in place of the forward's workspace), allocated once
+    svs = [torch.empty(ga.zgcm_attn_saved_size(Bw, Sw, HQ, HKV, D, 42, lw), dtype=torch.uint8, device=dev)
+           if kp else None for (lw, _), kp in zip(layers, keep)]
 
     def step(i=None, src=d, dst=None):
         o = dst or {"out": out, "lse": lse, "grads": grads}
@@ -564,13 +574,14 @@ def main():
             if i is not None:
                 ev_f[i][li][0].record(stream)
             ga.zgcm_attn_fwd(src["q"], src["k"], src["v"], src["g"], src["gamma_q"], src["gamma_k"],
-                             window=lw, out=o["out"], lse=o["lse"], workspace=fws[li], stream=stream)
+                             window=lw, out=o["out"], lse=o["lse"], workspace=fws[li], saved=svs[li],
+                             stream=stream)
             if i is not None:
                 ev_f[i][li][1].record(stream)
             if bwd:
                 ga.zgcm_attn_bwd(src["q"], src["k"], src["v"], src["g"], src["gamma_q"], src["gamma_k"],
                                  o["out"], o["lse"], src["dout"], window=lw, grads=o["grads"], workspace=ws,
-                                 stream=stream, kernel_events=None if i is None else ev_m[i][li])
+                                 saved=svs[li], stream=stream, kernel_events=None if i is None else ev_m[i][li])
 
     for _ in range(args.warmup):
         step()
@@ -703,9 +714,12 @@ def main():
                          "pair scaled to the workload's pairs per token"}
 
     # per layer: the forward's kernels (each tcgen05 forward runs the key preparation kernel
-    # first) + every backward kernel
-    fwd_launches = [1 if ga.zgcm_attn_fwd_kernel_name(Bw, Sw, HQ, HKV, 42, lw) == "fwd_mma_kernel" else 2
-                    for lw, _ in layers]
+    # first; the wide-window one, keeping its activations, also the query preparation) + every
+    # backward kernel
+    fwd_launches = []
+    for (lw, _), kp in zip(layers, keep):
+        fname = ga.zgcm_attn_fwd_kernel_name(Bw, Sw, HQ, HKV, 42, lw)
+        fwd_launches.append(1 if fname == "fwd_mma_kernel" else 3 if kp and fname == "fwd_glob_tc_kernel" else 2)
     launches_per_step = sum(f + len(n) for f, n in zip(fwd_launches, bwd_names))
     rec = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,

@@ -62,6 +62,15 @@ def load() -> ctypes.CDLL:
         lib.zgcm_attn_bwd_timed.restype = i
         lib.zgcm_attn_bwd_kernel_name.argtypes = [i, i, i, i]
         lib.zgcm_attn_bwd_kernel_name.restype = ctypes.c_char_p
+        lib.zgcm_attn_bwd_saved_kernel_name.argtypes = [i, i, i, i]
+        lib.zgcm_attn_bwd_saved_kernel_name.restype = ctypes.c_char_p
+        lib.zgcm_attn_saved_size.argtypes = [i, i, i, i, i, i, i]
+        lib.zgcm_attn_saved_size.restype = ctypes.c_size_t
+        lib.zgcm_attn_fwd_save.argtypes = lib.zgcm_attn_fwd_ws.argtypes
+        lib.zgcm_attn_fwd_save.restype = i
+        lib.zgcm_attn_bwd_saved.argtypes = (lib.zgcm_attn_bwd.argtypes[:-1] + [vp, ctypes.c_size_t, vp,
+                                                                               ctypes.POINTER(vp), i])
+        lib.zgcm_attn_bwd_saved.restype = i
         lib.zgcm_attn_fwd_kernel_name.argtypes = [i, i, i, i, i, i]
         lib.zgcm_attn_fwd_kernel_name.restype = ctypes.c_char_p
         lib.zgcm_attn_probe_ex2.argtypes = [vp, i, i, i, vp]
@@ -105,11 +114,20 @@ def zgcm_attn_fwd_workspace_size(B, S, Hq, Hkv, D=128, rope_dims=42, window=128)
                                                    int(window)))
 
 
+def zgcm_attn_saved_size(B, S, Hq, Hkv, D=128, rope_dims=42, window=128) -> int:
+    """Bytes of the activation store zgcm_attn_fwd(saved=...) fills for the backward (0 where
+    the pair does not apply)."""
+    return int(load().zgcm_attn_saved_size(int(B), int(S), int(Hq), int(Hkv), int(D), int(rope_dims),
+                                           int(window)))
+
+
 def zgcm_attn_fwd(q, k, v, g, gamma_q, gamma_k, *, rope_dims=42, rope_base=10000.0, window=128,
-                  causal=1, eps=1e-6, scale=None, out=None, lse=None, workspace=None, stream=None):
+                  causal=1, eps=1e-6, scale=None, out=None, lse=None, workspace=None, saved=None, stream=None):
     """Gated window-attention forward.  Returns (out bf16 [B,S,Hq,D], lse fp32 [B,Hq,S]).
     `workspace`: a uint8 device tensor of at least zgcm_attn_fwd_workspace_size bytes, or None
-    to allocate it here when the configuration needs one."""
+    to allocate it here when the configuration needs one.  `saved`: a uint8 device tensor of
+    zgcm_attn_saved_size bytes (zgcm_attn_fwd_save; then no workspace is used) that keeps the
+    activations zgcm_attn_bwd(saved=...) reads."""
     import torch
     for n, t in (("q", q), ("k", k), ("v", v), ("g", g)):
         _check(t, n, torch.bfloat16, 4)
@@ -123,6 +141,15 @@ def zgcm_attn_fwd(q, k, v, g, gamma_q, gamma_k, *, rope_dims=42, rope_base=10000
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    if saved is not None:
+        _check(saved, "saved", torch.uint8, 1)
+        st = load().zgcm_attn_fwd_save(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma_q), _ptr(gamma_k),
+                                       B, S, Hq, Hkv, D, int(rope_dims), float(rope_base), int(window),
+                                       int(causal), float(eps), float(scale), _ptr(out), _ptr(lse),
+                                       _ptr(saved), saved.numel(), _stream(stream))
+        if st != ZGCM_OK:
+            raise ZgcmError(st, "zgcm_attn_fwd_save")
+        return out, lse
     need = zgcm_attn_fwd_workspace_size(B, S, Hq, Hkv, D, rope_dims, window)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -195,11 +222,12 @@ def zgcm_attn_device_error() -> int:
     return int(load().zgcm_attn_device_error())
 
 
-def zgcm_attn_bwd_kernel_names(S, window, rope_dims=42):
-    """Names of the kernels zgcm_attn_bwd launches, in order."""
+def zgcm_attn_bwd_kernel_names(S, window, rope_dims=42, saved=False):
+    """Names of the kernels zgcm_attn_bwd launches (with `saved`: zgcm_attn_bwd_saved), in order."""
     names, i = [], 0
+    query = load().zgcm_attn_bwd_saved_kernel_name if saved else load().zgcm_attn_bwd_kernel_name
     while True:
-        n = load().zgcm_attn_bwd_kernel_name(i, int(S), int(rope_dims), int(window))
+        n = query(i, int(S), int(rope_dims), int(window))
         if n is None:
             return names
         names.append(n.decode())
@@ -207,13 +235,14 @@ def zgcm_attn_bwd_kernel_names(S, window, rope_dims=42):
 
 
 def zgcm_attn_bwd(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dims=42, rope_base=10000.0,
-                  window=128, causal=1, eps=1e-6, scale=None, grads=None, workspace=None, stream=None,
-                  kernel_events=None):
+                  window=128, causal=1, eps=1e-6, scale=None, grads=None, workspace=None, saved=None,
+                  stream=None, kernel_events=None):
     """Gated window-attention backward.  Returns dict dq, dk, dv, dg (bf16) and dgamma_q,
     dgamma_k (fp32 [D]).  `grads` may supply preallocated outputs, `workspace` a uint8
-    CUDA tensor of at least zgcm_attn_bwd_workspace_size(...) bytes.  `kernel_events`, a list
-    of (begin, end) torch.cuda.Event pairs, brackets the backward's kernels in launch order
-    (zgcm_attn_bwd_timed; names from zgcm_attn_bwd_kernel_names)."""
+    CUDA tensor of at least zgcm_attn_bwd_workspace_size(...) bytes.  `saved`: the store a
+    zgcm_attn_fwd(saved=...) of the same inputs filled (zgcm_attn_bwd_saved).  `kernel_events`,
+    a list of (begin, end) torch.cuda.Event pairs, brackets the backward's kernels in launch
+    order (zgcm_attn_bwd_timed; names from zgcm_attn_bwd_kernel_names)."""
     import torch
     B, S, Hq, D = q.shape
     Hkv = k.shape[2]
@@ -236,9 +265,8 @@ def zgcm_attn_bwd(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dims=42,
             _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]), _ptr(grads["dg"]),
             _ptr(grads["dgamma_q"]), _ptr(grads["dgamma_k"]), _ptr(workspace),
             workspace.numel(), _stream(stream))
-    if kernel_events is None:
-        st = load().zgcm_attn_bwd(*args)
-    else:
+    arr, n_pairs = None, 0
+    if kernel_events is not None:
         st_obj = stream if stream is not None else torch.cuda.current_stream()
         for pair in kernel_events:
             for e in pair:
@@ -246,7 +274,17 @@ def zgcm_attn_bwd(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dims=42,
                     e.record(st_obj)
         flat = [ctypes.c_void_p(e.cuda_event) for pair in kernel_events for e in pair]
         arr = (ctypes.c_void_p * max(1, len(flat)))(*flat)
-        st = load().zgcm_attn_bwd_timed(*args, arr, len(kernel_events))
+        n_pairs = len(kernel_events)
+    if saved is not None:
+        _check(saved, "saved", torch.uint8, 1)
+        st = load().zgcm_attn_bwd_saved(*args[:-1], _ptr(saved), saved.numel(), args[-1], arr, n_pairs)
+        if st != ZGCM_OK:
+            raise ZgcmError(st, "zgcm_attn_bwd_saved")
+        return grads
+    if kernel_events is None:
+        st = load().zgcm_attn_bwd(*args)
+    else:
+        st = load().zgcm_attn_bwd_timed(*args, arr, n_pairs)
     if st != ZGCM_OK:
         raise ZgcmError(st, "zgcm_attn_bwd")
     return grads

@@ -285,7 +285,8 @@ struct PrepSmem {
 // angles sit in registers here).  Also saved: each row's inverse RMS (RMSNorm backward of dq,
 // dk), the raw norm of each v row (dS^T scale) and the V tile scale.  Several CTAs per SM keep
 // tile loads, conversions and stores of different tiles in flight.
-template <bool IS_K>
+// WITH_K false (key tiles only): V alone, for a backward given the forward's K~ and inverse RMS.
+template <bool IS_K, bool WITH_K = true>
 __device__ __forceinline__ void prep_tile(const BwdTcParams& p) {
     const LayerParams& L = p.P.L;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -306,30 +307,36 @@ __device__ __forceinline__ void prep_tile(const BwdTcParams& p) {
     __syncthreads();
     if (r == 0) {
         const CUtensorMap* src = IS_K ? &p.tm_k : &p.tm_q;
-        mbar_expect_tx(&sm.bar, (IS_K ? 2 : 1) * TF_TILE_BYTES);
-        tma_load_4d(sm.X[0], src, &sm.bar, 0, h, t * TF_BN, b);
-        tma_load_4d(sm.X[1], src, &sm.bar, 64, h, t * TF_BN, b);
+        mbar_expect_tx(&sm.bar, ((IS_K ? 1 : 0) + (WITH_K ? 1 : 0)) * TF_TILE_BYTES);
+        if constexpr (WITH_K) {
+            tma_load_4d(sm.X[0], src, &sm.bar, 0, h, t * TF_BN, b);
+            tma_load_4d(sm.X[1], src, &sm.bar, 64, h, t * TF_BN, b);
+        }
         if constexpr (IS_K) {
             tma_load_4d(sm.V[0], &p.tm_v, &sm.bar, 0, h, t * TF_BN, b);
             tma_load_4d(sm.V[1], &p.tm_v, &sm.bar, 64, h, t * TF_BN, b);
         }
     }
     const int pos = t * TF_BN + r;
-    float2 csr[TF_HALF];  // (cos, sin) of the rotated pairs at this row's position
+    float2 csr[WITH_K ? TF_HALF : 1];  // (cos, sin) of the rotated pairs at this row's position
+    if constexpr (WITH_K) {
 #pragma unroll
-    for (int q = 0; q < TF_HALF; ++q) rope_cs(L.theta[q], pos, csr[q].x, csr[q].y);
+        for (int q = 0; q < TF_HALF; ++q) rope_cs(L.theta[q], pos, csr[q].x, csr[q].y);
+    }
     const float oscale = qk_fp16_scale(sm.gq, sm.gk);
     // one decision for the whole CTA (the V conversion below has a CTA-wide barrier)
     const bool ok = __syncthreads_and(mbar_wait(&sm.bar, 0, &abort, 250)) != 0;
     if (ok) {
-        const float rinv = tf_prologue_row_at<true>(sm.X[0], sm.X[1], r, IS_K ? sm.gk : sm.gq, L,
-                                                    [&](int q) { return csr[q]; }, oscale);
+        float rinv = 0.f;
+        if constexpr (WITH_K)
+            rinv = tf_prologue_row_at<true>(sm.X[0], sm.X[1], r, IS_K ? sm.gk : sm.gq, L,
+                                            [&](int q) { return csr[q]; }, oscale);
         const size_t ro = ((size_t)b * H + h) * L.S + pos;
         if constexpr (IS_K) {
             float vn = 0.f;
             const float vt = v_tile_to_f16(sm.V[0], sm.V[1], r, sm.vred, &vn);
             if (pos < L.S) {
-                p.krinv[ro] = rinv;
+                if constexpr (WITH_K) p.krinv[ro] = rinv;
                 p.vnorm[ro] = vn;
             }
             if (r == 0) p.vtinv[(size_t)chain * nt + t] = vt;
@@ -344,8 +351,10 @@ __device__ __forceinline__ void prep_tile(const BwdTcParams& p) {
     if (r == 0) {
         if (ok) {
             const CUtensorMap* dst = IS_K ? &p.tm_k16 : &p.tm_q16;
-            tma_store_4d(dst, sm.X[0], 0, h, t * TF_BN, b);
-            tma_store_4d(dst, sm.X[1], 64, h, t * TF_BN, b);
+            if constexpr (WITH_K) {
+                tma_store_4d(dst, sm.X[0], 0, h, t * TF_BN, b);
+                tma_store_4d(dst, sm.X[1], 64, h, t * TF_BN, b);
+            }
             if constexpr (IS_K) {
                 tma_store_4d(&p.tm_v16, sm.V[0], 0, h, t * TF_BN, b);
                 tma_store_4d(&p.tm_v16, sm.V[1], 64, h, t * TF_BN, b);
@@ -363,6 +372,9 @@ __global__ void __launch_bounds__(KP_THREADS, 3) bwd_prep_kv_kernel(const __grid
 }
 __global__ void __launch_bounds__(KP_THREADS, 4) bwd_prep_q_kernel(const __grid_constant__ BwdTcParams p) {
     prep_tile<false>(p);
+}
+__global__ void __launch_bounds__(KP_THREADS, 3) bwd_prep_v_kernel(const __grid_constant__ BwdTcParams p) {
+    prep_tile<true, false>(p);
 }
 
 __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_constant__ BwdTcParams p) {
@@ -1259,11 +1271,23 @@ extern const char* const kBwdWideKernelNames[] = {"bwd_gate_kernel",       "bwd_
                                                   "bwd_q_glob_kernel",     "bwd_kv_tc_kernel",
                                                   "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"};
 extern const int kBwdWideKernelCount = 8;
+// the same given the forward's saved Q~, K~ and inverse RMS: V alone is prepared
+extern const char* const kBwdTcSavedKernelNames[] = {"bwd_gate_kernel",  "bwd_prep_v_kernel",
+                                                     "bwd_q_tc_kernel",  "bwd_kv_tc_kernel",
+                                                     "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"};
+extern const int kBwdTcSavedKernelCount = 6;
+extern const char* const kBwdWideSavedKernelNames[] = {"bwd_gate_kernel",   "bwd_prep_v_kernel",
+                                                       "bwd_tile_stats_kernel", "bwd_q_glob_kernel",
+                                                       "bwd_kv_tc_kernel",  "dgamma_reduce_kernel(k)",
+                                                       "dgamma_reduce_kernel(q)"};
+extern const int kBwdWideSavedKernelCount = 7;
 
 __global__ void dgamma_reduce_kernel(const float* __restrict__ parts, int n, float* __restrict__ out);
 
+// Windows up to one key tile, 42 rotated dims.  A shape test only: without the driver's
+// tensor-map encoder the launch fails (ZGCM_ERR_CUDA).
 bool bwd_tc_supported(const LayerParams& L) {
-    return L.W <= TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1 && get_encode_b() != nullptr;
+    return L.W <= TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1;
 }
 
 // Windows wider than one tile (the global layer among them), 42 rotated dims.  A shape test
@@ -1295,8 +1319,29 @@ size_t bwd_tc_workspace_bytes(int B, int S, int Hq, int Hkv) {
            a(3 * tiles * sizeof(float)) + 2 * a(dgamma_slots(B, S, Hq) * kD * sizeof(float));
 }
 
+// Q~ fp16 [B,S,Hq,D] into q16 and each q row's inverse RMS into qrinv ([B,Hq,S]): the
+// backward's query preparation, run by a forward that keeps its activations.
+cudaError_t launch_prep_q_only(const LayerParams& L, void* q16, float* qrinv, int* err_word, cudaStream_t stream) {
+    BwdTcParams p;
+    p.P.L = L;
+    p.qrinv = qrinv;
+    p.err = err_word;
+    const long long q_tiles = (long long)L.B * L.Hq * ((L.S + TF_BN - 1) / TF_BN);
+    if (q_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+    if (!make_map_b(&p.tm_q, L.q, L.Hq, L.S, L.B) ||
+        !make_map_b(&p.tm_q16, q16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        return cudaErrorInvalidValue;
+    const size_t smem_pq = sizeof(PrepSmem<false>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(bwd_prep_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_pq);
+    if (e != cudaSuccess) return e;
+    bwd_prep_q_kernel<<<(int)q_tiles, KP_THREADS, smem_pq, stream>>>(p);
+    return cudaGetLastError();
+}
+
+// With `sv`, Q~, K~ and the rows' inverse RMS come from the forward: the K/V preparation
+// converts V alone and the Q preparation does not run.
 cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, cudaStream_t stream,
-                          void* const* events, int n_pairs) {
+                          void* const* events, int n_pairs, const SavedAct* sv) {
     BwdTcParams p;
     p.P = bp;
     // a window of S or more is the full causal one: clamped so that window arithmetic
@@ -1334,6 +1379,12 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     const size_t slots = dgamma_slots(L.B, L.S, L.Hq);
     p.P.dgq_part = reinterpret_cast<float*>(take(slots * kD * 4));
     p.P.dgk_part = reinterpret_cast<float*>(take(slots * kD * 4));
+    if (sv) {
+        q16 = sv->q16;
+        p.qrinv = sv->qrinv;
+        k16 = sv->k16;
+        p.krinv = sv->krinv;
+    }
     p.err = err_word;
     const bool wide = bp.L.W > TF_BN;  // as the kernel-name query decides: on the window given
     p.wide = wide ? 1 : 0;
@@ -1387,6 +1438,9 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     if ((e = cudaFuncSetAttribute(bwd_prep_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_pq)) !=
         cudaSuccess)
         return e;
+    if ((e = cudaFuncSetAttribute(bwd_prep_v_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_pk)) !=
+        cudaSuccess)
+        return e;
     const long long k_tiles = (long long)L.B * L.Hkv * nkt, q_tiles = (long long)L.B * L.Hq * nkt;
     if (q_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
     int i = 0;
@@ -1399,11 +1453,16 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
                                                                        p.domax, nullptr, (long long)rows, L.S, L.Hq);
     if ((e = after(i++)) != cudaSuccess) return e;
     if ((e = before(i)) != cudaSuccess) return e;
-    bwd_prep_kv_kernel<<<(int)k_tiles, KP_THREADS, smem_pk, stream>>>(p);
+    if (sv)
+        bwd_prep_v_kernel<<<(int)k_tiles, KP_THREADS, smem_pk, stream>>>(p);
+    else
+        bwd_prep_kv_kernel<<<(int)k_tiles, KP_THREADS, smem_pk, stream>>>(p);
     if ((e = after(i++)) != cudaSuccess) return e;
-    if ((e = before(i)) != cudaSuccess) return e;
-    bwd_prep_q_kernel<<<(int)q_tiles, KP_THREADS, smem_pq, stream>>>(p);
-    if ((e = after(i++)) != cudaSuccess) return e;
+    if (!sv) {
+        if ((e = before(i)) != cudaSuccess) return e;
+        bwd_prep_q_kernel<<<(int)q_tiles, KP_THREADS, smem_pq, stream>>>(p);
+        if ((e = after(i++)) != cudaSuccess) return e;
+    }
     if (wide) {
         // per-tile bounds, then the query-major sweep (one CTA per (b, head, block), heaviest
         // first) and the key-major one (one CTA per (b, KV head, tile), heaviest first)

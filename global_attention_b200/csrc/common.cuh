@@ -43,6 +43,16 @@ struct FwdParams {
     float* lse;   // [B,Hq,S]
 };
 
+// Activations the forward can leave for the backward (all null = none): the fp16 Q~
+// [B,S,Hq,D] and K~ [B,S,Hkv,D] that both passes form, and the inverse RMS of every q and k
+// row (fp32 [B,Hq,S], [B,Hkv,S]): the bits the backward's preparation would recompute.
+struct SavedAct {
+    void* q16 = nullptr;
+    float* qrinv = nullptr;
+    void* k16 = nullptr;
+    float* krinv = nullptr;
+};
+
 struct BwdParams {
     LayerParams L;
     const bf16* out;    // [B,S,Hq,D]

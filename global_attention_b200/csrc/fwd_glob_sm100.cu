@@ -50,6 +50,7 @@ struct FwdGlobParams {
     bf16* out;
     float* lse;
     int* err;
+    float* krinv;        // inverse RMS of each k row, [B,Hkv,S] (preparation kernel; null = not kept)
     int units;           // B * Hkv * (G / 2) * ceil(S / 128)
 };
 
@@ -132,7 +133,9 @@ __global__ void __launch_bounds__(FP_THREADS, 4) fwd_prep_k_kernel(const __grid_
     const float oscale = qk_fp16_scale(sm.gq, sm.gk);
     const bool ok = __syncthreads_and(mbar_wait(&sm.bar, 0, &abort, 260)) != 0;
     if (ok) {
-        tf_prologue_row_at<true>(sm.X[0], sm.X[1], r, sm.gk, L, [&](int q) { return csr[q]; }, oscale);
+        const float rinv = tf_prologue_row_at<true>(sm.X[0], sm.X[1], r, sm.gk, L, [&](int q) { return csr[q]; },
+                                                    oscale);
+        if (p.krinv && pos < L.S) p.krinv[(size_t)chain * L.S + pos] = rinv;
         fence_proxy_async_smem();
     } else if (r == 0) {
         mbar_wait_drain(&sm.bar, 0);
@@ -472,9 +475,15 @@ bool fwd_glob_supported(const LayerParams& L) {
 // K~ fp16 [B, S, Hkv, D] (both tcgen05 forwards)
 size_t fwd_glob_workspace_bytes(int B, int S, int Hkv) { return (size_t)B * S * Hkv * kD * 2; }
 
-cudaError_t launch_fwd_glob_tc(const FwdParams& fp, void* workspace, int* err_word, cudaStream_t stream) {
+cudaError_t launch_prep_q_only(const LayerParams& L, void* q16, float* qrinv, int* err_word, cudaStream_t stream);
+
+// With `sv`, K~ goes to sv->k16 (the caller passes it as `workspace`) with each k row's
+// inverse RMS, and a preparation pass leaves Q~ and the q rows' inverse RMS there too.
+cudaError_t launch_fwd_glob_tc(const FwdParams& fp, void* workspace, int* err_word, cudaStream_t stream,
+                               const SavedAct* sv) {
     FwdGlobParams p;
     p.L = fp.L;
+    p.krinv = sv ? sv->krinv : nullptr;
     // a window of S or more is the full causal one: clamped so that window arithmetic stays in range
     if (p.L.W > p.L.S) p.L.W = p.L.S;
     const LayerParams& L = p.L;
@@ -498,14 +507,18 @@ cudaError_t launch_fwd_glob_tc(const FwdParams& fp, void* workspace, int* err_wo
     if (e != cudaSuccess) return e;
     fwd_prep_k_kernel<<<(int)k_tiles, FP_THREADS, smem_p, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (sv && (e = launch_prep_q_only(fp.L, sv->q16, sv->qrinv, err_word, stream)) != cudaSuccess) return e;
     fwd_glob_tc_kernel<<<(int)units, FG_THREADS, smem_a, stream>>>(p);
     return cudaGetLastError();
 }
 
 // K~ fp16 of every key tile into `workspace` ([B,S,Hkv,D]) for the sliding-window forward.
-cudaError_t launch_fwd_prep_k(const LayerParams& L, void* workspace, int* err_word, cudaStream_t stream) {
+// With `krinv`, also each k row's inverse RMS ([B,Hkv,S]).
+cudaError_t launch_fwd_prep_k(const LayerParams& L, void* workspace, int* err_word, cudaStream_t stream,
+                              float* krinv) {
     FwdGlobParams p;
     p.L = L;
+    p.krinv = krinv;
     p.out = nullptr;
     p.lse = nullptr;
     p.err = err_word;

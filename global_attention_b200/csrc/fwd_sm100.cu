@@ -41,11 +41,14 @@ struct FwdTcParams {
     CUtensorMap tm_q;   // {D, Hq, S, B}, box {64, 1, 128, 1}, 128B swizzle
     CUtensorMap tm_k16; // K~ fp16 {D, Hkv, S, B} (fwd_prep_k_kernel, in the workspace)
     CUtensorMap tm_v;
+    CUtensorMap tm_q16s; // Q~ fp16 {D, Hq, S, B} kept for the backward, box {64, 1, 32, 1} (save_q)
     LayerParams L;
     bf16* out;
     float* lse;
+    float* qrinv;       // inverse RMS of each q row, [B,Hq,S] (save_q)
     int* err;           // device error word: site of an expired wait (0 = none)
     int total_steps;    // B * Hkv * ceil(S / 128)
+    int save_q;         // keep Q~ and the q rows' inverse RMS for the backward
 };
 
 enum Bar {
@@ -367,8 +370,23 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
             for (int h = 0; h < G; ++h, ++m) {
                 const int buf = m & 1;
                 if (!(ok = mbar_wait(&sm.bar[B_QFULL + buf], (m >> 1) & 1, abort, 33))) break;
-                tf_prologue_row<true>(sm.Q[buf][0], sm.Q[buf][1], r, sm.gq, L, sm.cs, oscale);
+                const float rinv = tf_prologue_row<true>(sm.Q[buf][0], sm.Q[buf][1], r, sm.gq, L, sm.cs, oscale);
                 fence_proxy_async_smem();
+                if (p.save_q) {
+                    // this warp's 32 rows of Q~ to the store the backward reads; their shared
+                    // memory is read before the tile is handed over (it is refilled after S)
+                    const int hg = st.kvh * G + h, i = st.qb * TF_BM + r, wq = warp - 8;
+                    const int row0 = st.qb * TF_BM + 32 * wq;
+                    if (i < L.S) p.qrinv[((size_t)st.b * L.Hq + hg) * L.S + i] = rinv;
+                    __syncwarp();
+                    if (lane == 0 && row0 < L.S) {
+                        tma_store_4d(&p.tm_q16s, sm.Q[buf][0] + wq * 32 * 128, 0, hg, row0, st.b);
+                        tma_store_4d(&p.tm_q16s, sm.Q[buf][1] + wq * 32 * 128, 64, hg, row0, st.b);
+                        tma_store_commit();
+                        tma_store_wait_read();
+                    }
+                    __syncwarp();
+                }
                 mbar_arrive(&sm.bar[B_QREADY + buf]);
             }
         }
@@ -455,14 +473,14 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-// 4-D 16-bit map {D, H, S, B} (innermost first), box {64, 1, 128, 1}, 128-byte swizzle
+// 4-D 16-bit map {D, H, S, B} (innermost first), box {64, 1, rows, 1}, 128-byte swizzle
 bool make_map(CUtensorMap* map, const void* base, int H, int S, int B,
-              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, int rows = 128) {
     auto enc = get_encode();
     if (!enc) return false;
     cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)S * H * kD * 2};
-    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(map, dtype, 4, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -480,15 +498,23 @@ bool fwd_tc_supported(const LayerParams& L) {
 
 size_t fwd_tc_smem_bytes() { return sizeof(FwdTcSmem) + 1024; }
 
-cudaError_t launch_fwd_prep_k(const LayerParams& L, void* workspace, int* err_word, cudaStream_t stream);
+cudaError_t launch_fwd_prep_k(const LayerParams& L, void* workspace, int* err_word, cudaStream_t stream,
+                              float* krinv);
 
-// fwd_prep_k_kernel (K~ into `workspace`, [B,S,Hkv,D] fp16), then the attention kernel
-cudaError_t launch_fwd_tc(const FwdParams& fp, void* workspace, int* err_word, cudaStream_t stream) {
+// fwd_prep_k_kernel (K~ into `workspace`, [B,S,Hkv,D] fp16), then the attention kernel.
+// With `sv` (whose k16 the caller passes as `workspace`), both also keep the inverse RMS of
+// every row, and the attention kernel stores Q~ for the backward.
+cudaError_t launch_fwd_tc(const FwdParams& fp, void* workspace, int* err_word, cudaStream_t stream,
+                          const SavedAct* sv) {
     FwdTcParams p;
     p.L = fp.L;
     p.out = fp.out;
     p.lse = fp.lse;
     p.err = err_word;
+    p.save_q = sv ? 1 : 0;
+    p.qrinv = sv ? sv->qrinv : nullptr;
+    if (sv && !make_map(&p.tm_q16s, sv->q16, fp.L.Hq, fp.L.S, fp.L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 32))
+        return cudaErrorInvalidValue;
     const int nqb = (fp.L.S + TF_BM - 1) / TF_BM;
     const long long total = (long long)fp.L.B * fp.L.Hkv * nqb;
     if (total > 0x7fffffffLL) return cudaErrorInvalidValue;
@@ -498,7 +524,7 @@ cudaError_t launch_fwd_tc(const FwdParams& fp, void* workspace, int* err_word, c
         !make_map(&p.tm_v, fp.L.v, fp.L.Hkv, fp.L.S, fp.L.B))
         return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
-    cudaError_t e = launch_fwd_prep_k(fp.L, workspace, err_word, stream);
+    cudaError_t e = launch_fwd_prep_k(fp.L, workspace, err_word, stream, sv ? sv->krinv : nullptr);
     if (e != cudaSuccess) return e;
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -10,9 +10,11 @@
 
 namespace zgcm {
 cudaError_t launch_fwd_mma(const FwdParams& p, cudaStream_t stream);
-cudaError_t launch_fwd_tc(const FwdParams& p, void* workspace, int* err_word, cudaStream_t stream);
+cudaError_t launch_fwd_tc(const FwdParams& p, void* workspace, int* err_word, cudaStream_t stream,
+                          const SavedAct* sv);
 bool fwd_tc_supported(const LayerParams& L);
-cudaError_t launch_fwd_glob_tc(const FwdParams& p, void* workspace, int* err_word, cudaStream_t stream);
+cudaError_t launch_fwd_glob_tc(const FwdParams& p, void* workspace, int* err_word, cudaStream_t stream,
+                               const SavedAct* sv);
 bool fwd_glob_supported(const LayerParams& L);
 size_t decode_workspace_bytes(int B, int Hq, int window, int C);
 cudaError_t launch_selftest_expired_wait(int* err_word, cudaStream_t stream);
@@ -24,7 +26,11 @@ cudaError_t launch_bwd_mma(const BwdParams& p, cudaStream_t stream, void* const*
 extern const char* const kBwdMmaKernelNames[];
 extern const int kBwdMmaKernelCount;
 cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, cudaStream_t stream,
-                          void* const* events, int n_pairs);
+                          void* const* events, int n_pairs, const SavedAct* sv);
+extern const char* const kBwdTcSavedKernelNames[];
+extern const int kBwdTcSavedKernelCount;
+extern const char* const kBwdWideSavedKernelNames[];
+extern const int kBwdWideSavedKernelCount;
 bool bwd_tc_supported(const LayerParams& L);
 bool bwd_wide_supported(const LayerParams& L);
 extern const char* const kBwdWideKernelNames[];
@@ -136,6 +142,31 @@ BwdWorkspace bwd_layout(int B, int S, int Hq, int Hkv) {
     return w;
 }
 
+// The activation store a forward leaves for the backward: Q~ fp16 [B,S,Hq,D], the q rows'
+// inverse RMS fp32 [B,Hq,S], K~ fp16 [B,S,Hkv,D] (the forward's own K~ workspace) and the k
+// rows' inverse RMS fp32 [B,Hkv,S], each 256-byte aligned.
+size_t saved_layout(int B, int S, int Hq, int Hkv, char* base, SavedAct* sv) {
+    const size_t rows = (size_t)B * S * Hq, krows = (size_t)B * S * Hkv;
+    size_t off = 0;
+    const size_t q16 = off;   off = align256(off + rows * kD * 2);
+    const size_t qrinv = off; off = align256(off + rows * 4);
+    const size_t k16 = off;   off = align256(off + krows * kD * 2);
+    const size_t krinv = off; off = align256(off + krows * 4);
+    if (sv) {
+        sv->q16 = base + q16;
+        sv->qrinv = reinterpret_cast<float*>(base + qrinv);
+        sv->k16 = base + k16;
+        sv->krinv = reinterpret_cast<float*>(base + krinv);
+    }
+    return off;
+}
+
+// The store applies where both passes run the tcgen05 kernels.
+bool saved_supported(const LayerParams& L) {
+    const FwdPath f = fwd_path(L);
+    return f != FwdPath::MMA && (bwd_tc_supported(L) || bwd_wide_supported(L));
+}
+
 }  // namespace
 
 extern "C" {
@@ -205,8 +236,8 @@ int zgcm_attn_fwd_ws(const void* q, const void* k, const void* v, const void* g,
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     cudaError_t e;
     switch (fwd_path(p.L)) {
-        case FwdPath::TC: e = launch_fwd_tc(p, workspace, device_error_word(), stream); break;
-        case FwdPath::GLOB: e = launch_fwd_glob_tc(p, workspace, device_error_word(), stream); break;
+        case FwdPath::TC: e = launch_fwd_tc(p, workspace, device_error_word(), stream, nullptr); break;
+        case FwdPath::GLOB: e = launch_fwd_glob_tc(p, workspace, device_error_word(), stream, nullptr); break;
         default: e = launch_fwd_mma(p, stream); break;
     }
     return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
@@ -232,6 +263,38 @@ int zgcm_attn_fwd(const void* q, const void* k, const void* v, const void* g,
                                     window, causal, eps, scale, out, lse, ws, need, cuda_stream);
     const cudaError_t e = cudaFreeAsync(ws, stream);
     if (st != ZGCM_OK) return st;
+    return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
+}
+
+size_t zgcm_attn_saved_size(int B, int S, int Hq, int Hkv, int D, int rope_dims, int window) {
+    if (check_shape(B, S, Hq, Hkv, D, rope_dims, 1.0, window, 1, 0.f, 1.f) != ZGCM_OK) return 0;
+    if ((long long)B * S == 0) return 0;
+    if (!saved_supported(shape_only(B, S, Hq, Hkv, rope_dims, window))) return 0;
+    return saved_layout(B, S, Hq, Hkv, nullptr, nullptr);
+}
+
+int zgcm_attn_fwd_save(const void* q, const void* k, const void* v, const void* g,
+                       const float* gamma_q, const float* gamma_k,
+                       int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                       double rope_base, int window, int causal, float eps, float scale,
+                       void* out, float* lse, void* saved, size_t saved_bytes, void* cuda_stream) {
+    int st = fwd_check(q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, D, rope_dims, rope_base, window, causal,
+                       eps, scale, out, lse);
+    if (st != ZGCM_OK) return st;
+    if ((long long)B * S == 0) return ZGCM_OK;
+    FwdParams p;
+    fill_layer(p.L, q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, rope_dims, rope_base, window, eps, scale);
+    if (!saved_supported(p.L)) return ZGCM_ERR_UNSUPPORTED;
+    if (!saved || saved_bytes < zgcm_attn_saved_size(B, S, Hq, Hkv, D, rope_dims, window)) return ZGCM_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(saved) & 255u) return ZGCM_ERR_ALIGNMENT;
+    SavedAct sv;
+    saved_layout(B, S, Hq, Hkv, static_cast<char*>(saved), &sv);
+    p.out = static_cast<bf16*>(out);
+    p.lse = lse;
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    const cudaError_t e = fwd_path(p.L) == FwdPath::TC
+                              ? launch_fwd_tc(p, sv.k16, device_error_word(), stream, &sv)
+                              : launch_fwd_glob_tc(p, sv.k16, device_error_word(), stream, &sv);
     return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
 }
 
@@ -301,15 +364,16 @@ size_t zgcm_attn_bwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int wi
     return a > b ? a : b;
 }
 
-int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void* g,
-                        const float* gamma_q, const float* gamma_k,
-                        const void* out, const float* lse, const void* dout,
-                        int B, int S, int Hq, int Hkv, int D, int rope_dims,
-                        double rope_base, int window, int causal, float eps, float scale,
-                        void* dq, void* dk, void* dv, void* dg,
-                        float* dgamma_q, float* dgamma_k,
-                        void* workspace, size_t workspace_bytes, void* cuda_stream,
-                        void* const* events, int n_pairs) {
+}  // extern "C"
+
+namespace {
+// The backward; with `saved` (non-null), from the activations zgcm_attn_fwd_save left there.
+int bwd_run(const void* q, const void* k, const void* v, const void* g, const float* gamma_q,
+            const float* gamma_k, const void* out, const float* lse, const void* dout, int B, int S, int Hq,
+            int Hkv, int D, int rope_dims, double rope_base, int window, int causal, float eps, float scale,
+            void* dq, void* dk, void* dv, void* dg, float* dgamma_q, float* dgamma_k, void* workspace,
+            size_t workspace_bytes, const void* saved, size_t saved_bytes, void* cuda_stream,
+            void* const* events, int n_pairs) {
     int st = check_shape(B, S, Hq, Hkv, D, rope_dims, rope_base, window, causal, eps, scale);
     if (st != ZGCM_OK) return st;
     if (!dgamma_q || !dgamma_k) return ZGCM_ERR_INVALID_ARG;
@@ -352,12 +416,66 @@ int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void*
     p.n_k_parts = w.n_k_parts;
     p.n_q_parts = (int)w.n_q_parts;
     if (n_pairs < 0 || (n_pairs > 0 && !events)) return ZGCM_ERR_INVALID_ARG;
+    SavedAct sv;
+    if (saved) {
+        if (!saved_supported(p.L)) return ZGCM_ERR_UNSUPPORTED;
+        if (saved_bytes < saved_layout(B, S, Hq, Hkv, nullptr, nullptr)) return ZGCM_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(saved) & 255u) return ZGCM_ERR_ALIGNMENT;
+        saved_layout(B, S, Hq, Hkv, static_cast<char*>(const_cast<void*>(saved)), &sv);
+    }
     cudaError_t e;
     if (!force_mma() && (bwd_tc_supported(p.L) || bwd_wide_supported(p.L)))
-        e = launch_bwd_tc(p, workspace, device_error_word(), stream, events, n_pairs);
+        e = launch_bwd_tc(p, workspace, device_error_word(), stream, events, n_pairs, saved ? &sv : nullptr);
     else
         e = launch_bwd_mma(p, stream, events, n_pairs);
     return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" {
+
+int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void* g,
+                        const float* gamma_q, const float* gamma_k,
+                        const void* out, const float* lse, const void* dout,
+                        int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                        double rope_base, int window, int causal, float eps, float scale,
+                        void* dq, void* dk, void* dv, void* dg,
+                        float* dgamma_q, float* dgamma_k,
+                        void* workspace, size_t workspace_bytes, void* cuda_stream,
+                        void* const* events, int n_pairs) {
+    return bwd_run(q, k, v, g, gamma_q, gamma_k, out, lse, dout, B, S, Hq, Hkv, D, rope_dims, rope_base, window,
+                   causal, eps, scale, dq, dk, dv, dg, dgamma_q, dgamma_k, workspace, workspace_bytes, nullptr, 0,
+                   cuda_stream, events, n_pairs);
+}
+
+int zgcm_attn_bwd_saved(const void* q, const void* k, const void* v, const void* g,
+                        const float* gamma_q, const float* gamma_k,
+                        const void* out, const float* lse, const void* dout,
+                        int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                        double rope_base, int window, int causal, float eps, float scale,
+                        void* dq, void* dk, void* dv, void* dg,
+                        float* dgamma_q, float* dgamma_k,
+                        void* workspace, size_t workspace_bytes, const void* saved, size_t saved_bytes,
+                        void* cuda_stream, void* const* events, int n_pairs) {
+    if (!saved) return ZGCM_ERR_INVALID_ARG;
+    return bwd_run(q, k, v, g, gamma_q, gamma_k, out, lse, dout, B, S, Hq, Hkv, D, rope_dims, rope_base, window,
+                   causal, eps, scale, dq, dk, dv, dg, dgamma_q, dgamma_k, workspace, workspace_bytes, saved,
+                   saved_bytes, cuda_stream, events, n_pairs);
+}
+
+const char* zgcm_attn_bwd_saved_kernel_name(int i, int S, int rope_dims, int window) {
+    LayerParams L{};
+    L.B = 1; L.S = S; L.rope_half = rope_dims / 2; L.W = window;
+    const char* const* names = nullptr;
+    int n = 0;
+    if (!force_mma() && S >= 1 && bwd_tc_supported(L)) {
+        names = kBwdTcSavedKernelNames;
+        n = kBwdTcSavedKernelCount;
+    } else if (!force_mma() && S >= 1 && bwd_wide_supported(L)) {
+        names = kBwdWideSavedKernelNames;
+        n = kBwdWideSavedKernelCount;
+    }
+    return (i >= 0 && i < n) ? names[i] : nullptr;
 }
 
 const char* zgcm_attn_bwd_kernel_name(int i, int S, int rope_dims, int window) {

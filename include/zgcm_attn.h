@@ -113,6 +113,50 @@ int zgcm_attn_fwd_ws(const void* q, const void* k, const void* v, const void* g,
                      void* out, float* lse, void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * Training-step pair: a forward that keeps the activations its backward would otherwise
+ * recompute.  Both passes form the same fp16 q~ = RoPE(gamma_q * q / rms(q)) and k~ (times
+ * the same power of two) and the same inverse RMS of every q and k row (RMSNorm backward);
+ * zgcm_attn_fwd_save leaves them in a caller-owned store and zgcm_attn_bwd_saved reads them
+ * there instead of converting q and k again (its preparation pass converts v alone).  The
+ * results are bit-identical to zgcm_attn_fwd + zgcm_attn_bwd on the same inputs.
+ *
+ * zgcm_attn_saved_size: bytes of the store for this problem; 0 for an empty problem and
+ *   where the pair does not apply (it needs the tcgen05 kernels: rope_dims == 42 and, for
+ *   windows wider than 128, an even Hq/Hkv; not with ZGCM_FORCE_MMA=1).
+ * Layout (each part 256-byte aligned, in this order): q~ fp16 [B,S,Hq,D], q inverse RMS fp32
+ *   [B,Hq,S], k~ fp16 [B,S,Hkv,D], k inverse RMS fp32 [B,Hkv,S].
+ * zgcm_attn_fwd_save: zgcm_attn_fwd_ws with the store as its workspace (k~ is the forward's
+ *   own key workspace).  `saved`: at least zgcm_attn_saved_size bytes, 256-byte aligned,
+ *   owned by the caller; after the call (in stream order) it holds this forward's
+ *   activations.  Returns ZGCM_ERR_UNSUPPORTED where zgcm_attn_saved_size is 0 for a
+ *   non-empty problem, ZGCM_ERR_WORKSPACE / ZGCM_ERR_ALIGNMENT for a store too small or
+ *   misaligned; otherwise as zgcm_attn_fwd.
+ * zgcm_attn_bwd_saved: zgcm_attn_bwd_timed given the store a zgcm_attn_fwd_save of the same
+ *   inputs and arguments filled (`saved`, read only; NULL returns ZGCM_ERR_INVALID_ARG).
+ *   Kernels: zgcm_attn_bwd_saved_kernel_name(i) (bwd_prep_v_kernel in place of the two
+ *   preparation kernels).  The workspace is the same as zgcm_attn_bwd's.
+ */
+size_t zgcm_attn_saved_size(int B, int S, int Hq, int Hkv, int D, int rope_dims, int window);
+
+int zgcm_attn_fwd_save(const void* q, const void* k, const void* v, const void* g,
+                       const float* gamma_q, const float* gamma_k,
+                       int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                       double rope_base, int window, int causal, float eps, float scale,
+                       void* out, float* lse, void* saved, size_t saved_bytes, void* cuda_stream);
+
+int zgcm_attn_bwd_saved(const void* q, const void* k, const void* v, const void* g,
+                        const float* gamma_q, const float* gamma_k,
+                        const void* out, const float* lse, const void* dout,
+                        int B, int S, int Hq, int Hkv, int D, int rope_dims,
+                        double rope_base, int window, int causal, float eps, float scale,
+                        void* dq, void* dk, void* dv, void* dg,
+                        float* dgamma_q, float* dgamma_k,
+                        void* workspace, size_t workspace_bytes, const void* saved, size_t saved_bytes,
+                        void* cuda_stream, void* const* events, int n_pairs);
+
+const char* zgcm_attn_bwd_saved_kernel_name(int i, int S, int rope_dims, int window);
+
+/*
  * Bytes of device workspace zgcm_attn_bwd needs for this problem (0 for an empty one).
  * Returns 0 as well for arguments zgcm_attn_bwd would reject.
  */

@@ -147,6 +147,57 @@ def test_fwd_ws_checks(lib):
     assert _fwd_ws(lib, P + 256 * 40, need, S=640, window=0) == -1
 
 
+def test_saved_size_query(lib):
+    sz = lambda *a: lib.zgcm_attn_saved_size(*a)
+    al = lambda x: (x + 255) // 256 * 256
+    # q~ fp16, q inverse RMS, k~ fp16, k inverse RMS, each 256-byte aligned
+    for B, S, W in ((4, 16384, 128), (1, 1000, 7), (2, 777, 10**6), (1, 1, 128), (3, 260, 129)):
+        rows, krows = B * S * 32, B * S * 8
+        assert sz(B, S, 32, 8, 128, 42, W) == al(rows * 256) + al(rows * 4) + al(krows * 256) + al(krows * 4)
+    assert sz(1, 1024, 32, 8, 128, 0, 128) == 0       # no rotation: the warp-MMA kernels
+    assert sz(1, 1024, 24, 8, 128, 42, 1024) == 0     # odd group size with a wide window: likewise
+    assert sz(0, 1024, 32, 8, 128, 42, 128) == 0      # empty
+    assert sz(1, 1024, 32, 8, 64, 42, 128) == 0       # invalid
+
+
+def _fwd_save(lib, saved, saved_bytes, **kw):
+    a = dict(ARGS, **kw)
+    vp = ctypes.c_void_p
+    p = [vp(P + 256 * i) for i in range(8)]
+    return lib.zgcm_attn_fwd_save(*p[:6], a["B"], a["S"], a["Hq"], a["Hkv"], a["D"], a["rope_dims"],
+                                  a["rope_base"], a["window"], a["causal"], a["eps"], a["scale"],
+                                  p[6], p[7], vp(saved), saved_bytes, None)
+
+
+def _bwd_saved(lib, ws_bytes, saved, saved_bytes, **kw):
+    a = dict(ARGS, **kw)
+    vp = ctypes.c_void_p
+    p = [vp(P + 256 * i) for i in range(15)]
+    return lib.zgcm_attn_bwd_saved(*p[:9], a["B"], a["S"], a["Hq"], a["Hkv"], a["D"], a["rope_dims"],
+                                   a["rope_base"], a["window"], a["causal"], a["eps"], a["scale"], *p[9:15],
+                                   vp(P + 256 * 40), ws_bytes, vp(saved), saved_bytes, None, None, 0)
+
+
+def test_saved_pair_checks(lib):
+    need = lib.zgcm_attn_saved_size(1, 64, 32, 8, 128, 42, 128)
+    assert need > 0
+    store = P + 2 ** 30
+    assert _fwd_save(lib, store, need - 1) == -4          # too small
+    assert _fwd_save(lib, 0, need) == -4                  # missing
+    assert _fwd_save(lib, store + 16, need) == -3         # not 256-byte aligned
+    assert _fwd_save(lib, store, need, rope_dims=0) == -2  # the pair needs the tcgen05 kernels
+    assert _fwd_save(lib, store, need, window=0) == -1
+    ws = lib.zgcm_attn_bwd_workspace_size(1, 64, 32, 8, 128, 128)
+    assert _bwd_saved(lib, ws, 0, need) == -1             # the store is required
+    assert _bwd_saved(lib, ws, store, need - 1) == -4
+    assert _bwd_saved(lib, ws, store + 16, need) == -3
+    assert _bwd_saved(lib, ws - 1, store, need) == -4     # the workspace is checked as before
+    assert _bwd_saved(lib, ws, store, need, rope_dims=0) == -2
+    names = ga.zgcm_attn_bwd_kernel_names(16384, 128, saved=True)
+    assert names[:4] == ["bwd_gate_kernel", "bwd_prep_v_kernel", "bwd_q_tc_kernel", "bwd_kv_tc_kernel"]
+    assert "bwd_prep_q_kernel" not in ga.zgcm_attn_bwd_kernel_names(4096, 4096, saved=True)
+
+
 def _dec(lib, ws_bytes, ptrs=None, ws=P + 256 * 40, **kw):
     a = dict(ARGS, **kw)
     vp = ctypes.c_void_p

@@ -219,6 +219,28 @@ def _decode_run(t, W, C, offsets=None, rope_dims=42):
     return torch.stack(outs), torch.stack(lses), torch.stack(poss)
 
 
+@pytest.mark.parametrize("B,S,W", [(1, 1024, 128), (2, 1000, 128), (1, 129, 7), (3, 260, 1), (1, 1, 128),
+                                   (1, 777, 777), (2, 640, 129), (1, 1300, 300)])
+def test_saved_activations_bit_identical(B, S, W, monkeypatch):
+    """zgcm_attn_fwd(saved=...) then zgcm_attn_bwd(saved=...) gives exactly the results of the
+    plain pair: the store holds the q~, k~ and inverse RMS values the backward's preparation
+    would form (the store starts out filled with garbage)."""
+    monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
+    t = make_inputs(B, S, seed=700 + S + W % 1000, with_dout=True)
+    d = _to_dev(t)
+    out, lse = _gpu_fwd(d, window=W)
+    gr = _gpu_bwd(d, out, lse, window=W)
+    n = ga.zgcm_attn_saved_size(B, S, 32, 8, window=W)
+    assert n > 0
+    saved = torch.full((n,), 0xAB, dtype=torch.uint8, device="cuda")
+    out_s, lse_s = _gpu_fwd(d, window=W, saved=saved)
+    assert torch.equal(out, out_s) and torch.equal(lse, lse_s)
+    gr_s = _gpu_bwd(d, out_s, lse_s, window=W, saved=saved)
+    assert ga.zgcm_attn_device_error() == 0
+    for name in gr:
+        assert torch.equal(gr[name], gr_s[name]), name
+
+
 @pytest.mark.parametrize("B,S,W,C", [(2, 300, 128, 128),     # sliding layer: a ring of W slots
                                      (1, 700, 700, 768),     # global layer: every token kept, 2 splits
                                      (3, 200, 50, 64),       # ring larger than the window
