@@ -56,7 +56,9 @@ enum Bar {
     B_QFULL = 8, B_QREADY = 10, B_QEMPTY = 12,
     B_SFULL = 14, B_PFULL = 15,
     B_OFULL = 16, B_OEMPTY = 18, B_LFULL = 20, B_LEMPTY = 22,
-    B_DONE = 24, B_COUNT = 25
+    B_DONE = 24,
+    B_QSTORED = 25,  // a Q buffer's rows were read by the stores that keep Q~ (save_q), by buffer
+    B_COUNT = 27
 };
 
 struct FwdTcSmem {
@@ -105,6 +107,7 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
         mbar_init(&sm.bar[B_SFULL], 1);
         mbar_init(&sm.bar[B_PFULL], 128);
         mbar_init(&sm.bar[B_DONE], 1);
+        for (int i = 0; i < 2; ++i) mbar_init(&sm.bar[B_QSTORED + i], 4);  // lane 0 of each prologue warp
         fence_barrier_init();
     }
     if (tid < kD) {
@@ -185,6 +188,8 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
                 for (int h = 0; h < G; ++h, ++m) {
                     const int buf = m & 1;
                     if (m >= 2 && !mbar_wait(&sm.bar[B_QEMPTY + buf], ((m >> 1) - 1) & 1, abort, 3)) break;
+                    if (p.save_q && m >= 2 && !mbar_wait(&sm.bar[B_QSTORED + buf], ((m >> 1) - 1) & 1, abort, 4))
+                        break;
                     mbar_expect_tx(&sm.bar[B_QFULL + buf], TF_TILE_BYTES);
                     const int hg = st.kvh * G + h;
                     tma_load_4d(sm.Q[buf][0], &p.tm_q, &sm.bar[B_QFULL + buf], 0, hg, st.qb * TF_BM, st.b);
@@ -373,8 +378,7 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
                 const float rinv = tf_prologue_row<true>(sm.Q[buf][0], sm.Q[buf][1], r, sm.gq, L, sm.cs, oscale);
                 fence_proxy_async_smem();
                 if (p.save_q) {
-                    // this warp's 32 rows of Q~ to the store the backward reads; their shared
-                    // memory is read before the tile is handed over (it is refilled after S)
+                    // this warp's 32 rows of Q~ to the store the backward reads
                     const int hg = st.kvh * G + h, i = st.qb * TF_BM + r, wq = warp - 8;
                     const int row0 = st.qb * TF_BM + 32 * wq;
                     if (i < L.S) p.qrinv[((size_t)st.b * L.Hq + hg) * L.S + i] = rinv;
@@ -383,11 +387,15 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
                         tma_store_4d(&p.tm_q16s, sm.Q[buf][0] + wq * 32 * 128, 0, hg, row0, st.b);
                         tma_store_4d(&p.tm_q16s, sm.Q[buf][1] + wq * 32 * 128, 64, hg, row0, st.b);
                         tma_store_commit();
-                        tma_store_wait_read();
                     }
-                    __syncwarp();
                 }
                 mbar_arrive(&sm.bar[B_QREADY + buf]);
+                if (p.save_q && lane == 0) {
+                    // the buffer is refilled (two heads on) only once the stores have read it
+                    tma_store_wait_read();
+                    mbar_arrive(&sm.bar[B_QSTORED + buf]);
+                }
+                __syncwarp();
             }
         }
     } else if (warp >= 12) {
