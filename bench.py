@@ -601,6 +601,11 @@ def main():
     if world > 1:
         dist.barrier()
     ms = t0.elapsed_time(t1)
+    # a bounded device wait that expired means a kernel gave up part of its work: no timing
+    derr = ga.zgcm_attn_device_error()
+    if derr != 0:
+        print(json.dumps({"error": f"device wait expired in the timed region ({ga.zgcm_status_string(derr)})"}))
+        return 1
     # per kernel and layer: (mean ms, algorithmic bytes, flops); the key names the kernel, and
     # the layer's window when the step runs more than one layer
     kern, layer_ms = {}, []

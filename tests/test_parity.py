@@ -32,6 +32,8 @@ def _to_dev(t):
 def _gpu_fwd(d, **kw):
     out, lse = ga.zgcm_attn_fwd(d["q"], d["k"], d["v"], d["g"], d["gamma_q"], d["gamma_k"], **kw)
     torch.cuda.synchronize()
+    # an expired bounded wait leaves outputs unwritten: never compare those
+    assert ga.zgcm_attn_device_error() == 0
     return out, lse
 
 
@@ -39,6 +41,7 @@ def _gpu_bwd(d, out, lse, **kw):
     gr = ga.zgcm_attn_bwd(d["q"], d["k"], d["v"], d["g"], d["gamma_q"], d["gamma_k"], out, lse,
                           d["dout"], **kw)
     torch.cuda.synchronize()
+    assert ga.zgcm_attn_device_error() == 0
     return gr
 
 
