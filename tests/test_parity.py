@@ -351,11 +351,20 @@ def test_forward_bitwise_repeatable():
 
 # ------------------------------------------------------------------ full-size workloads
 
-def _sampled_fwd_bwd(B, S, W, n_random, k_rows, check_bwd=True, seed=0, edge=256):
+def _sampled_fwd_bwd(B, S, W, n_random, k_rows, check_bwd=True, seed=0, edge=256, saved_pair=False):
     t = make_inputs(B, S, seed=seed, with_dout=check_bwd)
     d = _to_dev(t)
     out, lse = _gpu_fwd(d, window=W)
     gr = _gpu_bwd(d, out, lse, window=W) if check_bwd else None
+    if saved_pair:
+        # the training pair the benchmark times gives exactly these results at this size
+        sv = torch.empty(ga.zgcm_attn_saved_size(B, S, 32, 8, window=W), dtype=torch.uint8, device="cuda")
+        out_s, lse_s = _gpu_fwd(d, window=W, saved=sv)
+        assert torch.equal(out, out_s) and torch.equal(lse, lse_s)
+        gr_s = _gpu_bwd(d, out_s, lse_s, window=W, saved=sv)
+        for name in gr:
+            assert torch.equal(gr[name], gr_s[name]), name
+        del sv, out_s, lse_s, gr_s
     P = _problem(t, window=W)
     rows = sample_query_rows(B, S, n_random=n_random, edge=edge, seed=seed)
     b, i = rows // S, rows % S
@@ -392,7 +401,7 @@ def test_swa_16k_forward_backward():
     rng = np.random.default_rng(1)
     k_rows = np.unique(np.concatenate([np.arange(0, 64), np.arange(S * B - 64, S * B),
                                        rng.integers(0, B * S, 128)]))
-    _sampled_fwd_bwd(B, S, 128, n_random=512, k_rows=k_rows)
+    _sampled_fwd_bwd(B, S, 128, n_random=512, k_rows=k_rows, saved_pair=True)
 
 
 def test_global_64k_forward_backward():
@@ -400,7 +409,7 @@ def test_global_64k_forward_backward():
     oracle O(S) each, so fewer of them) + properties."""
     S = 65536
     k_rows = np.arange(S - 48, S)
-    _sampled_fwd_bwd(1, S, S, n_random=24, k_rows=k_rows, edge=12)
+    _sampled_fwd_bwd(1, S, S, n_random=24, k_rows=k_rows, edge=12, saved_pair=True)
 
 
 def test_256k_swa_and_global_forward():
