@@ -107,19 +107,25 @@ size_t bwd_q_glob_smem_bytes() { return sizeof(BwdQGlobSmem) + 1024; }
 template <bool MASK>
 __device__ __forceinline__ void qg_ds_chunk(const float* sv, const float* dv, uint32_t vm, float c2, float lse2,
                                             float kds, float dls, float (&ma)[2], uint32_t (&pk)[16]) {
+    // two keys per paired fp32 instruction
+    const float2 cc = make_float2(c2, c2), nl = make_float2(-lse2, -lse2);
+    const float2 kk = make_float2(kds, kds), nd = make_float2(-dls, -dls);
+    float2 acc = make_float2(ma[0], ma[1]);
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
-        const float s0 = sv[e], s1 = sv[e + 1];
-        float p0 = fast_exp2(fmaf(s0, c2, -lse2)), p1 = fast_exp2(fmaf(s1, c2, -lse2));
+        const float2 s = make_float2(sv[e], sv[e + 1]);
+        const float2 x = ffma2(s, cc, nl);
+        float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));
         if (MASK) {
-            p0 = ((vm >> e) & 1u) ? p0 : 0.f;  // (a masked score may overflow: selected away)
-            p1 = ((vm >> (e + 1)) & 1u) ? p1 : 0.f;
+            p.x = ((vm >> e) & 1u) ? p.x : 0.f;  // (a masked score may overflow: selected away)
+            p.y = ((vm >> (e + 1)) & 1u) ? p.y : 0.f;
         }
-        const float d0 = p0 * fmaf(dv[e], kds, -dls), d1 = p1 * fmaf(dv[e + 1], kds, -dls);
-        ma[0] = fmaf(d0, s0, ma[0]);
-        ma[1] = fmaf(d1, s1, ma[1]);
-        pk[e >> 1] = pack2<true>(d0, d1);
+        const float2 d = fmul2(p, ffma2(make_float2(dv[e], dv[e + 1]), kk, nd));
+        acc = ffma2(d, s, acc);
+        pk[e >> 1] = pack2<true>(d.x, d.y);
     }
+    ma[0] = acc.x;
+    ma[1] = acc.y;
 }
 
 __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid_constant__ BwdTcParams p) {
