@@ -354,20 +354,26 @@ __global__ void __launch_bounds__(FG_THREADS, 1) fwd_glob_tc_kernel(const __grid
             if (raise) m_ref = mt;
             l *= alpha;
             const float mb = m_ref == -INFINITY ? 0.f : m_ref;
-            float l4[4] = {0.f, 0.f, 0.f, 0.f};
+            // scores two at a time (paired fp32 instructions), the sum in two paired partials
+            const float2 cc = make_float2(c2, c2), nb = make_float2(-mb, -mb);
+            float2 la = make_float2(0.f, 0.f), lb = la;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float p0 = fast_exp2(fmaf(v[32 * c + e], c2, -mb));
-                    const float p1 = fast_exp2(fmaf(v[32 * c + e + 1], c2, -mb));
-                    l4[(e >> 1) & 3] += p0 + p1;
-                    pk[e >> 1] = pack_bf16(p0, p1);
+                for (int e = 0; e < 32; e += 4) {
+                    const float2 xa = ffma2(make_float2(v[32 * c + e], v[32 * c + e + 1]), cc, nb);
+                    const float2 xb = ffma2(make_float2(v[32 * c + e + 2], v[32 * c + e + 3]), cc, nb);
+                    const float2 pa = make_float2(fast_exp2(xa.x), fast_exp2(xa.y));
+                    const float2 pb = make_float2(fast_exp2(xb.x), fast_exp2(xb.y));
+                    la = fadd2(la, pa);
+                    lb = fadd2(lb, pb);
+                    pk[e >> 1] = pack_bf16(pa.x, pa.y);
+                    pk[(e >> 1) + 1] = pack_bf16(pb.x, pb.y);
                 }
                 tmem_st16(TM_S + lane_off + 16 * c, pk);
             }
-            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            l += (la.x + la.y) + (lb.x + lb.y);
             if (warp_raise && n > 0) {
                 // O_x holds PV_x(0..n-1), complete (S_x(n) was issued after PV_x(n-1))
 #pragma unroll 1
