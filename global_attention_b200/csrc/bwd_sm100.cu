@@ -2,7 +2,9 @@
 //
 // Exact gradients of L = sum(dout * out) for the ZGCM-1 layer (definition and page
 // citations in common.cuh), for windows W <= 128 and 42 rotated dims; other shapes run on
-// the warp-MMA kernels (bwd_mma.cu).  Three kernels:
+// the warp-MMA kernels (bwd_mma.cu).  The gate pass, the preparation passes (bwd_prep_kv,
+// bwd_prep_q: fp16 K~, V, Q~ with the rows' inverse RMS; bwd_prep_v alone when the forward
+// kept Q~ and K~) and the two score kernels:
 //
 //   bwd_gate   streaming pass over dout, g, out (coalesced, 16 lanes per row): the gate
 //              backward dg = dout*out*(1-sigmoid(g)), and dA = dout*sigmoid(g) stored as fp16

@@ -18,15 +18,18 @@
 //   S   = Q~ [K~_slot0; K~_slot1]^T          tcgen05.mma M=128 N=256 K=128, A,B in smem
 //                                            (fp16 q~, k~, the backward's operands, so the
 //                                            backward recomputes these scores bit for bit)
-//   P   = exp2(S*scale*log2e - max)          softmax warpgroup, thread = query row, fp32,
-//                                            written back as bf16 over the front of S
+//   P   = exp2(S*scale*log2e - m)            softmax warpgroup, thread = query row, fp32,
+//                                            written back as bf16 over the front of S; m is
+//                                            a bound on every score of the launch when that
+//                                            is small enough (one pass), else the row max
 //   O   = P [V_slot0; V_slot1]               tcgen05.mma M=128 N=128 K=256, A in TMEM,
 //                                            B (V, d-contiguous) MN-major in smem
 //   out = sigmoid(g) * O / l                 epilogue, 16-byte global loads/stores
 //
 // Warp roles (512 threads): w0 TMA K/V, w1 MMA issue + TMEM owner, w2 TMA Q, w3 idle,
-// w4-7 softmax, w8-11 prologue (Q~ in place), w12-15 gate epilogue.  Every wait is bounded;
-// on expiry the CTA records the site, drains, frees TMEM and returns.
+// w4-7 softmax, w8-11 prologue (Q~ in place; with save_q it also stores Q~ and the rows'
+// inverse RMS for the backward), w12-15 gate epilogue.  Every wait is bounded; on expiry
+// the CTA records the site, drains, frees TMEM and returns.
 #include <cudaTypedefs.h>
 
 #include "sm100.cuh"
