@@ -218,10 +218,12 @@ struct BwdQTcSmem {
     float dsinv[2][TF_BM];   // 2^-e of each dS row, by head number % 2
     float mdot[2][TF_BM];    // mean(dy gamma xhat) of each row (RMSNorm backward), by head % 2
     float dgq[4][kD];        // this CTA's d_gamma_q, one slice per epilogue warp
+    float2 cs[TF_HALF][TF_BM];  // epilogue: (cos, sin) of each row's rotated pairs, per step
     uint64_t bar[QB_COUNT];
     uint32_t tmem_base;
     int abort;
 };
+static_assert(sizeof(BwdQTcSmem) + 1024 <= 227 * 1024, "query-major shared memory over the 227 KB a CTA may use");
 
 // In-place fp16 conversion of a raw bf16 V tile by its 128 owner threads (thread r = row r;
 // the four warps of one warpgroup, named barrier 1), with one power-of-two scale for the whole
@@ -692,6 +694,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             const StepInfo st = decode_step(L, t, t_begin, t_end);
             const int i = st.qb * TF_BM + r;
             const bool valid = i < L.S;
+            // the row's rotation angles, shared by the G heads of the step (own column only)
+#pragma unroll 1
+            for (int q = 0; q < TF_HALF; ++q) rope_cs(L.theta[q], i, sm.cs[q][r].x, sm.cs[q][r].y);
             for (int h = 0; h < G; ++h, ++m) {
                 const int hg = st.kvh * G + h;
                 const size_t off = ((size_t)(st.b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hg) * kD;
@@ -713,7 +718,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                 const float mdot = sm.mdot[m & 1][r];
                 tc_fence_before();
                 mbar_arrive(&sm.bar[QB_DQEMPTY]);  // dQ(m) is in registers: TMEM free for dP(m+1)
-                row_rope_rms_backward_regs(dy, f, mdot, rinv, xv0, L.q + off, p.P.dq + off, valid, i, sm.gq, sm.dgq[wq], L);
+                row_rope_rms_backward_cs(dy, f, mdot, rinv, xv0, L.q + off, p.P.dq + off, valid,
+                                         [&](int q) { return sm.cs[q][r]; }, sm.gq, sm.dgq[wq]);
             }
         }
     }

@@ -99,10 +99,12 @@ __device__ __forceinline__ uint4* tile_chunk(unsigned char* h0, unsigned char* h
 // last 64 here.  d_gamma goes into this warp's slice `dgam` through warp-transposed sums
 // (lane L owns one dimension per 32-wide block: a fixed summation order, reproducible).
 // `valid` masks rows past the sequence (they still join the collectives).
-__device__ __forceinline__ void row_rope_rms_backward_regs(float (&dy)[128], float f, float mdot, float rinv,
-                                                           const uint4 (&xv0)[8], const bf16* x, bf16* dst,
-                                                           bool valid, int pos, const float* gamma, float* dgam,
-                                                           const LayerParams& L) {
+// cs_at(t): (cos, sin) of pair t at the row's position (rope_cs), so that a caller with
+// several heads of one row can form them once.
+template <class CsAt>
+__device__ __forceinline__ void row_rope_rms_backward_cs(float (&dy)[128], float f, float mdot, float rinv,
+                                                         const uint4 (&xv0)[8], const bf16* x, bf16* dst,
+                                                         bool valid, CsAt cs_at, const float* gamma, float* dgam) {
     const int lane = threadIdx.x & 31;
     const uint4* xr = reinterpret_cast<const uint4*>(x);
     uint4* dr = reinterpret_cast<uint4*>(dst);
@@ -111,8 +113,8 @@ __device__ __forceinline__ void row_rope_rms_backward_regs(float (&dy)[128], flo
     // transpose of the rotation of pairs (t, t + 21)
 #pragma unroll
     for (int t = 0; t < TF_HALF; ++t) {
-        float c, s;
-        rope_cs(L.theta[t], pos, c, s);
+        const float2 w = cs_at(t);
+        const float c = w.x, s = w.y;
         const float d1 = dy[t], d2 = dy[t + TF_HALF];
         dy[t] = d1 * c + d2 * s;
         dy[t + TF_HALF] = d2 * c - d1 * s;
@@ -142,6 +144,19 @@ __device__ __forceinline__ void row_rope_rms_backward_regs(float (&dy)[128], flo
         const float tot = warp_transpose_sum(v);
         dgam[32 * q + lane] += tot;
     }
+}
+
+__device__ __forceinline__ void row_rope_rms_backward_regs(float (&dy)[128], float f, float mdot, float rinv,
+                                                           const uint4 (&xv0)[8], const bf16* x, bf16* dst,
+                                                           bool valid, int pos, const float* gamma, float* dgam,
+                                                           const LayerParams& L) {
+    row_rope_rms_backward_cs(dy, f, mdot, rinv, xv0, x, dst, valid,
+                             [&](int t) {
+                                 float c, s;
+                                 rope_cs(L.theta[t], pos, c, s);
+                                 return make_float2(c, s);
+                             },
+                             gamma, dgam);
 }
 
 
