@@ -167,6 +167,34 @@ def test_rope_pairing_closed_form(oracle_mod):
     assert abs(y[42] - 1.0 / r) < 1e-12 and abs(y[127] - 2.0 / r) < 1e-12
 
 
+def test_score_bound_of_normalised_rows(oracle_mod):
+    """An RMS-normalised row has norm at most sqrt(D) before gamma (sum x^2 over mean x^2
+    + eps is at most D) and the rotation keeps norms, so every score is bounded by
+    |q~ . k~| <= D max|gamma_q| max|gamma_k|: the bound the sliding-window forward uses as
+    its softmax reference.  Random rows of any scale stay under it; one-hot rows in an
+    unrotated dimension with constant gamma and eps = 0 reach it exactly."""
+    D, R = 128, 42
+    t = _inputs(1, 4, 4, 1, D, seed=11)
+    gq, gk = t["gamma_q"].double().numpy(), t["gamma_k"].double().numpy()
+    P = _problem(oracle_mod, t, eps=1e-6)
+    bound = D * np.abs(gq).max() * np.abs(gk).max()
+    rng = np.random.default_rng(3)
+    worst = 0.0
+    for n in range(300):
+        x = rng.standard_normal(D) * (1e-3, 1.0, 1e3)[n % 3]
+        y = x + 0.1 * rng.standard_normal(D) if n % 2 else rng.standard_normal(D)
+        a, b = rng.integers(0, 262144, 2)
+        s = abs(float(np.dot(P.prologue_row(x, gq, int(a)), P.prologue_row(y, gk, int(b)))))
+        assert s <= bound * (1 + 1e-12)
+        worst = max(worst, s / bound)
+    assert worst > 0.05  # the random rows are not trivially far from the bound
+    cq, ck = 1.7, 0.6
+    P0 = _problem(oracle_mod, t, eps=0.0)
+    e = np.zeros(D); e[R + 5] = 3.0
+    s = float(np.dot(P0.prologue_row(e, np.full(D, cq), 77), P0.prologue_row(e, np.full(D, ck), 3)))
+    assert abs(s - D * cq * ck) < 1e-9 * D * cq * ck
+
+
 def test_rope_base_irrelevant_when_rotated_dims_are_zero(oracle_mod):
     t = _inputs(1, 50, 4, 1, 128, seed=10)
     for name in ("q", "k"):
