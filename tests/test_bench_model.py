@@ -1,0 +1,54 @@
+"""bench.py host logic on the CPU: the algorithmic byte model behind the roofline, and the
+lookup of ncu DRAM counters, which must ignore counters taken on another kernel source."""
+import hashlib
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+B, S = 4, 16384
+TOK = B * S
+QB = TOK * 32 * 128 * 2   # one [B,S,32,128] bf16 tensor
+KB = TOK * 8 * 128 * 2    # one [B,S,8,128] bf16 tensor
+LSE = TOK * 32 * 4
+
+
+def test_step_bytes_are_each_tensor_once():
+    """Forward: read q, k, v, g, write out, lse; backward: read q, k, v, g, out, dout, lse,
+    write dq, dk, dv, dg.  5.65e9 B at the 16K sliding workload: the roofline step."""
+    w = bench.work(B, S, 128, True)
+    assert w["fwd_bytes"] == 3 * QB + 2 * KB + LSE
+    assert w["bwd_bytes"] == 6 * QB + 4 * KB + LSE
+    assert w["fwd_bytes"] + w["bwd_bytes"] == pytest.approx(5.654e9, rel=1e-3)
+    assert bench.work(B, S, 128, False)["bwd_bytes"] == 0
+
+
+def test_kept_activations_change_kernels_not_the_step():
+    plain = bench.work(B, S, 128, True)
+    kept = bench.work(B, S, 128, True, saved=True)
+    # the forward that keeps q~ (fp16) and every q and k row's inverse RMS writes them once more
+    extra = QB + TOK * 32 * 4 + TOK * 8 * 4
+    assert kept["kernels"]["fwd_tc_kernel"][0] - plain["kernels"]["fwd_tc_kernel"][0] == extra
+    # the V-only preparation: read v, write V fp16 and a norm per row
+    assert kept["kernels"]["bwd_prep_v_kernel"][0] == 2 * KB + TOK * 8 * 4
+    # the roofline is the layer's, not this implementation's
+    assert (kept["fwd_bytes"], kept["bwd_bytes"]) == (plain["fwd_bytes"], plain["bwd_bytes"])
+
+
+def test_traffic_lookup_drops_counters_of_another_source(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    src = tmp_path / "k.cu"
+    src.write_text("kernel as captured")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    entry = {"kernel": "k", "workload": "w", "source": "k.cu", "source_sha": sha, "bytes_per_launch": 5.0}
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps([entry]))
+    assert bench.traffic_for("k", "w") == 5.0
+    assert bench.traffic_for("k", "other workload") is None
+    src.write_text("kernel changed since")
+    assert bench.traffic_for("k", "w") is None
