@@ -1,0 +1,105 @@
+"""Sequence sharding of the sliding-window layer (global_attention_b200.seqshard) as gloo
+process groups on the CPU: each rank computes its rows with the fp64 oracle through the
+halo exchange, and the results must equal the unsharded oracle on the whole sequence."""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _oracle_ops():
+    import oracle
+
+    def fwd(q, k, v, g, gq, gk, *, window, **kw):
+        out, lse = oracle.Problem(q, k, v, g, gq, gk, window=window, **kw).forward()
+        return torch.from_numpy(out), torch.from_numpy(lse)
+
+    def bwd(q, k, v, g, gq, gk, out, lse, dout, *, window, **kw):
+        r = oracle.Problem(q, k, v, g, gq, gk, window=window, **kw).backward(dout)
+        return {n: torch.from_numpy(x) for n, x in r.items()}
+
+    return fwd, bwd
+
+
+def _rank_main(rank, world, port, L, W, results):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    from datetime import timedelta
+    import oracle
+    from global_attention_b200 import seqshard
+    from global_attention_b200.synth import make_inputs
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=120))
+    try:
+        kw = dict(rope_dims=8, rope_base=10000.0)
+        B, Hq, Hkv, D = 2, 4, 2, 16
+        t = make_inputs(B, world * L, Hq=Hq, Hkv=Hkv, D=D, seed=21, with_dout=True)
+        rows = slice(rank * L, (rank + 1) * L)
+        mine = {n: t[n][:, rows].contiguous() for n in ("q", "k", "v", "g", "dout")}
+        ops = _oracle_ops()
+        out, lse, ctx = seqshard.halo_forward(mine["q"], mine["k"], mine["v"], mine["g"], t["gamma_q"],
+                                              t["gamma_k"], window=W, ops=ops, **kw)
+        gr = seqshard.halo_backward(ctx, mine["dout"], t["gamma_q"], t["gamma_k"], ops=ops)
+        # the whole sequence at once
+        P = oracle.Problem(t["q"], t["k"], t["v"], t["g"], t["gamma_q"], t["gamma_k"], window=W, **kw)
+        ref_out, ref_lse = P.forward()
+        ref = P.backward(t["dout"])
+        err = {
+            "out": np.abs(out.numpy() - ref_out[:, rows]).max(),
+            "lse": np.abs(lse.numpy() - ref_lse[:, :, rows]).max(),
+        }
+        for n in ("dq", "dk", "dv", "dg"):
+            err[n] = np.abs(gr[n].numpy() - ref[n][:, rows]).max()
+        for n in ("dgamma_q", "dgamma_k"):
+            err[n] = np.abs(gr[n].numpy() - ref[n]).max() / max(1.0, np.abs(ref[n]).max())
+        results[rank] = {k: float(v) for k, v in err.items()}
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,L,W", [(2, 24, 16), (3, 20, 16), (3, 15, 16), (2, 9, 1)])
+def test_halo_sharding_equals_whole_sequence(world, L, W):
+    """Ranks 0..world-1 each hold L rows; window W reaches W - 1 rows into the previous rank
+    (L = W - 1: exactly one whole rank of halo; W = 1: no halo, only the d_gamma sum).  Every
+    output and gradient equals the unsharded oracle to fp64 rounding (RoPE at shifted
+    positions differs only in the rounding of its angles)."""
+    mgr = mp.get_context("spawn").Manager()
+    results = mgr.dict()
+    mp.spawn(_rank_main, args=(world, _free_port(), L, W, results), nprocs=world, join=True)
+    assert len(results) == world
+    for rank in range(world):
+        for name, e in results[rank].items():
+            assert e < 1e-9, (rank, name, e)
+
+
+def test_halo_needs_window_rows_per_rank():
+    """A rank with fewer than W - 1 rows would need rows of two ranks back: refused."""
+    sys.path.insert(0, ROOT)
+    from global_attention_b200 import seqshard
+
+    class _G:  # a two-rank group seen from rank 1, without a process group
+        pass
+
+    orig = dist.get_rank, dist.get_world_size
+    try:
+        dist.get_rank = lambda group=None: 1
+        dist.get_world_size = lambda group=None: 2
+        x = torch.zeros(1, 10, 4, 16, dtype=torch.bfloat16)
+        with pytest.raises(ValueError):
+            seqshard.halo_forward(x, x[:, :, :2], x[:, :, :2], x, torch.ones(16), torch.ones(16), window=16,
+                                  ops=(None, None))
+    finally:
+        dist.get_rank, dist.get_world_size = orig
