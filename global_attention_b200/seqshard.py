@@ -1,5 +1,5 @@
-"""Sequence-sharded sliding-window layer: one long sequence split over the ranks of a process
-group, rank r holding positions [r L, (r + 1) L) of every batch row.
+"""Sequence-sharded layer: one long sequence split over the ranks of a process group, rank r
+holding positions [r L, (r + 1) L) of every batch row.
 
 A sliding window of W keys reaches W - 1 rows back, so each rank needs only the last W - 1
 key and value rows of the rank before it (a halo).  The forward receives that halo and runs
@@ -19,6 +19,13 @@ contribute nothing to any gradient.  The exchange is one send and one receive of
 2 (W - 1) B Hkv D values per rank and direction (torch.distributed point-to-point: NCCL over
 NVLink on GPUs, gloo on the CPU); there is no collective on the data path except the sum of
 d_gamma (2 x D values).
+
+A window longer than a rank's rows (the global layer, W >= S, among them) reaches further
+back: gathered_forward / gathered_backward gather every rank's key and value rows, run the
+layer on the rows the window reaches ([start, (r + 1) L), start = max(0, r L - (W - 1)),
+numbered from 0) with zero query rows before this rank's, and return the earlier rows' key
+gradients to their owners through one sum over the ranks.  The zero query rows are computed
+and dropped: a kernel that takes a first query row would skip that work.
 
 The compute is a pair of callables with the signatures of zgcm_attn_fwd / zgcm_attn_bwd of
 this package (the default); the tests pass others to check the sharding on the CPU.
@@ -107,6 +114,69 @@ def halo_backward(ctx, dout, gamma_q, gamma_k, *, group=None, ops=None):
                 tail = res[n][:, L - hw:]
                 acc = torch.float64 if tail.dtype == torch.float64 else torch.float32
                 res[n][:, L - hw:] = (tail.to(acc) + got[i].to(acc)).to(tail.dtype)
+    dgam = torch.stack([gr["dgamma_q"], gr["dgamma_k"]]).contiguous()
+    if world > 1:
+        dist.all_reduce(dgam, group=group)
+    res["dgamma_q"], res["dgamma_k"] = dgam[0], dgam[1]
+    return res
+
+
+def gathered_forward(q, k, v, g, gamma_q, gamma_k, *, window, group=None, ops=None, **kw):
+    """Forward of this rank's rows for any window: the key and value rows of the earlier
+    ranks that the window reaches are gathered (all ranks' rows travel; each keeps what it
+    needs).  Shapes as halo_forward; every rank has the same L."""
+    fwd, _ = ops or _default_ops()
+    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    B, L = q.shape[0], q.shape[1]
+    start = max(0, rank * L - (window - 1))
+    h = rank * L - start
+    if world == 1 or h == 0:
+        out, lse = fwd(q, k, v, g, gamma_q, gamma_k, window=window, **kw)
+        kv_all = None
+        if world > 1:  # the others still gather: take part with this rank's rows
+            kv_all = [torch.empty_like(torch.stack([k, v])) for _ in range(world)]
+            dist.all_gather(kv_all, torch.stack([k, v]).contiguous(), group=group)
+        return out, lse, HaloContext(0, (q, k, v, g), out, lse, window, dict(kw, _start=start))
+    kv_all = [torch.empty_like(torch.stack([k, v])) for _ in range(world)]
+    dist.all_gather(kv_all, torch.stack([k, v]).contiguous(), group=group)
+    before = torch.cat(kv_all[:rank], 2)[:, :, start:]  # [2, B, h, Hkv, D]
+    zq = torch.zeros((B, h) + tuple(q.shape[2:]), dtype=q.dtype, device=q.device)
+    ext = (torch.cat([zq, q], 1).contiguous(), torch.cat([before[0], k], 1).contiguous(),
+           torch.cat([before[1], v], 1).contiguous(), torch.cat([zq, g], 1).contiguous())
+    out_ext, lse_ext = fwd(*ext, gamma_q, gamma_k, window=window, **kw)
+    return (out_ext[:, h:].contiguous(), lse_ext[:, :, h:].contiguous(),
+            HaloContext(h, ext, out_ext, lse_ext, window, dict(kw, _start=start)))
+
+
+def gathered_backward(ctx, dout, gamma_q, gamma_k, *, group=None, ops=None):
+    """Backward of gathered_forward: this rank's dq, dk, dv, dg and the whole sequence's
+    dgamma_q, dgamma_k.  The key and value gradients of all rows are summed over the ranks
+    (each rank contributes the rows its window reached) and each keeps its own."""
+    _, bwd = ops or _default_ops()
+    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    kw = dict(ctx.kw)
+    start = kw.pop("_start")
+    h = ctx.h
+    q, k, v, g = ctx.ext
+    if h > 0:
+        zd = torch.zeros((dout.shape[0], h) + tuple(dout.shape[2:]), dtype=dout.dtype, device=dout.device)
+        dout = torch.cat([zd, dout], 1).contiguous()
+    gr = bwd(q, k, v, g, gamma_q, gamma_k, ctx.out_ext, ctx.lse_ext, dout, window=ctx.window, **kw)
+    res = {n: gr[n][:, h:].contiguous() for n in ("dq", "dg")}
+    L = res["dq"].shape[1]
+    dk_ext, dv_ext = gr["dk"], gr["dv"]
+    if world > 1:
+        acc = torch.float64 if dk_ext.dtype == torch.float64 else torch.float32
+        B = dk_ext.shape[0]
+        full = torch.zeros((2, B, world * L) + tuple(dk_ext.shape[2:]), dtype=acc, device=dk_ext.device)
+        full[0, :, start:(rank + 1) * L] = dk_ext.to(acc)
+        full[1, :, start:(rank + 1) * L] = dv_ext.to(acc)
+        dist.all_reduce(full, group=group)
+        mine = full[:, :, rank * L:(rank + 1) * L]
+        res["dk"] = mine[0].to(dk_ext.dtype).contiguous()
+        res["dv"] = mine[1].to(dv_ext.dtype).contiguous()
+    else:
+        res["dk"], res["dv"] = dk_ext[:, h:].contiguous(), dv_ext[:, h:].contiguous()
     dgam = torch.stack([gr["dgamma_q"], gr["dgamma_k"]]).contiguous()
     if world > 1:
         dist.all_reduce(dgam, group=group)

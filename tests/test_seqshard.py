@@ -1,6 +1,7 @@
-"""Sequence sharding of the sliding-window layer (global_attention_b200.seqshard) as gloo
-process groups on the CPU: each rank computes its rows with the fp64 oracle through the
-halo exchange, and the results must equal the unsharded oracle on the whole sequence."""
+"""Sequence sharding of the layer (global_attention_b200.seqshard) as gloo process groups on
+the CPU: each rank computes its rows with the fp64 oracle through the halo exchange (sliding
+windows) or the gathered earlier rows (any window, the global layer among them), and the
+results must equal the unsharded oracle on the whole sequence."""
 import os
 import socket
 import sys
@@ -34,7 +35,7 @@ def _oracle_ops():
     return fwd, bwd
 
 
-def _rank_main(rank, world, port, L, W, results):
+def _rank_main(rank, world, port, L, W, results, mode="halo"):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     from datetime import timedelta
@@ -50,9 +51,11 @@ def _rank_main(rank, world, port, L, W, results):
         rows = slice(rank * L, (rank + 1) * L)
         mine = {n: t[n][:, rows].contiguous() for n in ("q", "k", "v", "g", "dout")}
         ops = _oracle_ops()
-        out, lse, ctx = seqshard.halo_forward(mine["q"], mine["k"], mine["v"], mine["g"], t["gamma_q"],
-                                              t["gamma_k"], window=W, ops=ops, **kw)
-        gr = seqshard.halo_backward(ctx, mine["dout"], t["gamma_q"], t["gamma_k"], ops=ops)
+        fwd = seqshard.halo_forward if mode == "halo" else seqshard.gathered_forward
+        bwd = seqshard.halo_backward if mode == "halo" else seqshard.gathered_backward
+        out, lse, ctx = fwd(mine["q"], mine["k"], mine["v"], mine["g"], t["gamma_q"], t["gamma_k"], window=W,
+                            ops=ops, **kw)
+        gr = bwd(ctx, mine["dout"], t["gamma_q"], t["gamma_k"], ops=ops)
         # the whole sequence at once
         P = oracle.Problem(t["q"], t["k"], t["v"], t["g"], t["gamma_q"], t["gamma_k"], window=W, **kw)
         ref_out, ref_lse = P.forward()
@@ -85,14 +88,27 @@ def test_halo_sharding_equals_whole_sequence(world, L, W):
             assert e < 1e-9, (rank, name, e)
 
 
+@pytest.mark.parametrize("world,L,W", [(2, 16, 10**6), (3, 12, 36), (3, 10, 16), (3, 12, 8), (2, 9, 1)])
+def test_gathered_sharding_equals_whole_sequence(world, L, W):
+    """Windows that reach past the previous rank: the global layer (W >= the whole sequence),
+    W - 1 >= 2 L (every earlier row), and L = 10, W = 16, where rank 2's window covers rank 1
+    and rows 5..9 of rank 0; a short window and W = 1 take the same path.  Every output and
+    gradient equals the unsharded oracle to fp64 rounding."""
+    mgr = mp.get_context("spawn").Manager()
+    results = mgr.dict()
+    mp.spawn(_rank_main, args=(world, _free_port(), L, W, results, "gathered"), nprocs=world, join=True)
+    assert len(results) == world
+    for rank in range(world):
+        for name, e in results[rank].items():
+            assert e < 1e-9, (rank, name, e)
+
+
 def test_halo_needs_window_rows_per_rank():
     """A rank with fewer than W - 1 rows would need rows of two ranks back: refused."""
     sys.path.insert(0, ROOT)
     from global_attention_b200 import seqshard
 
-    class _G:  # a two-rank group seen from rank 1, without a process group
-        pass
-
+    # a two-rank group seen from rank 1, without a process group
     orig = dist.get_rank, dist.get_world_size
     try:
         dist.get_rank = lambda group=None: 1
