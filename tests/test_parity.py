@@ -296,6 +296,34 @@ def test_bounded_wait_expires_and_is_reported():
     assert_bf16_close("out after the expired wait", out, ref_out)
 
 
+def test_halo_rows_match_whole_sequence():
+    """The premise of the sliding layer's sequence sharding on the CUDA kernels: the rows of
+    a chunk computed from [the previous W - 1 key/value rows; the chunk], with zero query and
+    gate rows under the halo and positions numbered from 0, equal the same rows of the
+    whole-sequence call (outputs, lse, dq, dg, and dk, dv of the rows no later chunk sees)."""
+    B, L, W, R = 2, 640, 128, 3
+    t = make_inputs(B, R * L, seed=61, with_dout=True)
+    d = _to_dev(t)
+    out, lse = _gpu_fwd(d, window=W)
+    gr = _gpu_bwd(d, out, lse, window=W)
+    h = W - 1
+    for r in range(1, R):
+        a, s0, e = r * L - h, r * L, (r + 1) * L
+        zq = torch.zeros_like(d["q"][:, :h])
+        ext = dict(q=torch.cat([zq, d["q"][:, s0:e]], 1).contiguous(), k=d["k"][:, a:e].contiguous(),
+                   v=d["v"][:, a:e].contiguous(), g=torch.cat([zq, d["g"][:, s0:e]], 1).contiguous(),
+                   gamma_q=d["gamma_q"], gamma_k=d["gamma_k"],
+                   dout=torch.cat([zq, d["dout"][:, s0:e]], 1).contiguous())
+        o, l = _gpu_fwd(ext, window=W)
+        assert_bf16_close(f"out[{r}]", o[:, h:], f64(out)[:, s0:e])
+        assert_lse_close(f"lse[{r}]", l[:, :, h:], f64(lse)[:, :, s0:e])
+        g2 = _gpu_bwd(ext, o, l, window=W)
+        for n in ("dq", "dg"):
+            assert_bf16_close(f"{n}[{r}]", g2[n][:, h:], f64(gr[n])[:, s0:e])
+        for n in ("dk", "dv"):  # rows the next chunk's queries do not see
+            assert_bf16_close(f"{n}[{r}]", g2[n][:, h:L], f64(gr[n])[:, s0:e - h])
+
+
 def test_empty_problem():
     for B, S in ((0, 16), (2, 0)):
         t = make_inputs(max(B, 1), max(S, 1), with_dout=True)
