@@ -324,6 +324,61 @@ def test_halo_rows_match_whole_sequence():
             assert_bf16_close(f"{n}[{r}]", g2[n][:, h:L], f64(gr[n])[:, s0:e - h])
 
 
+def test_training_step_in_a_cuda_graph():
+    """The calls are stream-ordered, never synchronise and allocate nothing when given their
+    buffers, so a training step (the pair that keeps activations) captures into a CUDA graph;
+    a replay gives exactly the eager results, also after new inputs are copied in."""
+    B, S, W = 2, 1000, 128
+    d = _to_dev(make_inputs(B, S, seed=71, with_dout=True))
+    sv = torch.empty(ga.zgcm_attn_saved_size(B, S, 32, 8, window=W), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(ga.zgcm_attn_bwd_workspace_size(B, S, 32, 8, 128, W), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(d["q"])
+    lse = torch.empty((B, 32, S), dtype=torch.float32, device="cuda")
+    grads = dict(dq=torch.empty_like(d["q"]), dk=torch.empty_like(d["k"]), dv=torch.empty_like(d["v"]),
+                 dg=torch.empty_like(d["g"]), dgamma_q=torch.empty(128, device="cuda"),
+                 dgamma_k=torch.empty(128, device="cuda"))
+
+    def step():
+        ga.zgcm_attn_fwd(d["q"], d["k"], d["v"], d["g"], d["gamma_q"], d["gamma_k"], window=W, out=out,
+                         lse=lse, saved=sv)
+        ga.zgcm_attn_bwd(d["q"], d["k"], d["v"], d["g"], d["gamma_q"], d["gamma_k"], out, lse, d["dout"],
+                         window=W, grads=grads, workspace=ws, saved=sv)
+
+    def results():
+        return [out.clone(), lse.clone()] + [grads[n].clone() for n in sorted(grads)]
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()  # eager, outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    eager = results()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for x in [out, lse] + list(grads.values()):
+        x.fill_(float("nan"))
+    graph.replay()
+    torch.cuda.synchronize()
+    assert ga.zgcm_attn_device_error() == 0
+    for a, b in zip(eager, results()):
+        assert torch.equal(a, b)
+    # new inputs in the same buffers: the replay follows them
+    d2 = _to_dev(make_inputs(B, S, seed=72, with_dout=True))
+    for n in d:
+        d[n].copy_(d2[n])
+    graph.replay()
+    torch.cuda.synchronize()
+    replayed = results()
+    step()
+    torch.cuda.synchronize()
+    assert ga.zgcm_attn_device_error() == 0
+    for a, b in zip(replayed, results()):
+        assert torch.equal(a, b)
+    del graph
+
+
 def test_empty_problem():
     for B, S in ((0, 16), (2, 0)):
         t = make_inputs(max(B, 1), max(S, 1), with_dout=True)
