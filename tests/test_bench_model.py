@@ -52,3 +52,21 @@ def test_traffic_lookup_drops_counters_of_another_source(tmp_path, monkeypatch):
     assert bench.traffic_for("k", "other workload") is None
     src.write_text("kernel changed since")
     assert bench.traffic_for("k", "w") is None
+
+
+def _row(sm, reasons=()):
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    flags = ["Active" if n in reasons else "Not Active" for n in names]
+    return ["0", str(sm), "1965", "900.0", "0x0"] + flags
+
+
+def test_clock_summary_median_and_reasons():
+    """The clocks record of the JSON line: median SM clock over the samples, the maximum, and
+    every throttle reason seen active (a run showing a hardware or thermal one is re-taken)."""
+    cs = bench.ClockSampler("GPU-test")
+    cs.rows = [_row(1965), _row(1320, ("sw_power_cap",)), _row(1500, ("sw_power_cap",)), ["malformed"], []]
+    assert cs.summary() == {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    cs.rows = [_row(1100, ("hw_slowdown",)), _row(1200, ("sw_thermal_slowdown", "sw_power_cap"))]
+    assert cs.summary()["reasons"] == ["hw_slowdown", "sw_power_cap", "sw_thermal_slowdown"]
+    cs.rows = []
+    assert cs.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
