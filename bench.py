@@ -230,42 +230,60 @@ def pair_scaled(secs, B, S, W, S_full, W_full):
     return secs / (B * pairs(S, W)) * pairs(S_full, W_full) / S_full
 
 
-def cpu_sample_shape(Bw, Sw, W):
-    """A bounded sample of the workload for the oracle: same heads and window, fewer and
-    shorter sequences (window work per token is the same once past the first W tokens)."""
+# The oracle's bounded sample of one layer, shared by the reference arm (one sample per step)
+# and the GPU arm's cpu_baseline (samples until about 10 s of CPU time): same heads and
+# window as the workload, fewer and shorter sequences.  The oracle's work is proportional to
+# the visible (query, key) pairs, so a sample's time per pair scales to the workload's pairs
+# per token (a sliding layer past its first W tokens has the same pairs per token).
+ORACLE_SAMPLE_TOKENS = {"sliding": 4096, "global": 1024}
+
+
+def oracle_sample_shape(Sw, W):
     if W >= Sw:            # global layer: a shorter causal sequence
-        return 1, 2048, 2048
-    return 8, 8192, W
+        n = ORACLE_SAMPLE_TOKENS["global"]
+        return 1, n, n
+    return 1, ORACLE_SAMPLE_TOKENS["sliding"], W
+
+
+def oracle_sample(workload, seed=0):
+    """One sample of a whole step of `workload` on the fp64 oracle (every layer of the step,
+    each on its own sample).  Returns (seconds per workload token, seconds it took, text)."""
+    Bw, Sw, W, bwd = WORKLOADS[workload]
+    spt, took, parts = 0.0, 0.0, []
+    for lw, _ in layers_of(workload):
+        Bc, Sc, Wc = oracle_sample_shape(Sw, lw)
+        secs = cpu_oracle_run(Bc, Sc, Wc, bwd, seed=seed)
+        spt += pair_scaled(secs, Bc, Sc, Wc, Sw, lw)
+        took += secs
+        parts.append(f"{Bc}x{Sc} tokens, window {Wc}")
+    text = ("; ".join(parts) + f" per sample, fwd{'+bwd' if bwd else ''} in fp64; time per visible (query, key) "
+            "pair scaled to the workload's pairs per token")
+    return spt, took, text
 
 
 def run_reference(args):
-    """--impl reference: the fp64 CPU oracle as it stands, each step a bounded sample."""
+    """--impl reference: the fp64 CPU oracle as it stands, each step one bounded sample of the
+    workload (oracle_sample); the value is the workload's tokens/s at the sampled rate."""
     _, rank, _ = rank_env()
     if rank != 0:
         return 0
     import oracle
     oracle.build()
     Bw, Sw, W, bwd = WORKLOADS[args.workload]
-    # one sample per layer of the step: (B, S, window) with every layer's window kept
-    shapes = [(1, 512, 512) if lw >= Sw else (1, 1024, lw) for lw, _ in layers_of(args.workload)]
-
-    def one(seed=0):   # seconds per token of a whole step
-        return sum(pair_scaled(cpu_oracle_run(B, S, Wc, bwd, seed=seed), B, S, Wc, Sw, lw)
-                   for (B, S, Wc), (lw, _) in zip(shapes, layers_of(args.workload)))
-
-    for _ in range(args.warmup):
-        one()
-    spt = sum(one(seed=i) for i in range(args.steps)) / args.steps
+    for i in range(args.warmup):
+        oracle_sample(args.workload, seed=i)
+    runs = [oracle_sample(args.workload, seed=i) for i in range(args.steps)]
+    spt = sum(r[0] for r in runs) / len(runs)
     val = 1.0 / spt
-    ms = 1e3 * Bw * Sw * spt          # the workload's step at this rate
     cores = oracle.num_threads()
-    sample = "; ".join(f"{B}x{S} tokens, window {Wc}" for B, S, Wc in shapes)
-    sample += (f" per step, fwd{'+bwd' if bwd else ''}, fp64, {cores} threads; time per visible (query, key) "
-               "pair scaled to the workload's pairs per token")
+    sample = runs[0][2] + f"; {cores} threads"
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "steps": args.steps, "warmup": args.warmup,
+        # what one timed step (one sample) took; the workload's own step at this rate is scaled
+        "ms_per_step": 1e3 * sum(r[1] for r in runs) / len(runs),
+        "workload_ms_per_step_scaled": 1e3 * Bw * Sw * spt,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_name(args.workload), "sample": sample},
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -450,56 +468,19 @@ def decode_cpu_baseline(P, layers):
             "sample": "; ".join(parts) + " (the oracle's per-row forward, fp64, including its prologue)"}
 
 
-def run_probe_ex2(args):
-    """The MUFU exp2 rate of this GPU (the softmax kernels' exponential), at full occupancy
-    and with one warp per SM sub-partition; prints one JSON line."""
-    import torch
-    import global_attention_b200 as ga
-    lib = ga.load()
-    dev = torch.device("cuda", 0)
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    stream = torch.cuda.current_stream()
-    res = {}
-    for name, blocks, threads in (("full", sms * 8, 256), ("one_warp_per_smsp", sms, 128)):
-        iters = 4096
-        out = torch.empty(blocks * threads, dtype=torch.float32, device=dev)
-        call = lambda: lib.zgcm_attn_probe_ex2(ctypes.c_void_p(out.data_ptr()), blocks, threads, iters,
-                                               ctypes.c_void_p(stream.cuda_stream))
-        for _ in range(3):
-            assert call() == 0
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) as clk:
-            e0.record(stream)
-            for _ in range(args.steps):
-                assert call() == 0
-            e1.record(stream)
-            torch.cuda.synchronize()
-        secs = e0.elapsed_time(e1) / 1e3 / args.steps
-        n = blocks * threads * iters * 8
-        c = clk.summary()
-        mhz = c["sm_mhz"] or c["sm_max_mhz"] or 1965.0
-        res[name] = {"ex2_per_s": n / secs, "ex2_per_clock_per_sm": n / secs / (sms * mhz * 1e6),
-                     "ms": secs * 1e3, "sm_mhz": mhz}
-    print(json.dumps({"probe": "MUFU ex2.approx.ftz.f32 rate", "sms": sms, **res}))
-    return 0
-
-
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + ["probe_ex2"],
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS),
                     default="swa16k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=8)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.workload == "probe_ex2":
-        return run_probe_ex2(args)
     if args.workload in DECODE_WORKLOADS:
         if args.impl == "reference":
             _, rank, _ = rank_env()
@@ -707,16 +688,13 @@ def main():
     if world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        # seconds per token of each layer of the step, each on its own bounded sample
-        spt, parts = 0.0, []
-        for lw, _ in layers:
-            Bc, Sc, Wc = cpu_sample_shape(Bw, Sw, lw)
-            secs = cpu_oracle_run(Bc, Sc, Wc, bwd)
-            spt += pair_scaled(secs, Bc, Sc, Wc, Sw, lw)
-            parts.append(f"{Bc}x{Sc} tokens, window {Wc}, fwd{'+bwd' if bwd else ''} in fp64 ({secs:.1f} s)")
-        cpu = {"value": 1.0 / spt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-               "sample": "; ".join(parts) + "; same heads as the workload, time per visible (query, key) "
-                         "pair scaled to the workload's pairs per token"}
+        # the reference arm's samples (oracle_sample), repeated until about 10 s of CPU time
+        runs, took = [], 0.0
+        while took < 10.0 and len(runs) < 64:
+            runs.append(oracle_sample(args.workload, seed=len(runs)))
+            took += runs[-1][1]
+        cpu = {"value": len(runs) / sum(r[0] for r in runs), "unit": "tokens/s", "cores": oracle.num_threads(),
+               "kind": "oracle", "sample": f"{len(runs)} samples of " + runs[0][2] + f" ({took:.1f} s in all)"}
 
     # per layer: the forward's kernels (each tcgen05 forward runs the key preparation kernel
     # first; the wide-window one, keeping its activations, also the query preparation) + every

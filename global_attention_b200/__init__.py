@@ -73,8 +73,6 @@ def load() -> ctypes.CDLL:
         lib.zgcm_attn_bwd_saved.restype = i
         lib.zgcm_attn_fwd_kernel_name.argtypes = [i, i, i, i, i, i]
         lib.zgcm_attn_fwd_kernel_name.restype = ctypes.c_char_p
-        lib.zgcm_attn_probe_ex2.argtypes = [vp, i, i, i, vp]
-        lib.zgcm_attn_probe_ex2.restype = i
         lib.zgcm_attn_selftest_expired_wait.argtypes = [vp]
         lib.zgcm_attn_selftest_expired_wait.restype = i
         lib.zgcm_attn_device_error.argtypes = []
@@ -100,12 +98,36 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _check(t, name, dtype, ndim):
+def _check(t, name, dtype, ndim, cuda=True):
     import torch
-    if not isinstance(t, torch.Tensor) or not t.is_cuda:
-        raise TypeError(f"{name} must be a CUDA tensor")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
     if t.dtype != dtype or t.dim() != ndim or not t.is_contiguous():
         raise TypeError(f"{name} must be a contiguous {dtype} tensor of rank {ndim}")
+    if cuda and not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+
+
+def _check_bwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, dout, grads):
+    """Dtype, rank, layout and device of every backward tensor, before any launch."""
+    import torch
+    for n, t in (("q", q), ("k", k), ("v", v), ("g", g), ("out", out), ("dout", dout)):
+        _check(t, n, torch.bfloat16, 4, cuda=False)
+    _check(lse, "lse", torch.float32, 3, cuda=False)
+    _check(gamma_q, "gamma_q", torch.float32, 1, cuda=False)
+    _check(gamma_k, "gamma_k", torch.float32, 1, cuda=False)
+    if grads is not None:
+        for n, ref in (("dq", q), ("dk", k), ("dv", v), ("dg", g)):
+            _check(grads[n], n, torch.bfloat16, 4, cuda=False)
+            if grads[n].shape != ref.shape:
+                raise TypeError(f"{n} must have the shape of its input {tuple(ref.shape)}")
+        for n in ("dgamma_q", "dgamma_k"):
+            _check(grads[n], n, torch.float32, 1, cuda=False)
+    tensors = [q, k, v, g, gamma_q, gamma_k, out, lse, dout] + ([] if grads is None else list(grads.values()))
+    if not all(t.is_cuda for t in tensors):
+        raise TypeError("every tensor must be a CUDA tensor")
+    if any(t.device != q.device for t in tensors):
+        raise TypeError("every tensor must be on the device of q")
 
 
 def zgcm_attn_fwd_workspace_size(B, S, Hq, Hkv, D=128, rope_dims=42, window=128) -> int:
@@ -244,13 +266,11 @@ def zgcm_attn_bwd(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dims=42,
     a list of (begin, end) torch.cuda.Event pairs, brackets the backward's kernels in launch
     order (zgcm_attn_bwd_timed; names from zgcm_attn_bwd_kernel_names)."""
     import torch
+    _check_bwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, dout, grads)
     B, S, Hq, D = q.shape
     Hkv = k.shape[2]
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    for n, t in (("q", q), ("k", k), ("v", v), ("g", g), ("out", out), ("dout", dout)):
-        _check(t, n, torch.bfloat16, 4)
-    _check(lse, "lse", torch.float32, 3)
     if grads is None:
         grads = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
                      dg=torch.empty_like(g),
@@ -294,8 +314,11 @@ def zgcm_attn_bwd_noalloc(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_
                           window=128, causal=1, eps=1e-6, scale=None, grads=None, stream=None):
     """zgcm_attn_bwd without a workspace: for callers that cannot allocate device memory,
     the library's fixed 64 MiB per-device scratch array is used instead (problems needing
-    more raise ZgcmError with ZGCM_ERR_TOO_LARGE).  Calls that overlap on the GPU race."""
+    more raise ZgcmError with ZGCM_ERR_TOO_LARGE: at 32/8 heads and a window of at most 128,
+    B*S <= 3117 tokens fit).  The call runs with q's device current, so the array used is
+    that device's.  Calls that overlap on the GPU race."""
     import torch
+    _check_bwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, dout, grads)
     B, S, Hq, D = q.shape
     Hkv = k.shape[2]
     if scale is None:
@@ -305,11 +328,13 @@ def zgcm_attn_bwd_noalloc(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_
                      dg=torch.empty_like(g),
                      dgamma_q=torch.empty(D, dtype=torch.float32, device=q.device),
                      dgamma_k=torch.empty(D, dtype=torch.float32, device=q.device))
-    st = load().zgcm_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma_q), _ptr(gamma_k),
-                                      _ptr(out), _ptr(lse), _ptr(dout), B, S, Hq, Hkv, D, int(rope_dims),
-                                      float(rope_base), int(window), int(causal), float(eps), float(scale),
-                                      _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]), _ptr(grads["dg"]),
-                                      _ptr(grads["dgamma_q"]), _ptr(grads["dgamma_k"]), _stream(stream))
+    with torch.cuda.device(q.device):
+        st = load().zgcm_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma_q), _ptr(gamma_k),
+                                          _ptr(out), _ptr(lse), _ptr(dout), B, S, Hq, Hkv, D, int(rope_dims),
+                                          float(rope_base), int(window), int(causal), float(eps), float(scale),
+                                          _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]),
+                                          _ptr(grads["dg"]), _ptr(grads["dgamma_q"]), _ptr(grads["dgamma_k"]),
+                                          _stream(stream))
     if st != ZGCM_OK:
         raise ZgcmError(st, "zgcm_attn_bwd_noalloc")
     return grads

@@ -11,7 +11,9 @@
 // process exits.  Every call on a device shares it and it keeps the last call's contents:
 // the backward writes every scratch word it later reads (nothing in it must start at zero),
 // and two calls whose executions overlap on the GPU — on different streams, or from
-// different host threads — race on it.
+// different host threads — race on it.  The array used is the one of the calling thread's
+// current device, so the tensors and the stream must belong to that device (a call whose q
+// lives on another device is rejected with ZGCM_ERR_INVALID_ARG).
 #include <mutex>
 
 #include "../../include/zgcm_attn.h"
@@ -59,6 +61,16 @@ extern "C" int zgcm_attn_bwd_noalloc(const void* q, const void* k, const void* v
     if (need > kScratchBytes) return ZGCM_ERR_TOO_LARGE;
     void* ws = nullptr;
     if ((long long)B * S > 0) {
+        const void* ptrs[] = {q, k, v, g, gamma_q, gamma_k, out, lse, dout, dq, dk, dv, dg, dgamma_q, dgamma_k};
+        for (const void* p : ptrs)
+            if (!p) return ZGCM_ERR_INVALID_ARG;
+        // The scratch used is the current device's: the tensors must live there too.
+        int dev = 0;
+        cudaPointerAttributes attr;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaPointerGetAttributes(&attr, q) != cudaSuccess)
+            return ZGCM_ERR_CUDA;
+        if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) return ZGCM_ERR_INVALID_ARG;
+        if (attr.device != dev) return ZGCM_ERR_INVALID_ARG;
         int st = ZGCM_OK;
         ws = scratch_address(&st);
         if (st != ZGCM_OK) return st;

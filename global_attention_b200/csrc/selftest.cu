@@ -32,36 +32,3 @@ cudaError_t launch_selftest_expired_wait(int* err_word, cudaStream_t stream) {
 }
 
 }  // namespace zgcm
-
-// ------------------------------------------------------------------ MUFU exp2 rate probe
-
-namespace zgcm {
-
-// Each thread runs `iters` rounds of 8 independent exp2 chains (ex2.approx, the instruction
-// the softmax kernels use) and stores their sum, so nothing is optimised away: 8 * iters
-// exponentials per thread.  With enough warps the rate is the MUFU unit's throughput; with
-// one warp per SM sub-partition it is one warp's latency-bound rate.
-__global__ void probe_ex2_kernel(float* out, int iters) {
-    float a[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) a[k] = -1.0f - 0.001f * (threadIdx.x & 7) - 0.01f * k;
-    for (int it = 0; it < iters; ++it) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            float y;
-            asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(a[k]));
-            a[k] = y - 1.5f;  // stays in (-1.5, -0.5): a bounded, data-dependent chain
-        }
-    }
-    float s = 0.f;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) s += a[k];
-    out[blockIdx.x * blockDim.x + threadIdx.x] = s;
-}
-
-cudaError_t launch_probe_ex2(float* out, int blocks, int threads, int iters, cudaStream_t stream) {
-    probe_ex2_kernel<<<blocks, threads, 0, stream>>>(out, iters);
-    return cudaGetLastError();
-}
-
-}  // namespace zgcm

@@ -18,7 +18,6 @@ cudaError_t launch_fwd_glob_tc(const FwdParams& p, void* workspace, int* err_wor
 bool fwd_glob_supported(const LayerParams& L);
 size_t decode_workspace_bytes(int B, int Hq, int window, int C);
 cudaError_t launch_selftest_expired_wait(int* err_word, cudaStream_t stream);
-cudaError_t launch_probe_ex2(float* out, int blocks, int threads, int iters, cudaStream_t stream);
 cudaError_t launch_decode(const LayerParams& L, const int* pos, void* k_cache, void* v_cache, int C, void* out,
                           float* lse, void* workspace, cudaStream_t stream);
 size_t fwd_glob_workspace_bytes(int B, int S, int Hkv);
@@ -330,13 +329,6 @@ int zgcm_attn_decode(const void* q, const void* k, const void* v, const void* g,
 
 int zgcm_attn_selftest_expired_wait(void* cuda_stream) {
     return launch_selftest_expired_wait(device_error_word(), static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess
-               ? ZGCM_OK
-               : ZGCM_ERR_CUDA;
-}
-
-int zgcm_attn_probe_ex2(float* out, int blocks, int threads, int iters, void* cuda_stream) {
-    if (!out || blocks < 1 || threads < 32 || threads > 1024 || (threads & 31) || iters < 1) return ZGCM_ERR_INVALID_ARG;
-    return launch_probe_ex2(out, blocks, threads, iters, static_cast<cudaStream_t>(cuda_stream)) == cudaSuccess
                ? ZGCM_OK
                : ZGCM_ERR_CUDA;
 }

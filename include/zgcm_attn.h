@@ -214,8 +214,12 @@ int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void*
  * scratch array that lives in the library's device image on every GPU that loads the
  * library, until the process exits.  It allocates nothing.
  *
- * Limit: problems whose zgcm_attn_bwd_workspace_size exceeds 64 MiB (about 4K tokens
- * at 32 query heads) return ZGCM_ERR_TOO_LARGE before anything runs.
+ * Limit: problems whose zgcm_attn_bwd_workspace_size exceeds 64 MiB return
+ * ZGCM_ERR_TOO_LARGE before anything runs; at 32 query / 8 KV heads, D = 128 and a
+ * window of at most 128 that is B*S <= 3117 tokens (3118 is rejected).
+ * Device: the array used is the calling thread's current device's, so q (and every other
+ * tensor, and the stream) must be on the current device; a q that lives elsewhere returns
+ * ZGCM_ERR_INVALID_ARG.  Null tensor pointers return ZGCM_ERR_INVALID_ARG.
  * The first call on a device looks up the array's device address (once per device).
  * All calls on a device share the array, which keeps the last call's contents; every
  * scratch word is written before it is read, so nothing needs clearing.  Calls whose
@@ -291,14 +295,6 @@ int zgcm_attn_device_error(void);
  * ZGCM_ERR_TIMEOUT and the context stays usable.  Asynchronous on `cuda_stream`.
  */
 int zgcm_attn_selftest_expired_wait(void* cuda_stream);
-
-/*
- * Diagnostic: runs blocks x threads threads of `iters` rounds of 8 independent exp2 chains
- * (the MUFU instruction of the softmax kernels), 8 * iters exponentials per thread, and
- * writes one float per thread to `out` (device, blocks * threads floats).  Timed by the
- * caller, it measures the exponential rate the softmax kernels are budgeted against.
- */
-int zgcm_attn_probe_ex2(float* out, int blocks, int threads, int iters, void* cuda_stream);
 
 /* Name of the i-th kernel zgcm_attn_bwd launches for this configuration (static string),
  * or NULL when i is past the last one.  With 42 rotated dims, windows up to 128 run the

@@ -226,3 +226,49 @@ def test_decode_checks(lib):
         assert _dec(lib, need, ptrs=p) == -1
         p = list(good); p[i] = good[i] + 4
         assert _dec(lib, need, ptrs=p) == -3
+
+
+def _noalloc(lib, B, S, W=128):
+    null = [ctypes.c_void_p(0)] * 16
+    return lib.zgcm_attn_bwd_noalloc(*null[:9], B, S, 32, 8, 128, 42, 10000.0, W, 1, 1e-6, 0.0883883,
+                                     *null[9:16])
+
+
+def test_noalloc_size_bound(lib):
+    """The no-allocation backward takes every problem whose workspace fits its 64 MiB array and
+    rejects the rest with ZGCM_ERR_TOO_LARGE (-7) before looking at anything else; at 32/8
+    heads and a window of 128 the bound is B*S = 3117 tokens (the figure the header states)."""
+    lim = 64 << 20
+    ws = lambda B, S: lib.zgcm_attn_bwd_workspace_size(B, S, 32, 8, 128, 128)
+    s_ok = max(S for S in range(3000, 3300) if ws(1, S) <= lim)
+    assert s_ok == 3117
+    # accepted by the size check: the null tensor pointers are what it then rejects (-1)
+    assert _noalloc(lib, 1, s_ok) == -1
+    assert _noalloc(lib, 1, s_ok + 1) == -7
+    assert _noalloc(lib, 4, 16384) == -7
+
+
+def test_noalloc_binding_checks_before_any_launch(monkeypatch):
+    """The Python wrapper checks dtype, rank, layout and device of every tensor before it
+    reaches the C entry point: a float32 or a transposed q never gets to a kernel."""
+    import torch
+    from global_attention_b200.synth import make_inputs
+    reached = []
+
+    class NoLib:
+        def __getattr__(self, name):
+            reached.append(name)
+            raise AssertionError(f"reached the library ({name})")
+
+    monkeypatch.setattr(ga, "load", lambda: NoLib())
+    t = make_inputs(1, 8, with_dout=True)
+    lse = torch.zeros((1, 32, 8), dtype=torch.float32)
+    args = dict(q=t["q"], k=t["k"], v=t["v"], g=t["g"], gamma_q=t["gamma_q"], gamma_k=t["gamma_k"],
+                out=t["q"].clone(), lse=lse, dout=t["dout"])
+    for bad in (dict(q=t["q"].float()), dict(q=t["q"].transpose(1, 2)), dict(lse=lse.double()),
+                dict(gamma_k=t["gamma_k"].half()), dict(dout=t["dout"][:, :, :, :64])):
+        with pytest.raises(TypeError, match="contiguous"):
+            ga.zgcm_attn_bwd_noalloc(**dict(args, **bad))
+    with pytest.raises(TypeError, match="CUDA"):
+        ga.zgcm_attn_bwd_noalloc(**args)
+    assert not reached

@@ -488,11 +488,54 @@ def test_swa_16k_forward_backward():
 
 
 def test_global_64k_forward_backward():
-    """Global layer: B=1, S=65536, W=S, sampled rows (rows late in the sequence cost the
-    oracle O(S) each, so fewer of them) + properties."""
+    """Global layer: B=1, S=65536, W=S, sampled rows + properties.  A query row late in the
+    sequence costs the oracle O(S); a key row j needs the softmax statistics of every query
+    row after it, O(S^2) for an early key, so only the last keys are affordable here.  The
+    heaviest key tiles of the global backward (those that accumulate over the most query
+    blocks) are compared in test_global_8k_heaviest_key_tiles."""
     S = 65536
     k_rows = np.arange(S - 48, S)
-    _sampled_fwd_bwd(1, S, S, n_random=24, k_rows=k_rows, edge=12, saved_pair=True)
+    _sampled_fwd_bwd(1, S, S, n_random=96, k_rows=k_rows, edge=16, saved_pair=True)
+
+
+def test_global_8k_heaviest_key_tiles():
+    """Global layer at S=8192: dk and dv of the first three key tiles (rows 0..383), the units
+    of the key-major kernel that accumulate over the most query blocks (64, 63, 62 blocks of
+    128 queries x 4 heads) and run first on its heaviest-first schedule; plus sampled query rows."""
+    S = 8192
+    k_rows = np.arange(0, 384)
+    _sampled_fwd_bwd(1, S, S, n_random=64, k_rows=k_rows, edge=32, saved_pair=True, seed=3)
+
+
+def test_swa_16k_every_element():
+    """The headline workload compared in full: B=4, S=16384, W=128, every element of out, lse,
+    dq, dk, dv, dg and both d_gamma against the oracle's full forward and backward, computed by
+    the training pair the benchmark times (the forward keeping its activations)."""
+    import psutil
+    if psutil.virtual_memory().available < 48e9:
+        pytest.skip("needs ~30 GB of host RAM for the fp64 oracle arrays at B=4, S=16384")
+    B, S, W = 4, 16384, 128
+    t = make_inputs(B, S, seed=0, with_dout=True)
+    d = _to_dev(t)
+    sv = torch.empty(ga.zgcm_attn_saved_size(B, S, 32, 8, window=W), dtype=torch.uint8, device="cuda")
+    out, lse = _gpu_fwd(d, window=W, saved=sv)
+    gr = _gpu_bwd(d, out, lse, window=W, saved=sv)
+    got = {"out": out.cpu(), "lse": lse.cpu(), **{n: x.cpu() for n, x in gr.items()}}
+    del d, sv, out, lse, gr
+    P = _problem(t, window=W)
+    ref_out, ref_lse = P.forward()
+    for b in range(B):
+        assert_bf16_close(f"out[b={b}]", got["out"][b], ref_out[b])
+    assert_lse_close("lse", got["lse"], ref_lse)
+    del ref_out, ref_lse
+    ref = P.backward(t["dout"])
+    for n in ("dq", "dk", "dv", "dg"):
+        for b in range(B):
+            assert_bf16_close(f"{n}[b={b}]", got[n][b], ref[n][b])
+        # and over the whole tensor (rel-RMS of the full gradient)
+        assert_bf16_close(n, got[n], ref[n])
+    assert_dgamma_close("dgamma_q", got["dgamma_q"], ref["dgamma_q"])
+    assert_dgamma_close("dgamma_k", got["dgamma_k"], ref["dgamma_k"])
 
 
 def test_256k_swa_and_global_forward():

@@ -44,7 +44,8 @@ def _gpu():
 
 
 def test_noalloc_matches_workspace_backward_on_consecutive_calls():
-    for call, (B, S, W, seed) in enumerate(((1, 1000, 128, 11), (2, 700, 128, 12))):
+    # the last call is the largest problem the 64 MiB array takes at 32/8 heads and W = 128
+    for call, (B, S, W, seed) in enumerate(((1, 1000, 128, 11), (2, 700, 128, 12), (1, 3117, 128, 13))):
         t = make_inputs(B, S, seed=seed, with_dout=True)
         d = {k: v.cuda() for k, v in t.items()}
         out, lse = ga.zgcm_attn_fwd(d["q"], d["k"], d["v"], d["g"], d["gamma_q"], d["gamma_k"], window=W)
