@@ -107,6 +107,9 @@ def work(B, S, W, bwd, saved=False):
     keep = (qb + tok * HQ * 4 + tok * HKV * 4) if saved else 0
     kernels = {
         "fwd_mma_kernel": (fwd_bytes, fwd_flops),
+        # q, k, v, g -> out, lse (keys normalised in shared memory); keeping its activations it
+        # also writes q~ and k~ fp16 and each q and k row's inverse RMS
+        "fwd_strip_kernel": (fwd_bytes + (keep + kb if saved else 0), fwd_flops),
         "fwd_tc_kernel": (fwd_bytes + keep, fwd_flops),
         # tcgen05 forwards: q, K~16 (fp16, prepared from k by fwd_prep_k_kernel), v, g -> out, lse
         "fwd_glob_tc_kernel": (fwd_bytes + keep, fwd_flops),
@@ -126,6 +129,8 @@ def work(B, S, W, bwd, saved=False):
         # given the forward's q~, k~: v -> V fp16 (+ v norm per row, V scale per tile)
         "bwd_prep_v_kernel": (2 * kb + kb // (D // 2), 0),
         "bwd_q_tc_kernel": (4 * qb + 2 * kb + 3 * lse, 6 * D * npair),
+        # the same reads and writes, by strips of 32 positions x 4 heads
+        "bwd_strip_q_kernel": (4 * qb + 2 * kb + 3 * lse, 6 * D * npair),
         "bwd_kv_tc_kernel": (2 * qb + 5 * kb + 4 * lse, 8 * D * npair),
     }
     return dict(tokens=tok, npair=npair, fwd_bytes=fwd_bytes, fwd_flops=fwd_flops,
@@ -702,7 +707,8 @@ def main():
     fwd_launches = []
     for (lw, _), kp in zip(layers, keep):
         fname = ga.zgcm_attn_fwd_kernel_name(Bw, Sw, HQ, HKV, 42, lw)
-        fwd_launches.append(1 if fname == "fwd_mma_kernel" else 3 if kp and fname == "fwd_glob_tc_kernel" else 2)
+        fwd_launches.append(1 if fname in ("fwd_mma_kernel", "fwd_strip_kernel")
+                            else 3 if kp and fname == "fwd_glob_tc_kernel" else 2)
     launches_per_step = sum(f + len(n) for f, n in zip(fwd_launches, bwd_names))
     rec = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,

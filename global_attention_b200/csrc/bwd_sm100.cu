@@ -1242,12 +1242,12 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_b() {
 }
 
 bool make_map_b(CUtensorMap* map, const void* base, int H, int S, int B,
-                CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, int box_rows = 128) {
+                CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, int box_rows = 128, int box_heads = 1) {
     auto enc = get_encode_b();
     if (!enc) return false;
     cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)S * H * kD * 2};
-    cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+    cuuint32_t box[4] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(map, dtype, 4, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1284,6 +1284,16 @@ extern const char* const kBwdTcSavedKernelNames[] = {"bwd_gate_kernel",  "bwd_pr
                                                      "bwd_q_tc_kernel",  "bwd_kv_tc_kernel",
                                                      "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"};
 extern const int kBwdTcSavedKernelCount = 6;
+// 4 query heads per KV head: the query side runs by strips of positions
+extern const char* const kBwdStripKernelNames[] = {"bwd_gate_kernel",         "bwd_prep_kv_kernel",
+                                                   "bwd_prep_q_kernel",       "bwd_strip_q_kernel",
+                                                   "bwd_kv_tc_kernel",        "dgamma_reduce_kernel(k)",
+                                                   "dgamma_reduce_kernel(q)"};
+extern const int kBwdStripKernelCount = 7;
+extern const char* const kBwdStripSavedKernelNames[] = {"bwd_gate_kernel",  "bwd_prep_v_kernel",
+                                                        "bwd_strip_q_kernel", "bwd_kv_tc_kernel",
+                                                        "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"};
+extern const int kBwdStripSavedKernelCount = 6;
 extern const char* const kBwdWideSavedKernelNames[] = {"bwd_gate_kernel",   "bwd_prep_v_kernel",
                                                        "bwd_tile_stats_kernel", "bwd_q_glob_kernel",
                                                        "bwd_kv_tc_kernel",  "dgamma_reduce_kernel(k)",
@@ -1405,7 +1415,11 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
         !make_map_b(&p.tm_q16h, q16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 64) ||
         !make_map_b(&p.tm_dah, da16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 64) ||
         !make_map_rows(&p.tm_lse, p.lse2p, L.Hq, Spad, L.B) || !make_map_rows(&p.tm_delta, p.P.delta, L.Hq, Spad, L.B) ||
-        !make_map_rows(&p.tm_dainv, p.dainv, L.Hq, Spad, L.B))
+        !make_map_rows(&p.tm_dainv, p.dainv, L.Hq, Spad, L.B) ||
+        !make_map_b(&p.tm_q16s, q16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 32, 4 < L.Hq ? 4 : L.Hq) ||
+        !make_map_b(&p.tm_das, da16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 32, 4 < L.Hq ? 4 : L.Hq) ||
+        !make_map_b(&p.tm_k16c, k16, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 32) ||
+        !make_map_b(&p.tm_v16c, v16, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 32))
         return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1496,9 +1510,26 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
         dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgq_part, (int)units_q, bp.dgamma_q);
         return after(i);
     }
-    if ((e = before(i)) != cudaSuccess) return e;
-    bwd_q_tc_kernel<<<grid, TB_THREADS, smem_q, stream>>>(p);
-    if ((e = after(i++)) != cudaSuccess) return e;
+    int grid_q = grid;
+    if (bwd_strip_supported(L)) {
+        // the query side by strips of 32 positions x the group's 4 heads
+        const int strips = bwd_strip_total(L);
+        if (strips < 0) return cudaErrorInvalidValue;
+        const size_t smem_s = bwd_strip_smem_bytes();
+        if ((e = cudaFuncSetAttribute(bwd_strip_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s)) !=
+            cudaSuccess)
+            return e;
+        grid_q = strips < sms ? strips : sms;
+        BwdTcParams ps = p;
+        ps.total = strips;
+        if ((e = before(i)) != cudaSuccess) return e;
+        bwd_strip_q_kernel<<<grid_q, TB_THREADS, smem_s, stream>>>(ps);
+        if ((e = after(i++)) != cudaSuccess) return e;
+    } else {
+        if ((e = before(i)) != cudaSuccess) return e;
+        bwd_q_tc_kernel<<<grid, TB_THREADS, smem_q, stream>>>(p);
+        if ((e = after(i++)) != cudaSuccess) return e;
+    }
     if ((e = before(i)) != cudaSuccess) return e;
     bwd_kv_tc_kernel<false><<<grid, TB_THREADS, smem_k, stream>>>(p);
     if ((e = after(i++)) != cudaSuccess) return e;
@@ -1506,7 +1537,7 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgk_part, grid, bp.dgamma_k);
     if ((e = after(i++)) != cudaSuccess) return e;
     if ((e = before(i)) != cudaSuccess) return e;
-    dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgq_part, grid, bp.dgamma_q);
+    dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgq_part, grid_q, bp.dgamma_q);
     return after(i);
 }
 

@@ -115,7 +115,7 @@ __device__ __forceinline__ float tf_prologue_row_at(unsigned char* h0, unsigned 
         }
     }
     // a zero row (outside the sequence, zero-filled by TMA) stays zero even with eps = 0
-    const float rinv1 = ss > 0.f ? rsqrtf(ss * (1.0f / kD) + L.eps) : 0.f;
+    const float rinv1 = ss > 0.f ? rsqrtf(fmaf(ss, 1.0f / kD, L.eps)) : 0.f;
     const float rinv = rinv1 * oscale;
     // dims 0..47 (chunks 0..5): normalise, rotate the first 42
     float y[48];
@@ -131,12 +131,15 @@ __device__ __forceinline__ float tf_prologue_row_at(unsigned char* h0, unsigned 
             y[d + 1] = (f.y * rinv) * gamma[d + 1];
         }
     }
+    // explicit fused multiply-adds (here and in the mean square above): every kernel that forms
+    // q~ or k~ (the forwards, the backward's preparation, the strip kernels' in-place
+    // conversion) rounds identically, whatever contraction the compiler would pick at each site
 #pragma unroll
     for (int t = 0; t < TF_HALF; ++t) {
         const float a = y[t], bb = y[t + TF_HALF];
         const float2 w = cs_at(t);
-        y[t] = a * w.x - bb * w.y;
-        y[t + TF_HALF] = bb * w.x + a * w.y;
+        y[t] = fmaf(a, w.x, -(bb * w.y));
+        y[t + TF_HALF] = fmaf(bb, w.x, a * w.y);
     }
 #pragma unroll
     for (int ch = 0; ch < 6; ++ch) {

@@ -13,6 +13,8 @@ cudaError_t launch_fwd_mma(const FwdParams& p, cudaStream_t stream);
 cudaError_t launch_fwd_tc(const FwdParams& p, void* workspace, int* err_word, cudaStream_t stream,
                           const SavedAct* sv);
 bool fwd_tc_supported(const LayerParams& L);
+cudaError_t launch_fwd_strip(const FwdParams& fp, int* err_word, cudaStream_t stream, const SavedAct* sv);
+bool fwd_strip_supported(const LayerParams& L);
 cudaError_t launch_fwd_glob_tc(const FwdParams& p, void* workspace, int* err_word, cudaStream_t stream,
                                const SavedAct* sv);
 bool fwd_glob_supported(const LayerParams& L);
@@ -28,6 +30,11 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
                           void* const* events, int n_pairs, const SavedAct* sv);
 extern const char* const kBwdTcSavedKernelNames[];
 extern const int kBwdTcSavedKernelCount;
+extern const char* const kBwdStripKernelNames[];
+extern const int kBwdStripKernelCount;
+extern const char* const kBwdStripSavedKernelNames[];
+extern const int kBwdStripSavedKernelCount;
+bool bwd_strip_supported(const LayerParams& L);
 extern const char* const kBwdWideSavedKernelNames[];
 extern const int kBwdWideSavedKernelCount;
 bool bwd_tc_supported(const LayerParams& L);
@@ -63,12 +70,14 @@ bool force_mma() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Forward kernel for a layer: the sliding-window tcgen05 kernel (W <= 128), the wide-window /
-// global tcgen05 pair (W > 128), else (or with ZGCM_FORCE_MMA=1) the warp-MMA kernel.
-enum class FwdPath { TC, GLOB, MMA };
+// Forward kernel for a layer: the strip kernel (W <= 128, 4 query heads per KV head), the
+// sliding-window tcgen05 kernel (W <= 128, other group sizes), the wide-window / global
+// tcgen05 pair (W > 128), else (or with ZGCM_FORCE_MMA=1) the warp-MMA kernel.
+enum class FwdPath { STRIP, TC, GLOB, MMA };
 
 FwdPath fwd_path(const LayerParams& L) {
     if (force_mma()) return FwdPath::MMA;
+    if (fwd_strip_supported(L)) return FwdPath::STRIP;
     if (fwd_tc_supported(L)) return FwdPath::TC;
     if (fwd_glob_supported(L)) return FwdPath::GLOB;
     return FwdPath::MMA;
@@ -188,10 +197,10 @@ const char* zgcm_status_string(int status) {
 size_t zgcm_attn_fwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int rope_dims, int window) {
     if (check_shape(B, S, Hq, Hkv, D, rope_dims, 1.0, window, 1, 0.f, 1.f) != ZGCM_OK) return 0;
     if ((long long)B * S == 0) return 0;
-    // both tcgen05 forwards read K~ (fp16, normalised and rotated once per key tile) from it
-    return fwd_path(shape_only(B, S, Hq, Hkv, rope_dims, window)) != FwdPath::MMA
-               ? align256(fwd_glob_workspace_bytes(B, S, Hkv))
-               : 0;
+    // the tcgen05 forwards other than the strip kernel read K~ (fp16, normalised and rotated
+    // once per key tile) from it; the strip kernel normalises its key chunks in shared memory
+    const FwdPath f = fwd_path(shape_only(B, S, Hq, Hkv, rope_dims, window));
+    return (f == FwdPath::TC || f == FwdPath::GLOB) ? align256(fwd_glob_workspace_bytes(B, S, Hkv)) : 0;
 }
 
 }  // extern "C"
@@ -235,6 +244,7 @@ int zgcm_attn_fwd_ws(const void* q, const void* k, const void* v, const void* g,
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     cudaError_t e;
     switch (fwd_path(p.L)) {
+        case FwdPath::STRIP: e = launch_fwd_strip(p, device_error_word(), stream, nullptr); break;
         case FwdPath::TC: e = launch_fwd_tc(p, workspace, device_error_word(), stream, nullptr); break;
         case FwdPath::GLOB: e = launch_fwd_glob_tc(p, workspace, device_error_word(), stream, nullptr); break;
         default: e = launch_fwd_mma(p, stream); break;
@@ -291,9 +301,10 @@ int zgcm_attn_fwd_save(const void* q, const void* k, const void* v, const void* 
     p.out = static_cast<bf16*>(out);
     p.lse = lse;
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-    const cudaError_t e = fwd_path(p.L) == FwdPath::TC
-                              ? launch_fwd_tc(p, sv.k16, device_error_word(), stream, &sv)
-                              : launch_fwd_glob_tc(p, sv.k16, device_error_word(), stream, &sv);
+    const FwdPath f = fwd_path(p.L);
+    const cudaError_t e = f == FwdPath::STRIP ? launch_fwd_strip(p, device_error_word(), stream, &sv)
+                          : f == FwdPath::TC  ? launch_fwd_tc(p, sv.k16, device_error_word(), stream, &sv)
+                                              : launch_fwd_glob_tc(p, sv.k16, device_error_word(), stream, &sv);
     return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
 }
 
@@ -342,6 +353,7 @@ int zgcm_attn_device_error(void) {
 
 const char* zgcm_attn_fwd_kernel_name(int B, int S, int Hq, int Hkv, int rope_dims, int window) {
     switch (fwd_path(shape_only(B, S, Hq, Hkv, rope_dims, window))) {
+        case FwdPath::STRIP: return "fwd_strip_kernel";
         case FwdPath::TC: return "fwd_tc_kernel";
         case FwdPath::GLOB: return "fwd_glob_tc_kernel";
         default: return "fwd_mma_kernel";
@@ -457,10 +469,13 @@ int zgcm_attn_bwd_saved(const void* q, const void* k, const void* v, const void*
 
 const char* zgcm_attn_bwd_saved_kernel_name(int i, int S, int rope_dims, int window) {
     LayerParams L{};
-    L.B = 1; L.S = S; L.rope_half = rope_dims / 2; L.W = window;
+    L.B = 1; L.S = S; L.rope_half = rope_dims / 2; L.W = window; L.G = 4;
     const char* const* names = nullptr;
     int n = 0;
-    if (!force_mma() && S >= 1 && bwd_tc_supported(L)) {
+    if (!force_mma() && S >= 1 && bwd_strip_supported(L)) {
+        names = kBwdStripSavedKernelNames;
+        n = kBwdStripSavedKernelCount;
+    } else if (!force_mma() && S >= 1 && bwd_tc_supported(L)) {
         names = kBwdTcSavedKernelNames;
         n = kBwdTcSavedKernelCount;
     } else if (!force_mma() && S >= 1 && bwd_wide_supported(L)) {
@@ -472,10 +487,13 @@ const char* zgcm_attn_bwd_saved_kernel_name(int i, int S, int rope_dims, int win
 
 const char* zgcm_attn_bwd_kernel_name(int i, int S, int rope_dims, int window) {
     LayerParams L{};
-    L.B = 1; L.S = S; L.rope_half = rope_dims / 2; L.W = window;
+    L.B = 1; L.S = S; L.rope_half = rope_dims / 2; L.W = window; L.G = 4;
     const char* const* names = kBwdMmaKernelNames;
     int n = kBwdMmaKernelCount;
-    if (!force_mma() && S >= 1 && bwd_tc_supported(L)) {
+    if (!force_mma() && S >= 1 && bwd_strip_supported(L)) {
+        names = kBwdStripKernelNames;
+        n = kBwdStripKernelCount;
+    } else if (!force_mma() && S >= 1 && bwd_tc_supported(L)) {
         names = kBwdTcKernelNames;
         n = kBwdTcKernelCount;
     } else if (!force_mma() && S >= 1 && bwd_wide_supported(L)) {

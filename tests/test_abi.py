@@ -122,12 +122,17 @@ def _fwd_ws(lib, ws, ws_bytes, **kw):
 
 def test_fwd_workspace_size_query(lib):
     ws = lambda *a: lib.zgcm_attn_fwd_workspace_size(*a)
-    # both tcgen05 forwards (sliding windows and wider ones, the global layer among them) read
-    # the fp16 normalised keys, [B, S, Hkv, D]
-    for B, S, W in ((4, 16384, 128), (1, 1024, 7), (1, 65536, 65536), (2, 1000, 300), (1, 1, 10**6),
-                    (3, 777, 129)):
+    # the sliding layer (W <= 128, 4 query heads per KV head) needs none: the strip kernel
+    # normalises its key chunks in shared memory, so zgcm_attn_fwd allocates nothing there
+    for B, S, W in ((4, 16384, 128), (1, 1024, 7), (1, 1, 128), (2, 1000, 1)):
+        assert ws(B, S, 32, 8, 128, 42, W) == 0
+    # wider windows (the global layer among them) read the fp16 normalised keys, [B, S, Hkv, D],
+    # prepared once per key tile
+    for B, S, W in ((1, 65536, 65536), (2, 1000, 300), (1, 1, 10**6), (3, 777, 129)):
         n = B * S * 8 * 128 * 2
         assert ws(B, S, 32, 8, 128, 42, W) == (n + 255) // 256 * 256
+    # other group sizes of the sliding layer take the per-head tcgen05 kernel, which reads them too
+    assert ws(1, 1024, 16, 8, 128, 42, 128) == (1024 * 8 * 256 + 255) // 256 * 256
     # the warp-MMA kernel takes the rest (no rotation, odd group size) and needs none
     assert ws(1, 1024, 32, 8, 128, 0, 1024) == 0
     assert ws(1, 1024, 24, 8, 128, 42, 1024) == 0
@@ -194,7 +199,7 @@ def test_saved_pair_checks(lib):
     assert _bwd_saved(lib, ws - 1, store, need) == -4     # the workspace is checked as before
     assert _bwd_saved(lib, ws, store, need, rope_dims=0) == -2
     names = ga.zgcm_attn_bwd_kernel_names(16384, 128, saved=True)
-    assert names[:4] == ["bwd_gate_kernel", "bwd_prep_v_kernel", "bwd_q_tc_kernel", "bwd_kv_tc_kernel"]
+    assert names[:4] == ["bwd_gate_kernel", "bwd_prep_v_kernel", "bwd_strip_q_kernel", "bwd_kv_tc_kernel"]
     assert "bwd_prep_q_kernel" not in ga.zgcm_attn_bwd_kernel_names(4096, 4096, saved=True)
 
 

@@ -34,6 +34,9 @@ def test_kept_activations_change_kernels_not_the_step():
     # the forward that keeps q~ (fp16) and every q and k row's inverse RMS writes them once more
     extra = QB + TOK * 32 * 4 + TOK * 8 * 4
     assert kept["kernels"]["fwd_tc_kernel"][0] - plain["kernels"]["fwd_tc_kernel"][0] == extra
+    # the strip forward normalises its keys in shared memory and, keeping them, writes k~ too
+    assert kept["kernels"]["fwd_strip_kernel"][0] - plain["kernels"]["fwd_strip_kernel"][0] == extra + KB
+    assert plain["kernels"]["fwd_strip_kernel"][0] == plain["fwd_bytes"]
     # the V-only preparation: read v, write V fp16 and a norm per row
     assert kept["kernels"]["bwd_prep_v_kernel"][0] == 2 * KB + TOK * 8 * 4
     # the roofline is the layer's, not this implementation's

@@ -60,6 +60,9 @@ SMALL = [
     (1, 777, 32, 8, 777, 42, 1e4),       # global layer (W = S), ragged
     (1, 500, 16, 4, 10**6, 0, 1e4),      # global, W >> S, no rotation
     (3, 260, 32, 8, 200, 42, 1e4),       # window between one and two tiles
+    (2, 45, 4, 1, 128, 42, 1e4),         # strips: one KV head, sequences of 1.4 strips
+    (5, 77, 32, 8, 100, 42, 1e4),        # strips: one strip per CTA, every span loaded whole
+    (1, 3000, 16, 8, 128, 42, 1e4),      # two query heads per KV head: per-head tcgen05 kernel
 ]
 
 
@@ -84,13 +87,13 @@ def test_small_full_compare(B, S, Hq, Hkv, W, R, base):
 @pytest.mark.parametrize("B,S,W", [(1, 1024, 128), (2, 1000, 128), (1, 129, 7), (3, 260, 1), (1, 1, 128),
                                    (2, 384, 100)])
 def test_forward_both_kernel_paths(B, S, W, monkeypatch):
-    """The tcgen05 sliding-window kernel (default for W <= 128, 42 rotated dims) and the
-    warp-MMA kernel (forced) both match the oracle on the same inputs."""
+    """The tcgen05 strip kernel (default for W <= 128, 4 query heads per KV head, 42 rotated
+    dims) and the warp-MMA kernel (forced) both match the oracle on the same inputs."""
     t = make_inputs(B, S, seed=100 + S + W)
     d = _to_dev(t)
     ref_out, ref_lse = _problem(t, window=W).forward()
     monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
-    assert ga.zgcm_attn_fwd_kernel_name(B, S, 32, 8, 42, W) == "fwd_tc_kernel"
+    assert ga.zgcm_attn_fwd_kernel_name(B, S, 32, 8, 42, W) == "fwd_strip_kernel"
     out_tc, lse_tc = _gpu_fwd(d, window=W)
     assert ga.zgcm_attn_device_error() == 0
     monkeypatch.setenv("ZGCM_FORCE_MMA", "1")
@@ -120,7 +123,7 @@ def test_forward_score_bound_fallback(gq_all, spike, B, S, W, monkeypatch):
     d = _to_dev(t)
     ref_out, ref_lse = _problem(t, window=W).forward()
     monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
-    assert ga.zgcm_attn_fwd_kernel_name(B, S, 32, 8, 42, W) == "fwd_tc_kernel"
+    assert ga.zgcm_attn_fwd_kernel_name(B, S, 32, 8, 42, W) == "fwd_strip_kernel"
     out, lse = _gpu_fwd(d, window=W)
     assert ga.zgcm_attn_device_error() == 0
     assert_bf16_close("out", out, ref_out)
@@ -164,7 +167,7 @@ def test_backward_both_kernel_paths(B, S, W, monkeypatch):
     ref = _problem(t, window=W).backward(t["dout"])
     monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
     assert ga.zgcm_attn_bwd_kernel_names(S, W)[:5] == ["bwd_gate_kernel", "bwd_prep_kv_kernel", "bwd_prep_q_kernel",
-                                                        "bwd_q_tc_kernel", "bwd_kv_tc_kernel"]
+                                                        "bwd_strip_q_kernel", "bwd_kv_tc_kernel"]
     out, lse = _gpu_fwd(d, window=W)
     got_tc = _gpu_bwd(d, out, lse, window=W)
     assert ga.zgcm_attn_device_error() == 0
