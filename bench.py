@@ -707,7 +707,8 @@ def main():
     fwd_launches = []
     for (lw, _), kp in zip(layers, keep):
         fname = ga.zgcm_attn_fwd_kernel_name(Bw, Sw, HQ, HKV, 42, lw)
-        fwd_launches.append(1 if fname in ("fwd_mma_kernel", "fwd_strip_kernel")
+        # the strip forward keeping its activations runs the two preparation kernels first
+        fwd_launches.append(1 if fname == "fwd_mma_kernel" else (3 if kp else 1) if fname == "fwd_strip_kernel"
                             else 3 if kp and fname == "fwd_glob_tc_kernel" else 2)
     launches_per_step = sum(f + len(n) for f, n in zip(fwd_launches, bwd_names))
     rec = {

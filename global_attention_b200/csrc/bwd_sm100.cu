@@ -968,15 +968,13 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                     tc_fence_after();
                     const uint32_t tX = tmem + 128u * (uint32_t)c.half;
                     const uint32_t so = (uint32_t)slot * 2u * KV_SLOT_HALF;
+                    // S^T and dP^T step by step in turn: two independent accumulation chains keep the
+                    // tensor pipe busy where one dependent chain waits on each step
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t dh = kk >> 2, within = (kk & 3) * 32;
                         mma_ss(tX, sdesc_step(k_d, dh * TF_HALF_BYTES + within),
                                sdesc_step(q_d, so + dh * KV_SLOT_HALF + within), IDESC_S, kk > 0 ? 1u : 0u);
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t dh = kk >> 2, within = (kk & 3) * 32;
                         mma_ss(tX + 64, sdesc_step(v_d, dh * TF_HALF_BYTES + within),
                                sdesc_step(da_d, so + dh * KV_SLOT_HALF + within), IDESC_S, kk > 0 ? 1u : 0u);
                     }
@@ -996,13 +994,12 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                     const bool first = c.it == 0 && c.half == 0;
                     // A from TMEM (16 queries = 8 columns per step); B = dA / Q~ MN-major (N = d)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
+                    for (int kk = 0; kk < 4; ++kk) {  // dV and dK step by step in turn
                         mma_ts(TM_DV, tX + kk * 8, sdesc_step(da_mn, so + kk * 16 * 128), IDESC_MN,
                                (!first || kk > 0) ? 1u : 0u);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
                         mma_ts(TM_DK, tX + 64 + kk * 8, sdesc_step(q_mn, so + kk * 16 * 128), IDESC_MN,
                                (!first || kk > 0) ? 1u : 0u);
+                    }
                     mma_commit(&sm.bar[KB_QEMPTY + slot]);  // the half's Q~ and dA rows were read for the last time
                     if (last_of_unit(c)) mma_commit(&sm.bar[KB_DVKFULL]);
                     return true;

@@ -77,14 +77,23 @@ __device__ __forceinline__ BStrip bstrip_at(const LayerParams& L, int nst, int t
     return st;
 }
 
-// S (or dP) over a run of `nrun` ring slots starting at the given descriptors: 8 K-steps of 16 dims
-__device__ __forceinline__ void issue_span(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, int nrun) {
-    const uint32_t idesc = idesc_f16(128, 32 * nrun, false);
+// S = Q~ K~^T and dP = dA V^T over the span's ring slots (one run, or two around the ring's
+// end), K-step by K-step: the two (or four) independent accumulation chains are issued in
+// turn, so the tensor pipe overlaps them instead of waiting on each dependent step.
+__device__ __forceinline__ void issue_s_dp(uint32_t tS, uint32_t tP, uint64_t q_desc, uint64_t da_desc,
+                                           uint64_t k_desc0, uint64_t v_desc0, int s0, int run0, int nch) {
+    const uint32_t id0 = idesc_f16(128, 32 * run0, false), id1 = idesc_f16(128, 32 * (nch - run0), false);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
         const uint32_t half = kk >> 2, within = (kk & 3) * 32;
-        mma_ss(d_tmem, sdesc_step(a_desc, half * BQ_HALF + within),
-               sdesc_step(b_desc, half * BRING * BCH_HALF + within), idesc, kk > 0 ? 1u : 0u);
+        const uint32_t ao = half * BQ_HALF + within, bo = half * BRING * BCH_HALF + within;
+        const uint32_t acc = kk > 0 ? 1u : 0u;
+        mma_ss(tS, sdesc_step(q_desc, ao), sdesc_step(k_desc0, s0 * BCH_HALF + bo), id0, acc);
+        mma_ss(tP, sdesc_step(da_desc, ao), sdesc_step(v_desc0, s0 * BCH_HALF + bo), id0, acc);
+        if (run0 < nch) {
+            mma_ss(tS + 32 * run0, sdesc_step(q_desc, ao), sdesc_step(k_desc0, bo), id1, acc);
+            mma_ss(tP + 32 * run0, sdesc_step(da_desc, ao), sdesc_step(v_desc0, bo), id1, acc);
+        }
     }
 }
 
@@ -261,10 +270,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_strip_q_kernel(const __grid
                 tc_fence_after();
                 const int s0 = (le - (BNCH - 1)) % BRING;
                 const int run0 = min(BNCH, BRING - s0);
-                issue_span(tmem + BTM_S, q_d, sdesc_step(k_d, s0 * BCH_HALF), run0);
-                if (run0 < BNCH) issue_span(tmem + BTM_S + 32 * run0, q_d, k_d, BNCH - run0);
-                issue_span(tmem + BTM_P, da_d, sdesc_step(v_d, s0 * BCH_HALF), run0);
-                if (run0 < BNCH) issue_span(tmem + BTM_P + 32 * run0, da_d, v_d, BNCH - run0);
+                issue_s_dp(tmem + BTM_S, tmem + BTM_P, q_d, da_d, k_d, v_d, s0, run0, BNCH);
                 mma_commit(&sm.bar[SB_QE]);
                 mma_commit(&sm.bar[SB_SF]);
                 le_prev = le;

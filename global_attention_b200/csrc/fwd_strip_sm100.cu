@@ -116,19 +116,27 @@ __device__ __forceinline__ Strip strip_at(const StripParams& p, int t, int t_beg
     return st;
 }
 
-// K-step descriptors for S over a run of ring slots and for P V over one chunk
-__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc, int nrun) {
-    const uint32_t idesc = idesc_f16(128, 32 * nrun, false);
+// S = Q~ K~_span^T over the span's ring slots: one run, or two around the ring's end, issued
+// K-step by K-step in turn (independent accumulators, which the tensor pipe overlaps)
+__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc0, int s0, int run0) {
+    const uint32_t id0 = idesc_f16(128, 32 * run0, false), id1 = idesc_f16(128, 32 * (NCH - run0), false);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
         const uint32_t half = kk >> 2, within = (kk & 3) * 32;
-        mma_ss(d_tmem, sdesc_step(q_desc, half * QHALF + within),
-               sdesc_step(k_desc, half * RING * CHUNK_HALF + within), idesc, kk > 0 ? 1u : 0u);
+        const uint32_t ao = half * QHALF + within, bo = half * RING * CHUNK_HALF + within;
+        mma_ss(d_tmem, sdesc_step(q_desc, ao), sdesc_step(k_desc0, s0 * CHUNK_HALF + bo), id0, kk > 0 ? 1u : 0u);
+        if (run0 < NCH)
+            mma_ss(d_tmem + 32 * run0, sdesc_step(q_desc, ao), sdesc_step(k_desc0, bo), id1, kk > 0 ? 1u : 0u);
     }
 }
 
 }  // namespace
 
+// PREP: Q~ and K~ (fp16) were formed by the preparation kernels into the activation store and
+// arrive by TMA ready to use (the training pair, whose backward reads that store anyway): no
+// prologue or converter work in this kernel.  Otherwise q and k arrive raw and are converted
+// here.
+template <bool PREP>
 __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_constant__ StripParams p) {
     const LayerParams& L = p.L;
     extern __shared__ unsigned char smem_raw[];
@@ -211,7 +219,7 @@ __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_cons
                     const int buf = nq & 1;
                     const uint32_t ph = ((nq >> 1) - 1) & 1;
                     if (nq < 2 || (mbar_try_wait(&sm.bar[QE + buf], ph) &&
-                                   (!p.save || mbar_try_wait(&sm.bar[QS + buf], ph)))) {
+                                   (PREP || !p.save || mbar_try_wait(&sm.bar[QS + buf], ph)))) {
                         const Strip st = strip_at(p, tq, t_begin);
                         mbar_expect_tx(&sm.bar[QF + buf], 2 * QHALF);
                         tma_load_4d(sm.Q[buf][0], &p.tm_q, &sm.bar[QF + buf], 0, st.kvh * SG, st.s * SP, st.b);
@@ -231,8 +239,9 @@ __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_cons
                     const int slot = lk % RING;
                     if (lk < RING || mbar_try_wait(&sm.bar[KE + slot], ((lk / RING) - 1) & 1)) {
                         mbar_expect_tx(&sm.bar[KF + slot], CHUNK_BYTES);
-                        tma_load_4d(sm.K[0][slot], &p.tm_k, &sm.bar[KF + slot], 0, stk.kvh, ck * 32, stk.b);
-                        tma_load_4d(sm.K[1][slot], &p.tm_k, &sm.bar[KF + slot], 64, stk.kvh, ck * 32, stk.b);
+                        const CUtensorMap* km = PREP ? &p.tm_k16s : &p.tm_k;
+                        tma_load_4d(sm.K[0][slot], km, &sm.bar[KF + slot], 0, stk.kvh, ck * 32, stk.b);
+                        tma_load_4d(sm.K[1][slot], km, &sm.bar[KF + slot], 64, stk.kvh, ck * 32, stk.b);
                         mbar_expect_tx(&sm.bar[VF + slot], CHUNK_BYTES);
                         tma_load_4d(sm.V[0][slot], &p.tm_v, &sm.bar[VF + slot], 0, stk.kvh, ck * 32, stk.b);
                         tma_load_4d(sm.V[1][slot], &p.tm_v, &sm.bar[VF + slot], 64, stk.kvh, ck * 32, stk.b);
@@ -301,17 +310,15 @@ __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_cons
                 // Otherwise S(n) goes first, so this strip's softmax overlaps the previous P V.
                 const bool pv_first = st.fresh && n >= 1;
                 if (pv_first && !(ok = issue_pv(n - 1, false))) break;
-                if (!(ok = mbar_wait(&sm.bar[QR + buf], (n >> 1) & 1, abort, 43))) break;
+                if (!(ok = mbar_wait(&sm.bar[(PREP ? QF : QR) + buf], (n >> 1) & 1, abort, 43))) break;
                 for (; kc_waited <= le && ok; ++kc_waited)
-                    ok = mbar_wait(&sm.bar[KC + kc_waited % RING], (kc_waited / RING) & 1, abort, 44);
+                    ok = mbar_wait(&sm.bar[(PREP ? KF : KC) + kc_waited % RING], (kc_waited / RING) & 1, abort, 44);
                 if (!ok) break;
                 tc_fence_after();
                 // S = Q~ K~_span^T: the span's slots le-4 .. le, in one run or two around the ring end
                 const int s0 = (le - (NCH - 1)) % RING;
                 const int run0 = min(NCH, RING - s0);
-                const uint64_t qd = sdesc_step(q_desc0, buf * 2 * QHALF);
-                issue_s(tmem + X * SPAN, qd, sdesc_step(k_desc0, s0 * CHUNK_HALF), run0);
-                if (run0 < NCH) issue_s(tmem + X * SPAN + 32 * run0, qd, k_desc0, NCH - run0);
+                issue_s(tmem + X * SPAN, sdesc_step(q_desc0, buf * 2 * QHALF), k_desc0, s0, run0);
                 mma_commit(&sm.bar[QE + buf]);
                 mma_commit(&sm.bar[SF + X]);
                 if (n >= 1 && !pv_first) ok = issue_pv(n - 1, false);
@@ -321,7 +328,7 @@ __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_cons
             mma_commit(&sm.bar[DONE]);
             mbar_wait_drain(&sm.bar[DONE], 0);
         }
-    } else if (warp == 2 || warp == 3) {
+    } else if ((warp == 2 || warp == 3) && !PREP) {
         // ================================================ K converters: normalise + rotate in place
         // warp 2 takes the even loads, warp 3 the odd ones; thread = key row of the chunk
         const int mine = warp - 2;
@@ -360,7 +367,7 @@ __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_cons
             }
         }
         if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-    } else if (warp >= 12) {
+    } else if (warp >= 12 && !PREP) {
         // ================================================ Q prologue: Q~ normalised + rotated in place
         const int m = tid - 384, pos = m >> 2, wq = warp - 12;
         bool ok = true;
@@ -398,7 +405,7 @@ __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_cons
             __syncwarp();
         }
         if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-    } else {
+    } else if (warp >= 4 && warp < 12) {
         // ================================================ softmax + gate epilogue (thread = row)
         const int X = (warp - 4) >> 2;           // 0: even strips, 1: odd strips
         const int m = tid - 128 * (1 + X);       // row of the tile: 4 * position + head
@@ -567,8 +574,14 @@ bool fwd_strip_supported(const LayerParams& L) {
 
 size_t fwd_strip_smem_bytes() { return sizeof(StripSmem) + 1024; }
 
-// The strip forward; with `sv`, it also keeps Q~, K~ (fp16) and every q and k row's inverse
-// RMS in the caller's activation store for the backward.  Uses no scratch memory.
+cudaError_t launch_fwd_prep_k(const LayerParams& L, void* workspace, int* err_word, cudaStream_t stream,
+                              float* krinv);
+cudaError_t launch_prep_q_only(const LayerParams& L, void* q16, float* qrinv, int* err_word, cudaStream_t stream);
+
+// The strip forward.  With `sv` (the training pair) the preparation kernels first form Q~, K~
+// (fp16) and every q and k row's inverse RMS in the caller's activation store, which the
+// backward reads, and the attention kernel loads Q~ and K~ from there; without it the kernel
+// converts q and k itself and uses no scratch memory.
 cudaError_t launch_fwd_strip(const FwdParams& fp, int* err_word, cudaStream_t stream, const SavedAct* sv) {
     StripParams p;
     p.L = fp.L;
@@ -584,26 +597,36 @@ cudaError_t launch_fwd_strip(const FwdParams& fp, int* err_word, cudaStream_t st
     if (total > 0x7fffffffLL) return cudaErrorInvalidValue;
     p.total = (int)total;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    if (!strip_map(&p.tm_q, L.q, L.Hq, L.S, L.B, BF, SG, SP) || !strip_map(&p.tm_k, L.k, L.Hkv, L.S, L.B, BF, 1, 32) ||
-        !strip_map(&p.tm_v, L.v, L.Hkv, L.S, L.B, BF, 1, 32))
-        return cudaErrorInvalidValue;
-    if (sv) {
-        if (!strip_map(&p.tm_q16s, sv->q16, L.Hq, L.S, L.B, F16, SG, 8) ||
-            !strip_map(&p.tm_k16s, sv->k16, L.Hkv, L.S, L.B, F16, 1, 32))
-            return cudaErrorInvalidValue;
-    } else {
-        p.tm_q16s = p.tm_q;   // never used without save
-        p.tm_k16s = p.tm_k;
-    }
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     const size_t smem = fwd_strip_smem_bytes();
-    e = cudaFuncSetAttribute(fwd_strip_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     const int grid = (int)(total < sms ? total : sms);
-    fwd_strip_kernel<<<grid, THREADS, smem, stream>>>(p);
+    if (!strip_map(&p.tm_v, L.v, L.Hkv, L.S, L.B, BF, 1, 32)) return cudaErrorInvalidValue;
+    if (sv) {
+        // the training pair: Q~ and K~ (and the rows' inverse RMS) into the store first, then the
+        // attention kernel reads them from there
+        if ((e = launch_fwd_prep_k(L, sv->k16, err_word, stream, sv->krinv)) != cudaSuccess) return e;
+        if ((e = launch_prep_q_only(L, sv->q16, sv->qrinv, err_word, stream)) != cudaSuccess) return e;
+        if (!strip_map(&p.tm_q, sv->q16, L.Hq, L.S, L.B, F16, SG, SP) ||
+            !strip_map(&p.tm_k16s, sv->k16, L.Hkv, L.S, L.B, F16, 1, 32))
+            return cudaErrorInvalidValue;
+        p.tm_k = p.tm_k16s;
+        p.tm_q16s = p.tm_q;
+        p.save = 0;   // nothing left to store
+        e = cudaFuncSetAttribute(fwd_strip_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        fwd_strip_kernel<true><<<grid, THREADS, smem, stream>>>(p);
+        return cudaGetLastError();
+    }
+    if (!strip_map(&p.tm_q, L.q, L.Hq, L.S, L.B, BF, SG, SP) || !strip_map(&p.tm_k, L.k, L.Hkv, L.S, L.B, BF, 1, 32))
+        return cudaErrorInvalidValue;
+    p.tm_q16s = p.tm_q;   // never used without save
+    p.tm_k16s = p.tm_k;
+    e = cudaFuncSetAttribute(fwd_strip_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    fwd_strip_kernel<false><<<grid, THREADS, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
