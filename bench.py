@@ -129,8 +129,6 @@ def work(B, S, W, bwd, saved=False):
         # given the forward's q~, k~: v -> V fp16 (+ v norm per row, V scale per tile)
         "bwd_prep_v_kernel": (2 * kb + kb // (D // 2), 0),
         "bwd_q_tc_kernel": (4 * qb + 2 * kb + 3 * lse, 6 * D * npair),
-        # the same reads and writes, by strips of 32 positions x 4 heads
-        "bwd_strip_q_kernel": (4 * qb + 2 * kb + 3 * lse, 6 * D * npair),
         "bwd_kv_tc_kernel": (2 * qb + 5 * kb + 4 * lse, 8 * D * npair),
     }
     return dict(tokens=tok, npair=npair, fwd_bytes=fwd_bytes, fwd_flops=fwd_flops,

@@ -525,28 +525,24 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                     for (int h = 0; h < G && ok; ++h, ++m) {
                         const uint32_t tA = tm_half(m), tB = tm_half(m + 1);
                         if (!(ok = mbar_wait(&sm.bar[QB_QFULL], m & 1, abort, 114))) break;
+                        if (!(ok = mbar_wait(&sm.bar[QB_DAFULL], m & 1, abort, 118))) break;
+                        // dP(m) goes to tB once the epilogue of head m-1 has read dQ(m-1) there
+                        if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_DQEMPTY], (m - 1) & 1, abort, 115))) break;
                         tc_fence_after();
-                        // S = Q~ K~^T -> tA  (its columns were last read by the softmax of head m-1,
-                        // as dP, and by the epilogue of head m-2, both waited for already)
+                        // S = Q~ K~^T -> tA (its columns were last read by the softmax of head m-1, as
+                        // dP, and by the epilogue of head m-2) and dP = dA V^T -> tB, K-step by
+                        // K-step in turn: two independent accumulation chains overlap in the pipe
     #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
                             const uint32_t half = kk >> 2, within = (kk & 3) * 32;
                             const uint64_t aq = sdesc_sw128(q_base + half * TF_HALF_BYTES + within, 16, 1024);
                             const uint64_t bk = sdesc_sw128(k_base + half * TF_RING_HALF + within, 16, 1024);
                             mma_ss(tA, aq, bk, IDESC_N256, kk > 0 ? 1u : 0u);
-                        }
-                        mma_commit(&sm.bar[QB_QEMPTY]);
-                        // dP = dA V^T -> tB, once the epilogue of head m-1 has read dQ(m-1) there
-                        if (!(ok = mbar_wait(&sm.bar[QB_DAFULL], m & 1, abort, 118))) break;
-                        if (m >= 1 && !(ok = mbar_wait(&sm.bar[QB_DQEMPTY], (m - 1) & 1, abort, 115))) break;
-                        tc_fence_after();
-    #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t half = kk >> 2, within = (kk & 3) * 32;
                             const uint64_t ad = sdesc_sw128(da_base + half * TF_HALF_BYTES + within, 16, 1024);
                             const uint64_t bv = sdesc_sw128(v_base + half * TF_RING_HALF + within, 16, 1024);
                             mma_ss(tB, ad, bv, IDESC_N256, kk > 0 ? 1u : 0u);
                         }
+                        mma_commit(&sm.bar[QB_QEMPTY]);
                         mma_commit(&sm.bar[QB_DAEMPTY]);
                         mma_commit(&sm.bar[QB_DPFULL]);
                         if (h == G - 1) {
@@ -1239,12 +1235,12 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_b() {
 }
 
 bool make_map_b(CUtensorMap* map, const void* base, int H, int S, int B,
-                CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, int box_rows = 128, int box_heads = 1) {
+                CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, int box_rows = 128) {
     auto enc = get_encode_b();
     if (!enc) return false;
     cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)S * H * kD * 2};
-    cuuint32_t box[4] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows, 1};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(map, dtype, 4, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1281,16 +1277,6 @@ extern const char* const kBwdTcSavedKernelNames[] = {"bwd_gate_kernel",  "bwd_pr
                                                      "bwd_q_tc_kernel",  "bwd_kv_tc_kernel",
                                                      "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"};
 extern const int kBwdTcSavedKernelCount = 6;
-// 4 query heads per KV head: the query side runs by strips of positions
-extern const char* const kBwdStripKernelNames[] = {"bwd_gate_kernel",         "bwd_prep_kv_kernel",
-                                                   "bwd_prep_q_kernel",       "bwd_strip_q_kernel",
-                                                   "bwd_kv_tc_kernel",        "dgamma_reduce_kernel(k)",
-                                                   "dgamma_reduce_kernel(q)"};
-extern const int kBwdStripKernelCount = 7;
-extern const char* const kBwdStripSavedKernelNames[] = {"bwd_gate_kernel",  "bwd_prep_v_kernel",
-                                                        "bwd_strip_q_kernel", "bwd_kv_tc_kernel",
-                                                        "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"};
-extern const int kBwdStripSavedKernelCount = 6;
 extern const char* const kBwdWideSavedKernelNames[] = {"bwd_gate_kernel",   "bwd_prep_v_kernel",
                                                        "bwd_tile_stats_kernel", "bwd_q_glob_kernel",
                                                        "bwd_kv_tc_kernel",  "dgamma_reduce_kernel(k)",
@@ -1412,11 +1398,7 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
         !make_map_b(&p.tm_q16h, q16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 64) ||
         !make_map_b(&p.tm_dah, da16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 64) ||
         !make_map_rows(&p.tm_lse, p.lse2p, L.Hq, Spad, L.B) || !make_map_rows(&p.tm_delta, p.P.delta, L.Hq, Spad, L.B) ||
-        !make_map_rows(&p.tm_dainv, p.dainv, L.Hq, Spad, L.B) ||
-        !make_map_b(&p.tm_q16s, q16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 32, 4 < L.Hq ? 4 : L.Hq) ||
-        !make_map_b(&p.tm_das, da16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 32, 4 < L.Hq ? 4 : L.Hq) ||
-        !make_map_b(&p.tm_k16c, k16, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 32) ||
-        !make_map_b(&p.tm_v16c, v16, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 32))
+        !make_map_rows(&p.tm_dainv, p.dainv, L.Hq, Spad, L.B))
         return cudaErrorInvalidValue;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1507,26 +1489,9 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
         dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgq_part, (int)units_q, bp.dgamma_q);
         return after(i);
     }
-    int grid_q = grid;
-    if (bwd_strip_supported(L)) {
-        // the query side by strips of 32 positions x the group's 4 heads
-        const int strips = bwd_strip_total(L);
-        if (strips < 0) return cudaErrorInvalidValue;
-        const size_t smem_s = bwd_strip_smem_bytes();
-        if ((e = cudaFuncSetAttribute(bwd_strip_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_s)) !=
-            cudaSuccess)
-            return e;
-        grid_q = strips < sms ? strips : sms;
-        BwdTcParams ps = p;
-        ps.total = strips;
-        if ((e = before(i)) != cudaSuccess) return e;
-        bwd_strip_q_kernel<<<grid_q, TB_THREADS, smem_s, stream>>>(ps);
-        if ((e = after(i++)) != cudaSuccess) return e;
-    } else {
-        if ((e = before(i)) != cudaSuccess) return e;
-        bwd_q_tc_kernel<<<grid, TB_THREADS, smem_q, stream>>>(p);
-        if ((e = after(i++)) != cudaSuccess) return e;
-    }
+    if ((e = before(i)) != cudaSuccess) return e;
+    bwd_q_tc_kernel<<<grid, TB_THREADS, smem_q, stream>>>(p);
+    if ((e = after(i++)) != cudaSuccess) return e;
     if ((e = before(i)) != cudaSuccess) return e;
     bwd_kv_tc_kernel<false><<<grid, TB_THREADS, smem_k, stream>>>(p);
     if ((e = after(i++)) != cudaSuccess) return e;
@@ -1534,7 +1499,7 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgk_part, grid, bp.dgamma_k);
     if ((e = after(i++)) != cudaSuccess) return e;
     if ((e = before(i)) != cudaSuccess) return e;
-    dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgq_part, grid_q, bp.dgamma_q);
+    dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgq_part, grid, bp.dgamma_q);
     return after(i);
 }
 

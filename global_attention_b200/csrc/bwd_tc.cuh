@@ -26,10 +26,6 @@ struct BwdTcParams {
     CUtensorMap tm_lse;   // lse2p, Delta, 2^-e of the dA rows: fp32 {Spad, Hq, B}, box {64, 1, 1}
     CUtensorMap tm_delta;
     CUtensorMap tm_dainv;
-    CUtensorMap tm_q16s;  // Q~ fp16 with strip boxes {64, 4 heads, 32 positions, 1} (strip kernel)
-    CUtensorMap tm_das;   // dA16 with strip boxes
-    CUtensorMap tm_k16c;  // K~ fp16 with 32-row chunk boxes {64, 1, 32, 1}
-    CUtensorMap tm_v16c;  // V fp16 with 32-row chunk boxes
     BwdParams P;
     const __half* da16; // [B,S,Hq,D] dA * 2^e (e per row)
     float* dainv;       // [B,Hq,Spad] 2^-e of each dA row (0 for an all-zero row and past S)
@@ -168,11 +164,7 @@ __device__ __forceinline__ void row_rope_rms_backward_regs(float (&dy)[128], flo
 // sliding-window ones by launch_bwd_tc.
 __global__ void bwd_tile_stats_kernel(const __grid_constant__ BwdTcParams p);
 __global__ void bwd_q_glob_kernel(const __grid_constant__ BwdTcParams p);
-// Query side of the sliding-window backward by strips of positions (bwd_strip_sm100.cu).
-__global__ void bwd_strip_q_kernel(const __grid_constant__ BwdTcParams p);
-bool bwd_strip_supported(const LayerParams& L);
-size_t bwd_strip_smem_bytes();
-int bwd_strip_total(const LayerParams& L);
+
 size_t bwd_q_glob_smem_bytes();
 constexpr int BQG_THREADS = 384;
 constexpr int BTS_THREADS = 128;

@@ -14,25 +14,30 @@
 // positions x 4 heads) sees the same mask shape.  Consecutive strips of a chain share four of
 // their five chunks; K and V chunks stream through an 8-slot ring, one new chunk per strip.
 //
-// K is normalised and rotated in the ring, in place, by two converter warps (thread = key
-// row, the backward's device function, angles and fp16 scale, so the scores equal the
-// backward's bit for bit); no scratch memory is used.  Q is normalised in place by the
-// prologue warpgroup.  Per strip n (softmax warpgroup X = n mod 2, TMEM S_X):
+// Q~ and K~ are fp16 (times the power of two qk_fp16_scale picks), formed by the backward's own
+// device function, angles and scale, so the scores equal the backward's bit for bit.  Two modes:
+//   * plain forward: q and k arrive raw; K is normalised and rotated in the ring, in place, by
+//     two converter warps (thread = key row) and Q by the prologue warpgroup: no scratch memory;
+//   * the training pair (PREP): the preparation kernels have already formed Q~ and K~ (and every
+//     row's inverse RMS) in the caller's activation store, which the backward reads; they arrive
+//     by TMA ready to use and the converter and prologue warps stay idle.
+// Per strip n (softmax warpgroup X = n mod 2, TMEM S_X):
 //   S   = Q~ K~_span^T            tcgen05.mma M=128 N=160 K=128 (one or two runs of ring
-//                                  slots), fp16 operands in smem
+//                                  slots, issued in turn), fp16 operands in smem
 //   P   = exp2(S c - m)           softmax warpgroup X, thread = row, written as bf16 over the
 //                                  front of S_X; m a bound on every score when small enough
 //                                  (one pass), else the row maximum
 //   O   = P V_span                tcgen05.mma M=128 N=128 K=160, P from TMEM, V MN-major
 //   out = sigmoid(g) O / l        the same warpgroup, 16-byte loads and stores
 // Two softmax warpgroups take alternate strips, so one's exponentials overlap the other's
-// products and gate epilogue.  TMEM: S_0 [0,160), S_1 [160,320), O [320,448).
+// products and gate epilogue.  TMEM: S_0 [0,160), S_1 [160,320), O [320,448).  A strip that
+// starts a new chain finishes the previous strip's P V before its own S (its five new chunks
+// need the slots the previous strip holds).
 //
 // Warp roles (512 threads): w0 TMA producer (Q, K and V), w1 MMA issuer + TMEM owner, w2-3
 // K converters (alternate chunks), w4-7 softmax/epilogue of even strips, w8-11 of odd strips,
-// w12-15 Q prologue (with save_q it also stores Q~ and each row's inverse RMS for the
-// backward; the converters store K~ and the key rows' inverse RMS).  Every wait is bounded;
-// on expiry the CTA records the site, drains, frees TMEM and returns.
+// w12-15 Q prologue.  Every wait is bounded (and voted warp-uniform before warp-collective
+// instructions); on expiry the CTA records the site, drains, frees TMEM and returns.
 #include <cudaTypedefs.h>
 
 #include "sm100.cuh"
@@ -59,17 +64,12 @@ struct StripParams {
     CUtensorMap tm_q;    // raw q bf16 {D, Hq, S, B}, box {64, 4, 32, 1}
     CUtensorMap tm_k;    // raw k bf16 {D, Hkv, S, B}, box {64, 1, 32, 1}
     CUtensorMap tm_v;    // raw v bf16, box {64, 1, 32, 1}
-    CUtensorMap tm_q16s; // Q~ fp16 {D, Hq, S, B}, box {64, 4, 8, 1} (save: one warp's 32 rows)
-    CUtensorMap tm_k16s; // K~ fp16 {D, Hkv, S, B}, box {64, 1, 32, 1} (save)
     LayerParams L;
     bf16* out;
     float* lse;
-    float* qrinv;        // [B,Hq,S] inverse RMS of each q row (save)
-    float* krinv;        // [B,Hkv,S] inverse RMS of each k row (save)
     int* err;
     int nst;             // strips per (b, KV head) chain: ceil(S / 32)
     int total;           // B * Hkv * nst
-    int save;
 };
 
 enum Bar {
@@ -80,8 +80,7 @@ enum Bar {
     QF = KE + RING,         // [2] raw Q tile landed
     QR = QF + 2,            // [2] Q~ ready (prologue)
     QE = QR + 2,            // [2] Q buffer read by its S product
-    QS = QE + 2,            // [2] Q buffer read by the Q~ stores (save)
-    SF = QS + 2,            // [2] S_X complete
+    SF = QE + 2,            // [2] S_X complete
     PF = SF + 2,            // [2] P_X written
     OF = PF + 2,            // [2] O complete for a strip of warpgroup X
     OE = OF + 2,            // [2] O read by warpgroup X's epilogue
@@ -159,7 +158,6 @@ __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_cons
             mbar_init(&sm.bar[QF + i], 1);
             mbar_init(&sm.bar[QR + i], 128);
             mbar_init(&sm.bar[QE + i], 1);
-            mbar_init(&sm.bar[QS + i], 4);
             mbar_init(&sm.bar[SF + i], 1);
             mbar_init(&sm.bar[PF + i], 128);
             mbar_init(&sm.bar[OF + i], 1);
@@ -218,8 +216,7 @@ __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_cons
                 if (nq < nstrips) {
                     const int buf = nq & 1;
                     const uint32_t ph = ((nq >> 1) - 1) & 1;
-                    if (nq < 2 || (mbar_try_wait(&sm.bar[QE + buf], ph) &&
-                                   (PREP || !p.save || mbar_try_wait(&sm.bar[QS + buf], ph)))) {
+                    if (nq < 2 || mbar_try_wait(&sm.bar[QE + buf], ph)) {
                         const Strip st = strip_at(p, tq, t_begin);
                         mbar_expect_tx(&sm.bar[QF + buf], 2 * QHALF);
                         tma_load_4d(sm.Q[buf][0], &p.tm_q, &sm.bar[QF + buf], 0, st.kvh * SG, st.s * SP, st.b);
@@ -239,9 +236,8 @@ __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_cons
                     const int slot = lk % RING;
                     if (lk < RING || mbar_try_wait(&sm.bar[KE + slot], ((lk / RING) - 1) & 1)) {
                         mbar_expect_tx(&sm.bar[KF + slot], CHUNK_BYTES);
-                        const CUtensorMap* km = PREP ? &p.tm_k16s : &p.tm_k;
-                        tma_load_4d(sm.K[0][slot], km, &sm.bar[KF + slot], 0, stk.kvh, ck * 32, stk.b);
-                        tma_load_4d(sm.K[1][slot], km, &sm.bar[KF + slot], 64, stk.kvh, ck * 32, stk.b);
+                        tma_load_4d(sm.K[0][slot], &p.tm_k, &sm.bar[KF + slot], 0, stk.kvh, ck * 32, stk.b);
+                        tma_load_4d(sm.K[1][slot], &p.tm_k, &sm.bar[KF + slot], 64, stk.kvh, ck * 32, stk.b);
                         mbar_expect_tx(&sm.bar[VF + slot], CHUNK_BYTES);
                         tma_load_4d(sm.V[0][slot], &p.tm_v, &sm.bar[VF + slot], 0, stk.kvh, ck * 32, stk.b);
                         tma_load_4d(sm.V[1][slot], &p.tm_v, &sm.bar[VF + slot], 64, stk.kvh, ck * 32, stk.b);
@@ -340,36 +336,23 @@ __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_cons
             for (int c = 0; c < nl && ok; ++c, ++l) {
                 if ((l & 1) != mine) continue;
                 const int chunk = st.s - nl + 1 + c, slot = l % RING;
-                const bool own = (c == nl - 1);  // the strip's newest chunk: stored by this CTA
                 if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar[KF + slot], (l / RING) & 1, abort, 50)))) break;
                 const int pos = chunk * 32 + lane;
-                const float rinv = tf_prologue_row_at<true>(
-                    sm.K[0][slot], sm.K[1][slot], lane, sm.gk, L,
-                    [&](int q) {
-                        float2 w;
-                        rope_cs(L.theta[q], pos, w.x, w.y);
-                        return w;
-                    },
-                    oscale);
+                tf_prologue_row_at<true>(sm.K[0][slot], sm.K[1][slot], lane, sm.gk, L,
+                                         [&](int q) {
+                                             float2 w;
+                                             rope_cs(L.theta[q], pos, w.x, w.y);
+                                             return w;
+                                         },
+                                         oscale);
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (p.save && own) {
-                    if (pos < L.S) p.krinv[((size_t)st.b * L.Hkv + st.kvh) * L.S + pos] = rinv;
-                    if (lane == 0) {
-                        tma_store_4d(&p.tm_k16s, sm.K[0][slot], 0, st.kvh, chunk * 32, st.b);
-                        tma_store_4d(&p.tm_k16s, sm.K[1][slot], 64, st.kvh, chunk * 32, st.b);
-                        tma_store_commit();
-                        tma_store_wait_read();  // the slot is refilled only after the products read it
-                    }
-                    __syncwarp();
-                }
                 if (lane == 0) mbar_arrive(&sm.bar[KC + slot]);
             }
         }
-        if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     } else if (warp >= 12 && !PREP) {
         // ================================================ Q prologue: Q~ normalised + rotated in place
-        const int m = tid - 384, pos = m >> 2, wq = warp - 12;
+        const int m = tid - 384, pos = m >> 2;
         bool ok = true;
         for (int n = 0; n < nstrips && ok; ++n) {
             const Strip st = strip_at(p, t_begin + n, t_begin);
@@ -384,27 +367,11 @@ __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_cons
             }
             __syncwarp();
             if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar[QF + buf], (n >> 1) & 1, abort, 60)))) break;
-            const float rinv = tf_prologue_row_at<true>(sm.Q[buf][0], sm.Q[buf][1], m, sm.gq, L,
-                                                        [&](int q) { return sm.cs[pos][q]; }, oscale);
+            tf_prologue_row_at<true>(sm.Q[buf][0], sm.Q[buf][1], m, sm.gq, L, [&](int q) { return sm.cs[pos][q]; },
+                                     oscale);
             fence_proxy_async_smem();
-            if (p.save) {
-                const int i = p0 + pos, h = st.kvh * SG + (m & 3);
-                if (i < L.S) p.qrinv[((size_t)st.b * L.Hq + h) * L.S + i] = rinv;
-                __syncwarp();
-                if (lane == 0 && p0 + 8 * wq < L.S) {
-                    tma_store_4d(&p.tm_q16s, sm.Q[buf][0] + wq * 32 * 128, 0, st.kvh * SG, p0 + 8 * wq, st.b);
-                    tma_store_4d(&p.tm_q16s, sm.Q[buf][1] + wq * 32 * 128, 64, st.kvh * SG, p0 + 8 * wq, st.b);
-                    tma_store_commit();
-                }
-            }
             mbar_arrive(&sm.bar[QR + buf]);
-            if (p.save && lane == 0) {
-                tma_store_wait_read();  // the buffer is refilled two strips on, after this
-                mbar_arrive(&sm.bar[QS + buf]);
-            }
-            __syncwarp();
         }
-        if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     } else if (warp >= 4 && warp < 12) {
         // ================================================ softmax + gate epilogue (thread = row)
         const int X = (warp - 4) >> 2;           // 0: even strips, 1: odd strips
@@ -588,9 +555,6 @@ cudaError_t launch_fwd_strip(const FwdParams& fp, int* err_word, cudaStream_t st
     p.out = fp.out;
     p.lse = fp.lse;
     p.err = err_word;
-    p.save = sv ? 1 : 0;
-    p.qrinv = sv ? sv->qrinv : nullptr;
-    p.krinv = sv ? sv->krinv : nullptr;
     const LayerParams& L = fp.L;
     p.nst = (L.S + SP - 1) / SP;
     const long long total = (long long)L.B * L.Hkv * p.nst;
@@ -610,11 +574,8 @@ cudaError_t launch_fwd_strip(const FwdParams& fp, int* err_word, cudaStream_t st
         if ((e = launch_fwd_prep_k(L, sv->k16, err_word, stream, sv->krinv)) != cudaSuccess) return e;
         if ((e = launch_prep_q_only(L, sv->q16, sv->qrinv, err_word, stream)) != cudaSuccess) return e;
         if (!strip_map(&p.tm_q, sv->q16, L.Hq, L.S, L.B, F16, SG, SP) ||
-            !strip_map(&p.tm_k16s, sv->k16, L.Hkv, L.S, L.B, F16, 1, 32))
+            !strip_map(&p.tm_k, sv->k16, L.Hkv, L.S, L.B, F16, 1, 32))
             return cudaErrorInvalidValue;
-        p.tm_k = p.tm_k16s;
-        p.tm_q16s = p.tm_q;
-        p.save = 0;   // nothing left to store
         e = cudaFuncSetAttribute(fwd_strip_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         fwd_strip_kernel<true><<<grid, THREADS, smem, stream>>>(p);
@@ -622,8 +583,6 @@ cudaError_t launch_fwd_strip(const FwdParams& fp, int* err_word, cudaStream_t st
     }
     if (!strip_map(&p.tm_q, L.q, L.Hq, L.S, L.B, BF, SG, SP) || !strip_map(&p.tm_k, L.k, L.Hkv, L.S, L.B, BF, 1, 32))
         return cudaErrorInvalidValue;
-    p.tm_q16s = p.tm_q;   // never used without save
-    p.tm_k16s = p.tm_k;
     e = cudaFuncSetAttribute(fwd_strip_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     fwd_strip_kernel<false><<<grid, THREADS, smem, stream>>>(p);

@@ -30,11 +30,6 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
                           void* const* events, int n_pairs, const SavedAct* sv);
 extern const char* const kBwdTcSavedKernelNames[];
 extern const int kBwdTcSavedKernelCount;
-extern const char* const kBwdStripKernelNames[];
-extern const int kBwdStripKernelCount;
-extern const char* const kBwdStripSavedKernelNames[];
-extern const int kBwdStripSavedKernelCount;
-bool bwd_strip_supported(const LayerParams& L);
 extern const char* const kBwdWideSavedKernelNames[];
 extern const int kBwdWideSavedKernelCount;
 bool bwd_tc_supported(const LayerParams& L);
@@ -469,13 +464,10 @@ int zgcm_attn_bwd_saved(const void* q, const void* k, const void* v, const void*
 
 const char* zgcm_attn_bwd_saved_kernel_name(int i, int S, int rope_dims, int window) {
     LayerParams L{};
-    L.B = 1; L.S = S; L.rope_half = rope_dims / 2; L.W = window; L.G = 4;
+    L.B = 1; L.S = S; L.rope_half = rope_dims / 2; L.W = window;
     const char* const* names = nullptr;
     int n = 0;
-    if (!force_mma() && S >= 1 && bwd_strip_supported(L)) {
-        names = kBwdStripSavedKernelNames;
-        n = kBwdStripSavedKernelCount;
-    } else if (!force_mma() && S >= 1 && bwd_tc_supported(L)) {
+    if (!force_mma() && S >= 1 && bwd_tc_supported(L)) {
         names = kBwdTcSavedKernelNames;
         n = kBwdTcSavedKernelCount;
     } else if (!force_mma() && S >= 1 && bwd_wide_supported(L)) {
@@ -487,13 +479,10 @@ const char* zgcm_attn_bwd_saved_kernel_name(int i, int S, int rope_dims, int win
 
 const char* zgcm_attn_bwd_kernel_name(int i, int S, int rope_dims, int window) {
     LayerParams L{};
-    L.B = 1; L.S = S; L.rope_half = rope_dims / 2; L.W = window; L.G = 4;
+    L.B = 1; L.S = S; L.rope_half = rope_dims / 2; L.W = window;
     const char* const* names = kBwdMmaKernelNames;
     int n = kBwdMmaKernelCount;
-    if (!force_mma() && S >= 1 && bwd_strip_supported(L)) {
-        names = kBwdStripKernelNames;
-        n = kBwdStripKernelCount;
-    } else if (!force_mma() && S >= 1 && bwd_tc_supported(L)) {
+    if (!force_mma() && S >= 1 && bwd_tc_supported(L)) {
         names = kBwdTcKernelNames;
         n = kBwdTcKernelCount;
     } else if (!force_mma() && S >= 1 && bwd_wide_supported(L)) {

@@ -199,7 +199,7 @@ def test_saved_pair_checks(lib):
     assert _bwd_saved(lib, ws - 1, store, need) == -4     # the workspace is checked as before
     assert _bwd_saved(lib, ws, store, need, rope_dims=0) == -2
     names = ga.zgcm_attn_bwd_kernel_names(16384, 128, saved=True)
-    assert names[:4] == ["bwd_gate_kernel", "bwd_prep_v_kernel", "bwd_strip_q_kernel", "bwd_kv_tc_kernel"]
+    assert names[:4] == ["bwd_gate_kernel", "bwd_prep_v_kernel", "bwd_q_tc_kernel", "bwd_kv_tc_kernel"]
     assert "bwd_prep_q_kernel" not in ga.zgcm_attn_bwd_kernel_names(4096, 4096, saved=True)
 
 

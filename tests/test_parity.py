@@ -167,7 +167,7 @@ def test_backward_both_kernel_paths(B, S, W, monkeypatch):
     ref = _problem(t, window=W).backward(t["dout"])
     monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
     assert ga.zgcm_attn_bwd_kernel_names(S, W)[:5] == ["bwd_gate_kernel", "bwd_prep_kv_kernel", "bwd_prep_q_kernel",
-                                                        "bwd_strip_q_kernel", "bwd_kv_tc_kernel"]
+                                                        "bwd_q_tc_kernel", "bwd_kv_tc_kernel"]
     out, lse = _gpu_fwd(d, window=W)
     got_tc = _gpu_bwd(d, out, lse, window=W)
     assert ga.zgcm_attn_device_error() == 0
