@@ -106,19 +106,12 @@ def work(B, S, W, bwd, saved=False):
     # a forward that keeps its activations also writes q~ fp16 and each q and k row's inverse RMS
     keep = (qb + tok * HQ * 4 + tok * HKV * 4) if saved else 0
     kernels = {
-        "fwd_mma_kernel": (fwd_bytes, fwd_flops),
-        # q, k, v, g -> out, lse (keys normalised in shared memory); keeping its activations it
-        # also writes q~ and k~ fp16 and each q and k row's inverse RMS
-        "fwd_strip_kernel": (fwd_bytes + (keep + kb if saved else 0), fwd_flops),
+        # q, k, v, g -> out, lse (keys normalised in shared memory); in the training pair it
+        # reads q~ and k~ fp16 (same sizes) that the two preparation kernels wrote before it
+        "fwd_strip_kernel": (fwd_bytes, fwd_flops),
         "fwd_tc_kernel": (fwd_bytes + keep, fwd_flops),
         # tcgen05 forwards: q, K~16 (fp16, prepared from k by fwd_prep_k_kernel), v, g -> out, lse
         "fwd_glob_tc_kernel": (fwd_bytes + keep, fwd_flops),
-        # dout, out, g -> dg, dA
-        "bwd_pre_kernel": (5 * qb, 0),
-        # q, k, v, dA, lse -> dq, Delta ; S, dP, dQ
-        "bwd_dq_kernel": (qb + 2 * kb + qb + lse + qb + lse, 6 * D * npair),
-        # q, k, v, dA, lse, Delta -> dk, dv ; S, dP, dV, dK
-        "bwd_main_kernel": (qb + 2 * kb + qb + 2 * lse + 2 * kb, 8 * D * npair),
         # tcgen05 backward: gate pass dout, g, out -> dg, dA16 (fp16), 2^-e and max|dout| per row;
         # Q~16, K~16, V16, dA16, lse, 2^-e, raw q (RMSNorm backward) -> dq, Delta ; S, dP, dQ  |
         # Q~16, K~16, V16, dA16, lse, Delta, 2^-e, max|dout|, raw k -> dk, dv ; S, dP, dV, dK
@@ -165,19 +158,25 @@ def traffic_for(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks/throttle sampling during the timed region."""
+    """nvidia-smi clocks/throttle sampling around the timed region.  The sampler starts before
+    the warm-up and the timed region waits for its first row, so a short region is covered;
+    `mark_start` / `mark_end` bracket the region on the host clock and the summary takes the
+    rows inside it, or, when the region is shorter than the sampling interval, the last row
+    before it and the first row after it (reported as "window": "bracketing")."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 20
 
     def __init__(self, gpu_id: str):
         self.index, self.rows, self.proc = gpu_id, [], None
+        self.t_start = self.t_end = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", str(self.INTERVAL_MS)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except OSError:
@@ -186,7 +185,24 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.rows.append([x.strip() for x in line.split(",")])
+            self.rows.append((time.monotonic(), [x.strip() for x in line.split(",")]))
+
+    def _wait_rows(self, after, limit_s):
+        end = time.monotonic() + limit_s
+        while self.proc and self.proc.poll() is None and time.monotonic() < end:
+            if self.rows and self.rows[-1][0] > after:
+                return
+            time.sleep(0.005)
+
+    def wait_ready(self):
+        self._wait_rows(0.0, 10.0)  # nvidia-smi takes a moment to print its first row
+
+    def mark_start(self):
+        self.t_start = time.monotonic()
+
+    def mark_end(self):
+        self.t_end = time.monotonic()
+        self._wait_rows(self.t_end, 1.0)
 
     def __exit__(self, *a):
         if self.proc:
@@ -197,9 +213,18 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        rows, window = self.rows, "all"
+        if self.t_start is not None and self.t_end is not None:
+            inside = [r for r in rows if self.t_start <= r[0] <= self.t_end]
+            window = "timed region"
+            if not inside:
+                before = [r for r in rows if r[0] < self.t_start][-1:]
+                after = [r for r in rows if r[0] > self.t_end][:1]
+                inside, window = before + after, "bracketing"
+            rows = inside
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in self.rows:
+        for _, r in rows:
             try:
                 sm.append(float(r[1]))
                 mx = float(r[2])
@@ -211,7 +236,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "window": window}
 
 
 def cpu_oracle_run(B, S, W, bwd, seed=0):
@@ -370,11 +395,13 @@ def run_decode(args):
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in layers]
           for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize()
     with ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) as clk:
+        clk.wait_ready()
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+        clk.mark_start()
         t0.record(stream)
         for i in range(args.steps):
             for li in range(len(layers)):
@@ -383,6 +410,7 @@ def run_decode(args):
                 ev[i][li][1].record(stream)
         t1.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
     ms = max_over_ranks(t0.elapsed_time(t1), world, dev) / args.steps
     layer_ms = [statistics.mean(ev[i][li][0].elapsed_time(ev[i][li][1]) for i in range(args.steps))
                 for li in range(len(layers))]
@@ -573,15 +601,18 @@ def main():
 
     # ---- timed region: K steps, inputs resident in HBM (5.6 GB per step >> 126 MB L2)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
     with ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) as clk:
+        clk.wait_ready()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        clk.mark_start()
         t0.record(stream)
         for i in range(args.steps):
             step(i)
         t1.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
     if world > 1:
         dist.barrier()
     ms = t0.elapsed_time(t1)
@@ -706,7 +737,7 @@ def main():
     for (lw, _), kp in zip(layers, keep):
         fname = ga.zgcm_attn_fwd_kernel_name(Bw, Sw, HQ, HKV, 42, lw)
         # the strip forward keeping its activations runs the two preparation kernels first
-        fwd_launches.append(1 if fname == "fwd_mma_kernel" else (3 if kp else 1) if fname == "fwd_strip_kernel"
+        fwd_launches.append((3 if kp else 1) if fname == "fwd_strip_kernel"
                             else 3 if kp and fname == "fwd_glob_tc_kernel" else 2)
     launches_per_step = sum(f + len(n) for f, n in zip(fwd_launches, bwd_names))
     rec = {

@@ -137,8 +137,8 @@ def zgcm_attn_fwd_workspace_size(B, S, Hq, Hkv, D=128, rope_dims=42, window=128)
 
 
 def zgcm_attn_saved_size(B, S, Hq, Hkv, D=128, rope_dims=42, window=128) -> int:
-    """Bytes of the activation store zgcm_attn_fwd(saved=...) fills for the backward (0 where
-    the pair does not apply)."""
+    """Bytes of the activation store zgcm_attn_fwd(saved=...) fills for the backward (0 for an
+    empty problem)."""
     return int(load().zgcm_attn_saved_size(int(B), int(S), int(Hq), int(Hkv), int(D), int(rope_dims),
                                            int(window)))
 

@@ -128,6 +128,8 @@ __device__ __forceinline__ void qg_ds_chunk(const float* sv, const float* dv, ui
     ma[1] = acc.y;
 }
 
+// ANY: any number of rotated pairs in the dq epilogue (else the layer's 21, unrolled)
+template <bool ANY>
 __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid_constant__ BwdTcParams p) {
     const LayerParams& L = p.P.L;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -426,7 +428,8 @@ __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid
                 tmem_wait_ld();
                 const float f = L.scale / (dsc * oscale);
                 const float mdot = (macc + reinterpret_cast<const float*>(sm.V[1][0])[256 + r]) * mdot_f;
-                row_rope_rms_backward_regs(dy, f, mdot, rinv, xv0, L.q + off, p.P.dq + off, valid, i, sm.gq, dgam, L);
+                row_rope_rms_backward_regs<ANY ? 0 : TF_HALF>(dy, f, mdot, rinv, xv0, L.q + off, p.P.dq + off, valid, i,
+                                                              sm.gq, dgam, L);
             }
         }
     }
@@ -442,6 +445,17 @@ __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid
             sm.abort ? 0.f : (dg[tid] + dg[kD + tid]) + (dg[2 * kD + tid] + dg[3 * kD + tid]);
     }
     if (tid == 0 && sm.abort && p.err) atomicExch(p.err, sm.abort);
+}
+
+// The query-major kernel for windows wider than one tile: one CTA per unit, the instance for
+// the layer's 21 rotated pairs or for any other number.
+cudaError_t launch_bwd_q_glob(const BwdTcParams& p, int units, cudaStream_t stream) {
+    auto k = p.P.L.rope_half != TF_HALF ? bwd_q_glob_kernel<true> : bwd_q_glob_kernel<false>;
+    const size_t smem = bwd_q_glob_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<units, BQG_THREADS, smem, stream>>>(p);
+    return cudaGetLastError();
 }
 
 }  // namespace zgcm

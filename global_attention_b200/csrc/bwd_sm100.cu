@@ -1,8 +1,10 @@
 // bwd_sm100.cu — gated sliding-window attention backward on tcgen05 / TMEM / TMA (sm_100a).
 //
 // Exact gradients of L = sum(dout * out) for the ZGCM-1 layer (definition and page
-// citations in common.cuh), for windows W <= 128 and 42 rotated dims; other shapes run on
-// the warp-MMA kernels (bwd_mma.cu).  The gate pass, the preparation passes (bwd_prep_kv,
+// citations in common.cuh), for windows W <= 128 (wider ones: bwd_glob_sm100.cu with the
+// key-major kernel here in its wide mode).  Every kernel that rotates comes in two instances:
+// the layer's 21 rotated pairs, unrolled, and any other number (the angles formed where
+// needed).  The gate pass, the preparation passes (bwd_prep_kv,
 // bwd_prep_q: fp16 K~, V, Q~ with the rows' inverse RMS; bwd_prep_v alone when the forward
 // kept Q~ and K~) and the two score kernels:
 //
@@ -11,7 +13,8 @@
 //              scaled by a power of two per row (2^-e and max|dout| saved per row).
 //   bwd_q_tc   query-major sweep over (b, KV head, 128-query block) steps, all query heads
 //              of the group per step, key tiles qb-1 and qb in a 2-slot ring (as the forward).
-//              Per head: S = Q~ K~^T and dP = dA V^T (both M=128 N=256 into TMEM), then one
+//              Per head: S = Q~ K~^T and dP = dA V^T (both M=128 N=256 into TMEM, issued
+//              step by step in turn), then one
 //              warpgroup per row forms the log-sum-exp, Delta = sum_j P dP and dS = P(dP-Delta)
 //              from its own scores, dQ~ = dS K~ (M=128 N=128 K=256, dS from TMEM), and an
 //              epilogue warpgroup applies the RoPE / RMSNorm backward and writes dq.  Writes
@@ -290,7 +293,8 @@ struct PrepSmem {
 // dk), the raw norm of each v row (dS^T scale) and the V tile scale.  Several CTAs per SM keep
 // tile loads, conversions and stores of different tiles in flight.
 // WITH_K false (key tiles only): V alone, for a backward given the forward's K~ and inverse RMS.
-template <bool IS_K, bool WITH_K = true>
+// ANY: any number of rotated pairs, the angles formed as needed (else the layer's 21, in registers)
+template <bool IS_K, bool WITH_K, bool ANY>
 __device__ __forceinline__ void prep_tile(const BwdTcParams& p) {
     const LayerParams& L = p.P.L;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -322,8 +326,8 @@ __device__ __forceinline__ void prep_tile(const BwdTcParams& p) {
         }
     }
     const int pos = t * TF_BN + r;
-    float2 csr[WITH_K ? TF_HALF : 1];  // (cos, sin) of the rotated pairs at this row's position
-    if constexpr (WITH_K) {
+    float2 csr[WITH_K && !ANY ? TF_HALF : 1];  // (cos, sin) of the rotated pairs at this row's position
+    if constexpr (WITH_K && !ANY) {
 #pragma unroll
         for (int q = 0; q < TF_HALF; ++q) rope_cs(L.theta[q], pos, csr[q].x, csr[q].y);
     }
@@ -332,7 +336,9 @@ __device__ __forceinline__ void prep_tile(const BwdTcParams& p) {
     const bool ok = __syncthreads_and(mbar_wait(&sm.bar, 0, &abort, 250)) != 0;
     if (ok) {
         float rinv = 0.f;
-        if constexpr (WITH_K)
+        if constexpr (WITH_K && ANY)
+            rinv = tf_prologue_row_any<true>(sm.X[0], sm.X[1], r, IS_K ? sm.gk : sm.gq, L, pos, oscale);
+        else if constexpr (WITH_K)
             rinv = tf_prologue_row_at<true>(sm.X[0], sm.X[1], r, IS_K ? sm.gk : sm.gq, L,
                                             [&](int q) { return csr[q]; }, oscale);
         const size_t ro = ((size_t)b * H + h) * L.S + pos;
@@ -371,16 +377,20 @@ __device__ __forceinline__ void prep_tile(const BwdTcParams& p) {
     }
 }
 
+template <bool ANY>
 __global__ void __launch_bounds__(KP_THREADS, 3) bwd_prep_kv_kernel(const __grid_constant__ BwdTcParams p) {
-    prep_tile<true>(p);
+    prep_tile<true, true, ANY>(p);
 }
+template <bool ANY>
 __global__ void __launch_bounds__(KP_THREADS, 4) bwd_prep_q_kernel(const __grid_constant__ BwdTcParams p) {
-    prep_tile<false>(p);
+    prep_tile<false, true, ANY>(p);
 }
 __global__ void __launch_bounds__(KP_THREADS, 3) bwd_prep_v_kernel(const __grid_constant__ BwdTcParams p) {
-    prep_tile<true, false>(p);
+    prep_tile<true, false, false>(p);
 }
 
+// ANY: any number of rotated pairs in the dq epilogue (else the layer's 21, angles shared per step)
+template <bool ANY>
 __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_constant__ BwdTcParams p) {
     const LayerParams& L = p.P.L;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -692,7 +702,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
             const bool valid = i < L.S;
             // the row's rotation angles, shared by the G heads of the step (own column only)
 #pragma unroll 1
-            for (int q = 0; q < TF_HALF; ++q) rope_cs(L.theta[q], i, sm.cs[q][r].x, sm.cs[q][r].y);
+            for (int q = 0; !ANY && q < TF_HALF; ++q) rope_cs(L.theta[q], i, sm.cs[q][r].x, sm.cs[q][r].y);
             for (int h = 0; h < G; ++h, ++m) {
                 const int hg = st.kvh * G + h;
                 const size_t off = ((size_t)(st.b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hg) * kD;
@@ -714,8 +724,12 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_q_tc_kernel(const __grid_co
                 const float mdot = sm.mdot[m & 1][r];
                 tc_fence_before();
                 mbar_arrive(&sm.bar[QB_DQEMPTY]);  // dQ(m) is in registers: TMEM free for dP(m+1)
-                row_rope_rms_backward_cs(dy, f, mdot, rinv, xv0, L.q + off, p.P.dq + off, valid,
-                                         [&](int q) { return sm.cs[q][r]; }, sm.gq, sm.dgq[wq]);
+                if constexpr (ANY)
+                    row_rope_rms_backward_regs<0>(dy, f, mdot, rinv, xv0, L.q + off, p.P.dq + off, valid, i, sm.gq,
+                                                  sm.dgq[wq], L);
+                else
+                    row_rope_rms_backward_cs(dy, f, mdot, rinv, xv0, L.q + off, p.P.dq + off, valid,
+                                             [&](int q) { return sm.cs[q][r]; }, sm.gq, sm.dgq[wq]);
             }
         }
     }
@@ -807,7 +821,7 @@ __device__ __forceinline__ void decode_iter(const LayerParams& L, const UnitInfo
     hg = x.kvh * L.G + it % L.G;
 }
 
-template <bool WIDE>
+template <bool WIDE, bool ANY>
 __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_constant__ BwdTcParams p) {
     const LayerParams& L = p.P.L;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -1203,7 +1217,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             const float rinv = valid ? p.krinv[((size_t)x.b * L.Hkv + x.kvh) * L.S + j] : 0.f;
             tc_fence_before();
             mbar_arrive(&sm.bar[KB_DVKEMPTY]);  // dV, dK of the unit are out of TMEM
-            row_rope_rms_backward_regs(dy, f, mdot, rinv, xv0, L.k + off, p.P.dk + off, valid, j, sm.gk, sm.dgk[wq], L);
+            row_rope_rms_backward_regs<ANY ? 0 : TF_HALF>(dy, f, mdot, rinv, xv0, L.k + off, p.P.dk + off, valid, j,
+                                                          sm.gk, sm.dgk[wq], L);
         }
     }
 
@@ -1283,18 +1298,35 @@ extern const char* const kBwdWideSavedKernelNames[] = {"bwd_gate_kernel",   "bwd
                                                        "dgamma_reduce_kernel(q)"};
 extern const int kBwdWideSavedKernelCount = 7;
 
-__global__ void dgamma_reduce_kernel(const float* __restrict__ parts, int n, float* __restrict__ out);
-
-// Windows up to one key tile, 42 rotated dims.  A shape test only: without the driver's
-// tensor-map encoder the launch fails (ZGCM_ERR_CUDA).
-bool bwd_tc_supported(const LayerParams& L) {
-    return L.W <= TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1;
+// d_gamma[d] = sum over the n partial rows parts[i][d] (one per CTA of the kernel that wrote
+// them), in a fixed order so repeated runs give the same bits: eight groups of 128 threads
+// take every eighth row, then group 0 adds the eight group sums.  One CTA of 1024 threads.
+__global__ void __launch_bounds__(1024) dgamma_reduce_kernel(const float* __restrict__ parts, int n,
+                                                             float* __restrict__ out) {
+    __shared__ float acc[8][kD];
+    const int d = threadIdx.x & (kD - 1), grp = threadIdx.x >> 7;
+    float s = 0.f;
+    for (int i = grp; i < n; i += 8) s += parts[(size_t)i * kD + d];
+    acc[grp][d] = s;
+    __syncthreads();
+    if (grp == 0) {
+        float t = 0.f;
+#pragma unroll
+        for (int g2 = 0; g2 < 8; ++g2) t += acc[g2][d];
+        out[d] = t;
+    }
 }
 
-// Windows wider than one tile (the global layer among them), 42 rotated dims.  A shape test
+// Windows up to one key tile, any rotated dims and group size.  A shape test only: without
+// the driver's tensor-map encoder the launch fails (ZGCM_ERR_CUDA).
+bool bwd_tc_supported(const LayerParams& L) {
+    return L.W <= TF_BN && L.S >= 1 && L.B >= 1;
+}
+
+// Windows wider than one tile (the global layer among them), any rotated dims.  A shape test
 // only: without the driver's tensor-map encoder the launch fails (ZGCM_ERR_CUDA).
 bool bwd_wide_supported(const LayerParams& L) {
-    return L.W > TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1;
+    return L.W > TF_BN && L.S >= 1 && L.B >= 1;
 }
 
 namespace {
@@ -1333,9 +1365,10 @@ cudaError_t launch_prep_q_only(const LayerParams& L, void* q16, float* qrinv, in
         !make_map_b(&p.tm_q16, q16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return cudaErrorInvalidValue;
     const size_t smem_pq = sizeof(PrepSmem<false>) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(bwd_prep_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_pq);
+    auto prep_q = L.rope_half != TF_HALF ? bwd_prep_q_kernel<true> : bwd_prep_q_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(prep_q, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_pq);
     if (e != cudaSuccess) return e;
-    bwd_prep_q_kernel<<<(int)q_tiles, KP_THREADS, smem_pq, stream>>>(p);
+    prep_q<<<(int)q_tiles, KP_THREADS, smem_pq, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -1358,7 +1391,6 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
         off += a(bytes);
         return q;
     };
-    p.P.lse2 = nullptr;  // P is formed from the forward's lse
     const int Spad = row_stride(L.S);
     const size_t prows = (size_t)L.B * L.Hq * Spad;
     p.P.delta = reinterpret_cast<float*>(take(prows * 4));
@@ -1406,13 +1438,18 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     if (e != cudaSuccess) return e;
     sms = sms < TB_MAX_GRID ? sms : TB_MAX_GRID;
     const size_t smem_q = sizeof(BwdQTcSmem) + 1024, smem_k = sizeof(BwdKTcSmem) + 1024;
-    if ((e = cudaFuncSetAttribute(bwd_q_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_q)) != cudaSuccess)
+    // the layer's 21 rotated pairs take the unrolled instances, any other number the general ones
+    const bool any = L.rope_half != TF_HALF;
+    auto q_tc = any ? bwd_q_tc_kernel<true> : bwd_q_tc_kernel<false>;
+    auto kv_slide = any ? bwd_kv_tc_kernel<false, true> : bwd_kv_tc_kernel<false, false>;
+    auto kv_wide = any ? bwd_kv_tc_kernel<true, true> : bwd_kv_tc_kernel<true, false>;
+    auto prep_kv = any ? bwd_prep_kv_kernel<true> : bwd_prep_kv_kernel<false>;
+    auto prep_q = any ? bwd_prep_q_kernel<true> : bwd_prep_q_kernel<false>;
+    if ((e = cudaFuncSetAttribute(q_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_q)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(bwd_kv_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_k)) !=
-        cudaSuccess)
+    if ((e = cudaFuncSetAttribute(kv_slide, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_k)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(bwd_kv_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_k)) !=
-        cudaSuccess)
+    if ((e = cudaFuncSetAttribute(kv_wide, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_k)) != cudaSuccess)
         return e;
     // events[2i] / events[2i+1] bracket kernel i (i < n_pairs)
     auto before = [&](int i) -> cudaError_t {
@@ -1433,11 +1470,9 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     const long long gate_need = (half_warps * 16 + GATE_THREADS - 1) / GATE_THREADS;
     const int gate_grid = (int)(gate_need < 2LL * sms ? gate_need : 2LL * sms);
     const size_t smem_pk = sizeof(PrepSmem<true>) + 1024, smem_pq = sizeof(PrepSmem<false>) + 1024;
-    if ((e = cudaFuncSetAttribute(bwd_prep_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_pk)) !=
-        cudaSuccess)
+    if ((e = cudaFuncSetAttribute(prep_kv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_pk)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(bwd_prep_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_pq)) !=
-        cudaSuccess)
+    if ((e = cudaFuncSetAttribute(prep_q, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_pq)) != cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(bwd_prep_v_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_pk)) !=
         cudaSuccess)
@@ -1457,30 +1492,26 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     if (sv)
         bwd_prep_v_kernel<<<(int)k_tiles, KP_THREADS, smem_pk, stream>>>(p);
     else
-        bwd_prep_kv_kernel<<<(int)k_tiles, KP_THREADS, smem_pk, stream>>>(p);
+        prep_kv<<<(int)k_tiles, KP_THREADS, smem_pk, stream>>>(p);
     if ((e = after(i++)) != cudaSuccess) return e;
     if (!sv) {
         if ((e = before(i)) != cudaSuccess) return e;
-        bwd_prep_q_kernel<<<(int)q_tiles, KP_THREADS, smem_pq, stream>>>(p);
+        prep_q<<<(int)q_tiles, KP_THREADS, smem_pq, stream>>>(p);
         if ((e = after(i++)) != cudaSuccess) return e;
     }
     if (wide) {
         // per-tile bounds, then the query-major sweep (one CTA per (b, head, block), heaviest
         // first) and the key-major one (one CTA per (b, KV head, tile), heaviest first)
         const long long units_q = (long long)L.B * L.Hq * nqb;
-        const size_t smem_g = bwd_q_glob_smem_bytes();
-        if ((e = cudaFuncSetAttribute(bwd_q_glob_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_g)) !=
-            cudaSuccess)
-            return e;
         if ((e = before(i)) != cudaSuccess) return e;
         bwd_tile_stats_kernel<<<(int)k_tiles, BTS_THREADS, 0, stream>>>(p);
         if ((e = after(i++)) != cudaSuccess) return e;
         if ((e = before(i)) != cudaSuccess) return e;
-        bwd_q_glob_kernel<<<(int)units_q, BQG_THREADS, smem_g, stream>>>(p);
+        if ((e = launch_bwd_q_glob(p, (int)units_q, stream)) != cudaSuccess) return e;
         if ((e = after(i++)) != cudaSuccess) return e;
         p.total = (int)k_tiles;
         if ((e = before(i)) != cudaSuccess) return e;
-        bwd_kv_tc_kernel<true><<<(int)k_tiles, TB_THREADS, smem_k, stream>>>(p);
+        kv_wide<<<(int)k_tiles, TB_THREADS, smem_k, stream>>>(p);
         if ((e = after(i++)) != cudaSuccess) return e;
         if ((e = before(i)) != cudaSuccess) return e;
         dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgk_part, (int)k_tiles, bp.dgamma_k);
@@ -1490,10 +1521,10 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
         return after(i);
     }
     if ((e = before(i)) != cudaSuccess) return e;
-    bwd_q_tc_kernel<<<grid, TB_THREADS, smem_q, stream>>>(p);
+    q_tc<<<grid, TB_THREADS, smem_q, stream>>>(p);
     if ((e = after(i++)) != cudaSuccess) return e;
     if ((e = before(i)) != cudaSuccess) return e;
-    bwd_kv_tc_kernel<false><<<grid, TB_THREADS, smem_k, stream>>>(p);
+    kv_slide<<<grid, TB_THREADS, smem_k, stream>>>(p);
     if ((e = after(i++)) != cudaSuccess) return e;
     if ((e = before(i)) != cudaSuccess) return e;
     dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgk_part, grid, bp.dgamma_k);

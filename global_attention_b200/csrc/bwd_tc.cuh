@@ -101,23 +101,37 @@ __device__ __forceinline__ uint4* tile_chunk(unsigned char* h0, unsigned char* h
 // `valid` masks rows past the sequence (they still join the collectives).
 // cs_at(t): (cos, sin) of pair t at the row's position (rope_cs), so that a caller with
 // several heads of one row can form them once.
-template <class CsAt>
+// RH: the number of rotated pairs when known at compile time (the layer's 21, unrolled), or 0
+// for any number rh (0..64) given at run time.
+template <int RH = TF_HALF, class CsAt>
 __device__ __forceinline__ void row_rope_rms_backward_cs(float (&dy)[128], float f, float mdot, float rinv,
                                                          const uint4 (&xv0)[8], const bf16* x, bf16* dst,
-                                                         bool valid, CsAt cs_at, const float* gamma, float* dgam) {
+                                                         bool valid, CsAt cs_at, const float* gamma, float* dgam,
+                                                         int rh = RH) {
     const int lane = threadIdx.x & 31;
     const uint4* xr = reinterpret_cast<const uint4*>(x);
     uint4* dr = reinterpret_cast<uint4*>(dst);
 #pragma unroll
     for (int e = 0; e < 128; ++e) dy[e] *= f;
-    // transpose of the rotation of pairs (t, t + 21)
+    // transpose of the rotation of pairs (t, t + rh)
+    if constexpr (RH > 0) {
 #pragma unroll
-    for (int t = 0; t < TF_HALF; ++t) {
-        const float2 w = cs_at(t);
-        const float c = w.x, s = w.y;
-        const float d1 = dy[t], d2 = dy[t + TF_HALF];
-        dy[t] = d1 * c + d2 * s;
-        dy[t + TF_HALF] = d2 * c - d1 * s;
+        for (int t = 0; t < RH; ++t) {
+            const float2 w = cs_at(t);
+            const float c = w.x, s = w.y;
+            const float d1 = dy[t], d2 = dy[t + RH];
+            dy[t] = d1 * c + d2 * s;
+            dy[t + RH] = d2 * c - d1 * s;
+        }
+    } else {
+#pragma unroll 1
+        for (int t = 0; t < rh; ++t) {
+            const float2 w = cs_at(t);
+            const float c = w.x, s = w.y;
+            const float d1 = dy[t], d2 = dy[t + rh];
+            dy[t] = d1 * c + d2 * s;
+            dy[t + rh] = d2 * c - d1 * s;
+        }
     }
     uint4 xv1[8];
 #pragma unroll
@@ -146,26 +160,27 @@ __device__ __forceinline__ void row_rope_rms_backward_cs(float (&dy)[128], float
     }
 }
 
+template <int RH = TF_HALF>
 __device__ __forceinline__ void row_rope_rms_backward_regs(float (&dy)[128], float f, float mdot, float rinv,
                                                            const uint4 (&xv0)[8], const bf16* x, bf16* dst,
                                                            bool valid, int pos, const float* gamma, float* dgam,
                                                            const LayerParams& L) {
-    row_rope_rms_backward_cs(dy, f, mdot, rinv, xv0, x, dst, valid,
-                             [&](int t) {
-                                 float c, s;
-                                 rope_cs(L.theta[t], pos, c, s);
-                                 return make_float2(c, s);
-                             },
-                             gamma, dgam);
+    row_rope_rms_backward_cs<RH>(dy, f, mdot, rinv, xv0, x, dst, valid,
+                                 [&](int t) {
+                                     float c, s;
+                                     rope_cs(L.theta[t], pos, c, s);
+                                     return make_float2(c, s);
+                                 },
+                                 gamma, dgam, L.rope_half);
 }
 
 
 // Kernels of the wide-window / global backward (bwd_glob_sm100.cu), launched with the
 // sliding-window ones by launch_bwd_tc.
 __global__ void bwd_tile_stats_kernel(const __grid_constant__ BwdTcParams p);
-__global__ void bwd_q_glob_kernel(const __grid_constant__ BwdTcParams p);
+// the wide query-major kernel, its instance for the number of rotated pairs
+cudaError_t launch_bwd_q_glob(const BwdTcParams& p, int units, cudaStream_t stream);
 
-size_t bwd_q_glob_smem_bytes();
 constexpr int BQG_THREADS = 384;
 constexpr int BTS_THREADS = 128;
 

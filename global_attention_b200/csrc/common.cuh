@@ -64,14 +64,10 @@ struct BwdParams {
     bf16* dg;           // [B,S,Hq,D]
     float* dgamma_q;    // [D]
     float* dgamma_k;    // [D]
-    // workspace views
-    float* delta;       // [B,Hq,S]   sum_j P_ij dP_ij (formed by the dq kernel)
-    float* lse2;        // [B,Hq,S]   base-2 log-sum-exp of the backward's own scores
-    bf16* dA;           // [B,S,Hq,D] dout * sigmoid(g), rounded to bf16 ("hi")
-    bf16* dA_lo;        // [B,S,Hq,D] dout * sigmoid(g) - hi, rounded to bf16
-    float* dgk_part;    // [n_k_parts, D]
-    float* dgq_part;    // [n_q_parts, D]
-    int n_k_parts, n_q_parts;
+    // workspace views (set by the launcher)
+    float* delta;       // [B,Hq,Spad] Delta of each row
+    float* dgk_part;    // [slots, D] d_gamma_k partial sums
+    float* dgq_part;    // [slots, D] d_gamma_q partial sums
 };
 
 // ---------------------------------------------------------------- small helpers
@@ -171,99 +167,5 @@ __device__ __forceinline__ void prologue_row(uint2 raw, const float* gamma4, con
     }
 }
 
-// Backward of prologue_row for one row, warp-cooperative (lane l owns dims [4l, 4l+4)).
-// dyrot[4]: gradient w.r.t. the rotated row.  Writes dx[4] (gradient w.r.t. raw x) and
-// adds dy * xhat into dgamma_acc[4].
-//   dy = R^T dyrot ; dxhat = dy * gamma ; dx = (dxhat - xhat * mean(dxhat * xhat)) / r
-__device__ __forceinline__ void prologue_row_backward(uint2 raw, const float* gamma4,
-                                                      const LayerParams& L, int pos, float* ybuf,
-                                                      const float dyrot[4], float dx[4],
-                                                      float dgamma_acc[4]) {
-    const int lane = threadIdx.x & 31;
-    float2 a = unpack_bf16(raw.x), b = unpack_bf16(raw.y);
-    float x[4] = {a.x, a.y, b.x, b.y};
-    float ss = warp_sum(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
-    float r = sqrtf(ss * (1.0f / kD) + L.eps);
-    float rinv = 1.0f / r;
-    float dy[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dy[e] = dyrot[e];
-    const int half = L.rope_half;
-    if (half > 0) {
-        float ct = 1.f, st = 0.f, ct2 = 1.f, st2 = 0.f;
-        if (lane < half) rope_cs(L.theta[lane], pos, ct, st);
-        if (half > 32 && lane + 32 < half) rope_cs(L.theta[lane + 32], pos, ct2, st2);
-        *reinterpret_cast<float4*>(ybuf + 4 * lane) = make_float4(dyrot[0], dyrot[1], dyrot[2], dyrot[3]);
-        __syncwarp();
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            int d = 4 * lane + e;
-            int t = d < half ? d : d - half;
-            bool rot = d < 2 * half;
-            int src = t & 31;
-            float c0 = __shfl_sync(0xffffffffu, ct, src);
-            float s0 = __shfl_sync(0xffffffffu, st, src);
-            float c1 = __shfl_sync(0xffffffffu, ct2, src);
-            float s1 = __shfl_sync(0xffffffffu, st2, src);
-            float c = t < 32 ? c0 : c1, s = t < 32 ? s0 : s1;
-            if (rot) {
-                float partner = ybuf[d < half ? d + half : d - half];
-                // d <  half: dy_t      =  dyrot_t c + dyrot_{t+half} s
-                // d >= half: dy_{t+h}  = -dyrot_t s + dyrot_{t+half} c
-                dy[e] = d < half ? dyrot[e] * c + partner * s : dyrot[e] * c - partner * s;
-            }
-        }
-        __syncwarp();
-    }
-    float xhat[4], dxh[4];
-    float m = 0.f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        xhat[e] = x[e] * rinv;
-        dxh[e] = dy[e] * gamma4[e];
-        m += dxh[e] * xhat[e];
-        dgamma_acc[e] += dy[e] * xhat[e];
-    }
-    m = warp_sum(m) * (1.0f / kD);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dx[e] = (dxh[e] - xhat[e] * m) * rinv;
-}
-
-// ---------------------------------------------------------------- tensor-core (mma.sync) helpers
-
-__device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
-                                            uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                                  uint32_t& r3, uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-
-// D(16x8 fp32) += A(16x16 bf16, row) * B(16x8 bf16, col)
-__device__ __forceinline__ void mma_bf16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};\n"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Row-major [rows][128] bf16 tile in shared memory, 256 B per row, with the 16-byte chunk
-// index XOR-swizzled by (row & 7) so that 8 consecutive rows of one chunk column hit 8
-// different bank groups (ldmatrix reads conflict-free).
-__device__ __forceinline__ uint32_t tile_off(int row, int chunk) {
-    return (uint32_t)(row * 256 + ((chunk ^ (row & 7)) << 4));
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* gptr, bool pred) {
-    int n = pred ? 16 : 0;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(saddr), "l"(gptr), "r"(n));
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
 }  // namespace zgcm

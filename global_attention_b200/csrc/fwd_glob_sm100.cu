@@ -51,7 +51,7 @@ struct FwdGlobParams {
     float* lse;
     int* err;
     float* krinv;        // inverse RMS of each k row, [B,Hkv,S] (preparation kernel; null = not kept)
-    int units;           // B * Hkv * (G / 2) * ceil(S / 128)
+    int units;           // B * Hkv * ceil(G / 2) * ceil(S / 128)
 };
 
 enum FgBar {
@@ -72,14 +72,16 @@ struct FwdGlobSmem {
 };
 
 struct FgUnit {
-    int b, kvh, h0, qb, kt_lo, n_tiles;
+    int b, kvh, h0, h1, qb, kt_lo, n_tiles;   // h0, h1: the unit's two query heads
 };
 
-// Unit u, heaviest first: the query block runs from the last one down; the two head pairs of
-// a KV group are adjacent so that the CTAs reading the same K/V tiles run together.
+// Unit u, heaviest first: the query block runs from the last one down; the head pairs of a KV
+// group are adjacent so that the CTAs reading the same K/V tiles run together.  With an odd
+// number of heads per KV head the last pair repeats the last head (its two warpgroups compute,
+// and write, the same rows).
 __device__ __forceinline__ FgUnit fg_unit(const LayerParams& L, int u) {
     const int nqb = (L.S + TF_BM - 1) / TF_BM;
-    const int npair = L.G / 2, per_qb = L.B * L.Hkv * npair;
+    const int npair = (L.G + 1) / 2, per_qb = L.B * L.Hkv * npair;
     FgUnit w;
     w.qb = nqb - 1 - u / per_qb;
     const int rest = u - (nqb - 1 - w.qb) * per_qb;
@@ -87,6 +89,7 @@ __device__ __forceinline__ FgUnit fg_unit(const LayerParams& L, int u) {
     w.kvh = (rest / npair) % L.Hkv;
     w.b = rest / (npair * L.Hkv);
     w.h0 = w.kvh * L.G + 2 * hp;
+    w.h1 = w.kvh * L.G + min(2 * hp + 1, L.G - 1);
     const int q0 = w.qb * TF_BM;
     // first key tile holding a key visible to the block's first row: j > q0 - W
     w.kt_lo = (L.W >= L.S || q0 - L.W + 1 <= 0) ? 0 : (q0 - L.W + 1) / TF_BN;
@@ -105,6 +108,8 @@ struct FwdPrepSmem {
 };
 
 // One CTA per 128-row key tile (b, KV head, t): raw k -> K~ fp16 in place -> workspace.
+// ANY: any number of rotated pairs, the angles formed as needed (else the layer's 21, in registers)
+template <bool ANY>
 __global__ void __launch_bounds__(FP_THREADS, 4) fwd_prep_k_kernel(const __grid_constant__ FwdGlobParams p) {
     const LayerParams& L = p.L;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -127,14 +132,19 @@ __global__ void __launch_bounds__(FP_THREADS, 4) fwd_prep_k_kernel(const __grid_
         tma_load_4d(sm.X[1], &p.tm_k, &sm.bar, 64, h, t * TF_BN, b);
     }
     const int pos = t * TF_BN + r;
-    float2 csr[TF_HALF];
+    float2 csr[ANY ? 1 : TF_HALF];
+    if constexpr (!ANY) {
 #pragma unroll
-    for (int q = 0; q < TF_HALF; ++q) rope_cs(L.theta[q], pos, csr[q].x, csr[q].y);
+        for (int q = 0; q < TF_HALF; ++q) rope_cs(L.theta[q], pos, csr[q].x, csr[q].y);
+    }
     const float oscale = qk_fp16_scale(sm.gq, sm.gk);
     const bool ok = __syncthreads_and(mbar_wait(&sm.bar, 0, &abort, 260)) != 0;
     if (ok) {
-        const float rinv = tf_prologue_row_at<true>(sm.X[0], sm.X[1], r, sm.gk, L, [&](int q) { return csr[q]; },
-                                                    oscale);
+        float rinv;
+        if constexpr (ANY)
+            rinv = tf_prologue_row_any<true>(sm.X[0], sm.X[1], r, sm.gk, L, pos, oscale);
+        else
+            rinv = tf_prologue_row_at<true>(sm.X[0], sm.X[1], r, sm.gk, L, [&](int q) { return csr[q]; }, oscale);
         if (p.krinv && pos < L.S) p.krinv[(size_t)chain * L.S + pos] = rinv;
         fence_proxy_async_smem();
     } else if (r == 0) {
@@ -155,6 +165,7 @@ __global__ void __launch_bounds__(FP_THREADS, 4) fwd_prep_k_kernel(const __grid_
 
 // ------------------------------------------------------------------ attention kernel
 
+template <bool ANY>
 __global__ void __launch_bounds__(FG_THREADS, 1) fwd_glob_tc_kernel(const __grid_constant__ FwdGlobParams p) {
     const LayerParams& L = p.L;
     extern __shared__ unsigned char smem_raw[];
@@ -210,8 +221,8 @@ __global__ void __launch_bounds__(FG_THREADS, 1) fwd_glob_tc_kernel(const __grid
         if (lane == 0) {
             for (int x = 0; x < 2; ++x) {
                 mbar_expect_tx(&sm.bar[FG_QFULL + x], TF_TILE_BYTES);
-                tma_load_4d(sm.Q[x][0], &p.tm_q, &sm.bar[FG_QFULL + x], 0, w.h0 + x, q0, w.b);
-                tma_load_4d(sm.Q[x][1], &p.tm_q, &sm.bar[FG_QFULL + x], 64, w.h0 + x, q0, w.b);
+                tma_load_4d(sm.Q[x][0], &p.tm_q, &sm.bar[FG_QFULL + x], 0, x ? w.h1 : w.h0, q0, w.b);
+                tma_load_4d(sm.Q[x][1], &p.tm_q, &sm.bar[FG_QFULL + x], 64, x ? w.h1 : w.h0, q0, w.b);
             }
             int nk = 0, nv = 0;  // K~ / V tiles issued
             for (int n = 0; n < w.n_tiles; ++n) {
@@ -301,16 +312,20 @@ __global__ void __launch_bounds__(FG_THREADS, 1) fwd_glob_tc_kernel(const __grid
         // ================================================ softmax + epilogue of head x (thread = query row)
         reg_alloc<224>();
         const int x = (warp - 4) >> 2, wq = warp & 3;
-        const int r = 32 * wq + lane, i = q0 + r, hx = w.h0 + x;
+        const int r = 32 * wq + lane, i = q0 + r, hx = x ? w.h1 : w.h0;
         const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
         const uint32_t TM_S = tmem + 128 * x, TM_O = tmem + 256 + 128 * x;
         bool ok = mbar_wait(&sm.bar[FG_QFULL + x], 0, abort, 290);
         if (ok) {
             // Q~_x in place: the same device function, angles and scale as the backward's Q~
-            float2 csr[TF_HALF];
+            if constexpr (ANY) {
+                tf_prologue_row_any<true>(sm.Q[x][0], sm.Q[x][1], r, sm.gq, L, i, oscale);
+            } else {
+                float2 csr[TF_HALF];
 #pragma unroll
-            for (int t = 0; t < TF_HALF; ++t) rope_cs(L.theta[t], i, csr[t].x, csr[t].y);
-            tf_prologue_row_at<true>(sm.Q[x][0], sm.Q[x][1], r, sm.gq, L, [&](int t) { return csr[t]; }, oscale);
+                for (int t = 0; t < TF_HALF; ++t) rope_cs(L.theta[t], i, csr[t].x, csr[t].y);
+                tf_prologue_row_at<true>(sm.Q[x][0], sm.Q[x][1], r, sm.gq, L, [&](int t) { return csr[t]; }, oscale);
+            }
             fence_proxy_async_smem();
             mbar_arrive(&sm.bar[FG_QREADY + x]);
         }
@@ -471,11 +486,11 @@ bool make_map_g(CUtensorMap* map, const void* base, int H, int S, int B, CUtenso
 
 }  // namespace
 
-// Windows wider than one key tile (W > 128, including the global layer W >= S), 42 rotated
-// dims, an even number of query heads per KV head (heads are processed in pairs).  A shape
-// test only: without the driver's tensor-map encoder the launch fails (ZGCM_ERR_CUDA).
+// Windows wider than one key tile (W > 128, including the global layer W >= S): any number of
+// rotated dims and of query heads per KV head.  A shape test only: without the driver's
+// tensor-map encoder the launch fails (ZGCM_ERR_CUDA).
 bool fwd_glob_supported(const LayerParams& L) {
-    return L.W > TF_BN && L.rope_half == TF_HALF && L.G % 2 == 0 && L.S >= 1 && L.B >= 1;
+    return L.W > TF_BN && L.S >= 1 && L.B >= 1;
 }
 
 // K~ fp16 [B, S, Hkv, D] (both tcgen05 forwards)
@@ -497,7 +512,7 @@ cudaError_t launch_fwd_glob_tc(const FwdParams& fp, void* workspace, int* err_wo
     p.lse = fp.lse;
     p.err = err_word;
     const long long nqb = (L.S + TF_BM - 1) / TF_BM;
-    const long long units = (long long)L.B * L.Hkv * (L.G / 2) * nqb;
+    const long long units = (long long)L.B * L.Hkv * ((L.G + 1) / 2) * nqb;
     const long long k_tiles = (long long)L.B * L.Hkv * nqb;
     if (units > 0x7fffffffLL || k_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
     p.units = (int)units;
@@ -507,14 +522,17 @@ cudaError_t launch_fwd_glob_tc(const FwdParams& fp, void* workspace, int* err_wo
         !make_map_g(&p.tm_v, L.v, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
         return cudaErrorInvalidValue;
     const size_t smem_p = sizeof(FwdPrepSmem) + 1024, smem_a = sizeof(FwdGlobSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(fwd_prep_k_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p);
+    const bool any = L.rope_half != TF_HALF;
+    auto prep = any ? fwd_prep_k_kernel<true> : fwd_prep_k_kernel<false>;
+    auto attn = any ? fwd_glob_tc_kernel<true> : fwd_glob_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(fwd_glob_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
+    e = cudaFuncSetAttribute(attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
     if (e != cudaSuccess) return e;
-    fwd_prep_k_kernel<<<(int)k_tiles, FP_THREADS, smem_p, stream>>>(p);
+    prep<<<(int)k_tiles, FP_THREADS, smem_p, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (sv && (e = launch_prep_q_only(fp.L, sv->q16, sv->qrinv, err_word, stream)) != cudaSuccess) return e;
-    fwd_glob_tc_kernel<<<(int)units, FG_THREADS, smem_a, stream>>>(p);
+    attn<<<(int)units, FG_THREADS, smem_a, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -535,9 +553,10 @@ cudaError_t launch_fwd_prep_k(const LayerParams& L, void* workspace, int* err_wo
         !make_map_g(&p.tm_k16, workspace, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return cudaErrorInvalidValue;
     const size_t smem_p = sizeof(FwdPrepSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(fwd_prep_k_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p);
+    auto prep = L.rope_half != TF_HALF ? fwd_prep_k_kernel<true> : fwd_prep_k_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p);
     if (e != cudaSuccess) return e;
-    fwd_prep_k_kernel<<<(int)k_tiles, FP_THREADS, smem_p, stream>>>(p);
+    prep<<<(int)k_tiles, FP_THREADS, smem_p, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -2,8 +2,8 @@
 //
 // Layer (ZGCM-1; page citations in common.cuh): out = sigmoid(g) * softmax_window(q~ k~^T) v,
 // with q~, k~ the RMS-normalised (gamma) and partially rotated q, k, window i-W < j <= i.
-// This kernel takes windows W <= 128 (the 27 sliding layers use W = 128) and 42 rotated
-// dims; other shapes run on the warp-MMA kernel (fwd_mma.cu).
+// This kernel takes windows W <= 128 (the 27 sliding layers use W = 128) and any number of
+// query heads per KV head (the strip kernel, fwd_strip_sm100.cu, takes the layer's 4).
 //
 // Work decomposition: a "step" is (batch b, KV head, 128-query block qb) with all Hq/Hkv
 // query heads of the group.  With W <= 128 the window of block qb lies inside key tiles
@@ -81,6 +81,8 @@ struct FwdTcSmem {
 
 // ------------------------------------------------------------------ the kernel
 
+// ANY: any number of rotated pairs (L.rope_half), the angles formed per row as needed.
+template <bool ANY>
 __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_constant__ FwdTcParams p) {
     const LayerParams& L = p.L;
     extern __shared__ unsigned char smem_raw[];
@@ -374,11 +376,13 @@ __global__ void __launch_bounds__(TF_THREADS, 1) fwd_tc_kernel(const __grid_cons
         bool ok = true;
         for (int t = t_begin; t < t_end && ok; ++t) {
             const StepInfo st = decode_step(L, t, t_begin, t_end);
-            tf_angles(L, st.qb * TF_BM + r, sm.cs, r);  // this row's angles, shared by the G heads
+            if constexpr (!ANY) tf_angles(L, st.qb * TF_BM + r, sm.cs, r);  // this row's angles, shared by the G heads
             for (int h = 0; h < G; ++h, ++m) {
                 const int buf = m & 1;
                 if (!(ok = mbar_wait(&sm.bar[B_QFULL + buf], (m >> 1) & 1, abort, 33))) break;
-                const float rinv = tf_prologue_row<true>(sm.Q[buf][0], sm.Q[buf][1], r, sm.gq, L, sm.cs, oscale);
+                const float rinv =
+                    ANY ? tf_prologue_row_any<true>(sm.Q[buf][0], sm.Q[buf][1], r, sm.gq, L, st.qb * TF_BM + r, oscale)
+                        : tf_prologue_row<true>(sm.Q[buf][0], sm.Q[buf][1], r, sm.gq, L, sm.cs, oscale);
                 fence_proxy_async_smem();
                 if (p.save_q) {
                     // this warp's 32 rows of Q~ to the store the backward reads
@@ -501,10 +505,10 @@ bool make_map(CUtensorMap* map, const void* base, int H, int S, int B,
 
 }  // namespace
 
-// Windows up to one key tile with 42 rotated dims.  A shape test only: without the driver's
-// tensor-map encoder the launch fails (ZGCM_ERR_CUDA).
+// Windows up to one key tile, any rotated dims and group size.  A shape test only: without
+// the driver's tensor-map encoder the launch fails (ZGCM_ERR_CUDA).
 bool fwd_tc_supported(const LayerParams& L) {
-    return L.W <= TF_BN && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1;
+    return L.W <= TF_BN && L.S >= 1 && L.B >= 1;
 }
 
 size_t fwd_tc_smem_bytes() { return sizeof(FwdTcSmem) + 1024; }
@@ -541,10 +545,11 @@ cudaError_t launch_fwd_tc(const FwdParams& fp, void* workspace, int* err_word, c
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     const size_t smem = fwd_tc_smem_bytes();
-    e = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = fp.L.rope_half == TF_HALF ? fwd_tc_kernel<false> : fwd_tc_kernel<true>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = (int)(total < sms ? total : sms);
-    fwd_tc_kernel<<<grid, TF_THREADS, smem, stream>>>(p);
+    kern<<<grid, TF_THREADS, smem, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -4,15 +4,17 @@
 // Layer (ZGCM-1; page citations in common.cuh): out = sigmoid(g) * softmax_window(q~ k~^T) v,
 // q~, k~ the RMS-normalised (gamma) and partially rotated q, k; key j visible to query i iff
 // i-W < j <= i.  This kernel takes windows W <= 128 (the 27 sliding layers use W = 128),
-// 4 query heads per KV head (GQA 32/8) and 42 rotated dims.
+// 4 query heads per KV head (GQA 32/8) and any number of rotated dims.
 //
 // A strip is (batch b, KV head, 32 consecutive positions p0..p0+31) with the 4 query heads of
 // the KV group: 128 query rows that share one window of keys, positions p0-128 .. p0+31 —
 // five 32-key chunks.  The MMA tile's rows are (position, head) pairs, row = 4 pos + head (the
 // order one TMA box {64 d, 4 heads, 32 positions} lands in), so one M=128 product covers the
 // whole window of all 128 rows: no key tile is masked out entirely and every warp (8
-// positions x 4 heads) sees the same mask shape.  Consecutive strips of a chain share four of
-// their five chunks; K and V chunks stream through an 8-slot ring, one new chunk per strip.
+// positions x 4 heads) sees the same mask shape.  The layer's 42 rotated dims take an unrolled
+// prologue, other counts one that forms the angles where needed.  Consecutive strips of a
+// chain share four of their five chunks; K and V chunks stream through an 8-slot ring, one
+// new chunk per strip.
 //
 // Q~ and K~ are fp16 (times the power of two qk_fp16_scale picks), formed by the backward's own
 // device function, angles and scale, so the scores equal the backward's bit for bit.  Two modes:
@@ -135,7 +137,9 @@ __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t q_desc, uint64
 // arrive by TMA ready to use (the training pair, whose backward reads that store anyway): no
 // prologue or converter work in this kernel.  Otherwise q and k arrive raw and are converted
 // here.
-template <bool PREP>
+// ANY: any number of rotated pairs (L.rope_half), the rotation angles formed where needed;
+// otherwise the layer's 21 pairs, unrolled, with the angles of a strip shared by its heads.
+template <bool PREP, bool ANY>
 __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_constant__ StripParams p) {
     const LayerParams& L = p.L;
     extern __shared__ unsigned char smem_raw[];
@@ -338,13 +342,16 @@ __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_cons
                 const int chunk = st.s - nl + 1 + c, slot = l % RING;
                 if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar[KF + slot], (l / RING) & 1, abort, 50)))) break;
                 const int pos = chunk * 32 + lane;
-                tf_prologue_row_at<true>(sm.K[0][slot], sm.K[1][slot], lane, sm.gk, L,
-                                         [&](int q) {
-                                             float2 w;
-                                             rope_cs(L.theta[q], pos, w.x, w.y);
-                                             return w;
-                                         },
-                                         oscale);
+                if constexpr (ANY)
+                    tf_prologue_row_any<true>(sm.K[0][slot], sm.K[1][slot], lane, sm.gk, L, pos, oscale);
+                else
+                    tf_prologue_row_at<true>(sm.K[0][slot], sm.K[1][slot], lane, sm.gk, L,
+                                             [&](int q) {
+                                                 float2 w;
+                                                 rope_cs(L.theta[q], pos, w.x, w.y);
+                                                 return w;
+                                             },
+                                             oscale);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.bar[KC + slot]);
@@ -360,15 +367,18 @@ __global__ void __launch_bounds__(THREADS, 1) fwd_strip_kernel(const __grid_cons
             // angles of the strip's positions: the 4 threads of a position (its 4 heads, all in this
             // warp) take pairs t = head, head + 4, ..; only this warp reads its 8 positions' entries
             __syncwarp();   // the previous strip's rows have read the table
-            for (int q = m & 3; q < TF_HALF; q += 4) {
+            for (int q = m & 3; !ANY && q < TF_HALF; q += 4) {
                 float2 w;
                 rope_cs(L.theta[q], p0 + pos, w.x, w.y);
                 sm.cs[pos][q] = w;
             }
             __syncwarp();
             if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.bar[QF + buf], (n >> 1) & 1, abort, 60)))) break;
-            tf_prologue_row_at<true>(sm.Q[buf][0], sm.Q[buf][1], m, sm.gq, L, [&](int q) { return sm.cs[pos][q]; },
-                                     oscale);
+            if constexpr (ANY)
+                tf_prologue_row_any<true>(sm.Q[buf][0], sm.Q[buf][1], m, sm.gq, L, p0 + pos, oscale);
+            else
+                tf_prologue_row_at<true>(sm.Q[buf][0], sm.Q[buf][1], m, sm.gq, L, [&](int q) { return sm.cs[pos][q]; },
+                                         oscale);
             fence_proxy_async_smem();
             mbar_arrive(&sm.bar[QR + buf]);
         }
@@ -534,10 +544,21 @@ bool strip_map(CUtensorMap* map, const void* base, int H, int S, int B, CUtensor
 
 }  // namespace
 
-// Windows up to 128 keys, 4 query heads per KV head, 42 rotated dims.
+// Windows up to 128 keys, 4 query heads per KV head (any number of rotated dims).
 bool fwd_strip_supported(const LayerParams& L) {
-    return L.W <= 128 && L.G == SG && L.rope_half == TF_HALF && L.S >= 1 && L.B >= 1;
+    return L.W <= 128 && L.G == SG && L.S >= 1 && L.B >= 1;
 }
+
+namespace {
+template <bool PREP>
+cudaError_t launch_strip_kernel(const StripParams& p, int grid, size_t smem, cudaStream_t stream) {
+    auto k = p.L.rope_half == TF_HALF ? fwd_strip_kernel<PREP, false> : fwd_strip_kernel<PREP, true>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, THREADS, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+}  // namespace
 
 size_t fwd_strip_smem_bytes() { return sizeof(StripSmem) + 1024; }
 
@@ -576,17 +597,11 @@ cudaError_t launch_fwd_strip(const FwdParams& fp, int* err_word, cudaStream_t st
         if (!strip_map(&p.tm_q, sv->q16, L.Hq, L.S, L.B, F16, SG, SP) ||
             !strip_map(&p.tm_k, sv->k16, L.Hkv, L.S, L.B, F16, 1, 32))
             return cudaErrorInvalidValue;
-        e = cudaFuncSetAttribute(fwd_strip_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        fwd_strip_kernel<true><<<grid, THREADS, smem, stream>>>(p);
-        return cudaGetLastError();
+        return launch_strip_kernel<true>(p, grid, smem, stream);
     }
     if (!strip_map(&p.tm_q, L.q, L.Hq, L.S, L.B, BF, SG, SP) || !strip_map(&p.tm_k, L.k, L.Hkv, L.S, L.B, BF, 1, 32))
         return cudaErrorInvalidValue;
-    e = cudaFuncSetAttribute(fwd_strip_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    fwd_strip_kernel<false><<<grid, THREADS, smem, stream>>>(p);
-    return cudaGetLastError();
+    return launch_strip_kernel<false>(p, grid, smem, stream);
 }
 
 }  // namespace zgcm

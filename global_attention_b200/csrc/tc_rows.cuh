@@ -166,6 +166,55 @@ __device__ __forceinline__ float tf_prologue_row_at(unsigned char* h0, unsigned 
     return rinv1;  // 1 / sqrt(mean x^2 + eps) of the row (0 for a zero row)
 }
 
+// Element d (0..127) of row r in a two-half 128-row tile with 128-byte swizzle: its address.
+__device__ __forceinline__ unsigned char* tile_elem(unsigned char* h0, unsigned char* h1, int r, int d) {
+    unsigned char* hb = d < 64 ? h0 : h1;
+    const int dd = d & 63;
+    return hb + (uint32_t)r * 128u + (uint32_t)(((((dd >> 3) ^ (r & 7)) << 4)) + ((dd & 7) << 1));
+}
+
+// The same normalisation and rotation as tf_prologue_row_at for any number of rotated pairs
+// L.rope_half (0..64, pairs (t, t + rope_half)), the angles formed at `pos` as needed: each
+// pair's two elements are read, rotated and written back in place.  The arithmetic and its
+// rounding are those of tf_prologue_row_at, so for 21 pairs both give the same bits.
+template <bool F16>
+__device__ __forceinline__ float tf_prologue_row_any(unsigned char* h0, unsigned char* h1, int r, const float* gamma,
+                                                    const LayerParams& L, int pos, float oscale) {
+    float ss = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 16; ++ch) {
+        const uint4 u = *reinterpret_cast<const uint4*>(tile_elem(h0, h1, r, 8 * ch));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float2 f = unpack_bf16(w[e]);
+            ss = fmaf(f.x, f.x, ss);
+            ss = fmaf(f.y, f.y, ss);
+        }
+    }
+    const float rinv1 = ss > 0.f ? rsqrtf(fmaf(ss, 1.0f / kD, L.eps)) : 0.f;
+    const float rinv = rinv1 * oscale;
+    auto ld = [&](int d) { return __bfloat162float(*reinterpret_cast<const bf16*>(tile_elem(h0, h1, r, d))); };
+    auto st = [&](int d, float v) {
+        if constexpr (F16)
+            *reinterpret_cast<__half*>(tile_elem(h0, h1, r, d)) = __float2half_rn(v);
+        else
+            *reinterpret_cast<bf16*>(tile_elem(h0, h1, r, d)) = __float2bfloat16_rn(v);
+    };
+    const int rh = L.rope_half;
+#pragma unroll 1
+    for (int t = 0; t < rh; ++t) {
+        const float a = (ld(t) * rinv) * gamma[t], bb = (ld(t + rh) * rinv) * gamma[t + rh];
+        float c, sn;
+        rope_cs(L.theta[t], pos, c, sn);
+        st(t, fmaf(a, c, -(bb * sn)));
+        st(t + rh, fmaf(bb, c, a * sn));
+    }
+#pragma unroll 1
+    for (int d = 2 * rh; d < kD; ++d) st(d, (ld(d) * rinv) * gamma[d]);
+    return rinv1;
+}
+
 template <bool F16 = false>
 __device__ __forceinline__ float tf_prologue_row(unsigned char* h0, unsigned char* h1, int r, const float* gamma,
                                                 const LayerParams& L, const float2 (*cs)[TF_BM],

@@ -9,7 +9,6 @@
 #include "common.cuh"
 
 namespace zgcm {
-cudaError_t launch_fwd_mma(const FwdParams& p, cudaStream_t stream);
 cudaError_t launch_fwd_tc(const FwdParams& p, void* workspace, int* err_word, cudaStream_t stream,
                           const SavedAct* sv);
 bool fwd_tc_supported(const LayerParams& L);
@@ -23,9 +22,6 @@ cudaError_t launch_selftest_expired_wait(int* err_word, cudaStream_t stream);
 cudaError_t launch_decode(const LayerParams& L, const int* pos, void* k_cache, void* v_cache, int C, void* out,
                           float* lse, void* workspace, cudaStream_t stream);
 size_t fwd_glob_workspace_bytes(int B, int S, int Hkv);
-cudaError_t launch_bwd_mma(const BwdParams& p, cudaStream_t stream, void* const* events, int n_pairs);
-extern const char* const kBwdMmaKernelNames[];
-extern const int kBwdMmaKernelCount;
 cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, cudaStream_t stream,
                           void* const* events, int n_pairs, const SavedAct* sv);
 extern const char* const kBwdTcSavedKernelNames[];
@@ -39,8 +35,6 @@ extern const int kBwdWideKernelCount;
 size_t bwd_tc_workspace_bytes(int B, int S, int Hq, int Hkv);
 extern const char* const kBwdTcKernelNames[];
 extern const int kBwdTcKernelCount;
-int bwd_mma_n_k_parts(int B, int S, int Hkv);
-long long bwd_mma_n_q_parts(int B, int S, int Hq);
 }  // namespace zgcm
 
 using namespace zgcm;
@@ -56,26 +50,17 @@ int* device_error_word() {
     return cudaGetSymbolAddress(&ptr, zgcm_device_error_word) == cudaSuccess ? static_cast<int*>(ptr) : nullptr;
 }
 
-// Kernel choice: the tcgen05 sliding-window kernel where it applies, unless the caller
-// asks for the warp-MMA kernels with ZGCM_FORCE_MMA=1 (used to test both paths).
-bool force_mma() {
-    const char* e = getenv("ZGCM_FORCE_MMA");
-    return e && e[0] == '1';
-}
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Forward kernel for a layer: the strip kernel (W <= 128, 4 query heads per KV head), the
-// sliding-window tcgen05 kernel (W <= 128, other group sizes), the wide-window / global
-// tcgen05 pair (W > 128), else (or with ZGCM_FORCE_MMA=1) the warp-MMA kernel.
-enum class FwdPath { STRIP, TC, GLOB, MMA };
+// sliding-window tcgen05 kernel (W <= 128, other group sizes) or the wide-window / global
+// tcgen05 pair (W > 128).  Every shape the arguments allow has one of them.
+enum class FwdPath { STRIP, TC, GLOB };
 
 FwdPath fwd_path(const LayerParams& L) {
-    if (force_mma()) return FwdPath::MMA;
     if (fwd_strip_supported(L)) return FwdPath::STRIP;
     if (fwd_tc_supported(L)) return FwdPath::TC;
-    if (fwd_glob_supported(L)) return FwdPath::GLOB;
-    return FwdPath::MMA;
+    return FwdPath::GLOB;
 }
 
 LayerParams shape_only(int B, int S, int Hq, int Hkv, int rope_dims, int window) {
@@ -123,28 +108,6 @@ void fill_layer(LayerParams& L, const void* q, const void* k, const void* v, con
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-struct BwdWorkspace {
-    size_t delta, lse2, dA, dA_lo, dgk, dgq, total;
-    int n_k_parts;
-    long long n_q_parts;
-};
-
-BwdWorkspace bwd_layout(int B, int S, int Hq, int Hkv) {
-    BwdWorkspace w;
-    const size_t rows = (size_t)B * S * Hq;
-    w.n_k_parts = bwd_mma_n_k_parts(B, S, Hkv);
-    w.n_q_parts = bwd_mma_n_q_parts(B, S, Hq);
-    size_t off = 0;
-    w.delta = off; off = align256(off + rows * sizeof(float));
-    w.lse2 = off;  off = align256(off + rows * sizeof(float));
-    w.dA = off;    off = align256(off + rows * kD * sizeof(bf16));
-    w.dA_lo = off; off = align256(off + rows * kD * sizeof(bf16));
-    w.dgk = off;   off = align256(off + (size_t)w.n_k_parts * kD * sizeof(float));
-    w.dgq = off;   off = align256(off + (size_t)w.n_q_parts * kD * sizeof(float));
-    w.total = off;
-    return w;
-}
-
 // The activation store a forward leaves for the backward: Q~ fp16 [B,S,Hq,D], the q rows'
 // inverse RMS fp32 [B,Hq,S], K~ fp16 [B,S,Hkv,D] (the forward's own K~ workspace) and the k
 // rows' inverse RMS fp32 [B,Hkv,S], each 256-byte aligned.
@@ -164,11 +127,8 @@ size_t saved_layout(int B, int S, int Hq, int Hkv, char* base, SavedAct* sv) {
     return off;
 }
 
-// The store applies where both passes run the tcgen05 kernels.
-bool saved_supported(const LayerParams& L) {
-    const FwdPath f = fwd_path(L);
-    return f != FwdPath::MMA && (bwd_tc_supported(L) || bwd_wide_supported(L));
-}
+// The store applies to every shape (both passes run tcgen05 kernels throughout).
+bool saved_supported(const LayerParams& L) { return L.S >= 1 && L.B >= 1; }
 
 }  // namespace
 
@@ -195,7 +155,7 @@ size_t zgcm_attn_fwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int ro
     // the tcgen05 forwards other than the strip kernel read K~ (fp16, normalised and rotated
     // once per key tile) from it; the strip kernel normalises its key chunks in shared memory
     const FwdPath f = fwd_path(shape_only(B, S, Hq, Hkv, rope_dims, window));
-    return (f == FwdPath::TC || f == FwdPath::GLOB) ? align256(fwd_glob_workspace_bytes(B, S, Hkv)) : 0;
+    return f != FwdPath::STRIP ? align256(fwd_glob_workspace_bytes(B, S, Hkv)) : 0;
 }
 
 }  // extern "C"
@@ -241,8 +201,7 @@ int zgcm_attn_fwd_ws(const void* q, const void* k, const void* v, const void* g,
     switch (fwd_path(p.L)) {
         case FwdPath::STRIP: e = launch_fwd_strip(p, device_error_word(), stream, nullptr); break;
         case FwdPath::TC: e = launch_fwd_tc(p, workspace, device_error_word(), stream, nullptr); break;
-        case FwdPath::GLOB: e = launch_fwd_glob_tc(p, workspace, device_error_word(), stream, nullptr); break;
-        default: e = launch_fwd_mma(p, stream); break;
+        default: e = launch_fwd_glob_tc(p, workspace, device_error_word(), stream, nullptr); break;
     }
     return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
 }
@@ -350,17 +309,14 @@ const char* zgcm_attn_fwd_kernel_name(int B, int S, int Hq, int Hkv, int rope_di
     switch (fwd_path(shape_only(B, S, Hq, Hkv, rope_dims, window))) {
         case FwdPath::STRIP: return "fwd_strip_kernel";
         case FwdPath::TC: return "fwd_tc_kernel";
-        case FwdPath::GLOB: return "fwd_glob_tc_kernel";
-        default: return "fwd_mma_kernel";
+        default: return "fwd_glob_tc_kernel";
     }
 }
 
 size_t zgcm_attn_bwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int window) {
     if (check_shape(B, S, Hq, Hkv, D, 0, 1.0, window, 1, 0.f, 1.f) != ZGCM_OK) return 0;
     if ((long long)B * S == 0) return 0;
-    // enough for either backward (the kernel choice also depends on rope_dims)
-    const size_t a = bwd_layout(B, S, Hq, Hkv).total, b = bwd_tc_workspace_bytes(B, S, Hq, Hkv);
-    return a > b ? a : b;
+    return bwd_tc_workspace_bytes(B, S, Hq, Hkv);
 }
 
 }  // extern "C"
@@ -388,11 +344,9 @@ int bwd_run(const void* q, const void* k, const void* v, const void* g, const fl
         if (!p) return ZGCM_ERR_INVALID_ARG;
     for (const void* p : ptrs)
         if (!aligned16(p)) return ZGCM_ERR_ALIGNMENT;
-    const BwdWorkspace w = bwd_layout(B, S, Hq, Hkv);
     const size_t need = zgcm_attn_bwd_workspace_size(B, S, Hq, Hkv, D, window);
     if (!workspace || workspace_bytes < need) return ZGCM_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ZGCM_ERR_ALIGNMENT;
-    if (w.n_q_parts > 0x7fffffffLL) return ZGCM_ERR_UNSUPPORTED;
 
     BwdParams p;
     fill_layer(p.L, q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, rope_dims, rope_base, window, eps, scale);
@@ -405,15 +359,6 @@ int bwd_run(const void* q, const void* k, const void* v, const void* g, const fl
     p.dg = static_cast<bf16*>(dg);
     p.dgamma_q = dgamma_q;
     p.dgamma_k = dgamma_k;
-    char* ws = static_cast<char*>(workspace);
-    p.delta = reinterpret_cast<float*>(ws + w.delta);
-    p.lse2 = reinterpret_cast<float*>(ws + w.lse2);
-    p.dA = reinterpret_cast<bf16*>(ws + w.dA);
-    p.dA_lo = reinterpret_cast<bf16*>(ws + w.dA_lo);
-    p.dgk_part = reinterpret_cast<float*>(ws + w.dgk);
-    p.dgq_part = reinterpret_cast<float*>(ws + w.dgq);
-    p.n_k_parts = w.n_k_parts;
-    p.n_q_parts = (int)w.n_q_parts;
     if (n_pairs < 0 || (n_pairs > 0 && !events)) return ZGCM_ERR_INVALID_ARG;
     SavedAct sv;
     if (saved) {
@@ -422,11 +367,8 @@ int bwd_run(const void* q, const void* k, const void* v, const void* g, const fl
         if (reinterpret_cast<uintptr_t>(saved) & 255u) return ZGCM_ERR_ALIGNMENT;
         saved_layout(B, S, Hq, Hkv, static_cast<char*>(const_cast<void*>(saved)), &sv);
     }
-    cudaError_t e;
-    if (!force_mma() && (bwd_tc_supported(p.L) || bwd_wide_supported(p.L)))
-        e = launch_bwd_tc(p, workspace, device_error_word(), stream, events, n_pairs, saved ? &sv : nullptr);
-    else
-        e = launch_bwd_mma(p, stream, events, n_pairs);
+    const cudaError_t e =
+        launch_bwd_tc(p, workspace, device_error_word(), stream, events, n_pairs, saved ? &sv : nullptr);
     return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
 }
 }  // namespace
@@ -467,10 +409,10 @@ const char* zgcm_attn_bwd_saved_kernel_name(int i, int S, int rope_dims, int win
     L.B = 1; L.S = S; L.rope_half = rope_dims / 2; L.W = window;
     const char* const* names = nullptr;
     int n = 0;
-    if (!force_mma() && S >= 1 && bwd_tc_supported(L)) {
+    if (S >= 1 && bwd_tc_supported(L)) {
         names = kBwdTcSavedKernelNames;
         n = kBwdTcSavedKernelCount;
-    } else if (!force_mma() && S >= 1 && bwd_wide_supported(L)) {
+    } else if (S >= 1 && bwd_wide_supported(L)) {
         names = kBwdWideSavedKernelNames;
         n = kBwdWideSavedKernelCount;
     }
@@ -480,12 +422,12 @@ const char* zgcm_attn_bwd_saved_kernel_name(int i, int S, int rope_dims, int win
 const char* zgcm_attn_bwd_kernel_name(int i, int S, int rope_dims, int window) {
     LayerParams L{};
     L.B = 1; L.S = S; L.rope_half = rope_dims / 2; L.W = window;
-    const char* const* names = kBwdMmaKernelNames;
-    int n = kBwdMmaKernelCount;
-    if (!force_mma() && S >= 1 && bwd_tc_supported(L)) {
+    const char* const* names = nullptr;
+    int n = 0;
+    if (S >= 1 && bwd_tc_supported(L)) {
         names = kBwdTcKernelNames;
         n = kBwdTcKernelCount;
-    } else if (!force_mma() && S >= 1 && bwd_wide_supported(L)) {
+    } else if (S >= 1 && bwd_wide_supported(L)) {
         names = kBwdWideKernelNames;
         n = kBwdWideKernelCount;
     }

@@ -92,11 +92,14 @@ int zgcm_attn_fwd(const void* q, const void* k, const void* v, const void* g,
                   void* out, float* lse, void* cuda_stream);
 
 /*
- * Bytes of device scratch the forward needs for this configuration: B*S*Hkv*D*2 rounded up
- * to 256 wherever a tcgen05 forward runs (42 rotated dims; any window up to 128, or wider
- * windows with an even Hq/Hkv): the fp16 normalised, rotated keys, written once per key
- * tile by the forward's preparation kernel (fwd_prep_k_kernel) and read by its attention
- * kernel.  0 for the warp-MMA kernel and for invalid arguments.
+ * Bytes of device scratch the forward needs for this configuration.  0 for the sliding layer
+ * with 4 query heads per KV head (window up to 128: the strip kernel normalises its key
+ * chunks in shared memory, so zgcm_attn_fwd allocates nothing there), for an empty problem
+ * and for invalid arguments.  Otherwise (wider windows, the global layer among them, and
+ * sliding windows with another group size) B*S*Hkv*D*2 rounded up to 256: the fp16
+ * normalised, rotated keys, written once per key tile by the preparation kernel
+ * (fwd_prep_k_kernel) and read by every query block that sees the tile; zgcm_attn_fwd takes
+ * them from the stream-ordered pool of the caller's stream (cudaMallocAsync / cudaFreeAsync).
  */
 size_t zgcm_attn_fwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int rope_dims, int window);
 
@@ -120,17 +123,15 @@ int zgcm_attn_fwd_ws(const void* q, const void* k, const void* v, const void* g,
  * there instead of converting q and k again (its preparation pass converts v alone).  The
  * results are bit-identical to zgcm_attn_fwd + zgcm_attn_bwd on the same inputs.
  *
- * zgcm_attn_saved_size: bytes of the store for this problem; 0 for an empty problem and
- *   where the pair does not apply (it needs the tcgen05 kernels: rope_dims == 42 and, for
- *   windows wider than 128, an even Hq/Hkv; not with ZGCM_FORCE_MMA=1).
+ * zgcm_attn_saved_size: bytes of the store for this problem (every shape zgcm_attn_fwd
+ *   accepts); 0 for an empty problem and for invalid arguments.
  * Layout (each part 256-byte aligned, in this order): q~ fp16 [B,S,Hq,D], q inverse RMS fp32
  *   [B,Hq,S], k~ fp16 [B,S,Hkv,D], k inverse RMS fp32 [B,Hkv,S].
  * zgcm_attn_fwd_save: zgcm_attn_fwd_ws with the store as its workspace (k~ is the forward's
  *   own key workspace).  `saved`: at least zgcm_attn_saved_size bytes, 256-byte aligned,
  *   owned by the caller; after the call (in stream order) it holds this forward's
- *   activations.  Returns ZGCM_ERR_UNSUPPORTED where zgcm_attn_saved_size is 0 for a
- *   non-empty problem, ZGCM_ERR_WORKSPACE / ZGCM_ERR_ALIGNMENT for a store too small or
- *   misaligned; otherwise as zgcm_attn_fwd.
+ *   activations.  Returns ZGCM_ERR_WORKSPACE / ZGCM_ERR_ALIGNMENT for a store too
+ *   small or misaligned; otherwise as zgcm_attn_fwd.
  * zgcm_attn_bwd_saved: zgcm_attn_bwd_timed given the store a zgcm_attn_fwd_save of the same
  *   inputs and arguments filled (`saved`, read only; NULL returns ZGCM_ERR_INVALID_ARG).
  *   Kernels: zgcm_attn_bwd_saved_kernel_name(i) (bwd_prep_v_kernel in place of the two
@@ -271,12 +272,12 @@ int zgcm_attn_decode(const void* q, const void* k, const void* v, const void* g,
 size_t zgcm_attn_decode_workspace_size(int B, int Hq, int window, int cache_len);
 
 /*
- * Main kernel zgcm_attn_fwd launches for this configuration (static string):
- * "fwd_tc_kernel" (tcgen05/TMEM/TMA, sliding windows up to 128 with 42 rotated dims),
- * "fwd_glob_tc_kernel" (tcgen05, wider windows and the global layer, with 42 rotated dims
- * and an even Hq/Hkv), each preceded by the key preparation kernel fwd_prep_k_kernel, or
- * "fwd_mma_kernel" (warp MMA, every other shape).  Setting the environment variable
- * ZGCM_FORCE_MMA=1 selects the warp-MMA kernels.
+ * Main kernel zgcm_attn_fwd launches for this configuration (static string), all of them
+ * tcgen05 / TMEM / TMA kernels for any number of rotated dims: "fwd_strip_kernel" (windows
+ * up to 128 with 4 query heads per KV head; in the training pair the Q and K preparation
+ * kernels run before it), "fwd_tc_kernel" (windows up to 128, other group sizes) and
+ * "fwd_glob_tc_kernel" (wider windows and the global layer), these two preceded by the key
+ * preparation kernel fwd_prep_k_kernel.
  */
 const char* zgcm_attn_fwd_kernel_name(int B, int S, int Hq, int Hkv, int rope_dims, int window);
 
@@ -297,12 +298,11 @@ int zgcm_attn_device_error(void);
 int zgcm_attn_selftest_expired_wait(void* cuda_stream);
 
 /* Name of the i-th kernel zgcm_attn_bwd launches for this configuration (static string),
- * or NULL when i is past the last one.  With 42 rotated dims, windows up to 128 run the
- * gate pass, the K/V and Q preparation and the tcgen05 pair (bwd_gate_kernel,
- * bwd_prep_kv_kernel, bwd_prep_q_kernel, bwd_q_tc_kernel, bwd_kv_tc_kernel, then the two
- * d_gamma reductions); wider windows (the global layer among them) the same gate pass and
- * preparation, then bwd_tile_stats_kernel, bwd_q_glob_kernel, bwd_kv_tc_kernel and the two
- * reductions; other shapes, or ZGCM_FORCE_MMA=1, the warp-MMA kernels. */
+ * or NULL when i is past the last one.  Windows up to 128 run the gate pass, the K/V and Q
+ * preparation and the tcgen05 pair (bwd_gate_kernel, bwd_prep_kv_kernel, bwd_prep_q_kernel,
+ * bwd_q_tc_kernel, bwd_kv_tc_kernel, then the two d_gamma reductions); wider windows (the
+ * global layer among them) the same gate pass and preparation, then bwd_tile_stats_kernel,
+ * bwd_q_glob_kernel, bwd_kv_tc_kernel and the two reductions.  Any number of rotated dims. */
 const char* zgcm_attn_bwd_kernel_name(int i, int S, int rope_dims, int window);
 
 #ifdef __cplusplus

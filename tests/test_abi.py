@@ -133,9 +133,11 @@ def test_fwd_workspace_size_query(lib):
         assert ws(B, S, 32, 8, 128, 42, W) == (n + 255) // 256 * 256
     # other group sizes of the sliding layer take the per-head tcgen05 kernel, which reads them too
     assert ws(1, 1024, 16, 8, 128, 42, 128) == (1024 * 8 * 256 + 255) // 256 * 256
-    # the warp-MMA kernel takes the rest (no rotation, odd group size) and needs none
-    assert ws(1, 1024, 32, 8, 128, 0, 1024) == 0
-    assert ws(1, 1024, 24, 8, 128, 42, 1024) == 0
+    # any number of rotated dims and any group size: the same rule
+    assert ws(1, 1024, 32, 8, 128, 0, 1024) == (1024 * 8 * 256 + 255) // 256 * 256
+    assert ws(1, 1024, 32, 8, 128, 128, 128) == 0
+    assert ws(1, 1024, 24, 8, 128, 42, 1024) == (1024 * 8 * 256 + 255) // 256 * 256
+    assert ws(1, 1024, 8, 8, 128, 0, 64) == (1024 * 8 * 256 + 255) // 256 * 256
     # invalid or empty -> 0
     assert ws(1, 1024, 32, 8, 64, 42, 1024) == 0
     assert ws(0, 1024, 32, 8, 128, 42, 1024) == 0
@@ -159,8 +161,10 @@ def test_saved_size_query(lib):
     for B, S, W in ((4, 16384, 128), (1, 1000, 7), (2, 777, 10**6), (1, 1, 128), (3, 260, 129)):
         rows, krows = B * S * 32, B * S * 8
         assert sz(B, S, 32, 8, 128, 42, W) == al(rows * 256) + al(rows * 4) + al(krows * 256) + al(krows * 4)
-    assert sz(1, 1024, 32, 8, 128, 0, 128) == 0       # no rotation: the warp-MMA kernels
-    assert sz(1, 1024, 24, 8, 128, 42, 1024) == 0     # odd group size with a wide window: likewise
+    # every shape: no rotation, all dims rotated, an odd group size with a wide window
+    for Hq, R, W in ((32, 0, 128), (32, 128, 1024), (24, 42, 1024)):
+        rows, krows = 1024 * Hq, 1024 * 8
+        assert sz(1, 1024, Hq, 8, 128, R, W) == al(rows * 256) + al(rows * 4) + al(krows * 256) + al(krows * 4)
     assert sz(0, 1024, 32, 8, 128, 42, 128) == 0      # empty
     assert sz(1, 1024, 32, 8, 64, 42, 128) == 0       # invalid
 
@@ -190,14 +194,14 @@ def test_saved_pair_checks(lib):
     assert _fwd_save(lib, store, need - 1) == -4          # too small
     assert _fwd_save(lib, 0, need) == -4                  # missing
     assert _fwd_save(lib, store + 16, need) == -3         # not 256-byte aligned
-    assert _fwd_save(lib, store, need, rope_dims=0) == -2  # the pair needs the tcgen05 kernels
+    assert _fwd_save(lib, store, need, D=96) == -2        # head size other than 128
     assert _fwd_save(lib, store, need, window=0) == -1
     ws = lib.zgcm_attn_bwd_workspace_size(1, 64, 32, 8, 128, 128)
     assert _bwd_saved(lib, ws, 0, need) == -1             # the store is required
     assert _bwd_saved(lib, ws, store, need - 1) == -4
     assert _bwd_saved(lib, ws, store + 16, need) == -3
     assert _bwd_saved(lib, ws - 1, store, need) == -4     # the workspace is checked as before
-    assert _bwd_saved(lib, ws, store, need, rope_dims=0) == -2
+    assert _bwd_saved(lib, ws, store, need, D=96) == -2
     names = ga.zgcm_attn_bwd_kernel_names(16384, 128, saved=True)
     assert names[:4] == ["bwd_gate_kernel", "bwd_prep_v_kernel", "bwd_q_tc_kernel", "bwd_kv_tc_kernel"]
     assert "bwd_prep_q_kernel" not in ga.zgcm_attn_bwd_kernel_names(4096, 4096, saved=True)

@@ -34,8 +34,9 @@ def test_kept_activations_change_kernels_not_the_step():
     # the forward that keeps q~ (fp16) and every q and k row's inverse RMS writes them once more
     extra = QB + TOK * 32 * 4 + TOK * 8 * 4
     assert kept["kernels"]["fwd_tc_kernel"][0] - plain["kernels"]["fwd_tc_kernel"][0] == extra
-    # the strip forward normalises its keys in shared memory and, keeping them, writes k~ too
-    assert kept["kernels"]["fwd_strip_kernel"][0] - plain["kernels"]["fwd_strip_kernel"][0] == extra + KB
+    # the strip forward normalises its keys in shared memory; in the training pair it reads the
+    # q~ and k~ fp16 that the preparation kernels wrote, the same bytes as raw q and k
+    assert kept["kernels"]["fwd_strip_kernel"][0] == plain["kernels"]["fwd_strip_kernel"][0]
     assert plain["kernels"]["fwd_strip_kernel"][0] == plain["fwd_bytes"]
     # the V-only preparation: read v, write V fp16 and a norm per row
     assert kept["kernels"]["bwd_prep_v_kernel"][0] == 2 * KB + TOK * 8 * 4
@@ -67,9 +68,24 @@ def test_clock_summary_median_and_reasons():
     """The clocks record of the JSON line: median SM clock over the samples, the maximum, and
     every throttle reason seen active (a run showing a hardware or thermal one is re-taken)."""
     cs = bench.ClockSampler("GPU-test")
-    cs.rows = [_row(1965), _row(1320, ("sw_power_cap",)), _row(1500, ("sw_power_cap",)), ["malformed"], []]
-    assert cs.summary() == {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
-    cs.rows = [_row(1100, ("hw_slowdown",)), _row(1200, ("sw_thermal_slowdown", "sw_power_cap"))]
+    rows = [_row(1965), _row(1320, ("sw_power_cap",)), _row(1500, ("sw_power_cap",)), ["malformed"], []]
+    cs.rows = [(float(i), r) for i, r in enumerate(rows)]
+    assert cs.summary() == {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3,
+                            "window": "all"}
+    cs.rows = [(0.0, _row(1100, ("hw_slowdown",))), (1.0, _row(1200, ("sw_thermal_slowdown", "sw_power_cap")))]
     assert cs.summary()["reasons"] == ["hw_slowdown", "sw_power_cap", "sw_thermal_slowdown"]
     cs.rows = []
     assert cs.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+def test_clock_summary_keeps_the_timed_region():
+    """Rows inside the marked region count; the idle rows before it and the rows after it do
+    not.  A region shorter than the sampling interval takes the two rows around it."""
+    cs = bench.ClockSampler("GPU-test")
+    cs.rows = [(0.0, _row(900)), (1.0, _row(1900, ("sw_power_cap",))), (1.5, _row(1880)), (3.0, _row(700))]
+    cs.t_start, cs.t_end = 0.5, 2.0
+    assert cs.summary() == {"sm_mhz": 1890.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 2,
+                            "window": "timed region"}
+    cs.t_start, cs.t_end = 1.1, 1.2
+    sm = cs.summary()
+    assert (sm["samples"], sm["window"], sm["sm_mhz"]) == (2, "bracketing", 1890.0)

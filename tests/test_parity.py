@@ -86,22 +86,65 @@ def test_small_full_compare(B, S, Hq, Hkv, W, R, base):
 
 @pytest.mark.parametrize("B,S,W", [(1, 1024, 128), (2, 1000, 128), (1, 129, 7), (3, 260, 1), (1, 1, 128),
                                    (2, 384, 100)])
-def test_forward_both_kernel_paths(B, S, W, monkeypatch):
-    """The tcgen05 strip kernel (default for W <= 128, 4 query heads per KV head, 42 rotated
-    dims) and the warp-MMA kernel (forced) both match the oracle on the same inputs."""
+def test_forward_strip_kernel(B, S, W):
+    """The strip kernel (windows up to 128, 4 query heads per KV head) matches the oracle."""
     t = make_inputs(B, S, seed=100 + S + W)
     d = _to_dev(t)
     ref_out, ref_lse = _problem(t, window=W).forward()
-    monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
     assert ga.zgcm_attn_fwd_kernel_name(B, S, 32, 8, 42, W) == "fwd_strip_kernel"
-    out_tc, lse_tc = _gpu_fwd(d, window=W)
+    out, lse = _gpu_fwd(d, window=W)
     assert ga.zgcm_attn_device_error() == 0
-    monkeypatch.setenv("ZGCM_FORCE_MMA", "1")
-    assert ga.zgcm_attn_fwd_kernel_name(B, S, 32, 8, 42, W) == "fwd_mma_kernel"
-    out_mma, lse_mma = _gpu_fwd(d, window=W)
-    for name, o, l in (("tc", out_tc, lse_tc), ("mma", out_mma, lse_mma)):
-        assert_bf16_close(f"out[{name}]", o, ref_out)
-        assert_lse_close(f"lse[{name}]", l, ref_lse)
+    assert_bf16_close("out", out, ref_out)
+    assert_lse_close("lse", lse, ref_lse)
+
+
+# Shapes off the layer's own (42 rotated dims, 4 query heads per KV head): every kernel has a
+# second instance for any number of rotated pairs, and the per-head and wide-window kernels
+# take any group size (odd ones included).  (B, S, Hq, Hkv, W, rope_dims, forward kernel)
+OTHER_SHAPES = [
+    (1, 700, 32, 8, 128, 0, "fwd_strip_kernel"),       # no rotation
+    (2, 300, 32, 8, 77, 128, "fwd_strip_kernel"),      # every dim rotated
+    (1, 520, 32, 8, 128, 64, "fwd_strip_kernel"),
+    (1, 650, 24, 8, 128, 42, "fwd_tc_kernel"),         # 3 query heads per KV head
+    (2, 260, 16, 2, 100, 126, "fwd_tc_kernel"),        # 8 per KV head
+    (1, 300, 8, 8, 1, 2, "fwd_tc_kernel"),             # plain multi-head, window 1
+    (1, 900, 24, 8, 900, 42, "fwd_glob_tc_kernel"),    # odd group, global layer
+    (2, 400, 8, 8, 300, 2, "fwd_glob_tc_kernel"),      # one query head per KV head
+    (1, 333, 40, 8, 10**6, 0, "fwd_glob_tc_kernel"),   # 5 per KV head, no rotation
+    (1, 500, 6, 2, 200, 128, "fwd_glob_tc_kernel"),    # 3 per KV head, every dim rotated
+]
+
+
+@pytest.mark.parametrize("B,S,Hq,Hkv,W,R,kname", OTHER_SHAPES)
+def test_other_shapes_forward_backward(B, S, Hq, Hkv, W, R, kname):
+    """Forward and backward on the shapes above match the oracle, through the kernel named."""
+    t = make_inputs(B, S, Hq=Hq, Hkv=Hkv, seed=900 + S + R + W % 1000, with_dout=True)
+    kw = dict(window=W, rope_dims=R)
+    d = _to_dev(t)
+    P = _problem(t, **kw)
+    ref_out, ref_lse = P.forward()
+    assert ga.zgcm_attn_fwd_kernel_name(B, S, Hq, Hkv, R, W) == kname
+    out, lse = _gpu_fwd(d, **kw)
+    assert ga.zgcm_attn_device_error() == 0
+    assert_bf16_close("out", out, ref_out)
+    assert_lse_close("lse", lse, ref_lse)
+    gr = _gpu_bwd(d, out, lse, **kw)
+    assert ga.zgcm_attn_device_error() == 0
+    ref = P.backward(t["dout"])
+    for n in ("dq", "dk", "dv", "dg"):
+        assert_bf16_close(n, gr[n], ref[n])
+    assert_dgamma_close("dgamma_q", gr["dgamma_q"], ref["dgamma_q"])
+    assert_dgamma_close("dgamma_k", gr["dgamma_k"], ref["dgamma_k"])
+    # the training pair on the same shape: bit-identical to the plain pair
+    n = ga.zgcm_attn_saved_size(B, S, Hq, Hkv, rope_dims=R, window=W)
+    assert n > 0
+    saved = torch.full((n,), 0xAB, dtype=torch.uint8, device="cuda")
+    out_s, lse_s = _gpu_fwd(d, saved=saved, **kw)
+    assert torch.equal(out, out_s) and torch.equal(lse, lse_s)
+    gr_s = _gpu_bwd(d, out_s, lse_s, saved=saved, **kw)
+    assert ga.zgcm_attn_device_error() == 0
+    for name in gr:
+        assert torch.equal(gr[name], gr_s[name]), name
 
 
 @pytest.mark.parametrize("gq_all,spike,B,S,W", [
@@ -109,7 +152,7 @@ def test_forward_both_kernel_paths(B, S, W, monkeypatch):
     (1.9, None, 2, 700, 128),      # gamma 1.9 everywhere: bound just under the limit (59.2)
     (2.0, None, 1, 333, 37),       # gamma 2.0 everywhere: just over it (65.6)
 ])
-def test_forward_score_bound_fallback(gq_all, spike, B, S, W, monkeypatch):
+def test_forward_score_bound_fallback(gq_all, spike, B, S, W):
     """The sliding-window forward takes its exponentials' reference from a bound on every
     score, |scale| log2(e) D max|gamma_q| max|gamma_k|, when that bound is at most 60, and
     from each row's maximum otherwise.  Both sides of the limit, and a bound far above it,
@@ -122,7 +165,6 @@ def test_forward_score_bound_fallback(gq_all, spike, B, S, W, monkeypatch):
     t["gamma_k"] = torch.full((128,), gq_all, dtype=torch.float32)
     d = _to_dev(t)
     ref_out, ref_lse = _problem(t, window=W).forward()
-    monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
     assert ga.zgcm_attn_fwd_kernel_name(B, S, 32, 8, 42, W) == "fwd_strip_kernel"
     out, lse = _gpu_fwd(d, window=W)
     assert ga.zgcm_attn_device_error() == 0
@@ -132,13 +174,12 @@ def test_forward_score_bound_fallback(gq_all, spike, B, S, W, monkeypatch):
 
 @pytest.mark.parametrize("B,S,W", [(1, 777, 777), (2, 1000, 10**6), (1, 129, 129), (1, 1, 4096),
                                    (3, 260, 200), (1, 1300, 300), (2, 640, 129), (1, 2048, 2048)])
-def test_forward_wide_window_kernel(B, S, W, monkeypatch):
+def test_forward_wide_window_kernel(B, S, W):
     """Windows wider than one key tile (the global layer W >= S among them) run the tcgen05
-    wide-window forward; it matches the oracle and the forced warp-MMA kernel's tolerance."""
+    wide-window forward; it matches the oracle."""
     t = make_inputs(B, S, seed=300 + S + W % 1000)
     d = _to_dev(t)
     ref_out, ref_lse = _problem(t, window=W).forward()
-    monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
     assert ga.zgcm_attn_fwd_kernel_name(B, S, 32, 8, 42, W) == "fwd_glob_tc_kernel"
     out, lse = _gpu_fwd(d, window=W)
     assert ga.zgcm_attn_device_error() == 0
@@ -159,37 +200,31 @@ def test_forward_wide_window_kernel(B, S, W, monkeypatch):
 
 @pytest.mark.parametrize("B,S,W", [(1, 1024, 128), (2, 1000, 128), (1, 129, 7), (3, 260, 1), (1, 1, 128),
                                    (2, 384, 100)])
-def test_backward_both_kernel_paths(B, S, W, monkeypatch):
-    """The tcgen05 backward pair (default for W <= 128, 42 rotated dims) and the warp-MMA
-    backward (forced) both match the oracle's gradients on the same inputs."""
+def test_backward_sliding_kernels(B, S, W):
+    """The tcgen05 backward pair of windows up to 128 matches the oracle's gradients."""
     t = make_inputs(B, S, seed=200 + S + W, with_dout=True)
     d = _to_dev(t)
     ref = _problem(t, window=W).backward(t["dout"])
-    monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
     assert ga.zgcm_attn_bwd_kernel_names(S, W)[:5] == ["bwd_gate_kernel", "bwd_prep_kv_kernel", "bwd_prep_q_kernel",
                                                         "bwd_q_tc_kernel", "bwd_kv_tc_kernel"]
     out, lse = _gpu_fwd(d, window=W)
-    got_tc = _gpu_bwd(d, out, lse, window=W)
+    gr = _gpu_bwd(d, out, lse, window=W)
     assert ga.zgcm_attn_device_error() == 0
-    monkeypatch.setenv("ZGCM_FORCE_MMA", "1")
-    got_mma = _gpu_bwd(d, out, lse, window=W)
-    for name, gr in (("tc", got_tc), ("mma", got_mma)):
-        for n in ("dq", "dk", "dv", "dg"):
-            assert_bf16_close(f"{n}[{name}]", gr[n], ref[n])
-        assert_dgamma_close(f"dgamma_q[{name}]", gr["dgamma_q"], ref["dgamma_q"])
-        assert_dgamma_close(f"dgamma_k[{name}]", gr["dgamma_k"], ref["dgamma_k"])
+    for n in ("dq", "dk", "dv", "dg"):
+        assert_bf16_close(n, gr[n], ref[n])
+    assert_dgamma_close("dgamma_q", gr["dgamma_q"], ref["dgamma_q"])
+    assert_dgamma_close("dgamma_k", gr["dgamma_k"], ref["dgamma_k"])
 
 
 @pytest.mark.parametrize("B,S,W", [(1, 777, 777), (2, 1000, 10**6), (1, 129, 129), (1, 1, 4096),
                                    (3, 260, 200), (1, 1300, 300), (2, 640, 129), (1, 2048, 2048)])
-def test_backward_wide_window_kernels(B, S, W, monkeypatch):
+def test_backward_wide_window_kernels(B, S, W):
     """Windows wider than one key tile (the global layer among them) run the tcgen05
     wide-window backward (tile bounds, query-major dq sweep, key-major dk/dv sweep); every
     gradient matches the oracle."""
     t = make_inputs(B, S, seed=400 + S + W % 1000, with_dout=True)
     d = _to_dev(t)
     ref = _problem(t, window=W).backward(t["dout"])
-    monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
     assert ga.zgcm_attn_bwd_kernel_names(S, W) == [
         "bwd_gate_kernel", "bwd_prep_kv_kernel", "bwd_prep_q_kernel", "bwd_tile_stats_kernel",
         "bwd_q_glob_kernel", "bwd_kv_tc_kernel", "dgamma_reduce_kernel(k)", "dgamma_reduce_kernel(q)"]
@@ -227,11 +262,10 @@ def _decode_run(t, W, C, offsets=None, rope_dims=42):
 
 @pytest.mark.parametrize("B,S,W", [(1, 1024, 128), (2, 1000, 128), (1, 129, 7), (3, 260, 1), (1, 1, 128),
                                    (1, 777, 777), (2, 640, 129), (1, 1300, 300)])
-def test_saved_activations_bit_identical(B, S, W, monkeypatch):
+def test_saved_activations_bit_identical(B, S, W):
     """zgcm_attn_fwd(saved=...) then zgcm_attn_bwd(saved=...) gives exactly the results of the
     plain pair: the store holds the q~, k~ and inverse RMS values the backward's preparation
     would form (the store starts out filled with garbage)."""
-    monkeypatch.delenv("ZGCM_FORCE_MMA", raising=False)
     t = make_inputs(B, S, seed=700 + S + W % 1000, with_dout=True)
     d = _to_dev(t)
     out, lse = _gpu_fwd(d, window=W)
