@@ -79,6 +79,10 @@ def load() -> ctypes.CDLL:
         lib.zgcm_attn_device_error.restype = i
         lib.zgcm_attn_bwd_noalloc.argtypes = [vp] * 9 + [i] * 6 + [d, i, i, f, f] + [vp] * 7
         lib.zgcm_attn_bwd_noalloc.restype = i
+        lib.zgcm_attn_fwd_rows.argtypes = [vp] * 6 + [i] * 7 + [d, i, i, f, f] + [vp, vp, vp, ctypes.c_size_t, vp]
+        lib.zgcm_attn_fwd_rows.restype = i
+        lib.zgcm_attn_bwd_rows.argtypes = [vp] * 9 + [i] * 7 + [d, i, i, f, f] + [vp] * 7 + [ctypes.c_size_t, vp]
+        lib.zgcm_attn_bwd_rows.restype = i
         _lib = lib
     return _lib
 
@@ -307,6 +311,67 @@ def zgcm_attn_bwd(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dims=42,
         st = load().zgcm_attn_bwd_timed(*args, arr, n_pairs)
     if st != ZGCM_OK:
         raise ZgcmError(st, "zgcm_attn_bwd")
+    return grads
+
+
+def zgcm_attn_fwd_rows(q, k, v, g, gamma_q, gamma_k, *, rope_dims=42, rope_base=10000.0, window,
+                       causal=1, eps=1e-6, scale=None, out=None, lse=None, workspace=None, stream=None):
+    """Forward of the query rows at the end of a longer key sequence: q, g [B,Sq,Hq,D] are
+    positions S-Sq .. S-1 of k, v [B,S,Hkv,D] (S - Sq a multiple of 128 and window > 128 when
+    Sq < S).  Returns (out bf16 [B,Sq,Hq,D], lse fp32 [B,Hq,Sq]), the rows of the whole
+    sequence's forward."""
+    import torch
+    for n, t in (("q", q), ("k", k), ("v", v), ("g", g)):
+        _check(t, n, torch.bfloat16, 4)
+    _check(gamma_q, "gamma_q", torch.float32, 1)
+    _check(gamma_k, "gamma_k", torch.float32, 1)
+    B, Sq, Hq, D = q.shape
+    S, Hkv = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    need = zgcm_attn_fwd_workspace_size(B, S, Hq, Hkv, D, rope_dims, window)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel())
+    st = load().zgcm_attn_fwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma_q), _ptr(gamma_k),
+                                   B, Sq, S, Hq, Hkv, D, int(rope_dims), float(rope_base), int(window),
+                                   int(causal), float(eps), float(scale), _ptr(out), _ptr(lse),
+                                   ws_ptr, ws_bytes, _stream(stream))
+    if st != ZGCM_OK:
+        raise ZgcmError(st, "zgcm_attn_fwd_rows")
+    return out, lse
+
+
+def zgcm_attn_bwd_rows(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dims=42, rope_base=10000.0,
+                       window, causal=1, eps=1e-6, scale=None, grads=None, workspace=None, stream=None):
+    """Backward of zgcm_attn_fwd_rows: dq, dg of the query rows, dk, dv of every key row and
+    dgamma_q, dgamma_k, each the part these query rows contribute (a dict as zgcm_attn_bwd)."""
+    import torch
+    _check_bwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, dout, grads)
+    B, Sq, Hq, D = q.shape
+    S, Hkv = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if grads is None:
+        grads = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+                     dg=torch.empty_like(g),
+                     dgamma_q=torch.empty(D, dtype=torch.float32, device=q.device),
+                     dgamma_k=torch.empty(D, dtype=torch.float32, device=q.device))
+    need = zgcm_attn_bwd_workspace_size(B, S, Hq, Hkv, D, window)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    st = load().zgcm_attn_bwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma_q), _ptr(gamma_k),
+                                   _ptr(out), _ptr(lse), _ptr(dout), B, Sq, S, Hq, Hkv, D, int(rope_dims),
+                                   float(rope_base), int(window), int(causal), float(eps), float(scale),
+                                   _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]), _ptr(grads["dg"]),
+                                   _ptr(grads["dgamma_q"]), _ptr(grads["dgamma_k"]), _ptr(workspace),
+                                   workspace.numel(), _stream(stream))
+    if st != ZGCM_OK:
+        raise ZgcmError(st, "zgcm_attn_bwd_rows")
     return grads
 
 

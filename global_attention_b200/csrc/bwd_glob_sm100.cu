@@ -26,7 +26,8 @@ namespace zgcm {
 
 // One CTA of 128 threads per (b, KV head, tile t): thread r takes query row t*128 + r of each
 // head of the group and key row t*128 + r.  Writes p.tstat[k][(b*Hkv + kvh)*ntile + t] for
-// k = 0 (max |dout|), 1 (max |Delta|), 2 (max ||v||); rows past S contribute 0.
+// k = 0 (max |dout|), 1 (max |Delta|), 2 (max ||v||); rows past S, and query rows before the
+// first one (q_off), contribute 0.
 __global__ void __launch_bounds__(BTS_THREADS) bwd_tile_stats_kernel(const __grid_constant__ BwdTcParams p) {
     const LayerParams& L = p.P.L;
     const int r = threadIdx.x, lane = r & 31, warp = r >> 5;
@@ -36,7 +37,7 @@ __global__ void __launch_bounds__(BTS_THREADS) bwd_tile_stats_kernel(const __gri
     const int i = t * TF_BN + r;
     float dm = 0.f, dl = 0.f, vn = 0.f;
     if (i < L.S) {
-        for (int h = 0; h < L.G; ++h) {
+        for (int h = 0; h < L.G && i >= L.q_off; ++h) {
             const size_t rp = ((size_t)b * L.Hq + kvh * L.G + h) * Spad + i;
             dm = fmaxf(dm, p.domax[rp]);
             dl = fmaxf(dl, fabsf(p.P.delta[rp]));
@@ -136,7 +137,8 @@ __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid
     BwdQGlobSmem& sm = *reinterpret_cast<BwdQGlobSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     volatile int* abort = &sm.abort;
-    // unit, heaviest first: block qb from the last one down, then batch and head
+    // unit, heaviest first: block qb from the last one down (to the block of the first query
+    // row, q_off / 128: the launcher's unit count), then batch and head
     const int nqb = (L.S + TF_BM - 1) / TF_BM, nkt = nqb;
     const int per_qb = L.B * L.Hq;
     const int u = (int)blockIdx.x;
@@ -318,7 +320,8 @@ __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid
         const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
         const int Spad = row_stride(L.S);
         const size_t rp = ((size_t)b * L.Hq + hq) * Spad + i;
-        const size_t ro = ((size_t)b * L.Hq + hq) * L.S + (valid ? i : 0);
+        const int iq = valid ? i - L.q_off : 0;  // row of the query-side tensors (lse, q, dq)
+        const size_t ro = ((size_t)b * L.Hq + hq) * L.Sq + iq;
         // the forward's log-sum-exp (base 2): its scores are these, bit for bit
         const float lse2 = valid ? p.P.lse[ro] * kLog2e : INFINITY;
         const float dai = valid ? p.dainv[rp] : 0.f;       // undoes the dA row scale
@@ -408,7 +411,7 @@ __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid
             mbar_arrive(&sm.bar[QG_MDOT]);
         } else {
             // ------------------------------------------ dq epilogue: RoPE / RMSNorm backward
-            const size_t off = ((size_t)(b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hq) * kD;
+            const size_t off = ((size_t)(b * (size_t)L.Sq + iq) * L.Hq + hq) * kD;
             const float rinv = valid ? p.qrinv[((size_t)b * L.Hq + hq) * L.S + i] : 0.f;
             uint4 xv0[8];  // first half of the raw q row, in flight during the wait
 #pragma unroll

@@ -52,6 +52,8 @@ constexpr int GATE_UNROLL = 4;  // rows in flight per half-warp
 // fills the entries past S).  With DELTA (wide windows) also Delta = sum_d dout*out
 // per row, [B,Hq,Spad]: the row sum of dA * A (A = out / sigmoid(g)), which the wide-window
 // query-major kernel needs before its first key tile.
+// Rows: dout, g, out, dg are [B,Sq,Hq,D] (positions q_off .. S-1, Sq = S - q_off); da16 and
+// the row arrays are indexed by position ([B,S,Hq,D], [B,Hq,Spad]).
 template <bool DELTA>
 __global__ void __launch_bounds__(GATE_THREADS, 2) bwd_gate_kernel(const bf16* __restrict__ dout,
                                                                 const bf16* __restrict__ g,
@@ -60,7 +62,8 @@ __global__ void __launch_bounds__(GATE_THREADS, 2) bwd_gate_kernel(const bf16* _
                                                                 float* __restrict__ dainv,
                                                                 float* __restrict__ domax,
                                                                 float* __restrict__ delta, long long rows, int S,
-                                                                int Hq) {
+                                                                int Hq, int q_off) {
+    const int Sq = S - q_off;
     const int lane = threadIdx.x & 31, sub = lane & 15;
     const long long warp0 = ((long long)blockIdx.x * GATE_THREADS + threadIdx.x) >> 5;
     const long long nwarps = ((long long)gridDim.x * GATE_THREADS) >> 5;
@@ -109,24 +112,28 @@ __global__ void __launch_bounds__(GATE_THREADS, 2) bwd_gate_kernel(const bf16* _
                 for (int o = 8; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
             }
             if (r < rows) {
-                const size_t o = (size_t)r * (kD / 8) + sub;
-                reinterpret_cast<uint4*>(da16)[o] = make_uint4(da[0], da[1], da[2], da[3]);
-                reinterpret_cast<uint4*>(dg)[o] = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
-                if (sub == 0) {
-                    // row r = (b*S + s)*Hq + h  ->  [B,Hq,S] index (b*Hq + h)*S + s (32-bit
-                    // division where the row count allows: the 64-bit one is a long sequence)
-                    size_t ro;
+                // row r = (b*Sq + s)*Hq + h is position s + q_off: [B,Hq,Spad] index
+                // (b*Hq + h)*Spad + s + q_off, da16 row (b*S + s + q_off)*Hq + h (32-bit
+                // division where the row count allows: the 64-bit one is a long sequence)
+                size_t ro = 0, rda = (size_t)r;
+                if (q_off || sub == 0) {
                     if (rows <= 0xffffffffLL) {
-                        const uint32_t ru = (uint32_t)r, sh = (uint32_t)S * (uint32_t)Hq;
+                        const uint32_t ru = (uint32_t)r, sh = (uint32_t)Sq * (uint32_t)Hq;
                         const uint32_t b = ru / sh, rem = ru - b * sh;
                         const uint32_t s = rem / (uint32_t)Hq, h = rem - s * (uint32_t)Hq;
-                        ro = ((size_t)b * Hq + h) * row_stride(S) + s;
+                        ro = ((size_t)b * Hq + h) * row_stride(S) + s + q_off;
+                        if (q_off) rda = ((size_t)b * S + s + q_off) * Hq + h;
                     } else {
-                        const long long sh = (long long)S * Hq;
+                        const long long sh = (long long)Sq * Hq;
                         const long long b = r / sh, rem = r - b * sh;
                         const long long s = rem / Hq, h = rem - s * Hq;
-                        ro = (size_t)(b * Hq + h) * row_stride(S) + s;
+                        ro = (size_t)(b * Hq + h) * row_stride(S) + s + q_off;
+                        if (q_off) rda = ((size_t)b * S + s + q_off) * Hq + h;
                     }
+                }
+                reinterpret_cast<uint4*>(da16)[rda * (kD / 8) + sub] = make_uint4(da[0], da[1], da[2], da[3]);
+                reinterpret_cast<uint4*>(dg)[(size_t)r * (kD / 8) + sub] = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
+                if (sub == 0) {
                     dainv[ro] = mx > 0.f ? 1.0f / sc : 0.f;
                     domax[ro] = mx;
                     if constexpr (DELTA) delta[ro] = dsum;
@@ -301,7 +308,9 @@ __device__ __forceinline__ void prep_tile(const BwdTcParams& p) {
     PrepSmem<IS_K>& sm =
         *reinterpret_cast<PrepSmem<IS_K>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int r = threadIdx.x;
-    const int nt = (L.S + TF_BN - 1) / TF_BN;
+    // query tiles cover the query rows q_off .. S-1 (tile t at position q_off + 128 t; Q~ and
+    // the inverse RMS are stored by position), key tiles every position
+    const int nt = ((IS_K ? L.S : L.Sq) + TF_BN - 1) / TF_BN, x0 = IS_K ? 0 : L.q_off;
     const int H = IS_K ? L.Hkv : L.Hq;
     const int t = (int)blockIdx.x % nt, chain = (int)blockIdx.x / nt;
     const int h = chain % H, b = chain / H;
@@ -325,7 +334,7 @@ __device__ __forceinline__ void prep_tile(const BwdTcParams& p) {
             tma_load_4d(sm.V[1], &p.tm_v, &sm.bar, 64, h, t * TF_BN, b);
         }
     }
-    const int pos = t * TF_BN + r;
+    const int pos = x0 + t * TF_BN + r;
     float2 csr[WITH_K && !ANY ? TF_HALF : 1];  // (cos, sin) of the rotated pairs at this row's position
     if constexpr (WITH_K && !ANY) {
 #pragma unroll
@@ -362,8 +371,8 @@ __device__ __forceinline__ void prep_tile(const BwdTcParams& p) {
         if (ok) {
             const CUtensorMap* dst = IS_K ? &p.tm_k16 : &p.tm_q16;
             if constexpr (WITH_K) {
-                tma_store_4d(dst, sm.X[0], 0, h, t * TF_BN, b);
-                tma_store_4d(dst, sm.X[1], 64, h, t * TF_BN, b);
+                tma_store_4d(dst, sm.X[0], 0, h, x0 + t * TF_BN, b);
+                tma_store_4d(dst, sm.X[1], 64, h, x0 + t * TF_BN, b);
             }
             if constexpr (IS_K) {
                 tma_store_4d(&p.tm_v16, sm.V[0], 0, h, t * TF_BN, b);
@@ -788,36 +797,41 @@ struct BwdKTcSmem {
 
 struct UnitInfo {
     int b, kvh, kt, nit;   // nit = iterations: heads x query blocks that see the key tile
+    int qb0;               // the first of those query blocks
 };
 // Unit u: key tile kt of (b, KV head).  Sliding windows (W <= 128) sweep the units of a chain
 // in order (u = chain * tiles + kt), and query blocks kt and kt + 1 see the tile; wide windows
 // run one unit per CTA, heaviest (first tiles) first (u = kt * chains + chain), and the
-// query blocks that see tile kt run from kt to the block of the last query whose window
-// reaches the tile's last key, kt*128 + 127 + W - 1.
+// query blocks that see tile kt run from kt (or the block of the first query row, q_off / 128,
+// if later) to the block of the last query whose window reaches the tile's last key,
+// kt*128 + 127 + W - 1.  With q_off > 0 the tiles before wide_first_tile(L) have no query at
+// all: they take no unit (the launcher zeroes their dk and dv).
 __device__ __forceinline__ UnitInfo decode_unit(const LayerParams& L, int u, bool wide) {
     const int nkb = (L.S + TF_BN - 1) / TF_BN;
     UnitInfo x;
     int chain;
     if (wide) {
         const int chains = L.B * L.Hkv;
-        x.kt = u / chains;
-        chain = u - x.kt * chains;
+        x.kt = wide_first_tile(L) + u / chains;
+        chain = u % chains;
         // W <= S here (the launcher clamps it), so the sum stays in range
         const int last_q = x.kt * TF_BN + TF_BN - 1 + L.W - 1;
         const int qb_hi = min(nkb - 1, last_q / TF_BM);
-        x.nit = L.G * (qb_hi - x.kt + 1);
+        x.qb0 = max(x.kt, L.q_off / TF_BM);
+        x.nit = L.G * (qb_hi - x.qb0 + 1);
     } else {
         chain = u / nkb;
         x.kt = u - chain * nkb;
+        x.qb0 = x.kt;
         x.nit = L.G * ((x.kt + 1 < nkb) ? 2 : 1);  // W <= 128: blocks kt and kt + 1
     }
     x.b = chain / L.Hkv;
     x.kvh = chain - x.b * L.Hkv;
     return x;
 }
-// iteration it of a unit: query block kt + it / G, head it % G
+// iteration it of a unit: query block qb0 + it / G, head it % G
 __device__ __forceinline__ void decode_iter(const LayerParams& L, const UnitInfo& x, int it, int& qb, int& hg) {
-    qb = x.kt + it / L.G;
+    qb = x.qb0 + it / L.G;
     hg = x.kvh * L.G + it % L.G;
 }
 
@@ -1117,9 +1131,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
             const float vtile = p.vtinv[((size_t)x.b * L.Hkv + x.kvh) * nkt + x.kt];
             float domx = 0.f, dlmx = 0.f;
             if constexpr (WIDE) {
-                // per-tile maxima over the query blocks kt .. kt + nit/G - 1 (bwd_tile_stats_kernel)
+                // per-tile maxima over the query blocks qb0 .. qb0 + nit/G - 1 (bwd_tile_stats_kernel)
                 const size_t nst = (size_t)L.B * L.Hkv * nkt, base = ((size_t)x.b * L.Hkv + x.kvh) * nkt;
-                for (int t = x.kt + r; t < x.kt + x.nit / L.G; t += TF_BN) {
+                for (int t = x.qb0 + r; t < x.qb0 + x.nit / L.G; t += TF_BN) {
                     domx = fmaxf(domx, p.tstat[base + t]);
                     dlmx = fmaxf(dlmx, p.tstat[nst + base + t]);
                 }
@@ -1421,7 +1435,7 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     p.err = err_word;
     const bool wide = bp.L.W > TF_BN;  // as the kernel-name query decides: on the window given
     p.wide = wide ? 1 : 0;
-    if (!make_map_b(&p.tm_q, L.q, L.Hq, L.S, L.B) || !make_map_b(&p.tm_k, L.k, L.Hkv, L.S, L.B) ||
+    if (!make_map_b(&p.tm_q, L.q, L.Hq, L.Sq, L.B) || !make_map_b(&p.tm_k, L.k, L.Hkv, L.S, L.B) ||
         !make_map_b(&p.tm_v, L.v, L.Hkv, L.S, L.B) ||
         !make_map_b(&p.tm_da, da16, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
         !make_map_b(&p.tm_k16, k16, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
@@ -1465,8 +1479,10 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     if (steps > 0x7fffffffLL) return cudaErrorInvalidValue;
     p.total = (int)steps;
     const int grid = (int)(steps < sms ? steps : sms);
-    // gate pass: 2 resident blocks of 256 threads per SM, each half-warp GATE_UNROLL rows at a time
-    const long long half_warps = ((long long)rows + GATE_UNROLL - 1) / GATE_UNROLL;
+    // gate pass over the query rows: 2 resident blocks of 256 threads per SM, each half-warp
+    // GATE_UNROLL rows at a time
+    const long long qrows = (long long)L.B * L.Sq * L.Hq;
+    const long long half_warps = (qrows + GATE_UNROLL - 1) / GATE_UNROLL;
     const long long gate_need = (half_warps * 16 + GATE_THREADS - 1) / GATE_THREADS;
     const int gate_grid = (int)(gate_need < 2LL * sms ? gate_need : 2LL * sms);
     const size_t smem_pk = sizeof(PrepSmem<true>) + 1024, smem_pq = sizeof(PrepSmem<false>) + 1024;
@@ -1477,16 +1493,17 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     if ((e = cudaFuncSetAttribute(bwd_prep_v_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_pk)) !=
         cudaSuccess)
         return e;
-    const long long k_tiles = (long long)L.B * L.Hkv * nkt, q_tiles = (long long)L.B * L.Hq * nkt;
+    const long long k_tiles = (long long)L.B * L.Hkv * nkt;
+    const long long q_tiles = (long long)L.B * L.Hq * ((L.Sq + TF_BN - 1) / TF_BN);  // of the query rows
     if (q_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
     int i = 0;
     if ((e = before(i)) != cudaSuccess) return e;
     if (wide)
         bwd_gate_kernel<true><<<gate_grid, GATE_THREADS, 0, stream>>>(bp.dout, L.g, bp.out, bp.dg, da16, p.dainv,
-                                                                      p.domax, p.P.delta, (long long)rows, L.S, L.Hq);
+                                                                      p.domax, p.P.delta, qrows, L.S, L.Hq, L.q_off);
     else
         bwd_gate_kernel<false><<<gate_grid, GATE_THREADS, 0, stream>>>(bp.dout, L.g, bp.out, bp.dg, da16, p.dainv,
-                                                                       p.domax, nullptr, (long long)rows, L.S, L.Hq);
+                                                                       p.domax, nullptr, qrows, L.S, L.Hq, 0);
     if ((e = after(i++)) != cudaSuccess) return e;
     if ((e = before(i)) != cudaSuccess) return e;
     if (sv)
@@ -1502,19 +1519,29 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     if (wide) {
         // per-tile bounds, then the query-major sweep (one CTA per (b, head, block), heaviest
         // first) and the key-major one (one CTA per (b, KV head, tile), heaviest first)
-        const long long units_q = (long long)L.B * L.Hq * nqb;
+        // query blocks from the one of the first query row on; key tiles from the first one
+        // a query row sees (wide_first_tile), the ones before it get zero dk and dv
+        const long long units_q = (long long)L.B * L.Hq * (nqb - L.q_off / TF_BM);
+        const int kt0 = wide_first_tile(L);
+        const long long units_k = (long long)L.B * L.Hkv * (nkt - kt0);
+        if (kt0 > 0) {
+            const size_t pitch = (size_t)L.S * L.Hkv * kD * sizeof(bf16);
+            const size_t width = (size_t)kt0 * TF_BN * L.Hkv * kD * sizeof(bf16);
+            if ((e = cudaMemset2DAsync(bp.dk, pitch, 0, width, L.B, stream)) != cudaSuccess) return e;
+            if ((e = cudaMemset2DAsync(bp.dv, pitch, 0, width, L.B, stream)) != cudaSuccess) return e;
+        }
         if ((e = before(i)) != cudaSuccess) return e;
         bwd_tile_stats_kernel<<<(int)k_tiles, BTS_THREADS, 0, stream>>>(p);
         if ((e = after(i++)) != cudaSuccess) return e;
         if ((e = before(i)) != cudaSuccess) return e;
         if ((e = launch_bwd_q_glob(p, (int)units_q, stream)) != cudaSuccess) return e;
         if ((e = after(i++)) != cudaSuccess) return e;
-        p.total = (int)k_tiles;
+        p.total = (int)units_k;
         if ((e = before(i)) != cudaSuccess) return e;
-        kv_wide<<<(int)k_tiles, TB_THREADS, smem_k, stream>>>(p);
+        kv_wide<<<(int)units_k, TB_THREADS, smem_k, stream>>>(p);
         if ((e = after(i++)) != cudaSuccess) return e;
         if ((e = before(i)) != cudaSuccess) return e;
-        dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgk_part, (int)k_tiles, bp.dgamma_k);
+        dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgk_part, (int)units_k, bp.dgamma_k);
         if ((e = after(i++)) != cudaSuccess) return e;
         if ((e = before(i)) != cudaSuccess) return e;
         dgamma_reduce_kernel<<<1, 1024, 0, stream>>>(p.P.dgq_part, (int)units_q, bp.dgamma_q);

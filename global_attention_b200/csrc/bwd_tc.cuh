@@ -48,6 +48,13 @@ struct BwdTcParams {
 // global stride must be a multiple of 16 bytes).  Entries past S hold neutral values.
 __host__ __device__ __forceinline__ int row_stride(int S) { return (S + 63) & ~63; }
 
+// First key tile a query row sees in a wide-window problem whose query rows start at q_off
+// (window W <= S): the tile of key q_off - W + 1; 0 when that is before the sequence.
+__host__ __device__ __forceinline__ int wide_first_tile(const LayerParams& L) {
+    const int j = L.q_off - L.W + 1;
+    return j > 0 ? j / TF_BN : 0;
+}
+
 // power-of-two exponent e with |x| * 2^e in [2^13, 2^14); 0 for x == 0 or non-finite
 __device__ __forceinline__ int fit_exp(float x) {
     if (!(x > 0.f) || !isfinite(x)) return 0;

@@ -22,15 +22,19 @@ typedef __nv_bfloat16 bf16;
 
 // Everything a kernel needs, passed by value (__grid_constant__).
 struct LayerParams {
-    const bf16* q;       // [B,S,Hq,D]
+    const bf16* q;       // [B,Sq,Hq,D]: the query rows, positions q_off .. S-1
     const bf16* k;       // [B,S,Hkv,D]
     const bf16* v;       // [B,S,Hkv,D]
-    const bf16* g;       // [B,S,Hq,D]
+    const bf16* g;       // [B,Sq,Hq,D]
     const float* gamma_q;
     const float* gamma_k;
     int B, S, Hq, Hkv, G;   // G = Hq / Hkv
     int rope_half;          // rope_dims / 2
     int W;                  // window (>= S means full causal)
+    int q_off;              // position of the first query row (0: every position has one;
+                            // else a multiple of 128, wide windows only).  q, g, out, lse,
+                            // dout, dq, dg hold rows q_off .. S-1; k, v, dk, dv all S rows.
+    int Sq;                 // S - q_off
     float eps;
     float scale;            // softmax scale
     float scale_log2;       // scale * log2(e)
@@ -39,8 +43,8 @@ struct LayerParams {
 
 struct FwdParams {
     LayerParams L;
-    bf16* out;    // [B,S,Hq,D]
-    float* lse;   // [B,Hq,S]
+    bf16* out;    // [B,Sq,Hq,D]
+    float* lse;   // [B,Hq,Sq]
 };
 
 // Activations the forward can leave for the backward (all null = none): the fp16 Q~
@@ -55,13 +59,13 @@ struct SavedAct {
 
 struct BwdParams {
     LayerParams L;
-    const bf16* out;    // [B,S,Hq,D]
-    const float* lse;   // [B,Hq,S]
-    const bf16* dout;   // [B,S,Hq,D]
-    bf16* dq;           // [B,S,Hq,D]
+    const bf16* out;    // [B,Sq,Hq,D]
+    const float* lse;   // [B,Hq,Sq]
+    const bf16* dout;   // [B,Sq,Hq,D]
+    bf16* dq;           // [B,Sq,Hq,D]
     bf16* dk;           // [B,S,Hkv,D]
     bf16* dv;           // [B,S,Hkv,D]
-    bf16* dg;           // [B,S,Hq,D]
+    bf16* dg;           // [B,Sq,Hq,D]
     float* dgamma_q;    // [D]
     float* dgamma_k;    // [D]
     // workspace views (set by the launcher)

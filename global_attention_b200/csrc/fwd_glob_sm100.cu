@@ -75,8 +75,9 @@ struct FgUnit {
     int b, kvh, h0, h1, qb, kt_lo, n_tiles;   // h0, h1: the unit's two query heads
 };
 
-// Unit u, heaviest first: the query block runs from the last one down; the head pairs of a KV
-// group are adjacent so that the CTAs reading the same K/V tiles run together.  With an odd
+// Unit u, heaviest first: the query block runs from the last one down (to the block of the
+// first query row, q_off / 128); the head pairs of a KV group are adjacent so that the CTAs
+// reading the same K/V tiles run together.  With an odd
 // number of heads per KV head the last pair repeats the last head (its two warpgroups compute,
 // and write, the same rows).
 __device__ __forceinline__ FgUnit fg_unit(const LayerParams& L, int u) {
@@ -221,8 +222,9 @@ __global__ void __launch_bounds__(FG_THREADS, 1) fwd_glob_tc_kernel(const __grid
         if (lane == 0) {
             for (int x = 0; x < 2; ++x) {
                 mbar_expect_tx(&sm.bar[FG_QFULL + x], TF_TILE_BYTES);
-                tma_load_4d(sm.Q[x][0], &p.tm_q, &sm.bar[FG_QFULL + x], 0, x ? w.h1 : w.h0, q0, w.b);
-                tma_load_4d(sm.Q[x][1], &p.tm_q, &sm.bar[FG_QFULL + x], 64, x ? w.h1 : w.h0, q0, w.b);
+                // (q holds the rows from position q_off on)
+                tma_load_4d(sm.Q[x][0], &p.tm_q, &sm.bar[FG_QFULL + x], 0, x ? w.h1 : w.h0, q0 - L.q_off, w.b);
+                tma_load_4d(sm.Q[x][1], &p.tm_q, &sm.bar[FG_QFULL + x], 64, x ? w.h1 : w.h0, q0 - L.q_off, w.b);
             }
             int nk = 0, nv = 0;  // K~ / V tiles issued
             for (int n = 0; n < w.n_tiles; ++n) {
@@ -407,7 +409,8 @@ __global__ void __launch_bounds__(FG_THREADS, 1) fwd_glob_tc_kernel(const __grid
         }
         // ------------------------------------------ epilogue: out = sigmoid(g) * O / l, lse
         const bool valid = i < L.S;
-        const size_t off = ((size_t)(w.b * (size_t)L.S + (valid ? i : 0)) * L.Hq + hx) * kD;
+        const int iq = valid ? i - L.q_off : 0;  // row of the query-side tensors
+        const size_t off = ((size_t)(w.b * (size_t)L.Sq + iq) * L.Hq + hx) * kD;
         uint4 gr[16];
         if (valid) {
 #pragma unroll
@@ -441,7 +444,7 @@ __global__ void __launch_bounds__(FG_THREADS, 1) fwd_glob_tc_kernel(const __grid
                     }
                 }
             }
-            if (valid) p.lse[((size_t)w.b * L.Hq + hx) * L.S + i] = (m_ref + __log2f(l)) * kLn2;
+            if (valid) p.lse[((size_t)w.b * L.Hq + hx) * L.Sq + iq] = (m_ref + __log2f(l)) * kLn2;
         }
     }
 
@@ -512,11 +515,12 @@ cudaError_t launch_fwd_glob_tc(const FwdParams& fp, void* workspace, int* err_wo
     p.lse = fp.lse;
     p.err = err_word;
     const long long nqb = (L.S + TF_BM - 1) / TF_BM;
-    const long long units = (long long)L.B * L.Hkv * ((L.G + 1) / 2) * nqb;
+    // query blocks from the one of the first query row (q_off, a multiple of 128) on
+    const long long units = (long long)L.B * L.Hkv * ((L.G + 1) / 2) * (nqb - L.q_off / TF_BM);
     const long long k_tiles = (long long)L.B * L.Hkv * nqb;
     if (units > 0x7fffffffLL || k_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
     p.units = (int)units;
-    if (!make_map_g(&p.tm_q, L.q, L.Hq, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) ||
+    if (!make_map_g(&p.tm_q, L.q, L.Hq, L.Sq, L.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) ||
         !make_map_g(&p.tm_k, L.k, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) ||
         !make_map_g(&p.tm_k16, workspace, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
         !make_map_g(&p.tm_v, L.v, L.Hkv, L.S, L.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))

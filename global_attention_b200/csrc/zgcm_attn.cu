@@ -99,6 +99,8 @@ void fill_layer(LayerParams& L, const void* q, const void* k, const void* v, con
     L.B = B; L.S = S; L.Hq = Hq; L.Hkv = Hkv; L.G = Hq / Hkv;
     L.rope_half = rope_dims / 2;
     L.W = window;
+    L.q_off = 0;
+    L.Sq = S;
     L.eps = eps;
     L.scale = scale;
     L.scale_log2 = scale * kLog2e;
@@ -129,6 +131,18 @@ size_t saved_layout(int B, int S, int Hq, int Hkv, char* base, SavedAct* sv) {
 
 // The store applies to every shape (both passes run tcgen05 kernels throughout).
 bool saved_supported(const LayerParams& L) { return L.S >= 1 && L.B >= 1; }
+
+// Query rows Sq at the end of S key rows (the first at position q_off = S - Sq): every Sq
+// with q_off = 0, else q_off a multiple of 128 and a window wider than 128 (the wide-window
+// kernels take the offset; a window of at most 128 reaches 127 rows back, so a caller pads
+// those few rows instead).
+int rows_check(int S, int Sq, int window) {
+    if (Sq < 0 || Sq > S) return ZGCM_ERR_INVALID_ARG;
+    const int q_off = S - Sq;
+    if (q_off == 0) return ZGCM_OK;
+    if (q_off % 128 != 0 || window <= 128) return ZGCM_ERR_UNSUPPORTED;
+    return ZGCM_OK;
+}
 
 }  // namespace
 
@@ -229,6 +243,35 @@ int zgcm_attn_fwd(const void* q, const void* k, const void* v, const void* g,
     return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
 }
 
+int zgcm_attn_fwd_rows(const void* q, const void* k, const void* v, const void* g,
+                       const float* gamma_q, const float* gamma_k,
+                       int B, int Sq, int S, int Hq, int Hkv, int D, int rope_dims,
+                       double rope_base, int window, int causal, float eps, float scale,
+                       void* out, float* lse, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+    int st = check_shape(B, S, Hq, Hkv, D, rope_dims, rope_base, window, causal, eps, scale);
+    if (st != ZGCM_OK) return st;
+    if ((st = rows_check(S, Sq, window)) != ZGCM_OK) return st;
+    if ((long long)B * Sq == 0) return ZGCM_OK;  // no query row: nothing to compute
+    if (Sq == S)
+        return zgcm_attn_fwd_ws(q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, D, rope_dims, rope_base, window,
+                                causal, eps, scale, out, lse, workspace, workspace_bytes, cuda_stream);
+    st = fwd_check(q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, D, rope_dims, rope_base, window, causal, eps, scale,
+                   out, lse);
+    if (st != ZGCM_OK) return st;
+    const size_t need = zgcm_attn_fwd_workspace_size(B, S, Hq, Hkv, D, rope_dims, window);
+    if (!workspace || workspace_bytes < need) return ZGCM_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ZGCM_ERR_ALIGNMENT;
+    FwdParams p;
+    fill_layer(p.L, q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, rope_dims, rope_base, window, eps, scale);
+    p.L.q_off = S - Sq;
+    p.L.Sq = Sq;
+    p.out = static_cast<bf16*>(out);
+    p.lse = lse;
+    const cudaError_t e =
+        launch_fwd_glob_tc(p, workspace, device_error_word(), static_cast<cudaStream_t>(cuda_stream), nullptr);
+    return e == cudaSuccess ? ZGCM_OK : ZGCM_ERR_CUDA;
+}
+
 size_t zgcm_attn_saved_size(int B, int S, int Hq, int Hkv, int D, int rope_dims, int window) {
     if (check_shape(B, S, Hq, Hkv, D, rope_dims, 1.0, window, 1, 0.f, 1.f) != ZGCM_OK) return 0;
     if ((long long)B * S == 0) return 0;
@@ -323,18 +366,29 @@ size_t zgcm_attn_bwd_workspace_size(int B, int S, int Hq, int Hkv, int D, int wi
 
 namespace {
 // The backward; with `saved` (non-null), from the activations zgcm_attn_fwd_save left there.
+// Sq: the query rows (the last Sq of the S positions; Sq = S for every other entry).
 int bwd_run(const void* q, const void* k, const void* v, const void* g, const float* gamma_q,
-            const float* gamma_k, const void* out, const float* lse, const void* dout, int B, int S, int Hq,
+            const float* gamma_k, const void* out, const float* lse, const void* dout, int B, int Sq, int S, int Hq,
             int Hkv, int D, int rope_dims, double rope_base, int window, int causal, float eps, float scale,
             void* dq, void* dk, void* dv, void* dg, float* dgamma_q, float* dgamma_k, void* workspace,
             size_t workspace_bytes, const void* saved, size_t saved_bytes, void* cuda_stream,
             void* const* events, int n_pairs) {
     int st = check_shape(B, S, Hq, Hkv, D, rope_dims, rope_base, window, causal, eps, scale);
     if (st != ZGCM_OK) return st;
+    if ((st = rows_check(S, Sq, window)) != ZGCM_OK) return st;
+    if (saved && Sq != S) return ZGCM_ERR_UNSUPPORTED;
     if (!dgamma_q || !dgamma_k) return ZGCM_ERR_INVALID_ARG;
     if (!aligned16(dgamma_q) || !aligned16(dgamma_k)) return ZGCM_ERR_ALIGNMENT;
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-    if ((long long)B * S == 0) {
+    if ((long long)B * Sq == 0) {
+        // no query row: zero key gradients (when there are key rows) and d_gamma
+        if ((long long)B * S > 0) {
+            if (!dk || !dv) return ZGCM_ERR_INVALID_ARG;
+            if (!aligned16(dk) || !aligned16(dv)) return ZGCM_ERR_ALIGNMENT;
+            const size_t kv_bytes = (size_t)B * S * Hkv * kD * sizeof(bf16);
+            if (cudaMemsetAsync(dk, 0, kv_bytes, stream) != cudaSuccess) return ZGCM_ERR_CUDA;
+            if (cudaMemsetAsync(dv, 0, kv_bytes, stream) != cudaSuccess) return ZGCM_ERR_CUDA;
+        }
         if (cudaMemsetAsync(dgamma_q, 0, kD * sizeof(float), stream) != cudaSuccess) return ZGCM_ERR_CUDA;
         if (cudaMemsetAsync(dgamma_k, 0, kD * sizeof(float), stream) != cudaSuccess) return ZGCM_ERR_CUDA;
         return ZGCM_OK;
@@ -350,6 +404,8 @@ int bwd_run(const void* q, const void* k, const void* v, const void* g, const fl
 
     BwdParams p;
     fill_layer(p.L, q, k, v, g, gamma_q, gamma_k, B, S, Hq, Hkv, rope_dims, rope_base, window, eps, scale);
+    p.L.q_off = S - Sq;
+    p.L.Sq = Sq;
     p.out = static_cast<const bf16*>(out);
     p.lse = lse;
     p.dout = static_cast<const bf16*>(dout);
@@ -384,9 +440,22 @@ int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void*
                         float* dgamma_q, float* dgamma_k,
                         void* workspace, size_t workspace_bytes, void* cuda_stream,
                         void* const* events, int n_pairs) {
-    return bwd_run(q, k, v, g, gamma_q, gamma_k, out, lse, dout, B, S, Hq, Hkv, D, rope_dims, rope_base, window,
-                   causal, eps, scale, dq, dk, dv, dg, dgamma_q, dgamma_k, workspace, workspace_bytes, nullptr, 0,
-                   cuda_stream, events, n_pairs);
+    return bwd_run(q, k, v, g, gamma_q, gamma_k, out, lse, dout, B, S, S, Hq, Hkv, D, rope_dims, rope_base,
+                   window, causal, eps, scale, dq, dk, dv, dg, dgamma_q, dgamma_k, workspace, workspace_bytes, nullptr,
+                   0, cuda_stream, events, n_pairs);
+}
+
+int zgcm_attn_bwd_rows(const void* q, const void* k, const void* v, const void* g,
+                       const float* gamma_q, const float* gamma_k,
+                       const void* out, const float* lse, const void* dout,
+                       int B, int Sq, int S, int Hq, int Hkv, int D, int rope_dims,
+                       double rope_base, int window, int causal, float eps, float scale,
+                       void* dq, void* dk, void* dv, void* dg,
+                       float* dgamma_q, float* dgamma_k,
+                       void* workspace, size_t workspace_bytes, void* cuda_stream) {
+    return bwd_run(q, k, v, g, gamma_q, gamma_k, out, lse, dout, B, Sq, S, Hq, Hkv, D, rope_dims, rope_base,
+                   window, causal, eps, scale, dq, dk, dv, dg, dgamma_q, dgamma_k, workspace, workspace_bytes, nullptr,
+                   0, cuda_stream, nullptr, 0);
 }
 
 int zgcm_attn_bwd_saved(const void* q, const void* k, const void* v, const void* g,
@@ -399,8 +468,8 @@ int zgcm_attn_bwd_saved(const void* q, const void* k, const void* v, const void*
                         void* workspace, size_t workspace_bytes, const void* saved, size_t saved_bytes,
                         void* cuda_stream, void* const* events, int n_pairs) {
     if (!saved) return ZGCM_ERR_INVALID_ARG;
-    return bwd_run(q, k, v, g, gamma_q, gamma_k, out, lse, dout, B, S, Hq, Hkv, D, rope_dims, rope_base, window,
-                   causal, eps, scale, dq, dk, dv, dg, dgamma_q, dgamma_k, workspace, workspace_bytes, saved,
+    return bwd_run(q, k, v, g, gamma_q, gamma_k, out, lse, dout, B, S, S, Hq, Hkv, D, rope_dims, rope_base,
+                   window, causal, eps, scale, dq, dk, dv, dg, dgamma_q, dgamma_k, workspace, workspace_bytes, saved,
                    saved_bytes, cuda_stream, events, n_pairs);
 }
 

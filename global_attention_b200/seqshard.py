@@ -23,12 +23,16 @@ d_gamma (2 x D values).
 A window longer than a rank's rows (the global layer, W >= S, among them) reaches further
 back: gathered_forward / gathered_backward gather every rank's key and value rows, run the
 layer on the rows the window reaches ([start, (r + 1) L), start = max(0, r L - (W - 1)),
-numbered from 0) with zero query rows before this rank's, and return the earlier rows' key
-gradients to their owners through one sum over the ranks.  The zero query rows are computed
-and dropped: a kernel that takes a first query row would skip that work.
+numbered from 0) for this rank's query rows, and return the earlier rows' key gradients to
+their owners through one sum over the ranks.  With a window wider than 128 and r L a
+multiple of 128, start is rounded down to a multiple of 128 and the query-row entry points
+(zgcm_attn_fwd_rows / zgcm_attn_bwd_rows) take this rank's rows as the last ones of the
+gathered sequence, so no query row before them is computed; otherwise zero query rows stand
+before this rank's and their results are dropped.
 
-The compute is a pair of callables with the signatures of zgcm_attn_fwd / zgcm_attn_bwd of
-this package (the default); the tests pass others to check the sharding on the CPU.
+The compute is a tuple of callables with the signatures of zgcm_attn_fwd, zgcm_attn_bwd and
+(optionally) zgcm_attn_fwd_rows, zgcm_attn_bwd_rows of this package (the default); the tests
+pass others to check the sharding on the CPU.
 """
 from __future__ import annotations
 
@@ -38,7 +42,13 @@ import torch.distributed as dist
 
 def _default_ops():
     import global_attention_b200 as ga
-    return ga.zgcm_attn_fwd, ga.zgcm_attn_bwd
+    return ga.zgcm_attn_fwd, ga.zgcm_attn_bwd, ga.zgcm_attn_fwd_rows, ga.zgcm_attn_bwd_rows
+
+
+def _ops4(ops):
+    """(fwd, bwd, fwd_rows or None, bwd_rows or None)."""
+    ops = tuple(ops or _default_ops())
+    return ops + (None,) * (4 - len(ops))
 
 
 def _exchange(send, recv_shape, like, to_rank, from_rank, group):
@@ -68,7 +78,7 @@ def halo_forward(q, k, v, g, gamma_q, gamma_k, *, window, group=None, ops=None, 
     """Forward of this rank's rows.  q, g [B, L, Hq, D]; k, v [B, L, Hkv, D] are the rows of
     positions r L .. r L + L - 1; every rank has the same L >= window - 1.  Returns out
     [B, L, Hq, D], lse [B, Hq, L] of those rows and a HaloContext for halo_backward."""
-    fwd, _ = ops or _default_ops()
+    fwd = _ops4(ops)[0]
     rank, world = dist.get_rank(group), dist.get_world_size(group)
     B, L = q.shape[0], q.shape[1]
     h = window - 1
@@ -93,7 +103,7 @@ def halo_forward(q, k, v, g, gamma_q, gamma_k, *, window, group=None, ops=None, 
 def halo_backward(ctx, dout, gamma_q, gamma_k, *, group=None, ops=None):
     """Backward of halo_forward on this rank: dict of dq, dk, dv, dg for its rows and
     dgamma_q, dgamma_k of the whole sequence (summed over the ranks)."""
-    _, bwd = ops or _default_ops()
+    bwd = _ops4(ops)[1]
     rank, world = dist.get_rank(group), dist.get_world_size(group)
     h = ctx.h
     q, k, v, g = ctx.ext
@@ -125,10 +135,14 @@ def gathered_forward(q, k, v, g, gamma_q, gamma_k, *, window, group=None, ops=No
     """Forward of this rank's rows for any window: the key and value rows of the earlier
     ranks that the window reaches are gathered (all ranks' rows travel; each keeps what it
     needs).  Shapes as halo_forward; every rank has the same L."""
-    fwd, _ = ops or _default_ops()
+    fwd, _, fwd_rows, _ = _ops4(ops)
     rank, world = dist.get_rank(group), dist.get_world_size(group)
     B, L = q.shape[0], q.shape[1]
     start = max(0, rank * L - (window - 1))
+    # the query-row kernels take a first query row on a 128-row boundary, windows wider than 128
+    rows = fwd_rows is not None and window > 128 and (rank * L) % 128 == 0
+    if rows:
+        start -= start % 128
     h = rank * L - start
     if world == 1 or h == 0:
         out, lse = fwd(q, k, v, g, gamma_q, gamma_k, window=window, **kw)
@@ -140,6 +154,11 @@ def gathered_forward(q, k, v, g, gamma_q, gamma_k, *, window, group=None, ops=No
     kv_all = [torch.empty_like(torch.stack([k, v])) for _ in range(world)]
     dist.all_gather(kv_all, torch.stack([k, v]).contiguous(), group=group)
     before = torch.cat(kv_all[:rank], 2)[:, :, start:]  # [2, B, h, Hkv, D]
+    if rows:
+        ext_k = torch.cat([before[0], k], 1).contiguous()
+        ext_v = torch.cat([before[1], v], 1).contiguous()
+        out, lse = fwd_rows(q, ext_k, ext_v, g, gamma_q, gamma_k, window=window, **kw)
+        return out, lse, HaloContext(h, (q, ext_k, ext_v, g), out, lse, window, dict(kw, _start=start, _rows=True))
     zq = torch.zeros((B, h) + tuple(q.shape[2:]), dtype=q.dtype, device=q.device)
     ext = (torch.cat([zq, q], 1).contiguous(), torch.cat([before[0], k], 1).contiguous(),
            torch.cat([before[1], v], 1).contiguous(), torch.cat([zq, g], 1).contiguous())
@@ -152,17 +171,22 @@ def gathered_backward(ctx, dout, gamma_q, gamma_k, *, group=None, ops=None):
     """Backward of gathered_forward: this rank's dq, dk, dv, dg and the whole sequence's
     dgamma_q, dgamma_k.  The key and value gradients of all rows are summed over the ranks
     (each rank contributes the rows its window reached) and each keeps its own."""
-    _, bwd = ops or _default_ops()
+    _, bwd, _, bwd_rows = _ops4(ops)
     rank, world = dist.get_rank(group), dist.get_world_size(group)
     kw = dict(ctx.kw)
     start = kw.pop("_start")
+    rows = kw.pop("_rows", False)
     h = ctx.h
     q, k, v, g = ctx.ext
-    if h > 0:
-        zd = torch.zeros((dout.shape[0], h) + tuple(dout.shape[2:]), dtype=dout.dtype, device=dout.device)
-        dout = torch.cat([zd, dout], 1).contiguous()
-    gr = bwd(q, k, v, g, gamma_q, gamma_k, ctx.out_ext, ctx.lse_ext, dout, window=ctx.window, **kw)
-    res = {n: gr[n][:, h:].contiguous() for n in ("dq", "dg")}
+    if rows:  # this rank's query rows only, the gathered key rows before them
+        gr = bwd_rows(q, k, v, g, gamma_q, gamma_k, ctx.out_ext, ctx.lse_ext, dout, window=ctx.window, **kw)
+        res = {n: gr[n].contiguous() for n in ("dq", "dg")}
+    else:
+        if h > 0:
+            zd = torch.zeros((dout.shape[0], h) + tuple(dout.shape[2:]), dtype=dout.dtype, device=dout.device)
+            dout = torch.cat([zd, dout], 1).contiguous()
+        gr = bwd(q, k, v, g, gamma_q, gamma_k, ctx.out_ext, ctx.lse_ext, dout, window=ctx.window, **kw)
+        res = {n: gr[n][:, h:].contiguous() for n in ("dq", "dg")}
     L = res["dq"].shape[1]
     dk_ext, dv_ext = gr["dk"], gr["dv"]
     if world > 1:

@@ -207,6 +207,41 @@ int zgcm_attn_bwd_timed(const void* q, const void* k, const void* v, const void*
                         void* const* events, int n_pairs);
 
 /*
+ * Query rows at the end of a longer key sequence: a shard of one sequence whose earlier key
+ * and value rows (those its window reaches) were gathered from the ranks that own them.  The
+ * layer on positions 0 .. S-1 (k, v: [B,S,Hkv,D], every position) restricted to the query
+ * rows of positions q_off .. S-1, q_off = S - Sq: q, g, out, dout, dq, dg are [B,Sq,Hq,D],
+ * lse [B,Hq,Sq]; row i of them is position q_off + i (its RoPE angle, its window).  The
+ * rows before q_off cost nothing: no query block before them is computed.  (The shard
+ * layout of the sequence-sharded long-context stage: shibing624 review, section
+ * "数据与课程", the 256K stage; the global layers of the ZGCM-1 summary, section
+ * "前置知识 / 滑动窗口注意力(SWA)与混合注意力", see every earlier key.)
+ *
+ * Arguments as zgcm_attn_fwd_ws / zgcm_attn_bwd, with Sq and S in place of S; outputs are the
+ * rows zgcm_attn_fwd / zgcm_attn_bwd of the whole sequence would give for those positions,
+ * and dk, dv (every key row), dgamma_q, dgamma_k the parts the given query rows contribute.
+ * Workspace: zgcm_attn_fwd_workspace_size / zgcm_attn_bwd_workspace_size of (B, S, ...).
+ * Requires 0 <= Sq <= S (else ZGCM_ERR_INVALID_ARG) and, when Sq < S, q_off a multiple of
+ * 128 and window > 128 (else ZGCM_ERR_UNSUPPORTED: a window of at most 128 reaches 127 rows
+ * back, which a caller covers by padding its query rows with zeros).  Sq == S is
+ * zgcm_attn_fwd_ws / zgcm_attn_bwd.  Sq == 0: nothing to compute (the backward zeroes dk,
+ * dv and dgamma_*).
+ */
+int zgcm_attn_fwd_rows(const void* q, const void* k, const void* v, const void* g,
+                       const float* gamma_q, const float* gamma_k,
+                       int B, int Sq, int S, int Hq, int Hkv, int D, int rope_dims,
+                       double rope_base, int window, int causal, float eps, float scale,
+                       void* out, float* lse, void* workspace, size_t workspace_bytes, void* cuda_stream);
+int zgcm_attn_bwd_rows(const void* q, const void* k, const void* v, const void* g,
+                       const float* gamma_q, const float* gamma_k,
+                       const void* out, const float* lse, const void* dout,
+                       int B, int Sq, int S, int Hq, int Hkv, int D, int rope_dims,
+                       double rope_base, int window, int causal, float eps, float scale,
+                       void* dq, void* dk, void* dv, void* dg,
+                       float* dgamma_q, float* dgamma_k,
+                       void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
  * zgcm_attn_bwd for callers that cannot allocate device memory.  (No counterpart in the
  * paper: this is an interface convenience of this library.)  A process that has reserved
  * the GPU's memory for its own pool, or a plugin given no allocator, cannot provide the

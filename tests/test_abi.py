@@ -281,3 +281,38 @@ def test_noalloc_binding_checks_before_any_launch(monkeypatch):
     with pytest.raises(TypeError, match="CUDA"):
         ga.zgcm_attn_bwd_noalloc(**args)
     assert not reached
+
+
+def _fwd_rows(lib, ws, ws_bytes, Sq, S, window, **kw):
+    a = dict(ARGS, **kw)
+    vp = ctypes.c_void_p
+    p = [vp(P + 256 * i) for i in range(8)]
+    return lib.zgcm_attn_fwd_rows(*p[:6], a["B"], Sq, S, a["Hq"], a["Hkv"], a["D"], a["rope_dims"],
+                                  a["rope_base"], window, a["causal"], a["eps"], a["scale"], p[6], p[7],
+                                  vp(ws), ws_bytes, None)
+
+
+def _bwd_rows(lib, ws, ws_bytes, Sq, S, window, **kw):
+    a = dict(ARGS, **kw)
+    vp = ctypes.c_void_p
+    p = [vp(P + 256 * i) for i in range(15)]
+    return lib.zgcm_attn_bwd_rows(*p[:9], a["B"], Sq, S, a["Hq"], a["Hkv"], a["D"], a["rope_dims"],
+                                  a["rope_base"], window, a["causal"], a["eps"], a["scale"], *p[9:15],
+                                  vp(ws), ws_bytes, None)
+
+
+def test_query_rows_checks(lib):
+    """Query rows at the end of the key rows: Sq <= S, and a first query row off position 0
+    only on a 128-row boundary with a window wider than 128; the workspace is the one of the
+    whole key sequence.  Every call here fails validation before any launch."""
+    need = lib.zgcm_attn_fwd_workspace_size(1, 640, 32, 8, 128, 42, 640)
+    ws = P + 256 * 40
+    for fn, n in ((_fwd_rows, need), (_bwd_rows, lib.zgcm_attn_bwd_workspace_size(1, 640, 32, 8, 128, 640))):
+        assert fn(lib, ws, n, Sq=641, S=640, window=640) == -1     # more query rows than keys
+        assert fn(lib, ws, n, Sq=-1, S=640, window=640) == -1
+        assert fn(lib, ws, n, Sq=600, S=640, window=640) == -2     # first query row off a 128 boundary
+        assert fn(lib, ws, n, Sq=512, S=640, window=128) == -2     # a window of at most 128
+        assert fn(lib, ws, n, Sq=512, S=640, window=640, D=96) == -2
+        assert fn(lib, 0, n, Sq=512, S=640, window=640) == -4      # workspace missing
+        assert fn(lib, ws, n - 1, Sq=512, S=640, window=640) == -4
+        assert fn(lib, ws + 16, n, Sq=512, S=640, window=640) == -3

@@ -21,21 +21,48 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-def _oracle_ops():
+def _oracle_ops(calls=None):
+    """The layer's entry points restated with the fp64 oracle: fwd, bwd and the query-row pair
+    (query rows at the end of the key rows: zero query rows in front, results sliced), each
+    call counted in `calls` by name."""
     import oracle
 
+    def count(name):
+        if calls is not None:
+            calls[name] = calls.get(name, 0) + 1
+
     def fwd(q, k, v, g, gq, gk, *, window, **kw):
+        count("fwd")
         out, lse = oracle.Problem(q, k, v, g, gq, gk, window=window, **kw).forward()
         return torch.from_numpy(out), torch.from_numpy(lse)
 
     def bwd(q, k, v, g, gq, gk, out, lse, dout, *, window, **kw):
+        count("bwd")
         r = oracle.Problem(q, k, v, g, gq, gk, window=window, **kw).backward(dout)
         return {n: torch.from_numpy(x) for n, x in r.items()}
 
-    return fwd, bwd
+    def pad(x, h):
+        return torch.cat([torch.zeros((x.shape[0], h) + tuple(x.shape[2:]), dtype=x.dtype), x], 1)
+
+    def fwd_rows(q, k, v, g, gq, gk, *, window, **kw):
+        count("fwd_rows")
+        h = k.shape[1] - q.shape[1]
+        out, lse = oracle.Problem(pad(q, h), k, v, pad(g, h), gq, gk, window=window, **kw).forward()
+        return torch.from_numpy(out[:, h:]), torch.from_numpy(lse[:, :, h:])
+
+    def bwd_rows(q, k, v, g, gq, gk, out, lse, dout, *, window, **kw):
+        count("bwd_rows")
+        h = k.shape[1] - q.shape[1]
+        r = oracle.Problem(pad(q, h), k, v, pad(g, h), gq, gk, window=window, **kw).backward(pad(dout, h))
+        r = {n: torch.from_numpy(x) for n, x in r.items()}
+        for n in ("dq", "dg"):
+            r[n] = r[n][:, h:]
+        return r
+
+    return fwd, bwd, fwd_rows, bwd_rows
 
 
-def _rank_main(rank, world, port, L, W, results, mode="halo"):
+def _rank_main(rank, world, port, L, W, results, mode="halo", calls_out=None):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     from datetime import timedelta
@@ -50,7 +77,8 @@ def _rank_main(rank, world, port, L, W, results, mode="halo"):
         t = make_inputs(B, world * L, Hq=Hq, Hkv=Hkv, D=D, seed=21, with_dout=True)
         rows = slice(rank * L, (rank + 1) * L)
         mine = {n: t[n][:, rows].contiguous() for n in ("q", "k", "v", "g", "dout")}
-        ops = _oracle_ops()
+        calls = {}
+        ops = _oracle_ops(calls)
         fwd = seqshard.halo_forward if mode == "halo" else seqshard.gathered_forward
         bwd = seqshard.halo_backward if mode == "halo" else seqshard.gathered_backward
         out, lse, ctx = fwd(mine["q"], mine["k"], mine["v"], mine["g"], t["gamma_q"], t["gamma_k"], window=W,
@@ -69,6 +97,8 @@ def _rank_main(rank, world, port, L, W, results, mode="halo"):
         for n in ("dgamma_q", "dgamma_k"):
             err[n] = np.abs(gr[n].numpy() - ref[n]).max() / max(1.0, np.abs(ref[n]).max())
         results[rank] = {k: float(v) for k, v in err.items()}
+        if calls_out is not None:
+            calls_out[rank] = dict(calls)
     finally:
         dist.destroy_process_group()
 
@@ -101,6 +131,26 @@ def test_gathered_sharding_equals_whole_sequence(world, L, W):
     for rank in range(world):
         for name, e in results[rank].items():
             assert e < 1e-9, (rank, name, e)
+
+
+@pytest.mark.parametrize("world,L,W", [(2, 128, 10**6), (3, 128, 200)])
+def test_gathered_sharding_query_rows(world, L, W):
+    """With a window wider than 128 and rank boundaries on 128 rows the gathered shards go
+    through the query-row entry points (this rank's rows as the last ones of the gathered key
+    rows, whose start is rounded down to a 128-row boundary; no zero query rows): every rank
+    after the first calls them, and every output and gradient still equals the unsharded
+    oracle (global layer; W = 200, where rank 2's start 57 becomes 0 and rank 1's 0 stays)."""
+    mgr = mp.get_context("spawn").Manager()
+    results, calls = mgr.dict(), mgr.dict()
+    mp.spawn(_rank_main, args=(world, _free_port(), L, W, results, "gathered", calls), nprocs=world, join=True)
+    assert len(results) == world
+    for rank in range(world):
+        for name, e in results[rank].items():
+            assert e < 1e-9, (rank, name, e)
+        if rank > 0:
+            assert calls[rank] == {"fwd_rows": 1, "bwd_rows": 1}, calls[rank]
+        else:
+            assert calls[rank] == {"fwd": 1, "bwd": 1}, calls[rank]
 
 
 def test_halo_needs_window_rows_per_rank():
