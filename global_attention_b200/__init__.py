@@ -83,6 +83,14 @@ def load() -> ctypes.CDLL:
         lib.zgcm_attn_fwd_rows.restype = i
         lib.zgcm_attn_bwd_rows.argtypes = [vp] * 9 + [i] * 7 + [d, i, i, f, f] + [vp] * 7 + [ctypes.c_size_t, vp]
         lib.zgcm_attn_bwd_rows.restype = i
+        lib.zgcm_muon_workspace_size.argtypes = [i, i]
+        lib.zgcm_muon_workspace_size.restype = ctypes.c_size_t
+        lib.zgcm_muon_step.argtypes = [vp, vp, vp, i, i, f, f, f, i, f, f, f, f, vp, ctypes.c_size_t, vp]
+        lib.zgcm_muon_step.restype = i
+        lib.zgcm_muon_orthogonalize.argtypes = [vp, vp, i, i, i, f, f, f, f, vp, ctypes.c_size_t, vp]
+        lib.zgcm_muon_orthogonalize.restype = i
+        lib.zgcm_muon_gemm.argtypes = [vp, vp, vp, vp, i, i, i, f, f, i, vp]
+        lib.zgcm_muon_gemm.restype = i
         _lib = lib
     return _lib
 
@@ -403,3 +411,84 @@ def zgcm_attn_bwd_noalloc(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_
     if st != ZGCM_OK:
         raise ZgcmError(st, "zgcm_attn_bwd_noalloc")
     return grads
+
+
+# ---------------------------------------------------------------- Muon optimiser (zgcm_muon.h)
+
+# momentum, iterations, learning rate and weight decay of the ZGCM-1 summary, section
+# "前置知识 / Muon 优化器"; the classical Newton–Schulz coefficients (the pages give none)
+MUON_MOMENTUM, MUON_STEPS, MUON_LR, MUON_WEIGHT_DECAY = 0.9, 5, 2e-4, 0.1
+MUON_COEFFS = (1.5, -0.5, 0.0)
+
+
+def zgcm_muon_workspace_size(m, n) -> int:
+    """Bytes of workspace zgcm_muon_step / zgcm_muon_orthogonalize need for an m x n matrix."""
+    return int(load().zgcm_muon_workspace_size(int(m), int(n)))
+
+
+def _muon_ws(m, n, workspace, device):
+    import torch
+    need = zgcm_muon_workspace_size(m, n)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+    _check(workspace, "workspace", torch.uint8, 1)
+    return workspace
+
+
+def zgcm_muon_step(W, G, M, *, lr=MUON_LR, weight_decay=MUON_WEIGHT_DECAY, momentum=MUON_MOMENTUM,
+                   steps=MUON_STEPS, coeffs=MUON_COEFFS, eps=1e-7, workspace=None, stream=None):
+    """One Muon step in place: W fp32 [m, n], G bf16 [m, n], M fp32 [m, n] (momentum buffer)."""
+    import torch
+    _check(W, "W", torch.float32, 2)
+    _check(G, "G", torch.bfloat16, 2)
+    _check(M, "M", torch.float32, 2)
+    if G.shape != W.shape or M.shape != W.shape:
+        raise TypeError("W, G and M must have one shape")
+    m, n = W.shape
+    ws = _muon_ws(m, n, workspace, W.device)
+    a, b, c = (float(x) for x in coeffs)
+    st = load().zgcm_muon_step(_ptr(W), _ptr(G), _ptr(M), m, n, float(lr), float(weight_decay), float(momentum),
+                               int(steps), a, b, c, float(eps), _ptr(ws), ws.numel(), _stream(stream))
+    if st != ZGCM_OK:
+        raise ZgcmError(st, "zgcm_muon_step")
+    return W, M
+
+
+def zgcm_muon_orthogonalize(G, *, steps=MUON_STEPS, coeffs=MUON_COEFFS, eps=1e-7, out=None, workspace=None,
+                            stream=None):
+    """bf16 [m, n]: the Newton–Schulz iterate after `steps` steps from G / (||G||_F + eps)."""
+    import torch
+    _check(G, "G", torch.bfloat16, 2)
+    m, n = G.shape
+    if out is None:
+        out = torch.empty_like(G)
+    ws = _muon_ws(m, n, workspace, G.device)
+    a, b, c = (float(x) for x in coeffs)
+    st = load().zgcm_muon_orthogonalize(_ptr(G), _ptr(out), m, n, int(steps), a, b, c, float(eps), _ptr(ws),
+                                        ws.numel(), _stream(stream))
+    if st != ZGCM_OK:
+        raise ZgcmError(st, "zgcm_muon_orthogonalize")
+    return out
+
+
+def zgcm_muon_gemm(A, B, *, D=None, alpha=1.0, beta=0.0, b_kn=False, out=None, stream=None):
+    """C = alpha A op(B) + beta D in bf16 (fp32 accumulation): A [M, K]; B [K, N] if b_kn else
+    [N, K] (C = A B^T)."""
+    import torch
+    _check(A, "A", torch.bfloat16, 2)
+    _check(B, "B", torch.bfloat16, 2)
+    M, K = A.shape
+    N = B.shape[1] if b_kn else B.shape[0]
+    if (B.shape[0] if b_kn else B.shape[1]) != K:
+        raise TypeError("inner dimensions of A and B differ")
+    if D is not None:
+        _check(D, "D", torch.bfloat16, 2)
+        if D.shape != (M, N):
+            raise TypeError("D must be [M, N]")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    st = load().zgcm_muon_gemm(_ptr(A), _ptr(B), _ptr(D), _ptr(out), M, N, K, float(alpha), float(beta),
+                               1 if b_kn else 0, _stream(stream))
+    if st != ZGCM_OK:
+        raise ZgcmError(st, "zgcm_muon_gemm")
+    return out

@@ -52,6 +52,15 @@ int* device_error_word() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+}  // namespace
+
+namespace zgcm {
+// the error word for the library's other kernels (the Muon step)
+int* library_error_word() { return device_error_word(); }
+}  // namespace zgcm
+
+namespace {
+
 // Forward kernel for a layer: the strip kernel (W <= 128, 4 query heads per KV head), the
 // sliding-window tcgen05 kernel (W <= 128, other group sizes) or the wide-window / global
 // tcgen05 pair (W > 128).  Every shape the arguments allow has one of them.

@@ -316,3 +316,37 @@ def test_query_rows_checks(lib):
         assert fn(lib, 0, n, Sq=512, S=640, window=640) == -4      # workspace missing
         assert fn(lib, ws, n - 1, Sq=512, S=640, window=640) == -4
         assert fn(lib, ws + 16, n, Sq=512, S=640, window=640) == -3
+
+
+def test_muon_checks(lib):
+    """Muon calls reject bad dimensions, pointers, alignment and workspace before any launch."""
+    vp = ctypes.c_void_p
+    lib.zgcm_muon_workspace_size.restype = ctypes.c_size_t
+    ws = lib.zgcm_muon_workspace_size
+    assert ws(4096, 11008) == ws(11008, 4096) > 0
+    for m, n in ((7, 16), (16, 12), (0, 8), (8, -8)):
+        assert ws(m, n) == 0
+    need = ws(64, 128)
+    f = ctypes.c_float
+    step = lambda W, G, M, m, n, steps, wsp, wsb: lib.zgcm_muon_step(
+        vp(W), vp(G), vp(M), m, n, f(2e-4), f(0.1), f(0.9), steps, f(1.5), f(-0.5), f(0.0), f(1e-7), vp(wsp), wsb,
+        None)
+    orth = lambda G, O, m, n, steps, wsp, wsb: lib.zgcm_muon_orthogonalize(
+        vp(G), vp(O), m, n, steps, f(1.5), f(-0.5), f(0.0), f(1e-7), vp(wsp), wsb, None)
+    W, G, M, O, S = P, P + 2 ** 20, P + 2 ** 21, P + 2 ** 22, P + 2 ** 23
+    assert step(W, G, M, 64, 12, 5, S, need) == -1          # n not a multiple of 8
+    assert step(W, G, M, 64, 128, 101, S, need) == -1       # too many steps
+    assert step(0, G, M, 64, 128, 5, S, need) == -1
+    assert step(W + 4, G, M, 64, 128, 5, S, need) == -3
+    assert step(W, G, M, 64, 128, 5, S, need - 1) == -4
+    assert step(W, G, M, 64, 128, 5, S + 16, need) == -3
+    assert orth(G, O, 64, 124, 5, S, need) == -1
+    assert orth(G, 0, 64, 128, 5, S, need) == -1
+    assert orth(G, O, 64, 128, 5, 0, need) == -4
+    gemm = lambda A, B, D, C, M_, N_, K_, kn: lib.zgcm_muon_gemm(vp(A), vp(B), vp(D), vp(C), M_, N_, K_, f(1.0),
+                                                                 f(0.0), kn, None)
+    assert gemm(G, G, 0, O, 64, 12, 64, 0) == -1            # N not a multiple of 8
+    assert gemm(G, G, 0, O, 64, 64, 60, 0) == -1            # K neither
+    assert gemm(G, G, 0, O, 64, 64, 64, 2) == -1            # layout flag
+    assert gemm(G, G, 0, 0, 64, 64, 64, 0) == -1
+    assert gemm(G + 8, G, 0, O, 64, 64, 64, 0) == -3
