@@ -479,6 +479,143 @@ def run_decode(args):
     return 0
 
 
+# the Muon optimiser step on one matrix parameter: the SwiGLU projection of the model, hidden
+# 4096 x intermediate 11008 (ZGCM-1 summary, section "核心方法")
+MUON_WORKLOADS = {"muon4096x11008": (4096, 11008)}
+MUON_METRIC = "muon_step_newton_schulz_tflops"
+
+
+def muon_cpu_baseline(m, n):
+    """The fp64 oracle's Muon step on a bounded sample: the matrix at one sixteenth of each
+    dimension, in TFLOP/s of its Newton–Schulz products."""
+    import numpy as np
+    from oracle import muon
+    ms, ns = m // 16, n // 16
+    rng = np.random.default_rng(0)
+    W, G, M = (rng.standard_normal((ms, ns)) for _ in range(3))
+    t0 = time.perf_counter()
+    reps = 0
+    while time.perf_counter() - t0 < 2.0 or reps < 1:
+        muon.muon_step(W, G, M)
+        reps += 1
+    secs = (time.perf_counter() - t0) / reps
+    return {"value": muon.ns_flops(ms, ns) / secs / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
+            "kind": "oracle", "sample": f"{reps} steps on a {ms} x {ns} matrix (numpy fp64, its BLAS threads), "
+                                        f"{secs * 1e3:.1f} ms each"}
+
+
+def run_muon(args):
+    """K Muon steps of one matrix parameter (momentum, scaling, five Newton–Schulz iterations,
+    update), the inputs resident; the products' kernel timed on its own as well."""
+    import torch
+    import global_attention_b200 as ga
+    from oracle import muon
+    world, rank, local = rank_env()
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ga.load()
+    m, n = MUON_WORKLOADS[args.workload]
+    gen = torch.Generator().manual_seed(3000 + rank)
+    G_host = (torch.randn((m, n), generator=gen) * 1e-2).to(torch.bfloat16).pin_memory()
+    W = (torch.randn((m, n), generator=gen) * 2e-2).to(dev)
+    G = G_host.to(dev)
+    M = torch.zeros((m, n), device=dev)
+    ws = torch.empty(ga.zgcm_muon_workspace_size(m, n), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    step = lambda g=G: ga.zgcm_muon_step(W, g, M, workspace=ws, stream=stream)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) as clk:
+        clk.wait_ready()
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+        clk.mark_start()
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        clk.mark_end()
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev) / args.steps
+    if ga.zgcm_attn_device_error() != 0:
+        print(json.dumps({"error": "device wait expired in the timed region"}))
+        return 1
+    # the products' kernel alone, on the iteration's two shapes (p = min, q = max): X X^T and
+    # (A) X, each a 2 p^2 q multiply-add count
+    p_, q_ = min(m, n), max(m, n)
+    X = (torch.randn((p_, q_), generator=gen) * 1e-2).to(torch.bfloat16).to(dev)
+    A = (torch.randn((p_, p_), generator=gen) * 1e-2).to(torch.bfloat16).to(dev)
+    Cx, Ca = torch.empty_like(X), torch.empty_like(A)
+    gemms = {"X X^T": lambda: ga.zgcm_muon_gemm(X, X, out=Ca, stream=stream),
+             "A X": lambda: ga.zgcm_muon_gemm(A, X, D=X, alpha=-0.5, beta=1.5, b_kn=True, out=Cx, stream=stream)}
+    kms = {}
+    for name, f in gemms.items():
+        for _ in range(3):
+            f()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            f()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        kms[name] = e0.elapsed_time(e1) / args.steps
+    # end to end: the gradient from pinned host memory and the updated weights back, every step
+    W_host = torch.empty((m, n), dtype=torch.float32).pin_memory()
+    Gd = torch.empty_like(G)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        Gd.copy_(G_host, non_blocking=True)
+        step(Gd)
+        W_host.copy_(W, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        if rank != 0:
+            dist.destroy_process_group()
+            return 0
+    peaks, peak_src = load_peaks()
+    flops = muon.ns_flops(m, n)
+    name = max(kms, key=kms.get)
+    gflop = 2 * p_ * p_ * q_
+    roof = {"bound": "tensor", "achieved": gflop / (kms[name] / 1e3) / 1e12, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "traffic": None, "kernel": f"muon_gemm_kernel ({name}, {p_} x {q_})",
+            "kernel_ms": kms[name], "kernels_ms": kms, "algorithmic_flops": gflop,
+            "peak_source": f"{peak_src} (bf16 burst: the kernel timed back to back on its own)"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    cpu = None if (world > 1 or args.no_cpu_baseline) else muon_cpu_baseline(m, n)
+    launches = 3 + 2 * muon.NS_STEPS + 1  # momentum, norm, scaling; 2 products per step; update
+    rec = {
+        "metric": MUON_METRIC, "value": flops * world / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0, 0.01^2) bf16 gradient, N(0, 0.02^2) fp32 weights",
+        "config": {"workload": f"Muon step of one {m} x {n} matrix (momentum 0.9, Frobenius scaling, "
+                               f"{muon.NS_STEPS} Newton-Schulz steps {muon.NS_COEFFS}, lr 2e-4, wd 0.1)",
+                   "parallelism": f"dp{world} (one matrix per GPU)",
+                   "l2": f"operands larger than L2 ({m * n * 10 / 1e9:.2f} GB of W, G, M)"},
+        "roofline": roof, "cpu_baseline": cpu,
+        "e2e": {"value": flops * world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": G_host.numel() * 2, "d2h_bytes_per_step": W_host.numel() * 4,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(rec))
+    return 0
+
+
 def decode_cpu_baseline(P, layers):
     """The oracle's forward rows for a bounded sample: the last row of 2 sequences of P + 1
     tokens per layer (the row a decode step computes), tokens per second over both layers."""
@@ -505,7 +642,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS),
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(MUON_WORKLOADS),
                     default="swa16k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=8)
@@ -525,6 +662,18 @@ def main():
                                           "d2h_bytes_per_step": 0}}))
             return 0
         return run_decode(args)
+    if args.workload in MUON_WORKLOADS:
+        if args.impl == "reference":
+            _, rank, _ = rank_env()
+            if rank == 0:
+                cpu = muon_cpu_baseline(*MUON_WORKLOADS[args.workload])
+                print(json.dumps({"impl": "reference", "metric": MUON_METRIC, "value": cpu["value"],
+                                  "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": 1, "warmup": 0,
+                                  "higher_is_better": True, "dtype": "f64", "data": "synthetic",
+                                  "cpu_baseline": cpu, "e2e": {"value": cpu["value"], "unit": "TFLOP/s",
+                                                               "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+            return 0
+        return run_muon(args)
     if args.impl == "reference":
         return run_reference(args)
 

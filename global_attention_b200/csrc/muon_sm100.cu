@@ -50,6 +50,8 @@ struct GemmParams {
     int M, N, K;
     float alpha, beta;
     int b_kn;           // 1: B is [K, N] (C = A B), 0: B is [N, K] (C = A B^T)
+    int upper;          // 1: C is symmetric; tiles wholly below the diagonal are skipped (the
+                        // mirror kernel fills that half from the other)
     int* err;
 };
 
@@ -71,6 +73,7 @@ __global__ void __launch_bounds__(THREADS, 1) muon_gemm_kernel(const __grid_cons
     volatile int* abort = &sm.abort;
     const int n0 = (int)blockIdx.x * BN, m0 = (int)blockIdx.y * BM;
     const int nk = (p.K + BK - 1) / BK;
+    if (p.upper && n0 + BN <= m0) return;  // every column of the tile left of its first row
 
     if (tid == 0) {
         sm.abort = 0;
@@ -290,6 +293,23 @@ __global__ void __launch_bounds__(256) muon_scale_kernel(const T* __restrict__ s
     }
 }
 
+// C[r][c] = C[c][r] for every c < r of a symmetric p x p matrix whose upper triangle (and
+// diagonal) is computed: 32 x 32 tiles of the lower triangle through shared memory.
+__global__ void __launch_bounds__(256) muon_mirror_kernel(bf16* __restrict__ C, int p) {
+    __shared__ bf16 tile[32][34];
+    const int bx = (int)blockIdx.x, by = (int)blockIdx.y;  // destination tile: rows by*32, columns bx*32
+    if (bx > by) return;
+    for (int y = threadIdx.y; y < 32; y += 8) {  // source: rows bx*32.., columns by*32..
+        const int r = bx * 32 + y, c = by * 32 + threadIdx.x;
+        if (r < p && c < p) tile[y][threadIdx.x] = C[(size_t)r * p + c];
+    }
+    __syncthreads();
+    for (int y = threadIdx.y; y < 32; y += 8) {
+        const int r = by * 32 + y, c = bx * 32 + threadIdx.x;
+        if (r < p && c < r) C[(size_t)r * p + c] = tile[threadIdx.x][y];
+    }
+}
+
 // W <- W (1 - lr wd) - lr O for an m x n W; O = X ([m, n]) or X^T (X is [n, m] when transposed)
 __global__ void __launch_bounds__(256) muon_update_kernel(float* __restrict__ W, const bf16* __restrict__ X, int m,
                                                           int n, int transposed, float lr, float wd) {
@@ -344,8 +364,9 @@ bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_ro
 
 // C [M, N] = alpha A op(B) + beta D: A [M, K]; B [K, N] (b_kn) or [N, K]
 cudaError_t launch_gemm(const bf16* A, const bf16* B, const bf16* D, bf16* C, int M, int N, int K, float alpha,
-                        float beta, bool b_kn, cudaStream_t stream) {
+                        float beta, bool b_kn, cudaStream_t stream, bool upper = false) {
     GemmParams p;
+    p.upper = upper ? 1 : 0;
     if (!make_map(&p.tm_a, A, M, K, BM)) return cudaErrorInvalidValue;
     if (b_kn ? !make_map(&p.tm_b, B, K, N, BK) : !make_map(&p.tm_b, B, N, K, BN)) return cudaErrorInvalidValue;
     p.d = D;
@@ -362,6 +383,8 @@ cudaError_t launch_gemm(const bf16* A, const bf16* B, const bf16* D, bf16* C, in
     if (e != cudaSuccess) return e;
     const dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
     muon_gemm_kernel<<<grid, THREADS, smem, stream>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess || !upper) return e;
+    muon_mirror_kernel<<<dim3((M + 31) / 32, (M + 31) / 32), dim3(32, 8), 0, stream>>>(C, M);
     return cudaGetLastError();
 }
 
@@ -410,11 +433,11 @@ cudaError_t iterate(Ws& w, int p, int q, int steps, float a, float b, float c, c
     bf16* y = w.x1;
     cudaError_t e = cudaSuccess;
     for (int s = 0; s < steps && e == cudaSuccess; ++s) {
-        // A = X X^T
-        if ((e = launch_gemm(x, x, nullptr, w.a, p, p, q, 1.0f, 0.0f, false, stream)) != cudaSuccess) break;
+        // A = X X^T (symmetric: the upper tiles, then the mirror)
+        if ((e = launch_gemm(x, x, nullptr, w.a, p, p, q, 1.0f, 0.0f, false, stream, true)) != cudaSuccess) break;
         if (c != 0.0f) {
-            // B = b A + c A A  (A symmetric: A A = A A^T)
-            if ((e = launch_gemm(w.a, w.a, w.a, w.b, p, p, p, c, b, false, stream)) != cudaSuccess) break;
+            // B = b A + c A A  (A symmetric: A A = A A^T, and B symmetric)
+            if ((e = launch_gemm(w.a, w.a, w.a, w.b, p, p, p, c, b, false, stream, true)) != cudaSuccess) break;
             // X' = a X + B X
             e = launch_gemm(w.b, x, x, y, p, q, p, 1.0f, a, true, stream);
         } else {
