@@ -91,6 +91,14 @@ def load() -> ctypes.CDLL:
         lib.zgcm_muon_orthogonalize.restype = i
         lib.zgcm_muon_gemm.argtypes = [vp, vp, vp, vp, i, i, i, f, f, i, vp]
         lib.zgcm_muon_gemm.restype = i
+        lib.zgcm_proj_qkvg_fwd.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp, vp, vp]
+        lib.zgcm_proj_qkvg_fwd.restype = i
+        lib.zgcm_proj_qkvg_bwd.argtypes = [vp] * 6 + [i] * 5 + [vp, vp, vp]
+        lib.zgcm_proj_qkvg_bwd.restype = i
+        lib.zgcm_proj_out_fwd.argtypes = [vp, vp, i, i, i, vp, vp]
+        lib.zgcm_proj_out_fwd.restype = i
+        lib.zgcm_proj_out_bwd.argtypes = [vp, vp, vp, i, i, i, vp, vp, vp]
+        lib.zgcm_proj_out_bwd.restype = i
         _lib = lib
     return _lib
 
@@ -492,3 +500,66 @@ def zgcm_muon_gemm(A, B, *, D=None, alpha=1.0, beta=0.0, b_kn=False, out=None, s
     if st != ZGCM_OK:
         raise ZgcmError(st, "zgcm_muon_gemm")
     return out
+
+
+# ---------------------------------------------------------------- projections (zgcm_proj.h)
+
+def _proj_check(*named):
+    import torch
+    for n, t in named:
+        _check(t, n, torch.bfloat16, 2)
+
+
+def zgcm_proj_qkvg_fwd(x, w_qkvg, *, Hq=32, Hkv=8, D=128, out=None, stream=None):
+    """q, g [T, Hq*D] and k, v [T, Hkv*D] = the parts of x W_qkvg^T (x [T, d_model] bf16,
+    W_qkvg [(2 Hq + 2 Hkv) D, d_model] bf16, the rows of W_q, W_k, W_v, W_g)."""
+    import torch
+    _proj_check(("x", x), ("w_qkvg", w_qkvg))
+    T, dm = x.shape
+    if out is None:
+        out = tuple(torch.empty((T, h * D), dtype=torch.bfloat16, device=x.device) for h in (Hq, Hkv, Hkv, Hq))
+    st = load().zgcm_proj_qkvg_fwd(_ptr(x), _ptr(w_qkvg), T, dm, Hq, Hkv, D, *(_ptr(t) for t in out), _stream(stream))
+    if st != ZGCM_OK:
+        raise ZgcmError(st, "zgcm_proj_qkvg_fwd")
+    return out
+
+
+def zgcm_proj_qkvg_bwd(x, w_qkvg, dq, dk, dv, dg, *, Hq=32, Hkv=8, D=128, dx=None, dw=None, stream=None):
+    """dx = [dq|dk|dv|dg] W_qkvg and dW_qkvg = [dq|dk|dv|dg]^T x (bf16)."""
+    import torch
+    _proj_check(("x", x), ("w_qkvg", w_qkvg), ("dq", dq), ("dk", dk), ("dv", dv), ("dg", dg))
+    T, dm = x.shape
+    dx = torch.empty_like(x) if dx is None else dx
+    dw = torch.empty_like(w_qkvg) if dw is None else dw
+    st = load().zgcm_proj_qkvg_bwd(_ptr(x), _ptr(w_qkvg), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), T, dm, Hq, Hkv,
+                                   D, _ptr(dx), _ptr(dw), _stream(stream))
+    if st != ZGCM_OK:
+        raise ZgcmError(st, "zgcm_proj_qkvg_bwd")
+    return dx, dw
+
+
+def zgcm_proj_out_fwd(a, w_o, *, out=None, stream=None):
+    """y [T, d_model] = a W_o^T (a [T, d_in], W_o [d_model, d_in], bf16)."""
+    import torch
+    _proj_check(("a", a), ("w_o", w_o))
+    T, din = a.shape
+    dm = w_o.shape[0]
+    y = torch.empty((T, dm), dtype=torch.bfloat16, device=a.device) if out is None else out
+    st = load().zgcm_proj_out_fwd(_ptr(a), _ptr(w_o), T, din, dm, _ptr(y), _stream(stream))
+    if st != ZGCM_OK:
+        raise ZgcmError(st, "zgcm_proj_out_fwd")
+    return y
+
+
+def zgcm_proj_out_bwd(a, w_o, dy, *, da=None, dw=None, stream=None):
+    """da = dy W_o and dW_o = dy^T a (bf16)."""
+    import torch
+    _proj_check(("a", a), ("w_o", w_o), ("dy", dy))
+    T, din = a.shape
+    dm = w_o.shape[0]
+    da = torch.empty_like(a) if da is None else da
+    dw = torch.empty_like(w_o) if dw is None else dw
+    st = load().zgcm_proj_out_bwd(_ptr(a), _ptr(w_o), _ptr(dy), T, din, dm, _ptr(da), _ptr(dw), _stream(stream))
+    if st != ZGCM_OK:
+        raise ZgcmError(st, "zgcm_proj_out_bwd")
+    return da, dw

@@ -10,18 +10,16 @@
 //   X  <- a X + (b A + c A A) X,   A = X X^T          `steps` times, bf16 operands, fp32 sums
 //   W  <- W (1 - lr wd) - lr X^(T)                    (fp32 master weights)
 //
-// Products: one tcgen05 GEMM kernel, C = alpha A op(B) + beta D (bf16 in and out, fp32
-// accumulation in TMEM).  A is [M, K] row-major; B is [N, K] (C = A B^T: X X^T and A A, A
-// symmetric) or [K, N] (C = A B: (.) X).  One CTA per 128 x 256 output tile: a TMA warp
-// streams 64-wide K slabs of A and B through a 4-stage ring (128-byte swizzle), one thread
-// issues tcgen05.mma M=128 N=256 K=16 into a 256-column TMEM accumulator, and four epilogue
-// warps (thread = output row) apply alpha, beta and D and store bf16.  The elementwise steps
+// Products: the library's tcgen05 GEMM (gemm_sm100.cu), C = alpha A op(B) + beta D (bf16 in
+// and out, fp32 accumulation in TMEM): B is [N, K] for X X^T and A A (A symmetric: only the
+// upper tiles, then mirrored) and [K, N] for (.) X.  The elementwise steps
 // (momentum with the sum of squares, the scaling with the optional transpose, the update)
 // are plain streaming kernels; the norm is summed in a fixed order, so a step is
 // reproducible bit for bit.
 #include <cudaTypedefs.h>
 
 #include "../../include/zgcm_muon.h"
+#include "gemm_sm100.cuh"
 #include "sm100.cuh"
 
 namespace zgcm {
@@ -31,164 +29,8 @@ using namespace sm100;
 
 namespace muon {
 
-constexpr int BM = 128;                      // output rows of a CTA (MMA M)
-constexpr int BN = 256;                      // output columns of a CTA (MMA N)
-constexpr int BK = 64;                       // K of a stage: one 128-byte bf16 row
-constexpr int STAGES = 4;
-constexpr uint32_t A_STAGE = BM * BK * 2;    // 16 KB
-constexpr uint32_t B_STAGE = BN * BK * 2;    // 32 KB
-constexpr uint32_t B_CHUNK = BK * 128;       // [K, N] operand: one 64-column chunk of a stage, 8 KB
-constexpr int THREADS = 256;                 // w0 TMA, w1 MMA + TMEM, w2-3 idle, w4-7 epilogue
 constexpr int RED_THREADS = 256;
 constexpr int RED_BLOCKS = 296;              // partial sums of squares (2 blocks per SM)
-
-struct GemmParams {
-    CUtensorMap tm_a;   // A [M, K] bf16, box {64 (K), 128 (rows)}, 128-byte swizzle
-    CUtensorMap tm_b;   // [N, K]: box {64 (K), 256 (rows)};  [K, N]: box {64 (N), 64 (K rows)}
-    const bf16* d;      // [M, N], the beta term (null: none)
-    bf16* c;            // [M, N]
-    int M, N, K;
-    float alpha, beta;
-    int b_kn;           // 1: B is [K, N] (C = A B), 0: B is [N, K] (C = A B^T)
-    int upper;          // 1: C is symmetric; tiles wholly below the diagonal are skipped (the
-                        // mirror kernel fills that half from the other)
-    int* err;
-};
-
-enum { BAR_FULL = 0, BAR_EMPTY = STAGES, BAR_DONE = 2 * STAGES, NBAR = 2 * STAGES + 1 };
-
-struct GemmSmem {
-    alignas(1024) unsigned char A[STAGES][A_STAGE];
-    alignas(1024) unsigned char B[STAGES][B_STAGE];
-    uint64_t bar[NBAR];
-    uint32_t tmem_base;
-    int abort;
-};
-static_assert(sizeof(GemmSmem) + 1024 <= 232448, "beyond the 227 KB of shared memory a CTA can have");
-
-__global__ void __launch_bounds__(THREADS, 1) muon_gemm_kernel(const __grid_constant__ GemmParams p) {
-    extern __shared__ unsigned char smem_raw[];
-    GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    volatile int* abort = &sm.abort;
-    const int n0 = (int)blockIdx.x * BN, m0 = (int)blockIdx.y * BM;
-    const int nk = (p.K + BK - 1) / BK;
-    if (p.upper && n0 + BN <= m0) return;  // every column of the tile left of its first row
-
-    if (tid == 0) {
-        sm.abort = 0;
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&sm.bar[BAR_FULL + s], 1);
-            mbar_init(&sm.bar[BAR_EMPTY + s], 1);
-        }
-        mbar_init(&sm.bar[BAR_DONE], 1);
-        fence_barrier_init();
-    }
-    if (warp == 1) {
-        tmem_alloc(&sm.tmem_base, BN);
-        tmem_relinquish();
-    }
-    if (warp == 0 && lane == 0) {
-        prefetch_tmap(&p.tm_a);
-        prefetch_tmap(&p.tm_b);
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = sm.tmem_base;
-
-    if (warp == 0) {
-        // ================================================ TMA producer: the K slabs of A and B
-        if (lane == 0) {
-            int issued = 0;
-            for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % STAGES;
-                if (kb >= STAGES && !mbar_wait(&sm.bar[BAR_EMPTY + s], ((kb / STAGES) - 1) & 1, abort, 501)) break;
-                mbar_expect_tx(&sm.bar[BAR_FULL + s], A_STAGE + B_STAGE);
-                tma_load_2d(sm.A[s], &p.tm_a, &sm.bar[BAR_FULL + s], kb * BK, m0);
-                if (p.b_kn) {
-                    for (int j = 0; j < BN / 64; ++j)
-                        tma_load_2d(sm.B[s] + j * B_CHUNK, &p.tm_b, &sm.bar[BAR_FULL + s], n0 + 64 * j, kb * BK);
-                } else {
-                    tma_load_2d(sm.B[s], &p.tm_b, &sm.bar[BAR_FULL + s], kb * BK, n0);
-                }
-                issued = kb + 1;
-            }
-            // every copy issued lands before the CTA exits (matters after an abort)
-            for (int kb = issued > STAGES ? issued - STAGES : 0; kb < issued; ++kb)
-                mbar_wait_drain(&sm.bar[BAR_FULL + kb % STAGES], (kb / STAGES) & 1);
-        }
-    } else if (warp == 1) {
-        // ================================================ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(BM, BN, p.b_kn != 0);
-            bool ok = true;
-            for (int kb = 0; kb < nk && ok; ++kb) {
-                const int s = kb % STAGES;
-                if (!(ok = mbar_wait(&sm.bar[BAR_FULL + s], (kb / STAGES) & 1, abort, 502))) break;
-                tc_fence_after();
-                const uint32_t a0 = smem_u32(sm.A[s]), b0 = smem_u32(sm.B[s]);
-#pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk) {
-                    // A K-major: 16 elements = 32 bytes along the swizzled row.  B: K-major the
-                    // same; [K, N] (MN-major): 16 K rows = 2 KB on, 64-column chunks 8 KB apart
-                    const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
-                    const uint64_t bd = p.b_kn ? sdesc_sw128(b0 + kk * 16 * 128, B_CHUNK, 1024)
-                                               : sdesc_sw128(b0 + kk * 32, 16, 1024);
-                    mma_ss(tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(&sm.bar[BAR_EMPTY + s]);  // the stage is free once these products are done
-            }
-            // every MMA issued completes before TMEM is read or released
-            mma_commit(&sm.bar[BAR_DONE]);
-            if (!mbar_wait(&sm.bar[BAR_DONE], 0, abort, 504)) mbar_wait_drain(&sm.bar[BAR_DONE], 0);
-        }
-    } else if (warp >= 4) {
-        // ================================================ epilogue: thread = output row m0 + r
-        const int wq = warp - 4, r = 32 * wq + lane, row = m0 + r;
-        const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
-        const bool got = mbar_wait(&sm.bar[BAR_DONE], 0, abort, 503);
-        if (__all_sync(0xffffffffu, got)) {  // tcgen05.ld is warp-collective: one decision per warp
-            tc_fence_after();
-            for (int c = 0; c < BN / 32; ++c) {
-                float v[32];
-                tmem_ld32f(tmem + lane_off + 32 * c, v);
-                tmem_wait_ld();
-                if (row >= p.M) continue;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int col = n0 + 32 * c + 8 * q;  // N is a multiple of 8: whole chunks
-                    if (col >= p.N) break;
-                    const size_t off = (size_t)row * p.N + col;
-                    float dv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                    if (p.d) {
-                        const uint4 u = __ldg(reinterpret_cast<const uint4*>(p.d + off));
-                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = unpack_bf16(w[e]);
-                            dv[2 * e] = f.x;
-                            dv[2 * e + 1] = f.y;
-                        }
-                    }
-                    uint32_t o[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        o[e] = pack_bf16(fmaf(p.alpha, v[8 * q + 2 * e], p.beta * dv[2 * e]),
-                                         fmaf(p.alpha, v[8 * q + 2 * e + 1], p.beta * dv[2 * e + 1]));
-                    *reinterpret_cast<uint4*>(p.c + off) = make_uint4(o[0], o[1], o[2], o[3]);
-                }
-            }
-        }
-    }
-
-    // ------------------------------------------------ teardown
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, BN);
-    if (tid == 0 && sm.abort && p.err) atomicExch(p.err, sm.abort);
-}
 
 // ------------------------------------------------------------------ elementwise kernels
 
@@ -293,23 +135,6 @@ __global__ void __launch_bounds__(256) muon_scale_kernel(const T* __restrict__ s
     }
 }
 
-// C[r][c] = C[c][r] for every c < r of a symmetric p x p matrix whose upper triangle (and
-// diagonal) is computed: 32 x 32 tiles of the lower triangle through shared memory.
-__global__ void __launch_bounds__(256) muon_mirror_kernel(bf16* __restrict__ C, int p) {
-    __shared__ bf16 tile[32][34];
-    const int bx = (int)blockIdx.x, by = (int)blockIdx.y;  // destination tile: rows by*32, columns bx*32
-    if (bx > by) return;
-    for (int y = threadIdx.y; y < 32; y += 8) {  // source: rows bx*32.., columns by*32..
-        const int r = bx * 32 + y, c = by * 32 + threadIdx.x;
-        if (r < p && c < p) tile[y][threadIdx.x] = C[(size_t)r * p + c];
-    }
-    __syncthreads();
-    for (int y = threadIdx.y; y < 32; y += 8) {
-        const int r = by * 32 + y, c = bx * 32 + threadIdx.x;
-        if (r < p && c < r) C[(size_t)r * p + c] = tile[threadIdx.x][y];
-    }
-}
-
 // W <- W (1 - lr wd) - lr O for an m x n W; O = X ([m, n]) or X^T (X is [n, m] when transposed)
 __global__ void __launch_bounds__(256) muon_update_kernel(float* __restrict__ W, const bf16* __restrict__ X, int m,
                                                           int n, int transposed, float lr, float wd) {
@@ -335,57 +160,23 @@ __global__ void __launch_bounds__(256) muon_update_kernel(float* __restrict__ W,
 
 // ------------------------------------------------------------------ host side
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
-// 2-D bf16 map of a row-major [rows, cols] matrix, box {64 columns, box_rows rows}, 128-byte swizzle
-bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
-    auto enc = get_encode();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // C [M, N] = alpha A op(B) + beta D: A [M, K]; B [K, N] (b_kn) or [N, K]
 cudaError_t launch_gemm(const bf16* A, const bf16* B, const bf16* D, bf16* C, int M, int N, int K, float alpha,
                         float beta, bool b_kn, cudaStream_t stream, bool upper = false) {
-    GemmParams p;
-    p.upper = upper ? 1 : 0;
-    if (!make_map(&p.tm_a, A, M, K, BM)) return cudaErrorInvalidValue;
-    if (b_kn ? !make_map(&p.tm_b, B, K, N, BK) : !make_map(&p.tm_b, B, N, K, BN)) return cudaErrorInvalidValue;
-    p.d = D;
-    p.c = C;
-    p.M = M;
-    p.N = N;
-    p.K = K;
-    p.alpha = alpha;
-    p.beta = beta;
-    p.b_kn = b_kn ? 1 : 0;
-    p.err = library_error_word();
-    const size_t smem = sizeof(GemmSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(muon_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
-    muon_gemm_kernel<<<grid, THREADS, smem, stream>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess || !upper) return e;
-    muon_mirror_kernel<<<dim3((M + 31) / 32, (M + 31) / 32), dim3(32, 8), 0, stream>>>(C, M);
-    return cudaGetLastError();
+    GemmDesc g;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.a[0] = GemmSeg{A, M, K, 0};
+    g.b_kn = b_kn ? 1 : 0;
+    g.b = B;
+    g.c[0] = C;
+    g.c_ld[0] = N;
+    g.d = D;
+    g.alpha = alpha;
+    g.beta = beta;
+    g.upper = upper;
+    return zgcm::launch_gemm(g, library_error_word(), stream);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }

@@ -350,3 +350,21 @@ def test_muon_checks(lib):
     assert gemm(G, G, 0, O, 64, 64, 64, 2) == -1            # layout flag
     assert gemm(G, G, 0, 0, 64, 64, 64, 0) == -1
     assert gemm(G + 8, G, 0, O, 64, 64, 64, 0) == -3
+
+
+def test_proj_checks(lib):
+    """Projection calls reject shapes the tiles cannot split and bad pointers before any launch."""
+    vp = ctypes.c_void_p
+    x, w, q, k, v, g = (P + (1 << 22) * i for i in range(6))
+    fwd = lambda T, dm, Hq, Hkv, D, ptrs=(x, w, q, k, v, g): lib.zgcm_proj_qkvg_fwd(
+        vp(ptrs[0]), vp(ptrs[1]), T, dm, Hq, Hkv, D, *(vp(t) for t in ptrs[2:]), None)
+    assert fwd(0, 512, 4, 2, 128) == -1                      # no tokens
+    assert fwd(64, 500, 4, 2, 128) == -1                     # d_model not a multiple of 256
+    assert fwd(64, 512, 3, 1, 64) == -1                      # Hkv * D = 64
+    assert fwd(64, 512, 4, 2, 128, (x, w, q, 0, v, g)) == -1
+    assert fwd(64, 512, 4, 2, 128, (x, w + 8, q, k, v, g)) == -3
+    out = lambda T, din, dm, y=q: lib.zgcm_proj_out_fwd(vp(x), vp(w), T, din, dm, vp(y), None)
+    assert out(64, 512, 300) == -1
+    assert out(64, 512, 512, 0) == -1
+    bwd = lambda da: lib.zgcm_proj_out_bwd(vp(x), vp(w), vp(q), 64, 512, 512, vp(da), vp(k), None)
+    assert bwd(v + 4) == -3
