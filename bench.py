@@ -616,6 +616,136 @@ def run_muon(args):
     return 0
 
 
+# the projections around the layer for the 16K training batch: x [B*S, 4096] -> q, k, v, g
+# (heads 32 / 8 of 128) and the output projection, forward and backward
+PROJ_WORKLOADS = {"proj16k": (4 * 16384, 4096, 32, 8, 128)}
+PROJ_METRIC = "projections_fwd_bwd_tflops"
+
+
+def proj_cpu_baseline(T, dm, hq, hkv, d):
+    """The fp64 oracle's projections (forward and backward) on a bounded sample of the tokens."""
+    import numpy as np
+    from oracle import proj
+    Ts = 256
+    wq, wkv = hq * d, hkv * d
+    rng = np.random.default_rng(0)
+    x, a = rng.standard_normal((Ts, dm)), rng.standard_normal((Ts, wq))
+    w, wo = rng.standard_normal((2 * (wq + wkv), dm)), rng.standard_normal((dm, wq))
+    t0 = time.perf_counter()
+    q, k, v, g = proj.qkvg_forward(x, w, wq, wkv)
+    proj.qkvg_backward(x, w, q, k, v, g)
+    y = proj.out_forward(a, wo)
+    proj.out_backward(a, wo, y)
+    secs = time.perf_counter() - t0
+    fl = sum(proj.proj_flops(Ts, dm, wq, wkv, wq).values())
+    return {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{Ts} of the {T} tokens (numpy fp64), {secs:.2f} s"}
+
+
+def run_proj(args):
+    """K steps of the projections' forward and backward on resident inputs."""
+    import torch
+    import global_attention_b200 as ga
+    from oracle import proj
+    world, rank, local = rank_env()
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ga.load()
+    T, dm, hq, hkv, d = PROJ_WORKLOADS[args.workload]
+    wq, wkv = hq * d, hkv * d
+    gen = torch.Generator().manual_seed(4000 + rank)
+    rnd = lambda shape, sc=1.0: (torch.randn(shape, generator=gen) * sc).to(torch.bfloat16).to(dev)
+    x_host = torch.randn((T, dm), generator=gen).to(torch.bfloat16).pin_memory()
+    x, w, wo = x_host.to(dev), rnd((2 * (wq + wkv), dm), dm ** -0.5), rnd((dm, wq), wq ** -0.5)
+    a, dy = rnd((T, wq)), rnd((T, dm))
+    parts = tuple(torch.empty((T, h), dtype=torch.bfloat16, device=dev) for h in (wq, wkv, wkv, wq))
+    dparts = tuple(rnd(p.shape) for p in parts)
+    dx, dw, y, da, dwo = (torch.empty_like(t) for t in (x, w, dy, a, wo))
+    stream = torch.cuda.current_stream()
+    names = ("qkvg_fwd", "out_fwd", "out_bwd", "qkvg_bwd")
+    calls = {"qkvg_fwd": lambda src=x: ga.zgcm_proj_qkvg_fwd(src, w, Hq=hq, Hkv=hkv, D=d, out=parts, stream=stream),
+             "out_fwd": lambda: ga.zgcm_proj_out_fwd(a, wo, out=y, stream=stream),
+             "out_bwd": lambda: ga.zgcm_proj_out_bwd(a, wo, dy, da=da, dw=dwo, stream=stream),
+             "qkvg_bwd": lambda src=x: ga.zgcm_proj_qkvg_bwd(src, w, *dparts, Hq=hq, Hkv=hkv, D=d, dx=dx, dw=dw,
+                                                            stream=stream)}
+    for _ in range(args.warmup):
+        for n in names:
+            calls[n]()
+    torch.cuda.synchronize()
+    ev = {n: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)] for n in names}
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) as clk:
+        clk.wait_ready()
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+        clk.mark_start()
+        t0.record(stream)
+        for i in range(args.steps):
+            for n in names:
+                ev[n][i][0].record(stream)
+                calls[n]()
+                ev[n][i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        clk.mark_end()
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev) / args.steps
+    kms = {n: statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev[n]) for n in names}
+    # end to end: the layer input from pinned host memory, dx back to the host, every step
+    dx_host = torch.empty_like(dx, device="cpu").pin_memory()
+    xd = torch.empty_like(x)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        xd.copy_(x_host, non_blocking=True)
+        calls["qkvg_fwd"](xd)
+        calls["out_fwd"]()
+        calls["out_bwd"]()
+        calls["qkvg_bwd"](xd)
+        dx_host.copy_(dx, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        if rank != 0:
+            dist.destroy_process_group()
+            return 0
+    peaks, peak_src = load_peaks()
+    fl = proj.proj_flops(T, dm, wq, wkv, wq)
+    total = sum(fl.values())
+    top = max(kms, key=kms.get)
+    roof = {"bound": "tensor", "achieved": fl[top] / (kms[top] / 1e3) / 1e12, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "traffic": None, "kernel": f"gemm_kernel ({top}: {2 if top.endswith('bwd') else 1} launch(es))",
+            "kernel_ms": kms[top], "kernels_ms": kms, "algorithmic_flops": fl[top],
+            "peak_source": f"{peak_src} (bf16 burst)"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    cpu = None if (world > 1 or args.no_cpu_baseline) else proj_cpu_baseline(T, dm, hq, hkv, d)
+    rec = {
+        "metric": PROJ_METRIC, "value": total * world / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) bf16 activations and gradients, N(0, 1/fan_in) bf16 weights",
+        "config": {"workload": f"q/k/v/g and output projections fwd+bwd, {T} tokens, hidden {dm}, heads {hq}/{hkv}x{d}",
+                   "parallelism": f"dp{world}", "l2": f"operands larger than L2 ({(x.numel() + a.numel()) * 4 / 1e9:.2f} GB)"},
+        "roofline": roof, "cpu_baseline": cpu,
+        "e2e": {"value": total * world / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": dx_host.numel() * 2,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(rec))
+    return 0
+
+
 def decode_cpu_baseline(P, layers):
     """The oracle's forward rows for a bounded sample: the last row of 2 sequences of P + 1
     tokens per layer (the row a decode step computes), tokens per second over both layers."""
@@ -642,8 +772,8 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(MUON_WORKLOADS),
-                    default="swa16k")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(MUON_WORKLOADS)
+                    + sorted(PROJ_WORKLOADS), default="swa16k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=8)
     args = ap.parse_args()
@@ -662,6 +792,18 @@ def main():
                                           "d2h_bytes_per_step": 0}}))
             return 0
         return run_decode(args)
+    if args.workload in PROJ_WORKLOADS:
+        if args.impl == "reference":
+            _, rank, _ = rank_env()
+            if rank == 0:
+                cpu = proj_cpu_baseline(*PROJ_WORKLOADS[args.workload])
+                print(json.dumps({"impl": "reference", "metric": PROJ_METRIC, "value": cpu["value"],
+                                  "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": 1, "warmup": 0,
+                                  "higher_is_better": True, "dtype": "f64", "data": "synthetic",
+                                  "cpu_baseline": cpu, "e2e": {"value": cpu["value"], "unit": "TFLOP/s",
+                                                               "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+            return 0
+        return run_proj(args)
     if args.workload in MUON_WORKLOADS:
         if args.impl == "reference":
             _, rank, _ = rank_env()

@@ -60,3 +60,26 @@ def test_gradients_reach_their_inputs(store_bytes):
     for n, r in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("g", "dg"), ("gamma_q", "dgamma_q"),
                  ("gamma_k", "dgamma_k")):
         np.testing.assert_array_equal(x[n].grad.numpy(), ref[r], err_msg=n)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("S,W", [(700, 128), (500, 10**6)])
+def test_autograd_on_the_gpu_matches_oracle(S, W):
+    """zgcm_attention end to end on the B200 (the library's training pair under autograd):
+    a loss sum(dout * out) backpropagated to every input equals the oracle's gradients."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from tests.parity_util import assert_bf16_close, assert_dgamma_close
+    t = make_inputs(1, S, seed=31 + S, with_dout=True)
+    leaves = {n: t[n].cuda().requires_grad_(True) for n in ("q", "k", "v", "g", "gamma_q", "gamma_k")}
+    out = zgcm_attention(*(leaves[n] for n in ("q", "k", "v", "g", "gamma_q", "gamma_k")), window=W)
+    (out.float() * t["dout"].cuda().float()).sum().backward()
+    torch.cuda.synchronize()
+    P = oracle.Problem(t["q"], t["k"], t["v"], t["g"], t["gamma_q"], t["gamma_k"], window=W)
+    ref_out, _ = P.forward()
+    ref = P.backward(t["dout"])
+    assert_bf16_close("out", out.detach(), ref_out)
+    for n, r in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("g", "dg")):
+        assert_bf16_close(r, leaves[n].grad, ref[r])
+    assert_dgamma_close("dgamma_q", leaves["gamma_q"].grad, ref["dgamma_q"])
+    assert_dgamma_close("dgamma_k", leaves["gamma_k"].grad, ref["dgamma_k"])
