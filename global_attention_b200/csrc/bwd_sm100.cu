@@ -40,7 +40,7 @@ namespace zgcm {
 // =====================================================================  gate backward pass
 
 constexpr int GATE_THREADS = 256;
-constexpr int GATE_UNROLL = 4;  // rows in flight per half-warp
+constexpr int GATE_UNROLL = 2;  // rows in flight per half-warp
 
 // Sigmoid gate backward of out = sigmoid(g) * A (the gated-attention page, output gate):
 //   dA = dout * sigmoid(g)  -> da16 = fp16(dA * 2^e), e = fit_exp(max|dout| of the row)
@@ -55,7 +55,7 @@ constexpr int GATE_UNROLL = 4;  // rows in flight per half-warp
 // Rows: dout, g, out, dg are [B,Sq,Hq,D] (positions q_off .. S-1, Sq = S - q_off); da16 and
 // the row arrays are indexed by position ([B,S,Hq,D], [B,Hq,Spad]).
 template <bool DELTA>
-__global__ void __launch_bounds__(GATE_THREADS, 2) bwd_gate_kernel(const bf16* __restrict__ dout,
+__global__ void __launch_bounds__(GATE_THREADS, 4) bwd_gate_kernel(const bf16* __restrict__ dout,
                                                                 const bf16* __restrict__ g,
                                                                 const bf16* __restrict__ out,
                                                                 bf16* __restrict__ dg, __half* __restrict__ da16,
@@ -1479,12 +1479,12 @@ cudaError_t launch_bwd_tc(const BwdParams& bp, void* workspace, int* err_word, c
     if (steps > 0x7fffffffLL) return cudaErrorInvalidValue;
     p.total = (int)steps;
     const int grid = (int)(steps < sms ? steps : sms);
-    // gate pass over the query rows: 2 resident blocks of 256 threads per SM, each half-warp
+    // gate pass over the query rows: 4 resident blocks of 256 threads per SM, each half-warp
     // GATE_UNROLL rows at a time
     const long long qrows = (long long)L.B * L.Sq * L.Hq;
     const long long half_warps = (qrows + GATE_UNROLL - 1) / GATE_UNROLL;
     const long long gate_need = (half_warps * 16 + GATE_THREADS - 1) / GATE_THREADS;
-    const int gate_grid = (int)(gate_need < 2LL * sms ? gate_need : 2LL * sms);
+    const int gate_grid = (int)(gate_need < 4LL * sms ? gate_need : 4LL * sms);
     const size_t smem_pk = sizeof(PrepSmem<true>) + 1024, smem_pq = sizeof(PrepSmem<false>) + 1024;
     if ((e = cudaFuncSetAttribute(prep_kv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_pk)) != cudaSuccess)
         return e;
