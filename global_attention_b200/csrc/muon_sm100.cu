@@ -18,7 +18,7 @@
 // reproducible bit for bit.
 #include <cudaTypedefs.h>
 
-#include "../../include/zgcm_muon.h"
+#include "zgcm_muon.h"
 #include "gemm_sm100.cuh"
 #include "sm100.cuh"
 

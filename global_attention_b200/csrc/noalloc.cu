@@ -16,7 +16,7 @@
 // lives on another device is rejected with ZGCM_ERR_INVALID_ARG).
 #include <mutex>
 
-#include "../../include/zgcm_attn.h"
+#include "zgcm_attn.h"
 
 namespace {
 

@@ -3,7 +3,7 @@
 // (gemm_sm100.cu) with the q / k / v / g parts split in place.
 #include <stdint.h>
 
-#include "../../include/zgcm_proj.h"
+#include "zgcm_proj.h"
 #include "gemm_sm100.cuh"
 
 namespace zgcm {

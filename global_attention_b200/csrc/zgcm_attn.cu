@@ -5,7 +5,7 @@
 #include <stdint.h>
 #include <stdlib.h>
 
-#include "../../include/zgcm_attn.h"
+#include "zgcm_attn.h"
 #include "common.cuh"
 
 namespace zgcm {
