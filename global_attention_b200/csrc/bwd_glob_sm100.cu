@@ -79,7 +79,9 @@ enum QgBar {
     QG_DQFULL = QG_DSFULL + 1,                 // every product done: dQ~ final
     QG_MDOT = QG_DQFULL + 1,                   // the second warpgroup's RMSNorm row sums
     QG_DELTA = QG_MDOT + 1,                    // both halves of a one-tile sweep's sum P dP
-    QG_COUNT = QG_DELTA + 1
+    QG_DQDONE = QG_DELTA + 1,                  // dQ(n) has read dS(n): S buffer n % 2 free (2)
+    QG_SDONE = QG_DQDONE + 2,                  // the S / dP issuer's products are complete
+    QG_COUNT = QG_SDONE + 1
 };
 
 struct BwdQGlobSmem {
@@ -165,6 +167,9 @@ __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid
         mbar_init(&sm.bar[QG_DQFULL], 1);
         mbar_init(&sm.bar[QG_MDOT], 128);
         mbar_init(&sm.bar[QG_DELTA], 256);
+        mbar_init(&sm.bar[QG_DQDONE], 1);
+        mbar_init(&sm.bar[QG_DQDONE + 1], 1);
+        mbar_init(&sm.bar[QG_SDONE], 1);
         fence_barrier_init();
     }
     if (tid < kD) {
@@ -227,11 +232,12 @@ __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid
             for (int n = nv > QG_VSLOTS ? nv - QG_VSLOTS : 0; n < nv; ++n)
                 mbar_wait_drain(&sm.bar[QG_VFULL + n % QG_VSLOTS], (n / QG_VSLOTS) & 1);
         }
-    } else if (warp == 1) {
-        // ================================================ MMA issuer
-        // S(0) dP(0) S(1), then per tile n: dP(n+1) once dP(n) has been read, dQ(n) once dS(n)
-        // is written, S(n+2) over S(n) (after dQ(n), which reads dS(n) there: MMAs of one
-        // thread execute in order).
+    } else if (warp == 1 || warp == 2) {
+        // ================================================ MMA issuers
+        // warp 1: S(0) dP(0) S(1), then per tile n: dP(n+1) once dP(n) has been read, S(n+2)
+        // over S(n) once dQ(n), which reads dS(n) there, has completed (QG_DQDONE);
+        // warp 2: dQ(n) once dS(n) is written.  Two issuing threads, so that neither one's
+        // waits leave the tensor pipe without instructions.
         reg_dealloc<56>();
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_f16(128, 128, false);
@@ -267,7 +273,8 @@ __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid
                     mma_ts(TM_DQ, tm_s(n) + acol, sdesc_sw128(kb + kk * 16 * 128, TF_HALF_BYTES, 1024), IDESC_DQ,
                            (n > 0 || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(&sm.bar[QG_KEMPTY + n % QG_KSLOTS]);
+                mma_commit(&sm.bar[QG_KEMPTY + n % QG_KSLOTS]);  // (S(n) completed before dS(n) existed)
+                mma_commit(&sm.bar[QG_DQDONE + (n & 1)]);
             };
             auto kfull = [&](int n, int site) {
                 return mbar_wait(&sm.bar[QG_KFULL + n % QG_KSLOTS], (n / QG_KSLOTS) & 1, abort, site);
@@ -275,41 +282,53 @@ __global__ void __launch_bounds__(BQG_THREADS, 1) bwd_q_glob_kernel(const __grid
             auto vfull = [&](int n, int site) {
                 return mbar_wait(&sm.bar[QG_VFULL + n % QG_VSLOTS], (n / QG_VSLOTS) & 1, abort, site);
             };
-            bool ok = mbar_wait(&sm.bar[QG_QFULL], 0, abort, 310) && kfull(0, 311);
-            if (ok) {
-                tc_fence_after();
-                issue_s(0);
-                ok = vfull(0, 312);
-            }
-            if (ok) {
-                tc_fence_after();
-                issue_dp(0);
-                if (N > 1 && (ok = kfull(1, 313))) {
+            if (warp == 2) {
+                bool ok = true;
+                for (int n = 0; n < N && ok; ++n) {
+                    if (!(ok = mbar_wait(&sm.bar[QG_DSFULL], n & 1, abort, 316))) break;
                     tc_fence_after();
-                    issue_s(1);
+                    issue_dq(n);
                 }
-            }
-            for (int n = 0; n < N && ok; ++n) {
-                if (n + 1 < N) {
-                    if (!(ok = mbar_wait(&sm.bar[QG_DPFREE], n & 1, abort, 314) && vfull(n + 1, 315))) break;
+                // every MMA issued must complete before TMEM is released; DQFULL is that point
+                // for the dQ products (the S / dP ones complete before the last dS exists)
+                mma_commit(&sm.bar[QG_DQFULL]);
+                if (!mbar_wait(&sm.bar[QG_DQFULL], 0, abort, 318)) mbar_wait_drain(&sm.bar[QG_DQFULL], 0);
+            } else {
+                bool ok = mbar_wait(&sm.bar[QG_QFULL], 0, abort, 310) && kfull(0, 311);
+                if (ok) {
                     tc_fence_after();
-                    issue_dp(n + 1);
+                    issue_s(0);
+                    ok = vfull(0, 312);
                 }
-                if (!(ok = mbar_wait(&sm.bar[QG_DSFULL], n & 1, abort, 316))) break;
-                tc_fence_after();
-                issue_dq(n);
-                if (n + 2 < N) {
-                    if (!(ok = kfull(n + 2, 317))) break;
+                if (ok) {
                     tc_fence_after();
-                    issue_s(n + 2);
+                    issue_dp(0);
+                    if (N > 1 && (ok = kfull(1, 313))) {
+                        tc_fence_after();
+                        issue_s(1);
+                    }
                 }
+                for (int n = 0; n < N && ok; ++n) {
+                    if (n + 1 < N) {
+                        if (!(ok = mbar_wait(&sm.bar[QG_DPFREE], n & 1, abort, 314) && vfull(n + 1, 315))) break;
+                        tc_fence_after();
+                        issue_dp(n + 1);
+                    }
+                    if (n + 2 < N) {
+                        if (!(ok = mbar_wait(&sm.bar[QG_DQDONE + (n & 1)], (n >> 1) & 1, abort, 319) &&
+                                   kfull(n + 2, 317)))
+                            break;
+                        tc_fence_after();
+                        issue_s(n + 2);
+                    }
+                }
+                // this thread's products complete before TMEM is released (after an abort too)
+                mma_commit(&sm.bar[QG_SDONE]);
+                if (!mbar_wait(&sm.bar[QG_SDONE], 0, abort, 322)) mbar_wait_drain(&sm.bar[QG_SDONE], 0);
             }
-            // every MMA issued must complete before TMEM is released; DQFULL is that point
-            mma_commit(&sm.bar[QG_DQFULL]);
-            if (!mbar_wait(&sm.bar[QG_DQFULL], 0, abort, 318)) mbar_wait_drain(&sm.bar[QG_DQFULL], 0);
         }
     } else if (warp < 4) {
-        reg_dealloc<56>();  // warps 2-3: idle
+        reg_dealloc<56>();  // warp 3: idle
     } else {
         // ================================================ dS (thread = query row, 64 keys of each tile)
         const int hh = warp >= 8 ? 1 : 0, wq = warp & 3;

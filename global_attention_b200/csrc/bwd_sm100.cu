@@ -764,7 +764,8 @@ enum KBar {
     KB_SFULL = 15, KB_PFULL = 17,                 // by TMEM buffer (2 each)
     KB_DVKFULL = 19, KB_DVKEMPTY = 20, KB_DONE = 21, KB_RED = 22,
     KB_STATS = 23,  // a unit's scales are in shared memory; by unit number % 2
-    KB_COUNT = 25
+    KB_DVKDONE = 25,  // the dV / dK products of a half have read their TMEM buffer; by buffer (2)
+    KB_COUNT = 27
 };
 
 struct BwdKTcSmem {
@@ -859,7 +860,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
         }
         mbar_init(&sm.bar[KB_DVKFULL], 1);
         mbar_init(&sm.bar[KB_DVKEMPTY], 128);
-        mbar_init(&sm.bar[KB_DONE], 1);
+        mbar_init(&sm.bar[KB_DONE], 2);  // both MMA issuers
+        mbar_init(&sm.bar[KB_DVKDONE], 1);
+        mbar_init(&sm.bar[KB_DVKDONE + 1], 1);
         mbar_init(&sm.bar[KB_RED], 4);  // one arrival per epilogue warp
         mbar_init(&sm.bar[KB_STATS], 128);
         mbar_init(&sm.bar[KB_STATS + 1], 128);
@@ -947,13 +950,14 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                 for (int i = 0; i < KV_SLOTS; ++i)
                     if (last_q[i] >= 0) mbar_wait_drain(&sm.bar[KB_QFULL + i], (last_q[i] / KV_SLOTS) & 1);
             }
-        } else if (warp == 1) {
-            // ================================================ MMA issuer
+        } else if (warp == 1 || warp == 2) {
+            // ================================================ MMA issuers
             // Per 64-query half h (sweep order: unit, iteration, half), into TMEM buffer h % 2:
             //   S(h):   S^T = K~ Q~_h^T, dP^T = V dA_h^T      (M = 128 keys, N = 64, K = d)
             //   DVK(h): dV += P^T_h dA_h, dK~ += dS^T_h Q~_h  (K = 64 queries)
-            // issued as S(0) S(1) DVK(0) S(2) DVK(1) S(3) ...: the softmax of half h+1 runs while
-            // the tensor core does DVK(h) and S(h+2).
+            // warp 1 issues the S products, warp 2 the DVK ones, so that neither thread's waits
+            // and bookkeeping leave the tensor pipe without instructions: S(h+2) waits for
+            // DVK(h) to have read buffer h % 2 (KB_DVKDONE), DVK(h) for the softmax of half h.
             if (lane == 0) {
                 constexpr uint32_t IDESC_S = idesc_f16(128, 64, false);
                 constexpr uint32_t IDESC_MN = idesc_f16(128, 128, true);
@@ -1025,24 +1029,27 @@ __global__ void __launch_bounds__(TB_THREADS, 1) bwd_kv_tc_kernel(const __grid_c
                                (!first || kk > 0) ? 1u : 0u);
                     }
                     mma_commit(&sm.bar[KB_QEMPTY + slot]);  // the half's Q~ and dA rows were read for the last time
+                    mma_commit(&sm.bar[KB_DVKDONE + c.half]);  // TMEM buffer h % 2 read: free for S(h+2)
                     if (last_of_unit(c)) mma_commit(&sm.bar[KB_DVKFULL]);
                     return true;
                 };
-                Cursor cs_ = cur_first(), cd = cur_first();
                 bool ok = true;
-                for (int n = 0; n < 2 && ok && cs_.valid; ++n) {
-                    ok = issue_s(cs_);
-                    cur_next(cs_);
-                }
-                while (ok && cd.valid) {
-                    ok = issue_dvk(cd);
-                    if (ok && cs_.valid) {
+                if (warp == 1) {
+                    Cursor cs_ = cur_first();
+                    for (int hs = 0; ok && cs_.valid; ++hs) {
+                        if (hs >= 2 && !(ok = mbar_wait(&sm.bar[KB_DVKDONE + (hs & 1)], ((hs >> 1) - 1) & 1, abort, 215)))
+                            break;
                         ok = issue_s(cs_);
                         cur_next(cs_);
                     }
-                    cur_next(cd);
+                } else {
+                    Cursor cd = cur_first();
+                    while (ok && cd.valid) {
+                        ok = issue_dvk(cd);
+                        cur_next(cd);
+                    }
                 }
-                mma_commit(&sm.bar[KB_DONE]);
+                mma_commit(&sm.bar[KB_DONE]);  // this thread's products, all complete before teardown
                 mbar_wait(&sm.bar[KB_DONE], 0, abort, 214);
             }
         }
