@@ -128,26 +128,84 @@ def _check(t, name, dtype, ndim, cuda=True):
         raise TypeError(f"{name} must be a CUDA tensor")
 
 
-def _check_bwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, dout, grads):
-    """Dtype, rank, layout and device of every backward tensor, before any launch."""
+def _need(t, name, dtype, shape):
+    """t: a contiguous tensor of `dtype` and exactly `shape` (no device check)."""
+    _check(t, name, dtype, len(shape), cuda=False)
+    if tuple(t.shape) != tuple(shape):
+        raise TypeError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+
+
+def _one_device(*named):
+    """Every tensor given (None skipped) is a CUDA tensor on the device of the first one.
+    The library sees pointers and sizes only, so the shapes are checked before this, and
+    before any launch: a tensor smaller than the sizes passed would be read or written past
+    its end."""
+    ts = [(n, t) for n, t in named if t is not None]
+    for n, t in ts:
+        if not t.is_cuda:
+            raise TypeError(f"{n} must be a CUDA tensor")
+    n0, t0 = ts[0]
+    for n, t in ts:
+        if t.device != t0.device:
+            raise TypeError(f"{n} must be on the device of {n0} ({t0.device})")
+
+
+def _layer_shapes(q, k, v, g, gamma_q, gamma_k, rows=False):
+    """(B, Sq, S, Hq, Hkv, D) of a layer call: q, g [B,Sq,Hq,D] bf16, k, v [B,S,Hkv,D] bf16,
+    gamma_q, gamma_k [D] fp32; Sq = S unless `rows` (query rows at the end of the keys)."""
     import torch
-    for n, t in (("q", q), ("k", k), ("v", v), ("g", g), ("out", out), ("dout", dout)):
-        _check(t, n, torch.bfloat16, 4, cuda=False)
-    _check(lse, "lse", torch.float32, 3, cuda=False)
-    _check(gamma_q, "gamma_q", torch.float32, 1, cuda=False)
-    _check(gamma_k, "gamma_k", torch.float32, 1, cuda=False)
+    _check(q, "q", torch.bfloat16, 4, cuda=False)
+    _check(k, "k", torch.bfloat16, 4, cuda=False)
+    B, Sq, Hq, D = q.shape
+    S, Hkv = k.shape[1], k.shape[2]
+    if k.shape[0] != B or k.shape[3] != D:
+        raise TypeError(f"k must be [B, S, Hkv, D] with q's B = {B} and D = {D}, not {tuple(k.shape)}")
+    if not rows and S != Sq:
+        raise TypeError(f"q and k must have one sequence length ({Sq} != {S})")
+    _need(v, "v", torch.bfloat16, k.shape)
+    _need(g, "g", torch.bfloat16, q.shape)
+    _need(gamma_q, "gamma_q", torch.float32, (D,))
+    _need(gamma_k, "gamma_k", torch.float32, (D,))
+    return B, Sq, S, Hq, Hkv, D
+
+
+def _check_fwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, workspace, saved=None, rows=False):
+    """Dtype, layout and shape of every forward tensor, then their device, before any launch."""
+    import torch
+    B, Sq, S, Hq, Hkv, D = _layer_shapes(q, k, v, g, gamma_q, gamma_k, rows)
+    if out is not None:
+        _need(out, "out", torch.bfloat16, q.shape)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (B, Hq, Sq))
+    for n, t in (("workspace", workspace), ("saved", saved)):
+        if t is not None:
+            _check(t, n, torch.uint8, 1, cuda=False)
+    _one_device(("q", q), ("k", k), ("v", v), ("g", g), ("gamma_q", gamma_q), ("gamma_k", gamma_k),
+                ("out", out), ("lse", lse), ("workspace", workspace), ("saved", saved))
+    return B, Sq, S, Hq, Hkv, D
+
+
+def _check_bwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, dout, grads, workspace=None, saved=None,
+                    rows=False):
+    """Dtype, layout and shape of every backward tensor, then their device, before any launch."""
+    import torch
+    B, Sq, S, Hq, Hkv, D = _layer_shapes(q, k, v, g, gamma_q, gamma_k, rows)
+    _need(out, "out", torch.bfloat16, q.shape)
+    _need(dout, "dout", torch.bfloat16, q.shape)
+    _need(lse, "lse", torch.float32, (B, Hq, Sq))
+    gl = []
     if grads is not None:
         for n, ref in (("dq", q), ("dk", k), ("dv", v), ("dg", g)):
-            _check(grads[n], n, torch.bfloat16, 4, cuda=False)
-            if grads[n].shape != ref.shape:
-                raise TypeError(f"{n} must have the shape of its input {tuple(ref.shape)}")
+            _need(grads[n], n, torch.bfloat16, ref.shape)
         for n in ("dgamma_q", "dgamma_k"):
-            _check(grads[n], n, torch.float32, 1, cuda=False)
-    tensors = [q, k, v, g, gamma_q, gamma_k, out, lse, dout] + ([] if grads is None else list(grads.values()))
-    if not all(t.is_cuda for t in tensors):
-        raise TypeError("every tensor must be a CUDA tensor")
-    if any(t.device != q.device for t in tensors):
-        raise TypeError("every tensor must be on the device of q")
+            _need(grads[n], n, torch.float32, (D,))
+        gl = [(n, grads[n]) for n in ("dq", "dk", "dv", "dg", "dgamma_q", "dgamma_k")]
+    for n, t in (("workspace", workspace), ("saved", saved)):
+        if t is not None:
+            _check(t, n, torch.uint8, 1, cuda=False)
+    _one_device(("q", q), ("k", k), ("v", v), ("g", g), ("gamma_q", gamma_q), ("gamma_k", gamma_k), ("out", out),
+                ("lse", lse), ("dout", dout), *gl, ("workspace", workspace), ("saved", saved))
+    return B, Sq, S, Hq, Hkv, D
 
 
 def zgcm_attn_fwd_workspace_size(B, S, Hq, Hkv, D=128, rope_dims=42, window=128) -> int:
@@ -171,12 +229,7 @@ def zgcm_attn_fwd(q, k, v, g, gamma_q, gamma_k, *, rope_dims=42, rope_base=10000
     zgcm_attn_saved_size bytes (zgcm_attn_fwd_save; then no workspace is used) that keeps the
     activations zgcm_attn_bwd(saved=...) reads."""
     import torch
-    for n, t in (("q", q), ("k", k), ("v", v), ("g", g)):
-        _check(t, n, torch.bfloat16, 4)
-    _check(gamma_q, "gamma_q", torch.float32, 1)
-    _check(gamma_k, "gamma_k", torch.float32, 1)
-    B, S, Hq, D = q.shape
-    Hkv = k.shape[2]
+    B, S, _, Hq, Hkv, D = _check_fwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, workspace, saved)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if out is None:
@@ -184,7 +237,6 @@ def zgcm_attn_fwd(q, k, v, g, gamma_q, gamma_k, *, rope_dims=42, rope_base=10000
     if lse is None:
         lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
     if saved is not None:
-        _check(saved, "saved", torch.uint8, 1)
         st = load().zgcm_attn_fwd_save(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gamma_q), _ptr(gamma_k),
                                        B, S, Hq, Hkv, D, int(rope_dims), float(rope_base), int(window),
                                        int(causal), float(eps), float(scale), _ptr(out), _ptr(lse),
@@ -217,15 +269,27 @@ def zgcm_attn_decode(q, k, v, g, gamma_q, gamma_k, pos, k_cache, v_cache, *, rop
     pos int32 [B] (its position), k_cache fp16 / v_cache bf16 [B,C,Hkv,D] (updated in place).
     Returns (out bf16 [B,Hq,D], lse fp32 [B,Hq])."""
     import torch
-    for n, t in (("q", q), ("g", g), ("k", k), ("v", v)):
-        _check(t, n, torch.bfloat16, 3)
-    _check(gamma_q, "gamma_q", torch.float32, 1)
-    _check(gamma_k, "gamma_k", torch.float32, 1)
-    _check(pos, "pos", torch.int32, 1)
-    _check(k_cache, "k_cache", torch.float16, 4)
-    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(q, "q", torch.bfloat16, 3, cuda=False)
+    _check(k, "k", torch.bfloat16, 3, cuda=False)
+    _check(k_cache, "k_cache", torch.float16, 4, cuda=False)
     B, Hq, D = q.shape
     Hkv, C = k.shape[1], k_cache.shape[1]
+    _need(g, "g", torch.bfloat16, (B, Hq, D))
+    _need(k, "k", torch.bfloat16, (B, Hkv, D))
+    _need(v, "v", torch.bfloat16, (B, Hkv, D))
+    _need(gamma_q, "gamma_q", torch.float32, (D,))
+    _need(gamma_k, "gamma_k", torch.float32, (D,))
+    _need(pos, "pos", torch.int32, (B,))
+    _need(k_cache, "k_cache", torch.float16, (B, C, Hkv, D))
+    _need(v_cache, "v_cache", torch.bfloat16, (B, C, Hkv, D))
+    if out is not None:
+        _need(out, "out", torch.bfloat16, (B, Hq, D))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (B, Hq))
+    if workspace is not None:
+        _check(workspace, "workspace", torch.uint8, 1, cuda=False)
+    _one_device(("q", q), ("k", k), ("v", v), ("g", g), ("gamma_q", gamma_q), ("gamma_k", gamma_k), ("pos", pos),
+                ("k_cache", k_cache), ("v_cache", v_cache), ("out", out), ("lse", lse), ("workspace", workspace))
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if out is None:
@@ -286,9 +350,7 @@ def zgcm_attn_bwd(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dims=42,
     a list of (begin, end) torch.cuda.Event pairs, brackets the backward's kernels in launch
     order (zgcm_attn_bwd_timed; names from zgcm_attn_bwd_kernel_names)."""
     import torch
-    _check_bwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, dout, grads)
-    B, S, Hq, D = q.shape
-    Hkv = k.shape[2]
+    B, S, _, Hq, Hkv, D = _check_bwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, dout, grads, workspace, saved)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if grads is None:
@@ -316,7 +378,6 @@ def zgcm_attn_bwd(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dims=42,
         arr = (ctypes.c_void_p * max(1, len(flat)))(*flat)
         n_pairs = len(kernel_events)
     if saved is not None:
-        _check(saved, "saved", torch.uint8, 1)
         st = load().zgcm_attn_bwd_saved(*args[:-1], _ptr(saved), saved.numel(), args[-1], arr, n_pairs)
         if st != ZGCM_OK:
             raise ZgcmError(st, "zgcm_attn_bwd_saved")
@@ -337,12 +398,7 @@ def zgcm_attn_fwd_rows(q, k, v, g, gamma_q, gamma_k, *, rope_dims=42, rope_base=
     Sq < S).  Returns (out bf16 [B,Sq,Hq,D], lse fp32 [B,Hq,Sq]), the rows of the whole
     sequence's forward."""
     import torch
-    for n, t in (("q", q), ("k", k), ("v", v), ("g", g)):
-        _check(t, n, torch.bfloat16, 4)
-    _check(gamma_q, "gamma_q", torch.float32, 1)
-    _check(gamma_k, "gamma_k", torch.float32, 1)
-    B, Sq, Hq, D = q.shape
-    S, Hkv = k.shape[1], k.shape[2]
+    B, Sq, S, Hq, Hkv, D = _check_fwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, workspace, rows=True)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if out is None:
@@ -367,9 +423,8 @@ def zgcm_attn_bwd_rows(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_dim
     """Backward of zgcm_attn_fwd_rows: dq, dg of the query rows, dk, dv of every key row and
     dgamma_q, dgamma_k, each the part these query rows contribute (a dict as zgcm_attn_bwd)."""
     import torch
-    _check_bwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, dout, grads)
-    B, Sq, Hq, D = q.shape
-    S, Hkv = k.shape[1], k.shape[2]
+    B, Sq, S, Hq, Hkv, D = _check_bwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, dout, grads, workspace,
+                                           rows=True)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if grads is None:
@@ -399,9 +454,7 @@ def zgcm_attn_bwd_noalloc(q, k, v, g, gamma_q, gamma_k, out, lse, dout, *, rope_
     B*S <= 3117 tokens fit).  The call runs with q's device current, so the array used is
     that device's.  Calls that overlap on the GPU race."""
     import torch
-    _check_bwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, dout, grads)
-    B, S, Hq, D = q.shape
-    Hkv = k.shape[2]
+    B, S, _, Hq, Hkv, D = _check_bwd_args(q, k, v, g, gamma_q, gamma_k, out, lse, dout, grads)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if grads is None:
@@ -439,7 +492,9 @@ def _muon_ws(m, n, workspace, device):
     need = zgcm_muon_workspace_size(m, n)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
-    _check(workspace, "workspace", torch.uint8, 1)
+    _check(workspace, "workspace", torch.uint8, 1, cuda=False)
+    if not workspace.is_cuda or workspace.device != device:
+        raise TypeError(f"workspace must be a CUDA tensor on the matrix's device ({device})")
     return workspace
 
 
@@ -447,11 +502,10 @@ def zgcm_muon_step(W, G, M, *, lr=MUON_LR, weight_decay=MUON_WEIGHT_DECAY, momen
                    steps=MUON_STEPS, coeffs=MUON_COEFFS, eps=1e-7, workspace=None, stream=None):
     """One Muon step in place: W fp32 [m, n], G bf16 [m, n], M fp32 [m, n] (momentum buffer)."""
     import torch
-    _check(W, "W", torch.float32, 2)
-    _check(G, "G", torch.bfloat16, 2)
-    _check(M, "M", torch.float32, 2)
-    if G.shape != W.shape or M.shape != W.shape:
-        raise TypeError("W, G and M must have one shape")
+    _check(W, "W", torch.float32, 2, cuda=False)
+    _need(G, "G", torch.bfloat16, W.shape)
+    _need(M, "M", torch.float32, W.shape)
+    _one_device(("W", W), ("G", G), ("M", M))
     m, n = W.shape
     ws = _muon_ws(m, n, workspace, W.device)
     a, b, c = (float(x) for x in coeffs)
@@ -466,7 +520,10 @@ def zgcm_muon_orthogonalize(G, *, steps=MUON_STEPS, coeffs=MUON_COEFFS, eps=1e-7
                             stream=None):
     """bf16 [m, n]: the Newton–Schulz iterate after `steps` steps from G / (||G||_F + eps)."""
     import torch
-    _check(G, "G", torch.bfloat16, 2)
+    _check(G, "G", torch.bfloat16, 2, cuda=False)
+    if out is not None:
+        _need(out, "out", torch.bfloat16, G.shape)
+    _one_device(("G", G), ("out", out))
     m, n = G.shape
     if out is None:
         out = torch.empty_like(G)
@@ -483,16 +540,17 @@ def zgcm_muon_gemm(A, B, *, D=None, alpha=1.0, beta=0.0, b_kn=False, out=None, s
     """C = alpha A op(B) + beta D in bf16 (fp32 accumulation): A [M, K]; B [K, N] if b_kn else
     [N, K] (C = A B^T)."""
     import torch
-    _check(A, "A", torch.bfloat16, 2)
-    _check(B, "B", torch.bfloat16, 2)
+    _check(A, "A", torch.bfloat16, 2, cuda=False)
+    _check(B, "B", torch.bfloat16, 2, cuda=False)
     M, K = A.shape
     N = B.shape[1] if b_kn else B.shape[0]
     if (B.shape[0] if b_kn else B.shape[1]) != K:
         raise TypeError("inner dimensions of A and B differ")
     if D is not None:
-        _check(D, "D", torch.bfloat16, 2)
-        if D.shape != (M, N):
-            raise TypeError("D must be [M, N]")
+        _need(D, "D", torch.bfloat16, (M, N))
+    if out is not None:
+        _need(out, "out", torch.bfloat16, (M, N))
+    _one_device(("A", A), ("B", B), ("D", D), ("out", out))
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
     st = load().zgcm_muon_gemm(_ptr(A), _ptr(B), _ptr(D), _ptr(out), M, N, K, float(alpha), float(beta),
@@ -505,19 +563,29 @@ def zgcm_muon_gemm(A, B, *, D=None, alpha=1.0, beta=0.0, b_kn=False, out=None, s
 # ---------------------------------------------------------------- projections (zgcm_proj.h)
 
 def _proj_check(*named):
+    """(name, tensor, shape) triples: contiguous bf16 of that shape (None: not given), then one
+    CUDA device for all of them."""
     import torch
-    for n, t in named:
-        _check(t, n, torch.bfloat16, 2)
+    for n, t, shape in named:
+        if t is not None:
+            _need(t, n, torch.bfloat16, shape)
+    _one_device(*((n, t) for n, t, _ in named))
 
 
 def zgcm_proj_qkvg_fwd(x, w_qkvg, *, Hq=32, Hkv=8, D=128, out=None, stream=None):
     """q, g [T, Hq*D] and k, v [T, Hkv*D] = the parts of x W_qkvg^T (x [T, d_model] bf16,
     W_qkvg [(2 Hq + 2 Hkv) D, d_model] bf16, the rows of W_q, W_k, W_v, W_g)."""
     import torch
-    _proj_check(("x", x), ("w_qkvg", w_qkvg))
+    _check(x, "x", torch.bfloat16, 2, cuda=False)
     T, dm = x.shape
+    widths = (Hq * D, Hkv * D, Hkv * D, Hq * D)
+    if out is not None and len(out) != 4:
+        raise TypeError("out must be the four tensors q, k, v, g")
+    outs = (None,) * 4 if out is None else tuple(out)
+    _proj_check(("x", x, (T, dm)), ("w_qkvg", w_qkvg, (sum(widths), dm)),
+                *((n, t, (T, w)) for n, t, w in zip(("q", "k", "v", "g"), outs, widths)))
     if out is None:
-        out = tuple(torch.empty((T, h * D), dtype=torch.bfloat16, device=x.device) for h in (Hq, Hkv, Hkv, Hq))
+        out = tuple(torch.empty((T, w), dtype=torch.bfloat16, device=x.device) for w in widths)
     st = load().zgcm_proj_qkvg_fwd(_ptr(x), _ptr(w_qkvg), T, dm, Hq, Hkv, D, *(_ptr(t) for t in out), _stream(stream))
     if st != ZGCM_OK:
         raise ZgcmError(st, "zgcm_proj_qkvg_fwd")
@@ -527,8 +595,12 @@ def zgcm_proj_qkvg_fwd(x, w_qkvg, *, Hq=32, Hkv=8, D=128, out=None, stream=None)
 def zgcm_proj_qkvg_bwd(x, w_qkvg, dq, dk, dv, dg, *, Hq=32, Hkv=8, D=128, dx=None, dw=None, stream=None):
     """dx = [dq|dk|dv|dg] W_qkvg and dW_qkvg = [dq|dk|dv|dg]^T x (bf16)."""
     import torch
-    _proj_check(("x", x), ("w_qkvg", w_qkvg), ("dq", dq), ("dk", dk), ("dv", dv), ("dg", dg))
+    _check(x, "x", torch.bfloat16, 2, cuda=False)
     T, dm = x.shape
+    widths = (Hq * D, Hkv * D, Hkv * D, Hq * D)
+    _proj_check(("x", x, (T, dm)), ("w_qkvg", w_qkvg, (sum(widths), dm)),
+                *((n, t, (T, w)) for n, t, w in zip(("dq", "dk", "dv", "dg"), (dq, dk, dv, dg), widths)),
+                ("dx", dx, (T, dm)), ("dw", dw, (sum(widths), dm)))
     dx = torch.empty_like(x) if dx is None else dx
     dw = torch.empty_like(w_qkvg) if dw is None else dw
     st = load().zgcm_proj_qkvg_bwd(_ptr(x), _ptr(w_qkvg), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), T, dm, Hq, Hkv,
@@ -541,9 +613,11 @@ def zgcm_proj_qkvg_bwd(x, w_qkvg, dq, dk, dv, dg, *, Hq=32, Hkv=8, D=128, dx=Non
 def zgcm_proj_out_fwd(a, w_o, *, out=None, stream=None):
     """y [T, d_model] = a W_o^T (a [T, d_in], W_o [d_model, d_in], bf16)."""
     import torch
-    _proj_check(("a", a), ("w_o", w_o))
+    _check(a, "a", torch.bfloat16, 2, cuda=False)
+    _check(w_o, "w_o", torch.bfloat16, 2, cuda=False)
     T, din = a.shape
     dm = w_o.shape[0]
+    _proj_check(("a", a, (T, din)), ("w_o", w_o, (dm, din)), ("out", out, (T, dm)))
     y = torch.empty((T, dm), dtype=torch.bfloat16, device=a.device) if out is None else out
     st = load().zgcm_proj_out_fwd(_ptr(a), _ptr(w_o), T, din, dm, _ptr(y), _stream(stream))
     if st != ZGCM_OK:
@@ -554,9 +628,12 @@ def zgcm_proj_out_fwd(a, w_o, *, out=None, stream=None):
 def zgcm_proj_out_bwd(a, w_o, dy, *, da=None, dw=None, stream=None):
     """da = dy W_o and dW_o = dy^T a (bf16)."""
     import torch
-    _proj_check(("a", a), ("w_o", w_o), ("dy", dy))
+    _check(a, "a", torch.bfloat16, 2, cuda=False)
+    _check(w_o, "w_o", torch.bfloat16, 2, cuda=False)
     T, din = a.shape
     dm = w_o.shape[0]
+    _proj_check(("a", a, (T, din)), ("w_o", w_o, (dm, din)), ("dy", dy, (T, dm)), ("da", da, (T, din)),
+                ("dw", dw, (dm, din)))
     da = torch.empty_like(a) if da is None else da
     dw = torch.empty_like(w_o) if dw is None else dw
     st = load().zgcm_proj_out_bwd(_ptr(a), _ptr(w_o), _ptr(dy), T, din, dm, _ptr(da), _ptr(dw), _stream(stream))

@@ -368,3 +368,100 @@ def test_proj_checks(lib):
     assert out(64, 512, 512, 0) == -1
     bwd = lambda da: lib.zgcm_proj_out_bwd(vp(x), vp(w), vp(q), 64, 512, 512, vp(da), vp(k), None)
     assert bwd(v + 4) == -3
+
+
+def test_bindings_check_shapes_before_any_launch(monkeypatch):
+    """The library sees pointers and sizes only, so each Python wrapper checks that every tensor
+    has the shape the sizes it passes imply (and dtype, layout and one CUDA device) before the
+    C entry point: a tensor shorter than that would be read or written past its end.  Each bad
+    call below fails on the CPU with a shape error; the consistent one gets as far as the
+    device check."""
+    import torch
+    from global_attention_b200.synth import make_inputs
+    reached = []
+
+    class NoLib:
+        def __getattr__(self, name):
+            reached.append(name)
+            raise AssertionError(f"reached the library ({name})")
+
+    monkeypatch.setattr(ga, "load", lambda: NoLib())
+    t = make_inputs(1, 16, with_dout=True)
+    q, k, v, g, gq, gk, do = (t[n] for n in ("q", "k", "v", "g", "gamma_q", "gamma_k", "dout"))
+    lse = torch.zeros((1, 32, 16), dtype=torch.float32)
+    bf = dict(dtype=torch.bfloat16)
+
+    def shape_error(fn, *a, **kw):
+        with pytest.raises(TypeError, match="shape|sequence length|must be \\[|inner dimensions|four tensors"):
+            fn(*a, **kw)
+
+    def device_error(fn, *a, **kw):
+        with pytest.raises(TypeError, match="CUDA"):
+            fn(*a, **kw)
+
+    lay = dict(q=q, k=k, v=v, g=g, gamma_q=gq, gamma_k=gk)
+    # forward
+    for bad in (dict(v=v[:, :8].contiguous()), dict(g=g[:, :, :16].contiguous()), dict(gamma_q=gq[:64].contiguous()),
+                dict(k=k[:, :8].contiguous(), v=v[:, :8].contiguous()),
+                dict(k=torch.zeros((2, 16, 8, 128), **bf), v=torch.zeros((2, 16, 8, 128), **bf))):
+        shape_error(ga.zgcm_attn_fwd, **dict(lay, **bad))
+    shape_error(ga.zgcm_attn_fwd, **lay, out=torch.zeros((1, 8, 32, 128), **bf))
+    shape_error(ga.zgcm_attn_fwd, **lay, lse=torch.zeros((1, 32, 8)))
+    device_error(ga.zgcm_attn_fwd, **lay)
+    # backward (plain, query rows, no allocation)
+    bw = dict(lay, out=q.clone(), lse=lse, dout=do)
+    grads = dict(dq=torch.zeros_like(q), dk=torch.zeros_like(k), dv=torch.zeros_like(v), dg=torch.zeros_like(g),
+                 dgamma_q=torch.zeros(128), dgamma_k=torch.zeros(128))
+    for fn in (ga.zgcm_attn_bwd, ga.zgcm_attn_bwd_noalloc):
+        shape_error(fn, **dict(bw, lse=torch.zeros((1, 32, 8))))
+        shape_error(fn, **dict(bw, out=torch.zeros((1, 8, 32, 128), **bf)))
+        shape_error(fn, **dict(bw, dout=torch.zeros((1, 16, 16, 128), **bf)))
+        shape_error(fn, **bw, grads=dict(grads, dk=torch.zeros((1, 16, 4, 128), **bf)))
+        shape_error(fn, **bw, grads=dict(grads, dgamma_k=torch.zeros(64)))
+        device_error(fn, **bw, grads=grads)
+    rows = dict(lay, q=q[:, 8:].contiguous(), g=g[:, 8:].contiguous())
+    shape_error(ga.zgcm_attn_fwd_rows, **dict(rows, k=torch.zeros((1, 16, 8, 64), **bf)), window=4096)
+    shape_error(ga.zgcm_attn_fwd_rows, **rows, lse=lse, window=4096)
+    device_error(ga.zgcm_attn_fwd_rows, **rows, window=4096)
+    rows_b = dict(rows, out=rows["q"].clone(), lse=torch.zeros((1, 32, 8)), dout=do[:, 8:].contiguous())
+    shape_error(ga.zgcm_attn_bwd_rows, **dict(rows_b, lse=lse), window=4096)
+    device_error(ga.zgcm_attn_bwd_rows, **rows_b, window=4096)
+    # decode
+    dec = dict(q=q[:, 0].contiguous(), k=k[:, 0].contiguous(), v=v[:, 0].contiguous(), g=g[:, 0].contiguous(),
+               gamma_q=gq, gamma_k=gk, pos=torch.zeros(1, dtype=torch.int32),
+               k_cache=torch.zeros((1, 128, 8, 128), dtype=torch.float16), v_cache=torch.zeros((1, 128, 8, 128), **bf))
+    shape_error(ga.zgcm_attn_decode, **dict(dec, v_cache=torch.zeros((1, 64, 8, 128), **bf)))
+    shape_error(ga.zgcm_attn_decode, **dict(dec, pos=torch.zeros(2, dtype=torch.int32)))
+    shape_error(ga.zgcm_attn_decode, **dict(dec, g=torch.zeros((1, 16, 128), **bf)))
+    device_error(ga.zgcm_attn_decode, **dec)
+    # Muon
+    W, G, M = torch.zeros((64, 96)), torch.zeros((64, 96), **bf), torch.zeros((64, 96))
+    shape_error(ga.zgcm_muon_step, W, G[:32].contiguous(), M)
+    shape_error(ga.zgcm_muon_step, W, G, torch.zeros((96, 64)))
+    device_error(ga.zgcm_muon_step, W, G, M)
+    shape_error(ga.zgcm_muon_orthogonalize, G, out=torch.zeros((96, 64), **bf))
+    device_error(ga.zgcm_muon_orthogonalize, G)
+    A, Bm = torch.zeros((64, 32), **bf), torch.zeros((48, 32), **bf)
+    shape_error(ga.zgcm_muon_gemm, A, Bm, out=torch.zeros((64, 32), **bf))
+    shape_error(ga.zgcm_muon_gemm, A, Bm, D=torch.zeros((48, 64), **bf))
+    shape_error(ga.zgcm_muon_gemm, A, Bm, b_kn=True)
+    device_error(ga.zgcm_muon_gemm, A, Bm)
+    # projections (Hq = 4, Hkv = 2, D = 128: W_qkvg has 12 x 128 rows)
+    x, w = torch.zeros((8, 256), **bf), torch.zeros((12 * 128, 256), **bf)
+    pj = dict(Hq=4, Hkv=2, D=128)
+    shape_error(ga.zgcm_proj_qkvg_fwd, x, w[:-128].contiguous(), **pj)
+    shape_error(ga.zgcm_proj_qkvg_fwd, x, w, out=(torch.zeros((8, 512), **bf),) * 3, **pj)
+    shape_error(ga.zgcm_proj_qkvg_fwd, x, w, out=tuple(torch.zeros((8, 256), **bf) for _ in range(4)), **pj)
+    device_error(ga.zgcm_proj_qkvg_fwd, x, w, **pj)
+    dq_, dk_ = torch.zeros((8, 512), **bf), torch.zeros((8, 256), **bf)
+    shape_error(ga.zgcm_proj_qkvg_bwd, x, w, dq_, dk_, dk_, dk_, **pj)
+    shape_error(ga.zgcm_proj_qkvg_bwd, x, w, dq_, dk_, dk_, dq_, dx=torch.zeros((8, 128), **bf), **pj)
+    device_error(ga.zgcm_proj_qkvg_bwd, x, w, dq_, dk_, dk_, dq_, **pj)
+    a_, wo = torch.zeros((8, 512), **bf), torch.zeros((256, 512), **bf)
+    shape_error(ga.zgcm_proj_out_fwd, a_, torch.zeros((256, 384), **bf))
+    shape_error(ga.zgcm_proj_out_fwd, a_, wo, out=torch.zeros((8, 512), **bf))
+    device_error(ga.zgcm_proj_out_fwd, a_, wo)
+    shape_error(ga.zgcm_proj_out_bwd, a_, wo, torch.zeros((8, 512), **bf))
+    shape_error(ga.zgcm_proj_out_bwd, a_, wo, torch.zeros((8, 256), **bf), dw=torch.zeros((512, 256), **bf))
+    device_error(ga.zgcm_proj_out_bwd, a_, wo, torch.zeros((8, 256), **bf))
+    assert not reached
